@@ -1,0 +1,154 @@
+"""CPU oracle for paged KV-cache decode.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package.  It never touches a GPU
+and shares no code with the CUDA library under ``paged_kv_cache_348_b200/``.
+
+The arithmetic lives in ``pagedkv_oracle.c`` (plain C, fp64); this module only
+builds it with gcc and marshals numpy arrays through ctypes.  The copy-on-write
+planner (pure Python bookkeeping, no arithmetic on values) is in ``cow.py``.
+
+All 16-bit tensors are passed as ``numpy.uint16`` bit patterns; ``dtype`` is
+``"f16"`` or ``"bf16"``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "pagedkv_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+DTYPES = {"f16": 0, "bf16": 1}
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle into ``oracle/liboracle.so`` (gcc, -O2, no -ffast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp%d" % os.getpid()
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-o", tmp, _SRC,
+                               "-lm", "-lpthread"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        L = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        i32, i64, u16, f64 = ctypes.c_int, ctypes.c_int64, ctypes.c_uint16, ctypes.c_double
+        L.orc_f16_to_f64.argtypes = [u16]; L.orc_f16_to_f64.restype = f64
+        L.orc_bf16_to_f64.argtypes = [u16]; L.orc_bf16_to_f64.restype = f64
+        L.orc_f64_to_f16.argtypes = [f64]; L.orc_f64_to_f16.restype = u16
+        L.orc_f64_to_bf16.argtypes = [f64]; L.orc_f64_to_bf16.restype = u16
+        L.orc_kv_bytes_per_token.argtypes = [i32, i32, i32, i32]
+        L.orc_kv_bytes_per_token.restype = i64
+        L.orc_gather.argtypes = [P, P, i32, i32, i32, i32, i32, P, i32, i32]
+        L.orc_gather.restype = i32
+        L.orc_decode.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32,
+                                 f64, i32, P, i32, i32]
+        L.orc_decode.restype = i32
+        L.orc_cache_append.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32]
+        L.orc_cache_append.restype = i32
+        L.orc_copy_blocks.argtypes = [P, P, i32, P, i32, i64, i32]
+        L.orc_copy_blocks.restype = i32
+        _lib = L
+    return _lib
+
+
+def _p(a: np.ndarray):
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+def _c(a, dt):
+    return np.ascontiguousarray(a, dtype=dt)
+
+
+# ---- scalar conversions --------------------------------------------------------------
+def to_f64(bits: int, dtype: str) -> float:
+    L = _load()
+    return L.orc_bf16_to_f64(bits) if dtype == "bf16" else L.orc_f16_to_f64(bits)
+
+
+def from_f64(x: float, dtype: str) -> int:
+    L = _load()
+    return L.orc_f64_to_bf16(x) if dtype == "bf16" else L.orc_f64_to_f16(x)
+
+
+def kv_bytes_per_token(layers: int, kv_heads: int, head_dim: int, elem_bytes: int) -> int:
+    return _load().orc_kv_bytes_per_token(layers, kv_heads, head_dim, elem_bytes)
+
+
+# ---- gather / decode / append / copy -------------------------------------------------
+def gather(cache: np.ndarray, dtype: str, table_row: np.ndarray, ctx: int, kvh: int) -> np.ndarray:
+    """Logical rows 0..ctx-1 of one sequence/kv head, fp64 [ctx, D]."""
+    cache = _c(cache, np.uint16)
+    N, Hkv, bs, D = cache.shape
+    tr = _c(table_row, np.int32)
+    out = np.zeros((max(ctx, 0), D), dtype=np.float64)
+    rc = _load().orc_gather(_p(out), _p(cache), DTYPES[dtype], N, Hkv, bs, D, _p(tr), ctx, kvh)
+    if rc:
+        raise ValueError("oracle gather: block id out of range")
+    return out
+
+
+def decode(q, k_cache, v_cache, block_tables, context_lens, scale: float, dtype: str,
+           items=None, nthreads: int = 1):
+    """fp64 paged decode.  Returns (out64 [B,Hq,D] float64, out16 [B,Hq,D] uint16).
+
+    ``items`` restricts the computation to a list of sequence indices (the other
+    rows are returned as zeros)."""
+    q = _c(q, np.uint16)
+    k_cache = _c(k_cache, np.uint16)
+    v_cache = _c(v_cache, np.uint16)
+    bt = _c(block_tables, np.int32)
+    cl = _c(context_lens, np.int32)
+    B, Hq, D = q.shape
+    N, Hkv, bs, D2 = k_cache.shape
+    assert D2 == D and v_cache.shape == k_cache.shape and bt.shape[0] == B
+    out64 = np.zeros((B, Hq, D), dtype=np.float64)
+    out16 = np.zeros((B, Hq, D), dtype=np.uint16)
+    it = None if items is None else _c(items, np.int32)
+    rc = _load().orc_decode(_p(out64), _p(out16), _p(q), _p(k_cache), _p(v_cache), _p(bt), _p(cl),
+                            B, Hq, Hkv, D, bs, bt.shape[1], N, float(scale), DTYPES[dtype],
+                            None if it is None else _p(it), 0 if it is None else len(it),
+                            int(nthreads))
+    if rc == -1:
+        raise ValueError("oracle decode: block id out of range")
+    if rc:
+        raise ValueError("oracle decode: bad arguments (%d)" % rc)
+    return out64, out16
+
+
+def cache_append(k_cache, v_cache, k, v, slot_mapping):
+    """In-place scatter of k/v [T, Hkv, D] into the pools; negative slots are skipped."""
+    assert k_cache.flags.c_contiguous and v_cache.flags.c_contiguous
+    assert k_cache.dtype == np.uint16 and v_cache.dtype == np.uint16
+    N, Hkv, bs, D = k_cache.shape
+    k = _c(k, np.uint16); v = _c(v, np.uint16)
+    sm = _c(slot_mapping, np.int64)
+    rc = _load().orc_cache_append(_p(k_cache), _p(v_cache), _p(k), _p(v), _p(sm), len(sm), Hkv, D,
+                                  bs, N)
+    if rc:
+        raise ValueError("oracle append: slot out of range")
+
+
+def copy_blocks(k_caches, v_caches, pairs):
+    """In-place copy of block src -> dst for every (src, dst) pair and every layer."""
+    L = len(k_caches)
+    N = k_caches[0].shape[0]
+    block_elems = int(np.prod(k_caches[0].shape[1:]))
+    for a in list(k_caches) + list(v_caches):
+        assert a.flags.c_contiguous and a.dtype == np.uint16 and a.shape[0] == N
+    kp = (ctypes.c_void_p * L)(*[a.ctypes.data for a in k_caches])
+    vp = (ctypes.c_void_p * L)(*[a.ctypes.data for a in v_caches])
+    pr = _c(pairs, np.int32).reshape(-1, 2)
+    rc = _load().orc_copy_blocks(kp, vp, L, _p(pr), len(pr), block_elems, N)
+    if rc:
+        raise ValueError("oracle copy_blocks: block id out of range")
