@@ -1,0 +1,410 @@
+"""Paged decode benchmark: KV-read HBM GB/s (and % of peak) and seq-steps/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload llama70b|llama8b|heavytail|prefix] [--block-size BS]
+
+One step = one decode step of the workload over all its layers: pa_copy_blocks of the
+step's copy-on-write pairs (none unless the workload shares partial blocks), then per
+layer pa_cache_append of every sequence's newest token and pa_decode over all cached
+tokens.  Inputs are seeded synthetic tensors already resident in HBM; each layer's K/V
+pools (0.7 GB for the default workload) are larger than L2, so no flush is needed.
+
+With N > 1 (torchrun) every rank runs an independent replica of the workload (the
+path has no exchange step); value = all ranks' KV bytes / the slowest rank's time.
+`--impl reference` times the CPU oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attn: KV-read HBM GB/s (% of B200 peak) and seq-steps/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def workload_desc(w, bs):
+    from paged_kv_cache_348_b200 import inputs
+
+    ctx = {"tiny": "{5,16,17,40}", "llama8b": "U[128,2048]", "llama70b": "U[1000,8000]",
+           "heavytail": "lognormal(median 512, sigma 1.2) clipped [16,32768]",
+           "prefix": "2048 shared + U[0,512] private"}[w.name]
+    return ("%s-shape paged decode step: %d layer(s), batch %d, %d q / %d kv heads, head_dim %d, "
+            "block_size %d, %s, context lens %s, seed %d" % (
+                w.name, w.layers, w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, bs,
+                w.dtype, ctx, w.seed))
+
+
+def source_hash():
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "paged_kv_cache_348_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(d, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def measured_hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def ncu_traffic(workload_name, bs):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was taken on
+    the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        e = d["entries"]["%s_bs%d" % (workload_name, bs)]
+        if e.get("source_hash") != source_hash():
+            return None
+        return int(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id=None):
+        self.proc = None
+        self.bus_id = bus_id
+
+    def __enter__(self):
+        try:
+            cmd = ["nvidia-smi", "--query-gpu=pci.bus_id," + self.FIELDS,
+                   "--format=csv,noheader,nounits", "-lms", "200"]
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        rows = []
+        for l in self.lines:
+            parts = [p.strip() for p in l.split(",")]
+            if len(parts) < 9:
+                continue
+            if self.bus_id and parts[0].lower()[-12:] != self.bus_id.lower()[-12:]:
+                continue
+            rows.append(parts)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1])]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        loaded = [s for s in sm if s >= 0.5 * max(sm)] if sm else []
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": num(rows[0][2]), "reasons": reasons, "samples": len(rows)}
+
+
+def device_bus_id(torch):
+    try:
+        p = torch.cuda.get_device_properties(torch.cuda.current_device())
+        return "%08x:%02x:%02x.0" % (getattr(p, "pci_domain_id", 0), p.pci_bus_id, p.pci_device_id)
+    except Exception:
+        return None
+
+
+# ------------------------------------------------------------------------------- oracle
+def oracle_sample(w, bs, max_seconds=15.0, device_batch=None):
+    """Time the CPU oracle on whole sequences of layer 0 until ~max_seconds of work.
+    Returns (kv_bytes, seconds, seqs, threads)."""
+    import torch
+
+    import oracle
+    from paged_kv_cache_348_b200 import inputs
+
+    threads = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    if device_batch is not None:
+        b = device_batch
+        def bits(t):
+            return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+        q, k, v = bits(b.q[0]), bits(b.k_caches[0]), bits(b.v_caches[0])
+        tables, ctx = b.block_tables.cpu().numpy(), b.context_lens.cpu().numpy()
+    else:
+        from paged_kv_cache_348_b200 import workload as wl
+        b = wl.build(w, device="cpu", block_size=bs, layers=1) if w.name != "prefix" else \
+            wl.build_prefix_decode(w, device="cpu")
+        def bits(t):
+            return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+        q, k, v = bits(b.q[0]), bits(b.k_caches[0]), bits(b.v_caches[0])
+        tables, ctx = b.block_tables.numpy(), b.context_lens.numpy()
+    order = list(range(len(ctx)))
+    done_bytes, spent, seqs = 0, 0.0, 0
+    chunk = max(1, threads // 8)
+    i = 0
+    while i < len(order) and spent < max_seconds:
+        items = order[i:i + chunk]
+        t0 = time.perf_counter()
+        oracle.decode(q, k, v, tables, ctx, 1.0 / math.sqrt(w.head_dim), w.dtype, items=items,
+                      nthreads=threads)
+        spent += time.perf_counter() - t0
+        done_bytes += int(sum(int(ctx[s]) for s in items)) * w.num_kv_heads * w.head_dim * 4
+        seqs += len(items)
+        i += chunk
+    return done_bytes, spent, seqs, threads
+
+
+def run_reference(args, w, bs, rank, world):
+    if rank != 0:
+        return 0
+    for _ in range(args.warmup):
+        oracle_sample(w, bs, max_seconds=1.0)
+    t_all, b_all, s_all, threads = 0.0, 0, 0, 1
+    per = max(5.0, 20.0 / max(1, args.steps))
+    for _ in range(args.steps):
+        nbytes, sec, seqs, threads = oracle_sample(w, bs, max_seconds=per)
+        t_all += sec
+        b_all += nbytes
+        s_all += seqs
+    gbs = b_all / t_all / 1e9
+    # the metric's step is all layers of the workload: scale the sampled time
+    layer_bytes = b_all / max(1, s_all)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * (t_all / max(1, s_all)) * w.num_seqs * w.layers,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": workload_desc(w, bs), "parallelism": "cpu"},
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": "%d whole sequences of layer 0 per step (%.1f s of oracle "
+                                   "time per step), KV bytes of those sequences" % (
+                                       s_all // max(1, args.steps), t_all / max(1, args.steps))},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "seq_steps_per_s": (s_all / w.layers) / t_all,
+        "kv_bytes_per_seq_layer": layer_bytes,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------------------- ours
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="llama70b")
+    ap.add_argument("--block-size", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    from paged_kv_cache_348_b200 import inputs
+
+    w = inputs.WORKLOADS[args.workload]
+    bs = args.block_size or w.block_size
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.impl == "reference":
+        return run_reference(args, w, bs, rank, world)
+
+    import torch
+    import torch.distributed as dist
+
+    from paged_kv_cache_348_b200 import pagedkv as pk
+    from paged_kv_cache_348_b200 import workload as wl
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    pk.load()
+    if w.name == "prefix":
+        b = wl.build_prefix_decode(w, device="cuda")
+    else:
+        b = wl.build(w, device="cuda", block_size=bs)
+    stream = torch.cuda.current_stream()
+    L = b.layers
+    kv_step = b.kv_bytes_per_step()
+    kv_layer = kv_step // L
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        wl.run_step(b)
+    barrier()
+    if int(b.status.item()):
+        raise RuntimeError("device status 0x%x after warm-up" % int(b.status.item()))
+
+    # ---------------- timed region: K steps, per-decode-launch events inside
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps * L)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps * L)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    launches = 0
+    clocks = ClockSampler(device_bus_id(torch) if rank == 0 else None)
+    with clocks:
+        barrier()
+        t_start.record(stream)
+        for s in range(args.steps):
+            if b.cow_pairs is not None and b.cow_pairs.shape[0]:
+                pk.pa_copy_blocks(b.k_caches, b.v_caches, b.cow_pairs, b.status)
+                launches += 1
+            for l in range(L):
+                pk.pa_cache_append(b.k_caches[l], b.v_caches[l], b.k_new[l], b.v_new[l],
+                                   b.slot_mapping, b.status)
+                ev_s[s * L + l].record(stream)
+                pk.pa_decode(b.out[l], b.q[l], b.k_caches[l], b.v_caches[l], b.block_tables,
+                             b.context_lens, b.scale, b.workspace, b.status)
+                ev_e[s * L + l].record(stream)
+                launches += 3          # append, split pass, combine pass
+        t_end.record(stream)
+        barrier()
+    ms = t_start.elapsed_time(t_end)
+    dec_ms = [a.elapsed_time(e) for a, e in zip(ev_s, ev_e)]
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    st = int(b.status.item())
+    if st:
+        raise RuntimeError("device status 0x%x in the timed region" % st)
+    ms_step = ms / args.steps
+    value = world * kv_step / (ms_step * 1e-3) / 1e9
+    peak, peak_kind = measured_hbm_peak()
+    dec_avg = statistics.mean(dec_ms)
+    achieved = kv_layer / (dec_avg * 1e-3) / 1e9
+    traffic = ncu_traffic(w.name, bs)
+
+    # ---------------- end to end through the public API, host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(b, args, world, kv_step)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": workload_desc(w, bs), "global_batch": w.num_seqs * world,
+                   "seq_len": float(b.context_lens.float().mean().item()),
+                   "parallelism": "replicas" if world > 1 else "single gpu",
+                   "l2": "inputs larger than L2 (%.2f GB of K/V per layer)" % (kv_layer / 1e9)},
+        "pct_of_peak_hbm": 100.0 * value / world / peak,
+        "peak_hbm_gbs": peak, "peak_kind": peak_kind,
+        "seq_steps_per_s": world * w.num_seqs / (ms_step * 1e-3),
+        "kv_bytes_per_step": kv_step,
+        "roofline": {"bound": "hbm", "kernel": "pa_decode (split + combine passes)",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "algorithmic_bytes_per_launch": kv_layer,
+                     "avg_launch_ms": dec_avg, "peak_source": peak_kind},
+        "gpu_launches": launches,
+        "clocks": clocks.summary() if rank == 0 else None,
+        "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        nbytes, sec, seqs, threads = oracle_sample(w, bs, device_batch=b)
+        line["cpu_baseline"] = {
+            "value": nbytes / sec / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": "%d whole sequences (all %d q heads) of layer 0 of this workload, "
+                      "%.1f s" % (seqs, w.num_q_heads, sec)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def run_e2e(b, args, world, kv_step):
+    """Per step: pinned host -> device copies of every layer's new q / k / v, the
+    context lens, block tables and slot mapping; the step; device -> host copy of
+    every layer's output.  Timed with CUDA events on the stream."""
+    import torch
+
+    from paged_kv_cache_348_b200 import workload as wl
+
+    L = b.layers
+    hq = [t.cpu().pin_memory() for t in b.q]
+    hk = [t.cpu().pin_memory() for t in b.k_new]
+    hv = [t.cpu().pin_memory() for t in b.v_new]
+    hctx = b.context_lens.cpu().pin_memory()
+    htab = b.block_tables.cpu().pin_memory()
+    hslot = b.slot_mapping.cpu().pin_memory()
+    hout = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in b.out]
+    h2d = sum(t.numel() * t.element_size() for t in hq + hk + hv + [hctx, htab, hslot])
+    d2h = sum(t.numel() * t.element_size() for t in hout)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for l in range(L):
+            b.q[l].copy_(hq[l], non_blocking=True)
+            b.k_new[l].copy_(hk[l], non_blocking=True)
+            b.v_new[l].copy_(hv[l], non_blocking=True)
+        b.context_lens.copy_(hctx, non_blocking=True)
+        b.block_tables.copy_(htab, non_blocking=True)
+        b.slot_mapping.copy_(hslot, non_blocking=True)
+        wl.run_step(b)
+        for l in range(L):
+            hout[l].copy_(b.out[l], non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(args.steps):
+        step()
+    e.record(stream)
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e)
+    if world > 1:
+        import torch.distributed as dist
+
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+    return {"value": world * kv_step / (ms_step * 1e-3) / 1e9, "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_step}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,150 @@
+/*
+ * pagedkv.h -- C ABI of libpagedkv: paged KV-cache decode attention and its two
+ * companion kernels, for NVIDIA B200 (sm_100a).
+ *
+ * Pages the operations come from (cited by page title and section):
+ *  [P1] "Paged Attention and Memory Efficiency in Production LLM Serving"
+ *  [P2] "PagedAttention in Production: Boosting LLM Serving Throughput with Paged
+ *       KV Cache"
+ *  [P3] "PagedAttention -- The KV Cache Problem"
+ *
+ * Conventions shared by every call
+ *  - Pointers named *cache*, q, out, k, v, block_tables, context_lens, slot_mapping,
+ *    pairs, workspace and dev_status are DEVICE pointers on the current CUDA device;
+ *    k_caches / v_caches in pa_copy_blocks are HOST arrays holding device pointers.
+ *  - Ownership: the caller owns every buffer, including the workspace.  The library
+ *    allocates no device memory and keeps no state between calls.
+ *  - Synchrony: every call only enqueues work on `stream` (a cudaStream_t; NULL is
+ *    the legacy default stream) and returns; results are ready when the stream is.
+ *  - Errors: arguments are validated on the host before anything is enqueued; a
+ *    failed check returns an error code and enqueues nothing.  A CUDA launch error
+ *    returns PA_ERR_CUDA.  Range violations found on the device (a block id outside
+ *    [0, num_blocks), a slot outside [-1, num_blocks*block_size), a pair outside the
+ *    pool, a context length outside [0, max_blocks_per_seq*block_size]) never fault:
+ *    the offending access is skipped (or the length clamped) and, when dev_status is
+ *    not NULL, the matching PA_DEV_* bit is OR-ed into *dev_status.
+ *  - KV cache layout, per layer, separately for K and V (the pages only say
+ *    "fixed-size blocks"; this layout keeps each (block, kv head) slice contiguous):
+ *        cache[num_blocks][num_kv_heads][block_size][head_dim], 16-bit elements.
+ *  - Supported: head_dim in {64, 128}; block_size in {1, 8, 16, 32};
+ *    num_q_heads % num_kv_heads == 0 with a group of at most 16 q heads per kv head;
+ *    q, out and the caches share one dtype.  Pointers must be 16-byte aligned.
+ */
+#ifndef PAGEDKV_H
+#define PAGEDKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID = 1,      /* null/misaligned pointer, bad size, workspace too small */
+  PA_ERR_UNSUPPORTED = 2,  /* head_dim, block_size, dtype or group size not built */
+  PA_ERR_CUDA = 3          /* a CUDA runtime/driver call or launch failed */
+} pa_status;
+
+typedef enum { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
+
+/* Bits OR-ed into *dev_status by the kernels (see "Errors" above). */
+#define PA_DEV_BAD_BLOCK_ID 0x1
+#define PA_DEV_BAD_SLOT 0x2
+#define PA_DEV_BAD_PAIR 0x4
+#define PA_DEV_BAD_CONTEXT_LEN 0x8
+#define PA_DEV_TIMEOUT 0x10 /* a pipeline wait gave up after ~2 s; outputs are invalid */
+
+/* Library ABI version (major*100 + minor). */
+int pa_version(void);
+
+/* Short English text for a status code (static storage). */
+const char* pa_status_string(pa_status status);
+
+/*
+ * Bytes of workspace pa_decode needs for `num_seqs` sequences on the CURRENT
+ * device (the split schedule is sized by its SM count).  Returns 0 on bad arguments.
+ */
+size_t pa_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim);
+
+/*
+ * pa_decode -- attention of each sequence's newest query token over its paged KV.
+ *
+ * Defined by [P1] "How PagedAttention borrows OS paging": each request keeps a
+ * logical block table that the attention kernel resolves at run time, and the
+ * attention arithmetic itself (dot products, softmax, value-weighted sum) is the
+ * plain one; [P2] "Core Principle" (logical block i of a request -> physical block
+ * block_tables[i]); [P3] "How It Works" (the kernel reads the block table to gather
+ * KV from non-contiguous blocks).
+ *
+ * For sequence s and q head h (kv head kvh = h / (num_q_heads/num_kv_heads)):
+ *   K_s[t] = k_cache[block_tables[s][t / block_size]][kvh][t % block_size][:],
+ *   V_s[t] likewise, for t in [0, context_lens[s]);
+ *   out[s][h][:] = sum_t softmax_t(scale * <q[s][h], K_s[t]>) * V_s[t],
+ * computed with an fp32 online softmax and fp32 accumulation, rounded to the dtype.
+ * context_lens[s] counts every cached token, the newest one included (append runs
+ * first).  A length of 0 gives an all-zero output row.  Block-table entries past
+ * ceil(context_lens[s]/block_size) and cache slots past the last token are never read.
+ *
+ *   out            [num_seqs][num_q_heads][head_dim]            (written)
+ *   q              [num_seqs][num_q_heads][head_dim]
+ *   k_cache/v_cache  layout above, num_blocks blocks
+ *   block_tables   int32 [num_seqs][max_blocks_per_seq]
+ *   context_lens   int32 [num_seqs]
+ *   workspace      >= pa_decode_workspace_bytes(...) bytes, 256-byte aligned; its
+ *                  contents on entry do not matter and are clobbered.
+ *   dev_status     int32, nullable (see "Errors").
+ *
+ * The result is a deterministic function of the logical inputs: it does not depend
+ * on which physical blocks hold the data.
+ */
+pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+                    int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                    int max_blocks_per_seq, int num_blocks, float scale, pa_dtype dtype,
+                    void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                    void* stream);
+
+/*
+ * pa_cache_append -- write the new tokens' K and V into their cache slots.
+ *
+ * Defined by [P1] "How PagedAttention borrows OS paging" (blocks are filled on demand
+ * as decoding proceeds) and [P3] "How It Works" (allocate blocks on demand as tokens
+ * are generated).  For every token i with slot = slot_mapping[i] >= 0:
+ *   k_cache[slot / block_size][h][slot % block_size][:] = k[i][h][:]   for all h,
+ * and the same for v.  A negative slot marks a padding token and is skipped.
+ *
+ *   k, v           [num_tokens][num_kv_heads][head_dim], contiguous
+ *   slot_mapping   int64 [num_tokens]
+ * Two tokens naming the same slot in one call is undefined (one of them wins).
+ */
+pa_status pa_cache_append(void* k_cache, void* v_cache, const void* k, const void* v,
+                          const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
+                          int head_dim, int block_size, int num_blocks, pa_dtype dtype,
+                          int32_t* dev_status, void* stream);
+
+/*
+ * pa_copy_blocks -- the copy-on-write copy of shared blocks.
+ *
+ * Defined by [P1] "How PagedAttention borrows OS paging" (sequences sharing a prefix
+ * point at the same physical blocks; a new block is allocated when one diverges,
+ * as in OS copy-on-write) and [P3] "Why This Matters for Production" (parallel
+ * sampling and beam search share KV blocks copy-on-write).  For every layer l and
+ * pair p: block pairs[p][1] <- block pairs[p][0], byte for byte, in k_caches[l] and
+ * in v_caches[l].
+ *
+ *   k_caches, v_caches  HOST arrays of num_layers device pointers (one pool per layer)
+ *   pairs          device int32 [num_pairs][2] = (src, dst)
+ *   block_bytes    bytes of one block of one pool (num_kv_heads*block_size*head_dim*2),
+ *                  a multiple of 16
+ * A dst that is also a src, or appears twice, in one call is undefined.
+ */
+pa_status pa_copy_blocks(void* const* k_caches, void* const* v_caches, int num_layers,
+                         const int32_t* pairs, int num_pairs, int num_blocks,
+                         size_t block_bytes, int32_t* dev_status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PAGEDKV_H */

@@ -1,0 +1,260 @@
+// api.cu -- the extern "C" entry points of libpagedkv (declared in include/pagedkv.h):
+// argument validation, workspace layout, TMA descriptor encoding, template dispatch
+// and kernel launches.  No device memory is allocated here.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "decode.cuh"
+#include "kv_ops.cuh"
+#include "pagedkv.h"
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int sm_count() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return sms;
+}
+
+struct WsLayout {
+  size_t prefix_off, acc_off, ml_off, total;
+};
+
+// prefix: int32[num_seqs+1]; partial accumulators: float[G*2][16][D];
+// partial (max, sum): float[G*2][16][2].
+WsLayout ws_layout(int num_seqs, int head_dim, int grid) {
+  WsLayout w{};
+  size_t off = align256(sizeof(int32_t) * (size_t)(num_seqs + 1));
+  w.acc_off = off;
+  off = align256(off + sizeof(float) * (size_t)grid * 2 * pkv::kMaxGroup * head_dim);
+  w.ml_off = off;
+  off = align256(off + sizeof(float) * (size_t)grid * 2 * pkv::kMaxGroup * 2);
+  w.total = off;
+  return w;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D view of one pool: rows = num_blocks*kv_heads*block_size, each head_dim elements;
+// box = 64 dims x box_rows rows, 128-byte swizzle, out-of-range rows read as zero.
+bool encode_pool(CUtensorMap* map, const void* base, pa_dtype dtype, int head_dim,
+                 uint64_t rows, int box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
+  cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(map, dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                   2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <typename T, int D, int BS, int NT>
+pa_status launch_decode(const pkv::DecodeArgs& a, const CUtensorMap& mk, const CUtensorMap& mv,
+                        int grid, cudaStream_t stream) {
+  using L = pkv::Layout<D>;
+  auto split = pkv::pa_decode_split_kernel<T, D, BS, NT>;
+  if (cudaFuncSetAttribute(split, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynSmem) !=
+      cudaSuccess)
+    return PA_ERR_CUDA;
+  split<<<grid, pkv::kThreads, L::kDynSmem, stream>>>(a, mk, mv);
+  if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  pkv::pa_decode_combine_kernel<T, D><<<a.num_seqs * a.num_kv_heads, 128, 0, stream>>>(a, grid);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+template <typename T, int D, int BS>
+pa_status dispatch_nt(const pkv::DecodeArgs& a, const CUtensorMap& mk, const CUtensorMap& mv,
+                      int grid, cudaStream_t s) {
+  return a.group <= 8 ? launch_decode<T, D, BS, 1>(a, mk, mv, grid, s)
+                      : launch_decode<T, D, BS, 2>(a, mk, mv, grid, s);
+}
+
+template <typename T, int D>
+pa_status dispatch_bs(int bs, const pkv::DecodeArgs& a, const CUtensorMap& mk,
+                      const CUtensorMap& mv, int grid, cudaStream_t s) {
+  switch (bs) {
+    case 1: return dispatch_nt<T, D, 1>(a, mk, mv, grid, s);
+    case 8: return dispatch_nt<T, D, 8>(a, mk, mv, grid, s);
+    case 16: return dispatch_nt<T, D, 16>(a, mk, mv, grid, s);
+    case 32: return dispatch_nt<T, D, 32>(a, mk, mv, grid, s);
+  }
+  return PA_ERR_UNSUPPORTED;
+}
+
+template <typename T>
+pa_status dispatch_d(int d, int bs, const pkv::DecodeArgs& a, const CUtensorMap& mk,
+                     const CUtensorMap& mv, int grid, cudaStream_t s) {
+  return d == 64 ? dispatch_bs<T, 64>(bs, a, mk, mv, grid, s)
+                 : dispatch_bs<T, 128>(bs, a, mk, mv, grid, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+int pa_version(void) { return 100; }
+
+const char* pa_status_string(pa_status s) {
+  switch (s) {
+    case PA_OK: return "ok";
+    case PA_ERR_INVALID: return "invalid argument";
+    case PA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case PA_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+size_t pa_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim) {
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0) return 0;
+  const int sms = sm_count();
+  if (sms <= 0) return 0;
+  return ws_layout(num_seqs, head_dim, sms * pkv::kCtasPerSm).total;
+}
+
+pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+                    int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                    int max_blocks_per_seq, int num_blocks, float scale, pa_dtype dtype,
+                    void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                    void* stream) {
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0 ||
+      num_blocks <= 0 || !std::isfinite(scale))
+    return PA_ERR_INVALID;
+  if (num_q_heads % num_kv_heads) return PA_ERR_INVALID;
+  if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (block_size != 1 && block_size != 8 && block_size != 16 && block_size != 32)
+    return PA_ERR_UNSUPPORTED;
+  const int group = num_q_heads / num_kv_heads;
+  if (group > pkv::kMaxGroup) return PA_ERR_UNSUPPORTED;
+  if ((long long)num_blocks * num_kv_heads * block_size >= (1ll << 31) ||
+      (long long)max_blocks_per_seq * block_size >= (1ll << 31) ||
+      (long long)num_seqs * num_kv_heads >= (1ll << 31))
+    return PA_ERR_INVALID;
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !workspace)
+    return PA_ERR_INVALID;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      !aligned16(workspace))
+    return PA_ERR_INVALID;
+  const int sms = sm_count();
+  if (sms <= 0) return PA_ERR_CUDA;
+  const int grid = sms * pkv::kCtasPerSm;
+  const WsLayout w = ws_layout(num_seqs, head_dim, grid);
+  if (workspace_bytes < w.total) return PA_ERR_INVALID;
+
+  CUtensorMap mk, mv;
+  std::memset(&mk, 0, sizeof(mk));
+  std::memset(&mv, 0, sizeof(mv));
+  if (block_size != 1) {
+    const uint64_t rows = (uint64_t)num_blocks * num_kv_heads * block_size;
+    const int box_rows = block_size < 16 ? block_size : 16;
+    if (!encode_pool(&mk, k_cache, dtype, head_dim, rows, box_rows) ||
+        !encode_pool(&mv, v_cache, dtype, head_dim, rows, box_rows))
+      return PA_ERR_CUDA;
+  }
+  pkv::DecodeArgs a;
+  a.out = out;
+  a.q = q;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.prefix = reinterpret_cast<int32_t*>(ws + w.prefix_off);
+  a.part_acc = reinterpret_cast<float*>(ws + w.acc_off);
+  a.part_ml = reinterpret_cast<float*>(ws + w.ml_off);
+  a.status = dev_status;
+  a.num_seqs = num_seqs;
+  a.num_q_heads = num_q_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.group = group;
+  a.max_blocks = max_blocks_per_seq;
+  a.num_blocks = num_blocks;
+  a.ctx_cap = max_blocks_per_seq * block_size;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == PA_BF16) return dispatch_d<__nv_bfloat16>(head_dim, block_size, a, mk, mv, grid, st);
+  return dispatch_d<__half>(head_dim, block_size, a, mk, mv, grid, st);
+}
+
+pa_status pa_cache_append(void* k_cache, void* v_cache, const void* k, const void* v,
+                          const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
+                          int head_dim, int block_size, int num_blocks, pa_dtype dtype,
+                          int32_t* dev_status, void* stream) {
+  if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
+    return PA_ERR_INVALID;
+  if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  if ((head_dim * 2) % 16) return PA_ERR_UNSUPPORTED;
+  if (num_tokens == 0) return PA_OK;
+  if (!k_cache || !v_cache || !k || !v || !slot_mapping) return PA_ERR_INVALID;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k) || !aligned16(v))
+    return PA_ERR_INVALID;
+  const int cpr = head_dim * 2 / 16;
+  const long long total = (long long)num_tokens * num_kv_heads * cpr;
+  const int sms = sm_count();
+  if (sms <= 0) return PA_ERR_CUDA;
+  long long blocks = (total + 255) / 256;
+  if (blocks > (long long)sms * 16) blocks = (long long)sms * 16;
+  pkv::pa_cache_append_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), static_cast<const uint4*>(k),
+      static_cast<const uint4*>(v), slot_mapping, num_tokens, num_kv_heads, cpr, block_size,
+      num_blocks, dev_status);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_copy_blocks(void* const* k_caches, void* const* v_caches, int num_layers,
+                         const int32_t* pairs, int num_pairs, int num_blocks, size_t block_bytes,
+                         int32_t* dev_status, void* stream) {
+  if (num_layers < 0 || num_pairs < 0 || num_blocks <= 0 || block_bytes == 0 ||
+      block_bytes % 16)
+    return PA_ERR_INVALID;
+  if (num_layers == 0 || num_pairs == 0) return PA_OK;
+  if (!k_caches || !v_caches || !pairs) return PA_ERR_INVALID;
+  for (int l = 0; l < num_layers; ++l)
+    if (!k_caches[l] || !v_caches[l] || !aligned16(k_caches[l]) || !aligned16(v_caches[l]))
+      return PA_ERR_INVALID;
+  for (int l0 = 0; l0 < num_layers; l0 += pkv::kMaxLayersPerLaunch) {
+    const int n = (num_layers - l0) < pkv::kMaxLayersPerLaunch ? (num_layers - l0)
+                                                               : pkv::kMaxLayersPerLaunch;
+    pkv::LayerPtrs P;
+    std::memset(&P, 0, sizeof(P));
+    for (int i = 0; i < n; ++i) {
+      P.k[i] = static_cast<uint4*>(k_caches[l0 + i]);
+      P.v[i] = static_cast<uint4*>(v_caches[l0 + i]);
+    }
+    dim3 grid((unsigned)num_pairs, (unsigned)(2 * n));
+    pkv::pa_copy_blocks_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        P, pairs, num_blocks, (long long)(block_bytes / 16), dev_status);
+    if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  }
+  return PA_OK;
+}
+
+}  // extern "C"

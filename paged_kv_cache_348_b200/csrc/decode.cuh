@@ -1,0 +1,620 @@
+// decode.cuh -- paged decode attention for sm_100a.
+//
+// What it computes is defined in "Paged Attention and Memory Efficiency in Production
+// LLM Serving", section "How PagedAttention borrows OS paging": the attention kernel
+// resolves each request's block table at run time and the arithmetic is the plain
+// softmax(scale q K^T) V; "PagedAttention -- The KV Cache Problem", section "How It
+// Works": the kernel reads the block table to gather K/V from non-contiguous blocks.
+//
+// Design (B200):
+//  * Work is the set of (sequence, kv head) segments, cut into 16-token units.  The
+//    units of all segments are laid end to end and split into gridDim.x equal
+//    ranges, one per persistent CTA (2 per SM), so a batch with a heavy-tailed
+//    length mix still gives every SM the same number of KV bytes.  A segment that
+//    straddles CTA ranges is finished by the combine kernel (log-sum-exp merge).
+//  * Per CTA: one producer warp walks the CTA's range and streams K/V tiles of 64
+//    tokens into a 3-stage shared-memory ring: for block_size >= 8 with 2-D TMA
+//    tensor copies (128-byte swizzle, box = min(block_size,16) rows x 64 dims) whose
+//    row coordinate is the physical block id read from the block table; for
+//    block_size 1 with 16-byte cp.async copies.  Stages complete on mbarriers.
+//  * Four consumer warps each take one 16-token unit of a stage.  All q heads of
+//    the GQA group share every K/V byte: S^T = K q^T and O^T += V^T P^T run as
+//    m16n8k16 tensor-core MMAs with the tokens (resp. head dims) on M and the q heads
+//    on N, so a group of 8 heads fills N exactly.  Softmax is an fp32 online softmax
+//    in base 2; P is split into a 16-bit high part and a 16-bit residual so the PV
+//    product keeps ~16 mantissa bits.
+//  * Every wait is bounded (2 s); on give-up the CTA sets PA_DEV_TIMEOUT and leaves.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <cstdint>
+#include <type_traits>
+
+#include "ptx.cuh"
+
+namespace pkv {
+
+constexpr int kUnit = 16;                           // tokens per schedule unit
+constexpr int kConsumerWarps = 4;
+constexpr int kUnitsPerStage = kConsumerWarps;      // one unit per consumer warp
+constexpr int kTileTokens = kUnit * kUnitsPerStage; // 64 tokens per stage
+constexpr int kStages = 3;
+constexpr int kThreads = 32 * (1 + kConsumerWarps);
+constexpr int kCtasPerSm = 2;
+constexpr int kMaxGroup = 16;                       // q heads per kv head handled
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+constexpr int DEV_BAD_BLOCK_ID = 0x1;
+constexpr int DEV_BAD_CONTEXT_LEN = 0x8;
+constexpr int DEV_TIMEOUT = 0x10;
+
+enum : int { F_FIRST = 1, F_LAST = 2, F_END = 4, F_COMPLETE = 8 };
+
+struct StageMeta {
+  int seq, kvh, tok0, nunits, ctx, flags, pidx, pad;
+};
+
+struct DecodeArgs {
+  void* out;
+  const void* q;
+  const void* k_cache;          // used directly by the block_size-1 path
+  const void* v_cache;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  float* part_acc;              // [gridDim*2][kMaxGroup][D]
+  float* part_ml;               // [gridDim*2][kMaxGroup][2]  (max, sum) in base 2
+  int32_t* prefix;              // [num_seqs+1] units per kv head, exclusive scan
+  int32_t* status;              // nullable
+  int num_seqs, num_q_heads, num_kv_heads, group, max_blocks, num_blocks, ctx_cap;
+  float scale_log2;             // scale * log2(e)
+};
+
+template <int D>
+struct Layout {
+  static constexpr int kHalves = D / 64;                   // 128-byte swizzled column halves
+  static constexpr int kKvBytes = kHalves * kTileTokens * 128;
+  static constexpr int kQBytes = kMaxGroup * D * 2;
+  static constexpr int kStageBytes = 2 * kKvBytes + kQBytes;
+  static_assert(kStageBytes % 1024 == 0, "stage must keep 1024-byte alignment");
+  static constexpr int kMetaOff = kStages * kStageBytes;
+  static constexpr int kBarOff = kMetaOff + kStages * (int)sizeof(StageMeta);
+  static constexpr int kMlOff = kBarOff + 2 * kStages * 8 + 16;
+  static constexpr int kBytes = kMlOff + kConsumerWarps * kMaxGroup * 8;
+  static constexpr int kDynSmem = kBytes + 1024;           // slack for 1024-byte alignment
+};
+
+__device__ __forceinline__ int clamp_ctx(int c, int cap, int32_t* status) {
+  if (c < 0 || c > cap) {
+    if (status) atomicOr(status, DEV_BAD_CONTEXT_LEN);
+    c = c < 0 ? 0 : cap;
+  }
+  return c;
+}
+
+// Index of the CTA whose unit range [start(c), start(c+1)) holds unit x, where
+// start(c) = floor(c * total / G).
+__device__ __forceinline__ int cta_of(long long x, long long total, int G) {
+  return (int)(((x + 1) * (long long)G + total - 1) / total) - 1;
+}
+__device__ __forceinline__ long long cta_start(int c, long long total, int G) {
+  return (long long)c * total / G;
+}
+
+template <typename T>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  if constexpr (std::is_same_v<T, __nv_bfloat16>) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  } else {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  }
+}
+template <typename T>
+__device__ __forceinline__ float2 unpack2(uint32_t x) {
+  if constexpr (std::is_same_v<T, __nv_bfloat16>) {
+    return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&x));
+  } else {
+    return __half22float2(*reinterpret_cast<__half2*>(&x));
+  }
+}
+template <typename T>
+__device__ __forceinline__ T from_float(float x) {
+  if constexpr (std::is_same_v<T, __nv_bfloat16>) return __float2bfloat16_rn(x);
+  else return __float2half_rn(x);
+}
+
+__device__ __forceinline__ void cp_async_16_zfill(void* dst, const void* src, uint32_t src_bytes,
+                                                  uint64_t policy) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(src_bytes), "l"(policy)
+               : "memory");
+}
+
+// ------------------------------------------------------------------------------------
+// Split pass: every CTA processes its unit range and writes finished rows to `out`,
+// or (max, sum, unnormalised acc) partials for segments it shares with other CTAs.
+// ------------------------------------------------------------------------------------
+template <typename T, int D, int BS, int NT>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    pa_decode_split_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
+                           const __grid_constant__ CUtensorMap tmv) {
+  using L = Layout<D>;
+  constexpr bool kBF16 = std::is_same_v<T, __nv_bfloat16>;
+  constexpr int kFullCount = (BS == 1) ? 33 : 1;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  StageMeta* meta = reinterpret_cast<StageMeta*>(smem + L::kMetaOff);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* empty = full + kStages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kStages);
+  float2* mls = reinterpret_cast<float2*>(smem + L::kMlOff);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&full[i], kFullCount);
+      mbar_init(&empty[i], kConsumerWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (BS != 1 && threadIdx.x == 32) {
+    prefetch_tensormap(&tmk);
+    prefetch_tensormap(&tmv);
+  }
+  __syncthreads();
+
+  const int G = gridDim.x, c = blockIdx.x;
+  const int Hkv = a.num_kv_heads, group = a.group;
+
+  if (warp == 0) {
+    // ============================== producer ==============================
+    const int B = a.num_seqs;
+    // pass 1 over the batch: units per kv head, their exclusive scan (CTA 0 stores it)
+    long long run = 0;
+    for (int base = 0; base < B; base += 32) {
+      const int s = base + lane;
+      int u = 0;
+      if (s < B) u = (clamp_ctx(a.context_lens[s], a.ctx_cap, c == 0 ? a.status : nullptr) +
+                      kUnit - 1) / kUnit;
+      int x = u;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (c == 0 && s < B) a.prefix[s] = (int)(run + x - u);
+      run += __shfl_sync(0xffffffffu, x, 31);
+    }
+    if (c == 0 && lane == 0) a.prefix[B] = (int)run;
+    const long long total = (long long)Hkv * run;
+    const long long start = total ? cta_start(c, total, G) : 0;
+    const long long end = total ? cta_start(c + 1, total, G) : 0;
+
+    // pass 2: the sequence holding unit `start`
+    int s_cur = 0, u_cur = 0, ctx_cur = 0;
+    long long pbase = 0;
+    if (start < end) {
+      long long r2 = 0;
+      for (int base = 0; base < B; base += 32) {
+        const int s = base + lane;
+        int ctx = 0;
+        if (s < B) ctx = clamp_ctx(a.context_lens[s], a.ctx_cap, nullptr);
+        const int u = (ctx + kUnit - 1) / kUnit;
+        int x = u;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, x, o);
+          if (lane >= o) x += y;
+        }
+        const long long lo = (long long)Hkv * (r2 + x - u), hi = (long long)Hkv * (r2 + x);
+        const unsigned hit = __ballot_sync(0xffffffffu, s < B && u > 0 && lo <= start && start < hi);
+        if (hit) {
+          const int src = __ffs(hit) - 1;
+          s_cur = base + src;
+          u_cur = __shfl_sync(0xffffffffu, u, src);
+          ctx_cur = __shfl_sync(0xffffffffu, ctx, src);
+          pbase = __shfl_sync(0xffffffffu, lo, src);
+          break;
+        }
+        r2 += __shfl_sync(0xffffffffu, x, 31);
+      }
+    }
+
+    const uint64_t policy = policy_evict_first();
+    const int rows_total = a.num_blocks * Hkv * BS;
+    int st = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    long long x = start;
+    while (ok && x < end) {
+      while (x >= pbase + (long long)Hkv * u_cur) {   // next sequence with units
+        pbase += (long long)Hkv * u_cur;
+        ++s_cur;
+        ctx_cur = clamp_ctx(a.context_lens[s_cur], a.ctx_cap, nullptr);
+        u_cur = (ctx_cur + kUnit - 1) / kUnit;
+      }
+      const int kvh = (int)((x - pbase) / u_cur);
+      const long long seg0 = pbase + (long long)kvh * u_cur, seg1 = seg0 + u_cur;
+      const long long pe = seg1 < end ? seg1 : end;
+      const bool complete = seg0 >= start && seg1 <= end;
+      const int pidx = c * 2 + (start < seg0 ? 1 : 0);
+      const int32_t* trow = a.block_tables + (long long)s_cur * a.max_blocks;
+      for (long long tu = x; tu < pe; tu += kUnitsPerStage) {
+        const int nun = (int)((pe - tu) < kUnitsPerStage ? (pe - tu) : kUnitsPerStage);
+        const int tok0 = (int)(tu - seg0) * kUnit;
+        const int flags = (tu == x ? F_FIRST : 0) | (tu + kUnitsPerStage >= pe ? F_LAST : 0) |
+                          (complete ? F_COMPLETE : 0);
+        if (!mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        uint8_t* sK = smem + st * L::kStageBytes;
+        uint8_t* sV = sK + L::kKvBytes;
+        uint8_t* sQ = sV + L::kKvBytes;
+        const uint32_t qbytes = (flags & F_FIRST) ? (uint32_t)(group * D * 2) : 0u;
+        if (lane == 0) {
+          meta[st] = StageMeta{s_cur, kvh, tok0, nun, ctx_cur, flags, pidx, 0};
+        }
+        if constexpr (BS != 1) {
+          constexpr int H = BS < 16 ? BS : 16;     // rows per TMA box
+          constexpr int BPU = kUnit / H;           // boxes per unit and column half
+          constexpr int kBoxBytes = H * 128;
+          uint32_t bytes = qbytes;
+          for (int j = 0; j < nun; ++j) {
+            const int rem = ctx_cur - (tok0 + j * kUnit);
+            const int nb = (rem + H - 1) / H;
+            bytes += (uint32_t)((nb < BPU ? nb : BPU) * kBoxBytes * L::kHalves * 2);
+          }
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&full[st], bytes);
+            if (qbytes)
+              bulk_load(sQ,
+                        static_cast<const T*>(a.q) +
+                            ((long long)s_cur * a.num_q_heads + (long long)kvh * group) * D,
+                        qbytes, &full[st]);
+          }
+          __syncwarp();
+          const int nbox = nun * BPU * L::kHalves * 2;
+          for (int i = lane; i < nbox; i += 32) {
+            const int kv = i & 1;
+            const int hf = (i >> 1) % L::kHalves;
+            const int jb = (i >> 1) / L::kHalves;
+            const int j = jb / BPU, b = jb % BPU;
+            const int t = tok0 + j * kUnit + b * H;
+            if (t < ctx_cur) {
+              const int blk = trow[t / BS];
+              int y;
+              if ((unsigned)blk < (unsigned)a.num_blocks) {
+                y = (blk * Hkv + kvh) * BS + (t % BS);
+              } else {
+                if (a.status) atomicOr(a.status, DEV_BAD_BLOCK_ID);
+                y = rows_total;                      // out of range: TMA fills zeros
+              }
+              uint8_t* dst = (kv ? sV : sK) + hf * (kTileTokens * 128) + (j * kUnit + b * H) * 128;
+              tma_load_2d(dst, kv ? &tmv : &tmk, &full[st], hf * 64, y, policy);
+            }
+          }
+        } else {
+          // block_size 1: every token is its own block; 16-byte cp.async with the same
+          // 128-byte swizzle the TMA path produces.
+          constexpr int CPR = D * 2 / 16;          // 16-byte chunks per row
+          constexpr int RPI = 32 / CPR;            // rows per warp instruction
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&full[st], qbytes);
+            if (qbytes)
+              bulk_load(sQ,
+                        static_cast<const T*>(a.q) +
+                            ((long long)s_cur * a.num_q_heads + (long long)kvh * group) * D,
+                        qbytes, &full[st]);
+          }
+          const int ch = lane % CPR, hf = ch >> 3, cc = ch & 7;
+          for (int r0 = 0; r0 < nun * kUnit; r0 += RPI) {
+            const int r = r0 + lane / CPR;
+            const int t = tok0 + r;
+            if (t < ctx_cur) {
+              const int blk = trow[t];
+              uint32_t sz = 16;
+              long long row = 0;
+              if ((unsigned)blk < (unsigned)a.num_blocks) {
+                row = (long long)blk * Hkv + kvh;
+              } else {
+                if (a.status) atomicOr(a.status, DEV_BAD_BLOCK_ID);
+                sz = 0;                                // zero fill, no read
+              }
+              const long long off = row * D + ch * 8;
+              const int soff = hf * (kTileTokens * 128) + r * 128 + ((cc ^ (r & 7)) << 4);
+              cp_async_16_zfill(sK + soff, static_cast<const T*>(a.k_cache) + off, sz, policy);
+              cp_async_16_zfill(sV + soff, static_cast<const T*>(a.v_cache) + off, sz, policy);
+            }
+          }
+          cp_async_mbar_arrive_noinc(&full[st]);
+        }
+        if (++st == kStages) {
+          st = 0;
+          ph ^= 1u;
+        }
+      }
+      x = pe;
+    }
+    if (ok) ok = mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, kWaitLimitNs);
+    if (ok) {
+      if (lane == 0) meta[st].flags = F_END;
+      __syncwarp();
+      if (BS == 1 || lane == 0) mbar_arrive(&full[st]);
+      if (BS == 1 && lane == 0) mbar_arrive(&full[st]);
+    } else {
+      if (lane == 0) {
+        *abort_flag = 1;
+        if (a.status) atomicOr(a.status, DEV_TIMEOUT);
+      }
+    }
+    // drain: nothing this warp issued may still be landing when the CTA exits
+    if constexpr (BS == 1) asm volatile("cp.async.wait_all;" ::: "memory");
+    return;
+  }
+
+  // ============================== consumers ==============================
+  const int cw = warp - 1;
+  const int gid = lane >> 2, tig = lane & 3;
+  constexpr int KS = D / 16;            // k-steps of QK, m-tiles of PV
+  constexpr int NREG = KS * NT * 4;     // O^T accumulator registers per thread
+  float o[KS][NT][4];
+  float m[NT][2], l[NT][2];
+  uint32_t qf[KS][NT][2];
+#pragma unroll
+  for (int i = 0; i < KS; ++i)
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      qf[i][n][0] = qf[i][n][1] = 0u;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[i][n][e] = 0.f;
+    }
+#pragma unroll
+  for (int n = 0; n < NT; ++n) m[n][0] = m[n][1] = -INFINITY, l[n][0] = l[n][1] = 0.f;
+
+  int st = 0;
+  uint32_t ph = 0;
+  for (;;) {
+    if (!mbar_wait_bounded(&full[st], ph, abort_flag, kWaitLimitNs)) {
+      if (lane == 0) {
+        *abort_flag = 1;
+        if (a.status) atomicOr(a.status, DEV_TIMEOUT);
+      }
+      break;
+    }
+    const StageMeta mt = meta[st];
+    if (mt.flags & F_END) break;
+    uint8_t* sK = smem + st * L::kStageBytes;
+    uint8_t* sV = sK + L::kKvBytes;
+    const uint8_t* sQ = sV + L::kKvBytes;
+    if (mt.flags & F_FIRST) {
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        const int h = n * 8 + gid;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          uint32_t b0 = 0u, b1 = 0u;
+          if (h < group) {
+            const uint32_t* qrow = reinterpret_cast<const uint32_t*>(sQ + h * D * 2);
+            b0 = qrow[(ks * 16 + 2 * tig) >> 1];
+            b1 = qrow[(ks * 16 + 8 + 2 * tig) >> 1];
+          }
+          qf[ks][n][0] = b0;
+          qf[ks][n][1] = b1;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) o[ks][n][e] = 0.f;
+        }
+        m[n][0] = m[n][1] = -INFINITY;
+        l[n][0] = l[n][1] = 0.f;
+      }
+    }
+    if (cw < mt.nunits) {
+      const int t0 = mt.tok0 + cw * kUnit;
+      const int valid = (mt.ctx - t0) < kUnit ? (mt.ctx - t0) : kUnit;
+      const uint32_t kbase = smem_u32(sK), vbase = smem_u32(sV);
+      // ---- S^T[16 tokens][8*NT heads] = K_unit . q^T
+      float sacc[NT][4];
+#pragma unroll
+      for (int n = 0; n < NT; ++n) sacc[n][0] = sacc[n][1] = sacc[n][2] = sacc[n][3] = 0.f;
+      {
+        const int j = lane >> 3, i = lane & 7;
+        const int r = cw * kUnit + (j & 1) * 8 + i;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          const int d = ks * 16 + (j >> 1) * 8;
+          const uint32_t addr =
+              kbase + (d >> 6) * (kTileTokens * 128) + r * 128 + ((((d & 63) >> 3) ^ (r & 7)) << 4);
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(addr, a0, a1, a2, a3);
+#pragma unroll
+          for (int n = 0; n < NT; ++n) mma16816<kBF16>(sacc[n], a0, a1, a2, a3, qf[ks][n][0], qf[ks][n][1]);
+        }
+      }
+      // ---- online softmax (base 2) per head column
+      uint32_t bhi[NT][2], blo[NT][2];
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        float x[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int row = gid + (e >= 2 ? 8 : 0);
+          x[e] = row < valid ? sacc[n][e] * a.scale_log2 : -INFINITY;
+        }
+        float alpha[2], p[4];
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          float mx = fmaxf(x[cc], x[cc + 2]);
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+          const float mnew = fmaxf(m[n][cc], mx);
+          alpha[cc] = ex2(m[n][cc] - mnew);
+          m[n][cc] = mnew;
+          p[cc] = ex2(x[cc] - mnew);
+          p[cc + 2] = ex2(x[cc + 2] - mnew);
+          l[n][cc] = l[n][cc] * alpha[cc] + p[cc] + p[cc + 2];
+        }
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          o[ks][n][0] *= alpha[0];
+          o[ks][n][1] *= alpha[1];
+          o[ks][n][2] *= alpha[0];
+          o[ks][n][3] *= alpha[1];
+        }
+        const uint32_t h01 = pack2<T>(p[0], p[1]), h23 = pack2<T>(p[2], p[3]);
+        const float2 f01 = unpack2<T>(h01), f23 = unpack2<T>(h23);
+        const uint32_t l01 = pack2<T>(p[0] - f01.x, p[1] - f01.y);
+        const uint32_t l23 = pack2<T>(p[2] - f23.x, p[3] - f23.y);
+        bhi[n][0] = movmatrix_t(h01);
+        bhi[n][1] = movmatrix_t(h23);
+        blo[n][0] = movmatrix_t(l01);
+        blo[n][1] = movmatrix_t(l23);
+      }
+      // ---- O^T[D][8*NT] += V_unit^T . P^T
+      uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;   // token masks for V rows >= valid
+      if (valid < kUnit) {
+        const int t_a = 2 * tig, t_b = 8 + 2 * tig;
+        mlo = (t_a < valid ? 0x0000ffffu : 0u) | (t_a + 1 < valid ? 0xffff0000u : 0u);
+        mhi = (t_b < valid ? 0x0000ffffu : 0u) | (t_b + 1 < valid ? 0xffff0000u : 0u);
+      }
+      {
+        const int j = lane >> 3, i = lane & 7;
+        const int r = cw * kUnit + (j >> 1) * 8 + i;
+#pragma unroll
+        for (int mtile = 0; mtile < KS; ++mtile) {
+          const int d = mtile * 16 + (j & 1) * 8;
+          const uint32_t addr =
+              vbase + (d >> 6) * (kTileTokens * 128) + r * 128 + ((((d & 63) >> 3) ^ (r & 7)) << 4);
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_t(addr, a0, a1, a2, a3);
+          a0 &= mlo;
+          a1 &= mlo;
+          a2 &= mhi;
+          a3 &= mhi;
+#pragma unroll
+          for (int n = 0; n < NT; ++n) {
+            mma16816<kBF16>(o[mtile][n], a0, a1, a2, a3, bhi[n][0], bhi[n][1]);
+            mma16816<kBF16>(o[mtile][n], a0, a1, a2, a3, blo[n][0], blo[n][1]);
+          }
+        }
+      }
+    }
+    if (mt.flags & F_LAST) {
+      // ---- merge the four warps' (m, l, O) for this segment portion
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          float v = l[n][cc];
+          v += __shfl_xor_sync(0xffffffffu, v, 4);
+          v += __shfl_xor_sync(0xffffffffu, v, 8);
+          v += __shfl_xor_sync(0xffffffffu, v, 16);
+          l[n][cc] = v;
+        }
+      named_bar_sync(1, 32 * kConsumerWarps);      // all warps are done with this stage's K/V
+      float* scr = reinterpret_cast<float*>(sK);   // K and V tiles reused as scratch
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks)
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            scr[(cw * NREG + (ks * NT + n) * 4 + e) * 32 + lane] = o[ks][n][e];
+      if (gid == 0) {
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc)
+            mls[cw * kMaxGroup + n * 8 + 2 * tig + cc] = make_float2(m[n][cc], l[n][cc]);
+      }
+      named_bar_sync(1, 32 * kConsumerWarps);
+      const int tid = cw * 32 + lane;
+      const bool complete = mt.flags & F_COMPLETE;
+      T* outp = static_cast<T*>(a.out) +
+                ((long long)mt.seq * a.num_q_heads + (long long)mt.kvh * group) * D;
+      for (int pi = tid; pi < NREG * 32; pi += 32 * kConsumerWarps) {
+        const int r = pi >> 5, ln = pi & 31;
+        const int e = r & 3, n = (r >> 2) % NT, mtile = (r >> 2) / NT;
+        const int d = mtile * 16 + (ln >> 2) + (e >= 2 ? 8 : 0);
+        const int h = n * 8 + 2 * (ln & 3) + (e & 1);
+        if (h >= group) continue;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, mls[w * kMaxGroup + h].x);
+        float Lsum = 0.f, acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          const float2 ml = mls[w * kMaxGroup + h];
+          const float sc = ml.x == -INFINITY ? 0.f : ex2(ml.x - M);
+          Lsum += ml.y * sc;
+          acc += scr[(w * NREG + r) * 32 + ln] * sc;
+        }
+        if (complete) {
+          outp[h * D + d] = from_float<T>(acc / Lsum);
+        } else {
+          a.part_acc[((long long)mt.pidx * kMaxGroup + h) * D + d] = acc;
+          if (d == 0) {
+            a.part_ml[((long long)mt.pidx * kMaxGroup + h) * 2 + 0] = M;
+            a.part_ml[((long long)mt.pidx * kMaxGroup + h) * 2 + 1] = Lsum;
+          }
+        }
+      }
+      fence_proxy_async_smem();   // generic writes above precede the next TMA fill
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[st]);
+    if (++st == kStages) {
+      st = 0;
+      ph ^= 1u;
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------
+// Combine pass: for every segment split over several CTAs, merge the partials with a
+// log-sum-exp reduction in CTA order; also writes the zero rows of empty sequences.
+// ------------------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(128) pa_decode_combine_kernel(const DecodeArgs a, int G) {
+  const int Hkv = a.num_kv_heads, group = a.group;
+  const int s = blockIdx.x / Hkv, kvh = blockIdx.x % Hkv;
+  const int ctx = clamp_ctx(a.context_lens[s], a.ctx_cap, nullptr);
+  const int u = (ctx + kUnit - 1) / kUnit;
+  T* outp = static_cast<T*>(a.out) + ((long long)s * a.num_q_heads + (long long)kvh * group) * D;
+  if (u == 0) {
+    for (int i = threadIdx.x; i < group * D; i += blockDim.x) outp[i] = from_float<T>(0.f);
+    return;
+  }
+  const long long total = (long long)Hkv * a.prefix[a.num_seqs];
+  const long long seg0 = (long long)Hkv * a.prefix[s] + (long long)kvh * u;
+  const int cf = cta_of(seg0, total, G), cl = cta_of(seg0 + u - 1, total, G);
+  if (cf == cl) return;   // finished by a single CTA in the split pass
+  for (int i = threadIdx.x; i < group * D; i += blockDim.x) {
+    const int h = i / D, d = i % D;
+    float M = -INFINITY;
+    for (int cc = cf; cc <= cl; ++cc) {
+      const long long st0 = cta_start(cc, total, G);
+      if (st0 == cta_start(cc + 1, total, G)) continue;   // empty range
+      const int pidx = cc * 2 + (st0 < seg0 ? 1 : 0);
+      M = fmaxf(M, a.part_ml[((long long)pidx * kMaxGroup + h) * 2]);
+    }
+    float Lsum = 0.f, acc = 0.f;
+    for (int cc = cf; cc <= cl; ++cc) {
+      const long long st0 = cta_start(cc, total, G);
+      if (st0 == cta_start(cc + 1, total, G)) continue;
+      const int pidx = cc * 2 + (st0 < seg0 ? 1 : 0);
+      const float mp = a.part_ml[((long long)pidx * kMaxGroup + h) * 2];
+      const float sc = mp == -INFINITY ? 0.f : ex2(mp - M);
+      Lsum += a.part_ml[((long long)pidx * kMaxGroup + h) * 2 + 1] * sc;
+      acc += a.part_acc[((long long)pidx * kMaxGroup + h) * D + d] * sc;
+    }
+    outp[h * D + d] = from_float<T>(acc / Lsum);
+  }
+}
+
+}  // namespace pkv

@@ -1,0 +1,67 @@
+// kv_ops.cuh -- cache append (slot scatter) and copy-on-write block copy for sm_100a.
+// Both are pure byte movement: 16-byte vector loads/stores, consecutive threads on
+// consecutive 16-byte chunks of a row so every warp access is coalesced.
+#pragma once
+#include <cstdint>
+
+namespace pkv {
+
+constexpr int DEV_BAD_SLOT = 0x2;
+constexpr int DEV_BAD_PAIR = 0x4;
+constexpr int kMaxLayersPerLaunch = 128;
+
+// "Paged Attention and Memory Efficiency in Production LLM Serving", section "How
+// PagedAttention borrows OS paging": blocks are filled on demand as decoding proceeds.
+// Token i with slot s >= 0 lands at block s / block_size, offset s % block_size.
+__global__ void __launch_bounds__(256)
+    pa_cache_append_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
+                           const uint4* __restrict__ k, const uint4* __restrict__ v,
+                           const int64_t* __restrict__ slot_mapping, int num_tokens, int Hkv,
+                           int chunks_per_row, int block_size, int num_blocks,
+                           int32_t* status) {
+  const long long total = (long long)num_tokens * Hkv * chunks_per_row;
+  const long long limit = (long long)num_blocks * block_size;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int ch = (int)(i % chunks_per_row);
+    const long long rh = i / chunks_per_row;     // (token, kv head)
+    const int h = (int)(rh % Hkv);
+    const long long tok = rh / Hkv;
+    const long long slot = slot_mapping[tok];
+    if (slot < 0) continue;                      // padding token
+    if (slot >= limit) {
+      if (status && ch == 0) atomicOr(status, DEV_BAD_SLOT);
+      continue;
+    }
+    const long long b = slot / block_size, off = slot % block_size;
+    const long long dst = ((b * Hkv + h) * block_size + off) * chunks_per_row + ch;
+    k_cache[dst] = k[i];
+    v_cache[dst] = v[i];
+  }
+}
+
+struct LayerPtrs {
+  uint4* k[kMaxLayersPerLaunch];
+  uint4* v[kMaxLayersPerLaunch];
+};
+
+// "Paged Attention and Memory Efficiency in Production LLM Serving", section "How
+// PagedAttention borrows OS paging": a sequence that diverges from a shared prefix gets
+// a new block (copy-on-write).  grid = (pairs, layers * 2 pools).
+__global__ void __launch_bounds__(256)
+    pa_copy_blocks_kernel(const __grid_constant__ LayerPtrs P, const int32_t* __restrict__ pairs,
+                          int num_blocks, long long chunks_per_block, int32_t* status) {
+  const int p = blockIdx.x;
+  const int layer = blockIdx.y >> 1, pool = blockIdx.y & 1;
+  const int src = pairs[2 * p], dst = pairs[2 * p + 1];
+  if ((unsigned)src >= (unsigned)num_blocks || (unsigned)dst >= (unsigned)num_blocks) {
+    if (status && threadIdx.x == 0) atomicOr(status, DEV_BAD_PAIR);
+    return;
+  }
+  uint4* base = pool ? P.v[layer] : P.k[layer];
+  const uint4* s = base + (long long)src * chunks_per_block;
+  uint4* d = base + (long long)dst * chunks_per_block;
+  for (long long i = threadIdx.x; i < chunks_per_block; i += blockDim.x) d[i] = s[i];
+}
+
+}  // namespace pkv

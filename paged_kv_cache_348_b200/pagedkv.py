@@ -1,0 +1,176 @@
+"""ctypes binding of libpagedkv (the C ABI in include/pagedkv.h).
+
+Argument marshalling only: shapes are read from torch tensors, pointers and the
+current CUDA stream are passed through, and every step runs in the CUDA library.
+There is no fallback: if ``libpagedkv.so`` is missing or fails to load, every call
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpagedkv.so")
+
+PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_CUDA = 0, 1, 2, 3
+PA_F16, PA_BF16 = 0, 1
+DEV_BAD_BLOCK_ID, DEV_BAD_SLOT, DEV_BAD_PAIR, DEV_BAD_CONTEXT_LEN, DEV_TIMEOUT = (
+    0x1, 0x2, 0x4, 0x8, 0x10)
+
+# every symbol include/pagedkv.h declares
+EXPORTS = ("pa_version", "pa_status_string", "pa_decode_workspace_bytes", "pa_decode",
+           "pa_cache_append", "pa_copy_blocks")
+
+_lib = None
+_lock = threading.Lock()
+
+
+class PagedKVError(RuntimeError):
+    pass
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(path):
+            raise PagedKVError("libpagedkv.so not found at %s: build it with "
+                               "`python paged_kv_cache_348_b200/build.py`" % path)
+        L = ctypes.CDLL(path)
+        P, i32, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        L.pa_version.restype = i32
+        L.pa_version.argtypes = []
+        L.pa_status_string.restype = ctypes.c_char_p
+        L.pa_status_string.argtypes = [i32]
+        L.pa_decode_workspace_bytes.restype = sz
+        L.pa_decode_workspace_bytes.argtypes = [i32, i32, i32, i32]
+        L.pa_decode.restype = i32
+        L.pa_decode.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, f32, i32,
+                                P, sz, P, P]
+        L.pa_cache_append.restype = i32
+        L.pa_cache_append.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, P, P]
+        L.pa_copy_blocks.restype = i32
+        L.pa_copy_blocks.argtypes = [P, P, i32, P, i32, i32, sz, P, P]
+        _lib = L
+        return L
+
+
+def _check(rc: int, what: str):
+    if rc != PA_OK:
+        msg = load().pa_status_string(rc).decode()
+        raise PagedKVError("%s failed: %s (%d)" % (what, msg, rc))
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float16:
+        return PA_F16
+    if t.dtype == torch.bfloat16:
+        return PA_BF16
+    raise PagedKVError("unsupported dtype %s" % t.dtype)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _need(t: torch.Tensor, name: str, dtype=None, ndim=None):
+    if not t.is_cuda:
+        raise PagedKVError("%s must be a CUDA tensor" % name)
+    if not t.is_contiguous():
+        raise PagedKVError("%s must be contiguous" % name)
+    if dtype is not None and t.dtype != dtype:
+        raise PagedKVError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if ndim is not None and t.dim() != ndim:
+        raise PagedKVError("%s must have %d dims" % (name, ndim))
+
+
+def pa_version() -> int:
+    return load().pa_version()
+
+
+def pa_decode_workspace_bytes(num_seqs: int, num_q_heads: int, num_kv_heads: int,
+                              head_dim: int) -> int:
+    return int(load().pa_decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim))
+
+
+def new_workspace(num_seqs, num_q_heads, num_kv_heads, head_dim, device=None) -> torch.Tensor:
+    n = pa_decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim)
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def new_status(device=None) -> torch.Tensor:
+    return torch.zeros(1, dtype=torch.int32, device=device or "cuda")
+
+
+def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale: float, workspace,
+              status=None, stream=None):
+    """out[B,Hq,D] <- paged decode attention (see pa_decode in include/pagedkv.h)."""
+    _need(q, "q", ndim=3)
+    _need(out, "out", dtype=q.dtype, ndim=3)
+    _need(k_cache, "k_cache", dtype=q.dtype, ndim=4)
+    _need(v_cache, "v_cache", dtype=q.dtype, ndim=4)
+    _need(block_tables, "block_tables", dtype=torch.int32, ndim=2)
+    _need(context_lens, "context_lens", dtype=torch.int32, ndim=1)
+    _need(workspace, "workspace")
+    B, Hq, D = q.shape
+    N, Hkv, bs, D2 = k_cache.shape
+    if out.shape != q.shape or D2 != D or v_cache.shape != k_cache.shape or \
+            block_tables.shape[0] != B or context_lens.shape[0] != B:
+        raise PagedKVError("pa_decode: inconsistent shapes")
+    rc = load().pa_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                          _ptr(context_lens), B, Hq, Hkv, D, bs, block_tables.shape[1], N,
+                          float(scale), _dtype_code(q), _ptr(workspace),
+                          workspace.numel() * workspace.element_size(), _ptr(status),
+                          _stream(stream))
+    _check(rc, "pa_decode")
+    return out
+
+
+def pa_cache_append(k_cache, v_cache, k, v, slot_mapping, status=None, stream=None):
+    """Scatter k/v [T,Hkv,D] into the pools at slot_mapping (int64 [T])."""
+    _need(k_cache, "k_cache", ndim=4)
+    _need(v_cache, "v_cache", dtype=k_cache.dtype, ndim=4)
+    _need(k, "k", dtype=k_cache.dtype, ndim=3)
+    _need(v, "v", dtype=k_cache.dtype, ndim=3)
+    _need(slot_mapping, "slot_mapping", dtype=torch.int64, ndim=1)
+    N, Hkv, bs, D = k_cache.shape
+    T = k.shape[0]
+    if v_cache.shape != k_cache.shape or k.shape != (T, Hkv, D) or v.shape != k.shape or \
+            slot_mapping.shape[0] != T:
+        raise PagedKVError("pa_cache_append: inconsistent shapes")
+    rc = load().pa_cache_append(_ptr(k_cache), _ptr(v_cache), _ptr(k), _ptr(v), _ptr(slot_mapping),
+                                T, Hkv, D, bs, N, _dtype_code(k), _ptr(status), _stream(stream))
+    _check(rc, "pa_cache_append")
+
+
+def pa_copy_blocks(k_caches, v_caches, pairs, status=None, stream=None):
+    """Copy block pairs[:,0] -> pairs[:,1] in every layer's K and V pool."""
+    L = len(k_caches)
+    if L != len(v_caches) or L == 0:
+        raise PagedKVError("pa_copy_blocks: need the same non-zero number of K and V pools")
+    shape, dt = k_caches[0].shape, k_caches[0].dtype
+    for i, c in enumerate(list(k_caches) + list(v_caches)):
+        _need(c, "cache[%d]" % i, dtype=dt, ndim=4)
+        if c.shape != shape:
+            raise PagedKVError("pa_copy_blocks: all pools must have one shape")
+    _need(pairs, "pairs", dtype=torch.int32, ndim=2)
+    if pairs.shape[1] != 2:
+        raise PagedKVError("pairs must be [n, 2]")
+    kp = (ctypes.c_void_p * L)(*[c.data_ptr() for c in k_caches])
+    vp = (ctypes.c_void_p * L)(*[c.data_ptr() for c in v_caches])
+    block_bytes = shape[1] * shape[2] * shape[3] * k_caches[0].element_size()
+    rc = load().pa_copy_blocks(kp, vp, L, _ptr(pairs), pairs.shape[0], shape[0], block_bytes,
+                               _ptr(status), _stream(stream))
+    _check(rc, "pa_copy_blocks")

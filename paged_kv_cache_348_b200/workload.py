@@ -1,0 +1,171 @@
+"""Device-resident decode batches for the measured workloads.
+
+Builds, from the seeded generators in ``inputs`` and the host ``BlockManager``:
+per-layer K/V pools, one block table for all layers, context lengths, the newest
+token's q / k / v per layer and its slot mapping, output buffers, the decode
+workspace and a device status word.
+
+A decode step (``run_step``) is, for every layer: pa_cache_append of the newest
+token of every sequence, then pa_decode over all cached tokens (the newest one
+included).  Copy-on-write pairs, when the block manager produced some, are copied
+with one pa_copy_blocks call over all layers first.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+import torch
+
+from . import inputs
+from . import pagedkv as pk
+from .block_manager import BlockManager
+
+
+@dataclasses.dataclass
+class DecodeBatch:
+    w: inputs.Workload
+    block_size: int
+    bm: BlockManager
+    sids: list
+    num_blocks: int
+    k_caches: list
+    v_caches: list
+    block_tables: torch.Tensor
+    context_lens: torch.Tensor
+    slot_mapping: torch.Tensor
+    q: list
+    k_new: list
+    v_new: list
+    out: list
+    workspace: torch.Tensor
+    status: torch.Tensor
+    cow_pairs: torch.Tensor | None
+    scale: float
+
+    @property
+    def layers(self) -> int:
+        return len(self.k_caches)
+
+    def kv_bytes_per_step(self) -> int:
+        """Algorithmic KV bytes one decode step reads: every cached token of every
+        sequence, K and V, all kv heads, all layers."""
+        w = self.w
+        ctx = self.context_lens.cpu().numpy().astype(np.int64)
+        return int(ctx.sum()) * w.num_kv_heads * w.head_dim * 2 * 2 * self.layers
+
+    def unique_kv_bytes_per_step(self) -> int:
+        """KV bytes with every shared block counted once (blocks x fill)."""
+        seen = {}
+        for s in self.sids:
+            n = self.bm.context_len(s)
+            for i, b in enumerate(self.bm.table(s)):
+                seen[b] = max(seen.get(b, 0), min(self.block_size, n - i * self.block_size))
+        w = self.w
+        return sum(seen.values()) * w.num_kv_heads * w.head_dim * 2 * 2 * self.layers
+
+
+def _pool_size(w: inputs.Workload, need: int) -> int:
+    return w.pool_blocks if w.pool_blocks else int(math.ceil(w.pool_factor * need))
+
+
+def _alloc_layers(w, N, bs, layers, device, seed):
+    k, v = [], []
+    for l in range(layers):
+        k.append(inputs.randn((N, w.num_kv_heads, bs, w.head_dim), w.dtype, seed, device,
+                              stream=1000 + 2 * l))
+        v.append(inputs.randn((N, w.num_kv_heads, bs, w.head_dim), w.dtype, seed, device,
+                              stream=1001 + 2 * l))
+    return k, v
+
+
+def _finish(w, bs, bm, sids, N, layers, device, cow_pairs=None) -> DecodeBatch:
+    B = len(sids)
+    k_caches, v_caches = _alloc_layers(w, N, bs, layers, device, w.seed)
+    tables = torch.from_numpy(bm.block_tables(sids)).to(device)
+    ctx = torch.from_numpy(bm.context_lens(sids)).to(device)
+    slots = torch.tensor([bm.slot_of(s, bm.context_len(s) - 1) for s in sids], dtype=torch.int64,
+                         device=device)
+    q, kn, vn, out = [], [], [], []
+    for l in range(layers):
+        q.append(inputs.randn((B, w.num_q_heads, w.head_dim), w.dtype, w.seed, device,
+                              stream=5000 + 3 * l))
+        kn.append(inputs.randn((B, w.num_kv_heads, w.head_dim), w.dtype, w.seed, device,
+                               stream=5001 + 3 * l))
+        vn.append(inputs.randn((B, w.num_kv_heads, w.head_dim), w.dtype, w.seed, device,
+                               stream=5002 + 3 * l))
+        out.append(torch.empty((B, w.num_q_heads, w.head_dim), dtype=inputs.torch_dtype(w.dtype),
+                               device=device))
+    ws = pk.new_workspace(B, w.num_q_heads, w.num_kv_heads, w.head_dim, device)
+    st = pk.new_status(device)
+    pairs = None
+    if cow_pairs:
+        pairs = torch.tensor(cow_pairs, dtype=torch.int32, device=device).reshape(-1, 2)
+    return DecodeBatch(w, bs, bm, sids, N, k_caches, v_caches, tables, ctx, slots, q, kn, vn, out,
+                       ws, st, pairs, 1.0 / math.sqrt(w.head_dim))
+
+
+def build(w: inputs.Workload, device="cuda", block_size: int | None = None,
+          layers: int | None = None) -> DecodeBatch:
+    """Independent sequences (every workload but the shared-prefix one)."""
+    bs = block_size or w.block_size
+    ctx = inputs.context_lens(w)
+    need = int(sum(-(-int(c) // bs) for c in ctx))
+    N = _pool_size(w, need)
+    bm = BlockManager(N, bs, inputs.pool_order(N, w.seed))
+    sids = [bm.allocate(int(c)) for c in ctx]
+    return _finish(w, bs, bm, sids, N, layers or w.layers, device)
+
+
+def build_prefix_decode(w: inputs.Workload = inputs.PREFIX, device="cuda") -> DecodeBatch:
+    """Shared-prefix parallel sampling, decode phase: per prompt a 2048-token prefix
+    held once (refcount 8) and 0..512 private tokens per sample."""
+    bs = w.block_size
+    ctx = inputs.context_lens(w)                       # prefix + private, per sample
+    need = inputs.PREFIX_PROMPTS * (inputs.PREFIX_LEN // bs) + int(
+        sum(-(-int(c - inputs.PREFIX_LEN) // bs) for c in ctx))
+    N = _pool_size(w, need)
+    bm = BlockManager(N, bs, inputs.pool_order(N, w.seed))
+    sids = []
+    for p in range(inputs.PREFIX_PROMPTS):
+        root = bm.allocate(inputs.PREFIX_LEN)
+        kids = [root] + [bm.fork(root) for _ in range(inputs.PREFIX_SAMPLES - 1)]
+        for j, sid in enumerate(kids):
+            for _ in range(int(ctx[p * inputs.PREFIX_SAMPLES + j]) - inputs.PREFIX_LEN):
+                slot, cow = bm.append_token(sid)
+                assert cow is None                     # prefix is block aligned
+            sids.append(sid)
+    return _finish(w, bs, bm, sids, N, w.layers, device)
+
+
+def build_prefix_fork(w: inputs.Workload = inputs.PREFIX, device="cuda") -> DecodeBatch:
+    """Shared-prefix fork phase: each prompt's shared region is 2048 + t tokens
+    (t in 1..15), so its last block is partial and shared by 8 samples; every sample
+    then appends one token, and all but the last writer copy that block first."""
+    bs = w.block_size
+    tails = inputs.prefix_fork_tails(w)
+    per_prompt = -(-(inputs.PREFIX_LEN + int(tails.max())) // bs) + inputs.PREFIX_SAMPLES
+    N = _pool_size(w, inputs.PREFIX_PROMPTS * per_prompt)
+    bm = BlockManager(N, bs, inputs.pool_order(N, w.seed))
+    sids, pairs = [], []
+    for p in range(inputs.PREFIX_PROMPTS):
+        root = bm.allocate(inputs.PREFIX_LEN + int(tails[p]))
+        kids = [root] + [bm.fork(root) for _ in range(inputs.PREFIX_SAMPLES - 1)]
+        for sid in kids:
+            _, cow = bm.append_token(sid)
+            if cow:
+                pairs.append(cow)
+            sids.append(sid)
+    return _finish(w, bs, bm, sids, N, w.layers, device, cow_pairs=pairs)
+
+
+def run_step(b: DecodeBatch, stream=None, layers=None) -> None:
+    """One decode step over all layers (see module docstring)."""
+    if b.cow_pairs is not None and b.cow_pairs.shape[0]:
+        pk.pa_copy_blocks(b.k_caches, b.v_caches, b.cow_pairs, b.status, stream)
+    for l in range(layers if layers is not None else b.layers):
+        pk.pa_cache_append(b.k_caches[l], b.v_caches[l], b.k_new[l], b.v_new[l], b.slot_mapping,
+                           b.status, stream)
+        pk.pa_decode(b.out[l], b.q[l], b.k_caches[l], b.v_caches[l], b.block_tables,
+                     b.context_lens, b.scale, b.workspace, b.status, stream)
