@@ -144,6 +144,41 @@ pa_status pa_copy_blocks(void* const* k_caches, void* const* v_caches, int num_l
                          const int32_t* pairs, int num_pairs, int num_blocks,
                          size_t block_bytes, int32_t* dev_status, void* stream);
 
+/*
+ * pa_decode_noalloc -- pa_decode without a caller-provided workspace.
+ *
+ * The pages have no counterpart for this call; it exists for callers that cannot
+ * allocate device memory: a plug-in that runs inside a host serving process whose own
+ * allocator owns the device memory (most of it already handed to the KV pools, and
+ * raw cudaMalloc forbidden by that host), or a C caller on a path where cudaMalloc
+ * with its implicit device synchronisation is not allowed.  Such a caller still
+ * passes the inputs and the output; the scratch pa_decode takes as `workspace` lives
+ * instead in one fixed array of PA_NOALLOC_SCRATCH_BYTES bytes inside the library's
+ * device code.  Every GPU that loads the library holds that array until the process
+ * exits.  This call allocates nothing (no cudaMalloc, cudaFree or allocating library
+ * routine).
+ *
+ * Same arguments, results and errors as pa_decode, minus workspace/workspace_bytes,
+ * with these differences:
+ *  - num_seqs above PA_NOALLOC_MAX_SEQS returns PA_ERR_INVALID (the scratch is sized
+ *    for that many sequences and head_dim up to 128).
+ *  - The first call on a device looks up the device address of the array for that
+ *    device (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *    first call before any stream capture.
+ *  - All calls share the one array per device and it keeps whatever the previous call
+ *    left there.  Nothing in it needs to start at zero (each call writes every value
+ *    it later reads), but two calls that can run at the same time on one device (on
+ *    different streams, or from different host threads) race on it and give wrong
+ *    results: order them on one stream or with events.
+ */
+#define PA_NOALLOC_SCRATCH_BYTES 6291456
+#define PA_NOALLOC_MAX_SEQS 16384
+pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* block_tables, const int32_t* context_lens,
+                            int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                            int block_size, int max_blocks_per_seq, int num_blocks, float scale,
+                            pa_dtype dtype, int32_t* dev_status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -258,3 +258,106 @@ pa_status pa_copy_blocks(void* const* k_caches, void* const* v_caches, int num_l
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------
+// pa_decode_noalloc: pa_decode with its scratch in a fixed device array of this file, for
+// callers that cannot allocate device memory (see include/pagedkv.h).
+// ---------------------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoallocScratchBytes = PA_NOALLOC_SCRATCH_BYTES;
+static_assert(PA_NOALLOC_MAX_SEQS == 16384, "scratch sized for 16384 sequences");
+constexpr int kNoallocMaxGrid = 320;     // split CTAs the scratch is sized for
+constexpr int kNoallocMaxDevices = 64;
+
+// Lives in the module's global memory: every device that loads the library holds it
+// until the process exits.  Host code must not pass its name to a kernel (on the host
+// it is only a stand-in); the device address comes from cudaGetSymbolAddress.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoallocScratchBytes];
+
+// Device address of g_noalloc_scratch on the current device; looked up once per device
+// (the first call on a device does it) and cached.  nullptr on failure.
+void* noalloc_scratch(int dev) {
+  static std::mutex mu;
+  static void* addr[kNoallocMaxDevices] = {};
+  if (dev < 0 || dev >= kNoallocMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return nullptr;
+    addr[dev] = p;
+  }
+  return addr[dev];
+}
+
+}  // namespace
+
+extern "C" pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache,
+                                       const void* v_cache, const int32_t* block_tables,
+                                       const int32_t* context_lens, int num_seqs,
+                                       int num_q_heads, int num_kv_heads, int head_dim,
+                                       int block_size, int max_blocks_per_seq, int num_blocks,
+                                       float scale, pa_dtype dtype, int32_t* dev_status,
+                                       void* stream) {
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0 ||
+      num_blocks <= 0 || !std::isfinite(scale))
+    return PA_ERR_INVALID;
+  if (num_seqs > PA_NOALLOC_MAX_SEQS) return PA_ERR_INVALID;   // beyond the fixed scratch
+  if (num_q_heads % num_kv_heads) return PA_ERR_INVALID;
+  if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  if (block_size != 1 && block_size != 8 && block_size != 16 && block_size != 32)
+    return PA_ERR_UNSUPPORTED;
+  const int group = num_q_heads / num_kv_heads;
+  if (group > pkv::kMaxGroup) return PA_ERR_UNSUPPORTED;
+  if ((long long)num_blocks * num_kv_heads * block_size >= (1ll << 31) ||
+      (long long)max_blocks_per_seq * block_size >= (1ll << 31) ||
+      (long long)num_seqs * num_kv_heads >= (1ll << 31))
+    return PA_ERR_INVALID;
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PA_ERR_INVALID;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+  const int sms = sm_count();
+  if (sms <= 0) return PA_ERR_CUDA;
+  const int grid = sms * pkv::kCtasPerSm < kNoallocMaxGrid ? sms * pkv::kCtasPerSm : kNoallocMaxGrid;
+  const WsLayout w = ws_layout(num_seqs, head_dim, grid);
+  if (w.total > kNoallocScratchBytes) return PA_ERR_INVALID;
+  uint8_t* ws = static_cast<uint8_t*>(noalloc_scratch(dev));
+  if (!ws) return PA_ERR_CUDA;
+
+  CUtensorMap mk, mv;
+  std::memset(&mk, 0, sizeof(mk));
+  std::memset(&mv, 0, sizeof(mv));
+  if (block_size != 1) {
+    const uint64_t rows = (uint64_t)num_blocks * num_kv_heads * block_size;
+    const int box_rows = block_size < 16 ? block_size : 16;
+    if (!encode_pool(&mk, k_cache, dtype, head_dim, rows, box_rows) ||
+        !encode_pool(&mv, v_cache, dtype, head_dim, rows, box_rows))
+      return PA_ERR_CUDA;
+  }
+  pkv::DecodeArgs a;
+  a.out = out;
+  a.q = q;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.prefix = reinterpret_cast<int32_t*>(ws + w.prefix_off);
+  a.part_acc = reinterpret_cast<float*>(ws + w.acc_off);
+  a.part_ml = reinterpret_cast<float*>(ws + w.ml_off);
+  a.status = dev_status;
+  a.num_seqs = num_seqs;
+  a.num_q_heads = num_q_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.group = group;
+  a.max_blocks = max_blocks_per_seq;
+  a.num_blocks = num_blocks;
+  a.ctx_cap = max_blocks_per_seq * block_size;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == PA_BF16) return dispatch_d<__nv_bfloat16>(head_dim, block_size, a, mk, mv, grid, st);
+  return dispatch_d<__half>(head_dim, block_size, a, mk, mv, grid, st);
+}

@@ -23,7 +23,7 @@ DEV_BAD_BLOCK_ID, DEV_BAD_SLOT, DEV_BAD_PAIR, DEV_BAD_CONTEXT_LEN, DEV_TIMEOUT =
 
 # every symbol include/pagedkv.h declares
 EXPORTS = ("pa_version", "pa_status_string", "pa_decode_workspace_bytes", "pa_decode",
-           "pa_cache_append", "pa_copy_blocks")
+           "pa_cache_append", "pa_copy_blocks", "pa_decode_noalloc")
 
 _lib = None
 _lock = threading.Lock()
@@ -174,3 +174,36 @@ def pa_copy_blocks(k_caches, v_caches, pairs, status=None, stream=None):
     rc = load().pa_copy_blocks(kp, vp, L, _ptr(pairs), pairs.shape[0], shape[0], block_bytes,
                                _ptr(status), _stream(stream))
     _check(rc, "pa_copy_blocks")
+
+
+NOALLOC_MAX_SEQS = 16384
+
+
+def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, scale: float,
+                      status=None, stream=None):
+    """pa_decode with the library's fixed device scratch instead of a workspace, for
+    callers that cannot allocate device memory (see pa_decode_noalloc in
+    include/pagedkv.h: at most NOALLOC_MAX_SEQS sequences; calls that may run at the
+    same time on one device race on the shared scratch)."""
+    L = load()
+    fn = L.pa_decode_noalloc
+    if fn.argtypes is None:
+        P, i32, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        fn.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, f32, i32, P, P]
+        fn.restype = i32
+    _need(q, "q", ndim=3)
+    _need(out, "out", dtype=q.dtype, ndim=3)
+    _need(k_cache, "k_cache", dtype=q.dtype, ndim=4)
+    _need(v_cache, "v_cache", dtype=q.dtype, ndim=4)
+    _need(block_tables, "block_tables", dtype=torch.int32, ndim=2)
+    _need(context_lens, "context_lens", dtype=torch.int32, ndim=1)
+    B, Hq, D = q.shape
+    N, Hkv, bs, D2 = k_cache.shape
+    if out.shape != q.shape or D2 != D or v_cache.shape != k_cache.shape or \
+            block_tables.shape[0] != B or context_lens.shape[0] != B:
+        raise PagedKVError("pa_decode_noalloc: inconsistent shapes")
+    rc = fn(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+            _ptr(context_lens), B, Hq, Hkv, D, bs, block_tables.shape[1], N, float(scale),
+            _dtype_code(q), _ptr(status), _stream(stream))
+    _check(rc, "pa_decode_noalloc")
+    return out
