@@ -160,8 +160,9 @@ pa_status pa_copy_blocks(void* const* k_caches, void* const* v_caches, int num_l
  *
  * Same arguments, results and errors as pa_decode, minus workspace/workspace_bytes,
  * with these differences:
- *  - num_seqs above PA_NOALLOC_MAX_SEQS returns PA_ERR_INVALID (the scratch is sized
- *    for that many sequences and head_dim up to 128).
+ *  - num_seqs above PA_NOALLOC_MAX_SEQS returns PA_ERR_INVALID.  (The scratch holds
+ *    the split partials of at most 320 concurrently scheduled CTAs at head_dim <= 128;
+ *    on a larger GPU the call schedules 320 CTAs.)
  *  - The first call on a device looks up the device address of the array for that
  *    device (cudaGetSymbolAddress, with that device current) and caches it; make that
  *    first call before any stream capture.

@@ -5,8 +5,10 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -27,14 +29,15 @@ int sm_count() {
 }
 
 struct WsLayout {
-  size_t prefix_off, acc_off, ml_off, total;
+  size_t counters_off, acc_off, ml_off, total;
 };
 
-// prefix: int32[num_seqs+1]; partial accumulators: float[G*2][16][D];
-// partial (max, sum): float[G*2][16][2].
+// arrival counters: uint64[G]; partial accumulators: float[G*2][16][D];
+// partial (max, sum): float[G*2][16][2].  (num_seqs does not change the size.)
 WsLayout ws_layout(int num_seqs, int head_dim, int grid) {
+  (void)num_seqs;
   WsLayout w{};
-  size_t off = align256(sizeof(int32_t) * (size_t)(num_seqs + 1));
+  size_t off = align256(sizeof(unsigned long long) * (size_t)grid);
   w.acc_off = off;
   off = align256(off + sizeof(float) * (size_t)grid * 2 * pkv::kMaxGroup * head_dim);
   w.ml_off = off;
@@ -74,6 +77,41 @@ bool encode_pool(CUtensorMap* map, const void* base, pa_dtype dtype, int head_di
   return r == CUDA_SUCCESS;
 }
 
+// Every call gets its own epoch so arrival counters left by earlier calls (or by an
+// aborted one) read as zero; 0 is skipped so a zeroed workspace also reads as zero.
+uint32_t next_epoch() {
+  static std::atomic<uint32_t> epoch{0};
+  uint32_t e = ++epoch;
+  if (e == 0) e = ++epoch;
+  return e;
+}
+
+// Programmatic dependent launch lets a kernel's launch and prologue overlap the tail of
+// the kernel before it in the stream (PAGEDKV_NO_PDL=1 turns it off).
+bool use_pdl() {
+  static const bool on = [] {
+    const char* v = std::getenv("PAGEDKV_NO_PDL");
+    return !(v && v[0] && v[0] != '0');
+  }();
+  return on;
+}
+
+template <typename Kernel, typename... Args>
+cudaError_t launch(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                   Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = use_pdl() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 template <typename T, int D, int BS, int NT>
 pa_status launch_decode(const pkv::DecodeArgs& a, const CUtensorMap& mk, const CUtensorMap& mv,
                         int grid, cudaStream_t stream) {
@@ -82,9 +120,9 @@ pa_status launch_decode(const pkv::DecodeArgs& a, const CUtensorMap& mk, const C
   if (cudaFuncSetAttribute(split, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynSmem) !=
       cudaSuccess)
     return PA_ERR_CUDA;
-  split<<<grid, pkv::kThreads, L::kDynSmem, stream>>>(a, mk, mv);
-  if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
-  pkv::pa_decode_combine_kernel<T, D><<<a.num_seqs * a.num_kv_heads, 128, 0, stream>>>(a, grid);
+  if (launch(split, dim3(grid), dim3(pkv::kThreads), L::kDynSmem, stream, a, mk, mv) !=
+      cudaSuccess)
+    return PA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
@@ -187,7 +225,7 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
   a.block_tables = block_tables;
   a.context_lens = context_lens;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  a.prefix = reinterpret_cast<int32_t*>(ws + w.prefix_off);
+  a.counters = reinterpret_cast<unsigned long long*>(ws + w.counters_off);
   a.part_acc = reinterpret_cast<float*>(ws + w.acc_off);
   a.part_ml = reinterpret_cast<float*>(ws + w.ml_off);
   a.status = dev_status;
@@ -199,6 +237,7 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
   a.num_blocks = num_blocks;
   a.ctx_cap = max_blocks_per_seq * block_size;
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.epoch = next_epoch();
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dtype == PA_BF16) return dispatch_d<__nv_bfloat16>(head_dim, block_size, a, mk, mv, grid, st);
   return dispatch_d<__half>(head_dim, block_size, a, mk, mv, grid, st);
@@ -222,10 +261,12 @@ pa_status pa_cache_append(void* k_cache, void* v_cache, const void* k, const voi
   if (sms <= 0) return PA_ERR_CUDA;
   long long blocks = (total + 255) / 256;
   if (blocks > (long long)sms * 16) blocks = (long long)sms * 16;
-  pkv::pa_cache_append_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), static_cast<const uint4*>(k),
-      static_cast<const uint4*>(v), slot_mapping, num_tokens, num_kv_heads, cpr, block_size,
-      num_blocks, dev_status);
+  if (launch(pkv::pa_cache_append_kernel, dim3((unsigned)blocks), dim3(256), 0,
+             static_cast<cudaStream_t>(stream), static_cast<uint4*>(k_cache),
+             static_cast<uint4*>(v_cache), static_cast<const uint4*>(k),
+             static_cast<const uint4*>(v), slot_mapping, num_tokens, num_kv_heads, cpr,
+             block_size, num_blocks, dev_status) != cudaSuccess)
+    return PA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
@@ -250,9 +291,9 @@ pa_status pa_copy_blocks(void* const* k_caches, void* const* v_caches, int num_l
       P.v[i] = static_cast<uint4*>(v_caches[l0 + i]);
     }
     dim3 grid((unsigned)num_pairs, (unsigned)(2 * n));
-    pkv::pa_copy_blocks_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-        P, pairs, num_blocks, (long long)(block_bytes / 16), dev_status);
-    if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+    if (launch(pkv::pa_copy_blocks_kernel, grid, dim3(256), 0, static_cast<cudaStream_t>(stream),
+               P, pairs, num_blocks, (long long)(block_bytes / 16), dev_status) != cudaSuccess)
+      return PA_ERR_CUDA;
   }
   return PA_OK;
 }
@@ -345,7 +386,7 @@ extern "C" pa_status pa_decode_noalloc(void* out, const void* q, const void* k_c
   a.v_cache = v_cache;
   a.block_tables = block_tables;
   a.context_lens = context_lens;
-  a.prefix = reinterpret_cast<int32_t*>(ws + w.prefix_off);
+  a.counters = reinterpret_cast<unsigned long long*>(ws + w.counters_off);
   a.part_acc = reinterpret_cast<float*>(ws + w.acc_off);
   a.part_ml = reinterpret_cast<float*>(ws + w.ml_off);
   a.status = dev_status;
@@ -357,6 +398,7 @@ extern "C" pa_status pa_decode_noalloc(void* out, const void* q, const void* k_c
   a.num_blocks = num_blocks;
   a.ctx_cap = max_blocks_per_seq * block_size;
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.epoch = next_epoch();
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dtype == PA_BF16) return dispatch_d<__nv_bfloat16>(head_dim, block_size, a, mk, mv, grid, st);
   return dispatch_d<__half>(head_dim, block_size, a, mk, mv, grid, st);

@@ -11,7 +11,12 @@
 //    units of all segments are laid end to end and split into gridDim.x equal
 //    ranges, one per persistent CTA (2 per SM), so a batch with a heavy-tailed
 //    length mix still gives every SM the same number of KV bytes.  A segment that
-//    straddles CTA ranges is finished by the combine kernel (log-sum-exp merge).
+//    straddles CTA ranges leaves one (max, sum, acc) partial per CTA in the
+//    workspace; the last of those CTAs to finish (an epoch-tagged arrival counter,
+//    released and acquired at GPU scope) merges them with a log-sum-exp reduction in
+//    CTA order, so the result does not depend on which CTA came last and no second
+//    kernel is needed.  Every level of that merge issues its loads together: it sits
+//    at the end of most CTAs' ranges, on the kernel's critical path.
 //  * Per CTA: one producer warp walks the CTA's range and streams K/V tiles of 64
 //    tokens into a 3-stage shared-memory ring: for block_size >= 8 with 2-D TMA
 //    tensor copies (128-byte swizzle, box = min(block_size,16) rows x 64 dims) whose
@@ -24,6 +29,8 @@
 //    in base 2; P is split into a 16-bit high part and a 16-bit residual so the PV
 //    product keeps ~16 mantissa bits.
 //  * Every wait is bounded (2 s); on give-up the CTA sets PA_DEV_TIMEOUT and leaves.
+//  * Launched with programmatic dependent launch: the prologue overlaps the previous
+//    kernel's tail, and no global memory is touched before griddepcontrol.wait.
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -40,7 +47,8 @@ constexpr int kConsumerWarps = 4;
 constexpr int kUnitsPerStage = kConsumerWarps;      // one unit per consumer warp
 constexpr int kTileTokens = kUnit * kUnitsPerStage; // 64 tokens per stage
 constexpr int kStages = 3;
-constexpr int kThreads = 32 * (1 + kConsumerWarps);
+constexpr int kThreads = 32 * (1 + kConsumerWarps); // warp 0 produces, 1..4 consume
+constexpr int kMergeChunk = 32;                     // contributors whose weights sit in smem
 constexpr int kCtasPerSm = 2;
 constexpr int kMaxGroup = 16;                       // q heads per kv head handled
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
@@ -52,7 +60,13 @@ constexpr int DEV_TIMEOUT = 0x10;
 enum : int { F_FIRST = 1, F_LAST = 2, F_END = 4, F_COMPLETE = 8 };
 
 struct StageMeta {
-  int seq, kvh, tok0, nunits, ctx, flags, pidx, pad;
+  int seq, kvh, tok0, nunits, ctx, flags, pidx, qslot;
+};
+
+// A segment portion this CTA shares with other CTAs, handed to the merger warp.
+struct SplitDesc {
+  int seq, kvh, cf, cl, ncontrib, pad;  // first/last CTA of the segment, CTAs with units
+  long long seg0;                       // first unit of the segment
 };
 
 struct DecodeArgs {
@@ -64,10 +78,11 @@ struct DecodeArgs {
   const int32_t* context_lens;
   float* part_acc;              // [gridDim*2][kMaxGroup][D]
   float* part_ml;               // [gridDim*2][kMaxGroup][2]  (max, sum) in base 2
-  int32_t* prefix;              // [num_seqs+1] units per kv head, exclusive scan
+  unsigned long long* counters; // [gridDim] arrival counters: (epoch << 32) | arrivals
   int32_t* status;              // nullable
   int num_seqs, num_q_heads, num_kv_heads, group, max_blocks, num_blocks, ctx_cap;
   float scale_log2;             // scale * log2(e)
+  uint32_t epoch;               // distinct per call: counters of older calls read as zero
 };
 
 template <int D>
@@ -79,10 +94,33 @@ struct Layout {
   static_assert(kStageBytes % 1024 == 0, "stage must keep 1024-byte alignment");
   static constexpr int kMetaOff = kStages * kStageBytes;
   static constexpr int kBarOff = kMetaOff + kStages * (int)sizeof(StageMeta);
-  static constexpr int kMlOff = kBarOff + 2 * kStages * 8 + 16;
-  static constexpr int kBytes = kMlOff + kConsumerWarps * kMaxGroup * 8;
+  // full[kStages], empty[kStages]
+  static constexpr int kMiscOff = kBarOff + (2 * kStages + 1) * 8;
+  // abort flag, last-arrival flag, total units
+  static constexpr int kDescOff = kMiscOff + 16;
+  static constexpr int kMlOff = kDescOff + 2 * (int)sizeof(SplitDesc);
+  static constexpr int kMergeOff = kMlOff + kConsumerWarps * kMaxGroup * 8;
+  // merge: pidx[kMergeChunk], weights[kMergeChunk][kMaxGroup], max[16], 1/sum[16]
+  static constexpr int kBytes = kMergeOff + kMergeChunk * 4 + kMergeChunk * kMaxGroup * 4 + 2 * kMaxGroup * 4;
   static constexpr int kDynSmem = kBytes + 1024;           // slack for 1024-byte alignment
+  static_assert(2 * (kDynSmem + 1024) <= 233472, "two CTAs per SM must fit");
 };
+
+__device__ __forceinline__ unsigned long long ld_relaxed_gpu(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ unsigned long long cas_acq_rel_gpu(unsigned long long* p,
+                                                              unsigned long long cmp,
+                                                              unsigned long long val) {
+  unsigned long long old;
+  asm volatile("atom.acq_rel.gpu.global.cas.b64 %0, [%1], %2, %3;"
+               : "=l"(old)
+               : "l"(p), "l"(cmp), "l"(val)
+               : "memory");
+  return old;
+}
 
 __device__ __forceinline__ int clamp_ctx(int c, int cap, int32_t* status) {
   if (c < 0 || c > cap) {
@@ -134,9 +172,126 @@ __device__ __forceinline__ void cp_async_16_zfill(void* dst, const void* src, ui
 }
 
 // ------------------------------------------------------------------------------------
-// Split pass: every CTA processes its unit range and writes finished rows to `out`,
-// or (max, sum, unnormalised acc) partials for segments it shares with other CTAs.
+// The decode kernel: every CTA processes its unit range; rows of segments it covers
+// whole go straight to `out`, segments shared with other CTAs go through partials
+// and the last contributing CTA merges them.
 // ------------------------------------------------------------------------------------
+// Partial slot of CTA cc for the segment starting at unit seg0 (-1: CTA without units).
+__device__ __forceinline__ int partial_slot(int cc, long long seg0, long long total, int G) {
+  const long long s0 = cta_start(cc, total, G);
+  return s0 < cta_start(cc + 1, total, G) ? cc * 2 + (s0 < seg0 ? 1 : 0) : -1;
+}
+
+// Last arrival of a split segment: out = (sum_k acc_k 2^(m_k - M)) / (sum_k l_k 2^(m_k - M)),
+// M = max_k m_k, over the contributing CTAs k in CTA order; run by the 128 consumer
+// threads (bar.sync id 1).  Each level issues all of its loads before using them.
+template <typename T, int D>
+__device__ __forceinline__ void merge_split(const DecodeArgs& a, const SplitDesc& dsc,
+                                            long long total, int G, int group, int tid,
+                                            uint8_t* ws_smem) {
+  constexpr int kThr = 32 * kConsumerWarps;
+  int* plist = reinterpret_cast<int*>(ws_smem);
+  float* wgt = reinterpret_cast<float*>(plist + kMergeChunk);      // [kMergeChunk][kMaxGroup]
+  float* hmax = wgt + kMergeChunk * kMaxGroup;
+  float* hinv = hmax + kMaxGroup;
+  const int nr = dsc.cl - dsc.cf + 1;
+  // per head h (8 threads each): M and L
+  {
+    const int h = tid >> 3, sub = tid & 7;
+    const bool hv = h < group;
+    float mk = -INFINITY, lk = 0.f;
+    if (sub < nr && hv) {
+      const int p = partial_slot(dsc.cf + sub, dsc.seg0, total, G);
+      if (p >= 0) {
+        const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.part_ml) + (long long)p * kMaxGroup + h);
+        mk = ml.x;
+        lk = ml.y;
+      }
+    }
+    float M = mk;
+    for (int k = sub + 8; k < nr; k += 8) {
+      const int p = partial_slot(dsc.cf + k, dsc.seg0, total, G);
+      if (p >= 0 && hv) M = fmaxf(M, __ldcg(a.part_ml + ((long long)p * kMaxGroup + h) * 2));
+    }
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float Ls = mk == -INFINITY ? 0.f : lk * ex2(mk - M);
+    for (int k = sub + 8; k < nr; k += 8) {
+      const int p = partial_slot(dsc.cf + k, dsc.seg0, total, G);
+      if (p >= 0 && hv) {
+        const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.part_ml) + (long long)p * kMaxGroup + h);
+        Ls += ml.x == -INFINITY ? 0.f : ml.y * ex2(ml.x - M);
+      }
+    }
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
+    if (sub == 0 && hv) {
+      hmax[h] = M;
+      hinv[h] = 1.f / Ls;
+    }
+  }
+  constexpr int kF4 = D / 4;
+  constexpr int kPer = kMaxGroup * kF4 / kThr;          // float4 elements per thread (max)
+  const int nel = group * kF4;
+  float4 acc[kPer];
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) acc[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int k0 = 0; k0 < nr; k0 += kMergeChunk) {
+    const int kn = (nr - k0) < kMergeChunk ? (nr - k0) : kMergeChunk;
+    named_bar_sync(1, kThr);                           // hmax ready / previous chunk done
+    for (int i = tid; i < kn * kMaxGroup; i += kThr) {
+      const int k = i / kMaxGroup, h = i % kMaxGroup;
+      const int p = partial_slot(dsc.cf + k0 + k, dsc.seg0, total, G);
+      if (h == 0) plist[k] = p;
+      float w = 0.f;
+      if (p >= 0 && h < group) {
+        const float mp = __ldcg(a.part_ml + ((long long)p * kMaxGroup + h) * 2);
+        w = mp == -INFINITY ? 0.f : ex2(mp - hmax[h]);
+      }
+      wgt[k * kMaxGroup + h] = w;
+    }
+    named_bar_sync(1, kThr);
+    for (int k = 0; k < kn; k += 2) {
+      const int p0 = plist[k], p1 = k + 1 < kn ? plist[k + 1] : -1;
+      float4 v0[kPer], v1[kPer];
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) {
+        const int i = tid + kThr * e;
+        const int h = i / kF4, d4 = i % kF4;
+        v0[e] = v1[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (i < nel && p0 >= 0)
+          v0[e] = __ldcg(reinterpret_cast<const float4*>(a.part_acc + ((long long)p0 * kMaxGroup + h) * D) + d4);
+        if (i < nel && p1 >= 0)
+          v1[e] = __ldcg(reinterpret_cast<const float4*>(a.part_acc + ((long long)p1 * kMaxGroup + h) * D) + d4);
+      }
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) {
+        const int i = tid + kThr * e;
+        if (i >= nel) continue;
+        const int h = i / kF4;
+        const float w0 = p0 >= 0 ? wgt[k * kMaxGroup + h] : 0.f;
+        const float w1 = p1 >= 0 ? wgt[(k + 1) * kMaxGroup + h] : 0.f;
+        acc[e].x += v0[e].x * w0; acc[e].y += v0[e].y * w0;
+        acc[e].z += v0[e].z * w0; acc[e].w += v0[e].w * w0;
+        acc[e].x += v1[e].x * w1; acc[e].y += v1[e].y * w1;
+        acc[e].z += v1[e].z * w1; acc[e].w += v1[e].w * w1;
+      }
+    }
+  }
+  T* outp = static_cast<T*>(a.out) +
+            ((long long)dsc.seq * a.num_q_heads + (long long)dsc.kvh * group) * D;
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) {
+    const int i = tid + kThr * e;
+    if (i >= nel) continue;
+    const int h = i / kF4, d4 = i % kF4;
+    const float inv = hinv[h];
+    const uint32_t lo = pack2<T>(acc[e].x * inv, acc[e].y * inv);
+    const uint32_t hi = pack2<T>(acc[e].z * inv, acc[e].w * inv);
+    *reinterpret_cast<uint2*>(outp + h * D + d4 * 4) = make_uint2(lo, hi);
+  }
+}
+
 template <typename T, int D, int BS, int NT>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     pa_decode_split_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
@@ -144,13 +299,17 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   using L = Layout<D>;
   constexpr bool kBF16 = std::is_same_v<T, __nv_bfloat16>;
   constexpr int kFullCount = (BS == 1) ? 33 : 1;
+  constexpr int kConsumerThreads = 32 * kConsumerWarps;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   StageMeta* meta = reinterpret_cast<StageMeta*>(smem + L::kMetaOff);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   uint64_t* empty = full + kStages;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kStages);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff);
+  volatile int* last_flag = abort_flag + 1;
+  long long* total_s = reinterpret_cast<long long*>(smem + L::kMiscOff + 8);
+  SplitDesc* desc = reinterpret_cast<SplitDesc*>(smem + L::kDescOff);
   float2* mls = reinterpret_cast<float2*>(smem + L::kMlOff);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -160,6 +319,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       mbar_init(&empty[i], kConsumerWarps);
     }
     *abort_flag = 0;
+    *last_flag = 0;
     fence_mbar_init();
   }
   if (BS != 1 && threadIdx.x == 32) {
@@ -167,6 +327,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     prefetch_tensormap(&tmv);
   }
   __syncthreads();
+  pdl_wait();      // nothing global is read or written before the previous grid is done
+  pdl_trigger();
 
   const int G = gridDim.x, c = blockIdx.x;
   const int Hkv = a.num_kv_heads, group = a.group;
@@ -174,172 +336,217 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   if (warp == 0) {
     // ============================== producer ==============================
     const int B = a.num_seqs;
-    // pass 1 over the batch: units per kv head, their exclusive scan (CTA 0 stores it)
+    // pass 1 over the batch: total units; CTA 0 also writes the zero rows of empty
+    // sequences (they own no unit).  For B <= 32 the lane values are kept for pass 2.
     long long run = 0;
+    int keep_ctx = 0, keep_u = 0, keep_x = 0;
+#pragma unroll 4
     for (int base = 0; base < B; base += 32) {
       const int s = base + lane;
-      int u = 0;
-      if (s < B) u = (clamp_ctx(a.context_lens[s], a.ctx_cap, c == 0 ? a.status : nullptr) +
-                      kUnit - 1) / kUnit;
+      int ctx = 0;
+      if (s < B) ctx = clamp_ctx(a.context_lens[s], a.ctx_cap, c == 0 ? a.status : nullptr);
+      const int u = (ctx + kUnit - 1) / kUnit;
       int x = u;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, x, o);
         if (lane >= o) x += y;
       }
-      if (c == 0 && s < B) a.prefix[s] = (int)(run + x - u);
+      keep_ctx = ctx;
+      keep_u = u;
+      keep_x = x;
       run += __shfl_sync(0xffffffffu, x, 31);
+      if (c == 0) {
+        unsigned zero = __ballot_sync(0xffffffffu, s < B && u == 0);
+        while (zero) {
+          const int src = __ffs(zero) - 1;
+          zero &= zero - 1;
+          uint4* row = reinterpret_cast<uint4*>(static_cast<T*>(a.out) +
+                                                (long long)(base + src) * a.num_q_heads * D);
+          for (int i = lane; i < a.num_q_heads * D * 2 / 16; i += 32) row[i] = make_uint4(0, 0, 0, 0);
+        }
+      }
     }
-    if (c == 0 && lane == 0) a.prefix[B] = (int)run;
     const long long total = (long long)Hkv * run;
     const long long start = total ? cta_start(c, total, G) : 0;
     const long long end = total ? cta_start(c + 1, total, G) : 0;
 
     // pass 2: the sequence holding unit `start`
-    int s_cur = 0, u_cur = 0, ctx_cur = 0;
-    long long pbase = 0;
+    int s_a = 0, u_a = 0, ctx_a = 0;
+    long long pb_a = 0;
     if (start < end) {
       long long r2 = 0;
-      for (int base = 0; base < B; base += 32) {
+      bool got_a = false;
+      for (int base = 0; base < B && !got_a; base += 32) {
         const int s = base + lane;
-        int ctx = 0;
-        if (s < B) ctx = clamp_ctx(a.context_lens[s], a.ctx_cap, nullptr);
-        const int u = (ctx + kUnit - 1) / kUnit;
-        int x = u;
+        int ctx = keep_ctx, u = keep_u, x = keep_x;
+        if (B > 32) {
+          ctx = 0;
+          if (s < B) ctx = clamp_ctx(a.context_lens[s], a.ctx_cap, nullptr);
+          u = (ctx + kUnit - 1) / kUnit;
+          x = u;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(0xffffffffu, x, o);
-          if (lane >= o) x += y;
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+          }
         }
         const long long lo = (long long)Hkv * (r2 + x - u), hi = (long long)Hkv * (r2 + x);
-        const unsigned hit = __ballot_sync(0xffffffffu, s < B && u > 0 && lo <= start && start < hi);
-        if (hit) {
-          const int src = __ffs(hit) - 1;
-          s_cur = base + src;
-          u_cur = __shfl_sync(0xffffffffu, u, src);
-          ctx_cur = __shfl_sync(0xffffffffu, ctx, src);
-          pbase = __shfl_sync(0xffffffffu, lo, src);
-          break;
+        const unsigned ha = __ballot_sync(0xffffffffu, s < B && u > 0 && lo <= start && start < hi);
+        if (ha) {
+          const int src = __ffs(ha) - 1;
+          s_a = base + src;
+          u_a = __shfl_sync(0xffffffffu, u, src);
+          ctx_a = __shfl_sync(0xffffffffu, ctx, src);
+          pb_a = __shfl_sync(0xffffffffu, lo, src);
+          got_a = true;
         }
         r2 += __shfl_sync(0xffffffffu, x, 31);
       }
     }
+    if (lane == 0) *total_s = total;
+    __syncwarp();
 
     const uint64_t policy = policy_evict_first();
     const int rows_total = a.num_blocks * Hkv * BS;
-    int st = 0;
+    int st = 0, nq = 0;
     uint32_t ph = 0;
     bool ok = true;
-    long long x = start;
-    while (ok && x < end) {
-      while (x >= pbase + (long long)Hkv * u_cur) {   // next sequence with units
-        pbase += (long long)Hkv * u_cur;
-        ++s_cur;
-        ctx_cur = clamp_ctx(a.context_lens[s_cur], a.ctx_cap, nullptr);
-        u_cur = (ctx_cur + kUnit - 1) / kUnit;
-      }
-      const int kvh = (int)((x - pbase) / u_cur);
-      const long long seg0 = pbase + (long long)kvh * u_cur, seg1 = seg0 + u_cur;
-      const long long pe = seg1 < end ? seg1 : end;
-      const bool complete = seg0 >= start && seg1 <= end;
-      const int pidx = c * 2 + (start < seg0 ? 1 : 0);
-      const int32_t* trow = a.block_tables + (long long)s_cur * a.max_blocks;
-      for (long long tu = x; tu < pe; tu += kUnitsPerStage) {
-        const int nun = (int)((pe - tu) < kUnitsPerStage ? (pe - tu) : kUnitsPerStage);
-        const int tok0 = (int)(tu - seg0) * kUnit;
-        const int flags = (tu == x ? F_FIRST : 0) | (tu + kUnitsPerStage >= pe ? F_LAST : 0) |
-                          (complete ? F_COMPLETE : 0);
-        if (!mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, kWaitLimitNs)) {
-          ok = false;
-          break;
+    {
+      long long x = start;
+      const long long xend = end;
+      int s_cur = s_a, u_cur = u_a, ctx_cur = ctx_a;
+      long long pbase = pb_a;
+      while (ok && x < xend) {
+        while (x >= pbase + (long long)Hkv * u_cur) {   // next sequence with units
+          pbase += (long long)Hkv * u_cur;
+          ++s_cur;
+          ctx_cur = clamp_ctx(a.context_lens[s_cur], a.ctx_cap, nullptr);
+          u_cur = (ctx_cur + kUnit - 1) / kUnit;
         }
-        uint8_t* sK = smem + st * L::kStageBytes;
-        uint8_t* sV = sK + L::kKvBytes;
-        uint8_t* sQ = sV + L::kKvBytes;
-        const uint32_t qbytes = (flags & F_FIRST) ? (uint32_t)(group * D * 2) : 0u;
-        if (lane == 0) {
-          meta[st] = StageMeta{s_cur, kvh, tok0, nun, ctx_cur, flags, pidx, 0};
-        }
-        if constexpr (BS != 1) {
-          constexpr int H = BS < 16 ? BS : 16;     // rows per TMA box
-          constexpr int BPU = kUnit / H;           // boxes per unit and column half
-          constexpr int kBoxBytes = H * 128;
-          uint32_t bytes = qbytes;
-          for (int j = 0; j < nun; ++j) {
-            const int rem = ctx_cur - (tok0 + j * kUnit);
-            const int nb = (rem + H - 1) / H;
-            bytes += (uint32_t)((nb < BPU ? nb : BPU) * kBoxBytes * L::kHalves * 2);
-          }
+        const int kvh = (int)((x - pbase) / u_cur);
+        const long long seg0 = pbase + (long long)kvh * u_cur, seg1 = seg0 + u_cur;
+        const long long pe = seg1 < xend ? seg1 : xend;
+        const bool complete = seg0 >= start && seg1 <= end;
+        const int pidx = c * 2 + (start < seg0 ? 1 : 0);
+        int qslot = 0;
+        if (!complete) {
+          qslot = nq++;
           if (lane == 0) {
-            mbar_arrive_expect_tx(&full[st], bytes);
-            if (qbytes)
-              bulk_load(sQ,
-                        static_cast<const T*>(a.q) +
-                            ((long long)s_cur * a.num_q_heads + (long long)kvh * group) * D,
-                        qbytes, &full[st]);
+            const int cf = cta_of(seg0, total, G), cl = cta_of(seg1 - 1, total, G);
+            int ncontrib = 0;
+            for (int cc = cf; cc <= cl; ++cc)
+              ncontrib += cta_start(cc, total, G) < cta_start(cc + 1, total, G);
+            desc[qslot] = SplitDesc{s_cur, kvh, cf, cl, ncontrib, 0, seg0};
           }
-          __syncwarp();
-          const int nbox = nun * BPU * L::kHalves * 2;
-          for (int i = lane; i < nbox; i += 32) {
-            const int kv = i & 1;
-            const int hf = (i >> 1) % L::kHalves;
-            const int jb = (i >> 1) / L::kHalves;
+        }
+        const int32_t* trow = a.block_tables + (long long)s_cur * a.max_blocks;
+        for (long long tu = x; tu < pe; tu += kUnitsPerStage) {
+          const int nun = (int)((pe - tu) < kUnitsPerStage ? (pe - tu) : kUnitsPerStage);
+          const int tok0 = (int)(tu - seg0) * kUnit;
+          const int flags = (tu == x ? F_FIRST : 0) | (tu + kUnitsPerStage >= pe ? F_LAST : 0) |
+                            (complete ? F_COMPLETE : 0);
+          const uint32_t qbytes = (flags & F_FIRST) ? (uint32_t)(group * D * 2) : 0u;
+          const T* qsrc = static_cast<const T*>(a.q) +
+                          ((long long)s_cur * a.num_q_heads + (long long)kvh * group) * D;
+          if constexpr (BS != 1) {
+            constexpr int H = BS < 16 ? BS : 16;     // rows per TMA box
+            constexpr int BPU = kUnit / H;           // boxes per unit and column half
+            constexpr int kBoxBytes = H * 128;
+            static_assert(kUnitsPerStage * BPU * L::kHalves * 2 <= 32, "one box per lane");
+            // this lane's box and its block-table entry, read before the slot wait
+            const int nbox = nun * BPU * L::kHalves * 2;
+            const int kv = lane & 1;
+            const int hf = (lane >> 1) % L::kHalves;
+            const int jb = (lane >> 1) / L::kHalves;
             const int j = jb / BPU, b = jb % BPU;
             const int t = tok0 + j * kUnit + b * H;
-            if (t < ctx_cur) {
+            const bool mine = lane < nbox && t < ctx_cur;
+            int y = 0;
+            if (mine) {
               const int blk = trow[t / BS];
-              int y;
               if ((unsigned)blk < (unsigned)a.num_blocks) {
                 y = (blk * Hkv + kvh) * BS + (t % BS);
               } else {
                 if (a.status) atomicOr(a.status, DEV_BAD_BLOCK_ID);
-                y = rows_total;                      // out of range: TMA fills zeros
+                y = rows_total;                        // out of range: TMA fills zeros
               }
+            }
+            uint32_t bytes = qbytes;
+            for (int jj = 0; jj < nun; ++jj) {
+              const int rem = ctx_cur - (tok0 + jj * kUnit);
+              const int nb = (rem + H - 1) / H;
+              bytes += (uint32_t)((nb < BPU ? nb : BPU) * kBoxBytes * L::kHalves * 2);
+            }
+            if (!mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, kWaitLimitNs)) {
+              ok = false;
+              break;
+            }
+            uint8_t* sK = smem + st * L::kStageBytes;
+            uint8_t* sV = sK + L::kKvBytes;
+            uint8_t* sQ = sV + L::kKvBytes;
+            if (lane == 0) {
+              meta[st] = StageMeta{s_cur, kvh, tok0, nun, ctx_cur, flags, pidx, qslot};
+              mbar_arrive_expect_tx(&full[st], bytes);
+              if (qbytes) bulk_load(sQ, qsrc, qbytes, &full[st]);
+            }
+            __syncwarp();
+            if (mine) {
               uint8_t* dst = (kv ? sV : sK) + hf * (kTileTokens * 128) + (j * kUnit + b * H) * 128;
               tma_load_2d(dst, kv ? &tmv : &tmk, &full[st], hf * 64, y, policy);
             }
-          }
-        } else {
-          // block_size 1: every token is its own block; 16-byte cp.async with the same
-          // 128-byte swizzle the TMA path produces.
-          constexpr int CPR = D * 2 / 16;          // 16-byte chunks per row
-          constexpr int RPI = 32 / CPR;            // rows per warp instruction
-          if (lane == 0) {
-            mbar_arrive_expect_tx(&full[st], qbytes);
-            if (qbytes)
-              bulk_load(sQ,
-                        static_cast<const T*>(a.q) +
-                            ((long long)s_cur * a.num_q_heads + (long long)kvh * group) * D,
-                        qbytes, &full[st]);
-          }
-          const int ch = lane % CPR, hf = ch >> 3, cc = ch & 7;
-          for (int r0 = 0; r0 < nun * kUnit; r0 += RPI) {
-            const int r = r0 + lane / CPR;
-            const int t = tok0 + r;
-            if (t < ctx_cur) {
-              const int blk = trow[t];
-              uint32_t sz = 16;
-              long long row = 0;
-              if ((unsigned)blk < (unsigned)a.num_blocks) {
-                row = (long long)blk * Hkv + kvh;
-              } else {
-                if (a.status) atomicOr(a.status, DEV_BAD_BLOCK_ID);
-                sz = 0;                                // zero fill, no read
-              }
-              const long long off = row * D + ch * 8;
-              const int soff = hf * (kTileTokens * 128) + r * 128 + ((cc ^ (r & 7)) << 4);
-              cp_async_16_zfill(sK + soff, static_cast<const T*>(a.k_cache) + off, sz, policy);
-              cp_async_16_zfill(sV + soff, static_cast<const T*>(a.v_cache) + off, sz, policy);
+          } else {
+            // block_size 1: every token is its own block; 16-byte cp.async with the same
+            // 128-byte swizzle the TMA path produces.  Table entries of the tile's (up
+            // to) 64 tokens are read before the slot wait, two per lane, and handed out
+            // by shuffle.
+            constexpr int CPR = D * 2 / 16;          // 16-byte chunks per row
+            constexpr int RPI = 32 / CPR;            // rows per warp instruction
+            const int ntok = nun * kUnit;
+            int pre0 = -1, pre1 = -1;
+            if (lane < ntok && tok0 + lane < ctx_cur) pre0 = trow[tok0 + lane];
+            if (lane + 32 < ntok && tok0 + 32 + lane < ctx_cur) pre1 = trow[tok0 + 32 + lane];
+            if (!mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, kWaitLimitNs)) {
+              ok = false;
+              break;
             }
+            uint8_t* sK = smem + st * L::kStageBytes;
+            uint8_t* sV = sK + L::kKvBytes;
+            uint8_t* sQ = sV + L::kKvBytes;
+            if (lane == 0) {
+              meta[st] = StageMeta{s_cur, kvh, tok0, nun, ctx_cur, flags, pidx, qslot};
+              mbar_arrive_expect_tx(&full[st], qbytes);
+              if (qbytes) bulk_load(sQ, qsrc, qbytes, &full[st]);
+            }
+            const int ch = lane % CPR, hf = ch >> 3, cc = ch & 7;
+            for (int r0 = 0; r0 < ntok; r0 += RPI) {
+              const int r = r0 + lane / CPR;
+              const int blk = __shfl_sync(0xffffffffu, r0 >= 32 ? pre1 : pre0, r & 31);
+              const int t = tok0 + r;
+              if (r < ntok && t < ctx_cur) {
+                uint32_t sz = 16;
+                long long row = 0;
+                if ((unsigned)blk < (unsigned)a.num_blocks) {
+                  row = (long long)blk * Hkv + kvh;
+                } else {
+                  if (a.status) atomicOr(a.status, DEV_BAD_BLOCK_ID);
+                  sz = 0;                                // zero fill, no read
+                }
+                const long long off = row * D + ch * 8;
+                const int soff = hf * (kTileTokens * 128) + r * 128 + ((cc ^ (r & 7)) << 4);
+                cp_async_16_zfill(sK + soff, static_cast<const T*>(a.k_cache) + off, sz, policy);
+                cp_async_16_zfill(sV + soff, static_cast<const T*>(a.v_cache) + off, sz, policy);
+              }
+            }
+            cp_async_mbar_arrive_noinc(&full[st]);
           }
-          cp_async_mbar_arrive_noinc(&full[st]);
+          if (++st == kStages) {
+            st = 0;
+            ph ^= 1u;
+          }
         }
-        if (++st == kStages) {
-          st = 0;
-          ph ^= 1u;
-        }
+        x = pe;
       }
-      x = pe;
     }
     if (ok) ok = mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, kWaitLimitNs);
     if (ok) {
@@ -361,6 +568,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   // ============================== consumers ==============================
   const int cw = warp - 1;
   const int gid = lane >> 2, tig = lane & 3;
+  const int tid = cw * 32 + lane;
   constexpr int KS = D / 16;            // k-steps of QK, m-tiles of PV
   constexpr int NREG = KS * NT * 4;     // O^T accumulator registers per thread
   float o[KS][NT][4];
@@ -439,24 +647,24 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       uint32_t bhi[NT][2], blo[NT][2];
 #pragma unroll
       for (int n = 0; n < NT; ++n) {
-        float x[4];
+        float xs[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int row = gid + (e >= 2 ? 8 : 0);
-          x[e] = row < valid ? sacc[n][e] * a.scale_log2 : -INFINITY;
+          xs[e] = row < valid ? sacc[n][e] * a.scale_log2 : -INFINITY;
         }
         float alpha[2], p[4];
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
-          float mx = fmaxf(x[cc], x[cc + 2]);
+          float mx = fmaxf(xs[cc], xs[cc + 2]);
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
           const float mnew = fmaxf(m[n][cc], mx);
           alpha[cc] = ex2(m[n][cc] - mnew);
           m[n][cc] = mnew;
-          p[cc] = ex2(x[cc] - mnew);
-          p[cc + 2] = ex2(x[cc + 2] - mnew);
+          p[cc] = ex2(xs[cc] - mnew);
+          p[cc + 2] = ex2(xs[cc + 2] - mnew);
           l[n][cc] = l[n][cc] * alpha[cc] + p[cc] + p[cc + 2];
         }
 #pragma unroll
@@ -516,7 +724,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           v += __shfl_xor_sync(0xffffffffu, v, 16);
           l[n][cc] = v;
         }
-      named_bar_sync(1, 32 * kConsumerWarps);      // all warps are done with this stage's K/V
+      named_bar_sync(1, kConsumerThreads);         // all warps are done with this stage's K/V
       float* scr = reinterpret_cast<float*>(sK);   // K and V tiles reused as scratch
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks)
@@ -532,12 +740,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           for (int cc = 0; cc < 2; ++cc)
             mls[cw * kMaxGroup + n * 8 + 2 * tig + cc] = make_float2(m[n][cc], l[n][cc]);
       }
-      named_bar_sync(1, 32 * kConsumerWarps);
-      const int tid = cw * 32 + lane;
+      named_bar_sync(1, kConsumerThreads);
       const bool complete = mt.flags & F_COMPLETE;
       T* outp = static_cast<T*>(a.out) +
                 ((long long)mt.seq * a.num_q_heads + (long long)mt.kvh * group) * D;
-      for (int pi = tid; pi < NREG * 32; pi += 32 * kConsumerWarps) {
+      for (int pi = tid; pi < NREG * 32; pi += kConsumerThreads) {
         const int r = pi >> 5, ln = pi & 31;
         const int e = r & 3, n = (r >> 2) % NT, mtile = (r >> 2) / NT;
         const int d = mtile * 16 + (ln >> 2) + (e >= 2 ? 8 : 0);
@@ -564,6 +771,27 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           }
         }
       }
+      if (!complete) {
+        // ---- arrival on the segment's counter: bar.sync orders every thread's partial
+        // stores before thread 0's release at GPU scope; its acquire orders the other
+        // CTAs' partials before the reads below (they load through L2, bypassing L1).
+        named_bar_sync(1, kConsumerThreads);
+        const SplitDesc dsc = desc[mt.qslot];
+        if (tid == 0) {
+          unsigned long long* ctr = a.counters + dsc.cf;
+          unsigned long long old = ld_relaxed_gpu(ctr), nxt;
+          for (;;) {
+            nxt = (uint32_t)(old >> 32) == a.epoch ? old + 1
+                                                    : ((unsigned long long)a.epoch << 32) | 1ull;
+            const unsigned long long prev = cas_acq_rel_gpu(ctr, old, nxt);
+            if (prev == old) break;
+            old = prev;
+          }
+          *last_flag = (int)(uint32_t)nxt == dsc.ncontrib;
+        }
+        named_bar_sync(1, kConsumerThreads);
+        if (*last_flag) merge_split<T, D>(a, dsc, *total_s, G, group, tid, smem + L::kMergeOff);
+      }
       fence_proxy_async_smem();   // generic writes above precede the next TMA fill
     }
     __syncwarp();
@@ -572,48 +800,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       st = 0;
       ph ^= 1u;
     }
-  }
-}
-
-// ------------------------------------------------------------------------------------
-// Combine pass: for every segment split over several CTAs, merge the partials with a
-// log-sum-exp reduction in CTA order; also writes the zero rows of empty sequences.
-// ------------------------------------------------------------------------------------
-template <typename T, int D>
-__global__ void __launch_bounds__(128) pa_decode_combine_kernel(const DecodeArgs a, int G) {
-  const int Hkv = a.num_kv_heads, group = a.group;
-  const int s = blockIdx.x / Hkv, kvh = blockIdx.x % Hkv;
-  const int ctx = clamp_ctx(a.context_lens[s], a.ctx_cap, nullptr);
-  const int u = (ctx + kUnit - 1) / kUnit;
-  T* outp = static_cast<T*>(a.out) + ((long long)s * a.num_q_heads + (long long)kvh * group) * D;
-  if (u == 0) {
-    for (int i = threadIdx.x; i < group * D; i += blockDim.x) outp[i] = from_float<T>(0.f);
-    return;
-  }
-  const long long total = (long long)Hkv * a.prefix[a.num_seqs];
-  const long long seg0 = (long long)Hkv * a.prefix[s] + (long long)kvh * u;
-  const int cf = cta_of(seg0, total, G), cl = cta_of(seg0 + u - 1, total, G);
-  if (cf == cl) return;   // finished by a single CTA in the split pass
-  for (int i = threadIdx.x; i < group * D; i += blockDim.x) {
-    const int h = i / D, d = i % D;
-    float M = -INFINITY;
-    for (int cc = cf; cc <= cl; ++cc) {
-      const long long st0 = cta_start(cc, total, G);
-      if (st0 == cta_start(cc + 1, total, G)) continue;   // empty range
-      const int pidx = cc * 2 + (st0 < seg0 ? 1 : 0);
-      M = fmaxf(M, a.part_ml[((long long)pidx * kMaxGroup + h) * 2]);
-    }
-    float Lsum = 0.f, acc = 0.f;
-    for (int cc = cf; cc <= cl; ++cc) {
-      const long long st0 = cta_start(cc, total, G);
-      if (st0 == cta_start(cc + 1, total, G)) continue;
-      const int pidx = cc * 2 + (st0 < seg0 ? 1 : 0);
-      const float mp = a.part_ml[((long long)pidx * kMaxGroup + h) * 2];
-      const float sc = mp == -INFINITY ? 0.f : ex2(mp - M);
-      Lsum += a.part_ml[((long long)pidx * kMaxGroup + h) * 2 + 1] * sc;
-      acc += a.part_acc[((long long)pidx * kMaxGroup + h) * D + d] * sc;
-    }
-    outp[h * D + d] = from_float<T>(acc / Lsum);
   }
 }
 

@@ -4,6 +4,8 @@
 #pragma once
 #include <cstdint>
 
+#include "ptx.cuh"
+
 namespace pkv {
 
 constexpr int DEV_BAD_SLOT = 0x2;
@@ -19,6 +21,8 @@ __global__ void __launch_bounds__(256)
                            const int64_t* __restrict__ slot_mapping, int num_tokens, int Hkv,
                            int chunks_per_row, int block_size, int num_blocks,
                            int32_t* status) {
+  pdl_wait();
+  pdl_trigger();
   const long long total = (long long)num_tokens * Hkv * chunks_per_row;
   const long long limit = (long long)num_blocks * block_size;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
@@ -51,6 +55,8 @@ struct LayerPtrs {
 __global__ void __launch_bounds__(256)
     pa_copy_blocks_kernel(const __grid_constant__ LayerPtrs P, const int32_t* __restrict__ pairs,
                           int num_blocks, long long chunks_per_block, int32_t* status) {
+  pdl_wait();
+  pdl_trigger();
   const int p = blockIdx.x;
   const int layer = blockIdx.y >> 1, pool = blockIdx.y & 1;
   const int src = pairs[2 * p], dst = pairs[2 * p + 1];

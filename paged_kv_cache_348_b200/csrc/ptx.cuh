@@ -155,4 +155,13 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// Block until every grid this one depends on has completed and its memory is visible.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Allow the next grid in the stream (launched with programmatic serialisation) to start
+// its prologue; it still waits in pdl_wait() for this grid to finish.
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 }  // namespace pkv
