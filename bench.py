@@ -34,7 +34,7 @@ METRIC = "paged decode attn: KV-read HBM GB/s (% of B200 peak) and seq-steps/s"
 FALLBACK_HBM_GBS = 6650.0
 
 
-def workload_desc(w, bs):
+def workload_desc(w, bs, layers=0):
     from paged_kv_cache_348_b200 import inputs
 
     ctx = {"tiny": "{5,16,17,40}", "llama8b": "U[128,2048]", "llama70b": "U[1000,8000]",
@@ -42,7 +42,7 @@ def workload_desc(w, bs):
            "prefix": "2048 shared + U[0,512] private"}[w.name]
     return ("%s-shape paged decode step: %d layer(s), batch %d, %d q / %d kv heads, head_dim %d, "
             "block_size %d, %s, context lens %s, seed %d" % (
-                w.name, w.layers, w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, bs,
+                w.name, layers or w.layers, w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, bs,
                 w.dtype, ctx, w.seed))
 
 
@@ -225,6 +225,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama70b")
     ap.add_argument("--block-size", type=int, default=0)
+    ap.add_argument("--layers", type=int, default=0,
+                    help="layers of the workload to run (0: all; fewer only for profiling)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -255,7 +257,7 @@ def main():
     if w.name == "prefix":
         b = wl.build_prefix_decode(w, device="cuda")
     else:
-        b = wl.build(w, device="cuda", block_size=bs)
+        b = wl.build(w, device="cuda", block_size=bs, layers=args.layers or None)
     stream = torch.cuda.current_stream()
     L = b.layers
     kv_step = b.kv_bytes_per_step()
@@ -328,7 +330,7 @@ def main():
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-        "config": {"workload": workload_desc(w, bs), "global_batch": w.num_seqs * world,
+        "config": {"workload": workload_desc(w, bs, b.layers), "global_batch": w.num_seqs * world,
                    "seq_len": float(b.context_lens.float().mean().item()),
                    "parallelism": "replicas" if world > 1 else "single gpu",
                    "l2": "inputs larger than L2 (%.2f GB of K/V per layer)" % (kv_layer / 1e9)},
