@@ -15,8 +15,11 @@
 //    workspace; the last of those CTAs to finish (an epoch-tagged arrival counter,
 //    released and acquired at GPU scope) merges them with a log-sum-exp reduction in
 //    CTA order, so the result does not depend on which CTA came last and no second
-//    kernel is needed.  Every level of that merge issues its loads together: it sits
-//    at the end of most CTAs' ranges, on the kernel's critical path.
+//    kernel is needed.  The merge folds the partials in with a running maximum, several
+//    contributors per L2 round trip: it sits at the end of most CTAs' ranges, on the
+//    kernel's critical path.
+//  * The producer keeps a window of block-table entries in registers, loaded 64 blocks
+//    ahead of use, so the only table read a stage waits for is a portion's first.
 //  * Per CTA: one producer warp walks the CTA's range and streams K/V tiles of 64
 //    tokens into a 3-stage shared-memory ring: for block_size >= 8 with 2-D TMA
 //    tensor copies (128-byte swizzle, box = min(block_size,16) rows x 64 dims) whose
@@ -48,7 +51,6 @@ constexpr int kUnitsPerStage = kConsumerWarps;      // one unit per consumer war
 constexpr int kTileTokens = kUnit * kUnitsPerStage; // 64 tokens per stage
 constexpr int kStages = 3;
 constexpr int kThreads = 32 * (1 + kConsumerWarps); // warp 0 produces, 1..4 consume
-constexpr int kMergeChunk = 32;                     // contributors whose weights sit in smem
 constexpr int kCtasPerSm = 2;
 constexpr int kMaxGroup = 16;                       // q heads per kv head handled
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
@@ -99,9 +101,7 @@ struct Layout {
   // abort flag, last-arrival flag, total units
   static constexpr int kDescOff = kMiscOff + 16;
   static constexpr int kMlOff = kDescOff + 2 * (int)sizeof(SplitDesc);
-  static constexpr int kMergeOff = kMlOff + kConsumerWarps * kMaxGroup * 8;
-  // merge: pidx[kMergeChunk], weights[kMergeChunk][kMaxGroup], max[16], 1/sum[16]
-  static constexpr int kBytes = kMergeOff + kMergeChunk * 4 + kMergeChunk * kMaxGroup * 4 + 2 * kMaxGroup * 4;
+  static constexpr int kBytes = kMlOff + kConsumerWarps * kMaxGroup * 8;
   static constexpr int kDynSmem = kBytes + 1024;           // slack for 1024-byte alignment
   static_assert(2 * (kDynSmem + 1024) <= 233472, "two CTAs per SM must fit");
 };
@@ -171,6 +171,15 @@ __device__ __forceinline__ void cp_async_16_zfill(void* dst, const void* src, ui
                : "memory");
 }
 
+// Entry i (0 <= i < 96) of a block-table window held across the warp: lane l holds
+// entries l, 32+l and 64+l in x0, x1, x2.  Every lane must call it.
+__device__ __forceinline__ int win_lookup(int x0, int x1, int x2, int i) {
+  const int a = __shfl_sync(0xffffffffu, x0, i & 31);
+  const int b = __shfl_sync(0xffffffffu, x1, i & 31);
+  const int c = __shfl_sync(0xffffffffu, x2, i & 31);
+  return i < 32 ? a : (i < 64 ? b : c);
+}
+
 // ------------------------------------------------------------------------------------
 // The decode kernel: every CTA processes its unit range; rows of segments it covers
 // whole go straight to `out`, segments shared with other CTAs go through partials
@@ -183,100 +192,63 @@ __device__ __forceinline__ int partial_slot(int cc, long long seg0, long long to
 }
 
 // Last arrival of a split segment: out = (sum_k acc_k 2^(m_k - M)) / (sum_k l_k 2^(m_k - M)),
-// M = max_k m_k, over the contributing CTAs k in CTA order; run by the 128 consumer
-// threads (bar.sync id 1).  Each level issues all of its loads before using them.
-template <typename T, int D>
+// M = max_k m_k, over the contributing CTAs k.  Run by the 128 consumer threads; thread
+// tid owns output elements (head, 4 dims) e = tid + 128 i.  The partials are folded in
+// CTA order with a running maximum (so the result does not depend on which CTA arrived
+// last), kMC contributors at a time with every load of a group issued before any use:
+// one L2 round trip per group.
+template <typename T, int D, int NT>
 __device__ __forceinline__ void merge_split(const DecodeArgs& a, const SplitDesc& dsc,
-                                            long long total, int G, int group, int tid,
-                                            uint8_t* ws_smem) {
+                                            long long total, int G, int group, int tid) {
   constexpr int kThr = 32 * kConsumerWarps;
-  int* plist = reinterpret_cast<int*>(ws_smem);
-  float* wgt = reinterpret_cast<float*>(plist + kMergeChunk);      // [kMergeChunk][kMaxGroup]
-  float* hmax = wgt + kMergeChunk * kMaxGroup;
-  float* hinv = hmax + kMaxGroup;
-  const int nr = dsc.cl - dsc.cf + 1;
-  // per head h (8 threads each): M and L
-  {
-    const int h = tid >> 3, sub = tid & 7;
-    const bool hv = h < group;
-    float mk = -INFINITY, lk = 0.f;
-    if (sub < nr && hv) {
-      const int p = partial_slot(dsc.cf + sub, dsc.seg0, total, G);
-      if (p >= 0) {
-        const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.part_ml) + (long long)p * kMaxGroup + h);
-        mk = ml.x;
-        lk = ml.y;
-      }
-    }
-    float M = mk;
-    for (int k = sub + 8; k < nr; k += 8) {
-      const int p = partial_slot(dsc.cf + k, dsc.seg0, total, G);
-      if (p >= 0 && hv) M = fmaxf(M, __ldcg(a.part_ml + ((long long)p * kMaxGroup + h) * 2));
-    }
-#pragma unroll
-    for (int o = 1; o < 8; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float Ls = mk == -INFINITY ? 0.f : lk * ex2(mk - M);
-    for (int k = sub + 8; k < nr; k += 8) {
-      const int p = partial_slot(dsc.cf + k, dsc.seg0, total, G);
-      if (p >= 0 && hv) {
-        const float2 ml = __ldcg(reinterpret_cast<const float2*>(a.part_ml) + (long long)p * kMaxGroup + h);
-        Ls += ml.x == -INFINITY ? 0.f : ml.y * ex2(ml.x - M);
-      }
-    }
-#pragma unroll
-    for (int o = 1; o < 8; o <<= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
-    if (sub == 0 && hv) {
-      hmax[h] = M;
-      hinv[h] = 1.f / Ls;
-    }
-  }
   constexpr int kF4 = D / 4;
-  constexpr int kPer = kMaxGroup * kF4 / kThr;          // float4 elements per thread (max)
+  constexpr int kPer = (8 * NT * kF4 + kThr - 1) / kThr;  // float4 elements per thread (max)
+  constexpr int kMC = kPer >= 4 ? 2 : 4;                    // contributors per round trip
   const int nel = group * kF4;
+  const int nr = dsc.cl - dsc.cf + 1;
+  float M[kPer], Lsum[kPer];
   float4 acc[kPer];
 #pragma unroll
-  for (int e = 0; e < kPer; ++e) acc[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int k0 = 0; k0 < nr; k0 += kMergeChunk) {
-    const int kn = (nr - k0) < kMergeChunk ? (nr - k0) : kMergeChunk;
-    named_bar_sync(1, kThr);                           // hmax ready / previous chunk done
-    for (int i = tid; i < kn * kMaxGroup; i += kThr) {
-      const int k = i / kMaxGroup, h = i % kMaxGroup;
-      const int p = partial_slot(dsc.cf + k0 + k, dsc.seg0, total, G);
-      if (h == 0) plist[k] = p;
-      float w = 0.f;
-      if (p >= 0 && h < group) {
-        const float mp = __ldcg(a.part_ml + ((long long)p * kMaxGroup + h) * 2);
-        w = mp == -INFINITY ? 0.f : ex2(mp - hmax[h]);
-      }
-      wgt[k * kMaxGroup + h] = w;
-    }
-    named_bar_sync(1, kThr);
-    for (int k = 0; k < kn; k += 2) {
-      const int p0 = plist[k], p1 = k + 1 < kn ? plist[k + 1] : -1;
-      float4 v0[kPer], v1[kPer];
+  for (int e = 0; e < kPer; ++e) {
+    M[e] = -INFINITY;
+    Lsum[e] = 0.f;
+    acc[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int k0 = 0; k0 < nr; k0 += kMC) {
+    int pk[kMC];
+    float2 ml[kMC][kPer];
+    float4 v[kMC][kPer];
+#pragma unroll
+    for (int k = 0; k < kMC; ++k) {
+      pk[k] = k0 + k < nr ? partial_slot(dsc.cf + k0 + k, dsc.seg0, total, G) : -1;
 #pragma unroll
       for (int e = 0; e < kPer; ++e) {
         const int i = tid + kThr * e;
         const int h = i / kF4, d4 = i % kF4;
-        v0[e] = v1[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (i < nel && p0 >= 0)
-          v0[e] = __ldcg(reinterpret_cast<const float4*>(a.part_acc + ((long long)p0 * kMaxGroup + h) * D) + d4);
-        if (i < nel && p1 >= 0)
-          v1[e] = __ldcg(reinterpret_cast<const float4*>(a.part_acc + ((long long)p1 * kMaxGroup + h) * D) + d4);
-      }
-#pragma unroll
-      for (int e = 0; e < kPer; ++e) {
-        const int i = tid + kThr * e;
-        if (i >= nel) continue;
-        const int h = i / kF4;
-        const float w0 = p0 >= 0 ? wgt[k * kMaxGroup + h] : 0.f;
-        const float w1 = p1 >= 0 ? wgt[(k + 1) * kMaxGroup + h] : 0.f;
-        acc[e].x += v0[e].x * w0; acc[e].y += v0[e].y * w0;
-        acc[e].z += v0[e].z * w0; acc[e].w += v0[e].w * w0;
-        acc[e].x += v1[e].x * w1; acc[e].y += v1[e].y * w1;
-        acc[e].z += v1[e].z * w1; acc[e].w += v1[e].w * w1;
+        ml[k][e] = make_float2(-INFINITY, 0.f);
+        v[k][e] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (pk[k] >= 0 && i < nel) {
+          const long long row = (long long)pk[k] * kMaxGroup + h;
+          ml[k][e] = __ldcg(reinterpret_cast<const float2*>(a.part_ml) + row);
+          v[k][e] = __ldcg(reinterpret_cast<const float4*>(a.part_acc + row * D) + d4);
+        }
       }
     }
+#pragma unroll
+    for (int k = 0; k < kMC; ++k)
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) {
+        if (ml[k][e].x == -INFINITY) continue;          // no unit, or an empty partial
+        const float mn = fmaxf(M[e], ml[k][e].x);
+        const float sa = M[e] == -INFINITY ? 0.f : ex2(M[e] - mn);
+        const float sb = ex2(ml[k][e].x - mn);
+        Lsum[e] = Lsum[e] * sa + ml[k][e].y * sb;
+        acc[e].x = acc[e].x * sa + v[k][e].x * sb;
+        acc[e].y = acc[e].y * sa + v[k][e].y * sb;
+        acc[e].z = acc[e].z * sa + v[k][e].z * sb;
+        acc[e].w = acc[e].w * sa + v[k][e].w * sb;
+        M[e] = mn;
+      }
   }
   T* outp = static_cast<T*>(a.out) +
             ((long long)dsc.seq * a.num_q_heads + (long long)dsc.kvh * group) * D;
@@ -285,7 +257,7 @@ __device__ __forceinline__ void merge_split(const DecodeArgs& a, const SplitDesc
     const int i = tid + kThr * e;
     if (i >= nel) continue;
     const int h = i / kF4, d4 = i % kF4;
-    const float inv = hinv[h];
+    const float inv = 1.f / Lsum[e];
     const uint32_t lo = pack2<T>(acc[e].x * inv, acc[e].y * inv);
     const uint32_t hi = pack2<T>(acc[e].z * inv, acc[e].w * inv);
     *reinterpret_cast<uint2*>(outp + h * D + d4 * 4) = make_uint2(lo, hi);
@@ -440,10 +412,26 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             desc[qslot] = SplitDesc{s_cur, kvh, cf, cl, ncontrib, 0, seg0};
           }
         }
+        // Block-table window: lane l holds entries wb+l, wb+32+l (w0, w1) and the next 64
+        // entries (n0, n1), loaded 64 blocks before they are needed, so no stage waits on a
+        // table read except the portion's first.
         const int32_t* trow = a.block_tables + (long long)s_cur * a.max_blocks;
+        const int nblk = (ctx_cur + BS - 1) / BS;
+        int wb = (int)((x - seg0) * kUnit) / BS;
+        int w0 = wb + lane < nblk ? trow[wb + lane] : -1;
+        int w1 = wb + 32 + lane < nblk ? trow[wb + 32 + lane] : -1;
+        int n0 = wb + 64 + lane < nblk ? trow[wb + 64 + lane] : -1;
+        int n1 = wb + 96 + lane < nblk ? trow[wb + 96 + lane] : -1;
         for (long long tu = x; tu < pe; tu += kUnitsPerStage) {
           const int nun = (int)((pe - tu) < kUnitsPerStage ? (pe - tu) : kUnitsPerStage);
           const int tok0 = (int)(tu - seg0) * kUnit;
+          if (tok0 / BS >= wb + 64) {                 // warp-uniform: slide the window
+            w0 = n0;
+            w1 = n1;
+            wb += 64;
+            n0 = wb + 64 + lane < nblk ? trow[wb + 64 + lane] : -1;
+            n1 = wb + 96 + lane < nblk ? trow[wb + 96 + lane] : -1;
+          }
           const int flags = (tu == x ? F_FIRST : 0) | (tu + kUnitsPerStage >= pe ? F_LAST : 0) |
                             (complete ? F_COMPLETE : 0);
           const uint32_t qbytes = (flags & F_FIRST) ? (uint32_t)(group * D * 2) : 0u;
@@ -462,9 +450,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             const int j = jb / BPU, b = jb % BPU;
             const int t = tok0 + j * kUnit + b * H;
             const bool mine = lane < nbox && t < ctx_cur;
+            // the stage spans blocks tok0/BS .. +64/BS-1 < wb + 72: w0, w1 and, only when it
+            // runs past the window, n0 (whose load was issued 64 blocks ago)
+            const int wi = mine ? t / BS - wb : 0;
+            int blk;
+            if ((tok0 + kTileTokens - 1) / BS >= wb + 64)   // warp-uniform
+              blk = win_lookup(w0, w1, n0, wi);
+            else
+              blk = win_lookup(w0, w1, w1, wi);       // never touches n0 while it loads
             int y = 0;
             if (mine) {
-              const int blk = trow[t / BS];
               if ((unsigned)blk < (unsigned)a.num_blocks) {
                 y = (blk * Hkv + kvh) * BS + (t % BS);
               } else {
@@ -497,15 +492,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             }
           } else {
             // block_size 1: every token is its own block; 16-byte cp.async with the same
-            // 128-byte swizzle the TMA path produces.  Table entries of the tile's (up
-            // to) 64 tokens are read before the slot wait, two per lane, and handed out
-            // by shuffle.
+            // 128-byte swizzle the TMA path produces.  Stages are 64 tokens, so the window
+            // (w0, w1) holds exactly this stage's table entries, handed out by shuffle.
             constexpr int CPR = D * 2 / 16;          // 16-byte chunks per row
             constexpr int RPI = 32 / CPR;            // rows per warp instruction
             const int ntok = nun * kUnit;
-            int pre0 = -1, pre1 = -1;
-            if (lane < ntok && tok0 + lane < ctx_cur) pre0 = trow[tok0 + lane];
-            if (lane + 32 < ntok && tok0 + 32 + lane < ctx_cur) pre1 = trow[tok0 + 32 + lane];
             if (!mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, kWaitLimitNs)) {
               ok = false;
               break;
@@ -521,7 +512,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             const int ch = lane % CPR, hf = ch >> 3, cc = ch & 7;
             for (int r0 = 0; r0 < ntok; r0 += RPI) {
               const int r = r0 + lane / CPR;
-              const int blk = __shfl_sync(0xffffffffu, r0 >= 32 ? pre1 : pre0, r & 31);
+              const int blk = __shfl_sync(0xffffffffu, r0 >= 32 ? w1 : w0, r & 31);
               const int t = tok0 + r;
               if (r < ntok && t < ctx_cur) {
                 uint32_t sz = 16;
@@ -790,7 +781,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           *last_flag = (int)(uint32_t)nxt == dsc.ncontrib;
         }
         named_bar_sync(1, kConsumerThreads);
-        if (*last_flag) merge_split<T, D>(a, dsc, *total_s, G, group, tid, smem + L::kMergeOff);
+        if (*last_flag) merge_split<T, D, NT>(a, dsc, *total_s, G, group, tid);
       }
       fence_proxy_async_smem();   // generic writes above precede the next TMA fill
     }
