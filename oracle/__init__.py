@@ -54,6 +54,9 @@ def _load():
         L.orc_decode.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32,
                                  f64, i32, P, i32, i32]
         L.orc_decode.restype = i32
+        L.orc_decode_multi.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32,
+                                       i32, f64, i32, P, i32, i32]
+        L.orc_decode_multi.restype = i32
         L.orc_cache_append.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32]
         L.orc_cache_append.restype = i32
         L.orc_copy_blocks.argtypes = [P, P, i32, P, i32, i64, i32]
@@ -119,6 +122,35 @@ def decode(q, k_cache, v_cache, block_tables, context_lens, scale: float, dtype:
                             B, Hq, Hkv, D, bs, bt.shape[1], N, float(scale), DTYPES[dtype],
                             None if it is None else _p(it), 0 if it is None else len(it),
                             int(nthreads))
+    if rc == -1:
+        raise ValueError("oracle decode: block id out of range")
+    if rc:
+        raise ValueError("oracle decode: bad arguments (%d)" % rc)
+    return out64, out16
+
+
+def decode_multi(q, k_cache, v_cache, block_tables, context_lens, scale: float, dtype: str,
+                 items=None, nthreads: int = 1):
+    """fp64 paged decode of q_len new tokens per sequence, causal among them.
+
+    q is [B, q_len, Hq, D]; new token j of sequence s sits at position
+    ctx - q_len + j and attends to positions 0 .. ctx - q_len + j.  Returns
+    (out64 [B,q_len,Hq,D] float64, out16 [B,q_len,Hq,D] uint16)."""
+    q = _c(q, np.uint16)
+    k_cache = _c(k_cache, np.uint16)
+    v_cache = _c(v_cache, np.uint16)
+    bt = _c(block_tables, np.int32)
+    cl = _c(context_lens, np.int32)
+    B, QL, Hq, D = q.shape
+    N, Hkv, bs, D2 = k_cache.shape
+    assert D2 == D and v_cache.shape == k_cache.shape and bt.shape[0] == B
+    out64 = np.zeros((B, QL, Hq, D), dtype=np.float64)
+    out16 = np.zeros((B, QL, Hq, D), dtype=np.uint16)
+    it = None if items is None else _c(items, np.int32)
+    rc = _load().orc_decode_multi(_p(out64), _p(out16), _p(q), _p(k_cache), _p(v_cache), _p(bt),
+                                  _p(cl), B, QL, Hq, Hkv, D, bs, bt.shape[1], N, float(scale),
+                                  DTYPES[dtype], None if it is None else _p(it),
+                                  0 if it is None else len(it), int(nthreads))
     if rc == -1:
         raise ValueError("oracle decode: block id out of range")
     if rc:

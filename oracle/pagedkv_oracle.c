@@ -134,48 +134,55 @@ int orc_gather(double* out, const uint16_t* cache, int dtype, int num_blocks, in
 
 /* ---- decode attention: [P1] "How PagedAttention borrows OS paging" -- the math is
  *      the plain dot products, softmax and value-weighted sum, only the storage is
- *      paged; so this is softmax(scale * q K^T) V over the gathered rows. ---------- */
+ *      paged; so this is softmax(scale * q K^T) V over the gathered rows.
+ *      Several new tokens per sequence (q_len > 1): [P1] "Why KV cache memory was the
+ *      bottleneck" -- a generated token uses the keys and values of every token before
+ *      it.  The q_len new tokens occupy the last q_len cached positions, so new token j
+ *      (position ctx - q_len + j) attends to positions 0 .. ctx - q_len + j, i.e. to the
+ *      first n_j = ctx - q_len + 1 + j rows; n_j <= 0 gives an all-zero output row. -- */
 typedef struct {
   double* out64;
   uint16_t* out16;
   const uint16_t *q, *k_cache, *v_cache;
   const int32_t *block_tables, *context_lens, *items;
-  int n_items, Hq, Hkv, D, bs, max_blocks, num_blocks, dtype;
+  int n_items, q_len, Hq, Hkv, D, bs, max_blocks, num_blocks, dtype;
   double scale;
   atomic_int next;
   atomic_int err;
 } decode_job;
 
-static void decode_one(decode_job* J, int s, int h, double* kbuf, double* vbuf, double* w) {
+static void decode_one(decode_job* J, int s, int j, int h, double* kbuf, double* vbuf, double* w) {
   int D = J->D;
   int group = J->Hq / J->Hkv;
   int kvh = h / group;                      /* consecutive q heads share one kv head */
   int ctx = J->context_lens[s];
-  double* o64 = J->out64 + ((int64_t)s * J->Hq + h) * D;
+  int n = ctx - J->q_len + 1 + j;           /* rows this query token attends to */
+  int64_t row = ((int64_t)s * J->q_len + j) * J->Hq + h;
+  double* o64 = J->out64 + row * D;
   for (int d = 0; d < D; ++d) o64[d] = 0.0;
-  if (ctx > 0) {
+  if (n > 0) {
     const int32_t* table_row = J->block_tables + (int64_t)s * J->max_blocks;
-    if (orc_gather(kbuf, J->k_cache, J->dtype, J->num_blocks, J->Hkv, J->bs, D, table_row, ctx, kvh) ||
-        orc_gather(vbuf, J->v_cache, J->dtype, J->num_blocks, J->Hkv, J->bs, D, table_row, ctx, kvh)) {
+    if (orc_gather(kbuf, J->k_cache, J->dtype, J->num_blocks, J->Hkv, J->bs, D, table_row, n, kvh) ||
+        orc_gather(vbuf, J->v_cache, J->dtype, J->num_blocks, J->Hkv, J->bs, D, table_row, n, kvh)) {
       atomic_store(&J->err, 1);
       return;
     }
-    const uint16_t* qrow = J->q + ((int64_t)s * J->Hq + h) * D;
+    const uint16_t* qrow = J->q + row * D;
     double m = -INFINITY;
-    for (int t = 0; t < ctx; ++t) {         /* x_t = scale * <q, k_t> */
+    for (int t = 0; t < n; ++t) {           /* x_t = scale * <q, k_t> */
       double acc = 0.0;
       for (int d = 0; d < D; ++d) acc += to_f64(qrow[d], J->dtype) * kbuf[(int64_t)t * D + d];
       w[t] = J->scale * acc;
       if (w[t] > m) m = w[t];
     }
     double l = 0.0;
-    for (int t = 0; t < ctx; ++t) { w[t] = exp(w[t] - m); l += w[t]; }
-    for (int t = 0; t < ctx; ++t)
+    for (int t = 0; t < n; ++t) { w[t] = exp(w[t] - m); l += w[t]; }
+    for (int t = 0; t < n; ++t)
       for (int d = 0; d < D; ++d) o64[d] += w[t] * vbuf[(int64_t)t * D + d];
     for (int d = 0; d < D; ++d) o64[d] /= l;
   }
   if (J->out16) {
-    uint16_t* o16 = J->out16 + ((int64_t)s * J->Hq + h) * D;
+    uint16_t* o16 = J->out16 + row * D;
     for (int d = 0; d < D; ++d) o16[d] = from_f64(o64[d], J->dtype);
   }
 }
@@ -197,32 +204,34 @@ static void* decode_worker(void* arg) {
   double* vbuf = (double*)malloc(n * J->D * sizeof(double));
   double* w = (double*)malloc(n * sizeof(double));
   if (!kbuf || !vbuf || !w) { atomic_store(&J->err, 2); free(kbuf); free(vbuf); free(w); return NULL; }
-  int total = J->n_items * J->Hq;           /* work item = (sequence, q head) */
+  int per_seq = J->q_len * J->Hq;
+  int total = J->n_items * per_seq;         /* work item = (sequence, new token, q head) */
   for (;;) {
     int it = atomic_fetch_add(&J->next, 1);
     if (it >= total) break;
-    int i = it / J->Hq, h = it % J->Hq;
+    int i = it / per_seq, r = it % per_seq;
     int s = J->items ? J->items[i] : i;
-    decode_one(J, s, h, kbuf, vbuf, w);
+    decode_one(J, s, r / J->Hq, r % J->Hq, kbuf, vbuf, w);
   }
   free(kbuf); free(vbuf); free(w);
   return NULL;
 }
 
-/* out64[B][Hq][D] (and, if out16 != NULL, its round-to-nearest-even 16-bit copy).
- * `items` (nullable) restricts the work to the listed sequences (sampled checks);
- * rows of other sequences are left untouched.  Returns 0, -1 on a bad block id,
- * -2 on bad arguments or allocation failure. */
-int orc_decode(double* out64, uint16_t* out16, const uint16_t* q, const uint16_t* k_cache,
-               const uint16_t* v_cache, const int32_t* block_tables, const int32_t* context_lens,
-               int B, int Hq, int Hkv, int D, int bs, int max_blocks, int num_blocks,
-               double scale, int dtype, const int32_t* items, int n_items, int nthreads) {
-  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || D <= 0 || bs <= 0) return -2;
+/* q and out64 are [B][q_len][Hq][D] (out16, if not NULL, gets the round-to-nearest-even
+ * 16-bit copy).  `items` (nullable) restricts the work to the listed sequences (sampled
+ * checks); rows of other sequences are left untouched.  Returns 0, -1 on a bad block
+ * id, -2 on bad arguments or allocation failure. */
+int orc_decode_multi(double* out64, uint16_t* out16, const uint16_t* q, const uint16_t* k_cache,
+                     const uint16_t* v_cache, const int32_t* block_tables,
+                     const int32_t* context_lens, int B, int q_len, int Hq, int Hkv, int D, int bs,
+                     int max_blocks, int num_blocks, double scale, int dtype, const int32_t* items,
+                     int n_items, int nthreads) {
+  if (B < 0 || q_len < 1 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || D <= 0 || bs <= 0) return -2;
   decode_job J;
   J.out64 = out64; J.out16 = out16; J.q = q; J.k_cache = k_cache; J.v_cache = v_cache;
   J.block_tables = block_tables; J.context_lens = context_lens;
   J.items = items; J.n_items = items ? n_items : B;
-  J.Hq = Hq; J.Hkv = Hkv; J.D = D; J.bs = bs; J.max_blocks = max_blocks;
+  J.q_len = q_len; J.Hq = Hq; J.Hkv = Hkv; J.D = D; J.bs = bs; J.max_blocks = max_blocks;
   J.num_blocks = num_blocks; J.dtype = dtype; J.scale = scale;
   atomic_init(&J.next, 0);
   atomic_init(&J.err, 0);
@@ -243,6 +252,16 @@ int orc_decode(double* out64, uint16_t* out16, const uint16_t* q, const uint16_t
   }
   int e = atomic_load(&J.err);
   return e == 1 ? -1 : (e ? -2 : 0);
+}
+
+/* One new token per sequence: q and out are [B][Hq][D]. */
+int orc_decode(double* out64, uint16_t* out16, const uint16_t* q, const uint16_t* k_cache,
+               const uint16_t* v_cache, const int32_t* block_tables, const int32_t* context_lens,
+               int B, int Hq, int Hkv, int D, int bs, int max_blocks, int num_blocks,
+               double scale, int dtype, const int32_t* items, int n_items, int nthreads) {
+  return orc_decode_multi(out64, out16, q, k_cache, v_cache, block_tables, context_lens, B, 1, Hq,
+                          Hkv, D, bs, max_blocks, num_blocks, scale, dtype, items, n_items,
+                          nthreads);
 }
 
 /* ---- cache append: [P1] "How PagedAttention borrows OS paging" (blocks are filled
