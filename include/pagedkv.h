@@ -107,6 +107,29 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
                     void* stream);
 
 /*
+ * pa_decode_multi -- pa_decode for q_len new tokens per sequence (speculative, beam or
+ * chunked decoding), causal among them.
+ *
+ * Defined, besides the passages cited for pa_decode, by [P1] "Why KV cache memory was
+ * the bottleneck": a generated token uses the keys and values of every token before
+ * it.  The q_len new tokens of sequence s are its last q_len cached positions (append
+ * them first), so new token j sits at position p = context_lens[s] - q_len + j and
+ *   out[s][j][h][:] = sum_{t <= p} softmax_t(scale * <q[s][j][h], K_s[t]>) * V_s[t].
+ * A new token with p < 0 (context_lens[s] < q_len) sees nothing: its row is zero.
+ *
+ *   q, out         [num_seqs][q_len][num_q_heads][head_dim]
+ *   other arguments as for pa_decode; the workspace size does not depend on q_len.
+ * Limits: 1 <= q_len and (num_q_heads/num_kv_heads) * q_len <= 16 (PA_ERR_UNSUPPORTED
+ * otherwise).  q_len == 1 gives exactly the bits of pa_decode.
+ */
+pa_status pa_decode_multi(void* out, const void* q, const void* k_cache, const void* v_cache,
+                          const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+                          int q_len, int num_q_heads, int num_kv_heads, int head_dim,
+                          int block_size, int max_blocks_per_seq, int num_blocks, float scale,
+                          pa_dtype dtype, void* workspace, size_t workspace_bytes,
+                          int32_t* dev_status, void* stream);
+
+/*
  * pa_cache_append -- write the new tokens' K and V into their cache slots.
  *
  * Defined by [P1] "How PagedAttention borrows OS paging" (blocks are filled on demand

@@ -129,8 +129,8 @@ pa_status launch_decode(const pkv::DecodeArgs& a, const CUtensorMap& mk, const C
 template <typename T, int D, int BS>
 pa_status dispatch_nt(const pkv::DecodeArgs& a, const CUtensorMap& mk, const CUtensorMap& mv,
                       int grid, cudaStream_t s) {
-  return a.group <= 8 ? launch_decode<T, D, BS, 1>(a, mk, mv, grid, s)
-                      : launch_decode<T, D, BS, 2>(a, mk, mv, grid, s);
+  return a.ncol <= 8 ? launch_decode<T, D, BS, 1>(a, mk, mv, grid, s)
+                     : launch_decode<T, D, BS, 2>(a, mk, mv, grid, s);
 }
 
 template <typename T, int D>
@@ -152,37 +152,16 @@ pa_status dispatch_d(int d, int bs, const pkv::DecodeArgs& a, const CUtensorMap&
                  : dispatch_bs<T, 128>(bs, a, mk, mv, grid, s);
 }
 
-}  // namespace
-
-extern "C" {
-
-int pa_version(void) { return 100; }
-
-const char* pa_status_string(pa_status s) {
-  switch (s) {
-    case PA_OK: return "ok";
-    case PA_ERR_INVALID: return "invalid argument";
-    case PA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
-    case PA_ERR_CUDA: return "CUDA error";
-  }
-  return "unknown status";
-}
-
-size_t pa_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim) {
-  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0) return 0;
-  const int sms = sm_count();
-  if (sms <= 0) return 0;
-  return ws_layout(num_seqs, head_dim, sms * pkv::kCtasPerSm).total;
-}
-
-pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
-                    const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
-                    int num_q_heads, int num_kv_heads, int head_dim, int block_size,
-                    int max_blocks_per_seq, int num_blocks, float scale, pa_dtype dtype,
-                    void* workspace, size_t workspace_bytes, int32_t* dev_status,
-                    void* stream) {
-  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0 ||
-      num_blocks <= 0 || !std::isfinite(scale))
+// Validation, workspace layout, tensor maps and launch shared by the decode entry points.
+// grid_cap > 0 caps the number of split CTAs (the fixed scratch of pa_decode_noalloc).
+pa_status decode_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
+                      const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+                      int q_len, int num_q_heads, int num_kv_heads, int head_dim,
+                      int block_size, int max_blocks_per_seq, int num_blocks, float scale,
+                      pa_dtype dtype, void* workspace, size_t workspace_bytes, int grid_cap,
+                      int32_t* dev_status, void* stream) {
+  if (num_seqs < 0 || q_len < 1 || num_q_heads <= 0 || num_kv_heads <= 0 ||
+      max_blocks_per_seq <= 0 || num_blocks <= 0 || !std::isfinite(scale))
     return PA_ERR_INVALID;
   if (num_q_heads % num_kv_heads) return PA_ERR_INVALID;
   if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
@@ -190,7 +169,7 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
   if (block_size != 1 && block_size != 8 && block_size != 16 && block_size != 32)
     return PA_ERR_UNSUPPORTED;
   const int group = num_q_heads / num_kv_heads;
-  if (group > pkv::kMaxGroup) return PA_ERR_UNSUPPORTED;
+  if ((long long)group * q_len > pkv::kMaxGroup) return PA_ERR_UNSUPPORTED;
   if ((long long)num_blocks * num_kv_heads * block_size >= (1ll << 31) ||
       (long long)max_blocks_per_seq * block_size >= (1ll << 31) ||
       (long long)num_seqs * num_kv_heads >= (1ll << 31))
@@ -203,7 +182,8 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
     return PA_ERR_INVALID;
   const int sms = sm_count();
   if (sms <= 0) return PA_ERR_CUDA;
-  const int grid = sms * pkv::kCtasPerSm;
+  int grid = sms * pkv::kCtasPerSm;
+  if (grid_cap > 0 && grid > grid_cap) grid = grid_cap;
   const WsLayout w = ws_layout(num_seqs, head_dim, grid);
   if (workspace_bytes < w.total) return PA_ERR_INVALID;
 
@@ -236,11 +216,60 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
   a.max_blocks = max_blocks_per_seq;
   a.num_blocks = num_blocks;
   a.ctx_cap = max_blocks_per_seq * block_size;
+  a.q_len = q_len;
+  a.ncol = group * q_len;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.epoch = next_epoch();
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dtype == PA_BF16) return dispatch_d<__nv_bfloat16>(head_dim, block_size, a, mk, mv, grid, st);
   return dispatch_d<__half>(head_dim, block_size, a, mk, mv, grid, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int pa_version(void) { return 100; }
+
+const char* pa_status_string(pa_status s) {
+  switch (s) {
+    case PA_OK: return "ok";
+    case PA_ERR_INVALID: return "invalid argument";
+    case PA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case PA_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+size_t pa_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim) {
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0) return 0;
+  const int sms = sm_count();
+  if (sms <= 0) return 0;
+  return ws_layout(num_seqs, head_dim, sms * pkv::kCtasPerSm).total;
+}
+
+pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+                    int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                    int max_blocks_per_seq, int num_blocks, float scale, pa_dtype dtype,
+                    void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                    void* stream) {
+  return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, 1,
+                     num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                     num_blocks, scale, dtype, workspace, workspace_bytes, 0, dev_status,
+                     stream);
+}
+
+pa_status pa_decode_multi(void* out, const void* q, const void* k_cache, const void* v_cache,
+                          const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+                          int q_len, int num_q_heads, int num_kv_heads, int head_dim,
+                          int block_size, int max_blocks_per_seq, int num_blocks, float scale,
+                          pa_dtype dtype, void* workspace, size_t workspace_bytes,
+                          int32_t* dev_status, void* stream) {
+  return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, q_len,
+                     num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                     num_blocks, scale, dtype, workspace, workspace_bytes, 0, dev_status,
+                     stream);
 }
 
 pa_status pa_cache_append(void* k_cache, void* v_cache, const void* k, const void* v,
@@ -340,66 +369,20 @@ extern "C" pa_status pa_decode_noalloc(void* out, const void* q, const void* k_c
                                        int block_size, int max_blocks_per_seq, int num_blocks,
                                        float scale, pa_dtype dtype, int32_t* dev_status,
                                        void* stream) {
-  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0 ||
-      num_blocks <= 0 || !std::isfinite(scale))
-    return PA_ERR_INVALID;
   if (num_seqs > PA_NOALLOC_MAX_SEQS) return PA_ERR_INVALID;   // beyond the fixed scratch
-  if (num_q_heads % num_kv_heads) return PA_ERR_INVALID;
-  if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
-  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
-  if (block_size != 1 && block_size != 8 && block_size != 16 && block_size != 32)
-    return PA_ERR_UNSUPPORTED;
-  const int group = num_q_heads / num_kv_heads;
-  if (group > pkv::kMaxGroup) return PA_ERR_UNSUPPORTED;
-  if ((long long)num_blocks * num_kv_heads * block_size >= (1ll << 31) ||
-      (long long)max_blocks_per_seq * block_size >= (1ll << 31) ||
-      (long long)num_seqs * num_kv_heads >= (1ll << 31))
-    return PA_ERR_INVALID;
-  if (num_seqs == 0) return PA_OK;
-  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PA_ERR_INVALID;
-  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
-    return PA_ERR_INVALID;
+  if (num_seqs <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0)
+    return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, 1,
+                       num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                       num_blocks, scale, dtype, nullptr, 0, kNoallocMaxGrid, dev_status, stream);
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
-  const int sms = sm_count();
-  if (sms <= 0) return PA_ERR_CUDA;
-  const int grid = sms * pkv::kCtasPerSm < kNoallocMaxGrid ? sms * pkv::kCtasPerSm : kNoallocMaxGrid;
-  const WsLayout w = ws_layout(num_seqs, head_dim, grid);
-  if (w.total > kNoallocScratchBytes) return PA_ERR_INVALID;
-  uint8_t* ws = static_cast<uint8_t*>(noalloc_scratch(dev));
+  if (head_dim > 128) return PA_ERR_UNSUPPORTED;
+  // the scratch holds the layout of kNoallocMaxGrid CTAs at head_dim 128
+  if (ws_layout(num_seqs, 128, kNoallocMaxGrid).total > kNoallocScratchBytes) return PA_ERR_INVALID;
+  void* ws = noalloc_scratch(dev);
   if (!ws) return PA_ERR_CUDA;
-
-  CUtensorMap mk, mv;
-  std::memset(&mk, 0, sizeof(mk));
-  std::memset(&mv, 0, sizeof(mv));
-  if (block_size != 1) {
-    const uint64_t rows = (uint64_t)num_blocks * num_kv_heads * block_size;
-    const int box_rows = block_size < 16 ? block_size : 16;
-    if (!encode_pool(&mk, k_cache, dtype, head_dim, rows, box_rows) ||
-        !encode_pool(&mv, v_cache, dtype, head_dim, rows, box_rows))
-      return PA_ERR_CUDA;
-  }
-  pkv::DecodeArgs a;
-  a.out = out;
-  a.q = q;
-  a.k_cache = k_cache;
-  a.v_cache = v_cache;
-  a.block_tables = block_tables;
-  a.context_lens = context_lens;
-  a.counters = reinterpret_cast<unsigned long long*>(ws + w.counters_off);
-  a.part_acc = reinterpret_cast<float*>(ws + w.acc_off);
-  a.part_ml = reinterpret_cast<float*>(ws + w.ml_off);
-  a.status = dev_status;
-  a.num_seqs = num_seqs;
-  a.num_q_heads = num_q_heads;
-  a.num_kv_heads = num_kv_heads;
-  a.group = group;
-  a.max_blocks = max_blocks_per_seq;
-  a.num_blocks = num_blocks;
-  a.ctx_cap = max_blocks_per_seq * block_size;
-  a.scale_log2 = scale * 1.4426950408889634f;
-  a.epoch = next_epoch();
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (dtype == PA_BF16) return dispatch_d<__nv_bfloat16>(head_dim, block_size, a, mk, mv, grid, st);
-  return dispatch_d<__half>(head_dim, block_size, a, mk, mv, grid, st);
+  return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, 1,
+                     num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                     num_blocks, scale, dtype, ws, kNoallocScratchBytes, kNoallocMaxGrid,
+                     dev_status, stream);
 }

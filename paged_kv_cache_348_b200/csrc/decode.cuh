@@ -25,10 +25,12 @@
 //    tensor copies (128-byte swizzle, box = min(block_size,16) rows x 64 dims) whose
 //    row coordinate is the physical block id read from the block table; for
 //    block_size 1 with 16-byte cp.async copies.  Stages complete on mbarriers.
-//  * Four consumer warps each take one 16-token unit of a stage.  All q heads of
-//    the GQA group share every K/V byte: S^T = K q^T and O^T += V^T P^T run as
-//    m16n8k16 tensor-core MMAs with the tokens (resp. head dims) on M and the q heads
-//    on N, so a group of 8 heads fills N exactly.  Softmax is an fp32 online softmax
+//  * Four consumer warps each take one 16-token unit of a stage.  All query rows of a
+//    kv head -- the GQA group's heads times the new tokens of the sequence -- share
+//    every K/V byte: S^T = K q^T and O^T += V^T P^T run as m16n8k16 tensor-core MMAs
+//    with the tokens (resp. head dims) on M and those query rows on N (a group of 8
+//    heads fills one n-tile exactly; up to 16 rows are supported).  With several new
+//    tokens, token j is masked from the cached positions after its own.  Softmax is an fp32 online softmax
 //    in base 2; P is split into a 16-bit high part and a 16-bit residual so the PV
 //    product keeps ~16 mantissa bits.
 //  * Every wait is bounded (2 s); on give-up the CTA sets PA_DEV_TIMEOUT and leaves.
@@ -83,6 +85,8 @@ struct DecodeArgs {
   unsigned long long* counters; // [gridDim] arrival counters: (epoch << 32) | arrivals
   int32_t* status;              // nullable
   int num_seqs, num_q_heads, num_kv_heads, group, max_blocks, num_blocks, ctx_cap;
+  int q_len;                    // new tokens per sequence (query rows [seq][q_len][Hq][D])
+  int ncol;                     // query rows per kv head: group * q_len (MMA columns)
   float scale_log2;             // scale * log2(e)
   uint32_t epoch;               // distinct per call: counters of older calls read as zero
 };
@@ -204,7 +208,7 @@ __device__ __forceinline__ void merge_split(const DecodeArgs& a, const SplitDesc
   constexpr int kF4 = D / 4;
   constexpr int kPer = (8 * NT * kF4 + kThr - 1) / kThr;  // float4 elements per thread (max)
   constexpr int kMC = kPer >= 4 ? 2 : 4;                    // contributors per round trip
-  const int nel = group * kF4;
+  const int nel = a.ncol * kF4;
   const int nr = dsc.cl - dsc.cf + 1;
   float M[kPer], Lsum[kPer];
   float4 acc[kPer];
@@ -250,17 +254,18 @@ __device__ __forceinline__ void merge_split(const DecodeArgs& a, const SplitDesc
         M[e] = mn;
       }
   }
-  T* outp = static_cast<T*>(a.out) +
-            ((long long)dsc.seq * a.num_q_heads + (long long)dsc.kvh * group) * D;
 #pragma unroll
   for (int e = 0; e < kPer; ++e) {
     const int i = tid + kThr * e;
     if (i >= nel) continue;
-    const int h = i / kF4, d4 = i % kF4;
-    const float inv = 1.f / Lsum[e];
+    const int h = i / kF4, d4 = i % kF4;           // query column, 4-dim group
+    T* outp = static_cast<T*>(a.out) +
+              (((long long)dsc.seq * a.q_len + h / group) * a.num_q_heads +
+               (long long)dsc.kvh * group + h % group) * D;
+    const float inv = Lsum[e] > 0.f ? 1.f / Lsum[e] : 0.f;
     const uint32_t lo = pack2<T>(acc[e].x * inv, acc[e].y * inv);
     const uint32_t hi = pack2<T>(acc[e].z * inv, acc[e].w * inv);
-    *reinterpret_cast<uint2*>(outp + h * D + d4 * 4) = make_uint2(lo, hi);
+    *reinterpret_cast<uint2*>(outp + d4 * 4) = make_uint2(lo, hi);
   }
 }
 
@@ -334,8 +339,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           const int src = __ffs(zero) - 1;
           zero &= zero - 1;
           uint4* row = reinterpret_cast<uint4*>(static_cast<T*>(a.out) +
-                                                (long long)(base + src) * a.num_q_heads * D);
-          for (int i = lane; i < a.num_q_heads * D * 2 / 16; i += 32) row[i] = make_uint4(0, 0, 0, 0);
+                                                (long long)(base + src) * a.q_len * a.num_q_heads * D);
+          for (int i = lane; i < a.q_len * a.num_q_heads * D * 2 / 16; i += 32)
+            row[i] = make_uint4(0, 0, 0, 0);
         }
       }
     }
@@ -434,9 +440,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           }
           const int flags = (tu == x ? F_FIRST : 0) | (tu + kUnitsPerStage >= pe ? F_LAST : 0) |
                             (complete ? F_COMPLETE : 0);
-          const uint32_t qbytes = (flags & F_FIRST) ? (uint32_t)(group * D * 2) : 0u;
+          // the query rows of this kv head: group consecutive heads of each new token,
+          // one bulk copy per token, stored as columns c = token * group + head
+          const uint32_t qrow_bytes = (uint32_t)(group * D * 2);
+          const uint32_t qbytes = (flags & F_FIRST) ? qrow_bytes * (uint32_t)a.q_len : 0u;
           const T* qsrc = static_cast<const T*>(a.q) +
-                          ((long long)s_cur * a.num_q_heads + (long long)kvh * group) * D;
+                          ((long long)s_cur * a.q_len * a.num_q_heads + (long long)kvh * group) * D;
           if constexpr (BS != 1) {
             constexpr int H = BS < 16 ? BS : 16;     // rows per TMA box
             constexpr int BPU = kUnit / H;           // boxes per unit and column half
@@ -483,7 +492,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             if (lane == 0) {
               meta[st] = StageMeta{s_cur, kvh, tok0, nun, ctx_cur, flags, pidx, qslot};
               mbar_arrive_expect_tx(&full[st], bytes);
-              if (qbytes) bulk_load(sQ, qsrc, qbytes, &full[st]);
+              if (qbytes)
+                for (int j = 0; j < a.q_len; ++j)
+                  bulk_load(sQ + j * qrow_bytes, qsrc + (long long)j * a.num_q_heads * D,
+                            qrow_bytes, &full[st]);
             }
             __syncwarp();
             if (mine) {
@@ -507,7 +519,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             if (lane == 0) {
               meta[st] = StageMeta{s_cur, kvh, tok0, nun, ctx_cur, flags, pidx, qslot};
               mbar_arrive_expect_tx(&full[st], qbytes);
-              if (qbytes) bulk_load(sQ, qsrc, qbytes, &full[st]);
+              if (qbytes)
+                for (int j = 0; j < a.q_len; ++j)
+                  bulk_load(sQ + j * qrow_bytes, qsrc + (long long)j * a.num_q_heads * D,
+                            qrow_bytes, &full[st]);
             }
             const int ch = lane % CPR, hf = ch >> 3, cc = ch & 7;
             for (int r0 = 0; r0 < ntok; r0 += RPI) {
@@ -575,6 +590,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     }
 #pragma unroll
   for (int n = 0; n < NT; ++n) m[n][0] = m[n][1] = -INFINITY, l[n][0] = l[n][1] = 0.f;
+  // new-token index of this lane's two accumulator columns per n-tile
+  int jcol[NT][2];
+#pragma unroll
+  for (int n = 0; n < NT; ++n) {
+    jcol[n][0] = (n * 8 + 2 * tig) / group;
+    jcol[n][1] = (n * 8 + 2 * tig + 1) / group;
+  }
 
   int st = 0;
   uint32_t ph = 0;
@@ -594,12 +616,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     if (mt.flags & F_FIRST) {
 #pragma unroll
       for (int n = 0; n < NT; ++n) {
-        const int h = n * 8 + gid;
+        const int cq = n * 8 + gid;                  // this lane's query column
 #pragma unroll
         for (int ks = 0; ks < KS; ++ks) {
           uint32_t b0 = 0u, b1 = 0u;
-          if (h < group) {
-            const uint32_t* qrow = reinterpret_cast<const uint32_t*>(sQ + h * D * 2);
+          if (cq < a.ncol) {
+            const uint32_t* qrow = reinterpret_cast<const uint32_t*>(sQ + cq * D * 2);
             b0 = qrow[(ks * 16 + 2 * tig) >> 1];
             b1 = qrow[(ks * 16 + 8 + 2 * tig) >> 1];
           }
@@ -615,6 +637,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     if (cw < mt.nunits) {
       const int t0 = mt.tok0 + cw * kUnit;
       const int valid = (mt.ctx - t0) < kUnit ? (mt.ctx - t0) : kUnit;
+      // causal limit: new token j sees unit rows < ctx - q_len + 1 + j - t0
+      const int lim0 = mt.ctx - a.q_len + 1 - t0;
       const uint32_t kbase = smem_u32(sK), vbase = smem_u32(sV);
       // ---- S^T[16 tokens][8*NT heads] = K_unit . q^T
       float sacc[NT][4];
@@ -634,7 +658,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           for (int n = 0; n < NT; ++n) mma16816<kBF16>(sacc[n], a0, a1, a2, a3, qf[ks][n][0], qf[ks][n][1]);
         }
       }
-      // ---- online softmax (base 2) per head column
+      // ---- online softmax (base 2) per query column
       uint32_t bhi[NT][2], blo[NT][2];
 #pragma unroll
       for (int n = 0; n < NT; ++n) {
@@ -642,7 +666,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int row = gid + (e >= 2 ? 8 : 0);
-          xs[e] = row < valid ? sacc[n][e] * a.scale_log2 : -INFINITY;
+          const int lim = lim0 + jcol[n][e & 1];
+          xs[e] = (row < valid && row < lim) ? sacc[n][e] * a.scale_log2 : -INFINITY;
         }
         float alpha[2], p[4];
 #pragma unroll
@@ -652,10 +677,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
           const float mnew = fmaxf(m[n][cc], mx);
-          alpha[cc] = ex2(m[n][cc] - mnew);
+          // a column with no visible row yet keeps max -inf: use 0 as the reference
+          const float mref = mnew == -INFINITY ? 0.f : mnew;
+          alpha[cc] = ex2(m[n][cc] - mref);
           m[n][cc] = mnew;
-          p[cc] = ex2(xs[cc] - mnew);
-          p[cc + 2] = ex2(xs[cc + 2] - mnew);
+          p[cc] = ex2(xs[cc] - mref);
+          p[cc + 2] = ex2(xs[cc + 2] - mref);
           l[n][cc] = l[n][cc] * alpha[cc] + p[cc] + p[cc + 2];
         }
 #pragma unroll
@@ -733,14 +760,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       }
       named_bar_sync(1, kConsumerThreads);
       const bool complete = mt.flags & F_COMPLETE;
-      T* outp = static_cast<T*>(a.out) +
-                ((long long)mt.seq * a.num_q_heads + (long long)mt.kvh * group) * D;
       for (int pi = tid; pi < NREG * 32; pi += kConsumerThreads) {
         const int r = pi >> 5, ln = pi & 31;
         const int e = r & 3, n = (r >> 2) % NT, mtile = (r >> 2) / NT;
         const int d = mtile * 16 + (ln >> 2) + (e >= 2 ? 8 : 0);
-        const int h = n * 8 + 2 * (ln & 3) + (e & 1);
-        if (h >= group) continue;
+        const int h = n * 8 + 2 * (ln & 3) + (e & 1);   // query column
+        if (h >= a.ncol) continue;
         float M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, mls[w * kMaxGroup + h].x);
@@ -753,7 +778,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           acc += scr[(w * NREG + r) * 32 + ln] * sc;
         }
         if (complete) {
-          outp[h * D + d] = from_float<T>(acc / Lsum);
+          // column h = new token h / group, head kvh * group + h % group; a row that
+          // sees no token at all (a new token before the context start) is zero
+          T* outp = static_cast<T*>(a.out) +
+                    (((long long)mt.seq * a.q_len + h / group) * a.num_q_heads +
+                     (long long)mt.kvh * group + h % group) * D;
+          outp[d] = from_float<T>(Lsum > 0.f ? acc / Lsum : 0.f);
         } else {
           a.part_acc[((long long)mt.pidx * kMaxGroup + h) * D + d] = acc;
           if (d == 0) {

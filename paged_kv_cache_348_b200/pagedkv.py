@@ -23,7 +23,7 @@ DEV_BAD_BLOCK_ID, DEV_BAD_SLOT, DEV_BAD_PAIR, DEV_BAD_CONTEXT_LEN, DEV_TIMEOUT =
 
 # every symbol include/pagedkv.h declares
 EXPORTS = ("pa_version", "pa_status_string", "pa_decode_workspace_bytes", "pa_decode",
-           "pa_cache_append", "pa_copy_blocks", "pa_decode_noalloc")
+           "pa_decode_multi", "pa_cache_append", "pa_copy_blocks", "pa_decode_noalloc")
 
 _lib = None
 _lock = threading.Lock()
@@ -53,6 +53,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         L.pa_decode.restype = i32
         L.pa_decode.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, f32, i32,
                                 P, sz, P, P]
+        L.pa_decode_multi.restype = i32
+        L.pa_decode_multi.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, i32,
+                                      f32, i32, P, sz, P, P]
         L.pa_cache_append.restype = i32
         L.pa_cache_append.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, P, P]
         L.pa_copy_blocks.restype = i32
@@ -135,6 +138,31 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale: float
                           workspace.numel() * workspace.element_size(), _ptr(status),
                           _stream(stream))
     _check(rc, "pa_decode")
+    return out
+
+
+def pa_decode_multi(out, q, k_cache, v_cache, block_tables, context_lens, scale: float,
+                    workspace, status=None, stream=None):
+    """out[B,QL,Hq,D] <- paged decode of QL new tokens per sequence, causal among them
+    (see pa_decode_multi in include/pagedkv.h)."""
+    _need(q, "q", ndim=4)
+    _need(out, "out", dtype=q.dtype, ndim=4)
+    _need(k_cache, "k_cache", dtype=q.dtype, ndim=4)
+    _need(v_cache, "v_cache", dtype=q.dtype, ndim=4)
+    _need(block_tables, "block_tables", dtype=torch.int32, ndim=2)
+    _need(context_lens, "context_lens", dtype=torch.int32, ndim=1)
+    _need(workspace, "workspace")
+    B, QL, Hq, D = q.shape
+    N, Hkv, bs, D2 = k_cache.shape
+    if out.shape != q.shape or D2 != D or v_cache.shape != k_cache.shape or \
+            block_tables.shape[0] != B or context_lens.shape[0] != B:
+        raise PagedKVError("pa_decode_multi: inconsistent shapes")
+    rc = load().pa_decode_multi(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                _ptr(block_tables), _ptr(context_lens), B, QL, Hq, Hkv, D, bs,
+                                block_tables.shape[1], N, float(scale), _dtype_code(q),
+                                _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                _ptr(status), _stream(stream))
+    _check(rc, "pa_decode_multi")
     return out
 
 
