@@ -34,7 +34,7 @@ METRIC = "paged decode attn: KV-read HBM GB/s (% of B200 peak) and seq-steps/s"
 FALLBACK_HBM_GBS = 6650.0
 
 
-def workload_desc(w, bs, layers=0):
+def workload_desc(w, bs, layers=0, q_len=1):
     from paged_kv_cache_348_b200 import inputs
 
     ctx = {"tiny": "{5,16,17,40}", "llama8b": "U[128,2048]", "llama70b": "U[1000,8000]",
@@ -43,7 +43,8 @@ def workload_desc(w, bs, layers=0):
     return ("%s-shape paged decode step: %d layer(s), batch %d, %d q / %d kv heads, head_dim %d, "
             "block_size %d, %s, context lens %s, seed %d" % (
                 w.name, layers or w.layers, w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, bs,
-                w.dtype, ctx, w.seed))
+                w.dtype, ctx, w.seed)) + (", %d new tokens per sequence (causal)" % q_len
+                                          if q_len > 1 else "")
 
 
 def source_hash():
@@ -174,8 +175,9 @@ def oracle_sample(w, bs, max_seconds=15.0, device_batch=None):
     while i < len(order) and spent < max_seconds:
         items = order[i:i + chunk]
         t0 = time.perf_counter()
-        oracle.decode(q, k, v, tables, ctx, 1.0 / math.sqrt(w.head_dim), w.dtype, items=items,
-                      nthreads=threads)
+        fn = oracle.decode if q.ndim == 3 else oracle.decode_multi
+        fn(q, k, v, tables, ctx, 1.0 / math.sqrt(w.head_dim), w.dtype, items=items,
+           nthreads=threads)
         spent += time.perf_counter() - t0
         done_bytes += int(sum(int(ctx[s]) for s in items)) * w.num_kv_heads * w.head_dim * 4
         seqs += len(items)
@@ -225,6 +227,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama70b")
     ap.add_argument("--block-size", type=int, default=0)
+    ap.add_argument("--q-len", type=int, default=1,
+                    help="new tokens per sequence (pa_decode_multi when > 1)")
     ap.add_argument("--layers", type=int, default=0,
                     help="layers of the workload to run (0: all; fewer only for profiling)")
     ap.add_argument("--no-e2e", action="store_true")
@@ -257,7 +261,8 @@ def main():
     if w.name == "prefix":
         b = wl.build_prefix_decode(w, device="cuda")
     else:
-        b = wl.build(w, device="cuda", block_size=bs, layers=args.layers or None)
+        b = wl.build(w, device="cuda", block_size=bs, layers=args.layers or None,
+                     q_len=args.q_len)
     stream = torch.cuda.current_stream()
     L = b.layers
     kv_step = b.kv_bytes_per_step()
@@ -302,8 +307,7 @@ def main():
             pk.pa_cache_append(b.k_caches[l], b.v_caches[l], b.k_new[l], b.v_new[l],
                                b.slot_mapping, b.status)
             ev_s[s * L + l].record(stream)
-            pk.pa_decode(b.out[l], b.q[l], b.k_caches[l], b.v_caches[l], b.block_tables,
-                         b.context_lens, b.scale, b.workspace, b.status)
+            wl.decode_layer(b, l)
             ev_e[s * L + l].record(stream)
     barrier()
     dec_ms = [a.elapsed_time(e) for a, e in zip(ev_s, ev_e)]
@@ -330,7 +334,7 @@ def main():
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-        "config": {"workload": workload_desc(w, bs, b.layers), "global_batch": w.num_seqs * world,
+        "config": {"workload": workload_desc(w, bs, b.layers, b.q_len), "global_batch": w.num_seqs * world,
                    "seq_len": float(b.context_lens.float().mean().item()),
                    "parallelism": "replicas" if world > 1 else "single gpu",
                    "l2": "inputs larger than L2 (%.2f GB of K/V per layer)" % (kv_layer / 1e9)},
@@ -338,7 +342,8 @@ def main():
         "peak_hbm_gbs": peak, "peak_kind": peak_kind,
         "seq_steps_per_s": world * w.num_seqs / (ms_step * 1e-3),
         "kv_bytes_per_step": kv_step,
-        "roofline": {"bound": "hbm", "kernel": "pa_decode_split_kernel (one launch per pa_decode)",
+        "roofline": {"bound": "hbm", "kernel": "pa_decode_split_kernel (one launch per %s)" % (
+                         "pa_decode" if b.q_len == 1 else "pa_decode_multi"),
                      "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "algorithmic_bytes_per_launch": kv_layer,
@@ -415,8 +420,9 @@ def run_e2e(b, args, world, kv_step):
             comp.wait_event(ev_out[l])
             pk.pa_cache_append(b.k_caches[l], b.v_caches[l], b.k_new[l], b.v_new[l], slots[m],
                                b.status, comp)
-            pk.pa_decode(b.out[l], b.q[l], b.k_caches[l], b.v_caches[l], tabs[m], ctxs[m],
-                         b.scale, b.workspace, b.status, comp)
+            fn = pk.pa_decode if b.q_len == 1 else pk.pa_decode_multi
+            fn(b.out[l], b.q[l], b.k_caches[l], b.v_caches[l], tabs[m], ctxs[m], b.scale,
+               b.workspace, b.status, comp)
             ev_used[l].record(comp)
         ev_meta_free[m].record(comp)
         with torch.cuda.stream(down):

@@ -43,6 +43,7 @@ class DecodeBatch:
     status: torch.Tensor
     cow_pairs: torch.Tensor | None
     scale: float
+    q_len: int = 1
 
     @property
     def layers(self) -> int:
@@ -80,42 +81,44 @@ def _alloc_layers(w, N, bs, layers, device, seed):
     return k, v
 
 
-def _finish(w, bs, bm, sids, N, layers, device, cow_pairs=None) -> DecodeBatch:
+def _finish(w, bs, bm, sids, N, layers, device, cow_pairs=None, q_len=1) -> DecodeBatch:
     B = len(sids)
     k_caches, v_caches = _alloc_layers(w, N, bs, layers, device, w.seed)
     tables = torch.from_numpy(bm.block_tables(sids)).to(device)
     ctx = torch.from_numpy(bm.context_lens(sids)).to(device)
-    slots = torch.tensor([bm.slot_of(s, bm.context_len(s) - 1) for s in sids], dtype=torch.int64,
-                         device=device)
+    # the newest q_len tokens of every sequence are the ones appended and queried
+    slots = torch.tensor([bm.slot_of(s, bm.context_len(s) - q_len + j) for s in sids
+                          for j in range(q_len)], dtype=torch.int64, device=device)
+    qshape = (B, w.num_q_heads, w.head_dim) if q_len == 1 else \
+        (B, q_len, w.num_q_heads, w.head_dim)
     q, kn, vn, out = [], [], [], []
     for l in range(layers):
-        q.append(inputs.randn((B, w.num_q_heads, w.head_dim), w.dtype, w.seed, device,
-                              stream=5000 + 3 * l))
-        kn.append(inputs.randn((B, w.num_kv_heads, w.head_dim), w.dtype, w.seed, device,
+        q.append(inputs.randn(qshape, w.dtype, w.seed, device, stream=5000 + 3 * l))
+        kn.append(inputs.randn((B * q_len, w.num_kv_heads, w.head_dim), w.dtype, w.seed, device,
                                stream=5001 + 3 * l))
-        vn.append(inputs.randn((B, w.num_kv_heads, w.head_dim), w.dtype, w.seed, device,
+        vn.append(inputs.randn((B * q_len, w.num_kv_heads, w.head_dim), w.dtype, w.seed, device,
                                stream=5002 + 3 * l))
-        out.append(torch.empty((B, w.num_q_heads, w.head_dim), dtype=inputs.torch_dtype(w.dtype),
-                               device=device))
+        out.append(torch.empty(qshape, dtype=inputs.torch_dtype(w.dtype), device=device))
     ws = pk.new_workspace(B, w.num_q_heads, w.num_kv_heads, w.head_dim, device)
     st = pk.new_status(device)
     pairs = None
     if cow_pairs:
         pairs = torch.tensor(cow_pairs, dtype=torch.int32, device=device).reshape(-1, 2)
     return DecodeBatch(w, bs, bm, sids, N, k_caches, v_caches, tables, ctx, slots, q, kn, vn, out,
-                       ws, st, pairs, 1.0 / math.sqrt(w.head_dim))
+                       ws, st, pairs, 1.0 / math.sqrt(w.head_dim), q_len)
 
 
 def build(w: inputs.Workload, device="cuda", block_size: int | None = None,
-          layers: int | None = None) -> DecodeBatch:
-    """Independent sequences (every workload but the shared-prefix one)."""
+          layers: int | None = None, q_len: int = 1) -> DecodeBatch:
+    """Independent sequences (every workload but the shared-prefix one).  With q_len > 1
+    every sequence's newest q_len tokens are appended and queried each step."""
     bs = block_size or w.block_size
     ctx = inputs.context_lens(w)
     need = int(sum(-(-int(c) // bs) for c in ctx))
     N = _pool_size(w, need)
     bm = BlockManager(N, bs, inputs.pool_order(N, w.seed))
     sids = [bm.allocate(int(c)) for c in ctx]
-    return _finish(w, bs, bm, sids, N, layers or w.layers, device)
+    return _finish(w, bs, bm, sids, N, layers or w.layers, device, q_len=q_len)
 
 
 def build_prefix_decode(w: inputs.Workload = inputs.PREFIX, device="cuda") -> DecodeBatch:
@@ -167,5 +170,11 @@ def run_step(b: DecodeBatch, stream=None, layers=None) -> None:
     for l in range(layers if layers is not None else b.layers):
         pk.pa_cache_append(b.k_caches[l], b.v_caches[l], b.k_new[l], b.v_new[l], b.slot_mapping,
                            b.status, stream)
-        pk.pa_decode(b.out[l], b.q[l], b.k_caches[l], b.v_caches[l], b.block_tables,
-                     b.context_lens, b.scale, b.workspace, b.status, stream)
+        decode_layer(b, l, stream)
+
+
+def decode_layer(b: DecodeBatch, l: int, stream=None) -> None:
+    """pa_decode (one new token per sequence) or pa_decode_multi (q_len > 1) of layer l."""
+    fn = pk.pa_decode if b.q_len == 1 else pk.pa_decode_multi
+    fn(b.out[l], b.q[l], b.k_caches[l], b.v_caches[l], b.block_tables, b.context_lens, b.scale,
+       b.workspace, b.status, stream)
