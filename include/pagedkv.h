@@ -44,7 +44,9 @@ typedef enum {
   PA_OK = 0,
   PA_ERR_INVALID = 1,      /* null/misaligned pointer, bad size, workspace too small */
   PA_ERR_UNSUPPORTED = 2,  /* head_dim, block_size, dtype or group size not built */
-  PA_ERR_CUDA = 3          /* a CUDA runtime/driver call or launch failed */
+  PA_ERR_CUDA = 3,         /* a CUDA runtime/driver call or launch failed */
+  PA_ERR_NO_BLOCKS = 4,    /* block manager: not enough free blocks; nothing was changed */
+  PA_ERR_NO_MEMORY = 5     /* block manager: host memory allocation failed */
 } pa_status;
 
 typedef enum { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
@@ -202,6 +204,72 @@ pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache, const
                             int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                             int block_size, int max_blocks_per_seq, int num_blocks, float scale,
                             pa_dtype dtype, int32_t* dev_status, void* stream);
+
+/* ======================================================================================
+ * Host block manager (pa_bm_*): the bookkeeping that produces the kernels' inputs.
+ *
+ * Defined by [P2] "Core Principle" (logical blocks of a request map to physical blocks
+ * through its block table; blocks are allocated on demand and returned to the pool when
+ * the request finishes), [P1] "How PagedAttention borrows OS paging" (requests with an
+ * identical prefix point their tables at the same physical blocks; a new block is
+ * allocated only when a sequence diverges -- copy-on-write), [P3] "How It Works" and
+ * "Why This Matters for Production" (parallel sampling and beam search share blocks).
+ *
+ * Host-only: no call touches a GPU, and every pointer below is a HOST pointer.  A
+ * manager owns a pool of num_blocks block ids; free ids are handed out first-in
+ * first-out in the order given at creation (NULL: 0, 1, 2, ...), and released ids
+ * join the back of that queue.  Sequence ids are assigned 0, 1, 2, ... and never
+ * reused.  Not thread-safe: serialise calls on one manager.  Errors change nothing.
+ * ====================================================================================== */
+typedef struct pa_block_manager pa_block_manager;
+
+/* New manager over block ids 0..num_blocks-1 of block_size tokens each.  free_order,
+ * if not NULL, is a permutation of 0..num_blocks-1 (PA_ERR_INVALID otherwise). */
+pa_status pa_bm_create(int num_blocks, int block_size, const int32_t* free_order,
+                       pa_block_manager** out);
+void pa_bm_destroy(pa_block_manager* bm);
+
+/* Free blocks in the pool; the reference count of one block (-1: bad id). */
+int pa_bm_free_blocks(const pa_block_manager* bm);
+int pa_bm_refcount(const pa_block_manager* bm, int block);
+
+/* A new sequence holding num_tokens cached tokens (a prefill): ceil(num_tokens /
+ * block_size) fresh blocks.  PA_ERR_NO_BLOCKS if the pool cannot hold them. */
+pa_status pa_bm_allocate(pa_block_manager* bm, int num_tokens, int32_t* seq_id);
+
+/* A new sequence sharing every block of `seq` (each block's count goes up by one). */
+pa_status pa_bm_fork(pa_block_manager* bm, int32_t seq, int32_t* child);
+
+/* Reserve the slot of the next token of each of seqs[0..n) in order (a sequence may
+ * appear more than once).  For token i: slots[i] = physical block * block_size +
+ * offset.  A token that starts a new logical block gets a fresh block; a token that
+ * lands in a block shared with other sequences gets a private copy: the pair (shared
+ * block, fresh block) is written to cow_pairs[2k], cow_pairs[2k+1] (cow_pairs must
+ * hold 2n ints) and *num_cow counts them -- pass them to pa_copy_blocks before
+ * pa_cache_append.  If the pool cannot serve the whole batch, returns
+ * PA_ERR_NO_BLOCKS and changes nothing. */
+pa_status pa_bm_append_tokens(pa_block_manager* bm, const int32_t* seqs, int n, int64_t* slots,
+                              int32_t* cow_pairs, int* num_cow);
+
+/* Drop a sequence: every block's count goes down by one; blocks reaching zero return
+ * to the back of the free queue. */
+pa_status pa_bm_release(pa_block_manager* bm, int32_t seq);
+
+/* Cached tokens / blocks held by a sequence (-1: unknown sequence). */
+int64_t pa_bm_context_len(const pa_block_manager* bm, int32_t seq);
+int pa_bm_num_blocks_of(const pa_block_manager* bm, int32_t seq);
+
+/* Longest block table among seqs[0..n) (-1: an unknown sequence). */
+int pa_bm_max_blocks(const pa_block_manager* bm, const int32_t* seqs, int n);
+
+/* Fill tables[n][width] with the block tables of seqs[0..n) (entries past a table's
+ * end = fill) and, if not NULL, context_lens[n].  PA_ERR_INVALID if a table is wider
+ * than width or a sequence is unknown. */
+pa_status pa_bm_block_tables(const pa_block_manager* bm, const int32_t* seqs, int n, int width,
+                             int32_t fill, int32_t* tables, int32_t* context_lens);
+
+/* Flat slot of cached position pos (0 <= pos < context length) of seq. */
+pa_status pa_bm_slot_of(const pa_block_manager* bm, int32_t seq, int64_t pos, int64_t* slot);
 
 #ifdef __cplusplus
 }

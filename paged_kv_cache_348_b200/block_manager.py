@@ -14,16 +14,60 @@ Problem", section "How It Works".
 
 It produces exactly what the CUDA calls consume: int32 block tables, int32 context
 lengths, int64 slot mappings and int32 (src, dst) copy pairs.
+
+The bookkeeping itself is native: this class is a ctypes wrapper over the pa_bm_*
+calls of libpagedkv (include/pagedkv.h, csrc/block_manager.cpp).  It needs the
+library but no GPU.
 """
 from __future__ import annotations
 
-from collections import deque
+import ctypes
 
 import numpy as np
+
+from . import pagedkv as pk
 
 
 class PoolExhausted(MemoryError):
     pass
+
+
+def _lib():
+    L = pk.load()
+    if not getattr(L, "_bm_ready", False):
+        P, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+        L.pa_bm_create.argtypes = [i32, i32, P, ctypes.POINTER(P)]
+        L.pa_bm_create.restype = i32
+        L.pa_bm_destroy.argtypes = [P]
+        L.pa_bm_destroy.restype = None
+        L.pa_bm_free_blocks.argtypes = [P]
+        L.pa_bm_free_blocks.restype = i32
+        L.pa_bm_refcount.argtypes = [P, i32]
+        L.pa_bm_refcount.restype = i32
+        L.pa_bm_allocate.argtypes = [P, i32, P]
+        L.pa_bm_allocate.restype = i32
+        L.pa_bm_fork.argtypes = [P, i32, P]
+        L.pa_bm_fork.restype = i32
+        L.pa_bm_append_tokens.argtypes = [P, P, i32, P, P, P]
+        L.pa_bm_append_tokens.restype = i32
+        L.pa_bm_release.argtypes = [P, i32]
+        L.pa_bm_release.restype = i32
+        L.pa_bm_context_len.argtypes = [P, i32]
+        L.pa_bm_context_len.restype = i64
+        L.pa_bm_num_blocks_of.argtypes = [P, i32]
+        L.pa_bm_num_blocks_of.restype = i32
+        L.pa_bm_max_blocks.argtypes = [P, P, i32]
+        L.pa_bm_max_blocks.restype = i32
+        L.pa_bm_block_tables.argtypes = [P, P, i32, i32, i32, P, P]
+        L.pa_bm_block_tables.restype = i32
+        L.pa_bm_slot_of.argtypes = [P, i32, i64, P]
+        L.pa_bm_slot_of.restype = i32
+        L._bm_ready = True
+    return L
+
+
+def _ptr(a: np.ndarray):
+    return ctypes.c_void_p(a.ctypes.data)
 
 
 class BlockManager:
@@ -32,109 +76,124 @@ class BlockManager:
             raise ValueError("num_blocks and block_size must be positive")
         self.num_blocks = num_blocks
         self.block_size = block_size
-        order = range(num_blocks) if free_order is None else [int(b) for b in free_order]
-        self._free = deque(order)
-        if len(self._free) != num_blocks or len(set(self._free)) != num_blocks:
+        L = _lib()
+        order = None
+        if free_order is not None:
+            order = np.ascontiguousarray(np.asarray(free_order, dtype=np.int32))
+            if order.shape != (num_blocks,):
+                raise ValueError("free_order must be a permutation of the pool")
+        h = ctypes.c_void_p()
+        rc = L.pa_bm_create(num_blocks, block_size, None if order is None else _ptr(order),
+                            ctypes.byref(h))
+        if rc == pk.PA_ERR_INVALID:
             raise ValueError("free_order must be a permutation of the pool")
-        self._ref = np.zeros(num_blocks, dtype=np.int32)
-        self._tables: dict[int, list[int]] = {}
-        self._lens: dict[int, int] = {}
-        self._next_id = 0
+        if rc != pk.PA_OK:
+            raise RuntimeError("pa_bm_create failed (%d)" % rc)
+        self._h = h
+        self._L = L
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value:
+            self._L.pa_bm_destroy(h)
+            self._h = None
+
+    def _check(self, rc: int, what: str):
+        if rc == pk.PA_ERR_NO_BLOCKS:
+            raise PoolExhausted("%s: not enough free KV blocks (%d free)" % (what, self.free_blocks))
+        if rc != pk.PA_OK:
+            raise ValueError("%s failed (%d)" % (what, rc))
 
     # ---------------------------------------------------------------- allocation
     @property
     def free_blocks(self) -> int:
-        return len(self._free)
+        return int(self._L.pa_bm_free_blocks(self._h))
 
     def refcount(self, block: int) -> int:
-        return int(self._ref[block])
-
-    def _take(self) -> int:
-        if not self._free:
-            raise PoolExhausted("no free KV block left")
-        b = self._free.popleft()
-        self._ref[b] = 1
-        return b
-
-    def _blocks_for(self, n_tokens: int) -> int:
-        return -(-n_tokens // self.block_size)
+        r = int(self._L.pa_bm_refcount(self._h, int(block)))
+        if r < 0:
+            raise IndexError(block)
+        return r
 
     def allocate(self, n_tokens: int) -> int:
         """New sequence holding n_tokens cached tokens; returns its id."""
-        need = self._blocks_for(n_tokens)
-        if need > len(self._free):
-            raise PoolExhausted("need %d blocks, %d free" % (need, len(self._free)))
-        sid = self._next_id
-        self._next_id += 1
-        self._tables[sid] = [self._take() for _ in range(need)]
-        self._lens[sid] = n_tokens
-        return sid
+        sid = ctypes.c_int32()
+        self._check(self._L.pa_bm_allocate(self._h, int(n_tokens), ctypes.byref(sid)), "allocate")
+        return sid.value
 
     def fork(self, sid: int) -> int:
         """New sequence sharing every block of `sid` (parallel sampling / beams)."""
-        child = self._next_id
-        self._next_id += 1
-        self._tables[child] = list(self._tables[sid])
-        self._lens[child] = self._lens[sid]
-        for b in self._tables[child]:
-            self._ref[b] += 1
-        return child
+        child = ctypes.c_int32()
+        self._check(self._L.pa_bm_fork(self._h, int(sid), ctypes.byref(child)), "fork")
+        return child.value
+
+    def append_tokens(self, sids):
+        """Reserve the next slot of each listed sequence, in order.  Returns (slots
+        int64 [n], copy-on-write pairs int32 [k, 2]) -- the pairs must be copied before
+        the new tokens are written."""
+        s = np.ascontiguousarray(np.asarray(sids, dtype=np.int32))
+        n = s.shape[0]
+        slots = np.zeros(n, dtype=np.int64)
+        pairs = np.zeros((max(n, 1), 2), dtype=np.int32)
+        nc = ctypes.c_int()
+        self._check(self._L.pa_bm_append_tokens(self._h, _ptr(s), n, _ptr(slots), _ptr(pairs),
+                                                ctypes.byref(nc)), "append")
+        return slots, pairs[:nc.value].copy()
 
     def append_token(self, sid: int):
         """Reserve the slot of the next token of `sid`.
 
         Returns (slot, cow): slot = physical_block * block_size + offset, and cow is
         None or the (src, dst) block pair to copy before the new token is written."""
-        pos = self._lens[sid]
-        lb, off = divmod(pos, self.block_size)
-        table = self._tables[sid]
-        cow = None
-        if lb == len(table):
-            table.append(self._take())
-        elif self._ref[table[lb]] > 1:
-            src = table[lb]
-            dst = self._take()
-            self._ref[src] -= 1
-            table[lb] = dst
-            cow = (src, dst)
-        self._lens[sid] = pos + 1
-        return table[lb] * self.block_size + off, cow
+        slots, pairs = self.append_tokens([sid])
+        cow = (int(pairs[0, 0]), int(pairs[0, 1])) if len(pairs) else None
+        return int(slots[0]), cow
 
     def release(self, sid: int) -> None:
-        for b in self._tables.pop(sid):
-            self._ref[b] -= 1
-            if self._ref[b] == 0:
-                self._free.append(b)
-        del self._lens[sid]
+        self._check(self._L.pa_bm_release(self._h, int(sid)), "release")
 
     # ---------------------------------------------------------------- views
     def table(self, sid: int) -> list[int]:
-        return list(self._tables[sid])
+        n = int(self._L.pa_bm_num_blocks_of(self._h, int(sid)))
+        if n < 0:
+            raise KeyError(sid)
+        return [int(x) for x in self.block_tables([sid], width=max(n, 1))[0, :n]]
 
     def context_len(self, sid: int) -> int:
-        return self._lens[sid]
+        n = int(self._L.pa_bm_context_len(self._h, int(sid)))
+        if n < 0:
+            raise KeyError(sid)
+        return n
 
     def slot_of(self, sid: int, pos: int) -> int:
         """Flat slot of logical position `pos` of `sid`."""
-        lb, off = divmod(pos, self.block_size)
-        return self._tables[sid][lb] * self.block_size + off
+        out = ctypes.c_int64()
+        self._check(self._L.pa_bm_slot_of(self._h, int(sid), int(pos), ctypes.byref(out)),
+                    "slot_of")
+        return out.value
 
     def block_tables(self, sids, width: int | None = None, fill: int = 0) -> np.ndarray:
-        w = max([len(self._tables[s]) for s in sids] + [1]) if width is None else width
-        out = np.full((len(sids), w), fill, dtype=np.int32)
-        for i, s in enumerate(sids):
-            t = self._tables[s]
-            if len(t) > w:
-                raise ValueError("block table wider than width")
-            out[i, :len(t)] = t
-        return out
+        return self._tables(sids, width, fill)[0]
+
+    def _tables(self, sids, width, fill):
+        s = np.ascontiguousarray(np.asarray(list(sids), dtype=np.int32))
+        if width is None:
+            width = max(int(self._L.pa_bm_max_blocks(self._h, _ptr(s), len(s))), 1)
+        out = np.empty((len(s), width), dtype=np.int32)
+        lens = np.empty(len(s), dtype=np.int32)
+        rc = self._L.pa_bm_block_tables(self._h, _ptr(s), len(s), int(width), int(fill),
+                                        _ptr(out), _ptr(lens))
+        if rc != pk.PA_OK:
+            raise ValueError("block table wider than width, or unknown sequence")
+        return out, lens
 
     def context_lens(self, sids) -> np.ndarray:
-        return np.array([self._lens[s] for s in sids], dtype=np.int32)
+        return self._tables(sids, None, 0)[1]
 
     def tail_waste(self, sids) -> float:
         """Fraction of held slots that hold no token: only the unused tail of each
         sequence's last block (shared blocks counted once per sequence)."""
-        held = sum(len(self._tables[s]) * self.block_size for s in sids)
-        used = sum(self._lens[s] for s in sids)
+        held = sum(int(self._L.pa_bm_num_blocks_of(self._h, int(s))) * self.block_size
+                   for s in sids)
+        used = sum(self.context_len(s) for s in sids)
         return 0.0 if held == 0 else (held - used) / held

@@ -237,6 +237,8 @@ const char* pa_status_string(pa_status s) {
     case PA_ERR_INVALID: return "invalid argument";
     case PA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
     case PA_ERR_CUDA: return "CUDA error";
+    case PA_ERR_NO_BLOCKS: return "not enough free blocks";
+    case PA_ERR_NO_MEMORY: return "out of host memory";
   }
   return "unknown status";
 }

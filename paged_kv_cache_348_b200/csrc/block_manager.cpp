@@ -1,0 +1,242 @@
+// block_manager.cpp -- host-side block manager of a paged KV cache (declared in
+// include/pagedkv.h, pa_bm_*): a pool of fixed-size physical blocks, one block table per
+// sequence, reference counts, on-demand allocation, copy-on-write on divergence, and
+// release back to the pool.
+//
+// Follows "PagedAttention in Production: Boosting LLM Serving Throughput with Paged KV
+// Cache", section "Core Principle" (logical blocks map to physical blocks through a
+// per-request block table; blocks are allocated on demand and returned to the pool when
+// the request finishes); "Paged Attention and Memory Efficiency in Production LLM
+// Serving", section "How PagedAttention borrows OS paging" (requests with an identical
+// prefix point at the same physical blocks and a new block is allocated only when a
+// sequence diverges, as in copy-on-write); "PagedAttention -- The KV Cache Problem",
+// sections "How It Works" (fixed-size blocks, allocate on demand, free immediately) and
+// "Why This Matters for Production" (parallel sampling and beam search share blocks
+// copy-on-write).
+//
+// It produces what the CUDA calls consume: int32 block tables, int32 context lengths,
+// int64 slot mappings and int32 (src, dst) copy pairs.  Not thread-safe: a caller
+// serialises calls on one manager.
+#include <cstdint>
+#include <cstring>
+#include <deque>
+#include <new>
+#include <unordered_map>
+#include <vector>
+
+#include "pagedkv.h"
+
+struct pa_block_manager {
+  struct Seq {
+    std::vector<int32_t> table;  // logical block i -> physical block
+    int64_t len = 0;             // cached tokens
+  };
+  int32_t num_blocks = 0, block_size = 0;
+  std::vector<int32_t> ref;      // reference count per physical block
+  std::deque<int32_t> free;      // free blocks, handed out from the front
+  std::unordered_map<int32_t, Seq> seqs;
+  int32_t next_id = 0;
+
+  int32_t take() {               // caller has checked that a block is free
+    const int32_t b = free.front();
+    free.pop_front();
+    ref[b] = 1;
+    return b;
+  }
+  Seq* find(int32_t id) {
+    auto it = seqs.find(id);
+    return it == seqs.end() ? nullptr : &it->second;
+  }
+  const Seq* find(int32_t id) const {
+    auto it = seqs.find(id);
+    return it == seqs.end() ? nullptr : &it->second;
+  }
+  int64_t blocks_for(int64_t tokens) const { return (tokens + block_size - 1) / block_size; }
+};
+
+extern "C" {
+
+pa_status pa_bm_create(int num_blocks, int block_size, const int32_t* free_order,
+                       pa_block_manager** out) {
+  if (!out) return PA_ERR_INVALID;
+  *out = nullptr;
+  if (num_blocks <= 0 || block_size <= 0) return PA_ERR_INVALID;
+  pa_block_manager* bm = new (std::nothrow) pa_block_manager();
+  if (!bm) return PA_ERR_NO_MEMORY;
+  bm->num_blocks = num_blocks;
+  bm->block_size = block_size;
+  bm->ref.assign((size_t)num_blocks, 0);
+  if (free_order) {
+    std::vector<uint8_t> seen((size_t)num_blocks, 0);
+    for (int i = 0; i < num_blocks; ++i) {
+      const int32_t b = free_order[i];
+      if (b < 0 || b >= num_blocks || seen[(size_t)b]) {
+        delete bm;
+        return PA_ERR_INVALID;   // not a permutation of the pool
+      }
+      seen[(size_t)b] = 1;
+      bm->free.push_back(b);
+    }
+  } else {
+    for (int i = 0; i < num_blocks; ++i) bm->free.push_back(i);
+  }
+  *out = bm;
+  return PA_OK;
+}
+
+void pa_bm_destroy(pa_block_manager* bm) { delete bm; }
+
+int pa_bm_free_blocks(const pa_block_manager* bm) { return bm ? (int)bm->free.size() : -1; }
+
+int pa_bm_refcount(const pa_block_manager* bm, int block) {
+  if (!bm || block < 0 || block >= bm->num_blocks) return -1;
+  return bm->ref[(size_t)block];
+}
+
+pa_status pa_bm_allocate(pa_block_manager* bm, int num_tokens, int32_t* seq_id) {
+  if (!bm || !seq_id || num_tokens < 0) return PA_ERR_INVALID;
+  const int64_t need = bm->blocks_for(num_tokens);
+  if (need > (int64_t)bm->free.size()) return PA_ERR_NO_BLOCKS;
+  pa_block_manager::Seq s;
+  s.table.reserve((size_t)need);
+  for (int64_t i = 0; i < need; ++i) s.table.push_back(bm->take());
+  s.len = num_tokens;
+  const int32_t id = bm->next_id++;
+  bm->seqs.emplace(id, std::move(s));
+  *seq_id = id;
+  return PA_OK;
+}
+
+pa_status pa_bm_fork(pa_block_manager* bm, int32_t seq, int32_t* child) {
+  if (!bm || !child) return PA_ERR_INVALID;
+  const pa_block_manager::Seq* p = bm->find(seq);
+  if (!p) return PA_ERR_INVALID;
+  pa_block_manager::Seq c = *p;                  // shares every block of the parent
+  for (int32_t b : c.table) ++bm->ref[(size_t)b];
+  const int32_t id = bm->next_id++;
+  bm->seqs.emplace(id, std::move(c));
+  *child = id;
+  return PA_OK;
+}
+
+pa_status pa_bm_append_tokens(pa_block_manager* bm, const int32_t* seqs, int n, int64_t* slots,
+                              int32_t* cow_pairs, int* num_cow) {
+  if (!bm || n < 0 || (n && (!seqs || !slots || !cow_pairs || !num_cow))) return PA_ERR_INVALID;
+  if (num_cow) *num_cow = 0;
+  if (n == 0) return PA_OK;
+  // Dry run on copies of the touched state: how many fresh blocks the whole batch needs
+  // (a new logical block, or a private copy of a shared partial block), so that a batch
+  // the pool cannot serve changes nothing.
+  struct Sim {
+    int64_t len, nblk;
+    std::vector<int64_t> priv;   // logical blocks made private earlier in this batch
+  };
+  std::unordered_map<int32_t, Sim> sim;
+  std::unordered_map<int32_t, int32_t> ref;
+  int64_t need = 0;
+  for (int i = 0; i < n; ++i) {
+    const pa_block_manager::Seq* s = bm->find(seqs[i]);
+    if (!s) return PA_ERR_INVALID;
+    Sim& m = sim.try_emplace(seqs[i], Sim{s->len, (int64_t)s->table.size(), {}}).first->second;
+    const int64_t lb = m.len / bm->block_size;
+    if (lb == m.nblk) {
+      ++need;
+      ++m.nblk;
+      m.priv.push_back(lb);
+    } else {
+      bool priv = false;
+      for (int64_t x : m.priv) priv |= x == lb;
+      if (!priv) {
+        const int32_t b = s->table[(size_t)lb];
+        auto ri = ref.find(b);
+        const int32_t r = ri == ref.end() ? bm->ref[(size_t)b] : ri->second;
+        if (r > 1) {
+          ++need;
+          ref[b] = r - 1;
+          m.priv.push_back(lb);
+        }
+      }
+    }
+    ++m.len;
+  }
+  if (need > (int64_t)bm->free.size()) return PA_ERR_NO_BLOCKS;
+  int nc = 0;
+  for (int i = 0; i < n; ++i) {
+    pa_block_manager::Seq& s = *bm->find(seqs[i]);
+    const int64_t pos = s.len;
+    const int64_t lb = pos / bm->block_size, off = pos % bm->block_size;
+    if (lb == (int64_t)s.table.size()) {
+      s.table.push_back(bm->take());
+    } else if (bm->ref[(size_t)s.table[(size_t)lb]] > 1) {
+      const int32_t src = s.table[(size_t)lb];
+      const int32_t dst = bm->take();
+      --bm->ref[(size_t)src];
+      s.table[(size_t)lb] = dst;
+      cow_pairs[2 * nc] = src;
+      cow_pairs[2 * nc + 1] = dst;
+      ++nc;
+    }
+    s.len = pos + 1;
+    slots[i] = (int64_t)s.table[(size_t)lb] * bm->block_size + off;
+  }
+  *num_cow = nc;
+  return PA_OK;
+}
+
+pa_status pa_bm_release(pa_block_manager* bm, int32_t seq) {
+  if (!bm) return PA_ERR_INVALID;
+  auto it = bm->seqs.find(seq);
+  if (it == bm->seqs.end()) return PA_ERR_INVALID;
+  for (int32_t b : it->second.table)
+    if (--bm->ref[(size_t)b] == 0) bm->free.push_back(b);
+  bm->seqs.erase(it);
+  return PA_OK;
+}
+
+int64_t pa_bm_context_len(const pa_block_manager* bm, int32_t seq) {
+  const pa_block_manager::Seq* s = bm ? bm->find(seq) : nullptr;
+  return s ? s->len : -1;
+}
+
+int pa_bm_num_blocks_of(const pa_block_manager* bm, int32_t seq) {
+  const pa_block_manager::Seq* s = bm ? bm->find(seq) : nullptr;
+  return s ? (int)s->table.size() : -1;
+}
+
+int pa_bm_max_blocks(const pa_block_manager* bm, const int32_t* seqs, int n) {
+  if (!bm || n < 0 || (n && !seqs)) return -1;
+  int mx = 0;
+  for (int i = 0; i < n; ++i) {
+    const pa_block_manager::Seq* s = bm->find(seqs[i]);
+    if (!s) return -1;
+    if ((int)s->table.size() > mx) mx = (int)s->table.size();
+  }
+  return mx;
+}
+
+pa_status pa_bm_block_tables(const pa_block_manager* bm, const int32_t* seqs, int n, int width,
+                             int32_t fill, int32_t* tables, int32_t* context_lens) {
+  if (!bm || n < 0 || width <= 0 || (n && (!seqs || !tables))) return PA_ERR_INVALID;
+  for (int i = 0; i < n; ++i) {
+    const pa_block_manager::Seq* s = bm->find(seqs[i]);
+    if (!s || (int64_t)s->table.size() > width || s->len > INT32_MAX) return PA_ERR_INVALID;
+  }
+  for (int i = 0; i < n; ++i) {
+    const pa_block_manager::Seq* s = bm->find(seqs[i]);
+    int32_t* row = tables + (int64_t)i * width;
+    const size_t k = s->table.size();
+    if (k) std::memcpy(row, s->table.data(), k * sizeof(int32_t));
+    for (int j = (int)k; j < width; ++j) row[j] = fill;
+    if (context_lens) context_lens[i] = (int32_t)s->len;
+  }
+  return PA_OK;
+}
+
+pa_status pa_bm_slot_of(const pa_block_manager* bm, int32_t seq, int64_t pos, int64_t* slot) {
+  const pa_block_manager::Seq* s = bm ? bm->find(seq) : nullptr;
+  if (!s || !slot || pos < 0 || pos >= s->len) return PA_ERR_INVALID;
+  *slot = (int64_t)s->table[(size_t)(pos / bm->block_size)] * bm->block_size + pos % bm->block_size;
+  return PA_OK;
+}
+
+}  // extern "C"

@@ -16,14 +16,19 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libpagedkv.so")
 
-PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_CUDA = 0, 1, 2, 3
+PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_NO_BLOCKS, PA_ERR_NO_MEMORY = \
+    0, 1, 2, 3, 4, 5
 PA_F16, PA_BF16 = 0, 1
 DEV_BAD_BLOCK_ID, DEV_BAD_SLOT, DEV_BAD_PAIR, DEV_BAD_CONTEXT_LEN, DEV_TIMEOUT = (
     0x1, 0x2, 0x4, 0x8, 0x10)
 
 # every symbol include/pagedkv.h declares
 EXPORTS = ("pa_version", "pa_status_string", "pa_decode_workspace_bytes", "pa_decode",
-           "pa_decode_multi", "pa_cache_append", "pa_copy_blocks", "pa_decode_noalloc")
+           "pa_decode_multi", "pa_cache_append", "pa_copy_blocks", "pa_decode_noalloc",
+           "pa_bm_create", "pa_bm_destroy", "pa_bm_free_blocks", "pa_bm_refcount",
+           "pa_bm_allocate", "pa_bm_fork", "pa_bm_append_tokens", "pa_bm_release",
+           "pa_bm_context_len", "pa_bm_num_blocks_of", "pa_bm_max_blocks", "pa_bm_block_tables",
+           "pa_bm_slot_of")
 
 _lib = None
 _lock = threading.Lock()

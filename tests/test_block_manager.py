@@ -1,13 +1,20 @@
-"""Host block manager (product) against the oracle's reference planner, plus the
-workload generators' shapes.  CPU only."""
+"""Host block manager (product: the native pa_bm_* calls of libpagedkv, through its
+Python wrapper) against the oracle's reference planner, plus the workload generators'
+shapes.  CPU only: the manager never touches a GPU."""
 from __future__ import annotations
 
 import numpy as np
 import pytest
 
 from oracle.cow import RefBlockManager
+from paged_kv_cache_348_b200 import build as pbuild
 from paged_kv_cache_348_b200 import inputs
 from paged_kv_cache_348_b200.block_manager import BlockManager, PoolExhausted
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _library():
+    pbuild.build()
 
 
 def _scenario(mgr_cls, order):
@@ -96,3 +103,95 @@ def test_workload_generators():
     assert np.array_equal(inputs.context_lens(inputs.LLAMA8B), c1)        # seeded
     p = inputs.pool_order(64, 0)
     assert sorted(p) == list(range(64)) and not np.array_equal(p, np.arange(64))
+
+
+def test_random_operations_match_reference_planner():
+    """Differential run: the same random stream of prefills, forks, single and batched
+    appends and releases on the native manager and on the reference planner."""
+    rng = np.random.default_rng(123)
+    for trial in range(20):
+        N, bs = int(rng.integers(20, 120)), int(rng.choice([1, 4, 8, 16]))
+        order = rng.permutation(N).astype(np.int32)
+        m, r = BlockManager(N, bs, order), RefBlockManager(N, bs, order)
+        live = []
+        for _ in range(150):
+            op = rng.integers(0, 10)
+            if op < 2 or not live:
+                n = int(rng.integers(0, 3 * bs + 2))
+                try:
+                    sid = m.allocate(n)
+                except PoolExhausted:
+                    assert len(r.free) < -(-n // bs)     # the reference could not either
+                    continue
+                assert r.new_seq(n) == sid
+                live.append(sid)
+            elif op < 4:
+                p = int(rng.choice(live))
+                c = m.fork(p)
+                assert r.fork(p) == c
+                live.append(c)
+            elif op < 8:
+                batch = [int(x) for x in rng.choice(live, size=int(rng.integers(1, 5)))]
+                free0 = m.free_blocks
+                tables0 = {s: m.table(s) for s in live}
+                try:
+                    slots, pairs = m.append_tokens(batch)
+                except PoolExhausted:
+                    # nothing changed
+                    assert m.free_blocks == free0
+                    assert {s: m.table(s) for s in live} == tables0
+                    continue
+                ref_slots, ref_pairs = [], []
+                for sid in batch:
+                    sl, cow = r.append_slot(sid)
+                    ref_slots.append(sl)
+                    if cow:
+                        ref_pairs.append(cow)
+                assert list(slots) == ref_slots
+                assert [tuple(p) for p in pairs.tolist()] == ref_pairs
+            else:
+                sid = int(rng.choice(live))
+                m.release(sid)
+                r.release(sid)
+                live.remove(sid)
+            assert m.free_blocks == len(r.free)
+            for sid in live:
+                assert m.table(sid) == r.tables[sid]
+                assert m.context_len(sid) == r.ctx[sid]
+            for b in range(N):
+                assert m.refcount(b) == r.ref[b]
+
+
+def test_batch_append_that_does_not_fit_changes_nothing():
+    m = BlockManager(6, 4)
+    a = m.allocate(6)                      # 2 blocks, the second holds 2 of 4 tokens
+    kids = [m.fork(a) for _ in range(3)]   # all four share both blocks
+    assert m.free_blocks == 4
+    free0, t0 = m.free_blocks, {s: m.table(s) for s in [a] + kids}
+    # 3 copies of the shared partial block, then a and kids[0] each cross into a new
+    # block: 5 fresh blocks needed, 4 free
+    with pytest.raises(PoolExhausted):
+        m.append_tokens([a] + kids + [a, a, kids[0], kids[0]])
+    assert m.free_blocks == free0 and {s: m.table(s) for s in [a] + kids} == t0
+    assert [m.refcount(b) for b in t0[a]] == [4, 4]
+    slots, pairs = m.append_tokens([a] + kids)   # the last writer keeps the original
+    shared = t0[a][1]
+    assert [p[0] for p in pairs.tolist()] == [shared] * 3 and m.free_blocks == 1
+    assert m.table(kids[-1])[1] == shared and m.refcount(shared) == 1
+    assert slots[-1] == shared * 4 + 2
+
+
+def test_native_manager_rejects_bad_arguments():
+    with pytest.raises(ValueError):
+        BlockManager(4, 4, [0, 1, 1, 3])
+    m = BlockManager(8, 4)
+    with pytest.raises(ValueError):
+        m.fork(7)
+    with pytest.raises(ValueError):
+        m.release(3)
+    s = m.allocate(5)
+    with pytest.raises(ValueError):
+        m.slot_of(s, 5)
+    with pytest.raises(ValueError):
+        m.block_tables([s], width=1)
+    assert m.block_tables([s], width=3, fill=-1).tolist() == [[0, 1, -1]]
