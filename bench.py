@@ -227,6 +227,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama70b")
     ap.add_argument("--block-size", type=int, default=0)
+    ap.add_argument("--cascade", action="store_true",
+                    help="decode with pa_decode_cascade (shared prefixes read once per chunk)")
     ap.add_argument("--q-len", type=int, default=1,
                     help="new tokens per sequence (pa_decode_multi when > 1)")
     ap.add_argument("--layers", type=int, default=0,
@@ -263,6 +265,8 @@ def main():
     else:
         b = wl.build(w, device="cuda", block_size=bs, layers=args.layers or None,
                      q_len=args.q_len)
+    if args.cascade:
+        wl.use_cascade(b)
     stream = torch.cuda.current_stream()
     L = b.layers
     kv_step = b.kv_bytes_per_step()
@@ -342,8 +346,10 @@ def main():
         "peak_hbm_gbs": peak, "peak_kind": peak_kind,
         "seq_steps_per_s": world * w.num_seqs / (ms_step * 1e-3),
         "kv_bytes_per_step": kv_step,
-        "roofline": {"bound": "hbm", "kernel": "pa_decode_split_kernel (one launch per %s)" % (
-                         "pa_decode" if b.q_len == 1 else "pa_decode_multi"),
+        "roofline": {"bound": "hbm", "kernel": "pa_decode_split_kernel (%s)" % (
+                         "two launches per pa_decode_cascade" if b.cascade is not None else
+                         "one launch per pa_decode" if b.q_len == 1 else
+                         "one launch per pa_decode_multi"),
                      "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "algorithmic_bytes_per_launch": kv_layer,
@@ -353,6 +359,13 @@ def main():
         "clocks": clocks.summary() if rank == 0 else None,
         "e2e": e2e,
     }
+    if w.name == "prefix":
+        # shared blocks counted once: the bytes a read-once-per-block schedule needs
+        uniq = b.unique_kv_bytes_per_step()
+        line["kv_bytes_unique_per_step"] = uniq
+        line["roofline_unique_bytes"] = {
+            "achieved": uniq / L / (dec_avg * 1e-3) / 1e9, "peak": peak, "unit": "GB/s",
+            "frac": uniq / L / (dec_avg * 1e-3) / 1e9 / peak}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         nbytes, sec, seqs, threads = oracle_sample(w, bs, device_batch=b)
         line["cpu_baseline"] = {
@@ -420,9 +433,13 @@ def run_e2e(b, args, world, kv_step):
             comp.wait_event(ev_out[l])
             pk.pa_cache_append(b.k_caches[l], b.v_caches[l], b.k_new[l], b.v_new[l], slots[m],
                                b.status, comp)
-            fn = pk.pa_decode if b.q_len == 1 else pk.pa_decode_multi
-            fn(b.out[l], b.q[l], b.k_caches[l], b.v_caches[l], tabs[m], ctxs[m], b.scale,
-               b.workspace, b.status, comp)
+            if b.cascade is not None:
+                pk.pa_decode_cascade(b.out[l], b.q[l], b.k_caches[l], b.v_caches[l], tabs[m],
+                                     ctxs[m], *b.cascade, b.scale, b.workspace, b.status, comp)
+            else:
+                fn = pk.pa_decode if b.q_len == 1 else pk.pa_decode_multi
+                fn(b.out[l], b.q[l], b.k_caches[l], b.v_caches[l], tabs[m], ctxs[m], b.scale,
+                   b.workspace, b.status, comp)
             ev_used[l].record(comp)
         ev_meta_free[m].record(comp)
         with torch.cuda.stream(down):

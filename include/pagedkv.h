@@ -132,6 +132,52 @@ pa_status pa_decode_multi(void* out, const void* q, const void* k_cache, const v
                           int32_t* dev_status, void* stream);
 
 /*
+ * pa_decode_cascade -- pa_decode for a batch in which groups of sequences share a prefix
+ * of their KV blocks (parallel sampling, beams, a common system prompt), reading each
+ * shared block once per chunk of sharers instead of once per sequence.
+ *
+ * Defined by [P1] "How PagedAttention borrows OS paging" (requests with an identical
+ * prefix point their block tables at the same physical blocks) and [P3] "Why This
+ * Matters for Production" (parallel sampling and beam search share KV blocks).  The
+ * result is that of pa_decode on the same inputs (one new token per sequence): the
+ * softmax over a sequence's tokens is split at prefix_lens[s] into the shared part and
+ * the sequence's own part, each reduced to (max, sum, unnormalised acc), and the two
+ * are combined exactly (log-sum-exp); only the rounding order differs from pa_decode.
+ *
+ * Two launches on `stream`: pass 1 decodes every chunk's prefix (tokens
+ * 0..chunk_prefix_lens[c]-1, read through the block table of the chunk's first member)
+ * with the query rows of all its members at once; pass 2 decodes every sequence's
+ * tokens prefix_lens[s]..context_lens[s]-1 and merges the prefix result.
+ *
+ *   q, out, caches, block_tables, context_lens   as for pa_decode
+ *   prefix_lens        device int32 [num_seqs]: shared-prefix length of each sequence,
+ *                      0 for a sequence in no chunk
+ *   chunk_members      device int32 [num_chunks][chunk_width]: member sequence ids,
+ *                      padded with -1; the first slot must be a member.  1 <= chunk_width
+ *                      and (num_q_heads/num_kv_heads) * chunk_width <= 16: a chunk's query
+ *                      rows share the MMA N dimension (8 rows or fewer run the lighter
+ *                      kernel; up to 16 read the prefix half as often)
+ *   chunk_prefix_lens  device int32 [num_chunks]
+ *   workspace          >= pa_decode_cascade_workspace_bytes(...) bytes, 256-byte aligned
+ * Contract (not checked on the device): every sequence with prefix_lens[s] > 0 is a
+ * member of exactly one chunk, whose prefix length equals prefix_lens[s], and the block
+ * tables of a chunk's members agree on their first ceil(prefix/block_size) entries.
+ * Member ids outside [0, num_seqs) count as padding; a chunk whose first member is
+ * padding is empty.  Other arguments, limits and errors as for pa_decode.
+ */
+size_t pa_decode_cascade_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads,
+                                         int head_dim);
+pa_status pa_decode_cascade(void* out, const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* block_tables, const int32_t* context_lens,
+                            const int32_t* prefix_lens, int num_seqs,
+                            const int32_t* chunk_members, int chunk_width,
+                            const int32_t* chunk_prefix_lens, int num_chunks, int num_q_heads,
+                            int num_kv_heads, int head_dim, int block_size,
+                            int max_blocks_per_seq, int num_blocks, float scale, pa_dtype dtype,
+                            void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                            void* stream);
+
+/*
  * pa_cache_append -- write the new tokens' K and V into their cache slots.
  *
  * Defined by [P1] "How PagedAttention borrows OS paging" (blocks are filled on demand

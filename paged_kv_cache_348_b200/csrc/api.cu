@@ -112,11 +112,11 @@ cudaError_t launch(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
-template <typename T, int D, int BS, int NT>
+template <typename T, int D, int BS, int NT, int MODE>
 pa_status launch_decode(const pkv::DecodeArgs& a, const CUtensorMap& mk, const CUtensorMap& mv,
                         int grid, cudaStream_t stream) {
   using L = pkv::Layout<D>;
-  auto split = pkv::pa_decode_split_kernel<T, D, BS, NT>;
+  auto split = pkv::pa_decode_split_kernel<T, D, BS, NT, MODE>;
   if (cudaFuncSetAttribute(split, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynSmem) !=
       cudaSuccess)
     return PA_ERR_CUDA;
@@ -126,31 +126,52 @@ pa_status launch_decode(const pkv::DecodeArgs& a, const CUtensorMap& mk, const C
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
-template <typename T, int D, int BS>
+template <typename T, int D, int BS, int MODE>
 pa_status dispatch_nt(const pkv::DecodeArgs& a, const CUtensorMap& mk, const CUtensorMap& mv,
                       int grid, cudaStream_t s) {
-  return a.ncol <= 8 ? launch_decode<T, D, BS, 1>(a, mk, mv, grid, s)
-                     : launch_decode<T, D, BS, 2>(a, mk, mv, grid, s);
+  return a.ncol <= 8 ? launch_decode<T, D, BS, 1, MODE>(a, mk, mv, grid, s)
+                     : launch_decode<T, D, BS, 2, MODE>(a, mk, mv, grid, s);
 }
 
-template <typename T, int D>
+template <typename T, int D, int MODE>
 pa_status dispatch_bs(int bs, const pkv::DecodeArgs& a, const CUtensorMap& mk,
                       const CUtensorMap& mv, int grid, cudaStream_t s) {
   switch (bs) {
-    case 1: return dispatch_nt<T, D, 1>(a, mk, mv, grid, s);
-    case 8: return dispatch_nt<T, D, 8>(a, mk, mv, grid, s);
-    case 16: return dispatch_nt<T, D, 16>(a, mk, mv, grid, s);
-    case 32: return dispatch_nt<T, D, 32>(a, mk, mv, grid, s);
+    case 1: return dispatch_nt<T, D, 1, MODE>(a, mk, mv, grid, s);
+    case 8: return dispatch_nt<T, D, 8, MODE>(a, mk, mv, grid, s);
+    case 16: return dispatch_nt<T, D, 16, MODE>(a, mk, mv, grid, s);
+    case 32: return dispatch_nt<T, D, 32, MODE>(a, mk, mv, grid, s);
   }
   return PA_ERR_UNSUPPORTED;
 }
 
-template <typename T>
+template <typename T, int MODE>
 pa_status dispatch_d(int d, int bs, const pkv::DecodeArgs& a, const CUtensorMap& mk,
                      const CUtensorMap& mv, int grid, cudaStream_t s) {
-  return d == 64 ? dispatch_bs<T, 64>(bs, a, mk, mv, grid, s)
-                 : dispatch_bs<T, 128>(bs, a, mk, mv, grid, s);
+  return d == 64 ? dispatch_bs<T, 64, MODE>(bs, a, mk, mv, grid, s)
+                 : dispatch_bs<T, 128, MODE>(bs, a, mk, mv, grid, s);
 }
+
+template <typename T>
+pa_status dispatch_mode(int mode, int d, int bs, const pkv::DecodeArgs& a, const CUtensorMap& mk,
+                        const CUtensorMap& mv, int grid, cudaStream_t s) {
+  switch (mode) {
+    case pkv::kPlain: return dispatch_d<T, pkv::kPlain>(d, bs, a, mk, mv, grid, s);
+    case pkv::kPrefix: return dispatch_d<T, pkv::kPrefix>(d, bs, a, mk, mv, grid, s);
+    case pkv::kSuffix: return dispatch_d<T, pkv::kSuffix>(d, bs, a, mk, mv, grid, s);
+  }
+  return PA_ERR_INVALID;
+}
+
+// Cascade extras of one launch (kPlain: all null).
+struct CascadeArgs {
+  int mode = pkv::kPlain;
+  const int32_t* seq_start = nullptr;
+  const int32_t* chunk_members = nullptr;
+  int q_rows = 0;
+  float2* ext_ml = nullptr;
+  float* ext_acc = nullptr;
+};
 
 // Validation, workspace layout, tensor maps and launch shared by the decode entry points.
 // grid_cap > 0 caps the number of split CTAs (the fixed scratch of pa_decode_noalloc).
@@ -159,7 +180,7 @@ pa_status decode_impl(void* out, const void* q, const void* k_cache, const void*
                       int q_len, int num_q_heads, int num_kv_heads, int head_dim,
                       int block_size, int max_blocks_per_seq, int num_blocks, float scale,
                       pa_dtype dtype, void* workspace, size_t workspace_bytes, int grid_cap,
-                      int32_t* dev_status, void* stream) {
+                      int32_t* dev_status, void* stream, const CascadeArgs& cx = CascadeArgs()) {
   if (num_seqs < 0 || q_len < 1 || num_q_heads <= 0 || num_kv_heads <= 0 ||
       max_blocks_per_seq <= 0 || num_blocks <= 0 || !std::isfinite(scale))
     return PA_ERR_INVALID;
@@ -220,9 +241,29 @@ pa_status decode_impl(void* out, const void* q, const void* k_cache, const void*
   a.ncol = group * q_len;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.epoch = next_epoch();
+  a.seq_start = cx.seq_start;
+  a.chunk_members = cx.chunk_members;
+  a.q_rows = cx.q_rows;
+  a.ext_ml = cx.ext_ml;
+  a.ext_acc = cx.ext_acc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (dtype == PA_BF16) return dispatch_d<__nv_bfloat16>(head_dim, block_size, a, mk, mv, grid, st);
-  return dispatch_d<__half>(head_dim, block_size, a, mk, mv, grid, st);
+  if (dtype == PA_BF16)
+    return dispatch_mode<__nv_bfloat16>(cx.mode, head_dim, block_size, a, mk, mv, grid, st);
+  return dispatch_mode<__half>(cx.mode, head_dim, block_size, a, mk, mv, grid, st);
+}
+
+// Cascade workspace: the split scratch, then the external partials (max, sum)[B][Hq]
+// and acc[B][Hq][D].
+struct CascadeLayout {
+  size_t split, ml_off, acc_off, total;
+};
+CascadeLayout cascade_layout(int num_seqs, int num_q_heads, int head_dim, int grid) {
+  CascadeLayout c{};
+  c.split = ws_layout(num_seqs, head_dim, grid).total;
+  c.ml_off = align256(c.split);
+  c.acc_off = align256(c.ml_off + sizeof(float2) * (size_t)num_seqs * num_q_heads);
+  c.total = align256(c.acc_off + sizeof(float) * (size_t)num_seqs * num_q_heads * head_dim);
+  return c;
 }
 
 }  // namespace
@@ -272,6 +313,61 @@ pa_status pa_decode_multi(void* out, const void* q, const void* k_cache, const v
                      num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
                      num_blocks, scale, dtype, workspace, workspace_bytes, 0, dev_status,
                      stream);
+}
+
+size_t pa_decode_cascade_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads,
+                                         int head_dim) {
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0) return 0;
+  const int sms = sm_count();
+  if (sms <= 0) return 0;
+  return cascade_layout(num_seqs, num_q_heads, head_dim, sms * pkv::kCtasPerSm).total;
+}
+
+pa_status pa_decode_cascade(void* out, const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* block_tables, const int32_t* context_lens,
+                            const int32_t* prefix_lens, int num_seqs,
+                            const int32_t* chunk_members, int chunk_width,
+                            const int32_t* chunk_prefix_lens, int num_chunks, int num_q_heads,
+                            int num_kv_heads, int head_dim, int block_size,
+                            int max_blocks_per_seq, int num_blocks, float scale, pa_dtype dtype,
+                            void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                            void* stream) {
+  if (num_seqs < 0 || num_chunks < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+      num_q_heads % num_kv_heads || (num_chunks && chunk_width < 1))
+    return PA_ERR_INVALID;
+  if (num_seqs == 0) return PA_OK;
+  if (!prefix_lens || (num_chunks && (!chunk_members || !chunk_prefix_lens)) || !workspace ||
+      !aligned16(workspace))
+    return PA_ERR_INVALID;
+  const int sms = sm_count();
+  if (sms <= 0) return PA_ERR_CUDA;
+  const CascadeLayout cl = cascade_layout(num_seqs, num_q_heads, head_dim, sms * pkv::kCtasPerSm);
+  if (workspace_bytes < cl.total) return PA_ERR_INVALID;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  CascadeArgs cx;
+  cx.ext_ml = reinterpret_cast<float2*>(ws + cl.ml_off);
+  cx.ext_acc = reinterpret_cast<float*>(ws + cl.acc_off);
+  const int group = num_q_heads / num_kv_heads;
+  if (group > pkv::kMaxGroup || (num_chunks && (long long)group * chunk_width > pkv::kMaxGroup))
+    return PA_ERR_UNSUPPORTED;
+  if (num_chunks > 0) {
+    // pass 1: each chunk's shared prefix once, its members' query rows as MMA columns
+    cx.mode = pkv::kPrefix;
+    cx.chunk_members = chunk_members;
+    cx.q_rows = num_seqs;
+    const pa_status r = decode_impl(out, q, k_cache, v_cache, block_tables, chunk_prefix_lens,
+                                    num_chunks, chunk_width, num_q_heads, num_kv_heads,
+                                    head_dim, block_size, max_blocks_per_seq, num_blocks, scale,
+                                    dtype, workspace, cl.split, 0, dev_status, stream, cx);
+    if (r != PA_OK) return r;
+  }
+  // pass 2: every sequence's own tokens, merged with its prefix partial
+  cx.mode = pkv::kSuffix;
+  cx.chunk_members = nullptr;
+  cx.seq_start = prefix_lens;
+  return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, 1,
+                     num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                     num_blocks, scale, dtype, workspace, cl.split, 0, dev_status, stream, cx);
 }
 
 pa_status pa_cache_append(void* k_cache, void* v_cache, const void* k, const void* v,

@@ -63,8 +63,22 @@ constexpr int DEV_TIMEOUT = 0x10;
 
 enum : int { F_FIRST = 1, F_LAST = 2, F_END = 4, F_COMPLETE = 8 };
 
+// What a launch decodes (a template parameter, so the plain path carries none of the rest):
+//  kPlain   -- every sequence over its cached tokens 0..ctx-1; q_len new tokens, causal.
+//  kPrefix  -- cascade pass 1: "sequences" are chunks of sibling sequences sharing a prefix
+//              of ctx tokens (read through the first member's block table); the query
+//              columns are the members' rows, no causal mask, and the result is each
+//              member's unnormalised (max, sum, acc) written to the external partials.
+//  kSuffix  -- cascade pass 2: sequence s over its tokens seq_start[s]..ctx-1, merged with
+//              the external partial of its prefix when seq_start[s] > 0.
+enum : int { kPlain = 0, kPrefix = 1, kSuffix = 2 };
+
 struct StageMeta {
   int seq, kvh, tok0, nunits, ctx, flags, pidx, qslot;
+};
+
+struct SeqSpan {
+  int ctx, first;                       // tokens first..ctx-1 are decoded
 };
 
 // A segment portion this CTA shares with other CTAs, handed to the merger warp.
@@ -89,7 +103,14 @@ struct DecodeArgs {
   int ncol;                     // query rows per kv head: group * q_len (MMA columns)
   float scale_log2;             // scale * log2(e)
   uint32_t epoch;               // distinct per call: counters of older calls read as zero
+  // cascade (kPrefix / kSuffix launches only)
+  const int32_t* seq_start;     // kSuffix: first token of each sequence's own part
+  const int32_t* chunk_members; // kPrefix: [num_seqs][q_len] member sequences, -1 pad
+  int q_rows;                   // kPrefix: sequences in q / block_tables (valid member ids)
+  float2* ext_ml;               // [members][Hq] (max, sum) of the prefix part, base 2
+  float* ext_acc;               // [members][Hq][D] its unnormalised accumulator
 };
+
 
 template <int D>
 struct Layout {
@@ -134,6 +155,40 @@ __device__ __forceinline__ int clamp_ctx(int c, int cap, int32_t* status) {
   return c;
 }
 
+// Member slot j of chunk s in a prefix launch, or -1 (padding or out of range).
+__device__ __forceinline__ int chunk_member(const DecodeArgs& a, int s, int j) {
+  const int mem = a.chunk_members[(long long)s * a.q_len + j];
+  return (mem >= 0 && mem < a.q_rows) ? mem : -1;
+}
+
+template <int MODE>
+__device__ __forceinline__ SeqSpan span_of(const DecodeArgs& a, int s, int32_t* status) {
+  SeqSpan r;
+  r.ctx = clamp_ctx(a.context_lens[s], a.ctx_cap, status);
+  r.first = 0;
+  if constexpr (MODE == kPrefix) {
+    if (chunk_member(a, s, 0) < 0) r.ctx = 0;     // a chunk needs a valid first member
+  }
+  if constexpr (MODE == kSuffix) {
+    const int f = a.seq_start[s];
+    r.first = f < 0 ? 0 : (f > r.ctx ? r.ctx : f);
+  }
+  return r;
+}
+
+// Output row (sequence, head) of query column h of sequence/chunk `seq`, kv head kvh:
+// -1 when the column is a padding member slot of a chunk.
+template <int MODE>
+__device__ __forceinline__ long long out_row(const DecodeArgs& a, int seq, int kvh, int h) {
+  const int j = h / a.group, g = h % a.group;
+  if constexpr (MODE == kPrefix) {
+    const int mem = chunk_member(a, seq, j);
+    return mem < 0 ? -1ll : (long long)mem * a.num_q_heads + (long long)kvh * a.group + g;
+  } else {
+    return ((long long)seq * a.q_len + j) * a.num_q_heads + (long long)kvh * a.group + g;
+  }
+}
+
 // Index of the CTA whose unit range [start(c), start(c+1)) holds unit x, where
 // start(c) = floor(c * total / G).
 __device__ __forceinline__ int cta_of(long long x, long long total, int G) {
@@ -175,6 +230,75 @@ __device__ __forceinline__ void cp_async_16_zfill(void* dst, const void* src, ui
                : "memory");
 }
 
+// Finish one output value from this launch's (M, L, acc) of a column: kPlain writes
+// acc / L; kPrefix stores the unnormalised triple; kSuffix first folds in the prefix
+// partial (xm, xa), which the caller loaded beforehand (xm.x = -inf: none).  `d0` is the
+// first of `n` consecutive dims held in acc[] (n = 1 or 4).
+template <typename T, int MODE, int D>
+__device__ __forceinline__ void finish_row(const DecodeArgs& a, long long row, float M, float L,
+                                           float* acc, int d0, int n, float2 xm,
+                                           const float* xa) {
+  if constexpr (MODE == kPrefix) {
+    if (d0 == 0) a.ext_ml[row] = make_float2(M, L);
+    for (int i = 0; i < n; ++i) a.ext_acc[row * D + d0 + i] = acc[i];
+    return;
+  } else {
+    if constexpr (MODE == kSuffix) {
+      if (xm.x != -INFINITY) {
+        const float mn = fmaxf(M, xm.x);
+        const float sa = M == -INFINITY ? 0.f : ex2(M - mn);
+        const float sb = ex2(xm.x - mn);
+        L = L * sa + xm.y * sb;
+        for (int i = 0; i < n; ++i) acc[i] = acc[i] * sa + xa[i] * sb;
+        M = mn;
+      }
+    }
+    T* o = static_cast<T*>(a.out) + row * D + d0;
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    if (n == 4) {
+      *reinterpret_cast<uint2*>(o) = make_uint2(pack2<T>(acc[0] * inv, acc[1] * inv),
+                                                pack2<T>(acc[2] * inv, acc[3] * inv));
+    } else {
+      for (int i = 0; i < n; ++i) o[i] = from_float<T>(acc[i] * inv);
+    }
+  }
+}
+
+// Rows of a sequence (or chunk) that owns no unit, written by one warp: kPlain zeroes its
+// output rows; kPrefix marks its members' prefix partials empty; kSuffix normalises the
+// prefix partial (zero if there is none).
+template <typename T, int MODE, int D>
+__device__ __forceinline__ void empty_rows(const DecodeArgs& a, int s, int first, int lane) {
+  const int Hq = a.num_q_heads;
+  if constexpr (MODE == kPrefix) {
+    for (int j = 0; j < a.q_len; ++j) {
+      const int mem = chunk_member(a, s, j);
+      if (mem < 0) continue;
+      for (int h = lane; h < Hq; h += 32)
+        a.ext_ml[(long long)mem * Hq + h] = make_float2(-INFINITY, 0.f);
+    }
+  } else if constexpr (MODE == kSuffix) {
+    for (int i = lane; i < Hq * (D / 4); i += 32) {
+      const long long row = (long long)s * Hq + i / (D / 4);
+      const int d = (i % (D / 4)) * 4;
+      float v[4] = {0.f, 0.f, 0.f, 0.f};
+      if (first > 0) {
+        const float2 x = __ldcg(a.ext_ml + row);
+        const float4 y = __ldcg(reinterpret_cast<const float4*>(a.ext_acc + row * D + d));
+        if (x.x != -INFINITY && x.y > 0.f) {
+          const float inv = 1.f / x.y;
+          v[0] = y.x * inv, v[1] = y.y * inv, v[2] = y.z * inv, v[3] = y.w * inv;
+        }
+      }
+      *reinterpret_cast<uint2*>(static_cast<T*>(a.out) + row * D + d) =
+          make_uint2(pack2<T>(v[0], v[1]), pack2<T>(v[2], v[3]));
+    }
+  } else {
+    uint4* row = reinterpret_cast<uint4*>(static_cast<T*>(a.out) + (long long)s * a.q_len * Hq * D);
+    for (int i = lane; i < a.q_len * Hq * D * 2 / 16; i += 32) row[i] = make_uint4(0, 0, 0, 0);
+  }
+}
+
 // Entry i (0 <= i < 96) of a block-table window held across the warp: lane l holds
 // entries l, 32+l and 64+l in x0, x1, x2.  Every lane must call it.
 __device__ __forceinline__ int win_lookup(int x0, int x1, int x2, int i) {
@@ -201,7 +325,7 @@ __device__ __forceinline__ int partial_slot(int cc, long long seg0, long long to
 // CTA order with a running maximum (so the result does not depend on which CTA arrived
 // last), kMC contributors at a time with every load of a group issued before any use:
 // one L2 round trip per group.
-template <typename T, int D, int NT>
+template <typename T, int D, int NT, int MODE>
 __device__ __forceinline__ void merge_split(const DecodeArgs& a, const SplitDesc& dsc,
                                             long long total, int G, int group, int tid) {
   constexpr int kThr = 32 * kConsumerWarps;
@@ -254,22 +378,34 @@ __device__ __forceinline__ void merge_split(const DecodeArgs& a, const SplitDesc
         M[e] = mn;
       }
   }
+  const bool has_prefix = MODE == kSuffix && a.seq_start[dsc.seq] > 0;
+  float2 xm[kPer];
+  float4 xa[kPer];
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) {                // the prefix partials, all loads at once
+    const int i = tid + kThr * e;
+    xm[e] = make_float2(-INFINITY, 0.f);
+    xa[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (has_prefix && i < nel) {
+      const long long row = out_row<MODE>(a, dsc.seq, dsc.kvh, i / kF4);
+      xm[e] = __ldcg(a.ext_ml + row);
+      xa[e] = __ldcg(reinterpret_cast<const float4*>(a.ext_acc + row * D) + i % kF4);
+    }
+  }
 #pragma unroll
   for (int e = 0; e < kPer; ++e) {
     const int i = tid + kThr * e;
     if (i >= nel) continue;
     const int h = i / kF4, d4 = i % kF4;           // query column, 4-dim group
-    T* outp = static_cast<T*>(a.out) +
-              (((long long)dsc.seq * a.q_len + h / group) * a.num_q_heads +
-               (long long)dsc.kvh * group + h % group) * D;
-    const float inv = Lsum[e] > 0.f ? 1.f / Lsum[e] : 0.f;
-    const uint32_t lo = pack2<T>(acc[e].x * inv, acc[e].y * inv);
-    const uint32_t hi = pack2<T>(acc[e].z * inv, acc[e].w * inv);
-    *reinterpret_cast<uint2*>(outp + d4 * 4) = make_uint2(lo, hi);
+    const long long row = out_row<MODE>(a, dsc.seq, dsc.kvh, h);
+    if (row < 0) continue;
+    float v[4] = {acc[e].x, acc[e].y, acc[e].z, acc[e].w};
+    const float x4[4] = {xa[e].x, xa[e].y, xa[e].z, xa[e].w};
+    finish_row<T, MODE, D>(a, row, M[e], Lsum[e], v, d4 * 4, 4, xm[e], x4);
   }
 }
 
-template <typename T, int D, int BS, int NT>
+template <typename T, int D, int BS, int NT, int MODE>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     pa_decode_split_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
                            const __grid_constant__ CUtensorMap tmv) {
@@ -316,13 +452,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     // pass 1 over the batch: total units; CTA 0 also writes the zero rows of empty
     // sequences (they own no unit).  For B <= 32 the lane values are kept for pass 2.
     long long run = 0;
-    int keep_ctx = 0, keep_u = 0, keep_x = 0;
+    int keep_ctx = 0, keep_first = 0, keep_u = 0, keep_x = 0;
 #pragma unroll 4
     for (int base = 0; base < B; base += 32) {
       const int s = base + lane;
-      int ctx = 0;
-      if (s < B) ctx = clamp_ctx(a.context_lens[s], a.ctx_cap, c == 0 ? a.status : nullptr);
-      const int u = (ctx + kUnit - 1) / kUnit;
+      SeqSpan sp{0, 0};
+      if (s < B) sp = span_of<MODE>(a, s, c == 0 ? a.status : nullptr);
+      const int ctx = sp.ctx;
+      const int u = (ctx - sp.first + kUnit - 1) / kUnit;
       int x = u;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -330,6 +467,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         if (lane >= o) x += y;
       }
       keep_ctx = ctx;
+      keep_first = sp.first;
       keep_u = u;
       keep_x = x;
       run += __shfl_sync(0xffffffffu, x, 31);
@@ -338,10 +476,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         while (zero) {
           const int src = __ffs(zero) - 1;
           zero &= zero - 1;
-          uint4* row = reinterpret_cast<uint4*>(static_cast<T*>(a.out) +
-                                                (long long)(base + src) * a.q_len * a.num_q_heads * D);
-          for (int i = lane; i < a.q_len * a.num_q_heads * D * 2 / 16; i += 32)
-            row[i] = make_uint4(0, 0, 0, 0);
+          const int f = MODE == kSuffix ? __shfl_sync(0xffffffffu, sp.first, src) : 0;
+          empty_rows<T, MODE, D>(a, base + src, f, lane);
         }
       }
     }
@@ -350,18 +486,20 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     const long long end = total ? cta_start(c + 1, total, G) : 0;
 
     // pass 2: the sequence holding unit `start`
-    int s_a = 0, u_a = 0, ctx_a = 0;
+    int s_a = 0, u_a = 0, ctx_a = 0, first_a = 0;
     long long pb_a = 0;
     if (start < end) {
       long long r2 = 0;
       bool got_a = false;
       for (int base = 0; base < B && !got_a; base += 32) {
         const int s = base + lane;
-        int ctx = keep_ctx, u = keep_u, x = keep_x;
+        int ctx = keep_ctx, first = keep_first, u = keep_u, x = keep_x;
         if (B > 32) {
-          ctx = 0;
-          if (s < B) ctx = clamp_ctx(a.context_lens[s], a.ctx_cap, nullptr);
-          u = (ctx + kUnit - 1) / kUnit;
+          SeqSpan sp{0, 0};
+          if (s < B) sp = span_of<MODE>(a, s, nullptr);
+          ctx = sp.ctx;
+          first = sp.first;
+          u = (ctx - first + kUnit - 1) / kUnit;
           x = u;
 #pragma unroll
           for (int o = 1; o < 32; o <<= 1) {
@@ -376,6 +514,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           s_a = base + src;
           u_a = __shfl_sync(0xffffffffu, u, src);
           ctx_a = __shfl_sync(0xffffffffu, ctx, src);
+          if constexpr (MODE == kSuffix) first_a = __shfl_sync(0xffffffffu, first, src);
           pb_a = __shfl_sync(0xffffffffu, lo, src);
           got_a = true;
         }
@@ -393,14 +532,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     {
       long long x = start;
       const long long xend = end;
-      int s_cur = s_a, u_cur = u_a, ctx_cur = ctx_a;
+      int s_cur = s_a, u_cur = u_a, ctx_cur = ctx_a, first_cur = first_a;
       long long pbase = pb_a;
       while (ok && x < xend) {
         while (x >= pbase + (long long)Hkv * u_cur) {   // next sequence with units
           pbase += (long long)Hkv * u_cur;
           ++s_cur;
-          ctx_cur = clamp_ctx(a.context_lens[s_cur], a.ctx_cap, nullptr);
-          u_cur = (ctx_cur + kUnit - 1) / kUnit;
+          const SeqSpan sp = span_of<MODE>(a, s_cur, nullptr);
+          ctx_cur = sp.ctx;
+          if constexpr (MODE == kSuffix) first_cur = sp.first;
+          u_cur = (ctx_cur - first_cur + kUnit - 1) / kUnit;
         }
         const int kvh = (int)((x - pbase) / u_cur);
         const long long seg0 = pbase + (long long)kvh * u_cur, seg1 = seg0 + u_cur;
@@ -421,16 +562,18 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         // Block-table window: lane l holds entries wb+l, wb+32+l (w0, w1) and the next 64
         // entries (n0, n1), loaded 64 blocks before they are needed, so no stage waits on a
         // table read except the portion's first.
-        const int32_t* trow = a.block_tables + (long long)s_cur * a.max_blocks;
+        // a chunk of a prefix launch reads the prefix through its first member's table
+        const long long trow_seq = MODE == kPrefix ? (long long)chunk_member(a, s_cur, 0) : s_cur;
+        const int32_t* trow = a.block_tables + trow_seq * a.max_blocks;
         const int nblk = (ctx_cur + BS - 1) / BS;
-        int wb = (int)((x - seg0) * kUnit) / BS;
+        int wb = (first_cur + (int)(x - seg0) * kUnit) / BS;
         int w0 = wb + lane < nblk ? trow[wb + lane] : -1;
         int w1 = wb + 32 + lane < nblk ? trow[wb + 32 + lane] : -1;
         int n0 = wb + 64 + lane < nblk ? trow[wb + 64 + lane] : -1;
         int n1 = wb + 96 + lane < nblk ? trow[wb + 96 + lane] : -1;
         for (long long tu = x; tu < pe; tu += kUnitsPerStage) {
           const int nun = (int)((pe - tu) < kUnitsPerStage ? (pe - tu) : kUnitsPerStage);
-          const int tok0 = (int)(tu - seg0) * kUnit;
+          const int tok0 = first_cur + (int)(tu - seg0) * kUnit;
           if (tok0 / BS >= wb + 64) {                 // warp-uniform: slide the window
             w0 = n0;
             w1 = n1;
@@ -446,6 +589,18 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           const uint32_t qbytes = (flags & F_FIRST) ? qrow_bytes * (uint32_t)a.q_len : 0u;
           const T* qsrc = static_cast<const T*>(a.q) +
                           ((long long)s_cur * a.q_len * a.num_q_heads + (long long)kvh * group) * D;
+          // source of query-row token jq (in a prefix launch: the chunk's jq-th member; a
+          // padding slot repeats the first member's rows and its results are dropped)
+          auto qrow_src = [&](int jq) -> const T* {
+            if constexpr (MODE == kPrefix) {
+              int mem = chunk_member(a, s_cur, jq);
+              if (mem < 0) mem = (int)trow_seq;
+              return static_cast<const T*>(a.q) +
+                     ((long long)mem * a.num_q_heads + (long long)kvh * group) * D;
+            } else {
+              return qsrc + (long long)jq * a.num_q_heads * D;
+            }
+          };
           if constexpr (BS != 1) {
             constexpr int H = BS < 16 ? BS : 16;     // rows per TMA box
             constexpr int BPU = kUnit / H;           // boxes per unit and column half
@@ -493,9 +648,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
               meta[st] = StageMeta{s_cur, kvh, tok0, nun, ctx_cur, flags, pidx, qslot};
               mbar_arrive_expect_tx(&full[st], bytes);
               if (qbytes)
-                for (int j = 0; j < a.q_len; ++j)
-                  bulk_load(sQ + j * qrow_bytes, qsrc + (long long)j * a.num_q_heads * D,
-                            qrow_bytes, &full[st]);
+                for (int jq = 0; jq < a.q_len; ++jq)
+                  bulk_load(sQ + jq * qrow_bytes, qrow_src(jq), qrow_bytes, &full[st]);
             }
             __syncwarp();
             if (mine) {
@@ -520,9 +674,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
               meta[st] = StageMeta{s_cur, kvh, tok0, nun, ctx_cur, flags, pidx, qslot};
               mbar_arrive_expect_tx(&full[st], qbytes);
               if (qbytes)
-                for (int j = 0; j < a.q_len; ++j)
-                  bulk_load(sQ + j * qrow_bytes, qsrc + (long long)j * a.num_q_heads * D,
-                            qrow_bytes, &full[st]);
+                for (int jq = 0; jq < a.q_len; ++jq)
+                  bulk_load(sQ + jq * qrow_bytes, qrow_src(jq), qrow_bytes, &full[st]);
             }
             const int ch = lane % CPR, hf = ch >> 3, cc = ch & 7;
             for (int r0 = 0; r0 < ntok; r0 += RPI) {
@@ -637,8 +790,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     if (cw < mt.nunits) {
       const int t0 = mt.tok0 + cw * kUnit;
       const int valid = (mt.ctx - t0) < kUnit ? (mt.ctx - t0) : kUnit;
-      // causal limit: new token j sees unit rows < ctx - q_len + 1 + j - t0
-      const int lim0 = mt.ctx - a.q_len + 1 - t0;
+      // causal limit: new token j sees unit rows < ctx - q_len + 1 + j - t0 (a prefix
+      // launch's columns are different sequences: no mask)
+      const int lim0 = MODE == kPrefix ? (1 << 30) : mt.ctx - a.q_len + 1 - t0;
       const uint32_t kbase = smem_u32(sK), vbase = smem_u32(sV);
       // ---- S^T[16 tokens][8*NT heads] = K_unit . q^T
       float sacc[NT][4];
@@ -760,7 +914,32 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       }
       named_bar_sync(1, kConsumerThreads);
       const bool complete = mt.flags & F_COMPLETE;
-      for (int pi = tid; pi < NREG * 32; pi += kConsumerThreads) {
+      const bool has_prefix = MODE == kSuffix && complete && a.seq_start[mt.seq] > 0;
+      constexpr int kIt = NREG * 32 / kConsumerThreads;   // accumulator values per thread
+      static_assert(NREG * 32 % kConsumerThreads == 0, "");
+      float2 xm[kIt];
+      float xv[kIt];
+#pragma unroll
+      for (int it = 0; it < kIt; ++it) {            // the prefix partials, all loads at once
+        xm[it] = make_float2(-INFINITY, 0.f);
+        xv[it] = 0.f;
+        if (has_prefix) {
+          const int pi = tid + it * kConsumerThreads;
+          const int r = pi >> 5, ln = pi & 31;
+          const int e = r & 3, n = (r >> 2) % NT, mtile = (r >> 2) / NT;
+          const int d = mtile * 16 + (ln >> 2) + (e >= 2 ? 8 : 0);
+          const int h = n * 8 + 2 * (ln & 3) + (e & 1);
+          if (h < a.ncol) {
+            const long long row = out_row<MODE>(a, mt.seq, mt.kvh, h);
+            xm[it] = __ldcg(a.ext_ml + row);
+            xv[it] = __ldcg(a.ext_acc + row * D + d);
+          }
+        }
+      }
+      constexpr int kUnrollEpi = MODE == kSuffix ? kIt : 1;   // registers xm/xv need it
+#pragma unroll kUnrollEpi
+      for (int it = 0; it < kIt; ++it) {
+        const int pi = tid + it * kConsumerThreads;
         const int r = pi >> 5, ln = pi & 31;
         const int e = r & 3, n = (r >> 2) % NT, mtile = (r >> 2) / NT;
         const int d = mtile * 16 + (ln >> 2) + (e >= 2 ? 8 : 0);
@@ -778,12 +957,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           acc += scr[(w * NREG + r) * 32 + ln] * sc;
         }
         if (complete) {
-          // column h = new token h / group, head kvh * group + h % group; a row that
-          // sees no token at all (a new token before the context start) is zero
-          T* outp = static_cast<T*>(a.out) +
-                    (((long long)mt.seq * a.q_len + h / group) * a.num_q_heads +
-                     (long long)mt.kvh * group + h % group) * D;
-          outp[d] = from_float<T>(Lsum > 0.f ? acc / Lsum : 0.f);
+          // column h = new token (or chunk member) h / group, head kvh * group + h % group;
+          // a row that sees no token at all (a new token before the context start) is zero
+          const long long row = out_row<MODE>(a, mt.seq, mt.kvh, h);
+          if (row >= 0) {
+            if constexpr (MODE == kSuffix)
+              finish_row<T, MODE, D>(a, row, M, Lsum, &acc, d, 1, xm[it], &xv[it]);
+            else
+              finish_row<T, MODE, D>(a, row, M, Lsum, &acc, d, 1, make_float2(-INFINITY, 0.f),
+                                     nullptr);
+          }
         } else {
           a.part_acc[((long long)mt.pidx * kMaxGroup + h) * D + d] = acc;
           if (d == 0) {
@@ -811,7 +994,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           *last_flag = (int)(uint32_t)nxt == dsc.ncontrib;
         }
         named_bar_sync(1, kConsumerThreads);
-        if (*last_flag) merge_split<T, D, NT>(a, dsc, *total_s, G, group, tid);
+        if (*last_flag) merge_split<T, D, NT, MODE>(a, dsc, *total_s, G, group, tid);
       }
       fence_proxy_async_smem();   // generic writes above precede the next TMA fill
     }

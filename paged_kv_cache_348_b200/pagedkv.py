@@ -24,7 +24,8 @@ DEV_BAD_BLOCK_ID, DEV_BAD_SLOT, DEV_BAD_PAIR, DEV_BAD_CONTEXT_LEN, DEV_TIMEOUT =
 
 # every symbol include/pagedkv.h declares
 EXPORTS = ("pa_version", "pa_status_string", "pa_decode_workspace_bytes", "pa_decode",
-           "pa_decode_multi", "pa_cache_append", "pa_copy_blocks", "pa_decode_noalloc",
+           "pa_decode_multi", "pa_decode_cascade_workspace_bytes", "pa_decode_cascade",
+           "pa_cache_append", "pa_copy_blocks", "pa_decode_noalloc",
            "pa_bm_create", "pa_bm_destroy", "pa_bm_free_blocks", "pa_bm_refcount",
            "pa_bm_allocate", "pa_bm_fork", "pa_bm_append_tokens", "pa_bm_release",
            "pa_bm_context_len", "pa_bm_num_blocks_of", "pa_bm_max_blocks", "pa_bm_block_tables",
@@ -61,6 +62,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         L.pa_decode_multi.restype = i32
         L.pa_decode_multi.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, i32,
                                       f32, i32, P, sz, P, P]
+        L.pa_decode_cascade_workspace_bytes.restype = sz
+        L.pa_decode_cascade_workspace_bytes.argtypes = [i32, i32, i32, i32]
+        L.pa_decode_cascade.restype = i32
+        L.pa_decode_cascade.argtypes = [P, P, P, P, P, P, P, i32, P, i32, P, i32, i32, i32, i32,
+                                        i32, i32, i32, f32, i32, P, sz, P, P]
         L.pa_cache_append.restype = i32
         L.pa_cache_append.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, P, P]
         L.pa_copy_blocks.restype = i32
@@ -168,6 +174,46 @@ def pa_decode_multi(out, q, k_cache, v_cache, block_tables, context_lens, scale:
                                 _ptr(workspace), workspace.numel() * workspace.element_size(),
                                 _ptr(status), _stream(stream))
     _check(rc, "pa_decode_multi")
+    return out
+
+
+def new_cascade_workspace(num_seqs, num_q_heads, num_kv_heads, head_dim, device=None):
+    n = int(load().pa_decode_cascade_workspace_bytes(num_seqs, num_q_heads, num_kv_heads,
+                                                     head_dim))
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def pa_decode_cascade(out, q, k_cache, v_cache, block_tables, context_lens, prefix_lens,
+                      chunk_members, chunk_prefix_lens, scale: float, workspace, status=None,
+                      stream=None):
+    """out[B,Hq,D] <- paged decode where chunks of sequences share a KV prefix (see
+    pa_decode_cascade in include/pagedkv.h).  chunk_members is int32 [C, W] (-1 pad,
+    group * W <= 16), chunk_prefix_lens int32 [C], prefix_lens int32 [B]."""
+    _need(q, "q", ndim=3)
+    _need(out, "out", dtype=q.dtype, ndim=3)
+    _need(k_cache, "k_cache", dtype=q.dtype, ndim=4)
+    _need(v_cache, "v_cache", dtype=q.dtype, ndim=4)
+    _need(block_tables, "block_tables", dtype=torch.int32, ndim=2)
+    _need(context_lens, "context_lens", dtype=torch.int32, ndim=1)
+    _need(prefix_lens, "prefix_lens", dtype=torch.int32, ndim=1)
+    _need(chunk_members, "chunk_members", dtype=torch.int32, ndim=2)
+    _need(chunk_prefix_lens, "chunk_prefix_lens", dtype=torch.int32, ndim=1)
+    _need(workspace, "workspace")
+    B, Hq, D = q.shape
+    N, Hkv, bs, D2 = k_cache.shape
+    C = chunk_members.shape[0]
+    if out.shape != q.shape or D2 != D or v_cache.shape != k_cache.shape or \
+            block_tables.shape[0] != B or context_lens.shape[0] != B or \
+            prefix_lens.shape[0] != B or chunk_prefix_lens.shape[0] != C:
+        raise PagedKVError("pa_decode_cascade: inconsistent shapes")
+    rc = load().pa_decode_cascade(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                  _ptr(block_tables), _ptr(context_lens), _ptr(prefix_lens), B,
+                                  _ptr(chunk_members), chunk_members.shape[1],
+                                  _ptr(chunk_prefix_lens), C, Hq, Hkv, D, bs,
+                                  block_tables.shape[1], N, float(scale), _dtype_code(q),
+                                  _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                  _ptr(status), _stream(stream))
+    _check(rc, "pa_decode_cascade")
     return out
 
 

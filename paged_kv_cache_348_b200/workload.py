@@ -44,6 +44,7 @@ class DecodeBatch:
     cow_pairs: torch.Tensor | None
     scale: float
     q_len: int = 1
+    cascade: tuple | None = None     # (prefix_lens, chunk_members, chunk_prefix_lens) on device
 
     @property
     def layers(self) -> int:
@@ -173,8 +174,67 @@ def run_step(b: DecodeBatch, stream=None, layers=None) -> None:
         decode_layer(b, l, stream)
 
 
+def use_cascade(b: DecodeBatch, width: int | None = None) -> DecodeBatch:
+    """Decode this batch with pa_decode_cascade: plan the shared-prefix chunks from its
+    block tables (the workspace grows to the cascade size)."""
+    tables, ctx = b.block_tables.cpu().numpy(), b.context_lens.cpu().numpy()
+    w = b.w
+    prefix, members, plens = plan_cascade(tables, ctx, b.block_size,
+                                          w.num_q_heads // w.num_kv_heads, width)
+    dev = b.block_tables.device
+    b.cascade = (torch.from_numpy(prefix).to(dev), torch.from_numpy(members).to(dev),
+                 torch.from_numpy(plens).to(dev))
+    b.workspace = pk.new_cascade_workspace(len(ctx), w.num_q_heads, w.num_kv_heads, w.head_dim,
+                                           dev)
+    return b
+
+
 def decode_layer(b: DecodeBatch, l: int, stream=None) -> None:
-    """pa_decode (one new token per sequence) or pa_decode_multi (q_len > 1) of layer l."""
+    """pa_decode (one new token per sequence), pa_decode_multi (q_len > 1) or
+    pa_decode_cascade (after use_cascade) of layer l."""
+    if b.cascade is not None:
+        pk.pa_decode_cascade(b.out[l], b.q[l], b.k_caches[l], b.v_caches[l], b.block_tables,
+                             b.context_lens, *b.cascade, b.scale, b.workspace, b.status, stream)
+        return
     fn = pk.pa_decode if b.q_len == 1 else pk.pa_decode_multi
     fn(b.out[l], b.q[l], b.k_caches[l], b.v_caches[l], b.block_tables, b.context_lens, b.scale,
        b.workspace, b.status, stream)
+
+
+def plan_cascade(tables: np.ndarray, ctx: np.ndarray, block_size: int, group: int,
+                 width: int | None = None):
+    """Chunks of sequences that share a prefix of their block tables, for
+    pa_decode_cascade.  Sequences whose first block is the same physical block form a
+    sharing group; its prefix is the leading table entries common to all members,
+    capped at the shortest member's length.  Groups of one sequence get no chunk.
+    Returns (prefix_lens int32 [B], chunk_members int32 [C, width], chunk_prefix_lens
+    int32 [C]); a chunk holds at most `width` members (default: 8 query rows per chunk,
+    the lighter kernel; group * width <= 16)."""
+    B = len(ctx)
+    cap = width or max(1, 8 // group)
+    by_first = {}
+    for s in range(B):
+        if ctx[s] > 0:
+            by_first.setdefault(int(tables[s, 0]), []).append(s)
+    prefix = np.zeros(B, dtype=np.int32)
+    members, plens = [], []
+    for mem in by_first.values():
+        if len(mem) < 2:
+            continue
+        nb = min(-(-int(ctx[s]) // block_size) for s in mem)
+        common = 0
+        while common < nb and all(tables[s, common] == tables[mem[0], common] for s in mem):
+            common += 1
+        plen = min(common * block_size, min(int(ctx[s]) for s in mem))
+        if plen == 0:
+            continue
+        for i in range(0, len(mem), cap):
+            row = np.full(cap, -1, dtype=np.int32)
+            part = mem[i:i + cap]
+            row[:len(part)] = part
+            members.append(row)
+            plens.append(plen)
+            prefix[part] = plen
+    cm = np.stack(members) if members else np.zeros((0, cap), dtype=np.int32)
+    return prefix, cm, np.array(plens, dtype=np.int32)
+
