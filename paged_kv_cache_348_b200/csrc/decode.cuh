@@ -131,10 +131,8 @@ struct Layout {
   static_assert(2 * (kDynSmem + 1024) <= 233472, "two CTAs per SM must fit");
 };
 
-__device__ __forceinline__ unsigned long long ld_relaxed_gpu(const unsigned long long* p) {
-  unsigned long long v;
-  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
+__device__ __forceinline__ void st_relaxed_gpu(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 __device__ __forceinline__ unsigned long long cas_acq_rel_gpu(unsigned long long* p,
                                                               unsigned long long cmp,
@@ -915,63 +913,64 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       named_bar_sync(1, kConsumerThreads);
       const bool complete = mt.flags & F_COMPLETE;
       const bool has_prefix = MODE == kSuffix && complete && a.seq_start[mt.seq] > 0;
+      // Thread tid of warp cw holds, in scr, accumulator register e = cw of every (ks, n)
+      // tile of lane `lane`: query column h_n = n*8 + 2*(lane%4) + cw%2 and head dim
+      // d = ks*16 + lane/4 + 8*(cw/2).  So the column statistics (max, weights, sum)
+      // are computed once per n, and the loop over the dims only sums and stores.
       constexpr int kIt = NREG * 32 / kConsumerThreads;   // accumulator values per thread
-      static_assert(NREG * 32 % kConsumerThreads == 0, "");
-      float2 xm[kIt];
-      float xv[kIt];
+      static_assert(kIt == KS * NT, "one value per (ks, n) tile");
+      float cM[NT], cL[NT], cs[NT][kConsumerWarps];
+      long long crow[NT];
 #pragma unroll
-      for (int it = 0; it < kIt; ++it) {            // the prefix partials, all loads at once
-        xm[it] = make_float2(-INFINITY, 0.f);
-        xv[it] = 0.f;
-        if (has_prefix) {
-          const int pi = tid + it * kConsumerThreads;
-          const int r = pi >> 5, ln = pi & 31;
-          const int e = r & 3, n = (r >> 2) % NT, mtile = (r >> 2) / NT;
-          const int d = mtile * 16 + (ln >> 2) + (e >= 2 ? 8 : 0);
-          const int h = n * 8 + 2 * (ln & 3) + (e & 1);
-          if (h < a.ncol) {
-            const long long row = out_row<MODE>(a, mt.seq, mt.kvh, h);
-            xm[it] = __ldcg(a.ext_ml + row);
-            xv[it] = __ldcg(a.ext_acc + row * D + d);
-          }
-        }
-      }
-      constexpr int kUnrollEpi = MODE == kSuffix ? kIt : 1;   // registers xm/xv need it
-#pragma unroll kUnrollEpi
-      for (int it = 0; it < kIt; ++it) {
-        const int pi = tid + it * kConsumerThreads;
-        const int r = pi >> 5, ln = pi & 31;
-        const int e = r & 3, n = (r >> 2) % NT, mtile = (r >> 2) / NT;
-        const int d = mtile * 16 + (ln >> 2) + (e >= 2 ? 8 : 0);
-        const int h = n * 8 + 2 * (ln & 3) + (e & 1);   // query column
-        if (h >= a.ncol) continue;
+      for (int n = 0; n < NT; ++n) {
+        const int h = n * 8 + 2 * (lane & 3) + (cw & 1);
         float M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, mls[w * kMaxGroup + h].x);
-        float Lsum = 0.f, acc = 0.f;
+        float Ls = 0.f;
 #pragma unroll
         for (int w = 0; w < kConsumerWarps; ++w) {
           const float2 ml = mls[w * kMaxGroup + h];
-          const float sc = ml.x == -INFINITY ? 0.f : ex2(ml.x - M);
-          Lsum += ml.y * sc;
-          acc += scr[(w * NREG + r) * 32 + ln] * sc;
+          cs[n][w] = ml.x == -INFINITY ? 0.f : ex2(ml.x - M);
+          Ls += ml.y * cs[n][w];
         }
+        cM[n] = M;
+        cL[n] = Ls;
+        crow[n] = (complete && h < a.ncol) ? out_row<MODE>(a, mt.seq, mt.kvh, h) : -1ll;
+      }
+      float2 xm[NT];
+      float xv[kIt];
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+        xm[n] = (MODE == kSuffix && has_prefix && crow[n] >= 0) ? __ldcg(a.ext_ml + crow[n])
+                                                                 : make_float2(-INFINITY, 0.f);
+#pragma unroll
+      for (int it = 0; it < kIt; ++it) {            // the prefix partials, all loads at once
+        const int n = it % NT, ks = it / NT;
+        const int d = ks * 16 + (lane >> 2) + (cw >= 2 ? 8 : 0);
+        xv[it] = (MODE == kSuffix && has_prefix && crow[n] >= 0) ? __ldcg(a.ext_acc + crow[n] * D + d)
+                                                                  : 0.f;
+      }
+#pragma unroll
+      for (int it = 0; it < kIt; ++it) {
+        const int n = it % NT, ks = it / NT;
+        const int h = n * 8 + 2 * (lane & 3) + (cw & 1);   // query column
+        if (h >= a.ncol) continue;
+        const int d = ks * 16 + (lane >> 2) + (cw >= 2 ? 8 : 0);
+        const int r = cw + 4 * it;                   // scr register row of this value
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) acc += scr[(w * NREG + r) * 32 + lane] * cs[n][w];
         if (complete) {
           // column h = new token (or chunk member) h / group, head kvh * group + h % group;
           // a row that sees no token at all (a new token before the context start) is zero
-          const long long row = out_row<MODE>(a, mt.seq, mt.kvh, h);
-          if (row >= 0) {
-            if constexpr (MODE == kSuffix)
-              finish_row<T, MODE, D>(a, row, M, Lsum, &acc, d, 1, xm[it], &xv[it]);
-            else
-              finish_row<T, MODE, D>(a, row, M, Lsum, &acc, d, 1, make_float2(-INFINITY, 0.f),
-                                     nullptr);
-          }
+          if (crow[n] >= 0)
+            finish_row<T, MODE, D>(a, crow[n], cM[n], cL[n], &acc, d, 1, xm[n], &xv[it]);
         } else {
           a.part_acc[((long long)mt.pidx * kMaxGroup + h) * D + d] = acc;
           if (d == 0) {
-            a.part_ml[((long long)mt.pidx * kMaxGroup + h) * 2 + 0] = M;
-            a.part_ml[((long long)mt.pidx * kMaxGroup + h) * 2 + 1] = Lsum;
+            a.part_ml[((long long)mt.pidx * kMaxGroup + h) * 2 + 0] = cM[n];
+            a.part_ml[((long long)mt.pidx * kMaxGroup + h) * 2 + 1] = cL[n];
           }
         }
       }
@@ -982,8 +981,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         named_bar_sync(1, kConsumerThreads);
         const SplitDesc dsc = desc[mt.qslot];
         if (tid == 0) {
+          // One round trip in the usual case: the last arrival resets the counter to 0,
+          // and the first CTA of a segment (whose portion is the end of its range) is
+          // usually the last to arrive, the others the first.  A wrong guess only costs
+          // a retry with the value the CAS returned.
           unsigned long long* ctr = a.counters + dsc.cf;
-          unsigned long long old = ld_relaxed_gpu(ctr), nxt;
+          unsigned long long old =
+              dsc.cf == c ? ((unsigned long long)a.epoch << 32) | (uint32_t)(dsc.ncontrib - 1) : 0ull,
+              nxt;
           for (;;) {
             nxt = (uint32_t)(old >> 32) == a.epoch ? old + 1
                                                     : ((unsigned long long)a.epoch << 32) | 1ull;
@@ -991,7 +996,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             if (prev == old) break;
             old = prev;
           }
-          *last_flag = (int)(uint32_t)nxt == dsc.ncontrib;
+          const bool last = (int)(uint32_t)nxt == dsc.ncontrib;
+          if (last) st_relaxed_gpu(ctr, 0ull);     // every contributor has arrived
+          *last_flag = last;
         }
         named_bar_sync(1, kConsumerThreads);
         if (*last_flag) merge_split<T, D, NT, MODE>(a, dsc, *total_s, G, group, tid);
