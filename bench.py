@@ -5,9 +5,11 @@
 
 One step = one decode step of the workload over all its layers: pa_copy_blocks of the
 step's copy-on-write pairs (none unless the workload shares partial blocks), then per
-layer pa_cache_append of every sequence's newest token and pa_decode over all cached
-tokens.  Inputs are seeded synthetic tensors already resident in HBM; each layer's K/V
-pools (0.7 GB for the default workload) are larger than L2, so no flush is needed.
+layer the append of every sequence's newest token and decode over all cached tokens --
+by default one pa_decode_append launch per layer (the append fused into decode; same
+bits as the two calls), with --unfused pa_cache_append then pa_decode.  Inputs are
+seeded synthetic tensors already resident in HBM; each layer's K/V pools (0.7 GB for
+the default workload) are larger than L2, so no flush is needed.
 
 With N > 1 (torchrun) every rank runs an independent replica of the workload (the
 path has no exchange step); value = all ranks' KV bytes / the slowest rank's time.
@@ -227,6 +229,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama70b")
     ap.add_argument("--block-size", type=int, default=0)
+    ap.add_argument("--unfused", action="store_true",
+                    help="per layer pa_cache_append then pa_decode (default: pa_decode_append, "
+                         "one launch, where the step has one new token per sequence)")
     ap.add_argument("--cascade", action="store_true",
                     help="decode with pa_decode_cascade (shared prefixes read once per chunk)")
     ap.add_argument("--q-len", type=int, default=1,
@@ -269,6 +274,7 @@ def main():
         wl.use_cascade(b)
     stream = torch.cuda.current_stream()
     L = b.layers
+    fused = not args.unfused and b.q_len == 1 and b.cascade is None
     kv_step = b.kv_bytes_per_step()
     kv_layer = kv_step // L
 
@@ -278,7 +284,7 @@ def main():
             dist.barrier()
 
     for _ in range(args.warmup):
-        wl.run_step(b)
+        wl.run_step(b, fused=fused)
     barrier()
     if int(b.status.item()):
         raise RuntimeError("device status 0x%x after warm-up" % int(b.status.item()))
@@ -293,8 +299,9 @@ def main():
         barrier()
         t_start.record(stream)
         for s in range(args.steps):
-            wl.run_step(b)
-            launches += L * 2 + (1 if b.cow_pairs is not None and b.cow_pairs.shape[0] else 0)
+            wl.run_step(b, fused=fused)
+            launches += L * (1 if fused else 2) * (2 if b.cascade is not None else 1) + \
+                (1 if b.cow_pairs is not None and b.cow_pairs.shape[0] else 0)
         t_end.record(stream)
         barrier()
     ms = t_start.elapsed_time(t_end)
@@ -308,10 +315,14 @@ def main():
         if b.cow_pairs is not None and b.cow_pairs.shape[0]:
             pk.pa_copy_blocks(b.k_caches, b.v_caches, b.cow_pairs, b.status)
         for l in range(L):
-            pk.pa_cache_append(b.k_caches[l], b.v_caches[l], b.k_new[l], b.v_new[l],
-                               b.slot_mapping, b.status)
+            if not fused:
+                pk.pa_cache_append(b.k_caches[l], b.v_caches[l], b.k_new[l], b.v_new[l],
+                                   b.slot_mapping, b.status)
             ev_s[s * L + l].record(stream)
-            wl.decode_layer(b, l)
+            if fused:
+                wl.append_decode_layer(b, l)
+            else:
+                wl.decode_layer(b, l)
             ev_e[s * L + l].record(stream)
     barrier()
     dec_ms = [a.elapsed_time(e) for a, e in zip(ev_s, ev_e)]
@@ -332,7 +343,7 @@ def main():
     # ---------------- end to end through the public API, host buffers
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(b, args, world, kv_step)
+        e2e = run_e2e(b, args, world, kv_step, fused)
 
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -348,6 +359,7 @@ def main():
         "kv_bytes_per_step": kv_step,
         "roofline": {"bound": "hbm", "kernel": "pa_decode_split_kernel (%s)" % (
                          "two launches per pa_decode_cascade" if b.cascade is not None else
+                         "one launch per pa_decode_append" if fused else
                          "one launch per pa_decode" if b.q_len == 1 else
                          "one launch per pa_decode_multi"),
                      "achieved": achieved, "peak": peak, "unit": "GB/s",
@@ -380,7 +392,7 @@ def main():
     return 0
 
 
-def run_e2e(b, args, world, kv_step):
+def run_e2e(b, args, world, kv_step, fused=False):
     """The step through the public API with host buffers.  Every step copies, from pinned
     host memory, every layer's new q / k / v, the block tables, context lens and slot
     mapping, runs append + decode per layer, and copies every layer's output back.
@@ -391,6 +403,7 @@ def run_e2e(b, args, world, kv_step):
     import torch
 
     from paged_kv_cache_348_b200 import pagedkv as pk
+    from paged_kv_cache_348_b200 import workload as wl
 
     L = b.layers
     hq = [t.cpu().pin_memory() for t in b.q]
@@ -431,6 +444,10 @@ def run_e2e(b, args, world, kv_step):
         for l in range(L):
             comp.wait_event(ev_in[l])
             comp.wait_event(ev_out[l])
+            if fused:
+                wl.append_decode_layer(b, l, comp, tabs[m], ctxs[m])
+                ev_used[l].record(comp)
+                continue
             pk.pa_cache_append(b.k_caches[l], b.v_caches[l], b.k_new[l], b.v_new[l], slots[m],
                                b.status, comp)
             if b.cascade is not None:

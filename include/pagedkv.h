@@ -132,6 +132,31 @@ pa_status pa_decode_multi(void* out, const void* q, const void* k_cache, const v
                           int32_t* dev_status, void* stream);
 
 /*
+ * pa_decode_append -- pa_cache_append of each sequence's newest token fused into
+ * pa_decode: one launch instead of two for the usual decode step.
+ *
+ * Defined by the passages of pa_cache_append and pa_decode.  For every sequence s with
+ * context_lens[s] > 0, the newest token sits at position p = context_lens[s] - 1; its
+ * K and V (k_new[s], v_new[s]) are written to the cache row of p,
+ *   cache[block_tables[s][p / block_size]][h][p % block_size][:],
+ * and out is the pa_decode result over positions 0..p with that token included: the
+ * same bits as pa_cache_append (slot of position p) followed by pa_decode.
+ *
+ *   k_new, v_new   device [num_seqs][num_kv_heads][head_dim], 16-byte aligned
+ *   k_cache, v_cache  written at the newest token's rows only
+ *   other arguments, workspace and errors as for pa_decode; an out-of-range block id
+ *   for position p sets PA_DEV_BAD_BLOCK_ID and that token is not written.
+ * The newest token's block must not be shared with another sequence (copy it first,
+ * as for pa_cache_append).
+ */
+pa_status pa_decode_append(void* out, const void* q, void* k_cache, void* v_cache,
+                           const void* k_new, const void* v_new, const int32_t* block_tables,
+                           const int32_t* context_lens, int num_seqs, int num_q_heads,
+                           int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                           int num_blocks, float scale, pa_dtype dtype, void* workspace,
+                           size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
  * pa_decode_cascade -- pa_decode for a batch in which groups of sequences share a prefix
  * of their KV blocks (parallel sampling, beams, a common system prompt), reading each
  * shared block once per chunk of sharers instead of once per sequence.

@@ -159,6 +159,7 @@ pa_status dispatch_mode(int mode, int d, int bs, const pkv::DecodeArgs& a, const
     case pkv::kPlain: return dispatch_d<T, pkv::kPlain>(d, bs, a, mk, mv, grid, s);
     case pkv::kPrefix: return dispatch_d<T, pkv::kPrefix>(d, bs, a, mk, mv, grid, s);
     case pkv::kSuffix: return dispatch_d<T, pkv::kSuffix>(d, bs, a, mk, mv, grid, s);
+    case pkv::kAppend: return dispatch_d<T, pkv::kAppend>(d, bs, a, mk, mv, grid, s);
   }
   return PA_ERR_INVALID;
 }
@@ -171,6 +172,8 @@ struct CascadeArgs {
   int q_rows = 0;
   float2* ext_ml = nullptr;
   float* ext_acc = nullptr;
+  const void* k_new = nullptr;   // kAppend
+  const void* v_new = nullptr;
 };
 
 // Validation, workspace layout, tensor maps and launch shared by the decode entry points.
@@ -246,6 +249,8 @@ pa_status decode_impl(void* out, const void* q, const void* k_cache, const void*
   a.q_rows = cx.q_rows;
   a.ext_ml = cx.ext_ml;
   a.ext_acc = cx.ext_acc;
+  a.k_new = cx.k_new;
+  a.v_new = cx.v_new;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dtype == PA_BF16)
     return dispatch_mode<__nv_bfloat16>(cx.mode, head_dim, block_size, a, mk, mv, grid, st);
@@ -313,6 +318,24 @@ pa_status pa_decode_multi(void* out, const void* q, const void* k_cache, const v
                      num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
                      num_blocks, scale, dtype, workspace, workspace_bytes, 0, dev_status,
                      stream);
+}
+
+pa_status pa_decode_append(void* out, const void* q, void* k_cache, void* v_cache,
+                           const void* k_new, const void* v_new, const int32_t* block_tables,
+                           const int32_t* context_lens, int num_seqs, int num_q_heads,
+                           int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                           int num_blocks, float scale, pa_dtype dtype, void* workspace,
+                           size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  if (num_seqs > 0 && (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)))
+    return PA_ERR_INVALID;
+  CascadeArgs cx;
+  cx.mode = pkv::kAppend;
+  cx.k_new = k_new;
+  cx.v_new = v_new;
+  return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, 1,
+                     num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                     num_blocks, scale, dtype, workspace, workspace_bytes, 0, dev_status, stream,
+                     cx);
 }
 
 size_t pa_decode_cascade_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads,

@@ -71,10 +71,13 @@ enum : int { F_FIRST = 1, F_LAST = 2, F_END = 4, F_COMPLETE = 8 };
 //              member's unnormalised (max, sum, acc) written to the external partials.
 //  kSuffix  -- cascade pass 2: sequence s over its tokens seq_start[s]..ctx-1, merged with
 //              the external partial of its prefix when seq_start[s] > 0.
-enum : int { kPlain = 0, kPrefix = 1, kSuffix = 2 };
+//  kAppend  -- kPlain with one new token per sequence whose K/V (k_new, v_new) are patched
+//              into the tiles and written to the cache in the same launch.
+enum : int { kPlain = 0, kPrefix = 1, kSuffix = 2, kAppend = 3 };
 
 struct StageMeta {
   int seq, kvh, tok0, nunits, ctx, flags, pidx, qslot;
+  int newrow;                           // fused append: cache row of the new token, or -1
 };
 
 struct SeqSpan {
@@ -109,6 +112,9 @@ struct DecodeArgs {
   int q_rows;                   // kPrefix: sequences in q / block_tables (valid member ids)
   float2* ext_ml;               // [members][Hq] (max, sum) of the prefix part, base 2
   float* ext_acc;               // [members][Hq][D] its unnormalised accumulator
+  // kAppend: K/V of each sequence's newest token, [seqs][Hkv][D]
+  const void* k_new;
+  const void* v_new;
 };
 
 
@@ -120,14 +126,20 @@ struct Layout {
   static constexpr int kStageBytes = 2 * kKvBytes + kQBytes;
   static_assert(kStageBytes % 1024 == 0, "stage must keep 1024-byte alignment");
   static constexpr int kMetaOff = kStages * kStageBytes;
-  static constexpr int kBarOff = kMetaOff + kStages * (int)sizeof(StageMeta);
+  static constexpr int kBarOff = (kMetaOff + kStages * (int)sizeof(StageMeta) + 15) / 16 * 16;
   // full[kStages], empty[kStages]
   static constexpr int kMiscOff = kBarOff + (2 * kStages + 1) * 8;
   // abort flag, last-arrival flag, total units
   static constexpr int kDescOff = kMiscOff + 16;
   static constexpr int kMlOff = kDescOff + 2 * (int)sizeof(SplitDesc);
-  static constexpr int kBytes = kMlOff + kConsumerWarps * kMaxGroup * 8;
+  // fused append: per stage the new token's K and V rows, staged by the producer
+  static constexpr int kNewOff = (kMlOff + kConsumerWarps * kMaxGroup * 8 + 15) / 16 * 16;
+  static constexpr int kNewBytes = 2 * D * 2;
+  static constexpr int kBytes = kNewOff + kStages * kNewBytes;
   static constexpr int kDynSmem = kBytes + 1024;           // slack for 1024-byte alignment
+  static_assert(kBarOff % 8 == 0 && kMiscOff % 8 == 0 && kDescOff % 8 == 0 && kMlOff % 8 == 0 &&
+                    kNewOff % 16 == 0 && kNewBytes % 16 == 0,
+                "mbarriers and 64-bit fields need 8-byte, bulk-copy targets 16-byte alignment");
   static_assert(2 * (kDynSmem + 1024) <= 233472, "two CTAs per SM must fit");
 };
 
@@ -599,6 +611,33 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
               return qsrc + (long long)jq * a.num_q_heads * D;
             }
           };
+          // fused append: the stage holding a segment's newest token (position ctx-1)
+          // stages that token's K/V rows from k_new/v_new; its consumer patches them into
+          // the tile and writes them to the cache row found here
+          int newrow = -1;
+          if (MODE == kAppend && tok0 <= ctx_cur - 1 &&
+              ctx_cur - 1 < tok0 + nun * kUnit) {      // warp-uniform
+            const int tn = ctx_cur - 1;
+            int blk_n;
+            if constexpr (BS != 1) {
+              const int wi = tn / BS - wb;
+              if ((tok0 + kTileTokens - 1) / BS >= wb + 64)
+                blk_n = win_lookup(w0, w1, n0, wi);
+              else
+                blk_n = win_lookup(w0, w1, w1, wi);
+            } else {
+              const int r = tn - tok0;
+              blk_n = __shfl_sync(0xffffffffu, r >= 32 ? w1 : w0, r & 31);
+            }
+            if ((unsigned)blk_n < (unsigned)a.num_blocks) newrow = (blk_n * Hkv + kvh) * BS + tn % BS;
+          }
+          const uint32_t nbytes = newrow >= 0 ? (uint32_t)L::kNewBytes : 0u;
+          auto stage_new = [&](uint64_t* bar) {       // lane 0: the two staged rows
+            uint8_t* dst = smem + L::kNewOff + st * L::kNewBytes;
+            const long long src = ((long long)s_cur * Hkv + kvh) * D;
+            bulk_load(dst, static_cast<const T*>(a.k_new) + src, D * 2, bar);
+            bulk_load(dst + D * 2, static_cast<const T*>(a.v_new) + src, D * 2, bar);
+          };
           if constexpr (BS != 1) {
             constexpr int H = BS < 16 ? BS : 16;     // rows per TMA box
             constexpr int BPU = kUnit / H;           // boxes per unit and column half
@@ -629,7 +668,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 y = rows_total;                        // out of range: TMA fills zeros
               }
             }
-            uint32_t bytes = qbytes;
+            uint32_t bytes = qbytes + nbytes;
             for (int jj = 0; jj < nun; ++jj) {
               const int rem = ctx_cur - (tok0 + jj * kUnit);
               const int nb = (rem + H - 1) / H;
@@ -643,11 +682,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             uint8_t* sV = sK + L::kKvBytes;
             uint8_t* sQ = sV + L::kKvBytes;
             if (lane == 0) {
-              meta[st] = StageMeta{s_cur, kvh, tok0, nun, ctx_cur, flags, pidx, qslot};
+              meta[st] = StageMeta{s_cur, kvh, tok0, nun, ctx_cur, flags, pidx, qslot, newrow};
               mbar_arrive_expect_tx(&full[st], bytes);
               if (qbytes)
                 for (int jq = 0; jq < a.q_len; ++jq)
                   bulk_load(sQ + jq * qrow_bytes, qrow_src(jq), qrow_bytes, &full[st]);
+              if (nbytes) stage_new(&full[st]);
             }
             __syncwarp();
             if (mine) {
@@ -669,11 +709,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             uint8_t* sV = sK + L::kKvBytes;
             uint8_t* sQ = sV + L::kKvBytes;
             if (lane == 0) {
-              meta[st] = StageMeta{s_cur, kvh, tok0, nun, ctx_cur, flags, pidx, qslot};
-              mbar_arrive_expect_tx(&full[st], qbytes);
+              meta[st] = StageMeta{s_cur, kvh, tok0, nun, ctx_cur, flags, pidx, qslot, newrow};
+              mbar_arrive_expect_tx(&full[st], qbytes + nbytes);
               if (qbytes)
                 for (int jq = 0; jq < a.q_len; ++jq)
                   bulk_load(sQ + jq * qrow_bytes, qrow_src(jq), qrow_bytes, &full[st]);
+              if (nbytes) stage_new(&full[st]);
             }
             const int ch = lane % CPR, hf = ch >> 3, cc = ch & 7;
             for (int r0 = 0; r0 < ntok; r0 += RPI) {
@@ -785,12 +826,31 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         l[n][0] = l[n][1] = 0.f;
       }
     }
+    bool patched = false;
     if (cw < mt.nunits) {
       const int t0 = mt.tok0 + cw * kUnit;
       const int valid = (mt.ctx - t0) < kUnit ? (mt.ctx - t0) : kUnit;
       // causal limit: new token j sees unit rows < ctx - q_len + 1 + j - t0 (a prefix
       // launch's columns are different sequences: no mask)
       const int lim0 = MODE == kPrefix ? (1 << 30) : mt.ctx - a.q_len + 1 - t0;
+      if (MODE == kAppend && mt.newrow >= 0 && (mt.ctx - 1 - mt.tok0) / kUnit == cw) {
+        // fused append: this unit holds the newest token; its K/V rows come from the
+        // staging area (the cache row the TMA read may still be old) and are written to
+        // the cache
+        constexpr int CPR = D * 2 / 16;               // 16-byte chunks per row
+        const int rn = mt.ctx - 1 - mt.tok0;          // row in the stage tile
+        if (lane < 2 * CPR) {
+          const int kv = lane / CPR, ch = lane % CPR, hf = ch >> 3, cc = ch & 7;
+          const uint4 val = *reinterpret_cast<const uint4*>(smem + L::kNewOff + st * L::kNewBytes +
+                                                            kv * D * 2 + ch * 16);
+          *reinterpret_cast<uint4*>((kv ? sV : sK) + hf * (kTileTokens * 128) + rn * 128 +
+                                    ((cc ^ (rn & 7)) << 4)) = val;
+          T* cache = static_cast<T*>(const_cast<void*>(kv ? a.v_cache : a.k_cache));
+          *reinterpret_cast<uint4*>(cache + (long long)mt.newrow * D + ch * 8) = val;
+        }
+        __syncwarp();
+        patched = true;
+      }
       const uint32_t kbase = smem_u32(sK), vbase = smem_u32(sV);
       // ---- S^T[16 tokens][8*NT heads] = K_unit . q^T
       float sacc[NT][4];
@@ -1005,6 +1065,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       }
       fence_proxy_async_smem();   // generic writes above precede the next TMA fill
     }
+    if (patched) fence_proxy_async_smem();   // the patched row precedes the next TMA fill
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[st]);
     if (++st == kStages) {

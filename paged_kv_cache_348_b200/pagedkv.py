@@ -24,7 +24,8 @@ DEV_BAD_BLOCK_ID, DEV_BAD_SLOT, DEV_BAD_PAIR, DEV_BAD_CONTEXT_LEN, DEV_TIMEOUT =
 
 # every symbol include/pagedkv.h declares
 EXPORTS = ("pa_version", "pa_status_string", "pa_decode_workspace_bytes", "pa_decode",
-           "pa_decode_multi", "pa_decode_cascade_workspace_bytes", "pa_decode_cascade",
+           "pa_decode_multi", "pa_decode_append", "pa_decode_cascade_workspace_bytes",
+           "pa_decode_cascade",
            "pa_cache_append", "pa_copy_blocks", "pa_decode_noalloc",
            "pa_bm_create", "pa_bm_destroy", "pa_bm_free_blocks", "pa_bm_refcount",
            "pa_bm_allocate", "pa_bm_fork", "pa_bm_append_tokens", "pa_bm_release",
@@ -62,6 +63,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         L.pa_decode_multi.restype = i32
         L.pa_decode_multi.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, i32,
                                       f32, i32, P, sz, P, P]
+        L.pa_decode_append.restype = i32
+        L.pa_decode_append.argtypes = [P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32,
+                                       f32, i32, P, sz, P, P]
         L.pa_decode_cascade_workspace_bytes.restype = sz
         L.pa_decode_cascade_workspace_bytes.argtypes = [i32, i32, i32, i32]
         L.pa_decode_cascade.restype = i32
@@ -174,6 +178,35 @@ def pa_decode_multi(out, q, k_cache, v_cache, block_tables, context_lens, scale:
                                 _ptr(workspace), workspace.numel() * workspace.element_size(),
                                 _ptr(status), _stream(stream))
     _check(rc, "pa_decode_multi")
+    return out
+
+
+def pa_decode_append(out, q, k_cache, v_cache, k_new, v_new, block_tables, context_lens,
+                     scale: float, workspace, status=None, stream=None):
+    """Append each sequence's newest token (k_new/v_new [B,Hkv,D], at position
+    context_lens-1) into the caches and decode, in one launch (see pa_decode_append in
+    include/pagedkv.h)."""
+    _need(q, "q", ndim=3)
+    _need(out, "out", dtype=q.dtype, ndim=3)
+    _need(k_cache, "k_cache", dtype=q.dtype, ndim=4)
+    _need(v_cache, "v_cache", dtype=q.dtype, ndim=4)
+    _need(k_new, "k_new", dtype=q.dtype, ndim=3)
+    _need(v_new, "v_new", dtype=q.dtype, ndim=3)
+    _need(block_tables, "block_tables", dtype=torch.int32, ndim=2)
+    _need(context_lens, "context_lens", dtype=torch.int32, ndim=1)
+    _need(workspace, "workspace")
+    B, Hq, D = q.shape
+    N, Hkv, bs, D2 = k_cache.shape
+    if out.shape != q.shape or D2 != D or v_cache.shape != k_cache.shape or \
+            k_new.shape != (B, Hkv, D) or v_new.shape != k_new.shape or \
+            block_tables.shape[0] != B or context_lens.shape[0] != B:
+        raise PagedKVError("pa_decode_append: inconsistent shapes")
+    rc = load().pa_decode_append(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_new),
+                                 _ptr(v_new), _ptr(block_tables), _ptr(context_lens), B, Hq, Hkv,
+                                 D, bs, block_tables.shape[1], N, float(scale), _dtype_code(q),
+                                 _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                 _ptr(status), _stream(stream))
+    _check(rc, "pa_decode_append")
     return out
 
 

@@ -164,14 +164,29 @@ def build_prefix_fork(w: inputs.Workload = inputs.PREFIX, device="cuda") -> Deco
     return _finish(w, bs, bm, sids, N, w.layers, device, cow_pairs=pairs)
 
 
-def run_step(b: DecodeBatch, stream=None, layers=None) -> None:
-    """One decode step over all layers (see module docstring)."""
+def run_step(b: DecodeBatch, stream=None, layers=None, fused: bool = False) -> None:
+    """One decode step over all layers (see module docstring).  With fused=True each
+    layer is one pa_decode_append call (the newest token's append fused into decode;
+    one new token per sequence, no cascade)."""
     if b.cow_pairs is not None and b.cow_pairs.shape[0]:
         pk.pa_copy_blocks(b.k_caches, b.v_caches, b.cow_pairs, b.status, stream)
     for l in range(layers if layers is not None else b.layers):
+        if fused:
+            append_decode_layer(b, l, stream)
+            continue
         pk.pa_cache_append(b.k_caches[l], b.v_caches[l], b.k_new[l], b.v_new[l], b.slot_mapping,
                            b.status, stream)
         decode_layer(b, l, stream)
+
+
+def append_decode_layer(b: DecodeBatch, l: int, stream=None, block_tables=None,
+                        context_lens=None) -> None:
+    """pa_decode_append of layer l: append the newest token of every sequence and decode."""
+    assert b.q_len == 1 and b.cascade is None
+    pk.pa_decode_append(b.out[l], b.q[l], b.k_caches[l], b.v_caches[l], b.k_new[l], b.v_new[l],
+                        b.block_tables if block_tables is None else block_tables,
+                        b.context_lens if context_lens is None else context_lens, b.scale,
+                        b.workspace, b.status, stream)
 
 
 def use_cascade(b: DecodeBatch, width: int | None = None) -> DecodeBatch:
