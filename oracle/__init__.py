@@ -57,6 +57,15 @@ def _load():
         L.orc_decode_multi.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32,
                                        i32, f64, i32, P, i32, i32]
         L.orc_decode_multi.restype = i32
+        u8, f32 = ctypes.c_uint8, ctypes.c_float
+        L.orc_e4m3_to_f64.argtypes = [u8]; L.orc_e4m3_to_f64.restype = f64
+        L.orc_f64_to_e4m3.argtypes = [f64]; L.orc_f64_to_e4m3.restype = u8
+        L.orc_quantize_e4m3.argtypes = [u16, i32, f32]; L.orc_quantize_e4m3.restype = u8
+        L.orc_decode_e4m3.argtypes = [P, P, P, P, P, f64, f64, P, P, i32, i32, i32, i32, i32, i32,
+                                      i32, i32, f64, i32, P, i32, i32]
+        L.orc_decode_e4m3.restype = i32
+        L.orc_cache_append_e4m3.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, f32]
+        L.orc_cache_append_e4m3.restype = i32
         L.orc_cache_append.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32]
         L.orc_cache_append.restype = i32
         L.orc_copy_blocks.argtypes = [P, P, i32, P, i32, i64, i32]
@@ -156,6 +165,63 @@ def decode_multi(q, k_cache, v_cache, block_tables, context_lens, scale: float, 
     if rc:
         raise ValueError("oracle decode: bad arguments (%d)" % rc)
     return out64, out16
+
+
+# ---- 8-bit E4M3 cache ----------------------------------------------------------------
+def e4m3_to_f64(code: int) -> float:
+    return _load().orc_e4m3_to_f64(int(code))
+
+
+def f64_to_e4m3(x: float) -> int:
+    """Round to nearest even, magnitudes above 448 clamped to 448, NaN kept."""
+    return _load().orc_f64_to_e4m3(float(x))
+
+
+def quantize_e4m3(bits: int, dtype: str, scale: float) -> int:
+    """Code of a 16-bit value for a per-tensor scale (x / scale in binary32, then E4M3)."""
+    return _load().orc_quantize_e4m3(int(bits), DTYPES[dtype], float(scale))
+
+
+def cache_append_e4m3(k_cache8, v_cache8, k, v, slot_mapping, dtype: str, k_scale: float,
+                      v_scale: float):
+    """In-place quantising scatter of 16-bit k/v [T, Hkv, D] into uint8 E4M3 pools."""
+    assert k_cache8.flags.c_contiguous and v_cache8.flags.c_contiguous
+    assert k_cache8.dtype == np.uint8 and v_cache8.dtype == np.uint8
+    N, Hkv, bs, D = k_cache8.shape
+    k = _c(k, np.uint16); v = _c(v, np.uint16)
+    sm = _c(slot_mapping, np.int64)
+    rc = _load().orc_cache_append_e4m3(_p(k_cache8), _p(v_cache8), _p(k), _p(v), _p(sm), len(sm),
+                                       Hkv, D, bs, N, DTYPES[dtype], float(k_scale), float(v_scale))
+    if rc:
+        raise ValueError("oracle append: slot out of range")
+
+
+def decode_e4m3(q, k_cache8, v_cache8, k_scale: float, v_scale: float, block_tables,
+                context_lens, scale: float, dtype: str, items=None, nthreads: int = 1):
+    """fp64 paged decode over uint8 E4M3 pools (values k_scale * code, v_scale * code);
+    q [B, Hq, D] or [B, q_len, Hq, D] in `dtype`.  Returns (out64, out16) shaped like q."""
+    q = _c(q, np.uint16)
+    k8 = _c(k_cache8, np.uint8)
+    v8 = _c(v_cache8, np.uint8)
+    bt = _c(block_tables, np.int32)
+    cl = _c(context_lens, np.int32)
+    shape = q.shape
+    q4 = q.reshape(shape[0], 1, shape[1], shape[2]) if q.ndim == 3 else q
+    B, QL, Hq, D = q4.shape
+    N, Hkv, bs, D2 = k8.shape
+    assert D2 == D and v8.shape == k8.shape and bt.shape[0] == B
+    out64 = np.zeros((B, QL, Hq, D), dtype=np.float64)
+    out16 = np.zeros((B, QL, Hq, D), dtype=np.uint16)
+    it = None if items is None else _c(items, np.int32)
+    rc = _load().orc_decode_e4m3(_p(out64), _p(out16), _p(q4), _p(k8), _p(v8), float(k_scale),
+                                 float(v_scale), _p(bt), _p(cl), B, QL, Hq, Hkv, D, bs, bt.shape[1],
+                                 N, float(scale), DTYPES[dtype], None if it is None else _p(it),
+                                 0 if it is None else len(it), int(nthreads))
+    if rc == -1:
+        raise ValueError("oracle decode: block id out of range")
+    if rc:
+        raise ValueError("oracle decode: bad arguments (%d)" % rc)
+    return out64.reshape(shape), out16.reshape(shape)
 
 
 def cache_append(k_cache, v_cache, k, v, slot_mapping):

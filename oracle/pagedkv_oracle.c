@@ -97,6 +97,52 @@ static uint16_t f64_to_small(double x, int mant, int bias, int ebits) {
 uint16_t orc_f64_to_f16(double x) { return f64_to_small(x, 10, 15, 5); }
 uint16_t orc_f64_to_bf16(double x) { return f64_to_small(x, 7, 127, 8); }
 
+/* ---- 8-bit E4M3 (1 sign, 4 exponent bits with bias 7, 3 fraction bits; no infinity;
+ *      S.1111.111 is NaN, so the largest finite magnitude is 1.75 * 2^8 = 448) ------- */
+double orc_e4m3_to_f64(uint8_t b) {
+  int sign = (b >> 7) & 1;
+  int e = (b >> 3) & 0xf;
+  int f = b & 7;
+  double v;
+  if (e == 15 && f == 7)
+    v = NAN;
+  else if (e == 0)
+    v = ldexp((double)f, -9);              /* subnormal: f/8 * 2^-6 */
+  else
+    v = ldexp((double)(f | 8), e - 10);    /* (8+f)/8 * 2^(e-7) */
+  return sign ? -v : v;
+}
+
+/* Round to nearest, ties to even, then clamp magnitudes above 448 to 448 ("satfinite");
+ * NaN stays NaN. */
+uint8_t orc_f64_to_e4m3(double x) {
+  uint8_t sign = signbit(x) ? 0x80 : 0;
+  if (isnan(x)) return (uint8_t)(sign | 0x7f);
+  double ax = fabs(x);
+  if (ax == 0.0) return sign;
+  if (isinf(ax)) return (uint8_t)(sign | 0x7e);
+  int e;
+  frexp(ax, &e);
+  int unbiased = e - 1;                    /* ax in [2^unbiased, 2^(unbiased+1)) */
+  if (unbiased < -6) unbiased = -6;        /* subnormals share the 2^-9 step */
+  if (unbiased > 8) return (uint8_t)(sign | 0x7e);
+  double ulp = ldexp(1.0, unbiased - 3);
+  double n = rne_units(ax, ulp);           /* significand in units of ulp, 0..16 */
+  if (n >= 16.0) { n /= 2.0; unbiased += 1; }
+  if (unbiased > 8 || (unbiased == 8 && n > 14.0)) return (uint8_t)(sign | 0x7e);
+  uint32_t m = (uint32_t)n;
+  if (m < 8) return (uint8_t)(sign | m);   /* subnormal (unbiased == -6) */
+  return (uint8_t)(sign | (uint32_t)(unbiased + 7) << 3 | (m - 8));
+}
+
+/* The quantised code of a 16-bit cache input for a per-tensor scale: x / scale divided
+ * in binary32 (round to nearest), then rounded to E4M3 as above. */
+uint8_t orc_quantize_e4m3(uint16_t bits, int dtype, float scale) {
+  float xf = (float)(dtype == 1 ? orc_bf16_to_f64(bits) : orc_f16_to_f64(bits));
+  volatile float q = xf / scale;
+  return orc_f64_to_e4m3((double)q);
+}
+
 static double to_f64(uint16_t v, int dtype) {
   return dtype == ORC_BF16 ? orc_bf16_to_f64(v) : orc_f16_to_f64(v);
 }
@@ -119,17 +165,33 @@ static int64_t cache_row(int64_t b, int h, int o, int Hkv, int bs, int D) {
 }
 
 /* Gather the logical rows 0..ctx-1 of one sequence and kv head into out[ctx][D] (fp64).
+ * cache_dtype ORC_F16 / ORC_BF16: 16-bit elements; ORC_E4M3: 8-bit codes, each value
+ * multiplied by `scale` (the per-tensor dequantisation scale).
  * Returns 0, or -1 if a needed block-table entry lies outside [0, num_blocks). */
-int orc_gather(double* out, const uint16_t* cache, int dtype, int num_blocks, int Hkv,
-               int bs, int D, const int32_t* table_row, int ctx, int kvh) {
+#define ORC_E4M3 2
+int orc_gather_any(double* out, const void* cache, int cache_dtype, double scale,
+                   int num_blocks, int Hkv, int bs, int D, const int32_t* table_row, int ctx,
+                   int kvh) {
   for (int t = 0; t < ctx; ++t) {
     int32_t b = table_row[t / bs];          /* logical block t/bs -> physical block */
     int o = t % bs;                         /* position inside the block */
     if (b < 0 || b >= num_blocks) return -1;
-    const uint16_t* row = cache + cache_row(b, kvh, o, Hkv, bs, D);
-    for (int d = 0; d < D; ++d) out[(int64_t)t * D + d] = to_f64(row[d], dtype);
+    int64_t r = cache_row(b, kvh, o, Hkv, bs, D);
+    for (int d = 0; d < D; ++d) {
+      double v;
+      if (cache_dtype == ORC_E4M3)
+        v = scale * orc_e4m3_to_f64(((const uint8_t*)cache)[r + d]);
+      else
+        v = to_f64(((const uint16_t*)cache)[r + d], cache_dtype);
+      out[(int64_t)t * D + d] = v;
+    }
   }
   return 0;
+}
+
+int orc_gather(double* out, const uint16_t* cache, int dtype, int num_blocks, int Hkv,
+               int bs, int D, const int32_t* table_row, int ctx, int kvh) {
+  return orc_gather_any(out, cache, dtype, 1.0, num_blocks, Hkv, bs, D, table_row, ctx, kvh);
 }
 
 /* ---- decode attention: [P1] "How PagedAttention borrows OS paging" -- the math is
@@ -143,9 +205,12 @@ int orc_gather(double* out, const uint16_t* cache, int dtype, int num_blocks, in
 typedef struct {
   double* out64;
   uint16_t* out16;
-  const uint16_t *q, *k_cache, *v_cache;
+  const uint16_t* q;
+  const void *k_cache, *v_cache;
   const int32_t *block_tables, *context_lens, *items;
   int n_items, q_len, Hq, Hkv, D, bs, max_blocks, num_blocks, dtype;
+  int cache_dtype;                          /* dtype, or ORC_E4M3 with the scales below */
+  double k_scale, v_scale;
   double scale;
   atomic_int next;
   atomic_int err;
@@ -162,8 +227,10 @@ static void decode_one(decode_job* J, int s, int j, int h, double* kbuf, double*
   for (int d = 0; d < D; ++d) o64[d] = 0.0;
   if (n > 0) {
     const int32_t* table_row = J->block_tables + (int64_t)s * J->max_blocks;
-    if (orc_gather(kbuf, J->k_cache, J->dtype, J->num_blocks, J->Hkv, J->bs, D, table_row, n, kvh) ||
-        orc_gather(vbuf, J->v_cache, J->dtype, J->num_blocks, J->Hkv, J->bs, D, table_row, n, kvh)) {
+    if (orc_gather_any(kbuf, J->k_cache, J->cache_dtype, J->k_scale, J->num_blocks, J->Hkv, J->bs,
+                       D, table_row, n, kvh) ||
+        orc_gather_any(vbuf, J->v_cache, J->cache_dtype, J->v_scale, J->num_blocks, J->Hkv, J->bs,
+                       D, table_row, n, kvh)) {
       atomic_store(&J->err, 1);
       return;
     }
@@ -221,6 +288,26 @@ static void* decode_worker(void* arg) {
  * 16-bit copy).  `items` (nullable) restricts the work to the listed sequences (sampled
  * checks); rows of other sequences are left untouched.  Returns 0, -1 on a bad block
  * id, -2 on bad arguments or allocation failure. */
+static int run_decode(decode_job* J, int B, int nthreads);
+
+/* Decode over an 8-bit E4M3 cache: q and out as for orc_decode_multi (16-bit dtype), the
+ * cache values are k_scale * code and v_scale * code. */
+int orc_decode_e4m3(double* out64, uint16_t* out16, const uint16_t* q, const uint8_t* k_cache,
+                    const uint8_t* v_cache, double k_scale, double v_scale,
+                    const int32_t* block_tables, const int32_t* context_lens, int B, int q_len,
+                    int Hq, int Hkv, int D, int bs, int max_blocks, int num_blocks, double scale,
+                    int dtype, const int32_t* items, int n_items, int nthreads) {
+  if (B < 0 || q_len < 1 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || D <= 0 || bs <= 0) return -2;
+  decode_job J;
+  J.out64 = out64; J.out16 = out16; J.q = q; J.k_cache = k_cache; J.v_cache = v_cache;
+  J.cache_dtype = ORC_E4M3; J.k_scale = k_scale; J.v_scale = v_scale;
+  J.block_tables = block_tables; J.context_lens = context_lens;
+  J.items = items; J.n_items = items ? n_items : B;
+  J.q_len = q_len; J.Hq = Hq; J.Hkv = Hkv; J.D = D; J.bs = bs; J.max_blocks = max_blocks;
+  J.num_blocks = num_blocks; J.dtype = dtype; J.scale = scale;
+  return run_decode(&J, B, nthreads);
+}
+
 int orc_decode_multi(double* out64, uint16_t* out16, const uint16_t* q, const uint16_t* k_cache,
                      const uint16_t* v_cache, const int32_t* block_tables,
                      const int32_t* context_lens, int B, int q_len, int Hq, int Hkv, int D, int bs,
@@ -229,28 +316,34 @@ int orc_decode_multi(double* out64, uint16_t* out16, const uint16_t* q, const ui
   if (B < 0 || q_len < 1 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || D <= 0 || bs <= 0) return -2;
   decode_job J;
   J.out64 = out64; J.out16 = out16; J.q = q; J.k_cache = k_cache; J.v_cache = v_cache;
+  J.cache_dtype = dtype; J.k_scale = 1.0; J.v_scale = 1.0;
   J.block_tables = block_tables; J.context_lens = context_lens;
   J.items = items; J.n_items = items ? n_items : B;
   J.q_len = q_len; J.Hq = Hq; J.Hkv = Hkv; J.D = D; J.bs = bs; J.max_blocks = max_blocks;
   J.num_blocks = num_blocks; J.dtype = dtype; J.scale = scale;
-  atomic_init(&J.next, 0);
-  atomic_init(&J.err, 0);
-  for (int i = 0; i < J.n_items; ++i) {
-    int s = items ? items[i] : i;
+  return run_decode(&J, B, nthreads);
+}
+
+static int run_decode(decode_job* J, int B, int nthreads) {
+  atomic_init(&J->next, 0);
+  atomic_init(&J->err, 0);
+  for (int i = 0; i < J->n_items; ++i) {
+    int s = J->items ? J->items[i] : i;
     if (s < 0 || s >= B) return -2;
-    if (context_lens[s] < 0 || (int64_t)context_lens[s] > (int64_t)max_blocks * bs) return -2;
+    if (J->context_lens[s] < 0 || (int64_t)J->context_lens[s] > (int64_t)J->max_blocks * J->bs)
+      return -2;
   }
   if (nthreads < 1) nthreads = 1;
   if (nthreads == 1) {
-    decode_worker(&J);
+    decode_worker(J);
   } else {
     pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * nthreads);
     if (!th) return -2;
-    for (int i = 0; i < nthreads; ++i) pthread_create(&th[i], NULL, decode_worker, &J);
+    for (int i = 0; i < nthreads; ++i) pthread_create(&th[i], NULL, decode_worker, J);
     for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
     free(th);
   }
-  int e = atomic_load(&J.err);
+  int e = atomic_load(&J->err);
   return e == 1 ? -1 : (e ? -2 : 0);
 }
 
@@ -281,6 +374,30 @@ int orc_cache_append(uint16_t* k_cache, uint16_t* v_cache, const uint16_t* k, co
       int64_t src = ((int64_t)i * Hkv + h) * D;
       memcpy(k_cache + dst, k + src, (size_t)D * sizeof(uint16_t));
       memcpy(v_cache + dst, v + src, (size_t)D * sizeof(uint16_t));
+    }
+  }
+  return 0;
+}
+
+/* Quantising append into 8-bit E4M3 caches: for every token i with slot >= 0, the codes
+ * orc_quantize_e4m3(k[i][h][d], dtype, k_scale) (and likewise v) go to
+ * [slot/bs][h][slot%bs][d]; a negative slot is skipped. */
+int orc_cache_append_e4m3(uint8_t* k_cache, uint8_t* v_cache, const uint16_t* k, const uint16_t* v,
+                          const int64_t* slots, int T, int Hkv, int D, int bs, int num_blocks,
+                          int dtype, float k_scale, float v_scale) {
+  for (int i = 0; i < T; ++i) {
+    int64_t s = slots[i];
+    if (s < 0) continue;
+    if (s >= (int64_t)num_blocks * bs) return -1;
+    int64_t b = s / bs;
+    int o = (int)(s % bs);
+    for (int h = 0; h < Hkv; ++h) {
+      int64_t dst = cache_row(b, h, o, Hkv, bs, D);
+      int64_t src = ((int64_t)i * Hkv + h) * D;
+      for (int d = 0; d < D; ++d) {
+        k_cache[dst + d] = orc_quantize_e4m3(k[src + d], dtype, k_scale);
+        v_cache[dst + d] = orc_quantize_e4m3(v[src + d], dtype, v_scale);
+      }
     }
   }
   return 0;
