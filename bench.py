@@ -159,7 +159,10 @@ def oracle_sample(w, bs, max_seconds=15.0, device_batch=None):
     if device_batch is not None:
         b = device_batch
         def bits(t):
-            return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+            t = t.detach().cpu().contiguous()
+            if t.dtype == torch.uint8:
+                return t.numpy()
+            return t.view(torch.int16).numpy().view(np.uint16)
         q, k, v = bits(b.q[0]), bits(b.k_caches[0]), bits(b.v_caches[0])
         tables, ctx = b.block_tables.cpu().numpy(), b.context_lens.cpu().numpy()
     else:
@@ -177,11 +180,16 @@ def oracle_sample(w, bs, max_seconds=15.0, device_batch=None):
     while i < len(order) and spent < max_seconds:
         items = order[i:i + chunk]
         t0 = time.perf_counter()
-        fn = oracle.decode if q.ndim == 3 else oracle.decode_multi
-        fn(q, k, v, tables, ctx, 1.0 / math.sqrt(w.head_dim), w.dtype, items=items,
-           nthreads=threads)
+        if k.dtype == np.uint8:
+            oracle.decode_e4m3(q, k, v, *b.kv_scales, tables, ctx, 1.0 / math.sqrt(w.head_dim),
+                               w.dtype, items=items, nthreads=threads)
+        else:
+            fn = oracle.decode if q.ndim == 3 else oracle.decode_multi
+            fn(q, k, v, tables, ctx, 1.0 / math.sqrt(w.head_dim), w.dtype, items=items,
+               nthreads=threads)
         spent += time.perf_counter() - t0
-        done_bytes += int(sum(int(ctx[s]) for s in items)) * w.num_kv_heads * w.head_dim * 4
+        done_bytes += int(sum(int(ctx[s]) for s in items)) * w.num_kv_heads * w.head_dim * 2 * \
+            k.dtype.itemsize
         seqs += len(items)
         i += chunk
     return done_bytes, spent, seqs, threads
@@ -232,6 +240,8 @@ def main():
     ap.add_argument("--unfused", action="store_true",
                     help="per layer pa_cache_append then pa_decode (default: pa_decode_append, "
                          "one launch, where the step has one new token per sequence)")
+    ap.add_argument("--kv-fp8", action="store_true",
+                    help="8-bit E4M3 KV pools (pa_cache_append_e4m3 + pa_decode_e4m3)")
     ap.add_argument("--cascade", action="store_true",
                     help="decode with pa_decode_cascade (shared prefixes read once per chunk)")
     ap.add_argument("--q-len", type=int, default=1,
@@ -269,12 +279,12 @@ def main():
         b = wl.build_prefix_decode(w, device="cuda")
     else:
         b = wl.build(w, device="cuda", block_size=bs, layers=args.layers or None,
-                     q_len=args.q_len)
+                     q_len=args.q_len, kv8=args.kv_fp8)
     if args.cascade:
         wl.use_cascade(b)
     stream = torch.cuda.current_stream()
     L = b.layers
-    fused = not args.unfused and b.q_len == 1 and b.cascade is None
+    fused = not args.unfused and b.q_len == 1 and b.cascade is None and b.kv_scales is None
     kv_step = b.kv_bytes_per_step()
     kv_layer = kv_step // L
 
@@ -315,7 +325,10 @@ def main():
         if b.cow_pairs is not None and b.cow_pairs.shape[0]:
             pk.pa_copy_blocks(b.k_caches, b.v_caches, b.cow_pairs, b.status)
         for l in range(L):
-            if not fused:
+            if b.kv_scales is not None:
+                pk.pa_cache_append_e4m3(b.k_caches[l], b.v_caches[l], b.k_new[l], b.v_new[l],
+                                        b.slot_mapping, *b.kv_scales, b.status)
+            elif not fused:
                 pk.pa_cache_append(b.k_caches[l], b.v_caches[l], b.k_new[l], b.v_new[l],
                                    b.slot_mapping, b.status)
             ev_s[s * L + l].record(stream)
@@ -348,7 +361,8 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": w.dtype + ("+e4m3 kv" if b.kv_scales is not None else ""), "data": "synthetic",
         "config": {"workload": workload_desc(w, bs, b.layers, b.q_len), "global_batch": w.num_seqs * world,
                    "seq_len": float(b.context_lens.float().mean().item()),
                    "parallelism": "replicas" if world > 1 else "single gpu",
@@ -360,6 +374,7 @@ def main():
         "roofline": {"bound": "hbm", "kernel": "pa_decode_split_kernel (%s)" % (
                          "two launches per pa_decode_cascade" if b.cascade is not None else
                          "one launch per pa_decode_append" if fused else
+                         "one launch per pa_decode_e4m3" if b.kv_scales is not None else
                          "one launch per pa_decode" if b.q_len == 1 else
                          "one launch per pa_decode_multi"),
                      "achieved": achieved, "peak": peak, "unit": "GB/s",
@@ -446,6 +461,13 @@ def run_e2e(b, args, world, kv_step, fused=False):
             comp.wait_event(ev_out[l])
             if fused:
                 wl.append_decode_layer(b, l, comp, tabs[m], ctxs[m])
+                ev_used[l].record(comp)
+                continue
+            if b.kv_scales is not None:
+                pk.pa_cache_append_e4m3(b.k_caches[l], b.v_caches[l], b.k_new[l], b.v_new[l],
+                                        slots[m], *b.kv_scales, b.status, comp)
+                pk.pa_decode_e4m3(b.out[l], b.q[l], b.k_caches[l], b.v_caches[l], *b.kv_scales,
+                                  tabs[m], ctxs[m], b.scale, b.workspace, b.status, comp)
                 ev_used[l].record(comp)
                 continue
             pk.pa_cache_append(b.k_caches[l], b.v_caches[l], b.k_new[l], b.v_new[l], slots[m],

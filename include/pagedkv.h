@@ -157,6 +157,38 @@ pa_status pa_decode_append(void* out, const void* q, void* k_cache, void* v_cach
                            size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 /*
+ * 8-bit KV cache (E4M3): half the bytes per cached token.
+ *
+ * Defined by [P3] "What's Still Unsolved" (FP4/FP8 quantised KV cache: lower precision
+ * saves memory).  Format: E4M3 -- 1 sign bit, 4 exponent bits with bias 7, 3 fraction
+ * bits, no infinity, S.1111.111 = NaN; largest finite value 448.  A pool holds codes c
+ * with value scale * c for one per-tensor scale per pool (k_scale for K, v_scale for V,
+ * chosen by the caller, > 0).  Layout as for 16-bit pools with 1-byte elements.
+ *
+ * pa_cache_append_e4m3 -- pa_cache_append into E4M3 pools: every value x of k (v) is
+ * stored as the E4M3 code of x / k_scale (x / v_scale) computed in binary32 with IEEE
+ * division, rounded to nearest even, magnitudes above 448 clamped to 448.  k and v are
+ * 16-bit (dtype); head_dim a multiple of 16.  Other arguments and errors as for
+ * pa_cache_append.
+ *
+ * pa_decode_e4m3 -- pa_decode over E4M3 pools: K_s[t] = k_scale * code, V_s[t] = v_scale *
+ * code, everything else as for pa_decode (q and out 16-bit, dtype).  Inside, the codes
+ * are converted exactly to fp16 and the products use fp16 tensor-core MMAs with fp32
+ * accumulation (q is converted to fp16: values beyond fp16's range are not supported).
+ * head_dim 128 only (PA_ERR_UNSUPPORTED otherwise); workspace as for pa_decode.
+ */
+pa_status pa_cache_append_e4m3(void* k_cache, void* v_cache, const void* k, const void* v,
+                               const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
+                               int head_dim, int block_size, int num_blocks, pa_dtype dtype,
+                               float k_scale, float v_scale, int32_t* dev_status, void* stream);
+pa_status pa_decode_e4m3(void* out, const void* q, const void* k_cache, const void* v_cache,
+                         float k_scale, float v_scale, const int32_t* block_tables,
+                         const int32_t* context_lens, int num_seqs, int num_q_heads,
+                         int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                         int num_blocks, float scale, pa_dtype dtype, void* workspace,
+                         size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
  * pa_decode_cascade -- pa_decode for a batch in which groups of sequences share a prefix
  * of their KV blocks (parallel sampling, beams, a common system prompt), reading each
  * shared block once per chunk of sharers instead of once per sequence.

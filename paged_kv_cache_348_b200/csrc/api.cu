@@ -62,15 +62,18 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 // 2-D view of one pool: rows = num_blocks*kv_heads*block_size, each head_dim elements;
 // box = 64 dims x box_rows rows, 128-byte swizzle, out-of-range rows read as zero.
+// kv8: an 8-bit (E4M3) pool, rows of head_dim bytes, box = head_dim x box_rows (128 B).
 bool encode_pool(CUtensorMap* map, const void* base, pa_dtype dtype, int head_dim,
-                 uint64_t rows, int box_rows) {
+                 uint64_t rows, int box_rows, bool kv8 = false) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
-  cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+  cuuint64_t strides[1] = {(cuuint64_t)head_dim * (kv8 ? 1 : 2)};
+  cuuint32_t box[2] = {kv8 ? (cuuint32_t)head_dim : 64u, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1u, 1u};
-  CUresult r = enc(map, dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+  CUresult r = enc(map, kv8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                            : dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                               : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
                    2, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -112,11 +115,11 @@ cudaError_t launch(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
-template <typename T, int D, int BS, int NT, int MODE>
+template <typename T, int D, int BS, int NT, int MODE, bool KV8 = false>
 pa_status launch_decode(const pkv::DecodeArgs& a, const CUtensorMap& mk, const CUtensorMap& mv,
                         int grid, cudaStream_t stream) {
-  using L = pkv::Layout<D>;
-  auto split = pkv::pa_decode_split_kernel<T, D, BS, NT, MODE>;
+  using L = pkv::Layout<D, KV8>;
+  auto split = pkv::pa_decode_split_kernel<T, D, BS, NT, MODE, KV8>;
   if (cudaFuncSetAttribute(split, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynSmem) !=
       cudaSuccess)
     return PA_ERR_CUDA;
@@ -164,6 +167,24 @@ pa_status dispatch_mode(int mode, int d, int bs, const pkv::DecodeArgs& a, const
   return PA_ERR_INVALID;
 }
 
+// 8-bit (E4M3) caches: plain decode, head_dim 128.
+template <typename T>
+pa_status dispatch_e4m3(int bs, const pkv::DecodeArgs& a, const CUtensorMap& mk,
+                        const CUtensorMap& mv, int grid, cudaStream_t s) {
+  const bool nt1 = a.ncol <= 8;
+  switch (bs) {
+    case 1: return nt1 ? launch_decode<T, 128, 1, 1, pkv::kPlain, true>(a, mk, mv, grid, s)
+                       : launch_decode<T, 128, 1, 2, pkv::kPlain, true>(a, mk, mv, grid, s);
+    case 8: return nt1 ? launch_decode<T, 128, 8, 1, pkv::kPlain, true>(a, mk, mv, grid, s)
+                       : launch_decode<T, 128, 8, 2, pkv::kPlain, true>(a, mk, mv, grid, s);
+    case 16: return nt1 ? launch_decode<T, 128, 16, 1, pkv::kPlain, true>(a, mk, mv, grid, s)
+                        : launch_decode<T, 128, 16, 2, pkv::kPlain, true>(a, mk, mv, grid, s);
+    case 32: return nt1 ? launch_decode<T, 128, 32, 1, pkv::kPlain, true>(a, mk, mv, grid, s)
+                        : launch_decode<T, 128, 32, 2, pkv::kPlain, true>(a, mk, mv, grid, s);
+  }
+  return PA_ERR_UNSUPPORTED;
+}
+
 // Cascade extras of one launch (kPlain: all null).
 struct CascadeArgs {
   int mode = pkv::kPlain;
@@ -174,6 +195,8 @@ struct CascadeArgs {
   float* ext_acc = nullptr;
   const void* k_new = nullptr;   // kAppend
   const void* v_new = nullptr;
+  bool kv8 = false;              // 8-bit E4M3 caches with these scales
+  float k_scale = 1.f, v_scale = 1.f;
 };
 
 // Validation, workspace layout, tensor maps and launch shared by the decode entry points.
@@ -214,11 +237,12 @@ pa_status decode_impl(void* out, const void* q, const void* k_cache, const void*
   CUtensorMap mk, mv;
   std::memset(&mk, 0, sizeof(mk));
   std::memset(&mv, 0, sizeof(mv));
+  if (cx.kv8 && (head_dim != 128 || cx.mode != pkv::kPlain)) return PA_ERR_UNSUPPORTED;
   if (block_size != 1) {
     const uint64_t rows = (uint64_t)num_blocks * num_kv_heads * block_size;
     const int box_rows = block_size < 16 ? block_size : 16;
-    if (!encode_pool(&mk, k_cache, dtype, head_dim, rows, box_rows) ||
-        !encode_pool(&mv, v_cache, dtype, head_dim, rows, box_rows))
+    if (!encode_pool(&mk, k_cache, dtype, head_dim, rows, box_rows, cx.kv8) ||
+        !encode_pool(&mv, v_cache, dtype, head_dim, rows, box_rows, cx.kv8))
       return PA_ERR_CUDA;
   }
   pkv::DecodeArgs a;
@@ -242,7 +266,8 @@ pa_status decode_impl(void* out, const void* q, const void* k_cache, const void*
   a.ctx_cap = max_blocks_per_seq * block_size;
   a.q_len = q_len;
   a.ncol = group * q_len;
-  a.scale_log2 = scale * 1.4426950408889634f;
+  a.scale_log2 = scale * cx.k_scale * 1.4426950408889634f;
+  a.v_scale = cx.v_scale;
   a.epoch = next_epoch();
   a.seq_start = cx.seq_start;
   a.chunk_members = cx.chunk_members;
@@ -252,6 +277,9 @@ pa_status decode_impl(void* out, const void* q, const void* k_cache, const void*
   a.k_new = cx.k_new;
   a.v_new = cx.v_new;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cx.kv8)
+    return dtype == PA_BF16 ? dispatch_e4m3<__nv_bfloat16>(block_size, a, mk, mv, grid, st)
+                            : dispatch_e4m3<__half>(block_size, a, mk, mv, grid, st);
   if (dtype == PA_BF16)
     return dispatch_mode<__nv_bfloat16>(cx.mode, head_dim, block_size, a, mk, mv, grid, st);
   return dispatch_mode<__half>(cx.mode, head_dim, block_size, a, mk, mv, grid, st);
@@ -336,6 +364,63 @@ pa_status pa_decode_append(void* out, const void* q, void* k_cache, void* v_cach
                      num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
                      num_blocks, scale, dtype, workspace, workspace_bytes, 0, dev_status, stream,
                      cx);
+}
+
+pa_status pa_decode_e4m3(void* out, const void* q, const void* k_cache, const void* v_cache,
+                         float k_scale, float v_scale, const int32_t* block_tables,
+                         const int32_t* context_lens, int num_seqs, int num_q_heads,
+                         int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq,
+                         int num_blocks, float scale, pa_dtype dtype, void* workspace,
+                         size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  if (!std::isfinite(k_scale) || !std::isfinite(v_scale) || !(k_scale > 0.f) ||
+      !(v_scale > 0.f))
+    return PA_ERR_INVALID;
+  CascadeArgs cx;
+  cx.kv8 = true;
+  cx.k_scale = k_scale;
+  cx.v_scale = v_scale;
+  return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, 1,
+                     num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                     num_blocks, scale, dtype, workspace, workspace_bytes, 0, dev_status, stream,
+                     cx);
+}
+
+pa_status pa_cache_append_e4m3(void* k_cache, void* v_cache, const void* k, const void* v,
+                               const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
+                               int head_dim, int block_size, int num_blocks, pa_dtype dtype,
+                               float k_scale, float v_scale, int32_t* dev_status, void* stream) {
+  if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
+    return PA_ERR_INVALID;
+  if (!std::isfinite(k_scale) || !std::isfinite(v_scale) || !(k_scale > 0.f) || !(v_scale > 0.f))
+    return PA_ERR_INVALID;
+  if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  if (head_dim % 16) return PA_ERR_UNSUPPORTED;
+  if (num_tokens == 0) return PA_OK;
+  if (!k_cache || !v_cache || !k || !v || !slot_mapping) return PA_ERR_INVALID;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k) || !aligned16(v))
+    return PA_ERR_INVALID;
+  const int cpr = head_dim / 16;
+  const long long total = (long long)num_tokens * num_kv_heads * cpr;
+  const int sms = sm_count();
+  if (sms <= 0) return PA_ERR_CUDA;
+  long long blocks = (total + 255) / 256;
+  if (blocks > (long long)sms * 16) blocks = (long long)sms * 16;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (dtype == PA_BF16)
+    e = launch(pkv::pa_cache_append_e4m3_kernel<__nv_bfloat16>, dim3((unsigned)blocks), dim3(256),
+               0, st, static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
+               static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping,
+               num_tokens, num_kv_heads, cpr, block_size, num_blocks, k_scale, v_scale,
+               dev_status);
+  else
+    e = launch(pkv::pa_cache_append_e4m3_kernel<__half>, dim3((unsigned)blocks), dim3(256), 0, st,
+               static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
+               static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping,
+               num_tokens, num_kv_heads, cpr, block_size, num_blocks, k_scale, v_scale,
+               dev_status);
+  if (e != cudaSuccess) return PA_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 size_t pa_decode_cascade_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads,

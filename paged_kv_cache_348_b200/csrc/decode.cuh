@@ -115,13 +115,19 @@ struct DecodeArgs {
   // kAppend: K/V of each sequence's newest token, [seqs][Hkv][D]
   const void* k_new;
   const void* v_new;
+  float v_scale;                // 8-bit caches: value = v_scale * code (1 otherwise); the
+                                // K scale is folded into scale_log2
 };
 
 
-template <int D>
+// Shared-memory layout of a CTA.  16-bit caches: K and V tiles of 64 tokens in D/64
+// column halves of 128-byte lines; 8-bit (E4M3) caches: one line of D bytes per token
+// (D = 128), and a deeper ring since a stage is half the size.
+template <int D, bool KV8 = false>
 struct Layout {
+  static constexpr int kStages = KV8 ? 5 : 3;
   static constexpr int kHalves = D / 64;                   // 128-byte swizzled column halves
-  static constexpr int kKvBytes = kHalves * kTileTokens * 128;
+  static constexpr int kKvBytes = KV8 ? kTileTokens * D : kHalves * kTileTokens * 128;
   static constexpr int kQBytes = kMaxGroup * D * 2;
   static constexpr int kStageBytes = 2 * kKvBytes + kQBytes;
   static_assert(kStageBytes % 1024 == 0, "stage must keep 1024-byte alignment");
@@ -134,7 +140,7 @@ struct Layout {
   static constexpr int kMlOff = kDescOff + 2 * (int)sizeof(SplitDesc);
   // fused append: per stage the new token's K and V rows, staged by the producer
   static constexpr int kNewOff = (kMlOff + kConsumerWarps * kMaxGroup * 8 + 15) / 16 * 16;
-  static constexpr int kNewBytes = 2 * D * 2;
+  static constexpr int kNewBytes = KV8 ? 16 : 2 * D * 2;
   static constexpr int kBytes = kNewOff + kStages * kNewBytes;
   static constexpr int kDynSmem = kBytes + 1024;           // slack for 1024-byte alignment
   static_assert(kBarOff % 8 == 0 && kMiscOff % 8 == 0 && kDescOff % 8 == 0 && kMlOff % 8 == 0 &&
@@ -264,7 +270,7 @@ __device__ __forceinline__ void finish_row(const DecodeArgs& a, long long row, f
       }
     }
     T* o = static_cast<T*>(a.out) + row * D + d0;
-    const float inv = L > 0.f ? 1.f / L : 0.f;
+    const float inv = L > 0.f ? a.v_scale / L : 0.f;
     if (n == 4) {
       *reinterpret_cast<uint2*>(o) = make_uint2(pack2<T>(acc[0] * inv, acc[1] * inv),
                                                 pack2<T>(acc[2] * inv, acc[3] * inv));
@@ -307,6 +313,15 @@ __device__ __forceinline__ void empty_rows(const DecodeArgs& a, int s, int first
     uint4* row = reinterpret_cast<uint4*>(static_cast<T*>(a.out) + (long long)s * a.q_len * Hq * D);
     for (int i = lane; i < a.q_len * Hq * D * 2 / 16; i += 32) row[i] = make_uint4(0, 0, 0, 0);
   }
+}
+
+// Two E4M3 codes (low byte first) to two fp16 values, exactly.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t x16) {
+  uint32_t y;
+  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}"
+      : "=r"(y)
+      : "r"(x16));
+  return y;
 }
 
 // Entry i (0 <= i < 96) of a block-table window held across the warp: lane l holds
@@ -415,12 +430,15 @@ __device__ __forceinline__ void merge_split(const DecodeArgs& a, const SplitDesc
   }
 }
 
-template <typename T, int D, int BS, int NT, int MODE>
+template <typename T, int D, int BS, int NT, int MODE, bool KV8 = false>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     pa_decode_split_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
                            const __grid_constant__ CUtensorMap tmv) {
-  using L = Layout<D>;
-  constexpr bool kBF16 = std::is_same_v<T, __nv_bfloat16>;
+  using L = Layout<D, KV8>;
+  constexpr int kStages = L::kStages;
+  static_assert(!KV8 || (D == 128 && MODE == kPlain), "8-bit caches: head_dim 128, plain decode");
+  // MMA operand type: the cache's 16-bit type, or fp16 for E4M3 (exact there)
+  constexpr bool kBF16 = !KV8 && std::is_same_v<T, __nv_bfloat16>;
   constexpr int kFullCount = (BS == 1) ? 33 : 1;
   constexpr int kConsumerThreads = 32 * kConsumerWarps;
   extern __shared__ uint8_t smem_raw[];
@@ -641,13 +659,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           if constexpr (BS != 1) {
             constexpr int H = BS < 16 ? BS : 16;     // rows per TMA box
             constexpr int BPU = kUnit / H;           // boxes per unit and column half
-            constexpr int kBoxBytes = H * 128;
-            static_assert(kUnitsPerStage * BPU * L::kHalves * 2 <= 32, "one box per lane");
+            constexpr int kParts = KV8 ? 1 : L::kHalves;   // boxes per row of a token
+            constexpr int kBoxBytes = H * 128;       // D = 128 8-bit values or 64 16-bit
+            static_assert(kUnitsPerStage * BPU * kParts * 2 <= 32, "one box per lane");
             // this lane's box and its block-table entry, read before the slot wait
-            const int nbox = nun * BPU * L::kHalves * 2;
+            const int nbox = nun * BPU * kParts * 2;
             const int kv = lane & 1;
-            const int hf = (lane >> 1) % L::kHalves;
-            const int jb = (lane >> 1) / L::kHalves;
+            const int hf = (lane >> 1) % kParts;
+            const int jb = (lane >> 1) / kParts;
             const int j = jb / BPU, b = jb % BPU;
             const int t = tok0 + j * kUnit + b * H;
             const bool mine = lane < nbox && t < ctx_cur;
@@ -672,7 +691,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             for (int jj = 0; jj < nun; ++jj) {
               const int rem = ctx_cur - (tok0 + jj * kUnit);
               const int nb = (rem + H - 1) / H;
-              bytes += (uint32_t)((nb < BPU ? nb : BPU) * kBoxBytes * L::kHalves * 2);
+              bytes += (uint32_t)((nb < BPU ? nb : BPU) * kBoxBytes * kParts * 2);
             }
             if (!mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, kWaitLimitNs)) {
               ok = false;
@@ -692,13 +711,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             __syncwarp();
             if (mine) {
               uint8_t* dst = (kv ? sV : sK) + hf * (kTileTokens * 128) + (j * kUnit + b * H) * 128;
-              tma_load_2d(dst, kv ? &tmv : &tmk, &full[st], hf * 64, y, policy);
+              tma_load_2d(dst, kv ? &tmv : &tmk, &full[st], KV8 ? 0 : hf * 64, y, policy);
             }
           } else {
             // block_size 1: every token is its own block; 16-byte cp.async with the same
             // 128-byte swizzle the TMA path produces.  Stages are 64 tokens, so the window
             // (w0, w1) holds exactly this stage's table entries, handed out by shuffle.
-            constexpr int CPR = D * 2 / 16;          // 16-byte chunks per row
+            constexpr int CPR = D * (KV8 ? 1 : 2) / 16;   // 16-byte chunks per row
             constexpr int RPI = 32 / CPR;            // rows per warp instruction
             const int ntok = nun * kUnit;
             if (!mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, kWaitLimitNs)) {
@@ -730,10 +749,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                   if (a.status) atomicOr(a.status, DEV_BAD_BLOCK_ID);
                   sz = 0;                                // zero fill, no read
                 }
-                const long long off = row * D + ch * 8;
+                const long long off = (row * D + ch * 8) * 2;   // bytes; 8-bit: row * D + ch * 16
                 const int soff = hf * (kTileTokens * 128) + r * 128 + ((cc ^ (r & 7)) << 4);
-                cp_async_16_zfill(sK + soff, static_cast<const T*>(a.k_cache) + off, sz, policy);
-                cp_async_16_zfill(sV + soff, static_cast<const T*>(a.v_cache) + off, sz, policy);
+                const long long boff = KV8 ? row * D + ch * 16 : off;
+                cp_async_16_zfill(sK + soff, static_cast<const uint8_t*>(a.k_cache) + boff, sz, policy);
+                cp_async_16_zfill(sV + soff, static_cast<const uint8_t*>(a.v_cache) + boff, sz, policy);
               }
             }
             cp_async_mbar_arrive_noinc(&full[st]);
@@ -814,8 +834,19 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           uint32_t b0 = 0u, b1 = 0u;
           if (cq < a.ncol) {
             const uint32_t* qrow = reinterpret_cast<const uint32_t*>(sQ + cq * D * 2);
-            b0 = qrow[(ks * 16 + 2 * tig) >> 1];
-            b1 = qrow[(ks * 16 + 8 + 2 * tig) >> 1];
+            if constexpr (KV8) {
+              // k-step ks pairs with the 16 cache bytes of dims 16ks..16ks+15 as the
+              // converted fragments order them: logical k (2c, 2c+1) is dims (4c, 4c+1),
+              // logical k (2c+8, 2c+9) is dims (4c+2, 4c+3); q converted to fp16
+              const uint32_t u0 = qrow[(ks * 16 + 4 * tig) >> 1];
+              const uint32_t u1 = qrow[(ks * 16 + 4 * tig + 2) >> 1];
+              const float2 f0 = unpack2<T>(u0), f1 = unpack2<T>(u1);
+              b0 = pack2<__half>(f0.x, f0.y);
+              b1 = pack2<__half>(f1.x, f1.y);
+            } else {
+              b0 = qrow[(ks * 16 + 2 * tig) >> 1];
+              b1 = qrow[(ks * 16 + 8 + 2 * tig) >> 1];
+            }
           }
           qf[ks][n][0] = b0;
           qf[ks][n][1] = b1;
@@ -856,7 +887,28 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       float sacc[NT][4];
 #pragma unroll
       for (int n = 0; n < NT; ++n) sacc[n][0] = sacc[n][1] = sacc[n][2] = sacc[n][3] = 0.f;
-      {
+      if constexpr (KV8) {
+        // one ldmatrix.x4 = rows 0-7 / 8-15 of two 16-byte chunks (k-steps ks, ks+1); a
+        // thread's 32 bits are 4 codes, dims 4c..4c+3 of its row, converted in two halves
+        const int j = lane >> 3, i = lane & 7;
+        const int r = cw * kUnit + (j & 1) * 8 + i;
+#pragma unroll
+        for (int ks = 0; ks < KS; ks += 2) {
+          const int chunk = ks + (j >> 1);
+          const uint32_t addr = kbase + r * 128 + ((chunk ^ (r & 7)) << 4);
+          uint32_t m0, m1, m2, m3;
+          ldsm_x4(addr, m0, m1, m2, m3);
+          const uint32_t x0 = e4m3x2_to_f16x2(m0 & 0xffffu), x2 = e4m3x2_to_f16x2(m0 >> 16);
+          const uint32_t x1 = e4m3x2_to_f16x2(m1 & 0xffffu), x3 = e4m3x2_to_f16x2(m1 >> 16);
+          const uint32_t y0 = e4m3x2_to_f16x2(m2 & 0xffffu), y2 = e4m3x2_to_f16x2(m2 >> 16);
+          const uint32_t y1 = e4m3x2_to_f16x2(m3 & 0xffffu), y3 = e4m3x2_to_f16x2(m3 >> 16);
+#pragma unroll
+          for (int n = 0; n < NT; ++n) {
+            mma16816<false>(sacc[n], x0, x1, x2, x3, qf[ks][n][0], qf[ks][n][1]);
+            mma16816<false>(sacc[n], y0, y1, y2, y3, qf[ks + 1][n][0], qf[ks + 1][n][1]);
+          }
+        }
+      } else {
         const int j = lane >> 3, i = lane & 7;
         const int r = cw * kUnit + (j & 1) * 8 + i;
 #pragma unroll
@@ -904,14 +956,20 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           o[ks][n][2] *= alpha[0];
           o[ks][n][3] *= alpha[1];
         }
-        const uint32_t h01 = pack2<T>(p[0], p[1]), h23 = pack2<T>(p[2], p[3]);
-        const float2 f01 = unpack2<T>(h01), f23 = unpack2<T>(h23);
-        const uint32_t l01 = pack2<T>(p[0] - f01.x, p[1] - f01.y);
-        const uint32_t l23 = pack2<T>(p[2] - f23.x, p[3] - f23.y);
+        using TM = std::conditional_t<KV8, __half, T>;   // MMA operand type
+        const uint32_t h01 = pack2<TM>(p[0], p[1]), h23 = pack2<TM>(p[2], p[3]);
         bhi[n][0] = movmatrix_t(h01);
         bhi[n][1] = movmatrix_t(h23);
-        blo[n][0] = movmatrix_t(l01);
-        blo[n][1] = movmatrix_t(l23);
+        if constexpr (!KV8) {
+          // the rounding residual of P as a second 16-bit operand (~16 bits of P in all)
+          const float2 f01 = unpack2<TM>(h01), f23 = unpack2<TM>(h23);
+          const uint32_t l01 = pack2<TM>(p[0] - f01.x, p[1] - f01.y);
+          const uint32_t l23 = pack2<TM>(p[2] - f23.x, p[3] - f23.y);
+          blo[n][0] = movmatrix_t(l01);
+          blo[n][1] = movmatrix_t(l23);
+        } else {
+          blo[n][0] = blo[n][1] = 0u;   // fp16 P: 11 bits, next to 3-bit cache values
+        }
       }
       // ---- O^T[D][8*NT] += V_unit^T . P^T
       uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;   // token masks for V rows >= valid
@@ -920,7 +978,32 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         mlo = (t_a < valid ? 0x0000ffffu : 0u) | (t_a + 1 < valid ? 0xffff0000u : 0u);
         mhi = (t_b < valid ? 0x0000ffffu : 0u) | (t_b + 1 < valid ? 0xffff0000u : 0u);
       }
-      {
+      if constexpr (KV8) {
+        // ldmatrix.x4.trans of tokens 0-7 / 8-15 of two 16-byte chunks; a thread gets the
+        // codes of dims (2g, 2g+1) for tokens (2c, 2c+1): regrouped per dim they give the
+        // A fragments with M-row g = dim 2g and M-row g+8 = dim 2g+1 of the chunk
+        const int j = lane >> 3, i = lane & 7;
+        const int r = cw * kUnit + (j & 1) * 8 + i;
+#pragma unroll
+        for (int mtile = 0; mtile < KS; mtile += 2) {
+          const int chunk = mtile + (j >> 1);
+          const uint32_t addr = vbase + r * 128 + ((chunk ^ (r & 7)) << 4);
+          uint32_t m[4];
+          ldsm_x4_t(addr, m[0], m[1], m[2], m[3]);
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const uint32_t p0 = __byte_perm(m[2 * hh], 0u, 0x3120);       // tokens 2c, 2c+1
+            const uint32_t p1 = __byte_perm(m[2 * hh + 1], 0u, 0x3120);   // tokens 8+2c, ...
+            const uint32_t a0 = e4m3x2_to_f16x2(p0 & 0xffffu) & mlo;
+            const uint32_t a1 = e4m3x2_to_f16x2(p0 >> 16) & mlo;
+            const uint32_t a2 = e4m3x2_to_f16x2(p1 & 0xffffu) & mhi;
+            const uint32_t a3 = e4m3x2_to_f16x2(p1 >> 16) & mhi;
+#pragma unroll
+            for (int n = 0; n < NT; ++n)
+              mma16816<false>(o[mtile + hh][n], a0, a1, a2, a3, bhi[n][0], bhi[n][1]);
+          }
+        }
+      } else {
         const int j = lane >> 3, i = lane & 7;
         const int r = cw * kUnit + (j >> 1) * 8 + i;
 #pragma unroll
@@ -1007,7 +1090,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 #pragma unroll
       for (int it = 0; it < kIt; ++it) {            // the prefix partials, all loads at once
         const int n = it % NT, ks = it / NT;
-        const int d = ks * 16 + (lane >> 2) + (cw >= 2 ? 8 : 0);
+        const int d = ks * 16 + (KV8 ? 2 * (lane >> 2) + (cw >= 2 ? 1 : 0)
+                                     : (lane >> 2) + (cw >= 2 ? 8 : 0));
         xv[it] = (MODE == kSuffix && has_prefix && crow[n] >= 0) ? __ldcg(a.ext_acc + crow[n] * D + d)
                                                                   : 0.f;
       }
@@ -1016,7 +1100,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         const int n = it % NT, ks = it / NT;
         const int h = n * 8 + 2 * (lane & 3) + (cw & 1);   // query column
         if (h >= a.ncol) continue;
-        const int d = ks * 16 + (lane >> 2) + (cw >= 2 ? 8 : 0);
+        // head dim of this accumulator value (8-bit caches order the PV rows 2g, 2g+1)
+        const int d = ks * 16 + (KV8 ? 2 * (lane >> 2) + (cw >= 2 ? 1 : 0)
+                                     : (lane >> 2) + (cw >= 2 ? 8 : 0));
         const int r = cw + 4 * it;                   // scr register row of this value
         float acc = 0.f;
 #pragma unroll

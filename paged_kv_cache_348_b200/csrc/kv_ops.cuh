@@ -2,7 +2,11 @@
 // Both are pure byte movement: 16-byte vector loads/stores, consecutive threads on
 // consecutive 16-byte chunks of a row so every warp access is coalesced.
 #pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
 #include <cstdint>
+#include <type_traits>
 
 #include "ptx.cuh"
 
@@ -41,6 +45,74 @@ __global__ void __launch_bounds__(256)
     const long long dst = ((b * Hkv + h) * block_size + off) * chunks_per_row + ch;
     k_cache[dst] = k[i];
     v_cache[dst] = v[i];
+  }
+}
+
+// Two binary32 values to two E4M3 codes (x0 in the low byte): round to nearest even,
+// magnitudes above 448 clamped to 448.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float x0, float x1) {
+  uint32_t d;
+  asm("{\n\t.reg .b16 t;\n\tcvt.rn.satfinite.e4m3x2.f32 t, %2, %1;\n\tcvt.u32.u16 %0, t;\n\t}"
+      : "=r"(d)
+      : "f"(x0), "f"(x1));
+  return d;
+}
+
+// The append into 8-bit E4M3 caches: as pa_cache_append_kernel, each value quantised as
+// x / scale (binary32, IEEE division) rounded to E4M3.  One thread per 16 values: two
+// 16-byte loads of 16-bit input, one 16-byte store of codes.
+template <typename T>
+__global__ void __launch_bounds__(256)
+    pa_cache_append_e4m3_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
+                                const uint4* __restrict__ k, const uint4* __restrict__ v,
+                                const int64_t* __restrict__ slot_mapping, int num_tokens,
+                                int Hkv, int chunks_per_row, int block_size, int num_blocks,
+                                float k_scale, float v_scale, int32_t* status) {
+  pdl_wait();
+  pdl_trigger();
+  const long long total = (long long)num_tokens * Hkv * chunks_per_row;
+  const long long limit = (long long)num_blocks * block_size;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int ch = (int)(i % chunks_per_row);    // 16 values
+    const long long rh = i / chunks_per_row;
+    const int h = (int)(rh % Hkv);
+    const long long tok = rh / Hkv;
+    const long long slot = slot_mapping[tok];
+    if (slot < 0) continue;
+    if (slot >= limit) {
+      if (status && ch == 0) atomicOr(status, DEV_BAD_SLOT);
+      continue;
+    }
+    const long long b = slot / block_size, off = slot % block_size;
+    const long long dst = ((b * Hkv + h) * block_size + off) * chunks_per_row + ch;
+    for (int kv = 0; kv < 2; ++kv) {
+      const uint4* src = (kv ? v : k) + 2 * i;
+      const float sc = kv ? v_scale : k_scale;
+      const uint4 in[2] = {src[0], src[1]};
+      const uint32_t* w = reinterpret_cast<const uint32_t*>(in);
+      uint32_t q[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float f[4];
+        for (int u = 0; u < 2; ++u) {
+          uint32_t x = w[2 * e + u];
+          float lo, hi;
+          if constexpr (std::is_same_v<T, __nv_bfloat16>) {
+            lo = __uint_as_float(x << 16);
+            hi = __uint_as_float(x & 0xffff0000u);
+          } else {
+            const __half2 hx = *reinterpret_cast<const __half2*>(&x);
+            const float2 fx = __half22float2(hx);
+            lo = fx.x, hi = fx.y;
+          }
+          f[2 * u] = __fdiv_rn(lo, sc);
+          f[2 * u + 1] = __fdiv_rn(hi, sc);
+        }
+        q[e] = f32x2_to_e4m3x2(f[0], f[1]) | (f32x2_to_e4m3x2(f[2], f[3]) << 16);
+      }
+      (kv ? v_cache : k_cache)[dst] = make_uint4(q[0], q[1], q[2], q[3]);
+    }
   }
 }
 

@@ -106,6 +106,20 @@ def randn(shape, dtype: str, seed: int, device="cpu", stream: int = 0):
     return x.to(torch.bfloat16 if dtype == "bf16" else torch.float16)
 
 
+def randn_e4m3(shape, scale: float, seed: int, device="cpu", stream: int = 0):
+    """Random 8-bit E4M3 cache codes whose values (scale * code) follow N(0, 1): N(0, 1)
+    draws divided by `scale` and rounded to the nearest E4M3 code with torch's own
+    float8_e4m3fn type, as uint8.  (Input data only: the library quantises with its own
+    kernel.)"""
+    import torch
+
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed) * 1_000_003 + int(stream))
+    x = torch.randn(tuple(shape), generator=g, device=device, dtype=torch.float32) / scale
+    x = x.clamp(-448.0, 448.0)
+    return x.to(torch.float8_e4m3fn).view(torch.uint8)
+
+
 def torch_dtype(dtype: str):
     import torch
 

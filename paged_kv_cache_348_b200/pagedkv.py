@@ -24,7 +24,8 @@ DEV_BAD_BLOCK_ID, DEV_BAD_SLOT, DEV_BAD_PAIR, DEV_BAD_CONTEXT_LEN, DEV_TIMEOUT =
 
 # every symbol include/pagedkv.h declares
 EXPORTS = ("pa_version", "pa_status_string", "pa_decode_workspace_bytes", "pa_decode",
-           "pa_decode_multi", "pa_decode_append", "pa_decode_cascade_workspace_bytes",
+           "pa_decode_multi", "pa_decode_append", "pa_cache_append_e4m3", "pa_decode_e4m3",
+           "pa_decode_cascade_workspace_bytes",
            "pa_decode_cascade",
            "pa_cache_append", "pa_copy_blocks", "pa_decode_noalloc",
            "pa_bm_create", "pa_bm_destroy", "pa_bm_free_blocks", "pa_bm_refcount",
@@ -66,6 +67,12 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         L.pa_decode_append.restype = i32
         L.pa_decode_append.argtypes = [P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32,
                                        f32, i32, P, sz, P, P]
+        L.pa_cache_append_e4m3.restype = i32
+        L.pa_cache_append_e4m3.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, f32,
+                                           P, P]
+        L.pa_decode_e4m3.restype = i32
+        L.pa_decode_e4m3.argtypes = [P, P, P, P, f32, f32, P, P, i32, i32, i32, i32, i32, i32, i32,
+                                     f32, i32, P, sz, P, P]
         L.pa_decode_cascade_workspace_bytes.restype = sz
         L.pa_decode_cascade_workspace_bytes.argtypes = [i32, i32, i32, i32]
         L.pa_decode_cascade.restype = i32
@@ -207,6 +214,50 @@ def pa_decode_append(out, q, k_cache, v_cache, k_new, v_new, block_tables, conte
                                  _ptr(workspace), workspace.numel() * workspace.element_size(),
                                  _ptr(status), _stream(stream))
     _check(rc, "pa_decode_append")
+    return out
+
+
+def pa_cache_append_e4m3(k_cache8, v_cache8, k, v, slot_mapping, k_scale: float, v_scale: float,
+                         status=None, stream=None):
+    """Quantising scatter of 16-bit k/v [T,Hkv,D] into uint8 E4M3 pools (see
+    pa_cache_append_e4m3 in include/pagedkv.h)."""
+    _need(k_cache8, "k_cache", dtype=torch.uint8, ndim=4)
+    _need(v_cache8, "v_cache", dtype=torch.uint8, ndim=4)
+    _need(k, "k", ndim=3)
+    _need(v, "v", dtype=k.dtype, ndim=3)
+    _need(slot_mapping, "slot_mapping", dtype=torch.int64, ndim=1)
+    N, Hkv, bs, D = k_cache8.shape
+    T = k.shape[0]
+    if v_cache8.shape != k_cache8.shape or k.shape != (T, Hkv, D) or v.shape != k.shape or \
+            slot_mapping.shape[0] != T:
+        raise PagedKVError("pa_cache_append_e4m3: inconsistent shapes")
+    rc = load().pa_cache_append_e4m3(_ptr(k_cache8), _ptr(v_cache8), _ptr(k), _ptr(v),
+                                     _ptr(slot_mapping), T, Hkv, D, bs, N, _dtype_code(k),
+                                     float(k_scale), float(v_scale), _ptr(status), _stream(stream))
+    _check(rc, "pa_cache_append_e4m3")
+
+
+def pa_decode_e4m3(out, q, k_cache8, v_cache8, k_scale: float, v_scale: float, block_tables,
+                   context_lens, scale: float, workspace, status=None, stream=None):
+    """out[B,Hq,D] <- paged decode over uint8 E4M3 pools (see pa_decode_e4m3)."""
+    _need(q, "q", ndim=3)
+    _need(out, "out", dtype=q.dtype, ndim=3)
+    _need(k_cache8, "k_cache", dtype=torch.uint8, ndim=4)
+    _need(v_cache8, "v_cache", dtype=torch.uint8, ndim=4)
+    _need(block_tables, "block_tables", dtype=torch.int32, ndim=2)
+    _need(context_lens, "context_lens", dtype=torch.int32, ndim=1)
+    _need(workspace, "workspace")
+    B, Hq, D = q.shape
+    N, Hkv, bs, D2 = k_cache8.shape
+    if out.shape != q.shape or D2 != D or v_cache8.shape != k_cache8.shape or \
+            block_tables.shape[0] != B or context_lens.shape[0] != B:
+        raise PagedKVError("pa_decode_e4m3: inconsistent shapes")
+    rc = load().pa_decode_e4m3(_ptr(out), _ptr(q), _ptr(k_cache8), _ptr(v_cache8), float(k_scale),
+                               float(v_scale), _ptr(block_tables), _ptr(context_lens), B, Hq, Hkv,
+                               D, bs, block_tables.shape[1], N, float(scale), _dtype_code(q),
+                               _ptr(workspace), workspace.numel() * workspace.element_size(),
+                               _ptr(status), _stream(stream))
+    _check(rc, "pa_decode_e4m3")
     return out
 
 

@@ -45,6 +45,7 @@ class DecodeBatch:
     scale: float
     q_len: int = 1
     cascade: tuple | None = None     # (prefix_lens, chunk_members, chunk_prefix_lens) on device
+    kv_scales: tuple | None = None   # (k_scale, v_scale) of 8-bit E4M3 pools, else None
 
     @property
     def layers(self) -> int:
@@ -55,7 +56,8 @@ class DecodeBatch:
         sequence, K and V, all kv heads, all layers."""
         w = self.w
         ctx = self.context_lens.cpu().numpy().astype(np.int64)
-        return int(ctx.sum()) * w.num_kv_heads * w.head_dim * 2 * 2 * self.layers
+        elem = self.k_caches[0].element_size()
+        return int(ctx.sum()) * w.num_kv_heads * w.head_dim * 2 * elem * self.layers
 
     def unique_kv_bytes_per_step(self) -> int:
         """KV bytes with every shared block counted once (blocks x fill)."""
@@ -65,26 +67,34 @@ class DecodeBatch:
             for i, b in enumerate(self.bm.table(s)):
                 seen[b] = max(seen.get(b, 0), min(self.block_size, n - i * self.block_size))
         w = self.w
-        return sum(seen.values()) * w.num_kv_heads * w.head_dim * 2 * 2 * self.layers
+        elem = self.k_caches[0].element_size()
+        return sum(seen.values()) * w.num_kv_heads * w.head_dim * 2 * elem * self.layers
 
 
 def _pool_size(w: inputs.Workload, need: int) -> int:
     return w.pool_blocks if w.pool_blocks else int(math.ceil(w.pool_factor * need))
 
 
-def _alloc_layers(w, N, bs, layers, device, seed):
+KV8_SCALE = 1.0 / 64.0               # per-tensor scale of the synthetic 8-bit pools
+
+
+def _alloc_layers(w, N, bs, layers, device, seed, kv8=False):
     k, v = [], []
+    shape = (N, w.num_kv_heads, bs, w.head_dim)
     for l in range(layers):
-        k.append(inputs.randn((N, w.num_kv_heads, bs, w.head_dim), w.dtype, seed, device,
-                              stream=1000 + 2 * l))
-        v.append(inputs.randn((N, w.num_kv_heads, bs, w.head_dim), w.dtype, seed, device,
-                              stream=1001 + 2 * l))
+        if kv8:
+            k.append(inputs.randn_e4m3(shape, KV8_SCALE, seed, device, stream=1000 + 2 * l))
+            v.append(inputs.randn_e4m3(shape, KV8_SCALE, seed, device, stream=1001 + 2 * l))
+        else:
+            k.append(inputs.randn(shape, w.dtype, seed, device, stream=1000 + 2 * l))
+            v.append(inputs.randn(shape, w.dtype, seed, device, stream=1001 + 2 * l))
     return k, v
 
 
-def _finish(w, bs, bm, sids, N, layers, device, cow_pairs=None, q_len=1) -> DecodeBatch:
+def _finish(w, bs, bm, sids, N, layers, device, cow_pairs=None, q_len=1,
+            kv8=False) -> DecodeBatch:
     B = len(sids)
-    k_caches, v_caches = _alloc_layers(w, N, bs, layers, device, w.seed)
+    k_caches, v_caches = _alloc_layers(w, N, bs, layers, device, w.seed, kv8)
     tables = torch.from_numpy(bm.block_tables(sids)).to(device)
     ctx = torch.from_numpy(bm.context_lens(sids)).to(device)
     # the newest q_len tokens of every sequence are the ones appended and queried
@@ -106,11 +116,12 @@ def _finish(w, bs, bm, sids, N, layers, device, cow_pairs=None, q_len=1) -> Deco
     if cow_pairs:
         pairs = torch.tensor(cow_pairs, dtype=torch.int32, device=device).reshape(-1, 2)
     return DecodeBatch(w, bs, bm, sids, N, k_caches, v_caches, tables, ctx, slots, q, kn, vn, out,
-                       ws, st, pairs, 1.0 / math.sqrt(w.head_dim), q_len)
+                       ws, st, pairs, 1.0 / math.sqrt(w.head_dim), q_len,
+                       kv_scales=(KV8_SCALE, KV8_SCALE) if kv8 else None)
 
 
 def build(w: inputs.Workload, device="cuda", block_size: int | None = None,
-          layers: int | None = None, q_len: int = 1) -> DecodeBatch:
+          layers: int | None = None, q_len: int = 1, kv8: bool = False) -> DecodeBatch:
     """Independent sequences (every workload but the shared-prefix one).  With q_len > 1
     every sequence's newest q_len tokens are appended and queried each step."""
     bs = block_size or w.block_size
@@ -119,7 +130,7 @@ def build(w: inputs.Workload, device="cuda", block_size: int | None = None,
     N = _pool_size(w, need)
     bm = BlockManager(N, bs, inputs.pool_order(N, w.seed))
     sids = [bm.allocate(int(c)) for c in ctx]
-    return _finish(w, bs, bm, sids, N, layers or w.layers, device, q_len=q_len)
+    return _finish(w, bs, bm, sids, N, layers or w.layers, device, q_len=q_len, kv8=kv8)
 
 
 def build_prefix_decode(w: inputs.Workload = inputs.PREFIX, device="cuda") -> DecodeBatch:
@@ -171,11 +182,15 @@ def run_step(b: DecodeBatch, stream=None, layers=None, fused: bool = False) -> N
     if b.cow_pairs is not None and b.cow_pairs.shape[0]:
         pk.pa_copy_blocks(b.k_caches, b.v_caches, b.cow_pairs, b.status, stream)
     for l in range(layers if layers is not None else b.layers):
-        if fused:
+        if fused and b.kv_scales is None:
             append_decode_layer(b, l, stream)
             continue
-        pk.pa_cache_append(b.k_caches[l], b.v_caches[l], b.k_new[l], b.v_new[l], b.slot_mapping,
-                           b.status, stream)
+        if b.kv_scales is not None:
+            pk.pa_cache_append_e4m3(b.k_caches[l], b.v_caches[l], b.k_new[l], b.v_new[l],
+                                    b.slot_mapping, *b.kv_scales, b.status, stream)
+        else:
+            pk.pa_cache_append(b.k_caches[l], b.v_caches[l], b.k_new[l], b.v_new[l],
+                               b.slot_mapping, b.status, stream)
         decode_layer(b, l, stream)
 
 
@@ -210,6 +225,10 @@ def decode_layer(b: DecodeBatch, l: int, stream=None) -> None:
     if b.cascade is not None:
         pk.pa_decode_cascade(b.out[l], b.q[l], b.k_caches[l], b.v_caches[l], b.block_tables,
                              b.context_lens, *b.cascade, b.scale, b.workspace, b.status, stream)
+        return
+    if b.kv_scales is not None:
+        pk.pa_decode_e4m3(b.out[l], b.q[l], b.k_caches[l], b.v_caches[l], *b.kv_scales,
+                          b.block_tables, b.context_lens, b.scale, b.workspace, b.status, stream)
         return
     fn = pk.pa_decode if b.q_len == 1 else pk.pa_decode_multi
     fn(b.out[l], b.q[l], b.k_caches[l], b.v_caches[l], b.block_tables, b.context_lens, b.scale,
