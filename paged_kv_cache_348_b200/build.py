@@ -36,14 +36,40 @@ def _stale() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False, extra=()) -> str:
+    """Compile every source to an object in parallel (the decode kernel instances are
+    spread over several translation units), then link libpagedkv.so."""
     if not force and not _stale():
         return LIB
-    tmp = LIB + ".tmp%d" % os.getpid()
-    cmd = [NVCC, *FLAGS, *extra, "-o", tmp, *sources()]
-    if verbose:
-        print(" ".join(cmd), flush=True)
-    subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
+    import concurrent.futures
+    import tempfile
+
+    compile_flags = [f for f in FLAGS if f != "-shared"]
+    with tempfile.TemporaryDirectory(prefix="pagedkv_build_") as tmpdir:
+        def compile_one(src):
+            obj = os.path.join(tmpdir, os.path.basename(src) + ".o")
+            cmd = [NVCC, *compile_flags, *extra, "-c", "-o", obj, src]
+            r = subprocess.run(cmd, capture_output=True, text=True)
+            return src, obj, cmd, r
+        srcs = sources()
+        workers = max(1, min(len(srcs), os.cpu_count() or 1))
+        with concurrent.futures.ThreadPoolExecutor(workers) as ex:
+            results = list(ex.map(compile_one, srcs))
+        for src, obj, cmd, r in results:
+            if verbose:
+                print(" ".join(cmd), flush=True)
+                sys.stdout.write(r.stdout)
+                sys.stderr.write(r.stderr)
+            if r.returncode != 0:
+                if not verbose:
+                    sys.stderr.write(r.stderr)
+                raise subprocess.CalledProcessError(r.returncode, cmd)
+        tmp = LIB + ".tmp%d" % os.getpid()
+        link = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp,
+                *[obj for _, obj, _, _ in results]]
+        if verbose:
+            print(" ".join(link), flush=True)
+        subprocess.check_call(link)
+        os.replace(tmp, LIB)
     return LIB
 
 

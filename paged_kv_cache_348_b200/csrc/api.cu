@@ -14,6 +14,7 @@
 
 #include "decode.cuh"
 #include "kv_ops.cuh"
+#include "launch.cuh"
 #include "pagedkv.h"
 
 namespace {
@@ -89,100 +90,18 @@ uint32_t next_epoch() {
   return e;
 }
 
-// Programmatic dependent launch lets a kernel's launch and prologue overlap the tail of
-// the kernel before it in the stream (PAGEDKV_NO_PDL=1 turns it off).
-bool use_pdl() {
-  static const bool on = [] {
-    const char* v = std::getenv("PAGEDKV_NO_PDL");
-    return !(v && v[0] && v[0] != '0');
-  }();
-  return on;
-}
-
-template <typename Kernel, typename... Args>
-cudaError_t launch(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
-                   Args... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = use_pdl() ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kernel, args...);
-}
-
-template <typename T, int D, int BS, int NT, int MODE, bool KV8 = false>
-pa_status launch_decode(const pkv::DecodeArgs& a, const CUtensorMap& mk, const CUtensorMap& mv,
-                        int grid, cudaStream_t stream) {
-  using L = pkv::Layout<D, KV8>;
-  auto split = pkv::pa_decode_split_kernel<T, D, BS, NT, MODE, KV8>;
-  if (cudaFuncSetAttribute(split, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynSmem) !=
-      cudaSuccess)
-    return PA_ERR_CUDA;
-  if (launch(split, dim3(grid), dim3(pkv::kThreads), L::kDynSmem, stream, a, mk, mv) !=
-      cudaSuccess)
-    return PA_ERR_CUDA;
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
-}
-
-template <typename T, int D, int BS, int MODE>
-pa_status dispatch_nt(const pkv::DecodeArgs& a, const CUtensorMap& mk, const CUtensorMap& mv,
-                      int grid, cudaStream_t s) {
-  return a.ncol <= 8 ? launch_decode<T, D, BS, 1, MODE>(a, mk, mv, grid, s)
-                     : launch_decode<T, D, BS, 2, MODE>(a, mk, mv, grid, s);
-}
-
-template <typename T, int D, int MODE>
-pa_status dispatch_bs(int bs, const pkv::DecodeArgs& a, const CUtensorMap& mk,
-                      const CUtensorMap& mv, int grid, cudaStream_t s) {
-  switch (bs) {
-    case 1: return dispatch_nt<T, D, 1, MODE>(a, mk, mv, grid, s);
-    case 8: return dispatch_nt<T, D, 8, MODE>(a, mk, mv, grid, s);
-    case 16: return dispatch_nt<T, D, 16, MODE>(a, mk, mv, grid, s);
-    case 32: return dispatch_nt<T, D, 32, MODE>(a, mk, mv, grid, s);
-  }
-  return PA_ERR_UNSUPPORTED;
-}
-
-template <typename T, int MODE>
-pa_status dispatch_d(int d, int bs, const pkv::DecodeArgs& a, const CUtensorMap& mk,
-                     const CUtensorMap& mv, int grid, cudaStream_t s) {
-  return d == 64 ? dispatch_bs<T, 64, MODE>(bs, a, mk, mv, grid, s)
-                 : dispatch_bs<T, 128, MODE>(bs, a, mk, mv, grid, s);
-}
-
-template <typename T>
-pa_status dispatch_mode(int mode, int d, int bs, const pkv::DecodeArgs& a, const CUtensorMap& mk,
-                        const CUtensorMap& mv, int grid, cudaStream_t s) {
+// Kernel mode -> its translation unit's dispatcher.
+pa_status dispatch_mode(bool kv8, int mode, bool bf16, int d, int bs, const pkv::DecodeArgs& a,
+                        const CUtensorMap& mk, const CUtensorMap& mv, int grid, cudaStream_t s) {
+  using namespace pkv_host;
+  if (kv8) return run_decode_mode<pkv::kPlain, true>(bf16, d, bs, a, mk, mv, grid, s);
   switch (mode) {
-    case pkv::kPlain: return dispatch_d<T, pkv::kPlain>(d, bs, a, mk, mv, grid, s);
-    case pkv::kPrefix: return dispatch_d<T, pkv::kPrefix>(d, bs, a, mk, mv, grid, s);
-    case pkv::kSuffix: return dispatch_d<T, pkv::kSuffix>(d, bs, a, mk, mv, grid, s);
-    case pkv::kAppend: return dispatch_d<T, pkv::kAppend>(d, bs, a, mk, mv, grid, s);
+    case pkv::kPlain: return run_decode_mode<pkv::kPlain, false>(bf16, d, bs, a, mk, mv, grid, s);
+    case pkv::kPrefix: return run_decode_mode<pkv::kPrefix, false>(bf16, d, bs, a, mk, mv, grid, s);
+    case pkv::kSuffix: return run_decode_mode<pkv::kSuffix, false>(bf16, d, bs, a, mk, mv, grid, s);
+    case pkv::kAppend: return run_decode_mode<pkv::kAppend, false>(bf16, d, bs, a, mk, mv, grid, s);
   }
   return PA_ERR_INVALID;
-}
-
-// 8-bit (E4M3) caches: plain decode, head_dim 128.
-template <typename T>
-pa_status dispatch_e4m3(int bs, const pkv::DecodeArgs& a, const CUtensorMap& mk,
-                        const CUtensorMap& mv, int grid, cudaStream_t s) {
-  const bool nt1 = a.ncol <= 8;
-  switch (bs) {
-    case 1: return nt1 ? launch_decode<T, 128, 1, 1, pkv::kPlain, true>(a, mk, mv, grid, s)
-                       : launch_decode<T, 128, 1, 2, pkv::kPlain, true>(a, mk, mv, grid, s);
-    case 8: return nt1 ? launch_decode<T, 128, 8, 1, pkv::kPlain, true>(a, mk, mv, grid, s)
-                       : launch_decode<T, 128, 8, 2, pkv::kPlain, true>(a, mk, mv, grid, s);
-    case 16: return nt1 ? launch_decode<T, 128, 16, 1, pkv::kPlain, true>(a, mk, mv, grid, s)
-                        : launch_decode<T, 128, 16, 2, pkv::kPlain, true>(a, mk, mv, grid, s);
-    case 32: return nt1 ? launch_decode<T, 128, 32, 1, pkv::kPlain, true>(a, mk, mv, grid, s)
-                        : launch_decode<T, 128, 32, 2, pkv::kPlain, true>(a, mk, mv, grid, s);
-  }
-  return PA_ERR_UNSUPPORTED;
 }
 
 // Cascade extras of one launch (kPlain: all null).
@@ -277,12 +196,8 @@ pa_status decode_impl(void* out, const void* q, const void* k_cache, const void*
   a.k_new = cx.k_new;
   a.v_new = cx.v_new;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (cx.kv8)
-    return dtype == PA_BF16 ? dispatch_e4m3<__nv_bfloat16>(block_size, a, mk, mv, grid, st)
-                            : dispatch_e4m3<__half>(block_size, a, mk, mv, grid, st);
-  if (dtype == PA_BF16)
-    return dispatch_mode<__nv_bfloat16>(cx.mode, head_dim, block_size, a, mk, mv, grid, st);
-  return dispatch_mode<__half>(cx.mode, head_dim, block_size, a, mk, mv, grid, st);
+  return dispatch_mode(cx.kv8, cx.mode, dtype == PA_BF16, head_dim, block_size, a, mk, mv, grid,
+                       st);
 }
 
 // Cascade workspace: the split scratch, then the external partials (max, sum)[B][Hq]
@@ -408,13 +323,13 @@ pa_status pa_cache_append_e4m3(void* k_cache, void* v_cache, const void* k, cons
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (dtype == PA_BF16)
-    e = launch(pkv::pa_cache_append_e4m3_kernel<__nv_bfloat16>, dim3((unsigned)blocks), dim3(256),
+    e = pkv_host::launch(pkv::pa_cache_append_e4m3_kernel<__nv_bfloat16>, dim3((unsigned)blocks), dim3(256),
                0, st, static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
                static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping,
                num_tokens, num_kv_heads, cpr, block_size, num_blocks, k_scale, v_scale,
                dev_status);
   else
-    e = launch(pkv::pa_cache_append_e4m3_kernel<__half>, dim3((unsigned)blocks), dim3(256), 0, st,
+    e = pkv_host::launch(pkv::pa_cache_append_e4m3_kernel<__half>, dim3((unsigned)blocks), dim3(256), 0, st,
                static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
                static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping,
                num_tokens, num_kv_heads, cpr, block_size, num_blocks, k_scale, v_scale,
@@ -496,7 +411,7 @@ pa_status pa_cache_append(void* k_cache, void* v_cache, const void* k, const voi
   if (sms <= 0) return PA_ERR_CUDA;
   long long blocks = (total + 255) / 256;
   if (blocks > (long long)sms * 16) blocks = (long long)sms * 16;
-  if (launch(pkv::pa_cache_append_kernel, dim3((unsigned)blocks), dim3(256), 0,
+  if (pkv_host::launch(pkv::pa_cache_append_kernel, dim3((unsigned)blocks), dim3(256), 0,
              static_cast<cudaStream_t>(stream), static_cast<uint4*>(k_cache),
              static_cast<uint4*>(v_cache), static_cast<const uint4*>(k),
              static_cast<const uint4*>(v), slot_mapping, num_tokens, num_kv_heads, cpr,
@@ -526,7 +441,7 @@ pa_status pa_copy_blocks(void* const* k_caches, void* const* v_caches, int num_l
       P.v[i] = static_cast<uint4*>(v_caches[l0 + i]);
     }
     dim3 grid((unsigned)num_pairs, (unsigned)(2 * n));
-    if (launch(pkv::pa_copy_blocks_kernel, grid, dim3(256), 0, static_cast<cudaStream_t>(stream),
+    if (pkv_host::launch(pkv::pa_copy_blocks_kernel, grid, dim3(256), 0, static_cast<cudaStream_t>(stream),
                P, pairs, num_blocks, (long long)(block_bytes / 16), dev_status) != cudaSuccess)
       return PA_ERR_CUDA;
   }

@@ -1,0 +1,15 @@
+// decode_e4m3.cu -- the 8-bit (E4M3) pool decode kernel instances (see launch.cuh).
+#include "launch.cuh"
+
+namespace pkv_host {
+
+template <>
+pa_status run_decode_mode<pkv::kPlain, true>(bool bf16, int d, int bs, const pkv::DecodeArgs& a,
+                                       const CUtensorMap& mk, const CUtensorMap& mv, int grid,
+                                       cudaStream_t s) {
+  (void)d;
+  if (bf16) return dispatch_e4m3<__nv_bfloat16>(bs, a, mk, mv, grid, s);
+  return dispatch_e4m3<__half>(bs, a, mk, mv, grid, s);
+}
+
+}  // namespace pkv_host

@@ -1,0 +1,117 @@
+// launch.cuh -- host-side launch helpers and the template dispatch from runtime shape
+// arguments (dtype, head_dim, block_size, query columns) to a decode kernel instance.
+// The instances are spread over several translation units (decode_*.cu), one per kernel
+// mode, so that they compile in parallel; api.cu reaches them through run_decode_mode.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdlib>
+
+#include "decode.cuh"
+#include "pagedkv.h"
+
+namespace pkv_host {
+
+// Programmatic dependent launch lets a kernel's launch and prologue overlap the tail of
+// the kernel before it in the stream (PAGEDKV_NO_PDL=1 turns it off).
+inline bool use_pdl() {
+  static const bool on = [] {
+    const char* v = std::getenv("PAGEDKV_NO_PDL");
+    return !(v && v[0] && v[0] != '0');
+  }();
+  return on;
+}
+
+template <typename Kernel, typename... Args>
+cudaError_t launch(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                   Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = use_pdl() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+template <typename T, int D, int BS, int NT, int MODE, bool KV8 = false>
+pa_status launch_decode(const pkv::DecodeArgs& a, const CUtensorMap& mk, const CUtensorMap& mv,
+                        int grid, cudaStream_t stream) {
+  using L = pkv::Layout<D, KV8>;
+  auto split = pkv::pa_decode_split_kernel<T, D, BS, NT, MODE, KV8>;
+  if (cudaFuncSetAttribute(split, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynSmem) !=
+      cudaSuccess)
+    return PA_ERR_CUDA;
+  if (launch(split, dim3(grid), dim3(pkv::kThreads), L::kDynSmem, stream, a, mk, mv) !=
+      cudaSuccess)
+    return PA_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+template <typename T, int D, int BS, int MODE>
+pa_status dispatch_nt(const pkv::DecodeArgs& a, const CUtensorMap& mk, const CUtensorMap& mv,
+                      int grid, cudaStream_t s) {
+  return a.ncol <= 8 ? launch_decode<T, D, BS, 1, MODE>(a, mk, mv, grid, s)
+                     : launch_decode<T, D, BS, 2, MODE>(a, mk, mv, grid, s);
+}
+
+template <typename T, int D, int MODE>
+pa_status dispatch_bs(int bs, const pkv::DecodeArgs& a, const CUtensorMap& mk,
+                      const CUtensorMap& mv, int grid, cudaStream_t s) {
+  switch (bs) {
+    case 1: return dispatch_nt<T, D, 1, MODE>(a, mk, mv, grid, s);
+    case 8: return dispatch_nt<T, D, 8, MODE>(a, mk, mv, grid, s);
+    case 16: return dispatch_nt<T, D, 16, MODE>(a, mk, mv, grid, s);
+    case 32: return dispatch_nt<T, D, 32, MODE>(a, mk, mv, grid, s);
+  }
+  return PA_ERR_UNSUPPORTED;
+}
+
+template <typename T, int MODE>
+pa_status dispatch_d(int d, int bs, const pkv::DecodeArgs& a, const CUtensorMap& mk,
+                     const CUtensorMap& mv, int grid, cudaStream_t s) {
+  return d == 64 ? dispatch_bs<T, 64, MODE>(bs, a, mk, mv, grid, s)
+                 : dispatch_bs<T, 128, MODE>(bs, a, mk, mv, grid, s);
+}
+
+// 8-bit (E4M3) caches: plain decode, head_dim 128.
+template <typename T>
+pa_status dispatch_e4m3(int bs, const pkv::DecodeArgs& a, const CUtensorMap& mk,
+                        const CUtensorMap& mv, int grid, cudaStream_t s) {
+  const bool nt1 = a.ncol <= 8;
+  switch (bs) {
+    case 1: return nt1 ? launch_decode<T, 128, 1, 1, pkv::kPlain, true>(a, mk, mv, grid, s)
+                       : launch_decode<T, 128, 1, 2, pkv::kPlain, true>(a, mk, mv, grid, s);
+    case 8: return nt1 ? launch_decode<T, 128, 8, 1, pkv::kPlain, true>(a, mk, mv, grid, s)
+                       : launch_decode<T, 128, 8, 2, pkv::kPlain, true>(a, mk, mv, grid, s);
+    case 16: return nt1 ? launch_decode<T, 128, 16, 1, pkv::kPlain, true>(a, mk, mv, grid, s)
+                        : launch_decode<T, 128, 16, 2, pkv::kPlain, true>(a, mk, mv, grid, s);
+    case 32: return nt1 ? launch_decode<T, 128, 32, 1, pkv::kPlain, true>(a, mk, mv, grid, s)
+                        : launch_decode<T, 128, 32, 2, pkv::kPlain, true>(a, mk, mv, grid, s);
+  }
+  return PA_ERR_UNSUPPORTED;
+}
+
+// One kernel mode's instances, dispatched on the other parameters; defined in
+// decode_<mode>.cu.  kv8: 8-bit E4M3 pools (kPlain only).
+template <int MODE, bool KV8>
+pa_status run_decode_mode(bool bf16, int d, int bs, const pkv::DecodeArgs& a,
+                          const CUtensorMap& mk, const CUtensorMap& mv, int grid, cudaStream_t s);
+#define PKV_DECL_RUN(MODE, KV8)                                                              \
+  template <>                                                                                \
+  pa_status run_decode_mode<MODE, KV8>(bool bf16, int d, int bs, const pkv::DecodeArgs& a,   \
+                                       const CUtensorMap& mk, const CUtensorMap& mv, int grid, \
+                                       cudaStream_t s);
+PKV_DECL_RUN(pkv::kPlain, false)
+PKV_DECL_RUN(pkv::kPrefix, false)
+PKV_DECL_RUN(pkv::kSuffix, false)
+PKV_DECL_RUN(pkv::kAppend, false)
+PKV_DECL_RUN(pkv::kPlain, true)
+#undef PKV_DECL_RUN
+
+}  // namespace pkv_host

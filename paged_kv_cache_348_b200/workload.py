@@ -242,10 +242,10 @@ def plan_cascade(tables: np.ndarray, ctx: np.ndarray, block_size: int, group: in
     sharing group; its prefix is the leading table entries common to all members,
     capped at the shortest member's length.  Groups of one sequence get no chunk.
     Returns (prefix_lens int32 [B], chunk_members int32 [C, width], chunk_prefix_lens
-    int32 [C]); a chunk holds at most `width` members (default: 8 query rows per chunk,
-    the lighter kernel; group * width <= 16)."""
+    int32 [C]); a chunk holds at most `width` members (default: 16 query rows per chunk,
+    which reads each shared prefix least often; group * width <= 16)."""
     B = len(ctx)
-    cap = width or max(1, 8 // group)
+    cap = width or max(1, 16 // group)
     by_first = {}
     for s in range(B):
         if ctx[s] > 0:

@@ -124,7 +124,7 @@ def test_cascade_shared_prefix_workload_full_size():
     b = wl.build_prefix_decode()
     tables, ctx = b.block_tables.cpu().numpy(), b.context_lens.cpu().numpy()
     prefix, members, plens = wl.plan_cascade(tables, ctx, b.block_size, 4)
-    assert (prefix == inputs.PREFIX_LEN).all() and len(plens) == 64       # 4 chunks a prompt
+    assert (prefix == inputs.PREFIX_LEN).all() and len(plens) == 32       # 2 chunks a prompt
     out = torch.empty_like(b.q[0])
     ws = pk.new_cascade_workspace(128, 32, 8, 128)
     dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
