@@ -148,7 +148,7 @@ pa_status decode_impl(void* out, const void* q, const void* k_cache, const void*
     return PA_ERR_INVALID;
   const int sms = sm_count();
   if (sms <= 0) return PA_ERR_CUDA;
-  int grid = sms * pkv::kCtasPerSm;
+  int grid = sms * pkv::ctas_per_sm(cx.kv8, group * q_len <= 8 ? 1 : 2);   // as dispatch_nt
   if (grid_cap > 0 && grid > grid_cap) grid = grid_cap;
   const WsLayout w = ws_layout(num_seqs, head_dim, grid);
   if (workspace_bytes < w.total) return PA_ERR_INVALID;
@@ -236,7 +236,7 @@ size_t pa_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads
   if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0) return 0;
   const int sms = sm_count();
   if (sms <= 0) return 0;
-  return ws_layout(num_seqs, head_dim, sms * pkv::kCtasPerSm).total;
+  return ws_layout(num_seqs, head_dim, sms * pkv::kMaxCtasPerSm).total;
 }
 
 pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
@@ -343,7 +343,7 @@ size_t pa_decode_cascade_workspace_bytes(int num_seqs, int num_q_heads, int num_
   if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0) return 0;
   const int sms = sm_count();
   if (sms <= 0) return 0;
-  return cascade_layout(num_seqs, num_q_heads, head_dim, sms * pkv::kCtasPerSm).total;
+  return cascade_layout(num_seqs, num_q_heads, head_dim, sms * pkv::kMaxCtasPerSm).total;
 }
 
 pa_status pa_decode_cascade(void* out, const void* q, const void* k_cache, const void* v_cache,
@@ -364,7 +364,7 @@ pa_status pa_decode_cascade(void* out, const void* q, const void* k_cache, const
     return PA_ERR_INVALID;
   const int sms = sm_count();
   if (sms <= 0) return PA_ERR_CUDA;
-  const CascadeLayout cl = cascade_layout(num_seqs, num_q_heads, head_dim, sms * pkv::kCtasPerSm);
+  const CascadeLayout cl = cascade_layout(num_seqs, num_q_heads, head_dim, sms * pkv::kMaxCtasPerSm);
   if (workspace_bytes < cl.total) return PA_ERR_INVALID;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   CascadeArgs cx;

@@ -9,7 +9,8 @@
 // Design (B200):
 //  * Work is the set of (sequence, kv head) segments, cut into 16-token units.  The
 //    units of all segments are laid end to end and split into gridDim.x equal
-//    ranges, one per persistent CTA (2 per SM), so a batch with a heavy-tailed
+//    ranges, one per persistent CTA (2 per SM; 3 for 8-bit caches with one query-column
+//    tile, whose stages are half the size), so a batch with a heavy-tailed
 //    length mix still gives every SM the same number of KV bytes.  A segment that
 //    straddles CTA ranges leaves one (max, sum, acc) partial per CTA in the
 //    workspace; the last of those CTAs to finish (an epoch-tagged arrival counter,
@@ -53,7 +54,10 @@ constexpr int kUnitsPerStage = kConsumerWarps;      // one unit per consumer war
 constexpr int kTileTokens = kUnit * kUnitsPerStage; // 64 tokens per stage
 constexpr int kStages = 3;
 constexpr int kThreads = 32 * (1 + kConsumerWarps); // warp 0 produces, 1..4 consume
-constexpr int kCtasPerSm = 2;
+// Resident CTAs per SM: 2, or 3 for 8-bit caches with one query-column tile (their
+// consumers convert codes as well, and half-size stages let a third CTA's warps in).
+__host__ __device__ constexpr int ctas_per_sm(bool kv8, int nt) { return kv8 && nt == 1 ? 3 : 2; }
+constexpr int kMaxCtasPerSm = 3;        // the split workspace covers this many per SM
 constexpr int kMaxGroup = 16;                       // q heads per kv head handled
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
@@ -122,10 +126,10 @@ struct DecodeArgs {
 
 // Shared-memory layout of a CTA.  16-bit caches: K and V tiles of 64 tokens in D/64
 // column halves of 128-byte lines; 8-bit (E4M3) caches: one line of D bytes per token
-// (D = 128), and a deeper ring since a stage is half the size.
-template <int D, bool KV8 = false>
+// (D = 128), and, since a stage is half the size, a deeper ring at 2 CTAs per SM.
+template <int D, bool KV8 = false, int CPS = 2>
 struct Layout {
-  static constexpr int kStages = KV8 ? 5 : 3;
+  static constexpr int kStages = (KV8 && CPS == 2) ? 5 : 3;
   static constexpr int kHalves = D / 64;                   // 128-byte swizzled column halves
   static constexpr int kKvBytes = KV8 ? kTileTokens * D : kHalves * kTileTokens * 128;
   static constexpr int kQBytes = kMaxGroup * D * 2;
@@ -146,7 +150,7 @@ struct Layout {
   static_assert(kBarOff % 8 == 0 && kMiscOff % 8 == 0 && kDescOff % 8 == 0 && kMlOff % 8 == 0 &&
                     kNewOff % 16 == 0 && kNewBytes % 16 == 0,
                 "mbarriers and 64-bit fields need 8-byte, bulk-copy targets 16-byte alignment");
-  static_assert(2 * (kDynSmem + 1024) <= 233472, "two CTAs per SM must fit");
+  static_assert(CPS * (kDynSmem + 1024) <= 233472, "CPS CTAs per SM must fit");
 };
 
 __device__ __forceinline__ void st_relaxed_gpu(unsigned long long* p, unsigned long long v) {
@@ -431,10 +435,10 @@ __device__ __forceinline__ void merge_split(const DecodeArgs& a, const SplitDesc
 }
 
 template <typename T, int D, int BS, int NT, int MODE, bool KV8 = false>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+__global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT))
     pa_decode_split_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
                            const __grid_constant__ CUtensorMap tmv) {
-  using L = Layout<D, KV8>;
+  using L = Layout<D, KV8, ctas_per_sm(KV8, NT)>;
   constexpr int kStages = L::kStages;
   static_assert(!KV8 || (D == 128 && MODE == kPlain), "8-bit caches: head_dim 128, plain decode");
   // MMA operand type: the cache's 16-bit type, or fp16 for E4M3 (exact there)
