@@ -148,7 +148,7 @@ pa_status decode_impl(void* out, const void* q, const void* k_cache, const void*
     return PA_ERR_INVALID;
   const int sms = sm_count();
   if (sms <= 0) return PA_ERR_CUDA;
-  int grid = sms * pkv::ctas_per_sm(cx.kv8, group * q_len <= 8 ? 1 : 2);   // as dispatch_nt
+  int grid = sms * pkv::ctas_per_sm(cx.kv8, group * q_len <= 8 ? 1 : 2, block_size);   // as dispatch_nt
   if (grid_cap > 0 && grid > grid_cap) grid = grid_cap;
   const WsLayout w = ws_layout(num_seqs, head_dim, grid);
   if (workspace_bytes < w.total) return PA_ERR_INVALID;

@@ -9,8 +9,8 @@
 // Design (B200):
 //  * Work is the set of (sequence, kv head) segments, cut into 16-token units.  The
 //    units of all segments are laid end to end and split into gridDim.x equal
-//    ranges, one per persistent CTA (2 per SM; 3 for 8-bit caches with one query-column
-//    tile, whose stages are half the size), so a batch with a heavy-tailed
+//    ranges, one per persistent CTA (2 per SM; 3 with one query-column tile for 8-bit
+//    caches or block_size 1), so a batch with a heavy-tailed
 //    length mix still gives every SM the same number of KV bytes.  A segment that
 //    straddles CTA ranges leaves one (max, sum, acc) partial per CTA in the
 //    workspace; the last of those CTAs to finish (an epoch-tagged arrival counter,
@@ -54,9 +54,13 @@ constexpr int kUnitsPerStage = kConsumerWarps;      // one unit per consumer war
 constexpr int kTileTokens = kUnit * kUnitsPerStage; // 64 tokens per stage
 constexpr int kStages = 3;
 constexpr int kThreads = 32 * (1 + kConsumerWarps); // warp 0 produces, 1..4 consume
-// Resident CTAs per SM: 2, or 3 for 8-bit caches with one query-column tile (their
-// consumers convert codes as well, and half-size stages let a third CTA's warps in).
-__host__ __device__ constexpr int ctas_per_sm(bool kv8, int nt) { return kv8 && nt == 1 ? 3 : 2; }
+// Resident CTAs per SM: 2, or 3 with one query-column tile (128 registers a thread) when
+// the rate is set per CTA rather than by HBM: 8-bit caches, whose consumers also convert
+// codes (half-size stages keep a 3-deep ring), and block_size 1, whose producer issues a
+// 16-byte cp.async per 16 bytes of K/V (a 2-deep ring of 16-bit stages).
+__host__ __device__ constexpr int ctas_per_sm(bool kv8, int nt, int bs) {
+  return (kv8 || bs == 1) && nt == 1 ? 3 : 2;
+}
 constexpr int kMaxCtasPerSm = 3;        // the split workspace covers this many per SM
 constexpr int kMaxGroup = 16;                       // q heads per kv head handled
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
@@ -126,10 +130,11 @@ struct DecodeArgs {
 
 // Shared-memory layout of a CTA.  16-bit caches: K and V tiles of 64 tokens in D/64
 // column halves of 128-byte lines; 8-bit (E4M3) caches: one line of D bytes per token
-// (D = 128), and, since a stage is half the size, a deeper ring at 2 CTAs per SM.
+// (D = 128), and, since a stage is half the size, a deeper ring.  CPS = CTAs per SM.
 template <int D, bool KV8 = false, int CPS = 2>
 struct Layout {
-  static constexpr int kStages = (KV8 && CPS == 2) ? 5 : 3;
+  static constexpr int kStages = KV8 ? (CPS == 2 ? 5 : 3) : (CPS == 2 ? 3 : 2);
+  static_assert(CPS == 2 || CPS == 3, "2 or 3 CTAs per SM");
   static constexpr int kHalves = D / 64;                   // 128-byte swizzled column halves
   static constexpr int kKvBytes = KV8 ? kTileTokens * D : kHalves * kTileTokens * 128;
   static constexpr int kQBytes = kMaxGroup * D * 2;
@@ -435,10 +440,10 @@ __device__ __forceinline__ void merge_split(const DecodeArgs& a, const SplitDesc
 }
 
 template <typename T, int D, int BS, int NT, int MODE, bool KV8 = false>
-__global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT))
+__global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
     pa_decode_split_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
                            const __grid_constant__ CUtensorMap tmv) {
-  using L = Layout<D, KV8, ctas_per_sm(KV8, NT)>;
+  using L = Layout<D, KV8, ctas_per_sm(KV8, NT, BS)>;
   constexpr int kStages = L::kStages;
   static_assert(!KV8 || (D == 128 && MODE == kPlain), "8-bit caches: head_dim 128, plain decode");
   // MMA operand type: the cache's 16-bit type, or fp16 for E4M3 (exact there)
@@ -720,7 +725,9 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT))
           } else {
             // block_size 1: every token is its own block; 16-byte cp.async with the same
             // 128-byte swizzle the TMA path produces.  Stages are 64 tokens, so the window
-            // (w0, w1) holds exactly this stage's table entries, handed out by shuffle.
+            // (w0, w1) holds exactly this stage's table entries, handed out by shuffle.  The
+            // copy loop is unrolled: one warp issues all of a stage's copies, so their
+            // address arithmetic must overlap.
             constexpr int CPR = D * (KV8 ? 1 : 2) / 16;   // 16-byte chunks per row
             constexpr int RPI = 32 / CPR;            // rows per warp instruction
             const int ntok = nun * kUnit;
@@ -739,12 +746,20 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT))
                   bulk_load(sQ + jq * qrow_bytes, qrow_src(jq), qrow_bytes, &full[st]);
               if (nbytes) stage_new(&full[st]);
             }
-            const int ch = lane % CPR, hf = ch >> 3, cc = ch & 7;
-            for (int r0 = 0; r0 < ntok; r0 += RPI) {
-              const int r = r0 + lane / CPR;
+            const int ch = lane % CPR, hf = ch >> 3, cc = ch & 7, rl = lane / CPR;
+            constexpr long long kRowBytes = D * (KV8 ? 1 : 2);
+            const uint8_t* kb = static_cast<const uint8_t*>(a.k_cache) + ch * 16;
+            const uint8_t* vb = static_cast<const uint8_t*>(a.v_cache) + ch * 16;
+            uint8_t* sKl = sK + hf * (kTileTokens * 128) + rl * 128;
+            uint8_t* sVl = sV + hf * (kTileTokens * 128) + rl * 128;
+            const int nvalid = ntok < ctx_cur - tok0 ? ntok : ctx_cur - tok0;
+#pragma unroll
+            for (int i = 0; i < kTileTokens / RPI; ++i) {
+              const int r0 = i * RPI;
+              if (r0 >= ntok) break;
+              const int r = r0 + rl;
               const int blk = __shfl_sync(0xffffffffu, r0 >= 32 ? w1 : w0, r & 31);
-              const int t = tok0 + r;
-              if (r < ntok && t < ctx_cur) {
+              if (r < nvalid) {
                 uint32_t sz = 16;
                 long long row = 0;
                 if ((unsigned)blk < (unsigned)a.num_blocks) {
@@ -753,11 +768,9 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT))
                   if (a.status) atomicOr(a.status, DEV_BAD_BLOCK_ID);
                   sz = 0;                                // zero fill, no read
                 }
-                const long long off = (row * D + ch * 8) * 2;   // bytes; 8-bit: row * D + ch * 16
-                const int soff = hf * (kTileTokens * 128) + r * 128 + ((cc ^ (r & 7)) << 4);
-                const long long boff = KV8 ? row * D + ch * 16 : off;
-                cp_async_16_zfill(sK + soff, static_cast<const uint8_t*>(a.k_cache) + boff, sz, policy);
-                cp_async_16_zfill(sV + soff, static_cast<const uint8_t*>(a.v_cache) + boff, sz, policy);
+                const int soff = r0 * 128 + ((cc ^ (r & 7)) << 4);
+                cp_async_16_zfill(sKl + soff, kb + row * kRowBytes, sz, policy);
+                cp_async_16_zfill(sVl + soff, vb + row * kRowBytes, sz, policy);
               }
             }
             cp_async_mbar_arrive_noinc(&full[st]);
