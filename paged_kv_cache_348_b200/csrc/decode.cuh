@@ -10,7 +10,7 @@
 //  * Work is the set of (sequence, kv head) segments, cut into 16-token units.  The
 //    units of all segments are laid end to end and split into gridDim.x equal
 //    ranges, one per persistent CTA (2 per SM; 3 with one query-column tile for 8-bit
-//    caches or block_size 1), so a batch with a heavy-tailed
+//    caches or block_size <= 8), so a batch with a heavy-tailed
 //    length mix still gives every SM the same number of KV bytes.  A segment that
 //    straddles CTA ranges leaves one (max, sum, acc) partial per CTA in the
 //    workspace; the last of those CTAs to finish (an epoch-tagged arrival counter,
@@ -56,10 +56,11 @@ constexpr int kStages = 3;
 constexpr int kThreads = 32 * (1 + kConsumerWarps); // warp 0 produces, 1..4 consume
 // Resident CTAs per SM: 2, or 3 with one query-column tile (128 registers a thread) when
 // the rate is set per CTA rather than by HBM: 8-bit caches, whose consumers also convert
-// codes (half-size stages keep a 3-deep ring), and block_size 1, whose producer issues a
-// 16-byte cp.async per 16 bytes of K/V (a 2-deep ring of 16-bit stages).
+// codes (half-size stages keep a 3-deep ring), and block_size <= 8, whose producer issues
+// a copy per 16 bytes (block_size 1) or per 1 KB box (block_size 8); 16-bit stages then
+// form a 2-deep ring.
 __host__ __device__ constexpr int ctas_per_sm(bool kv8, int nt, int bs) {
-  return (kv8 || bs == 1) && nt == 1 ? 3 : 2;
+  return (kv8 || bs <= 8) && nt == 1 ? 3 : 2;
 }
 constexpr int kMaxCtasPerSm = 3;        // the split workspace covers this many per SM
 constexpr int kMaxGroup = 16;                       // q heads per kv head handled
@@ -324,13 +325,14 @@ __device__ __forceinline__ void empty_rows(const DecodeArgs& a, int s, int first
   }
 }
 
-// Two E4M3 codes (low byte first) to two fp16 values, exactly.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t x16) {
-  uint32_t y;
-  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}"
-      : "=r"(y)
-      : "r"(x16));
-  return y;
+// Four E4M3 codes (bytes 0..3 of x) to fp16 pairs (bytes 0, 1) and (bytes 2, 3), exactly.
+// Splitting the word with mov.b32 hands each conversion a register half directly (no
+// shift or mask to extract the upper pair).
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t x, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\tcvt.rn.f16x2.e4m3x2 %0, a;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(x));
 }
 
 // Entry i (0 <= i < 96) of a block-table window held across the warp: lane l holds
@@ -915,10 +917,11 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
           const uint32_t addr = kbase + r * 128 + ((chunk ^ (r & 7)) << 4);
           uint32_t m0, m1, m2, m3;
           ldsm_x4(addr, m0, m1, m2, m3);
-          const uint32_t x0 = e4m3x2_to_f16x2(m0 & 0xffffu), x2 = e4m3x2_to_f16x2(m0 >> 16);
-          const uint32_t x1 = e4m3x2_to_f16x2(m1 & 0xffffu), x3 = e4m3x2_to_f16x2(m1 >> 16);
-          const uint32_t y0 = e4m3x2_to_f16x2(m2 & 0xffffu), y2 = e4m3x2_to_f16x2(m2 >> 16);
-          const uint32_t y1 = e4m3x2_to_f16x2(m3 & 0xffffu), y3 = e4m3x2_to_f16x2(m3 >> 16);
+          uint32_t x0, x1, x2, x3, y0, y1, y2, y3;
+          e4m3x4_to_f16x2x2(m0, x0, x2);
+          e4m3x4_to_f16x2x2(m1, x1, x3);
+          e4m3x4_to_f16x2x2(m2, y0, y2);
+          e4m3x4_to_f16x2x2(m3, y1, y3);
 #pragma unroll
           for (int n = 0; n < NT; ++n) {
             mma16816<false>(sacc[n], x0, x1, x2, x3, qf[ks][n][0], qf[ks][n][1]);
@@ -995,51 +998,68 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
         mlo = (t_a < valid ? 0x0000ffffu : 0u) | (t_a + 1 < valid ? 0xffff0000u : 0u);
         mhi = (t_b < valid ? 0x0000ffffu : 0u) | (t_b + 1 < valid ? 0xffff0000u : 0u);
       }
+      // the PV product; with 8-bit caches (ALU-bound) the token masks are applied only to
+      // a unit with fewer than 16 valid rows (a lambda instantiated with and without them)
+      auto pv = [&](auto masked) {
+        if constexpr (KV8) {
+          // ldmatrix.x4.trans of tokens 0-7 / 8-15 of two 16-byte chunks; a thread gets the
+          // codes of dims (2g, 2g+1) for tokens (2c, 2c+1): regrouped per dim they give the
+          // A fragments with M-row g = dim 2g and M-row g+8 = dim 2g+1 of the chunk
+          const int j = lane >> 3, i = lane & 7;
+          const int r = cw * kUnit + (j & 1) * 8 + i;
+#pragma unroll
+          for (int mtile = 0; mtile < KS; mtile += 2) {
+            const int chunk = mtile + (j >> 1);
+            const uint32_t addr = vbase + r * 128 + ((chunk ^ (r & 7)) << 4);
+            uint32_t m[4];
+            ldsm_x4_t(addr, m[0], m[1], m[2], m[3]);
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              const uint32_t p0 = __byte_perm(m[2 * hh], 0u, 0x3120);       // tokens 2c, 2c+1
+              const uint32_t p1 = __byte_perm(m[2 * hh + 1], 0u, 0x3120);   // tokens 8+2c, ...
+              uint32_t a0, a1, a2, a3;
+              e4m3x4_to_f16x2x2(p0, a0, a1);
+              e4m3x4_to_f16x2x2(p1, a2, a3);
+              if constexpr (decltype(masked)::value) {
+                a0 &= mlo;
+                a1 &= mlo;
+                a2 &= mhi;
+                a3 &= mhi;
+              }
+#pragma unroll
+              for (int n = 0; n < NT; ++n)
+                mma16816<false>(o[mtile + hh][n], a0, a1, a2, a3, bhi[n][0], bhi[n][1]);
+            }
+          }
+        } else {
+          const int j = lane >> 3, i = lane & 7;
+          const int r = cw * kUnit + (j >> 1) * 8 + i;
+#pragma unroll
+          for (int mtile = 0; mtile < KS; ++mtile) {
+            const int d = mtile * 16 + (j & 1) * 8;
+            const uint32_t addr =
+                vbase + (d >> 6) * (kTileTokens * 128) + r * 128 + ((((d & 63) >> 3) ^ (r & 7)) << 4);
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4_t(addr, a0, a1, a2, a3);
+            if constexpr (decltype(masked)::value) {
+              a0 &= mlo;
+              a1 &= mlo;
+              a2 &= mhi;
+              a3 &= mhi;
+            }
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+              mma16816<kBF16>(o[mtile][n], a0, a1, a2, a3, bhi[n][0], bhi[n][1]);
+              mma16816<kBF16>(o[mtile][n], a0, a1, a2, a3, blo[n][0], blo[n][1]);
+            }
+          }
+        }
+      };
       if constexpr (KV8) {
-        // ldmatrix.x4.trans of tokens 0-7 / 8-15 of two 16-byte chunks; a thread gets the
-        // codes of dims (2g, 2g+1) for tokens (2c, 2c+1): regrouped per dim they give the
-        // A fragments with M-row g = dim 2g and M-row g+8 = dim 2g+1 of the chunk
-        const int j = lane >> 3, i = lane & 7;
-        const int r = cw * kUnit + (j & 1) * 8 + i;
-#pragma unroll
-        for (int mtile = 0; mtile < KS; mtile += 2) {
-          const int chunk = mtile + (j >> 1);
-          const uint32_t addr = vbase + r * 128 + ((chunk ^ (r & 7)) << 4);
-          uint32_t m[4];
-          ldsm_x4_t(addr, m[0], m[1], m[2], m[3]);
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const uint32_t p0 = __byte_perm(m[2 * hh], 0u, 0x3120);       // tokens 2c, 2c+1
-            const uint32_t p1 = __byte_perm(m[2 * hh + 1], 0u, 0x3120);   // tokens 8+2c, ...
-            const uint32_t a0 = e4m3x2_to_f16x2(p0 & 0xffffu) & mlo;
-            const uint32_t a1 = e4m3x2_to_f16x2(p0 >> 16) & mlo;
-            const uint32_t a2 = e4m3x2_to_f16x2(p1 & 0xffffu) & mhi;
-            const uint32_t a3 = e4m3x2_to_f16x2(p1 >> 16) & mhi;
-#pragma unroll
-            for (int n = 0; n < NT; ++n)
-              mma16816<false>(o[mtile + hh][n], a0, a1, a2, a3, bhi[n][0], bhi[n][1]);
-          }
-        }
+        if (valid < kUnit) pv(std::true_type{});
+        else pv(std::false_type{});
       } else {
-        const int j = lane >> 3, i = lane & 7;
-        const int r = cw * kUnit + (j >> 1) * 8 + i;
-#pragma unroll
-        for (int mtile = 0; mtile < KS; ++mtile) {
-          const int d = mtile * 16 + (j & 1) * 8;
-          const uint32_t addr =
-              vbase + (d >> 6) * (kTileTokens * 128) + r * 128 + ((((d & 63) >> 3) ^ (r & 7)) << 4);
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4_t(addr, a0, a1, a2, a3);
-          a0 &= mlo;
-          a1 &= mlo;
-          a2 &= mhi;
-          a3 &= mhi;
-#pragma unroll
-          for (int n = 0; n < NT; ++n) {
-            mma16816<kBF16>(o[mtile][n], a0, a1, a2, a3, bhi[n][0], bhi[n][1]);
-            mma16816<kBF16>(o[mtile][n], a0, a1, a2, a3, blo[n][0], blo[n][1]);
-          }
-        }
+        pv(std::true_type{});
       }
     }
     if (mt.flags & F_LAST) {
