@@ -954,6 +954,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
           xs[e] = (row < valid && row < lim) ? sacc[n][e] * a.scale_log2 : -INFINITY;
         }
         float alpha[2], p[4];
+        bool grew = false;
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
           float mx = fmaxf(xs[cc], xs[cc + 2]);
@@ -963,18 +964,23 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
           const float mnew = fmaxf(m[n][cc], mx);
           // a column with no visible row yet keeps max -inf: use 0 as the reference
           const float mref = mnew == -INFINITY ? 0.f : mnew;
+          grew |= mnew != m[n][cc];
           alpha[cc] = ex2(m[n][cc] - mref);
           m[n][cc] = mnew;
           p[cc] = ex2(xs[cc] - mref);
           p[cc + 2] = ex2(xs[cc + 2] - mref);
           l[n][cc] = l[n][cc] * alpha[cc] + p[cc] + p[cc + 2];
         }
+        // 8-bit caches (ALU-bound): rescale O only when a column's running max moved in
+        // this warp (alpha is exactly 1 otherwise)
+        if (!KV8 || __any_sync(0xffffffffu, grew)) {
 #pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-          o[ks][n][0] *= alpha[0];
-          o[ks][n][1] *= alpha[1];
-          o[ks][n][2] *= alpha[0];
-          o[ks][n][3] *= alpha[1];
+          for (int ks = 0; ks < KS; ++ks) {
+            o[ks][n][0] *= alpha[0];
+            o[ks][n][1] *= alpha[1];
+            o[ks][n][2] *= alpha[0];
+            o[ks][n][3] *= alpha[1];
+          }
         }
         using TM = std::conditional_t<KV8, __half, T>;   // MMA operand type
         const uint32_t h01 = pack2<TM>(p[0], p[1]), h23 = pack2<TM>(p[2], p[3]);
