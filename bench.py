@@ -67,14 +67,15 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def ncu_traffic(workload_name, bs):
+def ncu_traffic(workload_name, bs, variant):
     """DRAM bytes per decode launch from the committed ncu summary, if it was taken on
-    the current kernel source."""
+    the current kernel source for this workload, block size and entry point (variant:
+    append, decode, e4m3, multi, cascade)."""
     p = os.path.join(ROOT, "profiles", "decode_traffic.json")
     try:
         with open(p) as f:
             d = json.load(f)
-        e = d["entries"]["%s_bs%d" % (workload_name, bs)]
+        e = d["entries"]["%s_bs%d_%s" % (workload_name, bs, variant)]
         if e.get("source_hash") != source_hash():
             return None
         return int(e["dram_bytes_per_launch"])
@@ -351,7 +352,9 @@ def main():
     peak, peak_kind = measured_hbm_peak()
     dec_avg = statistics.mean(dec_ms)
     achieved = kv_layer / (dec_avg * 1e-3) / 1e9
-    traffic = ncu_traffic(w.name, bs)
+    variant = ("cascade" if b.cascade is not None else "append" if fused else
+               "e4m3" if b.kv_scales is not None else "decode" if b.q_len == 1 else "multi")
+    traffic = ncu_traffic(w.name, bs, variant)
 
     # ---------------- end to end through the public API, host buffers
     e2e = None
