@@ -148,15 +148,16 @@ def device_bus_id(torch):
 
 
 # ------------------------------------------------------------------------------- oracle
-def oracle_sample(w, bs, max_seconds=15.0, device_batch=None):
-    """Time the CPU oracle on whole sequences of layer 0 until ~max_seconds of work.
-    Returns (kv_bytes, seconds, seqs, threads)."""
+def oracle_sample(w, bs, max_seconds=15.0, device_batch=None, nthreads=None):
+    """Time the CPU oracle on whole sequences of layer 0 until ~max_seconds of work, on
+    all host cores (or nthreads).  Returns (kv_bytes, seconds, seqs, threads)."""
     import torch
 
     import oracle
     from paged_kv_cache_348_b200 import inputs
 
-    threads = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    threads = nthreads or (len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity")
+                           else os.cpu_count())
     if device_batch is not None:
         b = device_batch
         def bits(t):
@@ -398,10 +399,13 @@ def main():
             "frac": uniq / L / (dec_avg * 1e-3) / 1e9 / peak}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         nbytes, sec, seqs, threads = oracle_sample(w, bs, device_batch=b)
+        n1, sec1, seqs1, _ = oracle_sample(w, bs, max_seconds=3.0, device_batch=b, nthreads=1)
         line["cpu_baseline"] = {
             "value": nbytes / sec / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
             "sample": "%d whole sequences (all %d q heads) of layer 0 of this workload, "
-                      "%.1f s" % (seqs, w.num_q_heads, sec)}
+                      "%.1f s" % (seqs, w.num_q_heads, sec),
+            "value_1thread": n1 / sec1 / 1e9,
+            "sample_1thread": "%d whole sequences of layer 0, %.1f s on one thread" % (seqs1, sec1)}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
