@@ -807,26 +807,35 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
   const int gid = lane >> 2, tig = lane & 3;
   const int tid = cw * 32 + lane;
   constexpr int KS = D / 16;            // k-steps of QK, m-tiles of PV
-  constexpr int NREG = KS * NT * 4;     // O^T accumulator registers per thread
-  float o[KS][NT][4];
-  float m[NT][2], l[NT][2];
-  uint32_t qf[KS][NT][2];
+  constexpr int NREG = KS * NT * 4;     // O^T accumulator registers per thread (all n-tiles)
+  // With 16 query columns (NT = 2) a warp holding both n-tiles of O and q runs out of
+  // registers (spills in the unit loop), so with 16-bit caches the warps of a pair split
+  // the columns: warp cw takes n-tile cw & 1 of units 2 (cw >> 1) and 2 (cw >> 1) + 1 of
+  // every stage.  The fused append keeps one unit per warp (its patched row is written
+  // by the warp of its unit), as do 8-bit caches.
+  constexpr bool kColSplit = NT == 2 && !KV8 && MODE != kAppend;
+  constexpr int NTW = kColSplit ? 1 : NT;       // n-tiles a warp holds
+  constexpr int UPW = kColSplit ? 2 : 1;        // units a warp takes per stage
+  const int nb = kColSplit ? (cw & 1) : 0;      // its first n-tile
+  float o[KS][NTW][4];
+  float m[NTW][2], l[NTW][2];
+  uint32_t qf[KS][NTW][2];
 #pragma unroll
   for (int i = 0; i < KS; ++i)
 #pragma unroll
-    for (int n = 0; n < NT; ++n) {
+    for (int n = 0; n < NTW; ++n) {
       qf[i][n][0] = qf[i][n][1] = 0u;
 #pragma unroll
       for (int e = 0; e < 4; ++e) o[i][n][e] = 0.f;
     }
 #pragma unroll
-  for (int n = 0; n < NT; ++n) m[n][0] = m[n][1] = -INFINITY, l[n][0] = l[n][1] = 0.f;
+  for (int n = 0; n < NTW; ++n) m[n][0] = m[n][1] = -INFINITY, l[n][0] = l[n][1] = 0.f;
   // new-token index of this lane's two accumulator columns per n-tile
-  int jcol[NT][2];
+  int jcol[NTW][2];
 #pragma unroll
-  for (int n = 0; n < NT; ++n) {
-    jcol[n][0] = (n * 8 + 2 * tig) / group;
-    jcol[n][1] = (n * 8 + 2 * tig + 1) / group;
+  for (int n = 0; n < NTW; ++n) {
+    jcol[n][0] = ((nb + n) * 8 + 2 * tig) / group;
+    jcol[n][1] = ((nb + n) * 8 + 2 * tig + 1) / group;
   }
 
   int st = 0;
@@ -846,8 +855,8 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
     const uint8_t* sQ = sV + L::kKvBytes;
     if (mt.flags & F_FIRST) {
 #pragma unroll
-      for (int n = 0; n < NT; ++n) {
-        const int cq = n * 8 + gid;                  // this lane's query column
+      for (int n = 0; n < NTW; ++n) {
+        const int cq = (nb + n) * 8 + gid;           // this lane's query column
 #pragma unroll
         for (int ks = 0; ks < KS; ++ks) {
           uint32_t b0 = 0u, b1 = 0u;
@@ -877,155 +886,179 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
       }
     }
     bool patched = false;
-    if (cw < mt.nunits) {
-      const int t0 = mt.tok0 + cw * kUnit;
-      const int valid = (mt.ctx - t0) < kUnit ? (mt.ctx - t0) : kUnit;
-      // causal limit: new token j sees unit rows < ctx - q_len + 1 + j - t0 (a prefix
-      // launch's columns are different sequences: no mask)
-      const int lim0 = MODE == kPrefix ? (1 << 30) : mt.ctx - a.q_len + 1 - t0;
-      if (MODE == kAppend && mt.newrow >= 0 && (mt.ctx - 1 - mt.tok0) / kUnit == cw) {
-        // fused append: this unit holds the newest token; its K/V rows come from the
-        // staging area (the cache row the TMA read may still be old) and are written to
-        // the cache
-        constexpr int CPR = D * 2 / 16;               // 16-byte chunks per row
-        const int rn = mt.ctx - 1 - mt.tok0;          // row in the stage tile
-        if (lane < 2 * CPR) {
-          const int kv = lane / CPR, ch = lane % CPR, hf = ch >> 3, cc = ch & 7;
-          const uint4 val = *reinterpret_cast<const uint4*>(smem + L::kNewOff + st * L::kNewBytes +
-                                                            kv * D * 2 + ch * 16);
-          *reinterpret_cast<uint4*>((kv ? sV : sK) + hf * (kTileTokens * 128) + rn * 128 +
-                                    ((cc ^ (rn & 7)) << 4)) = val;
-          T* cache = static_cast<T*>(const_cast<void*>(kv ? a.v_cache : a.k_cache));
-          *reinterpret_cast<uint4*>(cache + (long long)mt.newrow * D + ch * 8) = val;
-        }
-        __syncwarp();
-        patched = true;
-      }
-      const uint32_t kbase = smem_u32(sK), vbase = smem_u32(sV);
-      // ---- S^T[16 tokens][8*NT heads] = K_unit . q^T
-      float sacc[NT][4];
-#pragma unroll
-      for (int n = 0; n < NT; ++n) sacc[n][0] = sacc[n][1] = sacc[n][2] = sacc[n][3] = 0.f;
-      if constexpr (KV8) {
-        // one ldmatrix.x4 = rows 0-7 / 8-15 of two 16-byte chunks (k-steps ks, ks+1); a
-        // thread's 32 bits are 4 codes, dims 4c..4c+3 of its row, converted in two halves
-        const int j = lane >> 3, i = lane & 7;
-        const int r = cw * kUnit + (j & 1) * 8 + i;
-#pragma unroll
-        for (int ks = 0; ks < KS; ks += 2) {
-          const int chunk = ks + (j >> 1);
-          const uint32_t addr = kbase + r * 128 + ((chunk ^ (r & 7)) << 4);
-          uint32_t m0, m1, m2, m3;
-          ldsm_x4(addr, m0, m1, m2, m3);
-          uint32_t x0, x1, x2, x3, y0, y1, y2, y3;
-          e4m3x4_to_f16x2x2(m0, x0, x2);
-          e4m3x4_to_f16x2x2(m1, x1, x3);
-          e4m3x4_to_f16x2x2(m2, y0, y2);
-          e4m3x4_to_f16x2x2(m3, y1, y3);
-#pragma unroll
-          for (int n = 0; n < NT; ++n) {
-            mma16816<false>(sacc[n], x0, x1, x2, x3, qf[ks][n][0], qf[ks][n][1]);
-            mma16816<false>(sacc[n], y0, y1, y2, y3, qf[ks + 1][n][0], qf[ks + 1][n][1]);
+#pragma unroll 1
+    for (int uk = 0; uk < UPW; ++uk) {
+      const int u = kColSplit ? (cw >> 1) * 2 + uk : cw;   // unit of the stage
+      if (u < mt.nunits) {
+        const int t0 = mt.tok0 + u * kUnit;
+        const int valid = (mt.ctx - t0) < kUnit ? (mt.ctx - t0) : kUnit;
+        // causal limit: new token j sees unit rows < ctx - q_len + 1 + j - t0 (a prefix
+        // launch's columns are different sequences: no mask)
+        const int lim0 = MODE == kPrefix ? (1 << 30) : mt.ctx - a.q_len + 1 - t0;
+        if (MODE == kAppend && mt.newrow >= 0 && (mt.ctx - 1 - mt.tok0) / kUnit == u) {
+          // fused append: this unit holds the newest token; its K/V rows come from the
+          // staging area (the cache row the TMA read may still be old) and are written to
+          // the cache
+          constexpr int CPR = D * 2 / 16;               // 16-byte chunks per row
+          const int rn = mt.ctx - 1 - mt.tok0;          // row in the stage tile
+          if (lane < 2 * CPR) {
+            const int kv = lane / CPR, ch = lane % CPR, hf = ch >> 3, cc = ch & 7;
+            const uint4 val = *reinterpret_cast<const uint4*>(smem + L::kNewOff + st * L::kNewBytes +
+                                                              kv * D * 2 + ch * 16);
+            *reinterpret_cast<uint4*>((kv ? sV : sK) + hf * (kTileTokens * 128) + rn * 128 +
+                                      ((cc ^ (rn & 7)) << 4)) = val;
+            T* cache = static_cast<T*>(const_cast<void*>(kv ? a.v_cache : a.k_cache));
+            *reinterpret_cast<uint4*>(cache + (long long)mt.newrow * D + ch * 8) = val;
           }
+          __syncwarp();
+          patched = true;
         }
-      } else {
-        const int j = lane >> 3, i = lane & 7;
-        const int r = cw * kUnit + (j & 1) * 8 + i;
+        const uint32_t kbase = smem_u32(sK), vbase = smem_u32(sV);
+        // ---- S^T[16 tokens][8*NT heads] = K_unit . q^T
+        float sacc[NTW][4];
 #pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-          const int d = ks * 16 + (j >> 1) * 8;
-          const uint32_t addr =
-              kbase + (d >> 6) * (kTileTokens * 128) + r * 128 + ((((d & 63) >> 3) ^ (r & 7)) << 4);
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4(addr, a0, a1, a2, a3);
+        for (int n = 0; n < NTW; ++n) sacc[n][0] = sacc[n][1] = sacc[n][2] = sacc[n][3] = 0.f;
+        if constexpr (KV8) {
+          // one ldmatrix.x4 = rows 0-7 / 8-15 of two 16-byte chunks (k-steps ks, ks+1); a
+          // thread's 32 bits are 4 codes, dims 4c..4c+3 of its row, converted in two halves
+          const int j = lane >> 3, i = lane & 7;
+          const int r = u * kUnit + (j & 1) * 8 + i;
 #pragma unroll
-          for (int n = 0; n < NT; ++n) mma16816<kBF16>(sacc[n], a0, a1, a2, a3, qf[ks][n][0], qf[ks][n][1]);
-        }
-      }
-      // ---- online softmax (base 2) per query column
-      uint32_t bhi[NT][2], blo[NT][2];
+          for (int ks = 0; ks < KS; ks += 2) {
+            const int chunk = ks + (j >> 1);
+            const uint32_t addr = kbase + r * 128 + ((chunk ^ (r & 7)) << 4);
+            uint32_t m0, m1, m2, m3;
+            ldsm_x4(addr, m0, m1, m2, m3);
+            uint32_t x0, x1, x2, x3, y0, y1, y2, y3;
+            e4m3x4_to_f16x2x2(m0, x0, x2);
+            e4m3x4_to_f16x2x2(m1, x1, x3);
+            e4m3x4_to_f16x2x2(m2, y0, y2);
+            e4m3x4_to_f16x2x2(m3, y1, y3);
 #pragma unroll
-      for (int n = 0; n < NT; ++n) {
-        float xs[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int row = gid + (e >= 2 ? 8 : 0);
-          const int lim = lim0 + jcol[n][e & 1];
-          xs[e] = (row < valid && row < lim) ? sacc[n][e] * a.scale_log2 : -INFINITY;
-        }
-        float alpha[2], p[4];
-        bool grew = false;
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          float mx = fmaxf(xs[cc], xs[cc + 2]);
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-          const float mnew = fmaxf(m[n][cc], mx);
-          // a column with no visible row yet keeps max -inf: use 0 as the reference
-          const float mref = mnew == -INFINITY ? 0.f : mnew;
-          grew |= mnew != m[n][cc];
-          alpha[cc] = ex2(m[n][cc] - mref);
-          m[n][cc] = mnew;
-          p[cc] = ex2(xs[cc] - mref);
-          p[cc + 2] = ex2(xs[cc + 2] - mref);
-          l[n][cc] = l[n][cc] * alpha[cc] + p[cc] + p[cc + 2];
-        }
-        // 8-bit caches (ALU-bound): rescale O only when a column's running max moved in
-        // this warp (alpha is exactly 1 otherwise)
-        if (!KV8 || __any_sync(0xffffffffu, grew)) {
+            for (int n = 0; n < NTW; ++n) {
+              mma16816<false>(sacc[n], x0, x1, x2, x3, qf[ks][n][0], qf[ks][n][1]);
+              mma16816<false>(sacc[n], y0, y1, y2, y3, qf[ks + 1][n][0], qf[ks + 1][n][1]);
+            }
+          }
+        } else {
+          const int j = lane >> 3, i = lane & 7;
+          const int r = u * kUnit + (j & 1) * 8 + i;
 #pragma unroll
           for (int ks = 0; ks < KS; ++ks) {
-            o[ks][n][0] *= alpha[0];
-            o[ks][n][1] *= alpha[1];
-            o[ks][n][2] *= alpha[0];
-            o[ks][n][3] *= alpha[1];
+            const int d = ks * 16 + (j >> 1) * 8;
+            const uint32_t addr =
+                kbase + (d >> 6) * (kTileTokens * 128) + r * 128 + ((((d & 63) >> 3) ^ (r & 7)) << 4);
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(addr, a0, a1, a2, a3);
+#pragma unroll
+            for (int n = 0; n < NTW; ++n) mma16816<kBF16>(sacc[n], a0, a1, a2, a3, qf[ks][n][0], qf[ks][n][1]);
           }
         }
-        using TM = std::conditional_t<KV8, __half, T>;   // MMA operand type
-        const uint32_t h01 = pack2<TM>(p[0], p[1]), h23 = pack2<TM>(p[2], p[3]);
-        bhi[n][0] = movmatrix_t(h01);
-        bhi[n][1] = movmatrix_t(h23);
-        if constexpr (!KV8) {
-          // the rounding residual of P as a second 16-bit operand (~16 bits of P in all)
-          const float2 f01 = unpack2<TM>(h01), f23 = unpack2<TM>(h23);
-          const uint32_t l01 = pack2<TM>(p[0] - f01.x, p[1] - f01.y);
-          const uint32_t l23 = pack2<TM>(p[2] - f23.x, p[3] - f23.y);
-          blo[n][0] = movmatrix_t(l01);
-          blo[n][1] = movmatrix_t(l23);
-        } else {
-          blo[n][0] = blo[n][1] = 0u;   // fp16 P: 11 bits, next to 3-bit cache values
+        // ---- online softmax (base 2) per query column
+        uint32_t bhi[NTW][2], blo[NTW][2];
+#pragma unroll
+        for (int n = 0; n < NTW; ++n) {
+          float xs[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int row = gid + (e >= 2 ? 8 : 0);
+            const int lim = lim0 + jcol[n][e & 1];
+            xs[e] = (row < valid && row < lim) ? sacc[n][e] * a.scale_log2 : -INFINITY;
+          }
+          float alpha[2], p[4];
+          bool grew = false;
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            float mx = fmaxf(xs[cc], xs[cc + 2]);
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+            const float mnew = fmaxf(m[n][cc], mx);
+            // a column with no visible row yet keeps max -inf: use 0 as the reference
+            const float mref = mnew == -INFINITY ? 0.f : mnew;
+            grew |= mnew != m[n][cc];
+            alpha[cc] = ex2(m[n][cc] - mref);
+            m[n][cc] = mnew;
+            p[cc] = ex2(xs[cc] - mref);
+            p[cc + 2] = ex2(xs[cc + 2] - mref);
+            l[n][cc] = l[n][cc] * alpha[cc] + p[cc] + p[cc + 2];
+          }
+          // 8-bit caches (ALU-bound): rescale O only when a column's running max moved in
+          // this warp (alpha is exactly 1 otherwise)
+          if (!KV8 || __any_sync(0xffffffffu, grew)) {
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+              o[ks][n][0] *= alpha[0];
+              o[ks][n][1] *= alpha[1];
+              o[ks][n][2] *= alpha[0];
+              o[ks][n][3] *= alpha[1];
+            }
+          }
+          using TM = std::conditional_t<KV8, __half, T>;   // MMA operand type
+          const uint32_t h01 = pack2<TM>(p[0], p[1]), h23 = pack2<TM>(p[2], p[3]);
+          bhi[n][0] = movmatrix_t(h01);
+          bhi[n][1] = movmatrix_t(h23);
+          if constexpr (!KV8) {
+            // the rounding residual of P as a second 16-bit operand (~16 bits of P in all)
+            const float2 f01 = unpack2<TM>(h01), f23 = unpack2<TM>(h23);
+            const uint32_t l01 = pack2<TM>(p[0] - f01.x, p[1] - f01.y);
+            const uint32_t l23 = pack2<TM>(p[2] - f23.x, p[3] - f23.y);
+            blo[n][0] = movmatrix_t(l01);
+            blo[n][1] = movmatrix_t(l23);
+          } else {
+            blo[n][0] = blo[n][1] = 0u;   // fp16 P: 11 bits, next to 3-bit cache values
+          }
         }
-      }
-      // ---- O^T[D][8*NT] += V_unit^T . P^T
-      uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;   // token masks for V rows >= valid
-      if (valid < kUnit) {
-        const int t_a = 2 * tig, t_b = 8 + 2 * tig;
-        mlo = (t_a < valid ? 0x0000ffffu : 0u) | (t_a + 1 < valid ? 0xffff0000u : 0u);
-        mhi = (t_b < valid ? 0x0000ffffu : 0u) | (t_b + 1 < valid ? 0xffff0000u : 0u);
-      }
-      // the PV product; with 8-bit caches (ALU-bound) the token masks are applied only to
-      // a unit with fewer than 16 valid rows (a lambda instantiated with and without them)
-      auto pv = [&](auto masked) {
-        if constexpr (KV8) {
-          // ldmatrix.x4.trans of tokens 0-7 / 8-15 of two 16-byte chunks; a thread gets the
-          // codes of dims (2g, 2g+1) for tokens (2c, 2c+1): regrouped per dim they give the
-          // A fragments with M-row g = dim 2g and M-row g+8 = dim 2g+1 of the chunk
-          const int j = lane >> 3, i = lane & 7;
-          const int r = cw * kUnit + (j & 1) * 8 + i;
+        // ---- O^T[D][8*NT] += V_unit^T . P^T
+        uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;   // token masks for V rows >= valid
+        if (valid < kUnit) {
+          const int t_a = 2 * tig, t_b = 8 + 2 * tig;
+          mlo = (t_a < valid ? 0x0000ffffu : 0u) | (t_a + 1 < valid ? 0xffff0000u : 0u);
+          mhi = (t_b < valid ? 0x0000ffffu : 0u) | (t_b + 1 < valid ? 0xffff0000u : 0u);
+        }
+        // the PV product; with 8-bit caches (ALU-bound) the token masks are applied only to
+        // a unit with fewer than 16 valid rows (a lambda instantiated with and without them)
+        auto pv = [&](auto masked) {
+          if constexpr (KV8) {
+            // ldmatrix.x4.trans of tokens 0-7 / 8-15 of two 16-byte chunks; a thread gets the
+            // codes of dims (2g, 2g+1) for tokens (2c, 2c+1): regrouped per dim they give the
+            // A fragments with M-row g = dim 2g and M-row g+8 = dim 2g+1 of the chunk
+            const int j = lane >> 3, i = lane & 7;
+            const int r = u * kUnit + (j & 1) * 8 + i;
 #pragma unroll
-          for (int mtile = 0; mtile < KS; mtile += 2) {
-            const int chunk = mtile + (j >> 1);
-            const uint32_t addr = vbase + r * 128 + ((chunk ^ (r & 7)) << 4);
-            uint32_t m[4];
-            ldsm_x4_t(addr, m[0], m[1], m[2], m[3]);
+            for (int mtile = 0; mtile < KS; mtile += 2) {
+              const int chunk = mtile + (j >> 1);
+              const uint32_t addr = vbase + r * 128 + ((chunk ^ (r & 7)) << 4);
+              uint32_t m[4];
+              ldsm_x4_t(addr, m[0], m[1], m[2], m[3]);
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              const uint32_t p0 = __byte_perm(m[2 * hh], 0u, 0x3120);       // tokens 2c, 2c+1
-              const uint32_t p1 = __byte_perm(m[2 * hh + 1], 0u, 0x3120);   // tokens 8+2c, ...
+              for (int hh = 0; hh < 2; ++hh) {
+                const uint32_t p0 = __byte_perm(m[2 * hh], 0u, 0x3120);       // tokens 2c, 2c+1
+                const uint32_t p1 = __byte_perm(m[2 * hh + 1], 0u, 0x3120);   // tokens 8+2c, ...
+                uint32_t a0, a1, a2, a3;
+                e4m3x4_to_f16x2x2(p0, a0, a1);
+                e4m3x4_to_f16x2x2(p1, a2, a3);
+                if constexpr (decltype(masked)::value) {
+                  a0 &= mlo;
+                  a1 &= mlo;
+                  a2 &= mhi;
+                  a3 &= mhi;
+                }
+#pragma unroll
+                for (int n = 0; n < NTW; ++n)
+                  mma16816<false>(o[mtile + hh][n], a0, a1, a2, a3, bhi[n][0], bhi[n][1]);
+              }
+            }
+          } else {
+            const int j = lane >> 3, i = lane & 7;
+            const int r = u * kUnit + (j >> 1) * 8 + i;
+#pragma unroll
+            for (int mtile = 0; mtile < KS; ++mtile) {
+              const int d = mtile * 16 + (j & 1) * 8;
+              const uint32_t addr =
+                  vbase + (d >> 6) * (kTileTokens * 128) + r * 128 + ((((d & 63) >> 3) ^ (r & 7)) << 4);
               uint32_t a0, a1, a2, a3;
-              e4m3x4_to_f16x2x2(p0, a0, a1);
-              e4m3x4_to_f16x2x2(p1, a2, a3);
+              ldsm_x4_t(addr, a0, a1, a2, a3);
               if constexpr (decltype(masked)::value) {
                 a0 &= mlo;
                 a1 &= mlo;
@@ -1033,45 +1066,25 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
                 a3 &= mhi;
               }
 #pragma unroll
-              for (int n = 0; n < NT; ++n)
-                mma16816<false>(o[mtile + hh][n], a0, a1, a2, a3, bhi[n][0], bhi[n][1]);
+              for (int n = 0; n < NTW; ++n) {
+                mma16816<kBF16>(o[mtile][n], a0, a1, a2, a3, bhi[n][0], bhi[n][1]);
+                mma16816<kBF16>(o[mtile][n], a0, a1, a2, a3, blo[n][0], blo[n][1]);
+              }
             }
           }
+        };
+        if constexpr (KV8) {
+          if (valid < kUnit) pv(std::true_type{});
+          else pv(std::false_type{});
         } else {
-          const int j = lane >> 3, i = lane & 7;
-          const int r = cw * kUnit + (j >> 1) * 8 + i;
-#pragma unroll
-          for (int mtile = 0; mtile < KS; ++mtile) {
-            const int d = mtile * 16 + (j & 1) * 8;
-            const uint32_t addr =
-                vbase + (d >> 6) * (kTileTokens * 128) + r * 128 + ((((d & 63) >> 3) ^ (r & 7)) << 4);
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4_t(addr, a0, a1, a2, a3);
-            if constexpr (decltype(masked)::value) {
-              a0 &= mlo;
-              a1 &= mlo;
-              a2 &= mhi;
-              a3 &= mhi;
-            }
-#pragma unroll
-            for (int n = 0; n < NT; ++n) {
-              mma16816<kBF16>(o[mtile][n], a0, a1, a2, a3, bhi[n][0], bhi[n][1]);
-              mma16816<kBF16>(o[mtile][n], a0, a1, a2, a3, blo[n][0], blo[n][1]);
-            }
-          }
+          pv(std::true_type{});
         }
-      };
-      if constexpr (KV8) {
-        if (valid < kUnit) pv(std::true_type{});
-        else pv(std::false_type{});
-      } else {
-        pv(std::true_type{});
       }
     }
     if (mt.flags & F_LAST) {
       // ---- merge the four warps' (m, l, O) for this segment portion
 #pragma unroll
-      for (int n = 0; n < NT; ++n)
+      for (int n = 0; n < NTW; ++n)
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
           float v = l[n][cc];
@@ -1082,19 +1095,27 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
         }
       named_bar_sync(1, kConsumerThreads);         // all warps are done with this stage's K/V
       float* scr = reinterpret_cast<float*>(sK);   // K and V tiles reused as scratch
+      // every warp stores all NT n-tiles; one it does not hold is empty (-inf, 0, zeros)
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks)
 #pragma unroll
         for (int n = 0; n < NT; ++n)
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            scr[(cw * NREG + (ks * NT + n) * 4 + e) * 32 + lane] = o[ks][n][e];
+          for (int e = 0; e < 4; ++e) {
+            const int w = n - nb;
+            scr[(cw * NREG + (ks * NT + n) * 4 + e) * 32 + lane] =
+                (w >= 0 && w < NTW) ? o[ks][w < NTW ? w : 0][e] : 0.f;
+          }
       if (gid == 0) {
 #pragma unroll
         for (int n = 0; n < NT; ++n)
 #pragma unroll
-          for (int cc = 0; cc < 2; ++cc)
-            mls[cw * kMaxGroup + n * 8 + 2 * tig + cc] = make_float2(m[n][cc], l[n][cc]);
+          for (int cc = 0; cc < 2; ++cc) {
+            const int w = n - nb;
+            mls[cw * kMaxGroup + n * 8 + 2 * tig + cc] =
+                (w >= 0 && w < NTW) ? make_float2(m[w < NTW ? w : 0][cc], l[w < NTW ? w : 0][cc])
+                                    : make_float2(-INFINITY, 0.f);
+          }
       }
       named_bar_sync(1, kConsumerThreads);
       const bool complete = mt.flags & F_COMPLETE;
