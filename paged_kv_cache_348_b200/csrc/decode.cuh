@@ -809,11 +809,9 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
   constexpr int KS = D / 16;            // k-steps of QK, m-tiles of PV
   constexpr int NREG = KS * NT * 4;     // O^T accumulator registers per thread (all n-tiles)
   // With 16 query columns (NT = 2) a warp holding both n-tiles of O and q runs out of
-  // registers (spills in the unit loop), so with 16-bit caches the warps of a pair split
-  // the columns: warp cw takes n-tile cw & 1 of units 2 (cw >> 1) and 2 (cw >> 1) + 1 of
-  // every stage.  The fused append keeps one unit per warp (its patched row is written
-  // by the warp of its unit), as do 8-bit caches.
-  constexpr bool kColSplit = NT == 2 && !KV8 && MODE != kAppend;
+  // registers (spills in the unit loop), so the warps of a pair split the columns: warp
+  // cw takes n-tile cw & 1 of units 2 (cw >> 1) and 2 (cw >> 1) + 1 of every stage.
+  constexpr bool kColSplit = NT == 2;
   constexpr int NTW = kColSplit ? 1 : NT;       // n-tiles a warp holds
   constexpr int UPW = kColSplit ? 2 : 1;        // units a warp takes per stage
   const int nb = kColSplit ? (cw & 1) : 0;      // its first n-tile
@@ -898,7 +896,8 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
         if (MODE == kAppend && mt.newrow >= 0 && (mt.ctx - 1 - mt.tok0) / kUnit == u) {
           // fused append: this unit holds the newest token; its K/V rows come from the
           // staging area (the cache row the TMA read may still be old) and are written to
-          // the cache
+          // the cache.  With split columns both warps of the unit patch their tile copy
+          // with the same bytes before reading it; the first writes the cache row.
           constexpr int CPR = D * 2 / 16;               // 16-byte chunks per row
           const int rn = mt.ctx - 1 - mt.tok0;          // row in the stage tile
           if (lane < 2 * CPR) {
@@ -907,8 +906,10 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
                                                               kv * D * 2 + ch * 16);
             *reinterpret_cast<uint4*>((kv ? sV : sK) + hf * (kTileTokens * 128) + rn * 128 +
                                       ((cc ^ (rn & 7)) << 4)) = val;
-            T* cache = static_cast<T*>(const_cast<void*>(kv ? a.v_cache : a.k_cache));
-            *reinterpret_cast<uint4*>(cache + (long long)mt.newrow * D + ch * 8) = val;
+            if (nb == 0) {
+              T* cache = static_cast<T*>(const_cast<void*>(kv ? a.v_cache : a.k_cache));
+              *reinterpret_cast<uint4*>(cache + (long long)mt.newrow * D + ch * 8) = val;
+            }
           }
           __syncwarp();
           patched = true;
