@@ -807,7 +807,6 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
   const int gid = lane >> 2, tig = lane & 3;
   const int tid = cw * 32 + lane;
   constexpr int KS = D / 16;            // k-steps of QK, m-tiles of PV
-  constexpr int NREG = KS * NT * 4;     // O^T accumulator registers per thread (all n-tiles)
   // With 16 query columns (NT = 2) a warp holding both n-tiles of O and q runs out of
   // registers (spills in the unit loop), so the warps of a pair split the columns: warp
   // cw takes n-tile cw & 1 of units 2 (cw >> 1) and 2 (cw >> 1) + 1 of every stage.
@@ -815,6 +814,10 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
   constexpr int NTW = kColSplit ? 1 : NT;       // n-tiles a warp holds
   constexpr int UPW = kColSplit ? 2 : 1;        // units a warp takes per stage
   const int nb = kColSplit ? (cw & 1) : 0;      // its first n-tile
+  constexpr int NREGW = KS * NTW * 4;           // O^T accumulator registers a thread holds
+  // the end-of-portion merge stages every warp's O in the stage's K and V tiles
+  static_assert(kConsumerWarps * NREGW * 32 * 4 <= 2 * L::kKvBytes,
+                "merge scratch must fit in the stage's K and V tiles");
   float o[KS][NTW][4];
   float m[NTW][2], l[NTW][2];
   uint32_t qf[KS][NTW][2];
@@ -1096,17 +1099,15 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
         }
       named_bar_sync(1, kConsumerThreads);         // all warps are done with this stage's K/V
       float* scr = reinterpret_cast<float*>(sK);   // K and V tiles reused as scratch
-      // every warp stores all NT n-tiles; one it does not hold is empty (-inf, 0, zeros)
+      // every warp stores the n-tiles it holds; its (max, sum) of a column it does not
+      // hold is empty (-inf, 0)
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks)
 #pragma unroll
-        for (int n = 0; n < NT; ++n)
+        for (int n = 0; n < NTW; ++n)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int w = n - nb;
-            scr[(cw * NREG + (ks * NT + n) * 4 + e) * 32 + lane] =
-                (w >= 0 && w < NTW) ? o[ks][w < NTW ? w : 0][e] : 0.f;
-          }
+          for (int e = 0; e < 4; ++e)
+            scr[(cw * NREGW + (ks * NTW + n) * 4 + e) * 32 + lane] = o[ks][n][e];
       if (gid == 0) {
 #pragma unroll
         for (int n = 0; n < NT; ++n)
@@ -1121,12 +1122,13 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
       named_bar_sync(1, kConsumerThreads);
       const bool complete = mt.flags & F_COMPLETE;
       const bool has_prefix = MODE == kSuffix && complete && a.seq_start[mt.seq] > 0;
-      // Thread tid of warp cw holds, in scr, accumulator register e = cw of every (ks, n)
-      // tile of lane `lane`: query column h_n = n*8 + 2*(lane%4) + cw%2 and head dim
-      // d = ks*16 + lane/4 + 8*(cw/2).  So the column statistics (max, weights, sum)
-      // are computed once per n, and the loop over the dims only sums and stores.
-      constexpr int kIt = NREG * 32 / kConsumerThreads;   // accumulator values per thread
-      static_assert(kIt == KS * NT, "one value per (ks, n) tile");
+      // Thread tid of warp cw combines accumulator register e = cw of every (ks, n) tile of
+      // lane `lane` over the warps holding n-tile n: query column h_n = n*8 + 2*(lane%4) +
+      // cw%2 and head dim d = ks*16 + lane/4 + 8*(cw/2).  So the column statistics (max,
+      // weights, sum) are computed once per n, and the loop over the dims only sums and
+      // stores.
+      constexpr int kIt = KS * NT;                  // accumulator values per thread
+      static_assert(kConsumerWarps == 4, "register e of a tile is combined by warp e");
       float cM[NT], cL[NT], cs[NT][kConsumerWarps];
       long long crow[NT];
 #pragma unroll
@@ -1168,10 +1170,13 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
         // head dim of this accumulator value (8-bit caches order the PV rows 2g, 2g+1)
         const int d = ks * 16 + (KV8 ? 2 * (lane >> 2) + (cw >= 2 ? 1 : 0)
                                      : (lane >> 2) + (cw >= 2 ? 8 : 0));
-        const int r = cw + 4 * it;                   // scr register row of this value
         float acc = 0.f;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) acc += scr[(w * NREG + r) * 32 + lane] * cs[n][w];
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          const int nl = n - (kColSplit ? (w & 1) : 0);    // n-tile n in warp w's registers
+          if (nl >= 0 && nl < NTW)
+            acc += scr[(w * NREGW + (ks * NTW + nl) * 4 + cw) * 32 + lane] * cs[n][w];
+        }
         if (complete) {
           // column h = new token (or chunk member) h / group, head kvh * group + h % group;
           // a row that sees no token at all (a new token before the context start) is zero

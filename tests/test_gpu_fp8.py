@@ -135,3 +135,21 @@ def test_e4m3_llama70b_shape_step_full_size():
                                     b.context_lens.cpu().numpy(), b.scale, "bf16",
                                     nthreads=NTHREADS)
         assert_attn_close(b.out[l], ref, what="70B e4m3 layer %d" % l)
+
+
+def test_e4m3_group16_llama70b_shape_full_size():
+    """16 query rows per kv head with 8-bit pools at full size (128 q / 8 kv heads, the
+    70B-shape lengths): the warp pairs' split columns and the end-of-portion merge of
+    every ring slot, every sequence checked."""
+    import dataclasses
+    w = dataclasses.replace(inputs.LLAMA70B, num_q_heads=128)
+    b = wl.build(w, layers=1, kv8=True)
+    wl.decode_layer(b, 0)
+    torch.cuda.synchronize()
+    assert int(b.status.item()) == 0
+    ks, vs = b.kv_scales
+    ref, _ = oracle.decode_e4m3(bits(b.q[0]), b.k_caches[0].cpu().numpy(),
+                                b.v_caches[0].cpu().numpy(), ks, vs,
+                                b.block_tables.cpu().numpy(), b.context_lens.cpu().numpy(),
+                                b.scale, "bf16", nthreads=NTHREADS)
+    assert_attn_close(b.out[0], ref, what="70B-shape group 16 e4m3")

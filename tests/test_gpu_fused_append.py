@@ -99,3 +99,21 @@ def test_fused_append_bad_block_id_is_flagged_and_not_written():
     assert torch.equal(sep[1].view(torch.int16), fused[1].view(torch.int16))
     assert torch.equal(sep[2].view(torch.int16), fused[2].view(torch.int16))
     assert torch.equal(sep[0][[0, 2]].view(torch.int16), fused[0][[0, 2]].view(torch.int16))
+
+
+def test_fused_append_group16_llama70b_shape_full_size():
+    """pa_decode_append with 16 query rows per kv head (128 q / 8 kv heads) at full size:
+    both warps of the newest token's unit patch their tile, one writes the cache."""
+    import dataclasses
+    w = dataclasses.replace(inputs.LLAMA70B, num_q_heads=128)
+    b = wl.build(w, layers=1)
+    hk, hv = bits(b.k_caches[0]), bits(b.v_caches[0])
+    pk.pa_decode_append(b.out[0], b.q[0], b.k_caches[0], b.v_caches[0], b.k_new[0], b.v_new[0],
+                        b.block_tables, b.context_lens, b.scale, b.workspace, b.status)
+    torch.cuda.synchronize()
+    assert int(b.status.item()) == 0
+    oracle.cache_append(hk, hv, bits(b.k_new[0]), bits(b.v_new[0]), b.slot_mapping.cpu().numpy())
+    assert np.array_equal(bits(b.k_caches[0]), hk) and np.array_equal(bits(b.v_caches[0]), hv)
+    ref, _ = oracle.decode(bits(b.q[0]), hk, hv, b.block_tables.cpu().numpy(),
+                           b.context_lens.cpu().numpy(), b.scale, "bf16", nthreads=8)
+    assert_attn_close(b.out[0], ref, what="70B-shape group 16 fused append")
