@@ -70,7 +70,7 @@ constexpr int DEV_BAD_BLOCK_ID = 0x1;
 constexpr int DEV_BAD_CONTEXT_LEN = 0x8;
 constexpr int DEV_TIMEOUT = 0x10;
 
-enum : int { F_FIRST = 1, F_LAST = 2, F_END = 4, F_COMPLETE = 8 };
+enum : int { F_FIRST = 1, F_LAST = 2, F_END = 4, F_COMPLETE = 8, F_PREFIX = 16 };
 
 // What a launch decodes (a template parameter, so the plain path carries none of the rest):
 //  kPlain   -- every sequence over its cached tokens 0..ctx-1; q_len new tokens, causal.
@@ -95,7 +95,8 @@ struct SeqSpan {
 
 // A segment portion this CTA shares with other CTAs, handed to the merger warp.
 struct SplitDesc {
-  int seq, kvh, cf, cl, ncontrib, pad;  // first/last CTA of the segment, CTAs with units
+  int seq, kvh, cf, cl, ncontrib;       // first/last CTA of the segment, CTAs with units
+  int has_prefix;                       // kSuffix: the sequence has a prefix partial
   long long seg0;                       // first unit of the segment
 };
 
@@ -414,7 +415,7 @@ __device__ __forceinline__ void merge_split(const DecodeArgs& a, const SplitDesc
         M[e] = mn;
       }
   }
-  const bool has_prefix = MODE == kSuffix && a.seq_start[dsc.seq] > 0;
+  const bool has_prefix = MODE == kSuffix && dsc.has_prefix;
   float2 xm[kPer];
   float4 xa[kPer];
 #pragma unroll
@@ -572,6 +573,11 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
       long long x = start;
       const long long xend = end;
       int s_cur = s_a, u_cur = u_a, ctx_cur = ctx_a, first_cur = first_a;
+      // the table window at the start of sequence s_win's segments, kept for its next kv
+      // head (whose segment starts at the same token), so only a CTA's first portion of a
+      // sequence waits on table reads
+      int s_win = -1, sw0 = 0, sw1 = 0, sn0 = 0, sn1 = 0;
+      const int32_t* s_trow = a.block_tables;
       long long pbase = pb_a;
       while (ok && x < xend) {
         while (x >= pbase + (long long)Hkv * u_cur) {   // next sequence with units
@@ -595,21 +601,40 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
             int ncontrib = 0;
             for (int cc = cf; cc <= cl; ++cc)
               ncontrib += cta_start(cc, total, G) < cta_start(cc + 1, total, G);
-            desc[qslot] = SplitDesc{s_cur, kvh, cf, cl, ncontrib, 0, seg0};
+            desc[qslot] = SplitDesc{s_cur, kvh, cf, cl, ncontrib, first_cur > 0 ? 1 : 0, seg0};
           }
         }
         // Block-table window: lane l holds entries wb+l, wb+32+l (w0, w1) and the next 64
         // entries (n0, n1), loaded 64 blocks before they are needed, so no stage waits on a
         // table read except the portion's first.
-        // a chunk of a prefix launch reads the prefix through its first member's table
-        const long long trow_seq = MODE == kPrefix ? (long long)chunk_member(a, s_cur, 0) : s_cur;
-        const int32_t* trow = a.block_tables + trow_seq * a.max_blocks;
         const int nblk = (ctx_cur + BS - 1) / BS;
         int wb = (first_cur + (int)(x - seg0) * kUnit) / BS;
-        int w0 = wb + lane < nblk ? trow[wb + lane] : -1;
-        int w1 = wb + 32 + lane < nblk ? trow[wb + 32 + lane] : -1;
-        int n0 = wb + 64 + lane < nblk ? trow[wb + 64 + lane] : -1;
-        int n1 = wb + 96 + lane < nblk ? trow[wb + 96 + lane] : -1;
+        const int32_t* trow;
+        int w0, w1, n0, n1;
+        if (x == seg0 && s_cur == s_win) {            // warp-uniform
+          trow = s_trow;
+          w0 = sw0;
+          w1 = sw1;
+          n0 = sn0;
+          n1 = sn1;
+        } else {
+          // a chunk of a prefix launch reads the prefix through its first member's table
+          const long long trow_seq =
+              MODE == kPrefix ? (long long)chunk_member(a, s_cur, 0) : s_cur;
+          trow = a.block_tables + trow_seq * a.max_blocks;
+          w0 = wb + lane < nblk ? trow[wb + lane] : -1;
+          w1 = wb + 32 + lane < nblk ? trow[wb + 32 + lane] : -1;
+          n0 = wb + 64 + lane < nblk ? trow[wb + 64 + lane] : -1;
+          n1 = wb + 96 + lane < nblk ? trow[wb + 96 + lane] : -1;
+          if (x == seg0) {
+            s_win = s_cur;
+            s_trow = trow;
+            sw0 = w0;
+            sw1 = w1;
+            sn0 = n0;
+            sn1 = n1;
+          }
+        }
         for (long long tu = x; tu < pe; tu += kUnitsPerStage) {
           const int nun = (int)((pe - tu) < kUnitsPerStage ? (pe - tu) : kUnitsPerStage);
           const int tok0 = first_cur + (int)(tu - seg0) * kUnit;
@@ -621,7 +646,8 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
             n1 = wb + 96 + lane < nblk ? trow[wb + 96 + lane] : -1;
           }
           const int flags = (tu == x ? F_FIRST : 0) | (tu + kUnitsPerStage >= pe ? F_LAST : 0) |
-                            (complete ? F_COMPLETE : 0);
+                            (complete ? F_COMPLETE : 0) |
+                            (MODE == kSuffix && first_cur > 0 ? F_PREFIX : 0);
           // the query rows of this kv head: group consecutive heads of each new token,
           // one bulk copy per token, stored as columns c = token * group + head
           const uint32_t qrow_bytes = (uint32_t)(group * D * 2);
@@ -633,7 +659,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
           auto qrow_src = [&](int jq) -> const T* {
             if constexpr (MODE == kPrefix) {
               int mem = chunk_member(a, s_cur, jq);
-              if (mem < 0) mem = (int)trow_seq;
+              if (mem < 0) mem = (int)((trow - a.block_tables) / a.max_blocks);   // first member
               return static_cast<const T*>(a.q) +
                      ((long long)mem * a.num_q_heads + (long long)kvh * group) * D;
             } else {
@@ -1121,7 +1147,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
       }
       named_bar_sync(1, kConsumerThreads);
       const bool complete = mt.flags & F_COMPLETE;
-      const bool has_prefix = MODE == kSuffix && complete && a.seq_start[mt.seq] > 0;
+      const bool has_prefix = MODE == kSuffix && complete && (mt.flags & F_PREFIX);
       // Thread tid of warp cw combines accumulator register e = cw of every (ks, n) tile of
       // lane `lane` over the warps holding n-tile n: query column h_n = n*8 + 2*(lane%4) +
       // cw%2 and head dim d = ks*16 + lane/4 + 8*(cw/2).  So the column statistics (max,
