@@ -49,6 +49,12 @@
 namespace pkv {
 
 constexpr int kUnit = 16;                           // tokens per schedule unit
+// Schedule weight of a segment beyond its units: a portion's fixed cost (first stage,
+// end-of-portion merge) is worth about this many units of streaming, so a CTA whose range
+// holds many short segments gets fewer units.  The weight is a tail of virtual units after
+// each segment's real ones; ranges that fall on it do no work.  With block_size 1 a unit
+// costs more (the producer issues a copy per 16 bytes), so the tail is shorter.
+__host__ __device__ constexpr int seg_weight(int bs) { return bs == 1 ? 2 : 8; }
 constexpr int kConsumerWarps = 4;
 constexpr int kUnitsPerStage = kConsumerWarps;      // one unit per consumer warp
 constexpr int kTileTokens = kUnit * kUnitsPerStage; // 64 tokens per stage
@@ -448,6 +454,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
                            const __grid_constant__ CUtensorMap tmv) {
   using L = Layout<D, KV8, ctas_per_sm(KV8, NT, BS)>;
   constexpr int kStages = L::kStages;
+  constexpr int kSegW = seg_weight(BS);
   static_assert(!KV8 || (D == 128 && MODE == kPlain), "8-bit caches: head_dim 128, plain decode");
   // MMA operand type: the cache's 16-bit type, or fp16 for E4M3 (exact there)
   constexpr bool kBF16 = !KV8 && std::is_same_v<T, __nv_bfloat16>;
@@ -500,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
       if (s < B) sp = span_of<MODE>(a, s, c == 0 ? a.status : nullptr);
       const int ctx = sp.ctx;
       const int u = (ctx - sp.first + kUnit - 1) / kUnit;
-      int x = u;
+      int x = u ? u + kSegW : 0;                     // weight of each of its segments
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, x, o);
@@ -540,14 +547,15 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
           ctx = sp.ctx;
           first = sp.first;
           u = (ctx - first + kUnit - 1) / kUnit;
-          x = u;
+          x = u ? u + kSegW : 0;
 #pragma unroll
           for (int o = 1; o < 32; o <<= 1) {
             const int y = __shfl_up_sync(0xffffffffu, x, o);
             if (lane >= o) x += y;
           }
         }
-        const long long lo = (long long)Hkv * (r2 + x - u), hi = (long long)Hkv * (r2 + x);
+        const int wt = u ? u + kSegW : 0;
+        const long long lo = (long long)Hkv * (r2 + x - wt), hi = (long long)Hkv * (r2 + x);
         const unsigned ha = __ballot_sync(0xffffffffu, s < B && u > 0 && lo <= start && start < hi);
         if (ha) {
           const int src = __ffs(ha) - 1;
@@ -580,16 +588,22 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
       const int32_t* s_trow = a.block_tables;
       long long pbase = pb_a;
       while (ok && x < xend) {
-        while (x >= pbase + (long long)Hkv * u_cur) {   // next sequence with units
-          pbase += (long long)Hkv * u_cur;
+        // a segment spans u_cur units and then kSegW virtual ones (weight w_cur)
+        while (x >= pbase + (long long)Hkv * (u_cur ? u_cur + kSegW : 0)) {   // next sequence
+          pbase += (long long)Hkv * (u_cur ? u_cur + kSegW : 0);
           ++s_cur;
           const SeqSpan sp = span_of<MODE>(a, s_cur, nullptr);
           ctx_cur = sp.ctx;
           if constexpr (MODE == kSuffix) first_cur = sp.first;
           u_cur = (ctx_cur - first_cur + kUnit - 1) / kUnit;
         }
-        const int kvh = (int)((x - pbase) / u_cur);
-        const long long seg0 = pbase + (long long)kvh * u_cur, seg1 = seg0 + u_cur;
+        const int w_cur = u_cur + kSegW;
+        const int kvh = (int)((x - pbase) / w_cur);
+        const long long seg0 = pbase + (long long)kvh * w_cur, seg1 = seg0 + u_cur;
+        if (x >= seg1) {                              // on the segment's virtual tail
+          x = seg0 + w_cur;
+          continue;
+        }
         const long long pe = seg1 < xend ? seg1 : xend;
         const bool complete = seg0 >= start && seg1 <= end;
         const int pidx = c * 2 + (start < seg0 ? 1 : 0);
@@ -808,7 +822,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
             ph ^= 1u;
           }
         }
-        x = pe;
+        x = pe == seg1 ? seg0 + w_cur : pe;          // past the virtual tail
       }
     }
     if (ok) ok = mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, kWaitLimitNs);
