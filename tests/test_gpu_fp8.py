@@ -153,3 +153,24 @@ def test_e4m3_group16_llama70b_shape_full_size():
                                 b.block_tables.cpu().numpy(), b.context_lens.cpu().numpy(),
                                 b.scale, "bf16", nthreads=NTHREADS)
     assert_attn_close(b.out[0], ref, what="70B-shape group 16 e4m3")
+
+
+@pytest.mark.parametrize("bs", [1, 16])
+def test_e4m3_heavytail_sampled(bs):
+    """The heavy-tailed batch with 8-bit pools at full size (256 sequences, lognormal
+    lengths up to the clip): the quantising append then decode, sequences sampled."""
+    b = wl.build(inputs.HEAVYTAIL, block_size=bs, kv8=True)
+    hk, hv = b.k_caches[0].cpu().numpy().copy(), b.v_caches[0].cpu().numpy().copy()
+    wl.run_step(b)
+    torch.cuda.synchronize()
+    assert int(b.status.item()) == 0
+    ks, vs = b.kv_scales
+    oracle.cache_append_e4m3(hk, hv, bits(b.k_new[0]), bits(b.v_new[0]),
+                             b.slot_mapping.cpu().numpy(), "f16", ks, vs)
+    assert np.array_equal(b.k_caches[0].cpu().numpy(), hk)
+    assert np.array_equal(b.v_caches[0].cpu().numpy(), hv)
+    ctx = b.context_lens.cpu().numpy()
+    items = sorted(set([int(i) for i in np.argsort(ctx)[-4:]] + list(range(0, 256, 23))))
+    ref, _ = oracle.decode_e4m3(bits(b.q[0]), hk, hv, ks, vs, b.block_tables.cpu().numpy(), ctx,
+                                b.scale, "f16", items=items, nthreads=NTHREADS)
+    assert_attn_close(b.out[0], ref, rows=items, what="heavytail e4m3 bs%d" % bs)

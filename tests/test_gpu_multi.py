@@ -119,3 +119,23 @@ def test_multi_llama8b_shape_four_new_tokens_full_size():
                                  b.block_tables.cpu().numpy(), b.context_lens.cpu().numpy(),
                                  b.scale, "f16", nthreads=NTHREADS)
     assert_attn_close(out, ref, what="llama8b q_len 4")
+
+
+def test_multi_llama70b_shape_two_new_tokens_two_layers_sampled():
+    """The bench's q_len-2 step at full size (70B shape, 16 query rows per kv head, warp
+    pairs splitting the columns): 2 layers through run_step, sequences sampled."""
+    b = wl.build(inputs.LLAMA70B, layers=2, q_len=2)
+    pre = [(bits(b.k_caches[l]), bits(b.v_caches[l])) for l in range(2)]
+    wl.run_step(b)
+    torch.cuda.synchronize()
+    assert int(b.status.item()) == 0
+    items = [0, 5, 11, 17, 23, 31]
+    for l in range(2):
+        hk, hv = pre[l]
+        oracle.cache_append(hk, hv, bits(b.k_new[l]), bits(b.v_new[l]),
+                            b.slot_mapping.cpu().numpy())
+        assert np.array_equal(bits(b.k_caches[l]), hk) and np.array_equal(bits(b.v_caches[l]), hv)
+        ref, _ = oracle.decode_multi(bits(b.q[l]), hk, hv, b.block_tables.cpu().numpy(),
+                                     b.context_lens.cpu().numpy(), b.scale, "bf16", items=items,
+                                     nthreads=NTHREADS)
+        assert_attn_close(b.out[l], ref, rows=items, what="70B q_len 2 layer %d" % l)
