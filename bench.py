@@ -36,6 +36,24 @@ METRIC = "paged decode attn: KV-read HBM GB/s (% of B200 peak) and seq-steps/s"
 FALLBACK_HBM_GBS = 6650.0
 
 
+def max_over_ranks(x: float, world: int, device="cuda") -> float:
+    """The largest x over all ranks of the process group (x itself with one rank): the
+    slowest rank's time is the job's time."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_gbs(world: int, bytes_per_rank_step: int, ms_per_step: float) -> float:
+    """Whole-job rate: every rank's bytes of one step over the (slowest rank's) step time."""
+    return world * bytes_per_rank_step / (ms_per_step * 1e-3) / 1e9
+
+
 def workload_desc(w, bs, layers=0, q_len=1):
     from paged_kv_cache_348_b200 import inputs
 
@@ -344,15 +362,12 @@ def main():
             ev_e[s * L + l].record(stream)
     barrier()
     dec_ms = [a.elapsed_time(e) for a, e in zip(ev_s, ev_e)]
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world)
     st = int(b.status.item())
     if st:
         raise RuntimeError("device status 0x%x in the timed region" % st)
     ms_step = ms / args.steps
-    value = world * kv_step / (ms_step * 1e-3) / 1e9
+    value = job_gbs(world, kv_step, ms_step)
     peak, peak_kind = measured_hbm_peak()
     dec_avg_events = statistics.mean(dec_ms)
     only_decode = fused and not (b.cow_pairs is not None and b.cow_pairs.shape[0])
@@ -519,15 +534,9 @@ def run_e2e(b, args, world, kv_step, fused=False):
     comp.wait_event(ev_out[L - 1])
     e.record(comp)
     torch.cuda.synchronize()
-    ms = s.elapsed_time(e)
-    if world > 1:
-        import torch.distributed as dist
-
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(s.elapsed_time(e), world)
     ms_step = ms / args.steps
-    return {"value": world * kv_step / (ms_step * 1e-3) / 1e9, "unit": "GB/s",
+    return {"value": job_gbs(world, kv_step, ms_step), "unit": "GB/s",
             "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,
             "ms_per_step": ms_step,
             "copies": "pinned host buffers; uploads and read-backs on two copy streams, "
