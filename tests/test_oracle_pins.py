@@ -336,3 +336,79 @@ def test_cow_fork_phase_copies_the_shared_partial_block():
     b = bm2.fork(a)
     s1, c1 = bm2.append_slot(b)
     assert c1 is None and s1 % bs == 0 and bm2.tables[b][:2] == bm2.tables[a][:2]
+
+
+# ---- RefBlockManager.release, pinned on its own: "PagedAttention in Production",
+# "Core Principle" (a finished request's blocks go back to the pool) and "Paged Attention
+# and Memory Efficiency in Production LLM Serving", "How PagedAttention borrows OS
+# paging" (shared blocks stay while any sharer holds them).
+
+def test_release_of_a_fork_keeps_the_shared_blocks():
+    bm = RefBlockManager(10, 4)
+    a = bm.new_seq(10)                                   # 3 blocks: 0, 1, 2
+    b = bm.fork(a)
+    assert [bm.ref[x] for x in bm.tables[a]] == [2, 2, 2]
+    free_before = list(bm.free)
+    bm.release(b)
+    # every block is still held by `a`: count down to 1, nothing returns to the pool
+    assert [bm.ref[x] for x in bm.tables[a]] == [1, 1, 1]
+    assert bm.free == free_before and b not in bm.tables and b not in bm.ctx
+    assert bm.tables[a] == [0, 1, 2] and bm.ctx[a] == 10
+
+
+def test_release_of_the_last_holder_frees_in_table_order_at_the_back():
+    order = [5, 2, 7, 0, 3, 1, 6, 4]
+    bm = RefBlockManager(8, 4, order)
+    a = bm.new_seq(9)                                     # takes 5, 2, 7
+    b = bm.new_seq(4)                                     # takes 0
+    assert bm.tables[a] == [5, 2, 7] and bm.tables[b] == [0] and bm.free == [3, 1, 6, 4]
+    bm.release(a)
+    assert bm.free == [3, 1, 6, 4, 5, 2, 7]               # back of the queue, table order
+    assert [bm.ref[x] for x in (5, 2, 7)] == [0, 0, 0] and bm.ref[0] == 1
+    # the released blocks are handed out again, after the older free ones
+    c = bm.new_seq(4 * 6)
+    assert bm.tables[c] == [3, 1, 6, 4, 5, 2]
+    assert bm.free == [7]
+
+
+def test_release_of_a_diverged_sample_returns_only_its_private_copy():
+    bm = RefBlockManager(12, 4)
+    root = bm.new_seq(6)                                   # blocks 0 (full), 1 (partial)
+    kid = bm.fork(root)
+    slot, cow = bm.append_slot(kid)                        # kid copies the partial block
+    assert cow == (1, 2) and bm.tables[kid] == [0, 2] and slot == 2 * 4 + 2
+    bm.release(kid)
+    assert bm.ref[0] == 1 and bm.ref[1] == 1 and bm.ref[2] == 0
+    assert bm.free[-1] == 2 and 0 not in bm.free and 1 not in bm.free
+
+
+def test_release_conserves_the_pool_under_random_forks_and_appends():
+    rng = np.random.default_rng(21)
+    for trial in range(20):
+        N, bs = 64, int(rng.choice([1, 2, 4, 8]))
+        bm = RefBlockManager(N, bs, list(rng.permutation(N)))
+        live = []
+        for _ in range(120):
+            op = rng.integers(0, 4)
+            try:
+                if op == 0 or not live:
+                    live.append(bm.new_seq(int(rng.integers(0, 3 * bs + 1))))
+                elif op == 1:
+                    live.append(bm.fork(live[int(rng.integers(len(live)))]))
+                elif op == 2:
+                    bm.append_slot(live[int(rng.integers(len(live)))])
+                else:
+                    bm.release(live.pop(int(rng.integers(len(live)))))
+            except MemoryError:
+                pass
+            # recount from the tables alone: a block's count is the number of table
+            # entries naming it, and a block is free exactly when nothing names it
+            held = {}
+            for t in bm.tables.values():
+                for x in t:
+                    held[x] = held.get(x, 0) + 1
+            assert all(bm.ref[x] == held.get(x, 0) for x in range(N))
+            assert sorted(bm.free + list(held)) == list(range(N))
+        for s in live:
+            bm.release(s)
+        assert sorted(bm.free) == list(range(N)) and not any(bm.ref) and not bm.tables
