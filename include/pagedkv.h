@@ -27,8 +27,15 @@
  *    "fixed-size blocks"; this layout keeps each (block, kv head) slice contiguous):
  *        cache[num_blocks][num_kv_heads][block_size][head_dim], 16-bit elements.
  *  - Supported: head_dim in {64, 128}; block_size in {1, 8, 16, 32};
- *    num_q_heads % num_kv_heads == 0 with a group of at most 16 q heads per kv head;
- *    q, out and the caches share one dtype.  Pointers must be 16-byte aligned.
+ *    num_q_heads % num_kv_heads == 0; q, out and the caches share one dtype.  The query
+ *    rows one kv head serves (q heads per kv head x new tokens per sequence, or x chunk
+ *    members in a cascade prefix pass) may number up to 64 for pa_decode,
+ *    pa_decode_multi and the cascade's prefix pass, up to 16 for pa_decode_append,
+ *    pa_decode_e4m3 and the cascade's per-sequence pass.  Up to 16 rows run on
+ *    warp-level tensor-core MMAs; 17 to 64 on the 5th-generation (tcgen05) tensor cores
+ *    with the accumulators in tensor memory (PAGEDKV_WIDE_MIN_COLS=n in the environment
+ *    moves that threshold, for comparing the two kernels).  Pointers must be 16-byte
+ *    aligned.
  */
 #ifndef PAGEDKV_H
 #define PAGEDKV_H
@@ -121,7 +128,7 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
  *
  *   q, out         [num_seqs][q_len][num_q_heads][head_dim]
  *   other arguments as for pa_decode; the workspace size does not depend on q_len.
- * Limits: 1 <= q_len and (num_q_heads/num_kv_heads) * q_len <= 16 (PA_ERR_UNSUPPORTED
+ * Limits: 1 <= q_len and (num_q_heads/num_kv_heads) * q_len <= 64 (PA_ERR_UNSUPPORTED
  * otherwise).  q_len == 1 gives exactly the bits of pa_decode.
  */
 pa_status pa_decode_multi(void* out, const void* q, const void* k_cache, const void* v_cache,
@@ -211,16 +218,17 @@ pa_status pa_decode_e4m3(void* out, const void* q, const void* k_cache, const vo
  *                      0 for a sequence in no chunk
  *   chunk_members      device int32 [num_chunks][chunk_width]: member sequence ids,
  *                      padded with -1; the first slot must be a member.  1 <= chunk_width
- *                      and (num_q_heads/num_kv_heads) * chunk_width <= 16: a chunk's query
- *                      rows share the MMA N dimension (8 rows or fewer run the lighter
- *                      kernel; up to 16 read the prefix half as often)
+ *                      and (num_q_heads/num_kv_heads) * chunk_width <= 64: a chunk's query
+ *                      rows share the MMA N dimension, so the prefix is read once for all
+ *                      of them (pa_plan_cascade plans such chunks)
  *   chunk_prefix_lens  device int32 [num_chunks]
  *   workspace          >= pa_decode_cascade_workspace_bytes(...) bytes, 256-byte aligned
  * Contract (not checked on the device): every sequence with prefix_lens[s] > 0 is a
  * member of exactly one chunk, whose prefix length equals prefix_lens[s], and the block
  * tables of a chunk's members agree on their first ceil(prefix/block_size) entries.
  * Member ids outside [0, num_seqs) count as padding; a chunk whose first member is
- * padding is empty.  Other arguments, limits and errors as for pa_decode.
+ * padding is empty.  num_q_heads/num_kv_heads must be <= 16 (the per-sequence pass).
+ * Other arguments, limits and errors as for pa_decode.
  */
 size_t pa_decode_cascade_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads,
                                          int head_dim);
@@ -273,6 +281,30 @@ pa_status pa_copy_blocks(void* const* k_caches, void* const* v_caches, int num_l
                          size_t block_bytes, int32_t* dev_status, void* stream);
 
 /*
+ * pa_swap_out_blocks / pa_swap_in_blocks -- the data side of preemption (see
+ * pa_bm_swap_out): copy n blocks of every layer's K and V pool to a buffer, or back.
+ *
+ * Defined by [P1] "Why KV cache memory was the bottleneck" (preempting in-flight
+ * requests when the cache runs out).  Buffer layout, block_bytes per block (as in
+ * pa_copy_blocks):  buf[layer][pool: 0 = K, 1 = V][i][block_bytes]  for i < n, entry i
+ * holding pool block blocks[i]; num_layers * 2 * n * block_bytes bytes in all.
+ *
+ *   host_dst / host_src  page-locked host memory the device can reach (cudaHostAlloc,
+ *                  cudaMallocHost, cudaHostRegister) or device memory, 16-byte aligned;
+ *                  pageable host memory is refused (PA_ERR_INVALID), not faulted on.
+ *   k_caches, v_caches  HOST arrays of num_layers device pointers (one pool per layer)
+ *   blocks         device int32 [n]; an id outside [0, num_blocks) sets PA_DEV_BAD_PAIR
+ *                  and that entry is skipped
+ * Stream-ordered like every call; the buffer is complete when the stream is.
+ */
+pa_status pa_swap_out_blocks(void* host_dst, void* const* k_caches, void* const* v_caches,
+                             int num_layers, const int32_t* blocks, int n, int num_blocks,
+                             size_t block_bytes, int32_t* dev_status, void* stream);
+pa_status pa_swap_in_blocks(void* const* k_caches, void* const* v_caches, int num_layers,
+                            const int32_t* blocks, int n, int num_blocks, const void* host_src,
+                            size_t block_bytes, int32_t* dev_status, void* stream);
+
+/*
  * pa_decode_noalloc -- pa_decode without a caller-provided workspace.
  *
  * The pages have no counterpart for this call; it exists for callers that cannot
@@ -288,19 +320,23 @@ pa_status pa_copy_blocks(void* const* k_caches, void* const* v_caches, int num_l
  *
  * Same arguments, results and errors as pa_decode, minus workspace/workspace_bytes,
  * with these differences:
- *  - num_seqs above PA_NOALLOC_MAX_SEQS returns PA_ERR_INVALID.  (The scratch holds
- *    the split partials of at most 320 concurrently scheduled CTAs at head_dim <= 128;
- *    on a larger GPU the call schedules 320 CTAs.)
+ *  - The scratch holds the split partials of at most 444 CTAs (3 per SM on a 148-SM
+ *    B200, the most pa_decode schedules there) at head_dim <= 128: head_dim above 128
+ *    returns PA_ERR_UNSUPPORTED, and a GPU with more SMs is scheduled with 444 CTAs.
+ *    The batch size does not change the scratch; num_seqs above PA_NOALLOC_MAX_SEQS
+ *    returns PA_ERR_INVALID as a stated limit of this call, not of the scratch.
  *  - The first call on a device looks up the device address of the array for that
- *    device (cudaGetSymbolAddress, with that device current) and caches it; make that
- *    first call before any stream capture.
+ *    device (cudaGetSymbolAddress, with that device current) and caches it for the life
+ *    of the process; make that first call before any stream capture, and do not use
+ *    this call after a cudaDeviceReset of that device (the cached address belongs to
+ *    the destroyed context).
  *  - All calls share the one array per device and it keeps whatever the previous call
  *    left there.  Nothing in it needs to start at zero (each call writes every value
  *    it later reads), but two calls that can run at the same time on one device (on
  *    different streams, or from different host threads) race on it and give wrong
  *    results: order them on one stream or with events.
  */
-#define PA_NOALLOC_SCRATCH_BYTES 6291456
+#define PA_NOALLOC_SCRATCH_BYTES 7864320
 #define PA_NOALLOC_MAX_SEQS 16384
 pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache, const void* v_cache,
                             const int32_t* block_tables, const int32_t* context_lens,
@@ -373,6 +409,66 @@ pa_status pa_bm_block_tables(const pa_block_manager* bm, const int32_t* seqs, in
 
 /* Flat slot of cached position pos (0 <= pos < context length) of seq. */
 pa_status pa_bm_slot_of(const pa_block_manager* bm, int32_t seq, int64_t pos, int64_t* slot);
+
+/*
+ * Preemption: swap a sequence's KV out of the pool and back.
+ *
+ * Defined by [P1] "Why KV cache memory was the bottleneck" (when the cache runs out,
+ * in-flight requests are preempted) together with the release rule of [P2] "Core
+ * Principle".  pa_bm_swap_out writes seq's blocks in table order to blocks[] (HOST,
+ * room for pa_bm_num_blocks_of(seq) entries), sets *num_blocks, and then gives them
+ * back exactly as pa_bm_release would (a block shared with another sequence stays with
+ * it); seq keeps its id and context length but holds no block.  Save the blocks'
+ * contents (pa_swap_out_blocks) before anything can reuse them: enqueue that copy
+ * before any later write into the pool on the same stream.  pa_bm_swap_in gives a
+ * swapped-out seq ceil(len/block_size) fresh blocks from the front of the free queue,
+ * written in table order to blocks[]; restore the saved contents into them
+ * (pa_swap_in_blocks) before the sequence is decoded.  A swapped-in sequence shares
+ * nothing.  Errors: PA_ERR_INVALID for an unknown sequence, swap_out of a swapped-out
+ * one or swap_in of a resident one; PA_ERR_NO_BLOCKS (nothing changed) when the pool
+ * cannot hold the blocks.  While swapped out, a sequence is refused by fork,
+ * append_tokens, block_tables, slot_of and plan_cascade (PA_ERR_INVALID);
+ * pa_bm_context_len still reports its length, pa_bm_num_blocks_of 0, and pa_bm_release
+ * drops it.
+ */
+pa_status pa_bm_swap_out(pa_block_manager* bm, int32_t seq, int32_t* blocks, int* num_blocks);
+pa_status pa_bm_swap_in(pa_block_manager* bm, int32_t seq, int32_t* blocks, int* num_blocks);
+
+/*
+ * Cascade planning: the inputs pa_decode_cascade takes (prefix_lens, chunk_members,
+ * chunk_prefix_lens) for a batch, from its block tables.
+ *
+ * Defined by [P1] "How PagedAttention borrows OS paging" (requests with an identical
+ * prefix point their block tables at the same physical blocks) and [P3] "Why This
+ * Matters for Production" (parallel sampling and beam search share blocks).  Batch rows
+ * with a non-empty context whose first table entry names the same physical block form a
+ * sharing group (groups in order of first appearance, members in row order).  A group's
+ * prefix is the leading table entries common to all its members, in tokens, capped at
+ * its shortest member's context length; a group of one row, or with a prefix of 0,
+ * gets no chunk.  Each group is cut, in row order, into chunks of at most chunk_width
+ * members (the last padded with -1), all with the group's prefix; prefix_lens[i] is the
+ * prefix of row i's chunk, 0 for a row in no chunk.  Identical blocks hold identical
+ * K/V, so this is exactly the contract pa_decode_cascade states.
+ *
+ *   group         q heads per kv head (num_q_heads / num_kv_heads), >= 1
+ *   chunk_width   members per chunk; <= 0 picks 64 / group (at least 1).  group *
+ *                 chunk_width must be <= 64 (PA_ERR_UNSUPPORTED otherwise).
+ *   prefix_lens   HOST int32 [num_seqs] (written)
+ *   chunk_members HOST int32 [num_seqs][chunk_width] (written: the first *num_chunks
+ *                 rows; there are never more chunks than rows)
+ *   chunk_prefix_lens  HOST int32 [num_seqs] (written: the first *num_chunks entries)
+ * Host-only, no GPU.  pa_plan_cascade reads the tables (HOST int32
+ * [num_seqs][max_blocks_per_seq], each holding ceil(context_lens[i]/block_size) valid
+ * entries, else PA_ERR_INVALID); pa_bm_plan_cascade reads the manager's tables of
+ * seqs[0..n), batch row i = seqs[i] (PA_ERR_INVALID for an unknown sequence).
+ */
+pa_status pa_plan_cascade(const int32_t* block_tables, int max_blocks_per_seq,
+                          const int32_t* context_lens, int num_seqs, int block_size, int group,
+                          int chunk_width, int32_t* prefix_lens, int32_t* chunk_members,
+                          int32_t* chunk_prefix_lens, int* num_chunks);
+pa_status pa_bm_plan_cascade(const pa_block_manager* bm, const int32_t* seqs, int n, int group,
+                             int chunk_width, int32_t* prefix_lens, int32_t* chunk_members,
+                             int32_t* chunk_prefix_lens, int* num_chunks);
 
 #ifdef __cplusplus
 }

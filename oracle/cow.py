@@ -12,6 +12,11 @@ Follows:
     a sequence diverges (copy-on-write).
   * "PagedAttention -- The KV Cache Problem", section "How It Works": fixed-size blocks,
     one block table per sequence, allocate on demand, free when the sequence finishes.
+  * "Paged Attention and Memory Efficiency in Production LLM Serving", section "Why KV
+    cache memory was the bottleneck": when the cache runs out, in-flight requests are
+    preempted.  Preemption here is a swap: the sequence's blocks are given back to the
+    pool (as on release) after their contents are saved, and the sequence, which keeps
+    its length, later takes fresh blocks for the saved contents.
 
 Free blocks are handed out in the order given to the constructor (lowest index of the
 remaining list first), so a run is fully determined by that order.
@@ -26,6 +31,7 @@ class RefBlockManager:
         self.ref = [0] * num_blocks
         self.tables: dict[int, list[int]] = {}
         self.ctx: dict[int, int] = {}
+        self.swapped: set[int] = set()
         self._next = 0
 
     def _alloc(self) -> int:
@@ -82,3 +88,30 @@ class RefBlockManager:
             if self.ref[b] == 0:
                 self.free.append(b)
         self.ctx.pop(sid)
+        self.swapped.discard(sid)
+
+    def swap_out(self, sid: int) -> list[int]:
+        """Preempt `sid`: returns its blocks in table order (their contents are to be
+        saved first); each block's count goes down by one, blocks reaching zero return to
+        the back of the free list, and `sid` keeps its length but holds no block."""
+        assert sid not in self.swapped
+        blocks = self.tables[sid]
+        self.tables[sid] = []
+        for b in blocks:
+            self.ref[b] -= 1
+            if self.ref[b] == 0:
+                self.free.append(b)
+        self.swapped.add(sid)
+        return list(blocks)
+
+    def swap_in(self, sid: int) -> list[int]:
+        """Resume a swapped-out `sid`: ceil(len / block_size) fresh blocks from the front
+        of the free list, in table order (the saved contents go there).  Raises
+        MemoryError and changes nothing if the pool cannot hold them."""
+        assert sid in self.swapped
+        need = -(-self.ctx[sid] // self.bs)
+        if len(self.free) < need:
+            raise MemoryError("block pool exhausted")
+        self.tables[sid] = [self._alloc() for _ in range(need)]
+        self.swapped.discard(sid)
+        return list(self.tables[sid])

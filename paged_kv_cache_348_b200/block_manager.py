@@ -62,12 +62,46 @@ def _lib():
         L.pa_bm_block_tables.restype = i32
         L.pa_bm_slot_of.argtypes = [P, i32, i64, P]
         L.pa_bm_slot_of.restype = i32
+        L.pa_bm_plan_cascade.argtypes = [P, P, i32, i32, i32, P, P, P, P]
+        L.pa_bm_plan_cascade.restype = i32
+        L.pa_plan_cascade.argtypes = [P, i32, P, i32, i32, i32, i32, P, P, P, P]
+        L.pa_plan_cascade.restype = i32
+        L.pa_bm_swap_out.argtypes = [P, i32, P, P]
+        L.pa_bm_swap_out.restype = i32
+        L.pa_bm_swap_in.argtypes = [P, i32, P, P]
+        L.pa_bm_swap_in.restype = i32
         L._bm_ready = True
     return L
 
 
 def _ptr(a: np.ndarray):
     return ctypes.c_void_p(a.ctypes.data)
+
+
+def _cascade_width(group: int, width: int | None) -> int:
+    return int(width) if width else max(1, 64 // int(group))
+
+
+def plan_cascade_tables(tables: np.ndarray, ctx: np.ndarray, block_size: int, group: int,
+                        width: int | None = None):
+    """Shared-prefix chunks of a batch for pa_decode_cascade, from its block tables
+    (pa_plan_cascade in include/pagedkv.h).  Returns (prefix_lens int32 [B],
+    chunk_members int32 [C, width], chunk_prefix_lens int32 [C]); the default width puts
+    64 query rows in a chunk (64 // group members)."""
+    t = np.ascontiguousarray(np.asarray(tables, dtype=np.int32))
+    c = np.ascontiguousarray(np.asarray(ctx, dtype=np.int32))
+    B = c.shape[0]
+    W = _cascade_width(group, width)
+    prefix = np.zeros(max(B, 1), dtype=np.int32)
+    members = np.zeros((max(B, 1), W), dtype=np.int32)
+    plens = np.zeros(max(B, 1), dtype=np.int32)
+    nc = ctypes.c_int()
+    rc = _lib().pa_plan_cascade(_ptr(t), t.shape[1] if t.ndim == 2 else 0, _ptr(c), B,
+                                int(block_size), int(group), W, _ptr(prefix), _ptr(members),
+                                _ptr(plens), ctypes.byref(nc))
+    if rc != pk.PA_OK:
+        raise ValueError("pa_plan_cascade failed (%d)" % rc)
+    return prefix[:B].copy(), members[:nc.value].copy(), plens[:nc.value].copy()
 
 
 class BlockManager:
@@ -152,6 +186,27 @@ class BlockManager:
     def release(self, sid: int) -> None:
         self._check(self._L.pa_bm_release(self._h, int(sid)), "release")
 
+    def swap_out(self, sid: int) -> np.ndarray:
+        """Preempt `sid` (pa_bm_swap_out): returns its blocks in table order, whose
+        contents must be saved (pa_swap_out_blocks) before the pool reuses them; the
+        blocks go back to the pool as on release and `sid` keeps its length."""
+        n = max(int(self._L.pa_bm_num_blocks_of(self._h, int(sid))), 1)
+        out = np.zeros(n, dtype=np.int32)
+        k = ctypes.c_int()
+        self._check(self._L.pa_bm_swap_out(self._h, int(sid), _ptr(out), ctypes.byref(k)),
+                    "swap_out")
+        return out[:k.value].copy()
+
+    def swap_in(self, sid: int) -> np.ndarray:
+        """Resume a swapped-out `sid` (pa_bm_swap_in): fresh blocks in table order, into
+        which the saved contents are restored (pa_swap_in_blocks)."""
+        n = max(-(-self.context_len(sid) // self.block_size), 1)
+        out = np.zeros(n, dtype=np.int32)
+        k = ctypes.c_int()
+        self._check(self._L.pa_bm_swap_in(self._h, int(sid), _ptr(out), ctypes.byref(k)),
+                    "swap_in")
+        return out[:k.value].copy()
+
     # ---------------------------------------------------------------- views
     def table(self, sid: int) -> list[int]:
         n = int(self._L.pa_bm_num_blocks_of(self._h, int(sid)))
@@ -189,6 +244,21 @@ class BlockManager:
 
     def context_lens(self, sids) -> np.ndarray:
         return self._tables(sids, None, 0)[1]
+
+    def plan_cascade(self, sids, group: int, width: int | None = None):
+        """Shared-prefix chunks of the batch sids (batch row i = sids[i]) from the
+        manager's own tables (pa_bm_plan_cascade); same result as plan_cascade_tables."""
+        s = np.ascontiguousarray(np.asarray(list(sids), dtype=np.int32))
+        B = s.shape[0]
+        W = _cascade_width(group, width)
+        prefix = np.zeros(max(B, 1), dtype=np.int32)
+        members = np.zeros((max(B, 1), W), dtype=np.int32)
+        plens = np.zeros(max(B, 1), dtype=np.int32)
+        nc = ctypes.c_int()
+        rc = self._L.pa_bm_plan_cascade(self._h, _ptr(s), B, int(group), W, _ptr(prefix),
+                                        _ptr(members), _ptr(plens), ctypes.byref(nc))
+        self._check(rc, "plan_cascade")
+        return prefix[:B].copy(), members[:nc.value].copy(), plens[:nc.value].copy()
 
     def tail_waste(self, sids) -> float:
         """Fraction of held slots that hold no token: only the unused tail of each

@@ -20,7 +20,7 @@
 namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+constexpr size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 int sm_count() {
   int dev = 0, sms = 0;
@@ -33,18 +33,37 @@ struct WsLayout {
   size_t counters_off, acc_off, ml_off, total;
 };
 
-// arrival counters: uint64[G]; partial accumulators: float[G*2][16][D];
-// partial (max, sum): float[G*2][16][2].  (num_seqs does not change the size.)
-WsLayout ws_layout(int num_seqs, int head_dim, int grid) {
-  (void)num_seqs;
+// arrival counters: uint64[G]; partial accumulators: float[G*2][rows][D]; partial (max,
+// sum): float[G*2][rows][2], rows = query columns a kernel's partial holds (16 for the
+// mma.sync kernel, 64 for the tcgen05 one).  The batch size does not change the size.
+constexpr WsLayout ws_layout(int head_dim, int grid, int rows) {
   WsLayout w{};
   size_t off = align256(sizeof(unsigned long long) * (size_t)grid);
   w.acc_off = off;
-  off = align256(off + sizeof(float) * (size_t)grid * 2 * pkv::kMaxGroup * head_dim);
+  off = align256(off + sizeof(float) * (size_t)grid * 2 * rows * head_dim);
   w.ml_off = off;
-  off = align256(off + sizeof(float) * (size_t)grid * 2 * pkv::kMaxGroup * 2);
+  off = align256(off + sizeof(float) * (size_t)grid * 2 * rows * 2);
   w.total = off;
   return w;
+}
+
+// The workspace pa_decode and its variants take covers either kernel: the mma.sync one at
+// up to 3 CTAs per SM with 16 query columns, the tcgen05 one at one CTA per SM with 64.
+size_t split_workspace_bytes(int head_dim, int sms) {
+  const size_t a = ws_layout(head_dim, sms * pkv::kMaxCtasPerSm, pkv::kMaxGroup).total;
+  const size_t b = ws_layout(head_dim, sms, pkv::kWideCols).total;
+  return a > b ? a : b;
+}
+
+// Query columns per kv head from which the tcgen05 kernel takes a launch (plain and prefix
+// modes; PAGEDKV_WIDE_MIN_COLS=n overrides it, for comparing the two kernels).
+int wide_min_cols() {
+  static const int v = [] {
+    const char* e = std::getenv("PAGEDKV_WIDE_MIN_COLS");
+    const int x = e ? std::atoi(e) : 0;
+    return (x >= 1 && x <= pkv::kWideCols + 1) ? x : pkv::kMaxGroup + 1;
+  }();
+  return v;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -91,9 +110,13 @@ uint32_t next_epoch() {
 }
 
 // Kernel mode -> its translation unit's dispatcher.
-pa_status dispatch_mode(bool kv8, int mode, bool bf16, int d, int bs, const pkv::DecodeArgs& a,
-                        const CUtensorMap& mk, const CUtensorMap& mv, int grid, cudaStream_t s) {
+pa_status dispatch_mode(bool kv8, bool wide, int mode, bool bf16, int d, int bs,
+                        const pkv::DecodeArgs& a, const CUtensorMap& mk, const CUtensorMap& mv,
+                        int grid, cudaStream_t s) {
   using namespace pkv_host;
+  if (wide)
+    return mode == pkv::kPrefix ? run_wide_mode<pkv::kPrefix>(bf16, d, bs, a, mk, mv, grid, s)
+                                : run_wide_mode<pkv::kPlain>(bf16, d, bs, a, mk, mv, grid, s);
   if (kv8) return run_decode_mode<pkv::kPlain, true>(bf16, d, bs, a, mk, mv, grid, s);
   switch (mode) {
     case pkv::kPlain: return run_decode_mode<pkv::kPlain, false>(bf16, d, bs, a, mk, mv, grid, s);
@@ -135,7 +158,12 @@ pa_status decode_impl(void* out, const void* q, const void* k_cache, const void*
   if (block_size != 1 && block_size != 8 && block_size != 16 && block_size != 32)
     return PA_ERR_UNSUPPORTED;
   const int group = num_q_heads / num_kv_heads;
-  if ((long long)group * q_len > pkv::kMaxGroup) return PA_ERR_UNSUPPORTED;
+  const long long ncol = (long long)group * q_len;
+  // query columns per kv head: up to 16 on the mma.sync kernel (every mode), up to 64 on
+  // the tcgen05 kernel (16-bit pools, plain and prefix modes)
+  const bool wide_mode = !cx.kv8 && (cx.mode == pkv::kPlain || cx.mode == pkv::kPrefix);
+  if (ncol > (wide_mode ? pkv::kWideCols : pkv::kMaxGroup)) return PA_ERR_UNSUPPORTED;
+  const bool wide = wide_mode && ncol >= wide_min_cols();
   if ((long long)num_blocks * num_kv_heads * block_size >= (1ll << 31) ||
       (long long)max_blocks_per_seq * block_size >= (1ll << 31) ||
       (long long)num_seqs * num_kv_heads >= (1ll << 31))
@@ -148,9 +176,9 @@ pa_status decode_impl(void* out, const void* q, const void* k_cache, const void*
     return PA_ERR_INVALID;
   const int sms = sm_count();
   if (sms <= 0) return PA_ERR_CUDA;
-  int grid = sms * pkv::ctas_per_sm(cx.kv8, group * q_len <= 8 ? 1 : 2, block_size);   // as dispatch_nt
+  int grid = wide ? sms : sms * pkv::ctas_per_sm(cx.kv8, ncol <= 8 ? 1 : 2, block_size);
   if (grid_cap > 0 && grid > grid_cap) grid = grid_cap;
-  const WsLayout w = ws_layout(num_seqs, head_dim, grid);
+  const WsLayout w = ws_layout(head_dim, grid, wide ? pkv::kWideCols : pkv::kMaxGroup);
   if (workspace_bytes < w.total) return PA_ERR_INVALID;
 
   CUtensorMap mk, mv;
@@ -196,8 +224,8 @@ pa_status decode_impl(void* out, const void* q, const void* k_cache, const void*
   a.k_new = cx.k_new;
   a.v_new = cx.v_new;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return dispatch_mode(cx.kv8, cx.mode, dtype == PA_BF16, head_dim, block_size, a, mk, mv, grid,
-                       st);
+  return dispatch_mode(cx.kv8, wide, cx.mode, dtype == PA_BF16, head_dim, block_size, a, mk, mv,
+                       grid, st);
 }
 
 // Cascade workspace: the split scratch, then the external partials (max, sum)[B][Hq]
@@ -205,9 +233,9 @@ pa_status decode_impl(void* out, const void* q, const void* k_cache, const void*
 struct CascadeLayout {
   size_t split, ml_off, acc_off, total;
 };
-CascadeLayout cascade_layout(int num_seqs, int num_q_heads, int head_dim, int grid) {
+CascadeLayout cascade_layout(int num_seqs, int num_q_heads, int head_dim, int sms) {
   CascadeLayout c{};
-  c.split = ws_layout(num_seqs, head_dim, grid).total;
+  c.split = split_workspace_bytes(head_dim, sms);
   c.ml_off = align256(c.split);
   c.acc_off = align256(c.ml_off + sizeof(float2) * (size_t)num_seqs * num_q_heads);
   c.total = align256(c.acc_off + sizeof(float) * (size_t)num_seqs * num_q_heads * head_dim);
@@ -236,7 +264,7 @@ size_t pa_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads
   if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0) return 0;
   const int sms = sm_count();
   if (sms <= 0) return 0;
-  return ws_layout(num_seqs, head_dim, sms * pkv::kMaxCtasPerSm).total;
+  return split_workspace_bytes(head_dim, sms);
 }
 
 pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
@@ -343,7 +371,7 @@ size_t pa_decode_cascade_workspace_bytes(int num_seqs, int num_q_heads, int num_
   if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0) return 0;
   const int sms = sm_count();
   if (sms <= 0) return 0;
-  return cascade_layout(num_seqs, num_q_heads, head_dim, sms * pkv::kMaxCtasPerSm).total;
+  return cascade_layout(num_seqs, num_q_heads, head_dim, sms).total;
 }
 
 pa_status pa_decode_cascade(void* out, const void* q, const void* k_cache, const void* v_cache,
@@ -364,14 +392,16 @@ pa_status pa_decode_cascade(void* out, const void* q, const void* k_cache, const
     return PA_ERR_INVALID;
   const int sms = sm_count();
   if (sms <= 0) return PA_ERR_CUDA;
-  const CascadeLayout cl = cascade_layout(num_seqs, num_q_heads, head_dim, sms * pkv::kMaxCtasPerSm);
+  const CascadeLayout cl = cascade_layout(num_seqs, num_q_heads, head_dim, sms);
   if (workspace_bytes < cl.total) return PA_ERR_INVALID;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   CascadeArgs cx;
   cx.ext_ml = reinterpret_cast<float2*>(ws + cl.ml_off);
   cx.ext_acc = reinterpret_cast<float*>(ws + cl.acc_off);
   const int group = num_q_heads / num_kv_heads;
-  if (group > pkv::kMaxGroup || (num_chunks && (long long)group * chunk_width > pkv::kMaxGroup))
+  // the prefix pass puts a chunk's members' query rows side by side (up to 64 columns);
+  // the suffix pass decodes one new token per sequence (up to 16)
+  if (group > pkv::kMaxGroup || (num_chunks && (long long)group * chunk_width > pkv::kWideCols))
     return PA_ERR_UNSUPPORTED;
   if (num_chunks > 0) {
     // pass 1: each chunk's shared prefix once, its members' query rows as MMA columns
@@ -450,6 +480,79 @@ pa_status pa_copy_blocks(void* const* k_caches, void* const* v_caches, int num_l
 
 }  // extern "C"
 
+namespace {
+
+// The device-side address of a swap buffer: page-locked host memory (cudaHostAlloc,
+// cudaMallocHost or cudaHostRegister) or device memory; nullptr for memory a kernel
+// cannot reach (pageable host memory), which is refused rather than faulted on.
+void* device_view(void* p) {
+  cudaPointerAttributes at;
+  if (!p || cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  if (at.type != cudaMemoryTypeHost && at.type != cudaMemoryTypeDevice &&
+      at.type != cudaMemoryTypeManaged)
+    return nullptr;
+  return at.devicePointer;
+}
+
+pa_status swap_blocks(bool out, void* buf, void* const* k_caches, void* const* v_caches,
+                      int num_layers, const int32_t* blocks, int n, int num_blocks,
+                      size_t block_bytes, int32_t* dev_status, void* stream) {
+  if (num_layers < 0 || n < 0 || num_blocks <= 0 || block_bytes == 0 || block_bytes % 16)
+    return PA_ERR_INVALID;
+  if (num_layers == 0 || n == 0) return PA_OK;
+  if (!k_caches || !v_caches || !blocks || !buf) return PA_ERR_INVALID;
+  for (int l = 0; l < num_layers; ++l)
+    if (!k_caches[l] || !v_caches[l] || !aligned16(k_caches[l]) || !aligned16(v_caches[l]))
+      return PA_ERR_INVALID;
+  void* dbuf = device_view(buf);
+  if (!dbuf || !aligned16(dbuf)) return PA_ERR_INVALID;
+  for (int l0 = 0; l0 < num_layers; l0 += pkv::kMaxLayersPerLaunch) {
+    const int m = (num_layers - l0) < pkv::kMaxLayersPerLaunch ? (num_layers - l0)
+                                                               : pkv::kMaxLayersPerLaunch;
+    pkv::LayerPtrs P;
+    std::memset(&P, 0, sizeof(P));
+    for (int i = 0; i < m; ++i) {
+      P.k[i] = static_cast<uint4*>(k_caches[l0 + i]);
+      P.v[i] = static_cast<uint4*>(v_caches[l0 + i]);
+    }
+    dim3 grid((unsigned)n, (unsigned)(2 * m));
+    const cudaError_t e =
+        out ? pkv_host::launch(pkv::pa_swap_blocks_kernel<true>, grid, dim3(256), 0,
+                               static_cast<cudaStream_t>(stream), P, blocks, n, num_blocks,
+                               (long long)(block_bytes / 16), l0, static_cast<uint4*>(dbuf),
+                               dev_status)
+            : pkv_host::launch(pkv::pa_swap_blocks_kernel<false>, grid, dim3(256), 0,
+                               static_cast<cudaStream_t>(stream), P, blocks, n, num_blocks,
+                               (long long)(block_bytes / 16), l0, static_cast<uint4*>(dbuf),
+                               dev_status);
+    if (e != cudaSuccess) return PA_ERR_CUDA;
+  }
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_swap_out_blocks(void* host_dst, void* const* k_caches, void* const* v_caches,
+                             int num_layers, const int32_t* blocks, int n, int num_blocks,
+                             size_t block_bytes, int32_t* dev_status, void* stream) {
+  return swap_blocks(true, host_dst, k_caches, v_caches, num_layers, blocks, n, num_blocks,
+                     block_bytes, dev_status, stream);
+}
+
+pa_status pa_swap_in_blocks(void* const* k_caches, void* const* v_caches, int num_layers,
+                            const int32_t* blocks, int n, int num_blocks, const void* host_src,
+                            size_t block_bytes, int32_t* dev_status, void* stream) {
+  return swap_blocks(false, const_cast<void*>(host_src), k_caches, v_caches, num_layers, blocks,
+                     n, num_blocks, block_bytes, dev_status, stream);
+}
+
+}  // extern "C"
+
 // ---------------------------------------------------------------------------------------
 // pa_decode_noalloc: pa_decode with its scratch in a fixed device array of this file, for
 // callers that cannot allocate device memory (see include/pagedkv.h).
@@ -457,9 +560,12 @@ pa_status pa_copy_blocks(void* const* k_caches, void* const* v_caches, int num_l
 namespace {
 
 constexpr size_t kNoallocScratchBytes = PA_NOALLOC_SCRATCH_BYTES;
-static_assert(PA_NOALLOC_MAX_SEQS == 16384, "scratch sized for 16384 sequences");
-constexpr int kNoallocMaxGrid = 320;     // split CTAs the scratch is sized for
+// split CTAs the scratch is sized for: 3 per SM on a 148-SM B200, the most pa_decode runs
+// there (block_size <= 8); a GPU with more SMs runs at most this many
+constexpr int kNoallocMaxGrid = 444;
 constexpr int kNoallocMaxDevices = 64;
+static_assert(ws_layout(128, kNoallocMaxGrid, pkv::kMaxGroup).total <= kNoallocScratchBytes,
+              "the scratch must hold the split partials of kNoallocMaxGrid CTAs at head_dim 128");
 
 // Lives in the module's global memory: every device that loads the library holds it
 // until the process exits.  Host code must not pass its name to a kernel (on the host
@@ -490,16 +596,14 @@ extern "C" pa_status pa_decode_noalloc(void* out, const void* q, const void* k_c
                                        int block_size, int max_blocks_per_seq, int num_blocks,
                                        float scale, pa_dtype dtype, int32_t* dev_status,
                                        void* stream) {
-  if (num_seqs > PA_NOALLOC_MAX_SEQS) return PA_ERR_INVALID;   // beyond the fixed scratch
+  if (num_seqs > PA_NOALLOC_MAX_SEQS) return PA_ERR_INVALID;   // the call's stated limit
   if (num_seqs <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0)
     return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, 1,
                        num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
                        num_blocks, scale, dtype, nullptr, 0, kNoallocMaxGrid, dev_status, stream);
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
-  if (head_dim > 128) return PA_ERR_UNSUPPORTED;
-  // the scratch holds the layout of kNoallocMaxGrid CTAs at head_dim 128
-  if (ws_layout(num_seqs, 128, kNoallocMaxGrid).total > kNoallocScratchBytes) return PA_ERR_INVALID;
+  if (head_dim > 128) return PA_ERR_UNSUPPORTED;   // the scratch holds head_dim <= 128
   void* ws = noalloc_scratch(dev);
   if (!ws) return PA_ERR_CUDA;
   return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, 1,

@@ -17,6 +17,7 @@
 // It produces what the CUDA calls consume: int32 block tables, int32 context lengths,
 // int64 slot mappings and int32 (src, dst) copy pairs.  Not thread-safe: a caller
 // serialises calls on one manager.
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <deque>
@@ -30,6 +31,7 @@ struct pa_block_manager {
   struct Seq {
     std::vector<int32_t> table;  // logical block i -> physical block
     int64_t len = 0;             // cached tokens
+    bool swapped = false;        // preempted: holds no block, keeps its length
   };
   int32_t num_blocks = 0, block_size = 0;
   std::vector<int32_t> ref;      // reference count per physical block
@@ -50,6 +52,14 @@ struct pa_block_manager {
   const Seq* find(int32_t id) const {
     auto it = seqs.find(id);
     return it == seqs.end() ? nullptr : &it->second;
+  }
+  // a sequence that holds its blocks (known and not swapped out)
+  const Seq* resident(int32_t id) const {
+    const Seq* s = find(id);
+    return s && !s->swapped ? s : nullptr;
+  }
+  void drop(int32_t b) {         // one reference less; a block nobody holds is free again
+    if (--ref[(size_t)b] == 0) free.push_back(b);
   }
   int64_t blocks_for(int64_t tokens) const { return (tokens + block_size - 1) / block_size; }
 };
@@ -109,7 +119,7 @@ pa_status pa_bm_allocate(pa_block_manager* bm, int num_tokens, int32_t* seq_id) 
 
 pa_status pa_bm_fork(pa_block_manager* bm, int32_t seq, int32_t* child) {
   if (!bm || !child) return PA_ERR_INVALID;
-  const pa_block_manager::Seq* p = bm->find(seq);
+  const pa_block_manager::Seq* p = bm->resident(seq);
   if (!p) return PA_ERR_INVALID;
   pa_block_manager::Seq c = *p;                  // shares every block of the parent
   for (int32_t b : c.table) ++bm->ref[(size_t)b];
@@ -135,7 +145,7 @@ pa_status pa_bm_append_tokens(pa_block_manager* bm, const int32_t* seqs, int n, 
   std::unordered_map<int32_t, int32_t> ref;
   int64_t need = 0;
   for (int i = 0; i < n; ++i) {
-    const pa_block_manager::Seq* s = bm->find(seqs[i]);
+    const pa_block_manager::Seq* s = bm->resident(seqs[i]);
     if (!s) return PA_ERR_INVALID;
     Sim& m = sim.try_emplace(seqs[i], Sim{s->len, (int64_t)s->table.size(), {}}).first->second;
     const int64_t lb = m.len / bm->block_size;
@@ -187,8 +197,7 @@ pa_status pa_bm_release(pa_block_manager* bm, int32_t seq) {
   if (!bm) return PA_ERR_INVALID;
   auto it = bm->seqs.find(seq);
   if (it == bm->seqs.end()) return PA_ERR_INVALID;
-  for (int32_t b : it->second.table)
-    if (--bm->ref[(size_t)b] == 0) bm->free.push_back(b);
+  for (int32_t b : it->second.table) bm->drop(b);
   bm->seqs.erase(it);
   return PA_OK;
 }
@@ -218,7 +227,7 @@ pa_status pa_bm_block_tables(const pa_block_manager* bm, const int32_t* seqs, in
                              int32_t fill, int32_t* tables, int32_t* context_lens) {
   if (!bm || n < 0 || width <= 0 || (n && (!seqs || !tables))) return PA_ERR_INVALID;
   for (int i = 0; i < n; ++i) {
-    const pa_block_manager::Seq* s = bm->find(seqs[i]);
+    const pa_block_manager::Seq* s = bm->resident(seqs[i]);
     if (!s || (int64_t)s->table.size() > width || s->len > INT32_MAX) return PA_ERR_INVALID;
   }
   for (int i = 0; i < n; ++i) {
@@ -233,10 +242,150 @@ pa_status pa_bm_block_tables(const pa_block_manager* bm, const int32_t* seqs, in
 }
 
 pa_status pa_bm_slot_of(const pa_block_manager* bm, int32_t seq, int64_t pos, int64_t* slot) {
-  const pa_block_manager::Seq* s = bm ? bm->find(seq) : nullptr;
+  const pa_block_manager::Seq* s = bm ? bm->resident(seq) : nullptr;
   if (!s || !slot || pos < 0 || pos >= s->len) return PA_ERR_INVALID;
   *slot = (int64_t)s->table[(size_t)(pos / bm->block_size)] * bm->block_size + pos % bm->block_size;
   return PA_OK;
+}
+
+// Preemption ("Paged Attention and Memory Efficiency in Production LLM Serving", section
+// "Why KV cache memory was the bottleneck": in-flight requests are preempted when the
+// cache runs out): the sequence's blocks go back to the pool as on release, after the
+// caller has saved their contents; it keeps its id and length and later takes fresh
+// blocks for the saved contents.
+pa_status pa_bm_swap_out(pa_block_manager* bm, int32_t seq, int32_t* blocks, int* num_blocks) {
+  if (!bm || !num_blocks) return PA_ERR_INVALID;
+  pa_block_manager::Seq* s = bm->find(seq);
+  if (!s || s->swapped || (!s->table.empty() && !blocks)) return PA_ERR_INVALID;
+  const size_t n = s->table.size();
+  if (n) std::memcpy(blocks, s->table.data(), n * sizeof(int32_t));
+  for (int32_t b : s->table) bm->drop(b);
+  s->table.clear();
+  s->swapped = true;
+  *num_blocks = (int)n;
+  return PA_OK;
+}
+
+pa_status pa_bm_swap_in(pa_block_manager* bm, int32_t seq, int32_t* blocks, int* num_blocks) {
+  if (!bm || !num_blocks) return PA_ERR_INVALID;
+  pa_block_manager::Seq* s = bm->find(seq);
+  if (!s || !s->swapped) return PA_ERR_INVALID;
+  const int64_t need = bm->blocks_for(s->len);
+  if (need && !blocks) return PA_ERR_INVALID;
+  if (need > (int64_t)bm->free.size()) return PA_ERR_NO_BLOCKS;
+  s->table.resize((size_t)need);
+  for (int64_t i = 0; i < need; ++i) s->table[(size_t)i] = blocks[i] = bm->take();
+  s->swapped = false;
+  *num_blocks = (int)need;
+  return PA_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------------------
+// Cascade planning: which sequences of a batch read the same physical blocks at the start
+// of their tables ("How PagedAttention borrows OS paging": requests with an identical
+// prefix point their block tables at the same physical blocks), grouped into chunks whose
+// members' query rows pa_decode_cascade decodes together over the shared prefix.
+// ---------------------------------------------------------------------------------------
+namespace {
+
+constexpr int kCascadeMaxRows = 64;     // query rows a prefix chunk holds (group x members)
+
+// Rows of one batch: table row i (entries row(i)[0..nblk(i))) and its length.
+template <typename RowFn, typename LenFn>
+pa_status plan_rows(int n, int block_size, int group, int chunk_width, RowFn row, LenFn len,
+                    int32_t* prefix_lens, int32_t* chunk_members, int32_t* chunk_prefix_lens,
+                    int* num_chunks) {
+  if (n < 0 || block_size <= 0 || group <= 0 || !num_chunks ||
+      (n && (!prefix_lens || !chunk_members || !chunk_prefix_lens)))
+    return PA_ERR_INVALID;
+  const int width = chunk_width > 0 ? chunk_width : std::max(1, kCascadeMaxRows / group);
+  if ((int64_t)group * width > kCascadeMaxRows) return PA_ERR_UNSUPPORTED;
+  *num_chunks = 0;
+  // sharing groups: rows with a non-empty context whose first physical block is the same,
+  // in order of first appearance, members in batch order
+  std::unordered_map<int32_t, int> by_first;
+  std::vector<std::vector<int>> groups;
+  for (int i = 0; i < n; ++i) {
+    prefix_lens[i] = 0;
+    if (len(i) <= 0) continue;
+    const int32_t b0 = row(i)[0];
+    auto it = by_first.find(b0);
+    if (it == by_first.end()) {
+      by_first.emplace(b0, (int)groups.size());
+      groups.push_back({i});
+    } else {
+      groups[(size_t)it->second].push_back(i);
+    }
+  }
+  int nc = 0;
+  for (const std::vector<int>& mem : groups) {
+    if (mem.size() < 2) continue;
+    // the leading table entries common to every member, capped at the shortest member
+    int64_t minlen = INT64_MAX;
+    for (int i : mem) minlen = std::min<int64_t>(minlen, len(i));
+    const int64_t nb = (minlen + block_size - 1) / block_size;
+    int64_t common = 0;
+    const int32_t* r0 = row(mem[0]);
+    while (common < nb) {
+      bool same = true;
+      for (int i : mem) same = same && row(i)[common] == r0[common];
+      if (!same) break;
+      ++common;
+    }
+    const int64_t plen = std::min<int64_t>(common * block_size, minlen);
+    if (plen == 0) continue;
+    for (size_t k = 0; k < mem.size(); k += (size_t)width) {
+      int32_t* out = chunk_members + (int64_t)nc * width;
+      for (int j = 0; j < width; ++j) {
+        const size_t m = k + (size_t)j;
+        out[j] = m < mem.size() ? mem[m] : -1;
+        if (m < mem.size()) prefix_lens[mem[m]] = (int32_t)plen;
+      }
+      chunk_prefix_lens[nc] = (int32_t)plen;
+      ++nc;
+    }
+  }
+  *num_chunks = nc;
+  return PA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_plan_cascade(const int32_t* block_tables, int max_blocks_per_seq,
+                          const int32_t* context_lens, int num_seqs, int block_size, int group,
+                          int chunk_width, int32_t* prefix_lens, int32_t* chunk_members,
+                          int32_t* chunk_prefix_lens, int* num_chunks) {
+  if (block_size <= 0 || (num_seqs > 0 && (!block_tables || !context_lens || max_blocks_per_seq <= 0)))
+    return PA_ERR_INVALID;
+  for (int i = 0; i < num_seqs; ++i) {     // every table must hold its sequence's blocks
+    const int64_t c = context_lens[i];
+    if (c < 0 || (c + block_size - 1) / block_size > max_blocks_per_seq) return PA_ERR_INVALID;
+  }
+  return plan_rows(
+      num_seqs, block_size, group, chunk_width,
+      [&](int i) { return block_tables + (int64_t)i * max_blocks_per_seq; },
+      [&](int i) { return (int64_t)context_lens[i]; }, prefix_lens, chunk_members,
+      chunk_prefix_lens, num_chunks);
+}
+
+pa_status pa_bm_plan_cascade(const pa_block_manager* bm, const int32_t* seqs, int n, int group,
+                             int chunk_width, int32_t* prefix_lens, int32_t* chunk_members,
+                             int32_t* chunk_prefix_lens, int* num_chunks) {
+  if (!bm || n < 0 || (n && !seqs)) return PA_ERR_INVALID;
+  std::vector<const pa_block_manager::Seq*> rows((size_t)n);
+  for (int i = 0; i < n; ++i) {
+    rows[(size_t)i] = bm->resident(seqs[i]);
+    if (!rows[(size_t)i]) return PA_ERR_INVALID;
+  }
+  return plan_rows(
+      n, bm->block_size, group, chunk_width,
+      [&](int i) { return rows[(size_t)i]->table.data(); },
+      [&](int i) { return rows[(size_t)i]->len; }, prefix_lens, chunk_members, chunk_prefix_lens,
+      num_chunks);
 }
 
 }  // extern "C"

@@ -1,0 +1,831 @@
+// decode_wide.cuh -- paged decode for many query rows per kv head on tcgen05 tensor cores.
+//
+// Same operation as decode.cuh ("Paged Attention and Memory Efficiency in Production LLM
+// Serving", section "How PagedAttention borrows OS paging": the kernel resolves each
+// request's block table at run time and computes the plain softmax(scale q K^T) V), for
+// the launches whose query rows per kv head -- the GQA group times the new tokens of a
+// sequence ("PagedAttention -- The KV Cache Problem", "Why This Matters for Production":
+// beam search and parallel sampling), or the members of a shared-prefix chunk -- number
+// 17..64.  There the contraction is a real dense tile (up to 64 flop per KV byte), too
+// much for warp-level mma.sync, so it runs on the 5th-generation tensor cores:
+//
+//  * One persistent CTA per SM takes an equal range of the batch's 16-token units (the
+//    schedule of decode.cuh: segments = (sequence, kv head), weighted split, partials of
+//    segments shared between CTAs merged by the last arrival).
+//  * Warp 0 streams 128-token K and V tiles into a 3-stage ring with 2-D TMA copies whose
+//    row coordinate comes from the block table (128-byte swizzle, tokens as rows), and the
+//    segment's query rows into a Q tile with cp.async (same swizzle).
+//  * Warp 1 (one thread) issues the MMAs: S^T[128 tokens][N] = K . Q^T with the tokens on
+//    M = 128 and the query rows on N = 16..64 (no padding of the query side to 64 or 128),
+//    accumulated in tensor memory; then O^T[D][N] += V^T . P^T with V read MN-major from
+//    the same tile.  The QK^T of stage i+2 is issued right after the PV of stage i, so the
+//    softmax of stage i+1 overlaps both.
+//  * Warps 2..5 (one thread per token row of S^T, i.e. per TMEM lane) run the softmax:
+//    base-2, fp32, with a lazily moved reference maximum per query row (a stage moves it
+//    only when some score exceeds it by more than 2^8, which after a portion's first stage
+//    is rare; O^T is then rescaled in tensor memory).  P^T is written in 16 bits as a high
+//    part and the rounding residual (~16 mantissa bits in all) into the stage's K tile,
+//    which QK^T no longer needs.  Row sums stay per thread and are reduced once per
+//    portion.  The same warps read O^T back at the end of a portion (one thread per head
+//    dim) and write the output or the split partial.
+//  * Every wait is bounded; tensor memory is released on every exit path.
+#pragma once
+#include "decode.cuh"
+
+namespace pkv {
+
+constexpr int kWideCols = 64;                     // query rows per kv head handled (MMA N)
+constexpr int kWideTile = 128;                    // tokens per stage (MMA M of QK^T)
+constexpr int kWideUnits = kWideTile / kUnit;     // 16-token units per stage
+constexpr int kWideStages = 3;
+constexpr int kWideSoftThreads = 128;             // softmax warps 2..5
+constexpr int kWideThreads = 64 + kWideSoftThreads;
+constexpr uint32_t kWideTmemCols = 256;           // S^T x 2 (cols 0..127), O^T (cols 128..191)
+constexpr float kRescaleLog2 = 8.f;               // a reference max moves past this gap only
+
+template <int D>
+struct WideLayout {
+  static constexpr int kHalves = D / 64;                        // 128-byte column halves
+  static constexpr int kKvBytes = kHalves * kWideTile * 128;    // one K or V tile
+  static constexpr int kPBytes = kWideTile * 128;               // P^T high or low part
+  // P^T (high, low) goes to the stage's K tile once QK^T has read it, when it fits
+  static constexpr bool kPInK = kKvBytes >= 2 * kPBytes;
+  static constexpr int kPOff = kPInK ? 0 : 2 * kKvBytes;
+  static constexpr int kStageBytes = 2 * kKvBytes + (kPInK ? 0 : 2 * kPBytes);
+  static constexpr int kQOff = kWideStages * kStageBytes;
+  static constexpr int kQBytes = kHalves * kWideCols * 128;
+  static constexpr int kMetaOff = kQOff + kQBytes;
+  static constexpr int kBarOff = (kMetaOff + kWideStages * (int)sizeof(StageMeta) + 15) / 16 * 16;
+  // full[3], empty[3], sfull[2], pfull[2], qempty, drain
+  static constexpr int kNumBars = 2 * kWideStages + 6;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;       // tmem base, abort, last, total
+  static constexpr int kDescOff = kMiscOff + 32;
+  static constexpr int kMrefOff = (kDescOff + 2 * (int)sizeof(SplitDesc) + 15) / 16 * 16;
+  static constexpr int kRedOff = kMrefOff + 2 * kWideCols * 4;  // float [64 cols][4 warps]
+  static constexpr int kAlphaOff = kRedOff + kWideCols * 4 * 4;
+  static constexpr int kBytes = kAlphaOff + kWideCols * 4;
+  static constexpr int kDynSmem = kBytes + 1024;                // slack for 1024-byte alignment
+  static_assert(kStageBytes % 1024 == 0 && kQOff % 1024 == 0 && kKvBytes % 1024 == 0,
+                "tiles need 1024-byte alignment (128-byte swizzle atoms)");
+  static_assert(kBarOff % 8 == 0 && kMiscOff % 8 == 0 && kDescOff % 8 == 0 && kMrefOff % 16 == 0,
+                "mbarriers and 64-bit fields need 8-byte alignment");
+  static_assert(kDynSmem <= 232448, "one CTA per SM must fit");
+};
+
+// Last arrival of a split segment (see merge_split in decode.cuh), for up to 64 query
+// columns: out = (sum_k acc_k 2^(m_k - M)) / (sum_k l_k 2^(m_k - M)), contributors folded
+// in CTA order.  Thread tid owns elements (column, 4 dims) e = tid + 128 i, 8 at a time.
+template <typename T, int D, int MODE>
+__device__ __forceinline__ void merge_wide(const DecodeArgs& a, const SplitDesc& dsc,
+                                           long long total, int G, int tid) {
+  constexpr int kF4 = D / 4;
+  constexpr int kB = 8;                                  // elements per batch
+  const int nel = a.ncol * kF4;
+  for (int e0 = tid; e0 < nel; e0 += kB * kWideSoftThreads) {
+    float M[kB], Ls[kB];
+    float4 acc[kB];
+#pragma unroll
+    for (int b = 0; b < kB; ++b) {
+      M[b] = -INFINITY;
+      Ls[b] = 0.f;
+      acc[b] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    for (int cc = dsc.cf; cc <= dsc.cl; ++cc) {
+      const int pk = partial_slot(cc, dsc.seg0, total, G);
+      if (pk < 0) continue;
+      float2 ml[kB];
+      float4 v[kB];
+#pragma unroll
+      for (int b = 0; b < kB; ++b) {
+        const int e = e0 + b * kWideSoftThreads;
+        ml[b] = make_float2(-INFINITY, 0.f);
+        v[b] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (e < nel) {
+          const long long row = (long long)pk * kWideCols + e / kF4;
+          ml[b] = __ldcg(reinterpret_cast<const float2*>(a.part_ml) + row);
+          v[b] = __ldcg(reinterpret_cast<const float4*>(a.part_acc + row * D) + e % kF4);
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < kB; ++b) {
+        if (ml[b].x == -INFINITY) continue;
+        const float mn = fmaxf(M[b], ml[b].x);
+        const float sa = M[b] == -INFINITY ? 0.f : ex2(M[b] - mn);
+        const float sb = ex2(ml[b].x - mn);
+        Ls[b] = Ls[b] * sa + ml[b].y * sb;
+        acc[b].x = acc[b].x * sa + v[b].x * sb;
+        acc[b].y = acc[b].y * sa + v[b].y * sb;
+        acc[b].z = acc[b].z * sa + v[b].z * sb;
+        acc[b].w = acc[b].w * sa + v[b].w * sb;
+        M[b] = mn;
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < kB; ++b) {
+      const int e = e0 + b * kWideSoftThreads;
+      if (e >= nel) continue;
+      const long long row = out_row<MODE>(a, dsc.seq, dsc.kvh, e / kF4);
+      if (row < 0) continue;
+      float v4[4] = {acc[b].x, acc[b].y, acc[b].z, acc[b].w};
+      finish_row<T, MODE, D>(a, row, M[b], Ls[b], v4, (e % kF4) * 4, 4, make_float2(-INFINITY, 0.f),
+                             v4);
+    }
+  }
+}
+
+template <typename T, int D, int BS, int MODE>
+__global__ void __launch_bounds__(kWideThreads, 1)
+    pa_decode_wide_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
+                          const __grid_constant__ CUtensorMap tmv) {
+  using L = WideLayout<D>;
+  static_assert(MODE == kPlain || MODE == kPrefix, "wide decode: plain (multi-token) or prefix");
+  constexpr int kSegW = seg_weight(BS);
+  constexpr uint32_t kAB = std::is_same_v<T, __nv_bfloat16> ? 1u : 0u;
+  constexpr int kFullCount = 33;       // lane 0's expect_tx arrival + 32 cp.async arrivals
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  StageMeta* meta = reinterpret_cast<StageMeta*>(smem + L::kMetaOff);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* empty = full + kWideStages;
+  uint64_t* sfull = empty + kWideStages;
+  uint64_t* pfull = sfull + 2;
+  uint64_t* qempty = pfull + 2;
+  uint64_t* drain = qempty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+  volatile int* last_flag = abort_flag + 1;
+  long long* total_s = reinterpret_cast<long long*>(smem + L::kMiscOff + 16);
+  SplitDesc* desc = reinterpret_cast<SplitDesc*>(smem + L::kDescOff);
+  float* mref = reinterpret_cast<float*>(smem + L::kMrefOff);      // [2][64]
+  float* red = reinterpret_cast<float*>(smem + L::kRedOff);        // [64][4]
+  float* alph = reinterpret_cast<float*>(smem + L::kAlphaOff);     // [64]
+  uint8_t* sQ = smem + L::kQOff;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kWideStages; ++i) {
+      mbar_init(&full[i], kFullCount);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sfull[i], 1);
+      mbar_init(&pfull[i], kWideSoftThreads);
+    }
+    mbar_init(qempty, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    *last_flag = 0;
+    fence_mbar_init();
+  }
+  if (BS != 1 && threadIdx.x == 32) {
+    prefetch_tensormap(&tmk);
+    prefetch_tensormap(&tmv);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kWideTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  pdl_wait();      // nothing global is read or written before the previous grid is done
+  pdl_trigger();
+
+  const int G = gridDim.x, c = blockIdx.x;
+  const int Hkv = a.num_kv_heads, group = a.group;
+  const int nq = (a.ncol + 15) & ~15;               // MMA N: query rows rounded up to 16
+
+  if (warp == 0) {
+    // ============================== producer ==============================
+    const int B = a.num_seqs;
+    long long run = 0;
+    int keep_ctx = 0, keep_u = 0, keep_x = 0;
+    for (int base = 0; base < B; base += 32) {
+      const int s = base + lane;
+      SeqSpan sp{0, 0};
+      if (s < B) sp = span_of<MODE>(a, s, c == 0 ? a.status : nullptr);
+      const int u = (sp.ctx + kUnit - 1) / kUnit;
+      int x = u ? u + kSegW : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      keep_ctx = sp.ctx;
+      keep_u = u;
+      keep_x = x;
+      run += __shfl_sync(0xffffffffu, x, 31);
+      if (c == 0) {
+        unsigned zero = __ballot_sync(0xffffffffu, s < B && u == 0);
+        while (zero) {
+          const int src = __ffs(zero) - 1;
+          zero &= zero - 1;
+          empty_rows<T, MODE, D>(a, base + src, 0, lane);
+        }
+      }
+    }
+    const long long total = (long long)Hkv * run;
+    const long long start = total ? cta_start(c, total, G) : 0;
+    const long long end = total ? cta_start(c + 1, total, G) : 0;
+
+    int s_a = 0, u_a = 0, ctx_a = 0;
+    long long pb_a = 0;
+    if (start < end) {
+      long long r2 = 0;
+      bool got_a = false;
+      for (int base = 0; base < B && !got_a; base += 32) {
+        const int s = base + lane;
+        int ctx = keep_ctx, u = keep_u, x = keep_x;
+        if (B > 32) {
+          SeqSpan sp{0, 0};
+          if (s < B) sp = span_of<MODE>(a, s, nullptr);
+          ctx = sp.ctx;
+          u = (ctx + kUnit - 1) / kUnit;
+          x = u ? u + kSegW : 0;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+          }
+        }
+        const int wt = u ? u + kSegW : 0;
+        const long long lo = (long long)Hkv * (r2 + x - wt), hi = (long long)Hkv * (r2 + x);
+        const unsigned ha = __ballot_sync(0xffffffffu, s < B && u > 0 && lo <= start && start < hi);
+        if (ha) {
+          const int src = __ffs(ha) - 1;
+          s_a = base + src;
+          u_a = __shfl_sync(0xffffffffu, u, src);
+          ctx_a = __shfl_sync(0xffffffffu, ctx, src);
+          pb_a = __shfl_sync(0xffffffffu, lo, src);
+          got_a = true;
+        }
+        r2 += __shfl_sync(0xffffffffu, x, 31);
+      }
+    }
+    if (lane == 0) *total_s = total;
+    __syncwarp();
+
+    const uint64_t policy = policy_evict_first();
+    const int rows_total = a.num_blocks * Hkv * BS;
+    int st = 0, nqs = 0, portions = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    {
+      long long x = start;
+      int s_cur = s_a, u_cur = u_a, ctx_cur = ctx_a;
+      long long pbase = pb_a;
+      while (ok && x < end) {
+        while (x >= pbase + (long long)Hkv * (u_cur ? u_cur + kSegW : 0)) {   // next sequence
+          pbase += (long long)Hkv * (u_cur ? u_cur + kSegW : 0);
+          ++s_cur;
+          ctx_cur = span_of<MODE>(a, s_cur, nullptr).ctx;
+          u_cur = (ctx_cur + kUnit - 1) / kUnit;
+        }
+        const int w_cur = u_cur + kSegW;
+        const int kvh = (int)((x - pbase) / w_cur);
+        const long long seg0 = pbase + (long long)kvh * w_cur, seg1 = seg0 + u_cur;
+        if (x >= seg1) {                              // on the segment's virtual tail
+          x = seg0 + w_cur;
+          continue;
+        }
+        const long long pe = seg1 < end ? seg1 : end;
+        const bool complete = seg0 >= start && seg1 <= end;
+        const int pidx = c * 2 + (start < seg0 ? 1 : 0);
+        int qslot = 0;
+        if (!complete) {
+          qslot = nqs++;
+          if (lane == 0) {
+            const int cf = cta_of(seg0, total, G), cl = cta_of(seg1 - 1, total, G);
+            int ncontrib = 0;
+            for (int cc = cf; cc <= cl; ++cc)
+              ncontrib += cta_start(cc, total, G) < cta_start(cc + 1, total, G);
+            desc[qslot] = SplitDesc{s_cur, kvh, cf, cl, ncontrib, 0, seg0};
+          }
+        }
+        // a chunk of a prefix launch reads the prefix through its first member's table
+        const long long trow_seq = MODE == kPrefix ? (long long)chunk_member(a, s_cur, 0) : s_cur;
+        const int32_t* trow = a.block_tables + trow_seq * a.max_blocks;
+        const int nblk = (ctx_cur + BS - 1) / BS;
+        for (long long tu = x; tu < pe; tu += kWideUnits) {
+          const int nun = (int)((pe - tu) < kWideUnits ? (pe - tu) : kWideUnits);
+          const int tok0 = (int)(tu - seg0) * kUnit;
+          const bool first_stage = tu == x;
+          const int flags = (first_stage ? F_FIRST : 0) | (tu + kWideUnits >= pe ? F_LAST : 0) |
+                            (complete ? F_COMPLETE : 0);
+          uint8_t* sK = smem + st * L::kStageBytes;
+          uint8_t* sV = sK + L::kKvBytes;
+          if constexpr (BS != 1) {
+            constexpr int H = BS < 16 ? BS : 16;     // rows per TMA box
+            constexpr int BPU = kUnit / H;           // boxes per unit and column half
+            constexpr int kBoxBytes = H * 128;
+            constexpr int kMaxBox = kWideUnits * BPU * L::kHalves * 2;
+            constexpr int kRep = (kMaxBox + 31) / 32;
+            const int nbox = nun * BPU * L::kHalves * 2;
+            // this lane's boxes and their block-table entries, read before the slot wait
+            int ys[kRep];
+#pragma unroll
+            for (int rp = 0; rp < kRep; ++rp) {
+              const int bi = lane + 32 * rp;
+              const int jb = (bi >> 1) / L::kHalves;
+              const int t = tok0 + (jb / BPU) * kUnit + (jb % BPU) * H;
+              ys[rp] = -1;
+              if (bi < nbox && t < ctx_cur) {
+                const int blk = t / BS < nblk ? __ldg(trow + t / BS) : -1;
+                if ((unsigned)blk < (unsigned)a.num_blocks) {
+                  ys[rp] = (blk * Hkv + kvh) * BS + (t % BS);
+                } else {
+                  if (a.status) atomicOr(a.status, DEV_BAD_BLOCK_ID);
+                  ys[rp] = rows_total;                 // out of range: TMA fills zeros
+                }
+              }
+            }
+            uint32_t bytes = 0;
+            for (int jj = 0; jj < nun; ++jj) {
+              const int rem = ctx_cur - (tok0 + jj * kUnit);
+              const int nb = (rem + H - 1) / H;
+              bytes += (uint32_t)((nb < BPU ? nb : BPU) * kBoxBytes * L::kHalves * 2);
+            }
+            if (!mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, kWaitLimitNs)) {
+              ok = false;
+              break;
+            }
+            if (lane == 0) {
+              meta[st] = StageMeta{s_cur, kvh, tok0, nun, ctx_cur, flags, pidx, qslot, -1};
+              mbar_arrive_expect_tx(&full[st], bytes);
+            }
+            __syncwarp();
+#pragma unroll
+            for (int rp = 0; rp < kRep; ++rp) {
+              const int bi = lane + 32 * rp;
+              if (ys[rp] >= 0) {
+                const int kv = bi & 1, hf = (bi >> 1) % L::kHalves, jb = (bi >> 1) / L::kHalves;
+                uint8_t* dst = (kv ? sV : sK) + hf * (kWideTile * 128) +
+                               ((jb / BPU) * kUnit + (jb % BPU) * H) * 128;
+                tma_load_2d(dst, kv ? &tmv : &tmk, &full[st], hf * 64, ys[rp], policy);
+              }
+            }
+          } else {
+            // block_size 1: each token is its own block; 16-byte cp.async into the same
+            // 128-byte-swizzled rows the TMA path produces.  Lane l reads the table entries
+            // of rows l, 32+l, 64+l, 96+l before the slot wait.
+            constexpr int CPR = D * 2 / 16;            // 16-byte chunks per row
+            constexpr int RPI = 32 / CPR;              // rows per warp instruction
+            const int nvalid = (nun * kUnit < ctx_cur - tok0) ? nun * kUnit : ctx_cur - tok0;
+            int wv[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int r = j * 32 + lane;
+              wv[j] = r < nvalid ? __ldg(trow + tok0 + r) : -1;
+            }
+            if (!mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, kWaitLimitNs)) {
+              ok = false;
+              break;
+            }
+            if (lane == 0) {
+              meta[st] = StageMeta{s_cur, kvh, tok0, nun, ctx_cur, flags, pidx, qslot, -1};
+              mbar_arrive_expect_tx(&full[st], 0u);
+            }
+            const int ch = lane % CPR, hf = ch >> 3, cc = ch & 7, rl = lane / CPR;
+            const uint8_t* kb = static_cast<const uint8_t*>(a.k_cache) + ch * 16;
+            const uint8_t* vb = static_cast<const uint8_t*>(a.v_cache) + ch * 16;
+            uint8_t* sKl = sK + hf * (kWideTile * 128) + rl * 128;
+            uint8_t* sVl = sV + hf * (kWideTile * 128) + rl * 128;
+#pragma unroll 4
+            for (int i = 0; i < kWideTile / RPI; ++i) {
+              const int r0 = i * RPI;
+              if (r0 >= nvalid) break;
+              const int r = r0 + rl;
+              const int v0 = __shfl_sync(0xffffffffu, wv[0], r & 31);
+              const int v1 = __shfl_sync(0xffffffffu, wv[1], r & 31);
+              const int v2 = __shfl_sync(0xffffffffu, wv[2], r & 31);
+              const int v3 = __shfl_sync(0xffffffffu, wv[3], r & 31);
+              const int blk = r < 32 ? v0 : (r < 64 ? v1 : (r < 96 ? v2 : v3));
+              if (r < nvalid) {
+                uint32_t sz = 16;
+                long long row = 0;
+                if ((unsigned)blk < (unsigned)a.num_blocks) {
+                  row = (long long)blk * Hkv + kvh;
+                } else {
+                  if (a.status) atomicOr(a.status, DEV_BAD_BLOCK_ID);
+                  sz = 0;                              // zero fill, no read
+                }
+                const int soff = r0 * 128 + ((cc ^ (r & 7)) << 4);
+                cp_async_16_zfill(sKl + soff, kb + row * (D * 2), sz, policy);
+                cp_async_16_zfill(sVl + soff, vb + row * (D * 2), sz, policy);
+              }
+            }
+          }
+          if (first_stage) {
+            // the segment's query rows: column cq = token (or chunk member) j * group + head,
+            // row cq of the Q tile, 128-byte swizzle.  The previous portion's last QK^T must
+            // be done with the single Q tile first.
+            if (portions > 0 &&
+                !mbar_wait_bounded(qempty, (uint32_t)((portions - 1) & 1), abort_flag,
+                                   kWaitLimitNs)) {
+              ok = false;
+              break;
+            }
+            constexpr int CPQ = D / 8;                 // 16-byte chunks per query row
+            const int nchunk = a.ncol * CPQ;
+            for (int k = lane; k < nchunk; k += 32) {
+              const int cq = k / CPQ, ch = k % CPQ;
+              const int jq = cq / group, g = cq % group;
+              const T* src;
+              if constexpr (MODE == kPrefix) {
+                int mem = chunk_member(a, s_cur, jq);
+                if (mem < 0) mem = (int)trow_seq;     // padding slot: the first member's rows
+                src = static_cast<const T*>(a.q) +
+                      ((long long)mem * a.num_q_heads + (long long)kvh * group + g) * D;
+              } else {
+                src = static_cast<const T*>(a.q) +
+                      (((long long)s_cur * a.q_len + jq) * a.num_q_heads + (long long)kvh * group + g) *
+                          D;
+              }
+              uint8_t* dst = sQ + (ch >> 3) * (kWideCols * 128) + cq * 128 + (((ch & 7) ^ (cq & 7)) << 4);
+              cp_async_16(dst, src + ch * 8, policy);
+            }
+            ++portions;
+          }
+          cp_async_mbar_arrive_noinc(&full[st]);
+          if (++st == kWideStages) {
+            st = 0;
+            ph ^= 1u;
+          }
+        }
+        x = pe == seg1 ? seg0 + w_cur : pe;          // past the virtual tail
+      }
+    }
+    if (ok) ok = mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, kWaitLimitNs);
+    if (ok) {
+      if (lane == 0) {
+        meta[st].flags = F_END;
+        mbar_arrive(&full[st]);
+      }
+      __syncwarp();
+      cp_async_mbar_arrive_noinc(&full[st]);
+    } else if (lane == 0) {
+      *abort_flag = 1;
+      if (a.status) atomicOr(a.status, DEV_TIMEOUT);
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+  } else if (warp == 1) {
+    // ============================== MMA issue ==============================
+    if (lane == 0) {
+      const uint32_t idesc_qk = idesc_f16(kAB, 0u, 0u, 128u, (uint32_t)nq);
+      const uint32_t idesc_pv = idesc_f16(kAB, 1u, 1u, (uint32_t)D, (uint32_t)nq);
+      const uint32_t sq = smem_u32(sQ);
+      auto qk = [&](int slot, int sb, int flags) {
+        const uint32_t sk = smem_u32(smem + slot * L::kStageBytes);
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (ks & 3) * 32;          // 16 dims = 32 bytes along a row
+          const uint64_t da = smem_desc_sw128(sk + (ks >> 2) * (kWideTile * 128) + off, 16u, 1024u);
+          const uint64_t db = smem_desc_sw128(sq + (ks >> 2) * (kWideCols * 128) + off, 16u, 1024u);
+          tc_mma_f16(tbase + (uint32_t)(sb * 64), da, db, idesc_qk, ks > 0);
+        }
+        tc_commit(&sfull[sb]);
+        if (flags & F_LAST) tc_commit(qempty);       // the Q tile may be refilled after this
+      };
+      auto pv = [&](int slot, bool first) {
+        const uint32_t sv = smem_u32(smem + slot * L::kStageBytes + L::kKvBytes);
+        const uint32_t sp = smem_u32(smem + slot * L::kStageBytes + L::kPOff);
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {         // P^T high part, then its residual
+#pragma unroll
+          for (int kk = 0; kk < kWideTile / 16; ++kk) {
+            const uint64_t da = smem_desc_sw128(sv + kk * 2048, kWideTile * 128, 1024u);
+            const uint64_t db = smem_desc_sw128(sp + part * L::kPBytes + kk * 2048, kWideTile * 128,
+                                                1024u);
+            tc_mma_f16(tbase + 128u, da, db, idesc_pv, !(first && part == 0 && kk == 0));
+          }
+        }
+      };
+      int sl[3] = {0, 0, 0}, fl[3] = {0, 0, 0};   // slots / flags of stages i, i+1, i+2
+      uint32_t phs = 0;
+      int st = 0;
+      bool ok = true, have_next = false;
+      auto next_stage = [&](int& slot, int& flags) -> bool {   // wait stage, false at END
+        if (!mbar_wait_bounded(&full[st], phs, abort_flag, kWaitLimitNs)) {
+          ok = false;
+          return false;
+        }
+        // Q (and, at block_size 1, K/V) arrive by cp.async, generic-proxy writes the
+        // tensor cores read through the async proxy
+        fence_proxy_async_smem();
+        slot = st;
+        flags = meta[st].flags;
+        if (++st == kWideStages) {
+          st = 0;
+          phs ^= 1u;
+        }
+        return !(flags & F_END);
+      };
+      if (next_stage(sl[0], fl[0])) {
+        tc_fence_after();
+        qk(sl[0], 0, fl[0]);
+        have_next = next_stage(sl[1], fl[1]);
+        if (have_next) qk(sl[1], 1, fl[1]);
+        for (int i = 0; ok; ++i) {
+          if (!mbar_wait_bounded(&pfull[i & 1], (uint32_t)((i >> 1) & 1), abort_flag,
+                                 kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          pv(sl[0], fl[0] & F_FIRST);
+          tc_commit(&empty[sl[0]]);                 // frees the stage (K, V and P tiles)
+          if (!have_next) break;
+          const bool more = next_stage(sl[2], fl[2]);
+          if (more) qk(sl[2], i & 1, fl[2]);
+          sl[0] = sl[1];
+          fl[0] = fl[1];
+          sl[1] = sl[2];
+          fl[1] = fl[2];
+          have_next = more;
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        if (a.status) atomicOr(a.status, DEV_TIMEOUT);
+      }
+      // nothing issued here may still be running when tensor memory is released (this
+      // wait ignores the abort flag: only its time limit ends it)
+      tc_commit(drain);
+      int no_abort = 0;
+      mbar_wait_bounded(drain, 0u, &no_abort, kWaitLimitNs);
+    }
+  } else {
+    // ============================== softmax / epilogue ==============================
+    const int q4 = warp & 3;                       // TMEM lane quadrant of this warp
+    const int r = q4 * 32 + lane;                  // token row of S^T (= head dim of O^T at D 128)
+    const int tid = threadIdx.x - 64;
+    const uint32_t trow_addr = tbase + ((uint32_t)(q4 * 32) << 16);
+    const int nchk = nq / 16;
+    float lp[kWideCols];
+#pragma unroll
+    for (int cq = 0; cq < kWideCols; ++cq) lp[cq] = 0.f;
+    int cur = 0;
+    int st = 0;
+    uint32_t ph = 0;
+    int pst = 0;
+    uint32_t pph = 0;                              // slot/parity of the previous stage
+    for (int i = 0;; ++i) {
+      if (!mbar_wait_bounded(&full[st], ph, abort_flag, kWaitLimitNs)) {
+        if (lane == 0) {
+          *abort_flag = 1;
+          if (a.status) atomicOr(a.status, DEV_TIMEOUT);
+        }
+        break;
+      }
+      const StageMeta mt = meta[st];
+      if (mt.flags & F_END) break;
+      const bool first = mt.flags & F_FIRST;
+      const int sb = i & 1;
+      if (first) {
+#pragma unroll
+        for (int cq = 0; cq < kWideCols; ++cq) lp[cq] = 0.f;
+      }
+      if (!mbar_wait_bounded(&sfull[sb], (uint32_t)((i >> 1) & 1), abort_flag, kWaitLimitNs)) {
+        if (lane == 0) {
+          *abort_flag = 1;
+          if (a.status) atomicOr(a.status, DEV_TIMEOUT);
+        }
+        break;
+      }
+      tc_fence_after();
+      float s[kWideCols];
+#pragma unroll
+      for (int k = 0; k < kWideCols / 16; ++k) {
+        if (k < nchk) {
+          float v[16];
+          tmem_ld16(trow_addr + (uint32_t)(sb * 64 + 16 * k), v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) s[16 * k + j] = v[j];
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) s[16 * k + j] = -INFINITY;
+        }
+      }
+      tmem_wait_ld();
+      const int nvalid = (mt.nunits * kUnit < mt.ctx - mt.tok0) ? mt.nunits * kUnit : mt.ctx - mt.tok0;
+      const bool tv = r < nvalid;
+      // causal limit: new token j sees stage rows < lim0 + j (a prefix launch: no mask)
+      const int lim0 = MODE == kPrefix ? (1 << 30) : mt.ctx - a.q_len + 1 - mt.tok0;
+      const float* mcur = mref + cur * kWideCols;
+      float e = -INFINITY;
+#pragma unroll
+      for (int cq = 0; cq < kWideCols; ++cq) {
+        bool vis = tv && cq < a.ncol;
+        if (MODE != kPrefix && r >= lim0) vis = vis && r < lim0 + cq / group;
+        s[cq] = vis ? s[cq] * a.scale_log2 : -INFINITY;
+        const float m = first ? -INFINITY : mcur[cq];
+        e = fmaxf(e, s[cq] - m);                  // NaN (-inf - -inf) is ignored
+      }
+      const bool slow = bar_red_or(1, kWideSoftThreads, first || e > kRescaleLog2);
+      if (slow) {
+        // move the reference maxima: stage column maxima over the 128 rows
+#pragma unroll
+        for (int cq = 0; cq < kWideCols; ++cq) {
+          if (cq < nq) {
+            const float wm = warp_max_f32(s[cq]);
+            if (lane == (cq & 31)) red[cq * 4 + q4] = wm;
+          }
+        }
+        named_bar_sync(1, kWideSoftThreads);
+        float* mnext = mref + (cur ^ 1) * kWideCols;
+#pragma unroll
+        for (int cq = 0; cq < kWideCols; ++cq) {
+          if (cq < nq) {
+            const float4 w4 = *reinterpret_cast<const float4*>(red + cq * 4);
+            const float cm = fmaxf(fmaxf(w4.x, w4.y), fmaxf(w4.z, w4.w));
+            const float mo = first ? -INFINITY : mcur[cq];
+            const float mn = fmaxf(mo, cm);
+            const float al = (mo == -INFINITY) ? 0.f : ex2(mo - mn);
+            lp[cq] *= al;
+            if (r == cq) {
+              mnext[cq] = mn;
+              alph[cq] = al;
+            }
+          }
+        }
+        named_bar_sync(1, kWideSoftThreads);
+        cur ^= 1;
+        if (!first) {
+          // O^T was accumulated against the old maxima: rescale it once the previous
+          // stage's PV is done (its commit freed that stage's slot)
+          if (!mbar_wait_bounded(&empty[pst], pph, abort_flag, kWaitLimitNs)) {
+            if (lane == 0) {
+              *abort_flag = 1;
+              if (a.status) atomicOr(a.status, DEV_TIMEOUT);
+            }
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < kWideCols / 16; ++k) {
+            if (k < nchk) {
+              float v[16];
+              tmem_ld16(trow_addr + (uint32_t)(128 + 16 * k), v);
+              tmem_wait_ld();
+#pragma unroll
+              for (int j = 0; j < 16; ++j) v[j] *= alph[16 * k + j];
+              tmem_st16(trow_addr + (uint32_t)(128 + 16 * k), v);
+            }
+          }
+          tmem_wait_st();
+        }
+      }
+      // P^T row r: p = 2^(x - m), 16-bit high part and residual, 8 columns per 16-byte chunk
+      {
+        const float* mc = mref + cur * kWideCols;
+        uint8_t* sP = smem + st * L::kStageBytes + L::kPOff;
+#pragma unroll
+        for (int ch = 0; ch < kWideCols / 8; ++ch) {
+          if (ch * 8 < nq) {
+            const float4 m0 = *reinterpret_cast<const float4*>(mc + ch * 8);
+            const float4 m1 = *reinterpret_cast<const float4*>(mc + ch * 8 + 4);
+            // a column with no visible row yet keeps max -inf: 0 as its reference gives p = 0
+            float mm[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+#pragma unroll
+            for (int j = 0; j < 8; ++j) mm[j] = mm[j] == -INFINITY ? 0.f : mm[j];
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int j = 0; j < 8; j += 2) {
+              const float p0 = ex2(s[ch * 8 + j] - mm[j]);
+              const float p1 = ex2(s[ch * 8 + j + 1] - mm[j + 1]);
+              lp[ch * 8 + j] += p0;
+              lp[ch * 8 + j + 1] += p1;
+              const uint32_t h = pack2<T>(p0, p1);
+              const float2 hf = unpack2<T>(h);
+              hi[j / 2] = h;
+              lo[j / 2] = pack2<T>(p0 - hf.x, p1 - hf.y);
+            }
+            const int off = r * 128 + ((ch ^ (r & 7)) << 4);
+            *reinterpret_cast<uint4*>(sP + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint4*>(sP + L::kPBytes + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          }
+        }
+        if (!tv) {
+          // a row past the stage's valid tokens may hold stale or NaN data: P is zero
+          // there, and V must be finite (0 x NaN would poison O)
+          uint8_t* sV = smem + st * L::kStageBytes + L::kKvBytes;
+#pragma unroll
+          for (int hf = 0; hf < L::kHalves; ++hf)
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch)
+              *reinterpret_cast<uint4*>(sV + hf * (kWideTile * 128) + r * 128 + ch * 16) =
+                  make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      fence_proxy_async_smem();                    // P and V rows -> the tensor cores
+      tc_fence_before();
+      mbar_arrive(&pfull[sb]);
+      if (mt.flags & F_LAST) {
+        // ---- end of a segment portion: row sums, then O^T back from tensor memory
+#pragma unroll
+        for (int cq = 0; cq < kWideCols; ++cq) {
+          if (cq < nq) {
+            float v = lp[cq];
+            v += __shfl_xor_sync(0xffffffffu, v, 16);
+            v += __shfl_xor_sync(0xffffffffu, v, 8);
+            v += __shfl_xor_sync(0xffffffffu, v, 4);
+            v += __shfl_xor_sync(0xffffffffu, v, 2);
+            v += __shfl_xor_sync(0xffffffffu, v, 1);
+            if (lane == (cq & 31)) red[cq * 4 + q4] = v;
+          }
+        }
+        named_bar_sync(1, kWideSoftThreads);
+        if (!mbar_wait_bounded(&empty[st], ph, abort_flag, kWaitLimitNs)) {   // this PV done
+          if (lane == 0) {
+            *abort_flag = 1;
+            if (a.status) atomicOr(a.status, DEV_TIMEOUT);
+          }
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < kWideCols / 16; ++k) {
+          if (k < nchk) {
+            float v[16];
+            tmem_ld16(trow_addr + (uint32_t)(128 + 16 * k), v);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) s[16 * k + j] = v[j];
+          }
+        }
+        tmem_wait_ld();
+        tc_fence_before();
+        // head dim of this thread's O^T lane: lane r at D 128; at D 64 (M = 64) dims
+        // 16 q4 .. 16 q4 + 15 sit in lanes 0..15 of quadrant q4
+        const int d = D == 128 ? r : (lane < 16 ? q4 * 16 + lane : -1);
+        const bool complete = mt.flags & F_COMPLETE;
+        const float* mc = mref + cur * kWideCols;
+#pragma unroll
+        for (int cq = 0; cq < kWideCols; ++cq) {
+          if (cq < a.ncol && d >= 0) {
+            const float4 w4 = *reinterpret_cast<const float4*>(red + cq * 4);
+            const float Ls = (w4.x + w4.y) + (w4.z + w4.w);
+            const float M = mc[cq];
+            if (complete) {
+              const long long row = out_row<MODE>(a, mt.seq, mt.kvh, cq);
+              if (row >= 0) {
+                if constexpr (MODE == kPrefix) {
+                  if (d == 0) a.ext_ml[row] = make_float2(M, Ls);
+                  a.ext_acc[row * D + d] = s[cq];
+                } else {
+                  static_cast<T*>(a.out)[row * D + d] = from_float<T>(Ls > 0.f ? s[cq] / Ls : 0.f);
+                }
+              }
+            } else {
+              const long long prow = (long long)mt.pidx * kWideCols + cq;
+              a.part_acc[prow * D + d] = s[cq];
+              if (d == 0) {
+                a.part_ml[prow * 2 + 0] = M;
+                a.part_ml[prow * 2 + 1] = Ls;
+              }
+            }
+          }
+        }
+        if (!complete) {
+          // arrival on the segment's counter (as in decode.cuh): the last contributor merges
+          named_bar_sync(1, kWideSoftThreads);
+          const SplitDesc dsc = desc[mt.qslot];
+          if (tid == 0) {
+            unsigned long long* ctr = a.counters + dsc.cf;
+            unsigned long long old =
+                dsc.cf == c ? ((unsigned long long)a.epoch << 32) | (uint32_t)(dsc.ncontrib - 1) : 0ull,
+                nxt;
+            for (;;) {
+              nxt = (uint32_t)(old >> 32) == a.epoch ? old + 1
+                                                      : ((unsigned long long)a.epoch << 32) | 1ull;
+              const unsigned long long prev = cas_acq_rel_gpu(ctr, old, nxt);
+              if (prev == old) break;
+              old = prev;
+            }
+            const bool last = (int)(uint32_t)nxt == dsc.ncontrib;
+            if (last) st_relaxed_gpu(ctr, 0ull);
+            *last_flag = last;
+          }
+          named_bar_sync(1, kWideSoftThreads);
+          if (*last_flag) merge_wide<T, D, MODE>(a, dsc, *total_s, G, tid);
+        }
+        named_bar_sync(1, kWideSoftThreads);       // red[] is reused by the next stage
+      }
+      pst = st;
+      pph = ph;
+      if (++st == kWideStages) {
+        st = 0;
+        ph ^= 1u;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, kWideTmemCols);
+  }
+}
+
+}  // namespace pkv

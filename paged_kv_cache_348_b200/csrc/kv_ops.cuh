@@ -142,4 +142,32 @@ __global__ void __launch_bounds__(256)
   for (long long i = threadIdx.x; i < chunks_per_block; i += blockDim.x) d[i] = s[i];
 }
 
+// Preemption ("Paged Attention and Memory Efficiency in Production LLM Serving", section
+// "Why KV cache memory was the bottleneck": requests are preempted when the cache runs
+// out): the blocks of a preempted sequence are saved to a buffer the device can reach
+// (page-locked host memory) and later restored into fresh blocks.  Buffer layout:
+// [layer][pool: K, V][i][block], blocks[i] naming the pool block of entry i.
+// grid = (n, layers * 2 pools); layer0 = the first layer of this launch's pointers.
+template <bool kOut>
+__global__ void __launch_bounds__(256)
+    pa_swap_blocks_kernel(const __grid_constant__ LayerPtrs P, const int32_t* __restrict__ blocks,
+                          int n, int num_blocks, long long chunks_per_block, int layer0,
+                          uint4* buf, int32_t* status) {
+  pdl_wait();
+  pdl_trigger();
+  const int i = blockIdx.x;
+  const int layer = blockIdx.y >> 1, pool = blockIdx.y & 1;
+  const int b = blocks[i];
+  if ((unsigned)b >= (unsigned)num_blocks) {
+    if (status && threadIdx.x == 0) atomicOr(status, DEV_BAD_PAIR);
+    return;
+  }
+  uint4* dev = (pool ? P.v[layer] : P.k[layer]) + (long long)b * chunks_per_block;
+  uint4* h = buf + (((long long)(layer0 + layer) * 2 + pool) * n + i) * chunks_per_block;
+  for (long long j = threadIdx.x; j < chunks_per_block; j += blockDim.x) {
+    if constexpr (kOut) h[j] = dev[j];
+    else dev[j] = h[j];
+  }
+}
+
 }  // namespace pkv

@@ -9,6 +9,7 @@
 #include <cstdlib>
 
 #include "decode.cuh"
+#include "decode_wide.cuh"
 #include "pagedkv.h"
 
 namespace pkv_host {
@@ -113,5 +114,54 @@ PKV_DECL_RUN(pkv::kSuffix, false)
 PKV_DECL_RUN(pkv::kAppend, false)
 PKV_DECL_RUN(pkv::kPlain, true)
 #undef PKV_DECL_RUN
+
+// ---- the tcgen05 kernel for 17..64 query rows per kv head (decode_wide.cuh)
+template <typename T, int D, int BS, int MODE>
+pa_status launch_wide(const pkv::DecodeArgs& a, const CUtensorMap& mk, const CUtensorMap& mv,
+                      int grid, cudaStream_t stream) {
+  using L = pkv::WideLayout<D>;
+  auto k = pkv::pa_decode_wide_kernel<T, D, BS, MODE>;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynSmem) !=
+      cudaSuccess)
+    return PA_ERR_CUDA;
+  if (launch(k, dim3(grid), dim3(pkv::kWideThreads), L::kDynSmem, stream, a, mk, mv) !=
+      cudaSuccess)
+    return PA_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+template <typename T, int MODE>
+pa_status dispatch_wide(int d, int bs, const pkv::DecodeArgs& a, const CUtensorMap& mk,
+                        const CUtensorMap& mv, int grid, cudaStream_t s) {
+  if (d == 64) {
+    switch (bs) {
+      case 1: return launch_wide<T, 64, 1, MODE>(a, mk, mv, grid, s);
+      case 8: return launch_wide<T, 64, 8, MODE>(a, mk, mv, grid, s);
+      case 16: return launch_wide<T, 64, 16, MODE>(a, mk, mv, grid, s);
+      case 32: return launch_wide<T, 64, 32, MODE>(a, mk, mv, grid, s);
+    }
+  } else {
+    switch (bs) {
+      case 1: return launch_wide<T, 128, 1, MODE>(a, mk, mv, grid, s);
+      case 8: return launch_wide<T, 128, 8, MODE>(a, mk, mv, grid, s);
+      case 16: return launch_wide<T, 128, 16, MODE>(a, mk, mv, grid, s);
+      case 32: return launch_wide<T, 128, 32, MODE>(a, mk, mv, grid, s);
+    }
+  }
+  return PA_ERR_UNSUPPORTED;
+}
+
+// One mode's wide instances (kPlain or kPrefix); defined in decode_wide_<mode>.cu.
+template <int MODE>
+pa_status run_wide_mode(bool bf16, int d, int bs, const pkv::DecodeArgs& a, const CUtensorMap& mk,
+                        const CUtensorMap& mv, int grid, cudaStream_t s);
+template <>
+pa_status run_wide_mode<pkv::kPlain>(bool bf16, int d, int bs, const pkv::DecodeArgs& a,
+                                     const CUtensorMap& mk, const CUtensorMap& mv, int grid,
+                                     cudaStream_t s);
+template <>
+pa_status run_wide_mode<pkv::kPrefix>(bool bf16, int d, int bs, const pkv::DecodeArgs& a,
+                                      const CUtensorMap& mk, const CUtensorMap& mv, int grid,
+                                      cudaStream_t s);
 
 }  // namespace pkv_host

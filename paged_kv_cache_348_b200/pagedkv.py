@@ -31,7 +31,8 @@ EXPORTS = ("pa_version", "pa_status_string", "pa_decode_workspace_bytes", "pa_de
            "pa_bm_create", "pa_bm_destroy", "pa_bm_free_blocks", "pa_bm_refcount",
            "pa_bm_allocate", "pa_bm_fork", "pa_bm_append_tokens", "pa_bm_release",
            "pa_bm_context_len", "pa_bm_num_blocks_of", "pa_bm_max_blocks", "pa_bm_block_tables",
-           "pa_bm_slot_of")
+           "pa_bm_slot_of", "pa_bm_plan_cascade", "pa_plan_cascade", "pa_bm_swap_out",
+           "pa_bm_swap_in", "pa_swap_out_blocks", "pa_swap_in_blocks")
 
 _lib = None
 _lock = threading.Lock()
@@ -82,6 +83,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         L.pa_cache_append.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, P, P]
         L.pa_copy_blocks.restype = i32
         L.pa_copy_blocks.argtypes = [P, P, i32, P, i32, i32, sz, P, P]
+        L.pa_swap_out_blocks.restype = i32
+        L.pa_swap_out_blocks.argtypes = [P, P, P, i32, P, i32, i32, sz, P, P]
+        L.pa_swap_in_blocks.restype = i32
+        L.pa_swap_in_blocks.argtypes = [P, P, i32, P, i32, i32, P, sz, P, P]
         _lib = L
         return L
 
@@ -337,6 +342,52 @@ def pa_copy_blocks(k_caches, v_caches, pairs, status=None, stream=None):
     rc = load().pa_copy_blocks(kp, vp, L, _ptr(pairs), pairs.shape[0], shape[0], block_bytes,
                                _ptr(status), _stream(stream))
     _check(rc, "pa_copy_blocks")
+
+
+def _pool_args(k_caches, v_caches):
+    L = len(k_caches)
+    if L != len(v_caches) or L == 0:
+        raise PagedKVError("need the same non-zero number of K and V pools")
+    shape, dt = k_caches[0].shape, k_caches[0].dtype
+    for i, c in enumerate(list(k_caches) + list(v_caches)):
+        _need(c, "cache[%d]" % i, dtype=dt, ndim=4)
+        if c.shape != shape:
+            raise PagedKVError("all pools must have one shape")
+    kp = (ctypes.c_void_p * L)(*[c.data_ptr() for c in k_caches])
+    vp = (ctypes.c_void_p * L)(*[c.data_ptr() for c in v_caches])
+    block_bytes = shape[1] * shape[2] * shape[3] * k_caches[0].element_size()
+    return L, kp, vp, shape[0], block_bytes
+
+
+def swap_buffer_bytes(k_caches, n: int) -> int:
+    """Bytes of the buffer that holds n blocks of every layer's K and V pool."""
+    c = k_caches[0]
+    return len(k_caches) * 2 * n * c.shape[1] * c.shape[2] * c.shape[3] * c.element_size()
+
+
+def pa_swap_out_blocks(buf, k_caches, v_caches, blocks, status=None, stream=None):
+    """Save blocks (device int32 [n]) of every layer's K and V pool into buf (pinned host
+    or device uint8, [layer][K|V][i][block]); see pa_swap_out_blocks in include/pagedkv.h."""
+    L, kp, vp, N, bb = _pool_args(k_caches, v_caches)
+    _need(blocks, "blocks", dtype=torch.int32, ndim=1)
+    n = blocks.shape[0]
+    if not buf.is_contiguous() or buf.numel() * buf.element_size() < L * 2 * n * bb:
+        raise PagedKVError("pa_swap_out_blocks: buffer too small or not contiguous")
+    rc = load().pa_swap_out_blocks(_ptr(buf), kp, vp, L, _ptr(blocks), n, N, bb, _ptr(status),
+                                   _stream(stream))
+    _check(rc, "pa_swap_out_blocks")
+
+
+def pa_swap_in_blocks(k_caches, v_caches, blocks, buf, status=None, stream=None):
+    """Restore buf (as written by pa_swap_out_blocks) into blocks (device int32 [n])."""
+    L, kp, vp, N, bb = _pool_args(k_caches, v_caches)
+    _need(blocks, "blocks", dtype=torch.int32, ndim=1)
+    n = blocks.shape[0]
+    if not buf.is_contiguous() or buf.numel() * buf.element_size() < L * 2 * n * bb:
+        raise PagedKVError("pa_swap_in_blocks: buffer too small or not contiguous")
+    rc = load().pa_swap_in_blocks(kp, vp, L, _ptr(blocks), n, N, _ptr(buf), bb, _ptr(status),
+                                  _stream(stream))
+    _check(rc, "pa_swap_in_blocks")
 
 
 NOALLOC_MAX_SEQS = 16384

@@ -121,14 +121,18 @@ def _finish(w, bs, bm, sids, N, layers, device, cow_pairs=None, q_len=1,
 
 
 def build(w: inputs.Workload, device="cuda", block_size: int | None = None,
-          layers: int | None = None, q_len: int = 1, kv8: bool = False) -> DecodeBatch:
+          layers: int | None = None, q_len: int = 1, kv8: bool = False,
+          contiguous: bool = False) -> DecodeBatch:
     """Independent sequences (every workload but the shared-prefix one).  With q_len > 1
-    every sequence's newest q_len tokens are appended and queried each step."""
+    every sequence's newest q_len tokens are appended and queried each step.  With
+    contiguous=True the pool hands out blocks in id order, so every sequence's table is
+    one run of consecutive blocks (the identity placement a contiguous cache would have)
+    instead of the seeded fragmented one."""
     bs = block_size or w.block_size
     ctx = inputs.context_lens(w)
     need = int(sum(-(-int(c) // bs) for c in ctx))
     N = _pool_size(w, need)
-    bm = BlockManager(N, bs, inputs.pool_order(N, w.seed))
+    bm = BlockManager(N, bs, None if contiguous else inputs.pool_order(N, w.seed))
     sids = [bm.allocate(int(c)) for c in ctx]
     return _finish(w, bs, bm, sids, N, layers or w.layers, device, q_len=q_len, kv8=kv8)
 
@@ -207,10 +211,9 @@ def append_decode_layer(b: DecodeBatch, l: int, stream=None, block_tables=None,
 def use_cascade(b: DecodeBatch, width: int | None = None) -> DecodeBatch:
     """Decode this batch with pa_decode_cascade: plan the shared-prefix chunks from its
     block tables (the workspace grows to the cascade size)."""
-    tables, ctx = b.block_tables.cpu().numpy(), b.context_lens.cpu().numpy()
     w = b.w
-    prefix, members, plens = plan_cascade(tables, ctx, b.block_size,
-                                          w.num_q_heads // w.num_kv_heads, width)
+    ctx = b.context_lens.cpu().numpy()
+    prefix, members, plens = b.bm.plan_cascade(b.sids, w.num_q_heads // w.num_kv_heads, width)
     dev = b.block_tables.device
     b.cascade = (torch.from_numpy(prefix).to(dev), torch.from_numpy(members).to(dev),
                  torch.from_numpy(plens).to(dev))
@@ -238,37 +241,10 @@ def decode_layer(b: DecodeBatch, l: int, stream=None) -> None:
 def plan_cascade(tables: np.ndarray, ctx: np.ndarray, block_size: int, group: int,
                  width: int | None = None):
     """Chunks of sequences that share a prefix of their block tables, for
-    pa_decode_cascade.  Sequences whose first block is the same physical block form a
-    sharing group; its prefix is the leading table entries common to all members,
-    capped at the shortest member's length.  Groups of one sequence get no chunk.
-    Returns (prefix_lens int32 [B], chunk_members int32 [C, width], chunk_prefix_lens
-    int32 [C]); a chunk holds at most `width` members (default: 16 query rows per chunk,
-    which reads each shared prefix least often; group * width <= 16)."""
-    B = len(ctx)
-    cap = width or max(1, 16 // group)
-    by_first = {}
-    for s in range(B):
-        if ctx[s] > 0:
-            by_first.setdefault(int(tables[s, 0]), []).append(s)
-    prefix = np.zeros(B, dtype=np.int32)
-    members, plens = [], []
-    for mem in by_first.values():
-        if len(mem) < 2:
-            continue
-        nb = min(-(-int(ctx[s]) // block_size) for s in mem)
-        common = 0
-        while common < nb and all(tables[s, common] == tables[mem[0], common] for s in mem):
-            common += 1
-        plen = min(common * block_size, min(int(ctx[s]) for s in mem))
-        if plen == 0:
-            continue
-        for i in range(0, len(mem), cap):
-            row = np.full(cap, -1, dtype=np.int32)
-            part = mem[i:i + cap]
-            row[:len(part)] = part
-            members.append(row)
-            plens.append(plen)
-            prefix[part] = plen
-    cm = np.stack(members) if members else np.zeros((0, cap), dtype=np.int32)
-    return prefix, cm, np.array(plens, dtype=np.int32)
+    pa_decode_cascade, planned by the library (pa_plan_cascade): sequences whose first
+    block is the same physical block form a sharing group; its prefix is the leading
+    table entries common to all members, capped at the shortest member's length; a
+    chunk holds at most `width` members (default 64 // group, 64 query rows)."""
+    from .block_manager import plan_cascade_tables
 
+    return plan_cascade_tables(tables, ctx, block_size, group, width)

@@ -53,7 +53,7 @@ def test_decode_host_validation(lib):
     assert _decode(lib, D=96) == pk.PA_ERR_UNSUPPORTED
     assert _decode(lib, bs=4) == pk.PA_ERR_UNSUPPORTED
     assert _decode(lib, Hq=9, Hkv=2) == pk.PA_ERR_INVALID
-    assert _decode(lib, Hq=64, Hkv=2) == pk.PA_ERR_UNSUPPORTED      # group 32 > 16
+    assert _decode(lib, Hq=72, Hkv=1) == pk.PA_ERR_UNSUPPORTED      # group 72 > 64
     assert _decode(lib, dtype=7) == pk.PA_ERR_UNSUPPORTED
     assert _decode(lib, B=0) == pk.PA_OK                              # nothing to do
     assert _decode(lib, ptr=P(0)) == pk.PA_ERR_INVALID                # null pointers

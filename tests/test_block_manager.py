@@ -195,3 +195,71 @@ def test_native_manager_rejects_bad_arguments():
     with pytest.raises(ValueError):
         m.block_tables([s], width=1)
     assert m.block_tables([s], width=3, fill=-1).tolist() == [[0, 1, -1]]
+
+
+def test_random_operations_with_preemption_match_reference_planner():
+    """Differential run as above with swap-outs and swap-ins mixed in: returned blocks,
+    tables, lengths, free and reference counts agree after every operation, and a
+    swapped-out sequence is refused by the calls that need its table."""
+    rng = np.random.default_rng(321)
+    for trial in range(20):
+        N, bs = int(rng.integers(20, 100)), int(rng.choice([1, 4, 8, 16]))
+        order = rng.permutation(N).astype(np.int32)
+        m, r = BlockManager(N, bs, order), RefBlockManager(N, bs, order)
+        live, out = [], []
+        for _ in range(200):
+            op = rng.integers(0, 12)
+            if op < 2 or not (live or out):
+                n = int(rng.integers(0, 3 * bs + 2))
+                try:
+                    sid = m.allocate(n)
+                except PoolExhausted:
+                    continue
+                assert r.new_seq(n) == sid
+                live.append(sid)
+            elif op < 3 and live:
+                p = int(rng.choice(live))
+                c = m.fork(p)
+                assert r.fork(p) == c
+                live.append(c)
+            elif op < 6 and live:
+                sid = int(rng.choice(live))
+                try:
+                    slot, cow = m.append_token(sid)
+                except PoolExhausted:
+                    continue
+                assert (slot, cow) == r.append_slot(sid)
+            elif op < 8 and live:
+                sid = live.pop(int(rng.integers(len(live))))
+                got = m.swap_out(sid)
+                assert got.tolist() == r.swap_out(sid)
+                out.append(sid)
+                with pytest.raises(ValueError):
+                    m.append_token(sid)
+                with pytest.raises(ValueError):
+                    m.fork(sid)
+                assert m.context_len(sid) == r.ctx[sid]
+            elif op < 10 and out:
+                sid = int(rng.choice(out))
+                try:
+                    got = m.swap_in(sid)
+                except PoolExhausted:
+                    with pytest.raises(MemoryError):
+                        r.swap_in(sid)
+                    continue
+                assert got.tolist() == r.swap_in(sid)
+                out.remove(sid)
+                live.append(sid)
+            else:
+                pool = live + out
+                if not pool:
+                    continue
+                sid = int(rng.choice(pool))
+                m.release(sid)
+                r.release(sid)
+                (live if sid in live else out).remove(sid)
+            assert m.free_blocks == len(r.free)
+            for sid in live:
+                assert m.table(sid) == r.tables[sid] and m.context_len(sid) == r.ctx[sid]
+            for b in range(N):
+                assert m.refcount(b) == r.ref[b]

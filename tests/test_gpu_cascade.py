@@ -88,7 +88,9 @@ GROUPS = [(40, [3, 0, 17, 1]), (0, [5]), (33, [0, 0]), (64, [1, 2, 3, 4, 5, 6, 7
 @pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("bs", [1, 8, 16, 32])
 @pytest.mark.parametrize("Hq,Hkv,width", [(8, 2, 2), (8, 2, 4), (32, 8, 2), (4, 4, 8), (4, 4, 16),
-                                          (16, 1, 1)])
+                                          (16, 1, 1),
+                                          # chunks wider than 16 query rows: tcgen05 prefix pass
+                                          (32, 8, 8), (8, 2, 16), (16, 1, 4)])
 def test_cascade_matches_oracle(dtype, D, bs, Hq, Hkv, width):
     case = shared_case(GROUPS, Hq, Hkv, D, bs, dtype, seed=400 + D + bs + Hq)
     plan = wl.plan_cascade(case["tables"], case["ctx"], bs, Hq // Hkv, width)
@@ -124,7 +126,7 @@ def test_cascade_shared_prefix_workload_full_size():
     b = wl.build_prefix_decode()
     tables, ctx = b.block_tables.cpu().numpy(), b.context_lens.cpu().numpy()
     prefix, members, plens = wl.plan_cascade(tables, ctx, b.block_size, 4)
-    assert (prefix == inputs.PREFIX_LEN).all() and len(plens) == 32       # 2 chunks a prompt
+    assert (prefix == inputs.PREFIX_LEN).all() and len(plens) == 16       # 1 chunk a prompt
     out = torch.empty_like(b.q[0])
     ws = pk.new_cascade_workspace(128, 32, 8, 128)
     dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()

@@ -412,3 +412,46 @@ def test_release_conserves_the_pool_under_random_forks_and_appends():
         for s in live:
             bm.release(s)
         assert sorted(bm.free) == list(range(N)) and not any(bm.ref) and not bm.tables
+
+
+# ---- RefBlockManager.swap_out / swap_in (preemption): "Paged Attention and Memory
+# Efficiency in Production LLM Serving", "Why KV cache memory was the bottleneck"
+# (requests are preempted when the cache runs out), with the release rule of
+# "PagedAttention in Production", "Core Principle".
+
+def test_swap_out_releases_like_release_and_keeps_the_length():
+    bm = RefBlockManager(10, 4, [9, 8, 7, 6, 5, 4, 3, 2, 1, 0])
+    a = bm.new_seq(9)                                      # 9, 8, 7
+    b = bm.fork(a)
+    bm.append_slot(b)                                      # b copies partial block 7 -> 6
+    assert bm.tables[b] == [9, 8, 6] and bm.free == [5, 4, 3, 2, 1, 0]
+    out = bm.swap_out(b)
+    assert out == [9, 8, 6]                                 # table order, to be saved
+    assert bm.ref[9] == 1 and bm.ref[8] == 1 and bm.ref[6] == 0   # shared ones stay with a
+    assert bm.free == [5, 4, 3, 2, 1, 0, 6] and bm.ctx[b] == 10 and bm.tables[b] == []
+    assert bm.tables[a] == [9, 8, 7] and bm.ctx[a] == 9
+
+
+def test_swap_in_takes_fresh_blocks_from_the_front():
+    bm = RefBlockManager(8, 4, [3, 1, 4, 0, 5, 2, 6, 7])
+    a = bm.new_seq(10)                                     # 3, 1, 4
+    out = bm.swap_out(a)
+    assert out == [3, 1, 4] and bm.free == [0, 5, 2, 6, 7, 3, 1, 4]
+    c = bm.new_seq(20)                                     # 0, 5, 2, 6, 7: reuses nothing yet
+    assert bm.tables[c] == [0, 5, 2, 6, 7]
+    back = bm.swap_in(a)
+    assert back == [3, 1, 4] and bm.tables[a] == [3, 1, 4] and bm.free == []
+    assert all(bm.ref[x] == 1 for x in back) and a not in bm.swapped and bm.ctx[a] == 10
+
+
+def test_swap_in_that_does_not_fit_changes_nothing():
+    bm = RefBlockManager(4, 4)
+    a = bm.new_seq(12)                                     # 0, 1, 2
+    bm.swap_out(a)
+    c = bm.new_seq(8)                                      # 3, 0
+    free0, ref0 = list(bm.free), list(bm.ref)
+    with pytest.raises(MemoryError):
+        bm.swap_in(a)                                      # needs 3, 2 free
+    assert bm.free == free0 and bm.ref == ref0 and a in bm.swapped and bm.tables[a] == []
+    bm.release(c)
+    assert len(bm.swap_in(a)) == 3
