@@ -34,6 +34,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "paged decode attn: KV-read HBM GB/s (% of B200 peak) and seq-steps/s"
 FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 1024 * 1024
 
 
 def max_over_ranks(x: float, world: int, device="cuda") -> float:
@@ -234,6 +235,10 @@ def run_reference(args, w, bs, rank, world):
         "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * (t_all / max(1, s_all)) * w.num_seqs * w.layers,
+        "ms_per_step_extrapolated": True,
+        "ms_per_step_basis": "oracle time per sampled whole sequence of layer 0, x %d sequences "
+                             "x %d layers (the step is never run whole on the CPU)" % (
+                                 w.num_seqs, w.layers),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": {"workload": workload_desc(w, bs), "parallelism": "cpu"},
         "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
@@ -252,7 +257,7 @@ def run_reference(args, w, bs, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=150)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama70b")
@@ -270,6 +275,9 @@ def main():
                     help="layers of the workload to run (0: all; fewer only for profiling)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the other workloads' per-launch measurements")
+    ap.add_argument("--secondary-iters", type=int, default=20)
     args = ap.parse_args()
 
     from paged_kv_cache_348_b200 import inputs
@@ -370,6 +378,7 @@ def main():
     value = job_gbs(world, kv_step, ms_step)
     peak, peak_kind = measured_hbm_peak()
     dec_avg_events = statistics.mean(dec_ms)
+    dec_med_events = statistics.median(dec_ms)
     only_decode = fused and not (b.cow_pairs is not None and b.cow_pairs.shape[0])
     if only_decode:
         dec_avg = ms_local / (args.steps * L)
@@ -411,6 +420,7 @@ def main():
                      "algorithmic_bytes_per_launch": kv_layer,
                      "avg_launch_ms": dec_avg, "avg_launch_ms_from": dec_src,
                      "avg_launch_ms_event_pairs": dec_avg_events,
+                     "median_launch_ms_event_pairs": dec_med_events,
                      "launches_timed": args.steps * L if only_decode else len(dec_ms),
                      "peak_source": peak_kind},
         "gpu_launches": launches,
@@ -424,6 +434,10 @@ def main():
         line["roofline_unique_bytes"] = {
             "achieved": uniq / L / (dec_avg * 1e-3) / 1e9, "peak": peak, "unit": "GB/s",
             "frac": uniq / L / (dec_avg * 1e-3) / 1e9 / peak}
+    if w.name == "llama70b" and not args.no_secondary and b.q_len == 1 and b.kv_scales is None \
+            and b.cascade is None:
+        # the other workloads, built one at a time beside the step's buffers
+        line["secondary"] = secondary_measurements(args, peak)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         nbytes, sec, seqs, threads = oracle_sample(w, bs, device_batch=b)
         n1, sec1, seqs1, _ = oracle_sample(w, bs, max_seconds=3.0, device_batch=b, nthreads=1)
@@ -542,6 +556,154 @@ def run_e2e(b, args, world, kv_step, fused=False):
             "copies": "pinned host buffers; uploads and read-backs on two copy streams, "
                       "overlapped with compute layer by layer"}
 
+
+
+# ------------------------------------------------------------------------------- secondary
+def time_launches(torch, fn, n, warmup, flush=None):
+    """Device time of fn() (one decode call: one or two library launches on the current
+    stream) with an event pair around each call; `flush` (an L2 flush) runs before each
+    timed call, outside the events.  Returns (median ms, mean ms)."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    evs = []
+    for _ in range(n):
+        if flush is not None:
+            flush()
+        a = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        e.record()
+        evs.append((a, e))
+    torch.cuda.synchronize()
+    ts = [a.elapsed_time(e) for a, e in evs]
+    return statistics.median(ts), statistics.mean(ts)
+
+
+def tail_waste_table():
+    """Fraction of held cache slots that hold no token (the unused tail of each
+    sequence's last block; shared blocks counted once per sequence), per workload and
+    block size: host bookkeeping only."""
+    from paged_kv_cache_348_b200 import inputs
+    from paged_kv_cache_348_b200.block_manager import BlockManager
+
+    out = {}
+    for name in ("tiny", "llama8b", "llama70b", "prefix", "heavytail"):
+        w = inputs.WORKLOADS[name]
+        ctx = [int(c) for c in inputs.context_lens(w)]
+        row = {}
+        for bs in (1, 8, 16, 32):
+            held = sum(-(-c // bs) * bs for c in ctx)
+            row["bs%d" % bs] = (held - sum(ctx)) / held
+        if name == "prefix":
+            # the shared 2048-token prefix is held once per prompt (block aligned at
+            # these sizes), the private tokens per sample
+            for bs in (1, 8, 16, 32):
+                bm = BlockManager(10 ** 6, bs)
+                sids = []
+                for p in range(inputs.PREFIX_PROMPTS):
+                    root = bm.allocate(inputs.PREFIX_LEN)
+                    kids = [root] + [bm.fork(root) for _ in range(inputs.PREFIX_SAMPLES - 1)]
+                    for j, sid in enumerate(kids):
+                        for _ in range(ctx[p * inputs.PREFIX_SAMPLES + j] - inputs.PREFIX_LEN):
+                            bm.append_token(sid)
+                        sids.append(sid)
+                held_slots = (10 ** 6 - bm.free_blocks) * bs
+                row["bs%d_unique" % bs] = (held_slots - (inputs.PREFIX_PROMPTS * inputs.PREFIX_LEN +
+                                                         sum(c - inputs.PREFIX_LEN for c in ctx))) \
+                    / held_slots
+        out[name] = row
+    return out
+
+
+def secondary_measurements(args, peak):
+    """Per-launch device time, KV-read rate and roofline fraction of the other workloads
+    (each built on its own, measured, and freed): the 8B shape, the heavy-tailed batch at
+    every block size, the shared-prefix batch (plain and cascade), 8-bit pools, several
+    new tokens per sequence, and identity (contiguous) against fragmented placement.  Calls
+    are timed one at a time with an event pair; when a layer's K/V pools are under 4x the
+    L2 size, a 256 MB buffer is written before each timed call so the pools come from
+    HBM."""
+    import torch
+
+    from paged_kv_cache_348_b200 import inputs
+    from paged_kv_cache_348_b200 import workload as wl
+
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    out = {}
+
+    def measure(name, b, fn, note, kv_bytes=None, unique=None, launches=1):
+        pool = 2 * b.k_caches[0].numel() * b.k_caches[0].element_size()
+        flush = pool < 4 * L2_BYTES
+        med, mean = time_launches(torch, fn, args.secondary_iters, 3,
+                                  (lambda: flush_buf.zero_()) if flush else None)
+        st = int(b.status.item())
+        if st:
+            raise RuntimeError("%s: device status 0x%x" % (name, st))
+        kvb = kv_bytes if kv_bytes is not None else b.kv_bytes_per_step() // b.layers
+        e = {"workload": note, "median_ms": med, "mean_ms": mean, "kv_bytes": kvb,
+             "gbs": kvb / (med * 1e-3) / 1e9, "frac": kvb / (med * 1e-3) / 1e9 / peak,
+             "launches_per_call": launches, "l2_flush": flush,
+             "seqs_per_s": len(b.sids) / (med * 1e-3)}
+        if unique is not None:
+            e["unique_kv_bytes"] = unique
+            e["unique_gbs"] = unique / (med * 1e-3) / 1e9
+            e["unique_frac"] = e["unique_gbs"] / peak
+        out[name] = e
+
+    def fused(b):
+        return lambda: wl.append_decode_layer(b, 0)
+
+    def plain(b):
+        return lambda: wl.decode_layer(b, 0)
+
+    runs = [
+        ("llama70b_layer", lambda: wl.build(inputs.LLAMA70B, layers=1), fused,
+         "70B shape, one layer, fragmented placement, pa_decode_append"),
+        ("llama70b_layer_identity", lambda: wl.build(inputs.LLAMA70B, layers=1, contiguous=True),
+         fused, "70B shape, one layer, identity (contiguous) placement, pa_decode_append"),
+        ("llama70b_q2", lambda: wl.build(inputs.LLAMA70B, layers=1, q_len=2), plain,
+         "70B shape, 2 new tokens a sequence (16 query rows per kv head), pa_decode_multi"),
+        ("llama70b_q4", lambda: wl.build(inputs.LLAMA70B, layers=1, q_len=4), plain,
+         "70B shape, 4 new tokens (32 rows), pa_decode_multi"),
+        ("llama70b_q8", lambda: wl.build(inputs.LLAMA70B, layers=1, q_len=8), plain,
+         "70B shape, 8 new tokens (64 rows), pa_decode_multi"),
+        ("llama70b_e4m3", lambda: wl.build(inputs.LLAMA70B, layers=1, kv8=True), plain,
+         "70B shape, one layer, 8-bit E4M3 pools (bytes counted at 1 per value), "
+         "pa_decode_e4m3"),
+        ("llama8b", lambda: wl.build(inputs.LLAMA8B), fused, "8B shape, pa_decode_append"),
+        ("llama8b_q4", lambda: wl.build(inputs.LLAMA8B, q_len=4), plain,
+         "8B shape, 4 new tokens (16 rows), pa_decode_multi"),
+        ("llama8b_e4m3", lambda: wl.build(inputs.LLAMA8B, kv8=True), plain,
+         "8B shape, 8-bit E4M3 pools, pa_decode_e4m3"),
+    ]
+    for bs in (1, 8, 16, 32):
+        runs.append(("heavytail_bs%d" % bs,
+                     (lambda bs=bs: wl.build(inputs.HEAVYTAIL, block_size=bs)), fused,
+                     "heavy-tailed 256 sequences, block_size %d, pa_decode_append" % bs))
+    runs.append(("heavytail_bs16_identity",
+                 lambda: wl.build(inputs.HEAVYTAIL, block_size=16, contiguous=True), fused,
+                 "heavy-tailed, block_size 16, identity (contiguous) placement"))
+    runs.append(("heavytail_bs1_e4m3",
+                 lambda: wl.build(inputs.HEAVYTAIL, block_size=1, kv8=True), plain,
+                 "heavy-tailed, block_size 1, 8-bit E4M3 pools"))
+    for name, mk, how, note in runs:
+        b = mk()
+        measure(name, b, how(b), note)
+        del b
+        torch.cuda.empty_cache()
+    b = wl.build_prefix_decode()
+    uniq = b.unique_kv_bytes_per_step()
+    measure("prefix_plain", b, plain(b), "shared prefix (16 prompts x 8 samples), pa_decode; "
+            "gbs on logical bytes (a shared block once per reader)", unique=uniq)
+    wl.use_cascade(b)
+    measure("prefix_cascade", b, plain(b), "shared prefix, pa_decode_cascade (prefix pass + "
+            "suffix pass)", unique=uniq, launches=2)
+    del b
+    torch.cuda.empty_cache()
+    out["tail_waste"] = tail_waste_table()
+    return out
 
 if __name__ == "__main__":
     sys.exit(main())

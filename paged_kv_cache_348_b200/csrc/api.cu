@@ -114,9 +114,16 @@ pa_status dispatch_mode(bool kv8, bool wide, int mode, bool bf16, int d, int bs,
                         const pkv::DecodeArgs& a, const CUtensorMap& mk, const CUtensorMap& mv,
                         int grid, cudaStream_t s) {
   using namespace pkv_host;
-  if (wide)
-    return mode == pkv::kPrefix ? run_wide_mode<pkv::kPrefix>(bf16, d, bs, a, mk, mv, grid, s)
-                                : run_wide_mode<pkv::kPlain>(bf16, d, bs, a, mk, mv, grid, s);
+  if (wide) {
+    const int nc = a.ncol <= 16 ? 16 : (a.ncol <= 32 ? 32 : 64);
+    if (mode == pkv::kPrefix)
+      return nc == 16 ? run_wide_mode<pkv::kPrefix, 16>(bf16, d, bs, a, mk, mv, grid, s)
+             : nc == 32 ? run_wide_mode<pkv::kPrefix, 32>(bf16, d, bs, a, mk, mv, grid, s)
+                        : run_wide_mode<pkv::kPrefix, 64>(bf16, d, bs, a, mk, mv, grid, s);
+    return nc == 16 ? run_wide_mode<pkv::kPlain, 16>(bf16, d, bs, a, mk, mv, grid, s)
+           : nc == 32 ? run_wide_mode<pkv::kPlain, 32>(bf16, d, bs, a, mk, mv, grid, s)
+                      : run_wide_mode<pkv::kPlain, 64>(bf16, d, bs, a, mk, mv, grid, s);
+  }
   if (kv8) return run_decode_mode<pkv::kPlain, true>(bf16, d, bs, a, mk, mv, grid, s);
   switch (mode) {
     case pkv::kPlain: return run_decode_mode<pkv::kPlain, false>(bf16, d, bs, a, mk, mv, grid, s);

@@ -20,14 +20,18 @@
 //    accumulated in tensor memory; then O^T[D][N] += V^T . P^T with V read MN-major from
 //    the same tile.  The QK^T of stage i+2 is issued right after the PV of stage i, so the
 //    softmax of stage i+1 overlaps both.
-//  * Warps 2..5 (one thread per token row of S^T, i.e. per TMEM lane) run the softmax:
-//    base-2, fp32, with a lazily moved reference maximum per query row (a stage moves it
-//    only when some score exceeds it by more than 2^8, which after a portion's first stage
-//    is rare; O^T is then rescaled in tensor memory).  P^T is written in 16 bits as a high
-//    part and the rounding residual (~16 mantissa bits in all) into the stage's K tile,
-//    which QK^T no longer needs.  Row sums stay per thread and are reduced once per
-//    portion.  The same warps read O^T back at the end of a portion (one thread per head
-//    dim) and write the output or the split partial.
+//  * Warps 2..9, two warpgroups that split the query columns, run the softmax: a thread
+//    owns one token row of S^T (one TMEM lane) and half of the columns.  Base 2, fp32, with
+//    a lazily moved reference maximum per query row (a stage moves it only when some score
+//    exceeds it by more than 2^8, which after a portion's first stage is rare; O^T is then
+//    rescaled in tensor memory).  P^T is written in 16 bits as a high part and the
+//    rounding residual (~16 mantissa bits in all) into the stage's K tile, which QK^T no
+//    longer needs.  Row sums stay per thread and are reduced once per portion.  The same
+//    warps read O^T back at the end of a portion (one thread per head dim and column half)
+//    and write the output or the split partial.  The column count NC (16, 32 or 64, the
+//    query rows rounded up) is a template parameter, so these loops are exactly as long
+//    as a launch needs: with one CTA per SM the softmax has only two warps per scheduler
+//    to hide latency with, and unused columns or runtime guards cost real time there.
 //  * Every wait is bounded; tensor memory is released on every exit path.
 #pragma once
 #include "decode.cuh"
@@ -38,7 +42,7 @@ constexpr int kWideCols = 64;                     // query rows per kv head hand
 constexpr int kWideTile = 128;                    // tokens per stage (MMA M of QK^T)
 constexpr int kWideUnits = kWideTile / kUnit;     // 16-token units per stage
 constexpr int kWideStages = 3;
-constexpr int kWideSoftThreads = 128;             // softmax warps 2..5
+constexpr int kWideSoftThreads = 256;             // softmax warps 2..9 (two warpgroups)
 constexpr int kWideThreads = 64 + kWideSoftThreads;
 constexpr uint32_t kWideTmemCols = 256;           // S^T x 2 (cols 0..127), O^T (cols 128..191)
 constexpr float kRescaleLog2 = 8.f;               // a reference max moves past this gap only
@@ -61,7 +65,8 @@ struct WideLayout {
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;       // tmem base, abort, last, total
   static constexpr int kDescOff = kMiscOff + 32;
   static constexpr int kMrefOff = (kDescOff + 2 * (int)sizeof(SplitDesc) + 15) / 16 * 16;
-  static constexpr int kRedOff = kMrefOff + 2 * kWideCols * 4;  // float [64 cols][4 warps]
+  // float [3][64]: two reference-max buffers and a row of -inf (a portion's first stage)
+  static constexpr int kRedOff = kMrefOff + 3 * kWideCols * 4;  // float [64 cols][4 warps]
   static constexpr int kAlphaOff = kRedOff + kWideCols * 4 * 4;
   static constexpr int kBytes = kAlphaOff + kWideCols * 4;
   static constexpr int kDynSmem = kBytes + 1024;                // slack for 1024-byte alignment
@@ -74,12 +79,12 @@ struct WideLayout {
 
 // Last arrival of a split segment (see merge_split in decode.cuh), for up to 64 query
 // columns: out = (sum_k acc_k 2^(m_k - M)) / (sum_k l_k 2^(m_k - M)), contributors folded
-// in CTA order.  Thread tid owns elements (column, 4 dims) e = tid + 128 i, 8 at a time.
+// in CTA order.  Thread tid owns elements (column, 4 dims) e = tid + 256 i, 4 at a time.
 template <typename T, int D, int MODE>
 __device__ __forceinline__ void merge_wide(const DecodeArgs& a, const SplitDesc& dsc,
                                            long long total, int G, int tid) {
   constexpr int kF4 = D / 4;
-  constexpr int kB = 8;                                  // elements per batch
+  constexpr int kB = 4;                                  // elements per batch
   const int nel = a.ncol * kF4;
   for (int e0 = tid; e0 < nel; e0 += kB * kWideSoftThreads) {
     float M[kB], Ls[kB];
@@ -133,12 +138,33 @@ __device__ __forceinline__ void merge_wide(const DecodeArgs& a, const SplitDesc&
   }
 }
 
-template <typename T, int D, int BS, int MODE>
+// 8 consecutive 32-bit TMEM columns of this warp's 32 lanes.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* v) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const float* v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(
+                   taddr),
+               "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+               "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+               "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7]))
+               : "memory");
+}
+
+template <typename T, int D, int BS, int MODE, int NC>
 __global__ void __launch_bounds__(kWideThreads, 1)
     pa_decode_wide_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
                           const __grid_constant__ CUtensorMap tmv) {
   using L = WideLayout<D>;
   static_assert(MODE == kPlain || MODE == kPrefix, "wide decode: plain (multi-token) or prefix");
+  static_assert(NC == 16 || NC == 32 || NC == 64, "16, 32 or 64 query columns");
+  constexpr int CW = NC / 2;                        // columns of one softmax warpgroup
   constexpr int kSegW = seg_weight(BS);
   constexpr uint32_t kAB = std::is_same_v<T, __nv_bfloat16> ? 1u : 0u;
   constexpr int kFullCount = 33;       // lane 0's expect_tx arrival + 32 cp.async arrivals
@@ -157,7 +183,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   volatile int* last_flag = abort_flag + 1;
   long long* total_s = reinterpret_cast<long long*>(smem + L::kMiscOff + 16);
   SplitDesc* desc = reinterpret_cast<SplitDesc*>(smem + L::kDescOff);
-  float* mref = reinterpret_cast<float*>(smem + L::kMrefOff);      // [2][64]
+  float* mref = reinterpret_cast<float*>(smem + L::kMrefOff);      // [3][64]
   float* red = reinterpret_cast<float*>(smem + L::kRedOff);        // [64][4]
   float* alph = reinterpret_cast<float*>(smem + L::kAlphaOff);     // [64]
   uint8_t* sQ = smem + L::kQOff;
@@ -174,6 +200,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     }
     mbar_init(qempty, 1);
     mbar_init(drain, 1);
+    for (int i = 0; i < kWideCols; ++i) mref[2 * kWideCols + i] = -INFINITY;
     *abort_flag = 0;
     *last_flag = 0;
     fence_mbar_init();
@@ -195,7 +222,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
 
   const int G = gridDim.x, c = blockIdx.x;
   const int Hkv = a.num_kv_heads, group = a.group;
-  const int nq = (a.ncol + 15) & ~15;               // MMA N: query rows rounded up to 16
+  constexpr int nq = NC;                            // MMA N: the query rows rounded up
 
   if (warp == 0) {
     // ============================== producer ==============================
@@ -558,25 +585,56 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     }
   } else {
     // ============================== softmax / epilogue ==============================
+    const int wg = (warp - 2) >> 2;                // softmax warpgroup: columns c0 .. c0+CW-1
+    const int c0 = wg * CW;
     const int q4 = warp & 3;                       // TMEM lane quadrant of this warp
     const int r = q4 * 32 + lane;                  // token row of S^T (= head dim of O^T at D 128)
     const int tid = threadIdx.x - 64;
     const uint32_t trow_addr = tbase + ((uint32_t)(q4 * 32) << 16);
-    const int nchk = nq / 16;
-    float lp[kWideCols];
+    float lp[CW];                                  // this row's share of the column sums
 #pragma unroll
-    for (int cq = 0; cq < kWideCols; ++cq) lp[cq] = 0.f;
+    for (int j = 0; j < CW; ++j) lp[j] = 0.f;
     int cur = 0;
     int st = 0;
     uint32_t ph = 0;
     int pst = 0;
     uint32_t pph = 0;                              // slot/parity of the previous stage
+    auto give_up = [&]() {
+      if (lane == 0) {
+        *abort_flag = 1;
+        if (a.status) atomicOr(a.status, DEV_TIMEOUT);
+      }
+    };
+    // CW consecutive TMEM columns starting at col of this warp's lanes
+    auto tld = [&](uint32_t col, float* v) {
+      if constexpr (CW == 8) {
+        tmem_ld8(trow_addr + col, v);
+      } else {
+#pragma unroll
+        for (int k = 0; k < CW / 16; ++k) {
+          float w[16];
+          tmem_ld16(trow_addr + col + 16 * k, w);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[16 * k + j] = w[j];
+        }
+      }
+    };
+    auto tst = [&](uint32_t col, const float* v) {
+      if constexpr (CW == 8) {
+        tmem_st8(trow_addr + col, v);
+      } else {
+#pragma unroll
+        for (int k = 0; k < CW / 16; ++k) {
+          float w[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) w[j] = v[16 * k + j];
+          tmem_st16(trow_addr + col + 16 * k, w);
+        }
+      }
+    };
     for (int i = 0;; ++i) {
       if (!mbar_wait_bounded(&full[st], ph, abort_flag, kWaitLimitNs)) {
-        if (lane == 0) {
-          *abort_flag = 1;
-          if (a.status) atomicOr(a.status, DEV_TIMEOUT);
-        }
+        give_up();
         break;
       }
       const StageMeta mt = meta[st];
@@ -585,95 +643,82 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       const int sb = i & 1;
       if (first) {
 #pragma unroll
-        for (int cq = 0; cq < kWideCols; ++cq) lp[cq] = 0.f;
+        for (int j = 0; j < CW; ++j) lp[j] = 0.f;
       }
       if (!mbar_wait_bounded(&sfull[sb], (uint32_t)((i >> 1) & 1), abort_flag, kWaitLimitNs)) {
-        if (lane == 0) {
-          *abort_flag = 1;
-          if (a.status) atomicOr(a.status, DEV_TIMEOUT);
-        }
+        give_up();
         break;
       }
       tc_fence_after();
-      float s[kWideCols];
-#pragma unroll
-      for (int k = 0; k < kWideCols / 16; ++k) {
-        if (k < nchk) {
-          float v[16];
-          tmem_ld16(trow_addr + (uint32_t)(sb * 64 + 16 * k), v);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) s[16 * k + j] = v[j];
-        } else {
-#pragma unroll
-          for (int j = 0; j < 16; ++j) s[16 * k + j] = -INFINITY;
-        }
-      }
+      float s[CW];
+      tld((uint32_t)(sb * 64 + c0), s);
       tmem_wait_ld();
       const int nvalid = (mt.nunits * kUnit < mt.ctx - mt.tok0) ? mt.nunits * kUnit : mt.ctx - mt.tok0;
       const bool tv = r < nvalid;
       // causal limit: new token j sees stage rows < lim0 + j (a prefix launch: no mask)
       const int lim0 = MODE == kPrefix ? (1 << 30) : mt.ctx - a.q_len + 1 - mt.tok0;
-      const float* mcur = mref + cur * kWideCols;
+      // reference maxima in force: a portion's first stage starts from the -inf row
+      const float* mcur = mref + (first ? 2 : cur) * kWideCols;
       float e = -INFINITY;
+      if (tv && (MODE == kPrefix || r < lim0)) {   // every column sees this row
 #pragma unroll
-      for (int cq = 0; cq < kWideCols; ++cq) {
-        bool vis = tv && cq < a.ncol;
-        if (MODE != kPrefix && r >= lim0) vis = vis && r < lim0 + cq / group;
-        s[cq] = vis ? s[cq] * a.scale_log2 : -INFINITY;
-        const float m = first ? -INFINITY : mcur[cq];
-        e = fmaxf(e, s[cq] - m);                  // NaN (-inf - -inf) is ignored
+        for (int j = 0; j < CW; j += 4) {
+          const float4 m4 = *reinterpret_cast<const float4*>(mcur + c0 + j);
+          const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            s[j + u] = c0 + j + u < a.ncol ? s[j + u] * a.scale_log2 : -INFINITY;
+            e = fmaxf(e, s[j + u] - mm[u]);       // NaN (-inf - -inf) is ignored
+          }
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < CW; ++j) {
+          const int cq = c0 + j;
+          const bool vis = tv && cq < a.ncol && (MODE == kPrefix || r < lim0 + cq / group);
+          s[j] = vis ? s[j] * a.scale_log2 : -INFINITY;
+          e = fmaxf(e, s[j] - mcur[cq]);
+        }
       }
       const bool slow = bar_red_or(1, kWideSoftThreads, first || e > kRescaleLog2);
       if (slow) {
-        // move the reference maxima: stage column maxima over the 128 rows
+        // move the reference maxima: this warpgroup's column maxima over the 128 rows
 #pragma unroll
-        for (int cq = 0; cq < kWideCols; ++cq) {
-          if (cq < nq) {
-            const float wm = warp_max_f32(s[cq]);
-            if (lane == (cq & 31)) red[cq * 4 + q4] = wm;
-          }
+        for (int j = 0; j < CW; ++j) {
+          const float wm = warp_max_f32(s[j]);
+          if (lane == j) red[(c0 + j) * 4 + q4] = wm;
         }
         named_bar_sync(1, kWideSoftThreads);
         float* mnext = mref + (cur ^ 1) * kWideCols;
 #pragma unroll
-        for (int cq = 0; cq < kWideCols; ++cq) {
-          if (cq < nq) {
-            const float4 w4 = *reinterpret_cast<const float4*>(red + cq * 4);
-            const float cm = fmaxf(fmaxf(w4.x, w4.y), fmaxf(w4.z, w4.w));
-            const float mo = first ? -INFINITY : mcur[cq];
-            const float mn = fmaxf(mo, cm);
-            const float al = (mo == -INFINITY) ? 0.f : ex2(mo - mn);
-            lp[cq] *= al;
-            if (r == cq) {
-              mnext[cq] = mn;
-              alph[cq] = al;
-            }
+        for (int j = 0; j < CW; ++j) {
+          const float4 w4 = *reinterpret_cast<const float4*>(red + (c0 + j) * 4);
+          const float cm = fmaxf(fmaxf(w4.x, w4.y), fmaxf(w4.z, w4.w));
+          const float mo = mcur[c0 + j];
+          const float mn = fmaxf(mo, cm);
+          const float al = (mo == -INFINITY) ? 0.f : ex2(mo - mn);
+          lp[j] *= al;
+          if (r == j) {
+            mnext[c0 + j] = mn;
+            alph[c0 + j] = al;
           }
         }
         named_bar_sync(1, kWideSoftThreads);
         cur ^= 1;
         if (!first) {
-          // O^T was accumulated against the old maxima: rescale it once the previous
-          // stage's PV is done (its commit freed that stage's slot)
+          // O^T was accumulated against the old maxima: rescale this warpgroup's columns
+          // once the previous stage's PV is done (its commit freed that stage's slot)
           if (!mbar_wait_bounded(&empty[pst], pph, abort_flag, kWaitLimitNs)) {
-            if (lane == 0) {
-              *abort_flag = 1;
-              if (a.status) atomicOr(a.status, DEV_TIMEOUT);
-            }
+            give_up();
             break;
           }
           tc_fence_after();
+          float o[CW];
+          tld((uint32_t)(128 + c0), o);
+          tmem_wait_ld();
 #pragma unroll
-          for (int k = 0; k < kWideCols / 16; ++k) {
-            if (k < nchk) {
-              float v[16];
-              tmem_ld16(trow_addr + (uint32_t)(128 + 16 * k), v);
-              tmem_wait_ld();
-#pragma unroll
-              for (int j = 0; j < 16; ++j) v[j] *= alph[16 * k + j];
-              tmem_st16(trow_addr + (uint32_t)(128 + 16 * k), v);
-            }
-          }
+          for (int j = 0; j < CW; ++j) o[j] *= alph[c0 + j];
+          tst((uint32_t)(128 + c0), o);
           tmem_wait_st();
         }
       }
@@ -682,41 +727,38 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         const float* mc = mref + cur * kWideCols;
         uint8_t* sP = smem + st * L::kStageBytes + L::kPOff;
 #pragma unroll
-        for (int ch = 0; ch < kWideCols / 8; ++ch) {
-          if (ch * 8 < nq) {
-            const float4 m0 = *reinterpret_cast<const float4*>(mc + ch * 8);
-            const float4 m1 = *reinterpret_cast<const float4*>(mc + ch * 8 + 4);
-            // a column with no visible row yet keeps max -inf: 0 as its reference gives p = 0
-            float mm[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+        for (int ch = 0; ch < CW / 8; ++ch) {
+          const float4 m0 = *reinterpret_cast<const float4*>(mc + c0 + ch * 8);
+          const float4 m1 = *reinterpret_cast<const float4*>(mc + c0 + ch * 8 + 4);
+          // a column with no visible row yet keeps max -inf: 0 as its reference gives p = 0
+          float mm[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
 #pragma unroll
-            for (int j = 0; j < 8; ++j) mm[j] = mm[j] == -INFINITY ? 0.f : mm[j];
-            uint32_t hi[4], lo[4];
+          for (int j = 0; j < 8; ++j) mm[j] = mm[j] == -INFINITY ? 0.f : mm[j];
+          uint32_t hi[4], lo[4];
 #pragma unroll
-            for (int j = 0; j < 8; j += 2) {
-              const float p0 = ex2(s[ch * 8 + j] - mm[j]);
-              const float p1 = ex2(s[ch * 8 + j + 1] - mm[j + 1]);
-              lp[ch * 8 + j] += p0;
-              lp[ch * 8 + j + 1] += p1;
-              const uint32_t h = pack2<T>(p0, p1);
-              const float2 hf = unpack2<T>(h);
-              hi[j / 2] = h;
-              lo[j / 2] = pack2<T>(p0 - hf.x, p1 - hf.y);
-            }
-            const int off = r * 128 + ((ch ^ (r & 7)) << 4);
-            *reinterpret_cast<uint4*>(sP + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-            *reinterpret_cast<uint4*>(sP + L::kPBytes + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          for (int j = 0; j < 8; j += 2) {
+            const float p0 = ex2(s[ch * 8 + j] - mm[j]);
+            const float p1 = ex2(s[ch * 8 + j + 1] - mm[j + 1]);
+            lp[ch * 8 + j] += p0;
+            lp[ch * 8 + j + 1] += p1;
+            const uint32_t h = pack2<T>(p0, p1);
+            const float2 hf = unpack2<T>(h);
+            hi[j / 2] = h;
+            lo[j / 2] = pack2<T>(p0 - hf.x, p1 - hf.y);
           }
+          const int chunk = c0 / 8 + ch;
+          const int off = r * 128 + ((chunk ^ (r & 7)) << 4);
+          *reinterpret_cast<uint4*>(sP + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4*>(sP + L::kPBytes + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
-        if (!tv) {
+        if (!tv && wg < L::kHalves) {
           // a row past the stage's valid tokens may hold stale or NaN data: P is zero
-          // there, and V must be finite (0 x NaN would poison O)
-          uint8_t* sV = smem + st * L::kStageBytes + L::kKvBytes;
+          // there, and V must be finite (0 x NaN would poison O); warpgroup wg clears
+          // column half wg of the row
+          uint8_t* sV = smem + st * L::kStageBytes + L::kKvBytes + wg * (kWideTile * 128) + r * 128;
 #pragma unroll
-          for (int hf = 0; hf < L::kHalves; ++hf)
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch)
-              *reinterpret_cast<uint4*>(sV + hf * (kWideTile * 128) + r * 128 + ch * 16) =
-                  make_uint4(0u, 0u, 0u, 0u);
+          for (int ch = 0; ch < 8; ++ch)
+            *reinterpret_cast<uint4*>(sV + ch * 16) = make_uint4(0u, 0u, 0u, 0u);
         }
       }
       fence_proxy_async_smem();                    // P and V rows -> the tensor cores
@@ -725,35 +767,22 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       if (mt.flags & F_LAST) {
         // ---- end of a segment portion: row sums, then O^T back from tensor memory
 #pragma unroll
-        for (int cq = 0; cq < kWideCols; ++cq) {
-          if (cq < nq) {
-            float v = lp[cq];
-            v += __shfl_xor_sync(0xffffffffu, v, 16);
-            v += __shfl_xor_sync(0xffffffffu, v, 8);
-            v += __shfl_xor_sync(0xffffffffu, v, 4);
-            v += __shfl_xor_sync(0xffffffffu, v, 2);
-            v += __shfl_xor_sync(0xffffffffu, v, 1);
-            if (lane == (cq & 31)) red[cq * 4 + q4] = v;
-          }
+        for (int j = 0; j < CW; ++j) {
+          float v = lp[j];
+          v += __shfl_xor_sync(0xffffffffu, v, 16);
+          v += __shfl_xor_sync(0xffffffffu, v, 8);
+          v += __shfl_xor_sync(0xffffffffu, v, 4);
+          v += __shfl_xor_sync(0xffffffffu, v, 2);
+          v += __shfl_xor_sync(0xffffffffu, v, 1);
+          if (lane == j) red[(c0 + j) * 4 + q4] = v;
         }
         named_bar_sync(1, kWideSoftThreads);
         if (!mbar_wait_bounded(&empty[st], ph, abort_flag, kWaitLimitNs)) {   // this PV done
-          if (lane == 0) {
-            *abort_flag = 1;
-            if (a.status) atomicOr(a.status, DEV_TIMEOUT);
-          }
+          give_up();
           break;
         }
         tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < kWideCols / 16; ++k) {
-          if (k < nchk) {
-            float v[16];
-            tmem_ld16(trow_addr + (uint32_t)(128 + 16 * k), v);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) s[16 * k + j] = v[j];
-          }
-        }
+        tld((uint32_t)(128 + c0), s);
         tmem_wait_ld();
         tc_fence_before();
         // head dim of this thread's O^T lane: lane r at D 128; at D 64 (M = 64) dims
@@ -762,7 +791,8 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         const bool complete = mt.flags & F_COMPLETE;
         const float* mc = mref + cur * kWideCols;
 #pragma unroll
-        for (int cq = 0; cq < kWideCols; ++cq) {
+        for (int j = 0; j < CW; ++j) {
+          const int cq = c0 + j;
           if (cq < a.ncol && d >= 0) {
             const float4 w4 = *reinterpret_cast<const float4*>(red + cq * 4);
             const float Ls = (w4.x + w4.y) + (w4.z + w4.w);
@@ -772,14 +802,14 @@ __global__ void __launch_bounds__(kWideThreads, 1)
               if (row >= 0) {
                 if constexpr (MODE == kPrefix) {
                   if (d == 0) a.ext_ml[row] = make_float2(M, Ls);
-                  a.ext_acc[row * D + d] = s[cq];
+                  a.ext_acc[row * D + d] = s[j];
                 } else {
-                  static_cast<T*>(a.out)[row * D + d] = from_float<T>(Ls > 0.f ? s[cq] / Ls : 0.f);
+                  static_cast<T*>(a.out)[row * D + d] = from_float<T>(Ls > 0.f ? s[j] / Ls : 0.f);
                 }
               }
             } else {
               const long long prow = (long long)mt.pidx * kWideCols + cq;
-              a.part_acc[prow * D + d] = s[cq];
+              a.part_acc[prow * D + d] = s[j];
               if (d == 0) {
                 a.part_ml[prow * 2 + 0] = M;
                 a.part_ml[prow * 2 + 1] = Ls;
@@ -811,6 +841,8 @@ __global__ void __launch_bounds__(kWideThreads, 1)
           if (*last_flag) merge_wide<T, D, MODE>(a, dsc, *total_s, G, tid);
         }
         named_bar_sync(1, kWideSoftThreads);       // red[] is reused by the next stage
+#pragma unroll
+        for (int j = 0; j < CW; ++j) lp[j] = 0.f;  // the next stage starts a portion
       }
       pst = st;
       pph = ph;

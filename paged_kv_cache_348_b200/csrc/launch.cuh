@@ -115,12 +115,13 @@ PKV_DECL_RUN(pkv::kAppend, false)
 PKV_DECL_RUN(pkv::kPlain, true)
 #undef PKV_DECL_RUN
 
-// ---- the tcgen05 kernel for 17..64 query rows per kv head (decode_wide.cuh)
-template <typename T, int D, int BS, int MODE>
+// ---- the tcgen05 kernel for 17..64 query rows per kv head (decode_wide.cuh); NC = the
+// query rows rounded up to 16, 32 or 64
+template <typename T, int D, int BS, int MODE, int NC>
 pa_status launch_wide(const pkv::DecodeArgs& a, const CUtensorMap& mk, const CUtensorMap& mv,
                       int grid, cudaStream_t stream) {
   using L = pkv::WideLayout<D>;
-  auto k = pkv::pa_decode_wide_kernel<T, D, BS, MODE>;
+  auto k = pkv::pa_decode_wide_kernel<T, D, BS, MODE, NC>;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynSmem) !=
       cudaSuccess)
     return PA_ERR_CUDA;
@@ -130,38 +131,42 @@ pa_status launch_wide(const pkv::DecodeArgs& a, const CUtensorMap& mk, const CUt
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
-template <typename T, int MODE>
+template <typename T, int MODE, int NC>
 pa_status dispatch_wide(int d, int bs, const pkv::DecodeArgs& a, const CUtensorMap& mk,
                         const CUtensorMap& mv, int grid, cudaStream_t s) {
   if (d == 64) {
     switch (bs) {
-      case 1: return launch_wide<T, 64, 1, MODE>(a, mk, mv, grid, s);
-      case 8: return launch_wide<T, 64, 8, MODE>(a, mk, mv, grid, s);
-      case 16: return launch_wide<T, 64, 16, MODE>(a, mk, mv, grid, s);
-      case 32: return launch_wide<T, 64, 32, MODE>(a, mk, mv, grid, s);
+      case 1: return launch_wide<T, 64, 1, MODE, NC>(a, mk, mv, grid, s);
+      case 8: return launch_wide<T, 64, 8, MODE, NC>(a, mk, mv, grid, s);
+      case 16: return launch_wide<T, 64, 16, MODE, NC>(a, mk, mv, grid, s);
+      case 32: return launch_wide<T, 64, 32, MODE, NC>(a, mk, mv, grid, s);
     }
   } else {
     switch (bs) {
-      case 1: return launch_wide<T, 128, 1, MODE>(a, mk, mv, grid, s);
-      case 8: return launch_wide<T, 128, 8, MODE>(a, mk, mv, grid, s);
-      case 16: return launch_wide<T, 128, 16, MODE>(a, mk, mv, grid, s);
-      case 32: return launch_wide<T, 128, 32, MODE>(a, mk, mv, grid, s);
+      case 1: return launch_wide<T, 128, 1, MODE, NC>(a, mk, mv, grid, s);
+      case 8: return launch_wide<T, 128, 8, MODE, NC>(a, mk, mv, grid, s);
+      case 16: return launch_wide<T, 128, 16, MODE, NC>(a, mk, mv, grid, s);
+      case 32: return launch_wide<T, 128, 32, MODE, NC>(a, mk, mv, grid, s);
     }
   }
   return PA_ERR_UNSUPPORTED;
 }
 
-// One mode's wide instances (kPlain or kPrefix); defined in decode_wide_<mode>.cu.
-template <int MODE>
+// One (mode, NC)'s wide instances; defined in decode_wide_<mode>_<NC>.cu.
+template <int MODE, int NC>
 pa_status run_wide_mode(bool bf16, int d, int bs, const pkv::DecodeArgs& a, const CUtensorMap& mk,
                         const CUtensorMap& mv, int grid, cudaStream_t s);
-template <>
-pa_status run_wide_mode<pkv::kPlain>(bool bf16, int d, int bs, const pkv::DecodeArgs& a,
-                                     const CUtensorMap& mk, const CUtensorMap& mv, int grid,
-                                     cudaStream_t s);
-template <>
-pa_status run_wide_mode<pkv::kPrefix>(bool bf16, int d, int bs, const pkv::DecodeArgs& a,
-                                      const CUtensorMap& mk, const CUtensorMap& mv, int grid,
-                                      cudaStream_t s);
+#define PKV_DECL_WIDE(MODE, NC)                                                               \
+  template <>                                                                                 \
+  pa_status run_wide_mode<MODE, NC>(bool bf16, int d, int bs, const pkv::DecodeArgs& a,       \
+                                    const CUtensorMap& mk, const CUtensorMap& mv, int grid,   \
+                                    cudaStream_t s);
+PKV_DECL_WIDE(pkv::kPlain, 16)
+PKV_DECL_WIDE(pkv::kPlain, 32)
+PKV_DECL_WIDE(pkv::kPlain, 64)
+PKV_DECL_WIDE(pkv::kPrefix, 16)
+PKV_DECL_WIDE(pkv::kPrefix, 32)
+PKV_DECL_WIDE(pkv::kPrefix, 64)
+#undef PKV_DECL_WIDE
 
 }  // namespace pkv_host

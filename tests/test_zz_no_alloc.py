@@ -65,3 +65,22 @@ def test_noalloc_rejects_batches_beyond_its_scratch():
     big_c = ctx[:1].expand(n).contiguous()
     with pytest.raises(pk.PagedKVError, match="invalid argument"):
         pk.pa_decode_noalloc(torch.empty_like(big_q), big_q, k, v, big_t, big_c, 0.1)
+
+
+def test_noalloc_allocates_no_device_memory():
+    # one warm-up call loads the kernel instance this configuration uses; after it, calls
+    # with other batch sizes (same dtype, head_dim, block_size and group) must leave the
+    # device's free memory exactly as it was
+    case = make_case(12, 32, 8, 128, 16, [900, 3, 4100, 17, 0, 2048, 65, 1, 700, 5000, 33, 129],
+                     dtype="f16", seed=84)
+    q, k, v, tables, ctx = _upload(case)
+    out = torch.empty_like(q)
+    st = pk.new_status()
+    pk.pa_decode_noalloc(out, q, k, v, tables, ctx, case["scale"], st)
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    for n in (1, 5, 12, 7, 12, 2):
+        pk.pa_decode_noalloc(out[:n], q[:n], k, v, tables[:n], ctx[:n], case["scale"], st)
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert int(st.item()) == 0
