@@ -17,16 +17,16 @@
 //    segment's query rows into a Q tile with cp.async (same swizzle).
 //  * Warp 1 (one thread) issues the MMAs: S^T[128 tokens][N] = K . Q^T with the tokens on
 //    M = 128 and the query rows on N = 16..64 (no padding of the query side to 64 or 128),
-//    accumulated in tensor memory; then O^T[D][N] += V^T . P^T with V read MN-major from
-//    the same tile.  The QK^T of stage i+2 is issued right after the PV of stage i, so the
-//    softmax of stage i+1 overlaps both.
+//    accumulated in tensor memory (one S^T buffer per ring slot); then O^T[D][N] +=
+//    V^T . P^T with V read MN-major from the same tile.  It is event driven: a stage's
+//    QK^T goes out as soon as its tiles land, its PV as soon as the softmax is done.
 //  * Warps 2..9, two warpgroups that split the query columns, run the softmax: a thread
 //    owns one token row of S^T (one TMEM lane) and half of the columns.  Base 2, fp32, with
 //    a lazily moved reference maximum per query row (a stage moves it only when some score
 //    exceeds it by more than 2^8, which after a portion's first stage is rare; O^T is then
-//    rescaled in tensor memory).  P^T is written in 16 bits as a high part and the
-//    rounding residual (~16 mantissa bits in all) into the stage's K tile, which QK^T no
-//    longer needs.  Row sums stay per thread and are reduced once per portion.  The same
+//    rescaled in tensor memory).  P^T is written in 16 bits into the stage's K tile, which
+//    QK^T no longer needs; with bf16 its rounding residual goes beside it as NC more
+//    columns, so one PV pass (N = 2 NC) accumulates both and ~16 bits of P count.  Row sums stay per thread and are reduced once per portion.  The same
 //    warps read O^T back at the end of a portion (one thread per head dim and column half)
 //    and write the output or the split partial.  The column count NC (16, 32 or 64, the
 //    query rows rounded up) is a template parameter, so these loops are exactly as long
@@ -44,7 +44,10 @@ constexpr int kWideUnits = kWideTile / kUnit;     // 16-token units per stage
 constexpr int kWideStages = 3;
 constexpr int kWideSoftThreads = 256;             // softmax warps 2..9 (two warpgroups)
 constexpr int kWideThreads = 64 + kWideSoftThreads;
-constexpr uint32_t kWideTmemCols = 256;           // S^T x 2 (cols 0..127), O^T (cols 128..191)
+// tensor memory: one S^T buffer per ring slot (columns 64 s .. 64 s + NC - 1) and O^T from
+// column 256 (NC columns, or 2 NC when P's residual is a second column block)
+constexpr uint32_t kWideTmemCols = 512;
+constexpr uint32_t kOCol = 256;
 constexpr float kRescaleLog2 = 8.f;               // a reference max moves past this gap only
 
 template <int D>
@@ -60,13 +63,14 @@ struct WideLayout {
   static constexpr int kQBytes = kHalves * kWideCols * 128;
   static constexpr int kMetaOff = kQOff + kQBytes;
   static constexpr int kBarOff = (kMetaOff + kWideStages * (int)sizeof(StageMeta) + 15) / 16 * 16;
-  // full[3], empty[3], sfull[2], pfull[2], qempty, drain
-  static constexpr int kNumBars = 2 * kWideStages + 6;
+  // full[3], empty[3], sfull[3], pfull[3], qempty, drain
+  static constexpr int kNumBars = 4 * kWideStages + 2;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;       // tmem base, abort, last, total
   static constexpr int kDescOff = kMiscOff + 32;
   static constexpr int kMrefOff = (kDescOff + 2 * (int)sizeof(SplitDesc) + 15) / 16 * 16;
-  // float [3][64]: two reference-max buffers and a row of -inf (a portion's first stage)
-  static constexpr int kRedOff = kMrefOff + 3 * kWideCols * 4;  // float [64 cols][4 warps]
+  // float [5][64]: two reference-max buffers, a row of -inf (a portion's first stage), and
+  // the two buffers again with -inf replaced by 0 (the reference p is computed against)
+  static constexpr int kRedOff = kMrefOff + 5 * kWideCols * 4;  // float [64 cols][4 warps]
   static constexpr int kAlphaOff = kRedOff + kWideCols * 4 * 4;
   static constexpr int kBytes = kAlphaOff + kWideCols * 4;
   static constexpr int kDynSmem = kBytes + 1024;                // slack for 1024-byte alignment
@@ -165,6 +169,10 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   static_assert(MODE == kPlain || MODE == kPrefix, "wide decode: plain (multi-token) or prefix");
   static_assert(NC == 16 || NC == 32 || NC == 64, "16, 32 or 64 query columns");
   constexpr int CW = NC / 2;                        // columns of one softmax warpgroup
+  // bf16 P keeps ~16 bits as a high part (columns 0..NC-1 of P^T and O^T) plus its rounding
+  // residual (columns NC..2NC-1, summed when O^T is read back); fp16 P has 11, enough here
+  constexpr bool kSplit = std::is_same_v<T, __nv_bfloat16>;
+  constexpr int kNPV = kSplit ? 2 * NC : NC;        // MMA N of PV
   constexpr int kSegW = seg_weight(BS);
   constexpr uint32_t kAB = std::is_same_v<T, __nv_bfloat16> ? 1u : 0u;
   constexpr int kFullCount = 33;       // lane 0's expect_tx arrival + 32 cp.async arrivals
@@ -175,15 +183,15 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   uint64_t* empty = full + kWideStages;
   uint64_t* sfull = empty + kWideStages;
-  uint64_t* pfull = sfull + 2;
-  uint64_t* qempty = pfull + 2;
+  uint64_t* pfull = sfull + kWideStages;
+  uint64_t* qempty = pfull + kWideStages;
   uint64_t* drain = qempty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
   volatile int* last_flag = abort_flag + 1;
   long long* total_s = reinterpret_cast<long long*>(smem + L::kMiscOff + 16);
   SplitDesc* desc = reinterpret_cast<SplitDesc*>(smem + L::kDescOff);
-  float* mref = reinterpret_cast<float*>(smem + L::kMrefOff);      // [3][64]
+  float* mref = reinterpret_cast<float*>(smem + L::kMrefOff);      // [5][64]
   float* red = reinterpret_cast<float*>(smem + L::kRedOff);        // [64][4]
   float* alph = reinterpret_cast<float*>(smem + L::kAlphaOff);     // [64]
   uint8_t* sQ = smem + L::kQOff;
@@ -194,7 +202,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       mbar_init(&full[i], kFullCount);
       mbar_init(&empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kWideStages; ++i) {
       mbar_init(&sfull[i], 1);
       mbar_init(&pfull[i], kWideSoftThreads);
     }
@@ -499,78 +507,85 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == 1) {
     // ============================== MMA issue ==============================
+    // Event driven: QK^T of a stage is issued as soon as its tiles have landed and its
+    // slot's S^T buffer is free (at most kWideStages stages ahead of PV), PV as soon as the
+    // softmax has written P^T.
     if (lane == 0) {
-      const uint32_t idesc_qk = idesc_f16(kAB, 0u, 0u, 128u, (uint32_t)nq);
-      const uint32_t idesc_pv = idesc_f16(kAB, 1u, 1u, (uint32_t)D, (uint32_t)nq);
-      const uint32_t sq = smem_u32(sQ);
-      auto qk = [&](int slot, int sb, int flags) {
-        const uint32_t sk = smem_u32(smem + slot * L::kStageBytes);
+      const uint32_t idesc_qk = idesc_f16(kAB, 0u, 0u, 128u, (uint32_t)NC);
+      const uint32_t idesc_pv = idesc_f16(kAB, 1u, 1u, (uint32_t)D, (uint32_t)kNPV);
+      // descriptors of slot 0; slots, k-steps and column halves add to the start-address
+      // field (16-byte units, bits 0..13; every address here is below 256 KB, so the sum
+      // never carries out of the field)
+      const uint64_t dq0 = smem_desc_sw128(smem_u32(sQ), 16u, 1024u);
+      const uint64_t dk0 = smem_desc_sw128(smem_u32(smem), 16u, 1024u);
+      const uint64_t dv0 = smem_desc_sw128(smem_u32(smem + L::kKvBytes), kWideTile * 128, 1024u);
+      const uint64_t dp0 = smem_desc_sw128(smem_u32(smem + L::kPOff), L::kPBytes, 1024u);
+      auto adv = [](uint64_t d, uint32_t bytes) { return d + (uint64_t)(bytes >> 4); };
+      auto qk = [&](int slot, int flags) {
+        const uint32_t so = (uint32_t)(slot * L::kStageBytes);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (ks & 3) * 32;          // 16 dims = 32 bytes along a row
-          const uint64_t da = smem_desc_sw128(sk + (ks >> 2) * (kWideTile * 128) + off, 16u, 1024u);
-          const uint64_t db = smem_desc_sw128(sq + (ks >> 2) * (kWideCols * 128) + off, 16u, 1024u);
-          tc_mma_f16(tbase + (uint32_t)(sb * 64), da, db, idesc_qk, ks > 0);
+          tc_mma_f16(tbase + (uint32_t)(slot * 64),
+                     adv(dk0, so + (ks >> 2) * (kWideTile * 128) + off),
+                     adv(dq0, (ks >> 2) * (kWideCols * 128) + off), idesc_qk, ks > 0);
         }
-        tc_commit(&sfull[sb]);
+        tc_commit(&sfull[slot]);
         if (flags & F_LAST) tc_commit(qempty);       // the Q tile may be refilled after this
       };
       auto pv = [&](int slot, bool first) {
-        const uint32_t sv = smem_u32(smem + slot * L::kStageBytes + L::kKvBytes);
-        const uint32_t sp = smem_u32(smem + slot * L::kStageBytes + L::kPOff);
+        const uint32_t so = (uint32_t)(slot * L::kStageBytes);
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {         // P^T high part, then its residual
-#pragma unroll
-          for (int kk = 0; kk < kWideTile / 16; ++kk) {
-            const uint64_t da = smem_desc_sw128(sv + kk * 2048, kWideTile * 128, 1024u);
-            const uint64_t db = smem_desc_sw128(sp + part * L::kPBytes + kk * 2048, kWideTile * 128,
-                                                1024u);
-            tc_mma_f16(tbase + 128u, da, db, idesc_pv, !(first && part == 0 && kk == 0));
-          }
-        }
+        for (int kk = 0; kk < kWideTile / 16; ++kk)
+          tc_mma_f16(tbase + kOCol, adv(dv0, so + kk * 2048), adv(dp0, so + kk * 2048), idesc_pv,
+                     !(first && kk == 0));
       };
-      int sl[3] = {0, 0, 0}, fl[3] = {0, 0, 0};   // slots / flags of stages i, i+1, i+2
-      uint32_t phs = 0;
-      int st = 0;
-      bool ok = true, have_next = false;
-      auto next_stage = [&](int& slot, int& flags) -> bool {   // wait stage, false at END
-        if (!mbar_wait_bounded(&full[st], phs, abort_flag, kWaitLimitNs)) {
-          ok = false;
-          return false;
-        }
-        // Q (and, at block_size 1, K/V) arrive by cp.async, generic-proxy writes the
-        // tensor cores read through the async proxy
-        fence_proxy_async_smem();
-        slot = st;
-        flags = meta[st].flags;
-        if (++st == kWideStages) {
-          st = 0;
-          phs ^= 1u;
-        }
-        return !(flags & F_END);
-      };
-      if (next_stage(sl[0], fl[0])) {
-        tc_fence_after();
-        qk(sl[0], 0, fl[0]);
-        have_next = next_stage(sl[1], fl[1]);
-        if (have_next) qk(sl[1], 1, fl[1]);
-        for (int i = 0; ok; ++i) {
-          if (!mbar_wait_bounded(&pfull[i & 1], (uint32_t)((i >> 1) & 1), abort_flag,
-                                 kWaitLimitNs)) {
-            ok = false;
-            break;
+      int q_slot = 0, p_slot = 0, n_qk = 0, n_pv = 0;
+      uint32_t q_ph = 0, p_ph = 0;
+      int fl[kWideStages] = {0, 0, 0};
+      bool q_end = false, ok = true;
+      uint64_t idle_since = 0;
+      while (ok) {
+        bool progress = false;
+        if (!q_end && n_qk - n_pv < kWideStages && mbar_try_wait(&full[q_slot], q_ph)) {
+          // Q (and, at block_size 1, K/V) arrive by cp.async: generic-proxy writes the
+          // tensor cores read through the async proxy
+          fence_proxy_async_smem();
+          const int f = meta[q_slot].flags;
+          if (f & F_END) {
+            q_end = true;
+          } else {
+            tc_fence_after();
+            qk(q_slot, f);
+            fl[q_slot] = f;
+            ++n_qk;
+            if (++q_slot == kWideStages) {
+              q_slot = 0;
+              q_ph ^= 1u;
+            }
           }
+          progress = true;
+        }
+        if (n_pv < n_qk && mbar_try_wait(&pfull[p_slot], p_ph)) {
           tc_fence_after();
-          pv(sl[0], fl[0] & F_FIRST);
-          tc_commit(&empty[sl[0]]);                 // frees the stage (K, V and P tiles)
-          if (!have_next) break;
-          const bool more = next_stage(sl[2], fl[2]);
-          if (more) qk(sl[2], i & 1, fl[2]);
-          sl[0] = sl[1];
-          fl[0] = fl[1];
-          sl[1] = sl[2];
-          fl[1] = fl[2];
-          have_next = more;
+          pv(p_slot, fl[p_slot] & F_FIRST);
+          tc_commit(&empty[p_slot]);                // frees the stage (K, V and P tiles)
+          ++n_pv;
+          if (++p_slot == kWideStages) {
+            p_slot = 0;
+            p_ph ^= 1u;
+          }
+          progress = true;
+        }
+        if (q_end && n_pv == n_qk) break;
+        if (progress) {
+          idle_since = 0;
+        } else if (*abort_flag) {
+          ok = false;
+        } else {
+          const uint64_t now = globaltimer_ns();
+          if (!idle_since) idle_since = now;
+          else if (now - idle_since > kWaitLimitNs) ok = false;
         }
       }
       if (!ok) {
@@ -640,44 +655,49 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       const StageMeta mt = meta[st];
       if (mt.flags & F_END) break;
       const bool first = mt.flags & F_FIRST;
-      const int sb = i & 1;
       if (first) {
 #pragma unroll
         for (int j = 0; j < CW; ++j) lp[j] = 0.f;
       }
-      if (!mbar_wait_bounded(&sfull[sb], (uint32_t)((i >> 1) & 1), abort_flag, kWaitLimitNs)) {
+      if (!mbar_wait_bounded(&sfull[st], ph, abort_flag, kWaitLimitNs)) {   // this slot's S^T
         give_up();
         break;
       }
       tc_fence_after();
       float s[CW];
-      tld((uint32_t)(sb * 64 + c0), s);
+      tld((uint32_t)(st * 64 + c0), s);
       tmem_wait_ld();
       const int nvalid = (mt.nunits * kUnit < mt.ctx - mt.tok0) ? mt.nunits * kUnit : mt.ctx - mt.tok0;
       const bool tv = r < nvalid;
       // causal limit: new token j sees stage rows < lim0 + j (a prefix launch: no mask)
       const int lim0 = MODE == kPrefix ? (1 << 30) : mt.ctx - a.q_len + 1 - mt.tok0;
-      // reference maxima in force: a portion's first stage starts from the -inf row
+      // reference maxima in force: a portion's first stage starts from the -inf row.  With
+      // x = scale * s (base 2), e = max_j (x_j - m_j) tells whether a reference must move;
+      // masked scores are -inf (NaN against a -inf reference, which fmaxf ignores)
+      const float sc = a.scale_log2;
       const float* mcur = mref + (first ? 2 : cur) * kWideCols;
       float e = -INFINITY;
       if (tv && (MODE == kPrefix || r < lim0)) {   // every column sees this row
+        if (a.ncol < c0 + CW) {                    // padding columns of this warpgroup
+#pragma unroll
+          for (int j = 0; j < CW; ++j)
+            if (c0 + j >= a.ncol) s[j] = -INFINITY;
+        }
 #pragma unroll
         for (int j = 0; j < CW; j += 4) {
           const float4 m4 = *reinterpret_cast<const float4*>(mcur + c0 + j);
-          const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            s[j + u] = c0 + j + u < a.ncol ? s[j + u] * a.scale_log2 : -INFINITY;
-            e = fmaxf(e, s[j + u] - mm[u]);       // NaN (-inf - -inf) is ignored
-          }
+          e = fmaxf(e, fmaf(s[j], sc, -m4.x));
+          e = fmaxf(e, fmaf(s[j + 1], sc, -m4.y));
+          e = fmaxf(e, fmaf(s[j + 2], sc, -m4.z));
+          e = fmaxf(e, fmaf(s[j + 3], sc, -m4.w));
         }
       } else {
 #pragma unroll
         for (int j = 0; j < CW; ++j) {
           const int cq = c0 + j;
           const bool vis = tv && cq < a.ncol && (MODE == kPrefix || r < lim0 + cq / group);
-          s[j] = vis ? s[j] * a.scale_log2 : -INFINITY;
-          e = fmaxf(e, s[j] - mcur[cq]);
+          if (!vis) s[j] = -INFINITY;
+          e = fmaxf(e, fmaf(s[j], sc, -mcur[cq]));
         }
       }
       const bool slow = bar_red_or(1, kWideSoftThreads, first || e > kRescaleLog2);
@@ -685,11 +705,12 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         // move the reference maxima: this warpgroup's column maxima over the 128 rows
 #pragma unroll
         for (int j = 0; j < CW; ++j) {
-          const float wm = warp_max_f32(s[j]);
+          const float wm = warp_max_f32(s[j] * sc);
           if (lane == j) red[(c0 + j) * 4 + q4] = wm;
         }
         named_bar_sync(1, kWideSoftThreads);
         float* mnext = mref + (cur ^ 1) * kWideCols;
+        float* mnext_p = mref + (3 + (cur ^ 1)) * kWideCols;
 #pragma unroll
         for (int j = 0; j < CW; ++j) {
           const float4 w4 = *reinterpret_cast<const float4*>(red + (c0 + j) * 4);
@@ -700,6 +721,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
           lp[j] *= al;
           if (r == j) {
             mnext[c0 + j] = mn;
+            mnext_p[c0 + j] = mn == -INFINITY ? 0.f : mn;   // p = 0 while nothing is visible
             alph[c0 + j] = al;
           }
         }
@@ -713,43 +735,49 @@ __global__ void __launch_bounds__(kWideThreads, 1)
             break;
           }
           tc_fence_after();
-          float o[CW];
-          tld((uint32_t)(128 + c0), o);
-          tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < CW; ++j) o[j] *= alph[c0 + j];
-          tst((uint32_t)(128 + c0), o);
+          for (int part = 0; part < (kSplit ? 2 : 1); ++part) {
+            float o[CW];
+            tld(kOCol + (uint32_t)(part * NC + c0), o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < CW; ++j) o[j] *= alph[c0 + j];
+            tst(kOCol + (uint32_t)(part * NC + c0), o);
+          }
           tmem_wait_st();
         }
       }
-      // P^T row r: p = 2^(x - m), 16-bit high part and residual, 8 columns per 16-byte chunk
+      // P^T row r: p = 2^(x - m), 16 bits per value in 16-byte chunks of 8 columns; P^T
+      // column col sits in 64-column block col / 64 (kPBytes apart), 128-byte swizzle
       {
-        const float* mc = mref + cur * kWideCols;
+        const float* mc = mref + (3 + cur) * kWideCols;   // -inf replaced by 0
         uint8_t* sP = smem + st * L::kStageBytes + L::kPOff;
+        auto put = [&](int col, uint4 v) {
+          const int chunk = (col & 63) >> 3;
+          *reinterpret_cast<uint4*>(sP + (col >> 6) * L::kPBytes + r * 128 +
+                                    ((chunk ^ (r & 7)) << 4)) = v;
+        };
 #pragma unroll
         for (int ch = 0; ch < CW / 8; ++ch) {
           const float4 m0 = *reinterpret_cast<const float4*>(mc + c0 + ch * 8);
           const float4 m1 = *reinterpret_cast<const float4*>(mc + c0 + ch * 8 + 4);
-          // a column with no visible row yet keeps max -inf: 0 as its reference gives p = 0
-          float mm[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
-#pragma unroll
-          for (int j = 0; j < 8; ++j) mm[j] = mm[j] == -INFINITY ? 0.f : mm[j];
+          const float mm[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
           uint32_t hi[4], lo[4];
 #pragma unroll
           for (int j = 0; j < 8; j += 2) {
-            const float p0 = ex2(s[ch * 8 + j] - mm[j]);
-            const float p1 = ex2(s[ch * 8 + j + 1] - mm[j + 1]);
+            const float p0 = ex2(fmaf(s[ch * 8 + j], sc, -mm[j]));
+            const float p1 = ex2(fmaf(s[ch * 8 + j + 1], sc, -mm[j + 1]));
             lp[ch * 8 + j] += p0;
             lp[ch * 8 + j + 1] += p1;
             const uint32_t h = pack2<T>(p0, p1);
-            const float2 hf = unpack2<T>(h);
             hi[j / 2] = h;
-            lo[j / 2] = pack2<T>(p0 - hf.x, p1 - hf.y);
+            if constexpr (kSplit) {
+              const float2 hf = unpack2<T>(h);
+              lo[j / 2] = pack2<T>(p0 - hf.x, p1 - hf.y);
+            }
           }
-          const int chunk = c0 / 8 + ch;
-          const int off = r * 128 + ((chunk ^ (r & 7)) << 4);
-          *reinterpret_cast<uint4*>(sP + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-          *reinterpret_cast<uint4*>(sP + L::kPBytes + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          put(c0 + ch * 8, make_uint4(hi[0], hi[1], hi[2], hi[3]));
+          if constexpr (kSplit) put(NC + c0 + ch * 8, make_uint4(lo[0], lo[1], lo[2], lo[3]));
         }
         if (!tv && wg < L::kHalves) {
           // a row past the stage's valid tokens may hold stale or NaN data: P is zero
@@ -763,7 +791,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       }
       fence_proxy_async_smem();                    // P and V rows -> the tensor cores
       tc_fence_before();
-      mbar_arrive(&pfull[sb]);
+      mbar_arrive(&pfull[st]);
       if (mt.flags & F_LAST) {
         // ---- end of a segment portion: row sums, then O^T back from tensor memory
 #pragma unroll
@@ -782,41 +810,54 @@ __global__ void __launch_bounds__(kWideThreads, 1)
           break;
         }
         tc_fence_after();
-        tld((uint32_t)(128 + c0), s);
-        tmem_wait_ld();
-        tc_fence_before();
         // head dim of this thread's O^T lane: lane r at D 128; at D 64 (M = 64) dims
         // 16 q4 .. 16 q4 + 15 sit in lanes 0..15 of quadrant q4
         const int d = D == 128 ? r : (lane < 16 ? q4 * 16 + lane : -1);
         const bool complete = mt.flags & F_COMPLETE;
         const float* mc = mref + cur * kWideCols;
+        // O^T back 8 columns at a time (the high part plus, with bf16, the residual part)
+#pragma unroll 1
+        for (int j0 = 0; j0 < CW; j0 += 8) {
+          float o[8];
+          tmem_ld8(trow_addr + kOCol + (uint32_t)(c0 + j0), o);
+          if constexpr (kSplit) {
+            float o2[8];
+            tmem_ld8(trow_addr + kOCol + (uint32_t)(NC + c0 + j0), o2);
+            tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < CW; ++j) {
-          const int cq = c0 + j;
-          if (cq < a.ncol && d >= 0) {
-            const float4 w4 = *reinterpret_cast<const float4*>(red + cq * 4);
-            const float Ls = (w4.x + w4.y) + (w4.z + w4.w);
-            const float M = mc[cq];
-            if (complete) {
-              const long long row = out_row<MODE>(a, mt.seq, mt.kvh, cq);
-              if (row >= 0) {
-                if constexpr (MODE == kPrefix) {
-                  if (d == 0) a.ext_ml[row] = make_float2(M, Ls);
-                  a.ext_acc[row * D + d] = s[j];
-                } else {
-                  static_cast<T*>(a.out)[row * D + d] = from_float<T>(Ls > 0.f ? s[j] / Ls : 0.f);
+            for (int j = 0; j < 8; ++j) o[j] += o2[j];
+          } else {
+            tmem_wait_ld();
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int cq = c0 + j0 + j;
+            if (cq < a.ncol && d >= 0) {
+              const float4 w4 = *reinterpret_cast<const float4*>(red + cq * 4);
+              const float Ls = (w4.x + w4.y) + (w4.z + w4.w);
+              const float M = mc[cq];
+              if (complete) {
+                const long long row = out_row<MODE>(a, mt.seq, mt.kvh, cq);
+                if (row >= 0) {
+                  if constexpr (MODE == kPrefix) {
+                    if (d == 0) a.ext_ml[row] = make_float2(M, Ls);
+                    a.ext_acc[row * D + d] = o[j];
+                  } else {
+                    static_cast<T*>(a.out)[row * D + d] = from_float<T>(Ls > 0.f ? o[j] / Ls : 0.f);
+                  }
                 }
-              }
-            } else {
-              const long long prow = (long long)mt.pidx * kWideCols + cq;
-              a.part_acc[prow * D + d] = s[j];
-              if (d == 0) {
-                a.part_ml[prow * 2 + 0] = M;
-                a.part_ml[prow * 2 + 1] = Ls;
+              } else {
+                const long long prow = (long long)mt.pidx * kWideCols + cq;
+                a.part_acc[prow * D + d] = o[j];
+                if (d == 0) {
+                  a.part_ml[prow * 2 + 0] = M;
+                  a.part_ml[prow * 2 + 1] = Ls;
+                }
               }
             }
           }
         }
+        tc_fence_before();
         if (!complete) {
           // arrival on the segment's counter (as in decode.cuh): the last contributor merges
           named_bar_sync(1, kWideSoftThreads);
