@@ -66,6 +66,12 @@ def _load():
         L.orc_decode_e4m3.restype = i32
         L.orc_cache_append_e4m3.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, f32]
         L.orc_cache_append_e4m3.restype = i32
+        L.orc_e4m3_block_scale.argtypes = [f32]; L.orc_e4m3_block_scale.restype = f32
+        L.orc_cache_append_e4m3_bs.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32]
+        L.orc_cache_append_e4m3_bs.restype = i32
+        L.orc_decode_e4m3_bs.argtypes = [P, P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32,
+                                         i32, i32, f64, i32, P, i32, i32]
+        L.orc_decode_e4m3_bs.restype = i32
         L.orc_cache_append.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32]
         L.orc_cache_append.restype = i32
         L.orc_copy_blocks.argtypes = [P, P, i32, P, i32, i64, i32]
@@ -217,6 +223,61 @@ def decode_e4m3(q, k_cache8, v_cache8, k_scale: float, v_scale: float, block_tab
                                  float(v_scale), _p(bt), _p(cl), B, QL, Hq, Hkv, D, bs, bt.shape[1],
                                  N, float(scale), DTYPES[dtype], None if it is None else _p(it),
                                  0 if it is None else len(it), int(nthreads))
+    if rc == -1:
+        raise ValueError("oracle decode: block id out of range")
+    if rc:
+        raise ValueError("oracle decode: bad arguments (%d)" % rc)
+    return out64.reshape(shape), out16.reshape(shape)
+
+
+def e4m3_block_scale(amax: float) -> float:
+    """Scale of an 8-bit block's (block, kv head) slice fixed by its offset-0 token, whose
+    row has largest magnitude amax: 2^(ceil(log2(amax / 448)) + 3), 1 for amax 0."""
+    return float(_load().orc_e4m3_block_scale(float(amax)))
+
+
+def cache_append_e4m3_bs(k_cache8, v_cache8, k_scales, v_scales, k, v, slot_mapping, dtype: str):
+    """In-place quantising scatter with per-(block, kv head) scales (float32 [N, Hkv],
+    updated for the blocks whose offset 0 is written here)."""
+    for a in (k_cache8, v_cache8, k_scales, v_scales):
+        assert a.flags.c_contiguous
+    assert k_cache8.dtype == np.uint8 and v_cache8.dtype == np.uint8
+    assert k_scales.dtype == np.float32 and v_scales.dtype == np.float32
+    N, Hkv, bs, D = k_cache8.shape
+    assert k_scales.shape == (N, Hkv) and v_scales.shape == (N, Hkv)
+    k = _c(k, np.uint16); v = _c(v, np.uint16)
+    sm = _c(slot_mapping, np.int64)
+    rc = _load().orc_cache_append_e4m3_bs(_p(k_cache8), _p(v_cache8), _p(k_scales), _p(v_scales),
+                                          _p(k), _p(v), _p(sm), len(sm), Hkv, D, bs, N,
+                                          DTYPES[dtype])
+    if rc:
+        raise ValueError("oracle append: slot out of range")
+
+
+def decode_e4m3_bs(q, k_cache8, v_cache8, k_scales, v_scales, block_tables, context_lens,
+                   scale: float, dtype: str, items=None, nthreads: int = 1):
+    """fp64 paged decode over uint8 E4M3 pools with per-(block, kv head) scales (value of
+    block b, head h = scales[b][h] * code); q [B, Hq, D] or [B, q_len, Hq, D]."""
+    q = _c(q, np.uint16)
+    k8 = _c(k_cache8, np.uint8)
+    v8 = _c(v_cache8, np.uint8)
+    ks = _c(k_scales, np.float32)
+    vs = _c(v_scales, np.float32)
+    bt = _c(block_tables, np.int32)
+    cl = _c(context_lens, np.int32)
+    shape = q.shape
+    q4 = q.reshape(shape[0], 1, shape[1], shape[2]) if q.ndim == 3 else q
+    B, QL, Hq, D = q4.shape
+    N, Hkv, bs, D2 = k8.shape
+    assert D2 == D and v8.shape == k8.shape and bt.shape[0] == B
+    assert ks.shape == (N, Hkv) and vs.shape == (N, Hkv)
+    out64 = np.zeros((B, QL, Hq, D), dtype=np.float64)
+    out16 = np.zeros((B, QL, Hq, D), dtype=np.uint16)
+    it = None if items is None else _c(items, np.int32)
+    rc = _load().orc_decode_e4m3_bs(_p(out64), _p(out16), _p(q4), _p(k8), _p(v8), _p(ks), _p(vs),
+                                    _p(bt), _p(cl), B, QL, Hq, Hkv, D, bs, bt.shape[1], N,
+                                    float(scale), DTYPES[dtype], None if it is None else _p(it),
+                                    0 if it is None else len(it), int(nthreads))
     if rc == -1:
         raise ValueError("oracle decode: block id out of range")
     if rc:

@@ -143,6 +143,28 @@ uint8_t orc_quantize_e4m3(uint16_t bits, int dtype, float scale) {
   return orc_f64_to_e4m3((double)q);
 }
 
+/* ---- per-(block, kv head) scales of an 8-bit cache.  The pages name an FP8 quantised
+ *      KV cache ("PagedAttention -- The KV Cache Problem", "What's Still Unsolved") but
+ *      no format; the reading: every (physical block, kv head) slice of a pool has its
+ *      own scale, fixed by the token written at offset 0 of the block (the first token a
+ *      block ever receives, since blocks fill in order): with amax the largest |x| of that
+ *      token's row for the head and y = amax / 448 in binary32, the scale is the power of
+ *      two 2^(ceil(log2 y) + 3) -- the smallest power of two that maps the row into
+ *      E4M3's range, times 8 of headroom for later tokens of the block (larger ones
+ *      saturate).  amax of 0 (or not finite) gives scale 1.  A power of two keeps x / scale
+ *      exact, so the code is the E4M3 rounding of the scaled value. ----------------- */
+float orc_e4m3_block_scale(float amax) {
+  volatile float y = amax / 448.0f;
+  if (!(y > 0.0f) || isinf(y)) return 1.0f;
+  int e;
+  float m = frexpf(y, &e);                 /* y = m 2^e, m in [0.5, 1) */
+  int c = (m == 0.5f) ? e - 1 : e;         /* ceil(log2 y) */
+  c += 3;
+  if (c < -126) c = -126;
+  if (c > 127) c = 127;
+  return ldexpf(1.0f, c);
+}
+
 static double to_f64(uint16_t v, int dtype) {
   return dtype == ORC_BF16 ? orc_bf16_to_f64(v) : orc_f16_to_f64(v);
 }
@@ -194,6 +216,21 @@ int orc_gather(double* out, const uint16_t* cache, int dtype, int num_blocks, in
   return orc_gather_any(out, cache, dtype, 1.0, num_blocks, Hkv, bs, D, table_row, ctx, kvh);
 }
 
+/* Gather over an 8-bit cache with per-(block, kv head) scales bscale[b][kvh]. */
+static int gather_block_scaled(double* out, const uint8_t* cache, const float* bscale,
+                               int num_blocks, int Hkv, int bs, int D, const int32_t* table_row,
+                               int ctx, int kvh) {
+  for (int t = 0; t < ctx; ++t) {
+    int32_t b = table_row[t / bs];
+    int o = t % bs;
+    if (b < 0 || b >= num_blocks) return -1;
+    double sc = (double)bscale[(int64_t)b * Hkv + kvh];
+    int64_t r = cache_row(b, kvh, o, Hkv, bs, D);
+    for (int d = 0; d < D; ++d) out[(int64_t)t * D + d] = sc * orc_e4m3_to_f64(cache[r + d]);
+  }
+  return 0;
+}
+
 /* ---- decode attention: [P1] "How PagedAttention borrows OS paging" -- the math is
  *      the plain dot products, softmax and value-weighted sum, only the storage is
  *      paged; so this is softmax(scale * q K^T) V over the gathered rows.
@@ -211,6 +248,7 @@ typedef struct {
   int n_items, q_len, Hq, Hkv, D, bs, max_blocks, num_blocks, dtype;
   int cache_dtype;                          /* dtype, or ORC_E4M3 with the scales below */
   double k_scale, v_scale;
+  const float *k_bscale, *v_bscale;         /* E4M3 with per-(block, kv head) scales */
   double scale;
   atomic_int next;
   atomic_int err;
@@ -227,10 +265,18 @@ static void decode_one(decode_job* J, int s, int j, int h, double* kbuf, double*
   for (int d = 0; d < D; ++d) o64[d] = 0.0;
   if (n > 0) {
     const int32_t* table_row = J->block_tables + (int64_t)s * J->max_blocks;
-    if (orc_gather_any(kbuf, J->k_cache, J->cache_dtype, J->k_scale, J->num_blocks, J->Hkv, J->bs,
-                       D, table_row, n, kvh) ||
-        orc_gather_any(vbuf, J->v_cache, J->cache_dtype, J->v_scale, J->num_blocks, J->Hkv, J->bs,
-                       D, table_row, n, kvh)) {
+    int bad;
+    if (J->k_bscale)
+      bad = gather_block_scaled(kbuf, (const uint8_t*)J->k_cache, J->k_bscale, J->num_blocks,
+                                J->Hkv, J->bs, D, table_row, n, kvh) ||
+            gather_block_scaled(vbuf, (const uint8_t*)J->v_cache, J->v_bscale, J->num_blocks,
+                                J->Hkv, J->bs, D, table_row, n, kvh);
+    else
+      bad = orc_gather_any(kbuf, J->k_cache, J->cache_dtype, J->k_scale, J->num_blocks, J->Hkv,
+                           J->bs, D, table_row, n, kvh) ||
+            orc_gather_any(vbuf, J->v_cache, J->cache_dtype, J->v_scale, J->num_blocks, J->Hkv,
+                           J->bs, D, table_row, n, kvh);
+    if (bad) {
       atomic_store(&J->err, 1);
       return;
     }
@@ -301,6 +347,29 @@ int orc_decode_e4m3(double* out64, uint16_t* out16, const uint16_t* q, const uin
   decode_job J;
   J.out64 = out64; J.out16 = out16; J.q = q; J.k_cache = k_cache; J.v_cache = v_cache;
   J.cache_dtype = ORC_E4M3; J.k_scale = k_scale; J.v_scale = v_scale;
+  J.k_bscale = NULL; J.v_bscale = NULL;
+  J.block_tables = block_tables; J.context_lens = context_lens;
+  J.items = items; J.n_items = items ? n_items : B;
+  J.q_len = q_len; J.Hq = Hq; J.Hkv = Hkv; J.D = D; J.bs = bs; J.max_blocks = max_blocks;
+  J.num_blocks = num_blocks; J.dtype = dtype; J.scale = scale;
+  return run_decode(&J, B, nthreads);
+}
+
+/* Decode over an 8-bit E4M3 cache with per-(block, kv head) scales: the cached value of
+ * (block b, kv head h) is k_bscale[b][h] * code (v likewise); q and out as for
+ * orc_decode_multi. */
+int orc_decode_e4m3_bs(double* out64, uint16_t* out16, const uint16_t* q, const uint8_t* k_cache,
+                       const uint8_t* v_cache, const float* k_bscale, const float* v_bscale,
+                       const int32_t* block_tables, const int32_t* context_lens, int B, int q_len,
+                       int Hq, int Hkv, int D, int bs, int max_blocks, int num_blocks, double scale,
+                       int dtype, const int32_t* items, int n_items, int nthreads) {
+  if (B < 0 || q_len < 1 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || D <= 0 || bs <= 0 || !k_bscale ||
+      !v_bscale)
+    return -2;
+  decode_job J;
+  J.out64 = out64; J.out16 = out16; J.q = q; J.k_cache = k_cache; J.v_cache = v_cache;
+  J.cache_dtype = ORC_E4M3; J.k_scale = 1.0; J.v_scale = 1.0;
+  J.k_bscale = k_bscale; J.v_bscale = v_bscale;
   J.block_tables = block_tables; J.context_lens = context_lens;
   J.items = items; J.n_items = items ? n_items : B;
   J.q_len = q_len; J.Hq = Hq; J.Hkv = Hkv; J.D = D; J.bs = bs; J.max_blocks = max_blocks;
@@ -317,6 +386,7 @@ int orc_decode_multi(double* out64, uint16_t* out16, const uint16_t* q, const ui
   decode_job J;
   J.out64 = out64; J.out16 = out16; J.q = q; J.k_cache = k_cache; J.v_cache = v_cache;
   J.cache_dtype = dtype; J.k_scale = 1.0; J.v_scale = 1.0;
+  J.k_bscale = NULL; J.v_bscale = NULL;
   J.block_tables = block_tables; J.context_lens = context_lens;
   J.items = items; J.n_items = items ? n_items : B;
   J.q_len = q_len; J.Hq = Hq; J.Hkv = Hkv; J.D = D; J.bs = bs; J.max_blocks = max_blocks;
@@ -421,5 +491,52 @@ int orc_copy_blocks(uint16_t** k_caches, uint16_t** v_caches, int L, const int32
       memcpy(v_caches[l] + dst * block_elems, v_caches[l] + src * block_elems,
              (size_t)block_elems * sizeof(uint16_t));
     }
+  return 0;
+}
+
+/* Quantising append into 8-bit pools with per-(block, kv head) scales (see
+ * orc_e4m3_block_scale).  First, every token whose slot is offset 0 of its block fixes
+ * that block's scales from its own rows (k_bscale[b][h] from k[i][h][:], v likewise);
+ * then every token's values are quantised with its block's scales, exactly as
+ * orc_quantize_e4m3 does for one scale.  Blocks whose offset 0 is not written here keep
+ * their scales.  Negative slots are padding.  Returns 0, or -1 on a slot outside the pool. */
+int orc_cache_append_e4m3_bs(uint8_t* k_cache, uint8_t* v_cache, float* k_bscale,
+                             float* v_bscale, const uint16_t* k, const uint16_t* v,
+                             const int64_t* slots, int T, int Hkv, int D, int bs, int num_blocks,
+                             int dtype) {
+  for (int i = 0; i < T; ++i)
+    if (slots[i] >= (int64_t)num_blocks * bs) return -1;
+  for (int i = 0; i < T; ++i) {
+    int64_t s = slots[i];
+    if (s < 0 || s % bs) continue;
+    int64_t b = s / bs;
+    for (int h = 0; h < Hkv; ++h) {
+      int64_t src = ((int64_t)i * Hkv + h) * D;
+      float ak = 0.0f, av = 0.0f;
+      for (int d = 0; d < D; ++d) {
+        float xk = fabsf((float)to_f64(k[src + d], dtype));
+        float xv = fabsf((float)to_f64(v[src + d], dtype));
+        if (xk > ak) ak = xk;
+        if (xv > av) av = xv;
+      }
+      k_bscale[b * Hkv + h] = orc_e4m3_block_scale(ak);
+      v_bscale[b * Hkv + h] = orc_e4m3_block_scale(av);
+    }
+  }
+  for (int i = 0; i < T; ++i) {
+    int64_t s = slots[i];
+    if (s < 0) continue;
+    int64_t b = s / bs;
+    int o = (int)(s % bs);
+    for (int h = 0; h < Hkv; ++h) {
+      int64_t dst = cache_row(b, h, o, Hkv, bs, D);
+      int64_t src = ((int64_t)i * Hkv + h) * D;
+      float sk = k_bscale[b * Hkv + h], sv = v_bscale[b * Hkv + h];
+      for (int d = 0; d < D; ++d) {
+        k_cache[dst + d] = orc_quantize_e4m3(k[src + d], dtype, sk);
+        v_cache[dst + d] = orc_quantize_e4m3(v[src + d], dtype, sv);
+      }
+    }
+  }
   return 0;
 }

@@ -146,3 +146,113 @@ def test_e4m3_append_writes_the_quantised_codes_and_nothing_else():
     mask = ~touched
     assert np.array_equal(k8.transpose(0, 2, 1, 3)[mask], before_k.transpose(0, 2, 1, 3)[mask])
     assert np.array_equal(v8.transpose(0, 2, 1, 3)[mask], before_v.transpose(0, 2, 1, 3)[mask])
+
+
+# ---- per-(block, kv head) scales: the scale a block's offset-0 token fixes is the power
+# of two s with s/16 < amax/448 <= s/8 (amax/448 in binary32), 1 for an all-zero row.
+
+def _is_pow2(x: float) -> bool:
+    m, _ = np.frexp(x)
+    return x > 0 and m == 0.5
+
+
+def test_block_scale_closed_forms_and_boundaries():
+    assert oracle.e4m3_block_scale(448.0) == 8.0                  # amax/448 = 1 = 2^0
+    assert oracle.e4m3_block_scale(14.0) == 0.25                  # 2^-5 exactly
+    nxt = float(np.nextafter(np.float32(14.0), np.float32(20.0)))
+    assert oracle.e4m3_block_scale(nxt) == 0.5                    # just above: next power
+    assert oracle.e4m3_block_scale(0.0) == 1.0
+    assert oracle.e4m3_block_scale(448.0 * 2.0 ** -20) == 2.0 ** -17
+
+
+def test_block_scale_brackets_the_row_for_any_amax():
+    rng = np.random.default_rng(7)
+    amax = np.concatenate([10.0 ** rng.uniform(-30, 4, 4000),
+                           np.float32(448.0) * 2.0 ** rng.integers(-40, 8, 200)]).astype(np.float32)
+    for a in amax:
+        s = oracle.e4m3_block_scale(float(a))
+        y = float(np.float32(a) / np.float32(448.0))
+        assert _is_pow2(s) and s / 16 < y <= s / 8, (a, s)
+
+
+def _bs_case(dtype, seed, N=12, Hkv=2, bs=4, D=32):
+    rng = np.random.default_rng(seed)
+    k8 = rng.integers(0, 256, size=(N, Hkv, bs, D), dtype=np.uint8)
+    v8 = rng.integers(0, 256, size=(N, Hkv, bs, D), dtype=np.uint8)
+    ks = np.full((N, Hkv), 3.0, np.float32)
+    vs = np.full((N, Hkv), 5.0, np.float32)
+    return k8, v8, ks, vs
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_block_scaled_append_fixes_scales_at_offset_zero_in_any_order(dtype):
+    N, Hkv, bs, D = 12, 2, 4, 32
+    k8, v8, ks, vs = _bs_case(dtype, 1)
+    rng = np.random.default_rng(2)
+    T = 5
+    k = bits(torch.from_numpy(rng.standard_normal((T, Hkv, D)) * 3).to(
+        torch.float16 if dtype == "f16" else torch.bfloat16))
+    v = bits(torch.from_numpy(rng.standard_normal((T, Hkv, D)) * 0.01).to(
+        torch.float16 if dtype == "f16" else torch.bfloat16))
+    # block 7 gets offsets 3 then 0 (the offset-0 token comes later in the batch), block 2
+    # gets offset 1 only (keeps its scale), one padding token
+    slots = np.array([7 * bs + 3, 2 * bs + 1, -1, 7 * bs + 0, 9 * bs + 0], np.int64)
+    k8b, v8b, ksb, vsb = k8.copy(), v8.copy(), ks.copy(), vs.copy()
+    oracle.cache_append_e4m3_bs(k8b, v8b, ksb, vsb, k, v, slots, dtype)
+    kf, vf = bits_to_f64(k, dtype), bits_to_f64(v, dtype)
+    for blk, tok in ((7, 3), (9, 4)):
+        for h in range(Hkv):
+            for x, scl in ((kf[tok, h], ksb[blk, h]), (vf[tok, h], vsb[blk, h])):
+                y = float(np.float32(np.abs(x).max()) / np.float32(448.0))
+                assert _is_pow2(float(scl)) and scl / 16 < y <= scl / 8
+    assert ksb[2].tolist() == [3.0, 3.0] and vsb[2].tolist() == [5.0, 5.0]
+    changed = {7, 9}
+    assert all(ksb[b].tolist() == ks[b].tolist() for b in range(N) if b not in changed)
+    # every written code is the pinned quantiser's code with its block's scale
+    for i, sl in enumerate(slots):
+        if sl < 0:
+            continue
+        b, o = divmod(int(sl), bs)
+        for h in range(Hkv):
+            for d in range(D):
+                assert k8b[b, h, o, d] == oracle.quantize_e4m3(k[i, h, d], dtype, ksb[b, h])
+                assert v8b[b, h, o, d] == oracle.quantize_e4m3(v[i, h, d], dtype, vsb[b, h])
+    # nothing else in the pools changed
+    mask = np.zeros((N, Hkv, bs), bool)
+    for sl in slots:
+        if sl >= 0:
+            mask[int(sl) // bs, :, int(sl) % bs] = True
+    assert np.array_equal(k8b[~mask], k8[~mask]) and np.array_equal(v8b[~mask], v8[~mask])
+    # the first row of a block: its largest value maps into (28, 56] of the code range
+    top = max(abs(oracle.e4m3_to_f64(c)) for c in k8b[9, 0, 0])
+    assert 28 <= top <= 56
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_block_scaled_decode_equals_16bit_decode_of_the_dequantised_pools(dtype):
+    # power-of-two scales keep scale * code exact in fp16 / bf16 at these magnitudes, so
+    # the 8-bit decode must give exactly the pinned 16-bit decode of the dequantised rows
+    case = make_case(4, 8, 2, 64, 8, [5, 16, 17, 40], dtype=dtype, seed=31, poison=False)
+    rng = np.random.default_rng(3)
+    N, Hkv, bs, D = case["k"].shape
+    k8 = rng.integers(0, 0x78, size=(N, Hkv, bs, D), dtype=np.uint8) | \
+        (rng.integers(0, 2, size=(N, Hkv, bs, D), dtype=np.uint8) << 7)
+    v8 = rng.integers(0, 0x78, size=(N, Hkv, bs, D), dtype=np.uint8)
+    ks = (2.0 ** rng.integers(-6, 1, size=(N, Hkv))).astype(np.float32)
+    vs = (2.0 ** rng.integers(-6, 1, size=(N, Hkv))).astype(np.float32)
+    deq = lambda c8, sc: np.vectorize(oracle.e4m3_to_f64)(c8) * sc[:, :, None, None]
+    tdt = torch.float16 if dtype == "f16" else torch.bfloat16
+    k16 = bits(torch.from_numpy(deq(k8, ks)).to(tdt))
+    v16 = bits(torch.from_numpy(deq(v8, vs)).to(tdt))
+    assert np.array_equal(bits_to_f64(k16, dtype), deq(k8, ks))      # exact in 16 bits
+    a, _ = oracle.decode_e4m3_bs(case["q"], k8, v8, ks, vs, case["tables"], case["ctx"],
+                                 case["scale"], dtype)
+    b, _ = oracle.decode(case["q"], k16, v16, case["tables"], case["ctx"], case["scale"], dtype)
+    assert np.array_equal(a, b)
+    # equal block scales everywhere: exactly the per-tensor-scale decode
+    c, _ = oracle.decode_e4m3_bs(case["q"], k8, v8, np.full_like(ks, 0.25),
+                                 np.full_like(vs, 0.5), case["tables"], case["ctx"],
+                                 case["scale"], dtype)
+    e, _ = oracle.decode_e4m3(case["q"], k8, v8, 0.25, 0.5, case["tables"], case["ctx"],
+                              case["scale"], dtype)
+    assert np.array_equal(c, e)
