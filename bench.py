@@ -201,7 +201,12 @@ def oracle_sample(w, bs, max_seconds=15.0, device_batch=None, nthreads=None):
     while i < len(order) and spent < max_seconds:
         items = order[i:i + chunk]
         t0 = time.perf_counter()
-        if k.dtype == np.uint8:
+        if k.dtype == np.uint8 and getattr(b, "kv_bscales", None) is not None:
+            oracle.decode_e4m3_bs(q, k, v, b.kv_bscales[0][0].cpu().numpy(),
+                                  b.kv_bscales[0][1].cpu().numpy(), tables, ctx,
+                                  1.0 / math.sqrt(w.head_dim), w.dtype, items=items,
+                                  nthreads=threads)
+        elif k.dtype == np.uint8:
             oracle.decode_e4m3(q, k, v, *b.kv_scales, tables, ctx, 1.0 / math.sqrt(w.head_dim),
                                w.dtype, items=items, nthreads=threads)
         else:
@@ -267,6 +272,9 @@ def main():
                          "one launch, where the step has one new token per sequence)")
     ap.add_argument("--kv-fp8", action="store_true",
                     help="8-bit E4M3 KV pools (pa_cache_append_e4m3 + pa_decode_e4m3)")
+    ap.add_argument("--kv-fp8-block", action="store_true",
+                    help="8-bit E4M3 KV pools with per-(block, kv head) scales "
+                         "(pa_cache_append_e4m3_bs + pa_decode_e4m3_bs)")
     ap.add_argument("--cascade", action="store_true",
                     help="decode with pa_decode_cascade (shared prefixes read once per chunk)")
     ap.add_argument("--q-len", type=int, default=1,
@@ -307,12 +315,13 @@ def main():
         b = wl.build_prefix_decode(w, device="cuda")
     else:
         b = wl.build(w, device="cuda", block_size=bs, layers=args.layers or None,
-                     q_len=args.q_len, kv8=args.kv_fp8)
+                     q_len=args.q_len, kv8="block" if args.kv_fp8_block else args.kv_fp8)
     if args.cascade:
         wl.use_cascade(b)
     stream = torch.cuda.current_stream()
     L = b.layers
-    fused = not args.unfused and b.q_len == 1 and b.cascade is None and b.kv_scales is None
+    fused = not args.unfused and b.q_len == 1 and b.cascade is None and b.kv_scales is None \
+        and b.kv_bscales is None
     kv_step = b.kv_bytes_per_step()
     kv_layer = kv_step // L
 
@@ -356,7 +365,10 @@ def main():
         if b.cow_pairs is not None and b.cow_pairs.shape[0]:
             pk.pa_copy_blocks(b.k_caches, b.v_caches, b.cow_pairs, b.status)
         for l in range(L):
-            if b.kv_scales is not None:
+            if b.kv_bscales is not None:
+                pk.pa_cache_append_e4m3_bs(b.k_caches[l], b.v_caches[l], *b.kv_bscales[l],
+                                           b.k_new[l], b.v_new[l], b.slot_mapping, b.status)
+            elif b.kv_scales is not None:
                 pk.pa_cache_append_e4m3(b.k_caches[l], b.v_caches[l], b.k_new[l], b.v_new[l],
                                         b.slot_mapping, *b.kv_scales, b.status)
             elif not fused:
@@ -388,6 +400,7 @@ def main():
         dec_src = "an event pair around each launch"
     achieved = kv_layer / (dec_avg * 1e-3) / 1e9
     variant = ("cascade" if b.cascade is not None else "append" if fused else
+               "e4m3bs" if b.kv_bscales is not None else
                "e4m3" if b.kv_scales is not None else "decode" if b.q_len == 1 else "multi")
     traffic = ncu_traffic(w.name, bs, variant)
 
@@ -400,7 +413,9 @@ def main():
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
-        "dtype": w.dtype + ("+e4m3 kv" if b.kv_scales is not None else ""), "data": "synthetic",
+        "dtype": w.dtype + ("+e4m3 kv, per-(block, kv head) scales" if b.kv_bscales is not None
+                            else "+e4m3 kv" if b.kv_scales is not None else ""),
+        "data": "synthetic",
         "config": {"workload": workload_desc(w, bs, b.layers, b.q_len), "global_batch": w.num_seqs * world,
                    "seq_len": float(b.context_lens.float().mean().item()),
                    "parallelism": "replicas" if world > 1 else "single gpu",
@@ -412,6 +427,7 @@ def main():
         "roofline": {"bound": "hbm", "kernel": "pa_decode_split_kernel (%s)" % (
                          "two launches per pa_decode_cascade" if b.cascade is not None else
                          "one launch per pa_decode_append" if fused else
+                         "one launch per pa_decode_e4m3_bs" if b.kv_bscales is not None else
                          "one launch per pa_decode_e4m3" if b.kv_scales is not None else
                          "one launch per pa_decode" if b.q_len == 1 else
                          "one launch per pa_decode_multi"),
@@ -509,6 +525,14 @@ def run_e2e(b, args, world, kv_step, fused=False):
             comp.wait_event(ev_out[l])
             if fused:
                 wl.append_decode_layer(b, l, comp, tabs[m], ctxs[m])
+                ev_used[l].record(comp)
+                continue
+            if b.kv_bscales is not None:
+                pk.pa_cache_append_e4m3_bs(b.k_caches[l], b.v_caches[l], *b.kv_bscales[l],
+                                           b.k_new[l], b.v_new[l], slots[m], b.status, comp)
+                pk.pa_decode_e4m3_bs(b.out[l], b.q[l], b.k_caches[l], b.v_caches[l],
+                                     *b.kv_bscales[l], tabs[m], ctxs[m], b.scale, b.workspace,
+                                     b.status, comp)
                 ev_used[l].record(comp)
                 continue
             if b.kv_scales is not None:
@@ -672,6 +696,9 @@ def secondary_measurements(args, peak):
         ("llama70b_e4m3", lambda: wl.build(inputs.LLAMA70B, layers=1, kv8=True), plain,
          "70B shape, one layer, 8-bit E4M3 pools (bytes counted at 1 per value), "
          "pa_decode_e4m3"),
+        ("llama70b_e4m3_bs", lambda: wl.build(inputs.LLAMA70B, layers=1, kv8="block"), plain,
+         "70B shape, one layer, 8-bit E4M3 pools with per-(block, kv head) scales, "
+         "pa_decode_e4m3_bs"),
         ("llama8b", lambda: wl.build(inputs.LLAMA8B), fused, "8B shape, pa_decode_append"),
         ("llama8b_q4", lambda: wl.build(inputs.LLAMA8B, q_len=4), plain,
          "8B shape, 4 new tokens (16 rows), pa_decode_multi"),
@@ -685,6 +712,9 @@ def secondary_measurements(args, peak):
     runs.append(("heavytail_bs16_identity",
                  lambda: wl.build(inputs.HEAVYTAIL, block_size=16, contiguous=True), fused,
                  "heavy-tailed, block_size 16, identity (contiguous) placement"))
+    runs.append(("heavytail_bs16_e4m3_bs",
+                 lambda: wl.build(inputs.HEAVYTAIL, block_size=16, kv8="block"), plain,
+                 "heavy-tailed, block_size 16, 8-bit pools with per-(block, kv head) scales"))
     runs.append(("heavytail_bs1_e4m3",
                  lambda: wl.build(inputs.HEAVYTAIL, block_size=1, kv8=True), plain,
                  "heavy-tailed, block_size 1, 8-bit E4M3 pools"))

@@ -196,6 +196,46 @@ pa_status pa_decode_e4m3(void* out, const void* q, const void* k_cache, const vo
                          size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 /*
+ * 8-bit KV cache (E4M3) with per-(block, kv head) scales.
+ *
+ * Defined by [P3] "What's Still Unsolved" (FP8 quantised KV cache); the pages give no
+ * format or scale granularity, and this reading gives every (physical block, kv head)
+ * slice of a pool its own scale: k_scales / v_scales, float32 [num_blocks][num_kv_heads]
+ * device arrays beside the pools (value = scale * code).  A block's scale is fixed when
+ * its offset-0 token is written: with amax the largest |x| of that token's row for the
+ * head and y = amax / 448 in binary32, scale = 2^(ceil(log2 y) + 3) -- the power of two s
+ * with s/16 < y <= s/8, leaving 8x headroom for later tokens of the block (larger values
+ * saturate at 448 * s); 1 for an all-zero row.  Blocks fill in order, so every token of a
+ * block is quantised with the scale its first token set.
+ *
+ * pa_cache_append_e4m3_bs -- the quantising append: first every token whose slot is
+ * offset 0 of its block sets that block's scales (in the same call, before any value is
+ * quantised, whatever the order of the tokens), then every value x becomes the E4M3
+ * code of x / scale (binary32 IEEE division, round to nearest even, clamped to 448).
+ * Arguments as for pa_cache_append_e4m3, with the scale arrays in place of the two
+ * per-pool scales; blocks whose offset 0 is not written keep their scales.  Two tokens at
+ * offset 0 of one block in one call are undefined (as are duplicate slots).
+ *
+ * pa_decode_e4m3_bs -- decode of q_len new tokens per sequence (as pa_decode_multi;
+ * q_len = 1 is pa_decode) over such pools: K_s[t] = k_scales[b][h] * code with b the
+ * physical block of position t, V likewise.  Inside, each token row's K scale multiplies
+ * its scores and its V scale its softmax weights before the fp16 tensor-core PV product.
+ * head_dim 128, (num_q_heads/num_kv_heads) * q_len <= 16; workspace as for pa_decode.
+ */
+pa_status pa_cache_append_e4m3_bs(void* k_cache, void* v_cache, float* k_scales,
+                                  float* v_scales, const void* k, const void* v,
+                                  const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
+                                  int head_dim, int block_size, int num_blocks, pa_dtype dtype,
+                                  int32_t* dev_status, void* stream);
+pa_status pa_decode_e4m3_bs(void* out, const void* q, const void* k_cache, const void* v_cache,
+                            const float* k_scales, const float* v_scales,
+                            const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+                            int q_len, int num_q_heads, int num_kv_heads, int head_dim,
+                            int block_size, int max_blocks_per_seq, int num_blocks, float scale,
+                            pa_dtype dtype, void* workspace, size_t workspace_bytes,
+                            int32_t* dev_status, void* stream);
+
+/*
  * pa_decode_cascade -- pa_decode for a batch in which groups of sequences share a prefix
  * of their KV blocks (parallel sampling, beams, a common system prompt), reading each
  * shared block once per chunk of sharers instead of once per sequence.

@@ -146,6 +146,8 @@ struct CascadeArgs {
   const void* v_new = nullptr;
   bool kv8 = false;              // 8-bit E4M3 caches with these scales
   float k_scale = 1.f, v_scale = 1.f;
+  const float* k_bscale = nullptr;   // 8-bit caches: per-(block, kv head) scales instead
+  const float* v_bscale = nullptr;
 };
 
 // Validation, workspace layout, tensor maps and launch shared by the decode entry points.
@@ -230,6 +232,8 @@ pa_status decode_impl(void* out, const void* q, const void* k_cache, const void*
   a.ext_acc = cx.ext_acc;
   a.k_new = cx.k_new;
   a.v_new = cx.v_new;
+  a.k_bscale = cx.k_bscale;
+  a.v_bscale = cx.v_bscale;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return dispatch_mode(cx.kv8, wide, cx.mode, dtype == PA_BF16, head_dim, block_size, a, mk, mv,
                        grid, st);
@@ -362,15 +366,85 @@ pa_status pa_cache_append_e4m3(void* k_cache, void* v_cache, const void* k, cons
                0, st, static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
                static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping,
                num_tokens, num_kv_heads, cpr, block_size, num_blocks, k_scale, v_scale,
-               dev_status);
+               (const float*)nullptr, (const float*)nullptr, dev_status);
   else
     e = pkv_host::launch(pkv::pa_cache_append_e4m3_kernel<__half>, dim3((unsigned)blocks), dim3(256), 0, st,
                static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
                static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping,
                num_tokens, num_kv_heads, cpr, block_size, num_blocks, k_scale, v_scale,
-               dev_status);
+               (const float*)nullptr, (const float*)nullptr, dev_status);
   if (e != cudaSuccess) return PA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_cache_append_e4m3_bs(void* k_cache, void* v_cache, float* k_scales,
+                                  float* v_scales, const void* k, const void* v,
+                                  const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
+                                  int head_dim, int block_size, int num_blocks, pa_dtype dtype,
+                                  int32_t* dev_status, void* stream) {
+  if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
+    return PA_ERR_INVALID;
+  if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  if (head_dim % 16) return PA_ERR_UNSUPPORTED;
+  if (num_tokens == 0) return PA_OK;
+  if (!k_cache || !v_cache || !k || !v || !slot_mapping || !k_scales || !v_scales)
+    return PA_ERR_INVALID;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k) || !aligned16(v))
+    return PA_ERR_INVALID;
+  const int sms = sm_count();
+  if (sms <= 0) return PA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // 1. the blocks whose offset 0 is written here take their scales from that token
+  const long long warps = (long long)num_tokens * num_kv_heads;
+  const unsigned sblocks = (unsigned)((warps * 32 + 255) / 256);
+  cudaError_t e =
+      dtype == PA_BF16
+          ? pkv_host::launch(pkv::pa_e4m3_block_scale_kernel<__nv_bfloat16>, dim3(sblocks), dim3(256),
+                             0, st, k_scales, v_scales, static_cast<const __nv_bfloat16*>(k),
+                             static_cast<const __nv_bfloat16*>(v), slot_mapping, num_tokens,
+                             num_kv_heads, head_dim, block_size, num_blocks)
+          : pkv_host::launch(pkv::pa_e4m3_block_scale_kernel<__half>, dim3(sblocks), dim3(256), 0, st,
+                             k_scales, v_scales, static_cast<const __half*>(k),
+                             static_cast<const __half*>(v), slot_mapping, num_tokens, num_kv_heads,
+                             head_dim, block_size, num_blocks);
+  if (e != cudaSuccess) return PA_ERR_CUDA;
+  // 2. every token quantised with its block's scales
+  const int cpr = head_dim / 16;
+  const long long total = (long long)num_tokens * num_kv_heads * cpr;
+  long long blocks = (total + 255) / 256;
+  if (blocks > (long long)sms * 16) blocks = (long long)sms * 16;
+  if (dtype == PA_BF16)
+    e = pkv_host::launch(pkv::pa_cache_append_e4m3_kernel<__nv_bfloat16>, dim3((unsigned)blocks),
+                         dim3(256), 0, st, static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
+                         static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping,
+                         num_tokens, num_kv_heads, cpr, block_size, num_blocks, 1.f, 1.f,
+                         (const float*)k_scales, (const float*)v_scales, dev_status);
+  else
+    e = pkv_host::launch(pkv::pa_cache_append_e4m3_kernel<__half>, dim3((unsigned)blocks), dim3(256),
+                         0, st, static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
+                         static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping,
+                         num_tokens, num_kv_heads, cpr, block_size, num_blocks, 1.f, 1.f,
+                         (const float*)k_scales, (const float*)v_scales, dev_status);
+  if (e != cudaSuccess) return PA_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_decode_e4m3_bs(void* out, const void* q, const void* k_cache, const void* v_cache,
+                            const float* k_scales, const float* v_scales,
+                            const int32_t* block_tables, const int32_t* context_lens, int num_seqs,
+                            int q_len, int num_q_heads, int num_kv_heads, int head_dim,
+                            int block_size, int max_blocks_per_seq, int num_blocks, float scale,
+                            pa_dtype dtype, void* workspace, size_t workspace_bytes,
+                            int32_t* dev_status, void* stream) {
+  if (num_seqs > 0 && (!k_scales || !v_scales)) return PA_ERR_INVALID;
+  CascadeArgs cx;
+  cx.kv8 = true;
+  cx.k_bscale = k_scales;
+  cx.v_bscale = v_scales;
+  return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, q_len,
+                     num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                     num_blocks, scale, dtype, workspace, workspace_bytes, 0, dev_status, stream,
+                     cx);
 }
 
 size_t pa_decode_cascade_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads,

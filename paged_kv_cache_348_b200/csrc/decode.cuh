@@ -133,6 +133,9 @@ struct DecodeArgs {
   const void* v_new;
   float v_scale;                // 8-bit caches: value = v_scale * code (1 otherwise); the
                                 // K scale is folded into scale_log2
+  // 8-bit caches with per-(block, kv head) scales [num_blocks][Hkv] (null: per-tensor)
+  const float* k_bscale;
+  const float* v_bscale;
 };
 
 
@@ -158,7 +161,11 @@ struct Layout {
   // fused append: per stage the new token's K and V rows, staged by the producer
   static constexpr int kNewOff = (kMlOff + kConsumerWarps * kMaxGroup * 8 + 15) / 16 * 16;
   static constexpr int kNewBytes = KV8 ? 16 : 2 * D * 2;
-  static constexpr int kBytes = kNewOff + kStages * kNewBytes;
+  // 8-bit caches with per-(block, kv head) scales: per stage the K and V scale of every
+  // token row, staged by the producer
+  static constexpr int kScOff = kNewOff + kStages * kNewBytes;
+  static constexpr int kScBytes = KV8 ? 2 * kTileTokens * 4 : 0;
+  static constexpr int kBytes = kScOff + kStages * kScBytes;
   static constexpr int kDynSmem = kBytes + 1024;           // slack for 1024-byte alignment
   static_assert(kBarOff % 8 == 0 && kMiscOff % 8 == 0 && kDescOff % 8 == 0 && kMlOff % 8 == 0 &&
                     kNewOff % 16 == 0 && kNewBytes % 16 == 0,
@@ -448,7 +455,7 @@ __device__ __forceinline__ void merge_split(const DecodeArgs& a, const SplitDesc
   }
 }
 
-template <typename T, int D, int BS, int NT, int MODE, bool KV8 = false>
+template <typename T, int D, int BS, int NT, int MODE, bool KV8 = false, bool KSC = false>
 __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
     pa_decode_split_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
                            const __grid_constant__ CUtensorMap tmv) {
@@ -456,6 +463,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
   constexpr int kStages = L::kStages;
   constexpr int kSegW = seg_weight(BS);
   static_assert(!KV8 || (D == 128 && MODE == kPlain), "8-bit caches: head_dim 128, plain decode");
+  static_assert(!KSC || KV8, "per-block scales belong to 8-bit caches");
   // MMA operand type: the cache's 16-bit type, or fp16 for E4M3 (exact there)
   constexpr bool kBF16 = !KV8 && std::is_same_v<T, __nv_bfloat16>;
   constexpr int kFullCount = (BS == 1) ? 33 : 1;
@@ -730,9 +738,11 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
             else
               blk = win_lookup(w0, w1, w1, wi);       // never touches n0 while it loads
             int y = 0;
+            float scv = 0.f;                           // KSC: this box's block scale
             if (mine) {
               if ((unsigned)blk < (unsigned)a.num_blocks) {
                 y = (blk * Hkv + kvh) * BS + (t % BS);
+                if constexpr (KSC) scv = __ldg((kv ? a.v_bscale : a.k_bscale) + blk * Hkv + kvh);
               } else {
                 if (a.status) atomicOr(a.status, DEV_BAD_BLOCK_ID);
                 y = rows_total;                        // out of range: TMA fills zeros
@@ -751,6 +761,17 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
             uint8_t* sK = smem + st * L::kStageBytes;
             uint8_t* sV = sK + L::kKvBytes;
             uint8_t* sQ = sV + L::kKvBytes;
+            if constexpr (KSC) {
+              // every row's K / V scale: box lane (kv, j, b) covers rows j*16 + b*H .. +H-1
+              // of pool kv (0 for rows past the valid tokens)
+              if (lane < kUnitsPerStage * BPU * 2) {
+                float* sc = reinterpret_cast<float*>(smem + L::kScOff + st * L::kScBytes) +
+                            kv * kTileTokens + j * kUnit + b * H;
+#pragma unroll
+                for (int rr = 0; rr < H; ++rr) sc[rr] = scv;
+              }
+              __syncwarp();
+            }
             if (lane == 0) {
               meta[st] = StageMeta{s_cur, kvh, tok0, nun, ctx_cur, flags, pidx, qslot, newrow};
               mbar_arrive_expect_tx(&full[st], bytes);
@@ -773,6 +794,20 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
             constexpr int CPR = D * (KV8 ? 1 : 2) / 16;   // 16-byte chunks per row
             constexpr int RPI = 32 / CPR;            // rows per warp instruction
             const int ntok = nun * kUnit;
+            // KSC: the K / V scales of rows lane and 32+lane (this stage's table entries
+            // are w0, w1), read before the slot wait
+            float sck0 = 0.f, sck1 = 0.f, scv0 = 0.f, scv1 = 0.f;
+            if constexpr (KSC) {
+              const int nv = ntok < ctx_cur - tok0 ? ntok : ctx_cur - tok0;
+              if (lane < nv && (unsigned)w0 < (unsigned)a.num_blocks) {
+                sck0 = __ldg(a.k_bscale + w0 * Hkv + kvh);
+                scv0 = __ldg(a.v_bscale + w0 * Hkv + kvh);
+              }
+              if (32 + lane < nv && (unsigned)w1 < (unsigned)a.num_blocks) {
+                sck1 = __ldg(a.k_bscale + w1 * Hkv + kvh);
+                scv1 = __ldg(a.v_bscale + w1 * Hkv + kvh);
+              }
+            }
             if (!mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, kWaitLimitNs)) {
               ok = false;
               break;
@@ -780,6 +815,14 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
             uint8_t* sK = smem + st * L::kStageBytes;
             uint8_t* sV = sK + L::kKvBytes;
             uint8_t* sQ = sV + L::kKvBytes;
+            if constexpr (KSC) {
+              float* sc = reinterpret_cast<float*>(smem + L::kScOff + st * L::kScBytes);
+              sc[lane] = sck0;
+              sc[32 + lane] = sck1;
+              sc[kTileTokens + lane] = scv0;
+              sc[kTileTokens + 32 + lane] = scv1;
+              __syncwarp();
+            }
             if (lane == 0) {
               meta[st] = StageMeta{s_cur, kvh, tok0, nun, ctx_cur, flags, pidx, qslot, newrow};
               mbar_arrive_expect_tx(&full[st], qbytes + nbytes);
@@ -999,6 +1042,17 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
           }
         }
         // ---- online softmax (base 2) per query column
+        // KSC: this lane's two rows (gid, gid + 8) carry their blocks' K scales into the
+        // scores and their V scales into P (the row sums keep the unscaled weights)
+        float sl_lo = a.scale_log2, sl_hi = a.scale_log2, vs_lo = 1.f, vs_hi = 1.f;
+        if constexpr (KSC) {
+          const float* sc = reinterpret_cast<const float*>(smem + L::kScOff + st * L::kScBytes);
+          const int r0 = u * kUnit + gid;
+          sl_lo = a.scale_log2 * sc[r0];
+          sl_hi = a.scale_log2 * sc[r0 + 8];
+          vs_lo = sc[kTileTokens + r0];
+          vs_hi = sc[kTileTokens + r0 + 8];
+        }
         uint32_t bhi[NTW][2], blo[NTW][2];
 #pragma unroll
         for (int n = 0; n < NTW; ++n) {
@@ -1007,7 +1061,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
           for (int e = 0; e < 4; ++e) {
             const int row = gid + (e >= 2 ? 8 : 0);
             const int lim = lim0 + jcol[n][e & 1];
-            xs[e] = (row < valid && row < lim) ? sacc[n][e] * a.scale_log2 : -INFINITY;
+            xs[e] = (row < valid && row < lim) ? sacc[n][e] * (e >= 2 ? sl_hi : sl_lo) : -INFINITY;
           }
           float alpha[2], p[4];
           bool grew = false;
@@ -1039,7 +1093,8 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
             }
           }
           using TM = std::conditional_t<KV8, __half, T>;   // MMA operand type
-          const uint32_t h01 = pack2<TM>(p[0], p[1]), h23 = pack2<TM>(p[2], p[3]);
+          const uint32_t h01 = pack2<TM>(p[0] * vs_lo, p[1] * vs_lo);
+          const uint32_t h23 = pack2<TM>(p[2] * vs_hi, p[3] * vs_hi);
           bhi[n][0] = movmatrix_t(h01);
           bhi[n][1] = movmatrix_t(h23);
           if constexpr (!KV8) {

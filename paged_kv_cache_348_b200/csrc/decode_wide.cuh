@@ -49,6 +49,7 @@ constexpr int kWideThreads = 64 + kWideSoftThreads;
 constexpr uint32_t kWideTmemCols = 512;
 constexpr uint32_t kOCol = 256;
 constexpr float kRescaleLog2 = 8.f;               // a reference max moves past this gap only
+constexpr int kWideSegWeight = 40;                // see pa_decode_wide_kernel
 
 template <int D>
 struct WideLayout {
@@ -72,7 +73,9 @@ struct WideLayout {
   // the two buffers again with -inf replaced by 0 (the reference p is computed against)
   static constexpr int kRedOff = kMrefOff + 5 * kWideCols * 4;  // float [64 cols][4 warps]
   static constexpr int kAlphaOff = kRedOff + kWideCols * 4 * 4;
-  static constexpr int kBytes = kAlphaOff + kWideCols * 4;
+  // per query column: new token (or chunk member) j and head g within the group
+  static constexpr int kColOff = kAlphaOff + kWideCols * 4;
+  static constexpr int kBytes = kColOff + 2 * kWideCols * 4;
   static constexpr int kDynSmem = kBytes + 1024;                // slack for 1024-byte alignment
   static_assert(kStageBytes % 1024 == 0 && kQOff % 1024 == 0 && kKvBytes % 1024 == 0,
                 "tiles need 1024-byte alignment (128-byte swizzle atoms)");
@@ -173,7 +176,11 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   // residual (columns NC..2NC-1, summed when O^T is read back); fp16 P has 11, enough here
   constexpr bool kSplit = std::is_same_v<T, __nv_bfloat16>;
   constexpr int kNPV = kSplit ? 2 * NC : NC;        // MMA N of PV
-  constexpr int kSegW = seg_weight(BS);
+  // a segment's schedule weight beyond its units: a portion's fixed cost here (first stage
+  // with its reference-max pass and Q load, end-of-portion epilogue) is worth about this
+  // many 16-token units of streaming, several stages' worth (measured per CTA with
+  // global-timer stamps), far more than in the mma.sync kernel
+  constexpr int kSegW = kWideSegWeight;
   constexpr uint32_t kAB = std::is_same_v<T, __nv_bfloat16> ? 1u : 0u;
   constexpr int kFullCount = 33;       // lane 0's expect_tx arrival + 32 cp.async arrivals
   extern __shared__ uint8_t smem_raw[];
@@ -194,6 +201,8 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   float* mref = reinterpret_cast<float*>(smem + L::kMrefOff);      // [5][64]
   float* red = reinterpret_cast<float*>(smem + L::kRedOff);        // [64][4]
   float* alph = reinterpret_cast<float*>(smem + L::kAlphaOff);     // [64]
+  int* colj = reinterpret_cast<int*>(smem + L::kColOff);           // [64] column -> j
+  int* colg = colj + kWideCols;                                    // [64] column -> head in group
   uint8_t* sQ = smem + L::kQOff;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -220,6 +229,11 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   if (warp == 1) {
     tmem_alloc(tmem_slot, kWideTmemCols);
     tmem_relinquish();
+  }
+  if (threadIdx.x >= 64 && threadIdx.x < 64 + kWideCols) {
+    const int cq = threadIdx.x - 64;
+    colj[cq] = cq / a.group;
+    colg[cq] = cq % a.group;
   }
   tc_fence_before();
   __syncthreads();
@@ -598,6 +612,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       int no_abort = 0;
       mbar_wait_bounded(drain, 0u, &no_abort, kWaitLimitNs);
     }
+    __syncwarp();      // the warp reaches the CTA barrier below together, lane 0 included
   } else {
     // ============================== softmax / epilogue ==============================
     const int wg = (warp - 2) >> 2;                // softmax warpgroup: columns c0 .. c0+CW-1
@@ -695,7 +710,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
 #pragma unroll
         for (int j = 0; j < CW; ++j) {
           const int cq = c0 + j;
-          const bool vis = tv && cq < a.ncol && (MODE == kPrefix || r < lim0 + cq / group);
+          const bool vis = tv && cq < a.ncol && (MODE == kPrefix || r < lim0 + colj[cq]);
           if (!vis) s[j] = -INFINITY;
           e = fmaxf(e, fmaf(s[j], sc, -mcur[cq]));
         }
@@ -837,7 +852,16 @@ __global__ void __launch_bounds__(kWideThreads, 1)
               const float Ls = (w4.x + w4.y) + (w4.z + w4.w);
               const float M = mc[cq];
               if (complete) {
-                const long long row = out_row<MODE>(a, mt.seq, mt.kvh, cq);
+                // output row of column cq: out_row without its divisions
+                long long row;
+                if constexpr (MODE == kPrefix) {
+                  const int mem = chunk_member(a, mt.seq, colj[cq]);
+                  row = mem < 0 ? -1ll
+                                : (long long)mem * a.num_q_heads + (long long)mt.kvh * group + colg[cq];
+                } else {
+                  row = ((long long)mt.seq * a.q_len + colj[cq]) * a.num_q_heads +
+                        (long long)mt.kvh * group + colg[cq];
+                }
                 if (row >= 0) {
                   if constexpr (MODE == kPrefix) {
                     if (d == 0) a.ext_ml[row] = make_float2(M, Ls);

@@ -58,16 +58,75 @@ __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float x0, float x1) {
   return d;
 }
 
+// Scale of a (block, kv head) slice of an 8-bit cache, fixed by the block's offset-0 token
+// ("PagedAttention -- The KV Cache Problem", "What's Still Unsolved": FP8 quantised KV
+// cache): the power of two s with s/16 < amax/448 <= s/8, i.e. 2^(ceil(log2 y) + 3) with
+// y = amax / 448 in binary32; 1 for a zero (or non-finite) amax.  ceil(log2 y) comes from
+// y's bits: a power of two gives its exponent, anything else one more.
+__device__ __forceinline__ float e4m3_block_scale(float amax) {
+  const float y = __fdiv_rn(amax, 448.f);
+  if (!(y > 0.f) || isinf(y)) return 1.f;
+  const uint32_t u = __float_as_uint(y);
+  const int ex = (int)((u >> 23) & 0xffu);
+  const uint32_t man = u & 0x7fffffu;
+  int c;
+  if (ex == 0) {                                  // subnormal: y = man * 2^-149
+    const int p = 31 - __clz(man);
+    c = man == (1u << p) ? p - 149 : p - 148;
+  } else {
+    c = ex - 127 + (man ? 1 : 0);
+  }
+  c += 3;
+  c = c < -126 ? -126 : (c > 127 ? 127 : c);
+  return __uint_as_float((uint32_t)(c + 127) << 23);
+}
+
+// First step of the block-scaled 8-bit append: every token whose slot is offset 0 of its
+// block fixes that block's (K and V) scales for each kv head from its own rows.  One warp
+// per (token, kv head); 16-bit input rows of D values.
+template <typename T>
+__global__ void __launch_bounds__(256)
+    pa_e4m3_block_scale_kernel(float* __restrict__ k_bscale, float* __restrict__ v_bscale,
+                               const T* __restrict__ k, const T* __restrict__ v,
+                               const int64_t* __restrict__ slot_mapping, int num_tokens, int Hkv,
+                               int D, int block_size, int num_blocks) {
+  pdl_wait();
+  pdl_trigger();
+  const int lane = threadIdx.x & 31;
+  const long long w = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
+  if (w >= (long long)num_tokens * Hkv) return;
+  const int h = (int)(w % Hkv);
+  const long long tok = w / Hkv;
+  const long long slot = slot_mapping[tok];
+  if (slot < 0 || slot >= (long long)num_blocks * block_size || slot % block_size) return;
+  const long long b = slot / block_size;
+  float ak = 0.f, av = 0.f;
+  for (int d = lane; d < D; d += 32) {
+    const long long i = (tok * Hkv + h) * D + d;
+    ak = fmaxf(ak, fabsf((float)k[i]));
+    av = fmaxf(av, fabsf((float)v[i]));
+  }
+  ak = warp_max_f32(ak);
+  av = warp_max_f32(av);
+  if (lane == 0) {
+    k_bscale[b * Hkv + h] = e4m3_block_scale(ak);
+    v_bscale[b * Hkv + h] = e4m3_block_scale(av);
+  }
+}
+
 // The append into 8-bit E4M3 caches: as pa_cache_append_kernel, each value quantised as
-// x / scale (binary32, IEEE division) rounded to E4M3.  One thread per 16 values: two
-// 16-byte loads of 16-bit input, one 16-byte store of codes.
+// x / scale (binary32, IEEE division) rounded to E4M3, with one scale per pool (k_scale,
+// v_scale) or, when k_bscale is not null, the scale of the destination (block, kv head)
+// (set beforehand for blocks whose offset 0 is written in the same call).  One thread per
+// 16 values: two 16-byte loads of 16-bit input, one 16-byte store of codes.
 template <typename T>
 __global__ void __launch_bounds__(256)
     pa_cache_append_e4m3_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
                                 const uint4* __restrict__ k, const uint4* __restrict__ v,
                                 const int64_t* __restrict__ slot_mapping, int num_tokens,
                                 int Hkv, int chunks_per_row, int block_size, int num_blocks,
-                                float k_scale, float v_scale, int32_t* status) {
+                                float k_scale, float v_scale, const float* __restrict__ k_bscale,
+                                const float* __restrict__ v_bscale, int32_t* status) {
   pdl_wait();
   pdl_trigger();
   const long long total = (long long)num_tokens * Hkv * chunks_per_row;
@@ -88,7 +147,7 @@ __global__ void __launch_bounds__(256)
     const long long dst = ((b * Hkv + h) * block_size + off) * chunks_per_row + ch;
     for (int kv = 0; kv < 2; ++kv) {
       const uint4* src = (kv ? v : k) + 2 * i;
-      const float sc = kv ? v_scale : k_scale;
+      const float sc = k_bscale ? (kv ? v_bscale : k_bscale)[b * Hkv + h] : (kv ? v_scale : k_scale);
       const uint4 in[2] = {src[0], src[1]};
       const uint32_t* w = reinterpret_cast<const uint32_t*>(in);
       uint32_t q[4];

@@ -40,11 +40,11 @@ cudaError_t launch(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
-template <typename T, int D, int BS, int NT, int MODE, bool KV8 = false>
+template <typename T, int D, int BS, int NT, int MODE, bool KV8 = false, bool KSC = false>
 pa_status launch_decode(const pkv::DecodeArgs& a, const CUtensorMap& mk, const CUtensorMap& mv,
                         int grid, cudaStream_t stream) {
   using L = pkv::Layout<D, KV8, pkv::ctas_per_sm(KV8, NT, BS)>;
-  auto split = pkv::pa_decode_split_kernel<T, D, BS, NT, MODE, KV8>;
+  auto split = pkv::pa_decode_split_kernel<T, D, BS, NT, MODE, KV8, KSC>;
   if (cudaFuncSetAttribute(split, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynSmem) !=
       cudaSuccess)
     return PA_ERR_CUDA;
@@ -80,23 +80,28 @@ pa_status dispatch_d(int d, int bs, const pkv::DecodeArgs& a, const CUtensorMap&
                  : dispatch_bs<T, 128, MODE>(bs, a, mk, mv, grid, s);
 }
 
-// 8-bit (E4M3) caches: plain decode, head_dim 128.
-template <typename T>
+// 8-bit (E4M3) caches: plain decode (one or several new tokens), head_dim 128; KSC: per-
+// (block, kv head) scales instead of one per pool.
+template <typename T, bool KSC = false>
 pa_status dispatch_e4m3(int bs, const pkv::DecodeArgs& a, const CUtensorMap& mk,
                         const CUtensorMap& mv, int grid, cudaStream_t s) {
   const bool nt1 = a.ncol <= 8;
   switch (bs) {
-    case 1: return nt1 ? launch_decode<T, 128, 1, 1, pkv::kPlain, true>(a, mk, mv, grid, s)
-                       : launch_decode<T, 128, 1, 2, pkv::kPlain, true>(a, mk, mv, grid, s);
-    case 8: return nt1 ? launch_decode<T, 128, 8, 1, pkv::kPlain, true>(a, mk, mv, grid, s)
-                       : launch_decode<T, 128, 8, 2, pkv::kPlain, true>(a, mk, mv, grid, s);
-    case 16: return nt1 ? launch_decode<T, 128, 16, 1, pkv::kPlain, true>(a, mk, mv, grid, s)
-                        : launch_decode<T, 128, 16, 2, pkv::kPlain, true>(a, mk, mv, grid, s);
-    case 32: return nt1 ? launch_decode<T, 128, 32, 1, pkv::kPlain, true>(a, mk, mv, grid, s)
-                        : launch_decode<T, 128, 32, 2, pkv::kPlain, true>(a, mk, mv, grid, s);
+    case 1: return nt1 ? launch_decode<T, 128, 1, 1, pkv::kPlain, true, KSC>(a, mk, mv, grid, s)
+                       : launch_decode<T, 128, 1, 2, pkv::kPlain, true, KSC>(a, mk, mv, grid, s);
+    case 8: return nt1 ? launch_decode<T, 128, 8, 1, pkv::kPlain, true, KSC>(a, mk, mv, grid, s)
+                       : launch_decode<T, 128, 8, 2, pkv::kPlain, true, KSC>(a, mk, mv, grid, s);
+    case 16: return nt1 ? launch_decode<T, 128, 16, 1, pkv::kPlain, true, KSC>(a, mk, mv, grid, s)
+                        : launch_decode<T, 128, 16, 2, pkv::kPlain, true, KSC>(a, mk, mv, grid, s);
+    case 32: return nt1 ? launch_decode<T, 128, 32, 1, pkv::kPlain, true, KSC>(a, mk, mv, grid, s)
+                        : launch_decode<T, 128, 32, 2, pkv::kPlain, true, KSC>(a, mk, mv, grid, s);
   }
   return PA_ERR_UNSUPPORTED;
 }
+
+// The block-scaled 8-bit instances; defined in decode_e4m3_bs.cu.
+pa_status run_e4m3_bs(bool bf16, int bs, const pkv::DecodeArgs& a, const CUtensorMap& mk,
+                      const CUtensorMap& mv, int grid, cudaStream_t s);
 
 // One kernel mode's instances, dispatched on the other parameters; defined in
 // decode_<mode>.cu.  kv8: 8-bit E4M3 pools (kPlain only).

@@ -32,7 +32,8 @@ EXPORTS = ("pa_version", "pa_status_string", "pa_decode_workspace_bytes", "pa_de
            "pa_bm_allocate", "pa_bm_fork", "pa_bm_append_tokens", "pa_bm_release",
            "pa_bm_context_len", "pa_bm_num_blocks_of", "pa_bm_max_blocks", "pa_bm_block_tables",
            "pa_bm_slot_of", "pa_bm_plan_cascade", "pa_plan_cascade", "pa_bm_swap_out",
-           "pa_bm_swap_in", "pa_swap_out_blocks", "pa_swap_in_blocks")
+           "pa_bm_swap_in", "pa_swap_out_blocks", "pa_swap_in_blocks", "pa_cache_append_e4m3_bs",
+           "pa_decode_e4m3_bs")
 
 _lib = None
 _lock = threading.Lock()
@@ -74,6 +75,12 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         L.pa_decode_e4m3.restype = i32
         L.pa_decode_e4m3.argtypes = [P, P, P, P, f32, f32, P, P, i32, i32, i32, i32, i32, i32, i32,
                                      f32, i32, P, sz, P, P]
+        L.pa_cache_append_e4m3_bs.restype = i32
+        L.pa_cache_append_e4m3_bs.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32,
+                                              P, P]
+        L.pa_decode_e4m3_bs.restype = i32
+        L.pa_decode_e4m3_bs.argtypes = [P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32,
+                                        i32, f32, i32, P, sz, P, P]
         L.pa_decode_cascade_workspace_bytes.restype = sz
         L.pa_decode_cascade_workspace_bytes.argtypes = [i32, i32, i32, i32]
         L.pa_decode_cascade.restype = i32
@@ -263,6 +270,64 @@ def pa_decode_e4m3(out, q, k_cache8, v_cache8, k_scale: float, v_scale: float, b
                                _ptr(workspace), workspace.numel() * workspace.element_size(),
                                _ptr(status), _stream(stream))
     _check(rc, "pa_decode_e4m3")
+    return out
+
+
+def pa_cache_append_e4m3_bs(k_cache8, v_cache8, k_scales, v_scales, k, v, slot_mapping,
+                            status=None, stream=None):
+    """Quantising scatter of 16-bit k/v [T,Hkv,D] into uint8 E4M3 pools with per-(block,
+    kv head) scales (float32 [N,Hkv], set for blocks whose offset 0 is written); see
+    pa_cache_append_e4m3_bs in include/pagedkv.h."""
+    _need(k_cache8, "k_cache", dtype=torch.uint8, ndim=4)
+    _need(v_cache8, "v_cache", dtype=torch.uint8, ndim=4)
+    _need(k_scales, "k_scales", dtype=torch.float32, ndim=2)
+    _need(v_scales, "v_scales", dtype=torch.float32, ndim=2)
+    _need(k, "k", ndim=3)
+    _need(v, "v", dtype=k.dtype, ndim=3)
+    _need(slot_mapping, "slot_mapping", dtype=torch.int64, ndim=1)
+    N, Hkv, bs, D = k_cache8.shape
+    T = k.shape[0]
+    if v_cache8.shape != k_cache8.shape or k.shape != (T, Hkv, D) or v.shape != k.shape or \
+            slot_mapping.shape[0] != T or k_scales.shape != (N, Hkv) or \
+            v_scales.shape != (N, Hkv):
+        raise PagedKVError("pa_cache_append_e4m3_bs: inconsistent shapes")
+    rc = load().pa_cache_append_e4m3_bs(_ptr(k_cache8), _ptr(v_cache8), _ptr(k_scales),
+                                        _ptr(v_scales), _ptr(k), _ptr(v), _ptr(slot_mapping), T,
+                                        Hkv, D, bs, N, _dtype_code(k), _ptr(status),
+                                        _stream(stream))
+    _check(rc, "pa_cache_append_e4m3_bs")
+
+
+def pa_decode_e4m3_bs(out, q, k_cache8, v_cache8, k_scales, v_scales, block_tables,
+                      context_lens, scale: float, workspace, status=None, stream=None):
+    """out <- paged decode over uint8 E4M3 pools with per-(block, kv head) scales; q and
+    out [B,Hq,D] (one new token) or [B,QL,Hq,D] (QL new tokens, causal); see
+    pa_decode_e4m3_bs in include/pagedkv.h."""
+    if q.dim() not in (3, 4):
+        raise PagedKVError("q must have 3 or 4 dims")
+    _need(q, "q")
+    _need(out, "out", dtype=q.dtype, ndim=q.dim())
+    _need(k_cache8, "k_cache", dtype=torch.uint8, ndim=4)
+    _need(v_cache8, "v_cache", dtype=torch.uint8, ndim=4)
+    _need(k_scales, "k_scales", dtype=torch.float32, ndim=2)
+    _need(v_scales, "v_scales", dtype=torch.float32, ndim=2)
+    _need(block_tables, "block_tables", dtype=torch.int32, ndim=2)
+    _need(context_lens, "context_lens", dtype=torch.int32, ndim=1)
+    _need(workspace, "workspace")
+    B, QL = q.shape[0], (q.shape[1] if q.dim() == 4 else 1)
+    Hq, D = q.shape[-2], q.shape[-1]
+    N, Hkv, bs, D2 = k_cache8.shape
+    if out.shape != q.shape or D2 != D or v_cache8.shape != k_cache8.shape or \
+            block_tables.shape[0] != B or context_lens.shape[0] != B or \
+            k_scales.shape != (N, Hkv) or v_scales.shape != (N, Hkv):
+        raise PagedKVError("pa_decode_e4m3_bs: inconsistent shapes")
+    rc = load().pa_decode_e4m3_bs(_ptr(out), _ptr(q), _ptr(k_cache8), _ptr(v_cache8),
+                                  _ptr(k_scales), _ptr(v_scales), _ptr(block_tables),
+                                  _ptr(context_lens), B, QL, Hq, Hkv, D, bs,
+                                  block_tables.shape[1], N, float(scale), _dtype_code(q),
+                                  _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                  _ptr(status), _stream(stream))
+    _check(rc, "pa_decode_e4m3_bs")
     return out
 
 

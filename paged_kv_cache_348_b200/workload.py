@@ -46,6 +46,7 @@ class DecodeBatch:
     q_len: int = 1
     cascade: tuple | None = None     # (prefix_lens, chunk_members, chunk_prefix_lens) on device
     kv_scales: tuple | None = None   # (k_scale, v_scale) of 8-bit E4M3 pools, else None
+    kv_bscales: list | None = None   # per layer (k_scales, v_scales) [N, Hkv] of block-scaled pools
 
     @property
     def layers(self) -> int:
@@ -91,10 +92,40 @@ def _alloc_layers(w, N, bs, layers, device, seed, kv8=False):
     return k, v
 
 
+def _fill_block_scaled(w, bs, bm, sids, N, layers, device, seed):
+    """8-bit pools with per-(block, kv head) scales, filled the way a server fills them:
+    every cached token's 16-bit K/V rows (N(0,1)) appended in position order with
+    pa_cache_append_e4m3_bs, so each block's scale is the one its first token fixed."""
+    import torch
+
+    slots = torch.tensor([bm.slot_of(s, p) for s in sids for p in range(bm.context_len(s))],
+                         dtype=torch.int64, device=device)
+    T = slots.shape[0]
+    k8, v8, sc = [], [], []
+    for l in range(layers):
+        kc = torch.zeros((N, w.num_kv_heads, bs, w.head_dim), dtype=torch.uint8, device=device)
+        vc = torch.zeros_like(kc)
+        ks = torch.ones((N, w.num_kv_heads), dtype=torch.float32, device=device)
+        vs = torch.ones_like(ks)
+        kr = inputs.randn((T, w.num_kv_heads, w.head_dim), w.dtype, seed, device, stream=1000 + 2 * l)
+        vr = inputs.randn((T, w.num_kv_heads, w.head_dim), w.dtype, seed, device, stream=1001 + 2 * l)
+        pk.pa_cache_append_e4m3_bs(kc, vc, ks, vs, kr, vr, slots)
+        del kr, vr
+        k8.append(kc)
+        v8.append(vc)
+        sc.append((ks, vs))
+    return k8, v8, sc
+
+
 def _finish(w, bs, bm, sids, N, layers, device, cow_pairs=None, q_len=1,
             kv8=False) -> DecodeBatch:
     B = len(sids)
-    k_caches, v_caches = _alloc_layers(w, N, bs, layers, device, w.seed, kv8)
+    if kv8 == "block":
+        k_caches, v_caches, bscales = _fill_block_scaled(w, bs, bm, sids, N, layers, device,
+                                                         w.seed)
+    else:
+        k_caches, v_caches = _alloc_layers(w, N, bs, layers, device, w.seed, kv8)
+        bscales = None
     tables = torch.from_numpy(bm.block_tables(sids)).to(device)
     ctx = torch.from_numpy(bm.context_lens(sids)).to(device)
     # the newest q_len tokens of every sequence are the ones appended and queried
@@ -117,14 +148,17 @@ def _finish(w, bs, bm, sids, N, layers, device, cow_pairs=None, q_len=1,
         pairs = torch.tensor(cow_pairs, dtype=torch.int32, device=device).reshape(-1, 2)
     return DecodeBatch(w, bs, bm, sids, N, k_caches, v_caches, tables, ctx, slots, q, kn, vn, out,
                        ws, st, pairs, 1.0 / math.sqrt(w.head_dim), q_len,
-                       kv_scales=(KV8_SCALE, KV8_SCALE) if kv8 else None)
+                       kv_scales=(KV8_SCALE, KV8_SCALE) if kv8 is True else None,
+                       kv_bscales=bscales)
 
 
 def build(w: inputs.Workload, device="cuda", block_size: int | None = None,
-          layers: int | None = None, q_len: int = 1, kv8: bool = False,
+          layers: int | None = None, q_len: int = 1, kv8=False,
           contiguous: bool = False) -> DecodeBatch:
     """Independent sequences (every workload but the shared-prefix one).  With q_len > 1
-    every sequence's newest q_len tokens are appended and queried each step.  With
+    every sequence's newest q_len tokens are appended and queried each step.  kv8: False
+    (16-bit pools), True (8-bit pools, one scale per pool) or "block" (8-bit pools with
+    per-(block, kv head) scales, filled by the quantising append).  With
     contiguous=True the pool hands out blocks in id order, so every sequence's table is
     one run of consecutive blocks (the identity placement a contiguous cache would have)
     instead of the seeded fragmented one."""
@@ -186,10 +220,13 @@ def run_step(b: DecodeBatch, stream=None, layers=None, fused: bool = False) -> N
     if b.cow_pairs is not None and b.cow_pairs.shape[0]:
         pk.pa_copy_blocks(b.k_caches, b.v_caches, b.cow_pairs, b.status, stream)
     for l in range(layers if layers is not None else b.layers):
-        if fused and b.kv_scales is None:
+        if fused and b.kv_scales is None and b.kv_bscales is None:
             append_decode_layer(b, l, stream)
             continue
-        if b.kv_scales is not None:
+        if b.kv_bscales is not None:
+            pk.pa_cache_append_e4m3_bs(b.k_caches[l], b.v_caches[l], *b.kv_bscales[l], b.k_new[l],
+                                       b.v_new[l], b.slot_mapping, b.status, stream)
+        elif b.kv_scales is not None:
             pk.pa_cache_append_e4m3(b.k_caches[l], b.v_caches[l], b.k_new[l], b.v_new[l],
                                     b.slot_mapping, *b.kv_scales, b.status, stream)
         else:
@@ -228,6 +265,10 @@ def decode_layer(b: DecodeBatch, l: int, stream=None) -> None:
     if b.cascade is not None:
         pk.pa_decode_cascade(b.out[l], b.q[l], b.k_caches[l], b.v_caches[l], b.block_tables,
                              b.context_lens, *b.cascade, b.scale, b.workspace, b.status, stream)
+        return
+    if b.kv_bscales is not None:
+        pk.pa_decode_e4m3_bs(b.out[l], b.q[l], b.k_caches[l], b.v_caches[l], *b.kv_bscales[l],
+                             b.block_tables, b.context_lens, b.scale, b.workspace, b.status, stream)
         return
     if b.kv_scales is not None:
         pk.pa_decode_e4m3(b.out[l], b.q[l], b.k_caches[l], b.v_caches[l], *b.kv_scales,
