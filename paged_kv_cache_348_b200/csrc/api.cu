@@ -100,6 +100,27 @@ bool encode_pool(CUtensorMap* map, const void* base, pa_dtype dtype, int head_di
   return r == CUDA_SUCCESS;
 }
 
+// The tcgen05 kernel's 4-D view of a 16-bit pool: (64 dims, 8 rows, column halves, 8-row
+// groups) with byte strides (row D*2, half 128, group 8*D*2); a box of box_groups groups
+// lands in shared memory as [group][half][8 rows][128 bytes], 128-byte swizzle.  rows must
+// be a multiple of 8 (block_size >= 8).
+bool encode_pool_wide(CUtensorMap* map, const void* base, pa_dtype dtype, int head_dim,
+                      uint64_t rows, int box_groups) {
+  auto enc = tensor_map_encoder();
+  if (!enc || rows % 8) return false;
+  const int halves = head_dim / 64;
+  cuuint64_t dims[4] = {64u, 8u, (cuuint64_t)halves, (cuuint64_t)(rows / 8)};
+  cuuint64_t strides[3] = {(cuuint64_t)head_dim * 2, 128u, (cuuint64_t)head_dim * 2 * 8};
+  cuuint32_t box[4] = {64u, 8u, (cuuint32_t)halves, (cuuint32_t)box_groups};
+  cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  CUresult r = enc(map, dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                         : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                   4, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // Every call gets its own epoch so arrival counters left by earlier calls (or by an
 // aborted one) read as zero; 0 is skipped so a zeroed workspace also reads as zero.
 uint32_t next_epoch() {
@@ -197,9 +218,14 @@ pa_status decode_impl(void* out, const void* q, const void* k_cache, const void*
   if (block_size != 1) {
     const uint64_t rows = (uint64_t)num_blocks * num_kv_heads * block_size;
     const int box_rows = block_size < 16 ? block_size : 16;
-    if (!encode_pool(&mk, k_cache, dtype, head_dim, rows, box_rows, cx.kv8) ||
-        !encode_pool(&mv, v_cache, dtype, head_dim, rows, box_rows, cx.kv8))
+    if (wide) {
+      if (!encode_pool_wide(&mk, k_cache, dtype, head_dim, rows, box_rows / 8) ||
+          !encode_pool_wide(&mv, v_cache, dtype, head_dim, rows, box_rows / 8))
+        return PA_ERR_CUDA;
+    } else if (!encode_pool(&mk, k_cache, dtype, head_dim, rows, box_rows, cx.kv8) ||
+               !encode_pool(&mv, v_cache, dtype, head_dim, rows, box_rows, cx.kv8)) {
       return PA_ERR_CUDA;
+    }
   }
   pkv::DecodeArgs a;
   a.out = out;

@@ -51,10 +51,15 @@ constexpr uint32_t kOCol = 256;
 constexpr float kRescaleLog2 = 8.f;               // a reference max moves past this gap only
 constexpr int kWideSegWeight = 40;                // see pa_decode_wide_kernel
 
+// K and V tiles: token row r, 64-dim half h (128 bytes, 128-byte swizzle) at
+// ((r / 8) * kHalves + h) * 1024 + (r % 8) * 128: 8-row atoms with the halves side by side,
+// so one TMA box (a 4-D view of the pool) brings a 16-row unit's both halves, and the
+// MMA descriptors see 8-row groups at a stride of kHalves * 1024 bytes.
 template <int D>
 struct WideLayout {
   static constexpr int kHalves = D / 64;                        // 128-byte column halves
   static constexpr int kKvBytes = kHalves * kWideTile * 128;    // one K or V tile
+  static constexpr int kGroupBytes = kHalves * 1024;            // one 8-row group, all halves
   static constexpr int kPBytes = kWideTile * 128;               // P^T high or low part
   // P^T (high, low) goes to the stage's K tile once QK^T has read it, when it fits
   static constexpr bool kPInK = kKvBytes >= 2 * kPBytes;
@@ -366,18 +371,18 @@ __global__ void __launch_bounds__(kWideThreads, 1)
           uint8_t* sK = smem + st * L::kStageBytes;
           uint8_t* sV = sK + L::kKvBytes;
           if constexpr (BS != 1) {
-            constexpr int H = BS < 16 ? BS : 16;     // rows per TMA box
-            constexpr int BPU = kUnit / H;           // boxes per unit and column half
-            constexpr int kBoxBytes = H * 128;
-            constexpr int kMaxBox = kWideUnits * BPU * L::kHalves * 2;
+            constexpr int H = BS < 16 ? BS : 16;     // rows per TMA box (all column halves)
+            constexpr int BPU = kUnit / H;           // boxes per unit
+            constexpr int kBoxBytes = H * 128 * L::kHalves;
+            constexpr int kMaxBox = kWideUnits * BPU * 2;
             constexpr int kRep = (kMaxBox + 31) / 32;
-            const int nbox = nun * BPU * L::kHalves * 2;
+            const int nbox = nun * BPU * 2;
             // this lane's boxes and their block-table entries, read before the slot wait
             int ys[kRep];
 #pragma unroll
             for (int rp = 0; rp < kRep; ++rp) {
               const int bi = lane + 32 * rp;
-              const int jb = (bi >> 1) / L::kHalves;
+              const int jb = bi >> 1;
               const int t = tok0 + (jb / BPU) * kUnit + (jb % BPU) * H;
               ys[rp] = -1;
               if (bi < nbox && t < ctx_cur) {
@@ -394,7 +399,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
             for (int jj = 0; jj < nun; ++jj) {
               const int rem = ctx_cur - (tok0 + jj * kUnit);
               const int nb = (rem + H - 1) / H;
-              bytes += (uint32_t)((nb < BPU ? nb : BPU) * kBoxBytes * L::kHalves * 2);
+              bytes += (uint32_t)((nb < BPU ? nb : BPU) * kBoxBytes * 2);
             }
             if (!mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, kWaitLimitNs)) {
               ok = false;
@@ -409,10 +414,10 @@ __global__ void __launch_bounds__(kWideThreads, 1)
             for (int rp = 0; rp < kRep; ++rp) {
               const int bi = lane + 32 * rp;
               if (ys[rp] >= 0) {
-                const int kv = bi & 1, hf = (bi >> 1) % L::kHalves, jb = (bi >> 1) / L::kHalves;
-                uint8_t* dst = (kv ? sV : sK) + hf * (kWideTile * 128) +
-                               ((jb / BPU) * kUnit + (jb % BPU) * H) * 128;
-                tma_load_2d(dst, kv ? &tmv : &tmk, &full[st], hf * 64, ys[rp], policy);
+                const int kv = bi & 1, jb = bi >> 1;
+                const int row0 = (jb / BPU) * kUnit + (jb % BPU) * H;   // a multiple of 8
+                uint8_t* dst = (kv ? sV : sK) + (row0 >> 3) * L::kGroupBytes;
+                tma_load_4d(dst, kv ? &tmv : &tmk, &full[st], ys[rp] >> 3, policy);
               }
             }
           } else {
@@ -439,8 +444,6 @@ __global__ void __launch_bounds__(kWideThreads, 1)
             const int ch = lane % CPR, hf = ch >> 3, cc = ch & 7, rl = lane / CPR;
             const uint8_t* kb = static_cast<const uint8_t*>(a.k_cache) + ch * 16;
             const uint8_t* vb = static_cast<const uint8_t*>(a.v_cache) + ch * 16;
-            uint8_t* sKl = sK + hf * (kWideTile * 128) + rl * 128;
-            uint8_t* sVl = sV + hf * (kWideTile * 128) + rl * 128;
 #pragma unroll 4
             for (int i = 0; i < kWideTile / RPI; ++i) {
               const int r0 = i * RPI;
@@ -460,9 +463,10 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                   if (a.status) atomicOr(a.status, DEV_BAD_BLOCK_ID);
                   sz = 0;                              // zero fill, no read
                 }
-                const int soff = r0 * 128 + ((cc ^ (r & 7)) << 4);
-                cp_async_16_zfill(sKl + soff, kb + row * (D * 2), sz, policy);
-                cp_async_16_zfill(sVl + soff, vb + row * (D * 2), sz, policy);
+                const int soff = ((r >> 3) * L::kHalves + hf) * 1024 + (r & 7) * 128 +
+                                 ((cc ^ (r & 7)) << 4);
+                cp_async_16_zfill(sK + soff, kb + row * (D * 2), sz, policy);
+                cp_async_16_zfill(sV + soff, vb + row * (D * 2), sz, policy);
               }
             }
           }
@@ -531,8 +535,8 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       // field (16-byte units, bits 0..13; every address here is below 256 KB, so the sum
       // never carries out of the field)
       const uint64_t dq0 = smem_desc_sw128(smem_u32(sQ), 16u, 1024u);
-      const uint64_t dk0 = smem_desc_sw128(smem_u32(smem), 16u, 1024u);
-      const uint64_t dv0 = smem_desc_sw128(smem_u32(smem + L::kKvBytes), kWideTile * 128, 1024u);
+      const uint64_t dk0 = smem_desc_sw128(smem_u32(smem), 16u, L::kGroupBytes);
+      const uint64_t dv0 = smem_desc_sw128(smem_u32(smem + L::kKvBytes), 1024u, L::kGroupBytes);
       const uint64_t dp0 = smem_desc_sw128(smem_u32(smem + L::kPOff), L::kPBytes, 1024u);
       auto adv = [](uint64_t d, uint32_t bytes) { return d + (uint64_t)(bytes >> 4); };
       auto qk = [&](int slot, int flags) {
@@ -541,7 +545,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint32_t off = (ks & 3) * 32;          // 16 dims = 32 bytes along a row
           tc_mma_f16(tbase + (uint32_t)(slot * 64),
-                     adv(dk0, so + (ks >> 2) * (kWideTile * 128) + off),
+                     adv(dk0, so + (ks >> 2) * 1024 + off),
                      adv(dq0, (ks >> 2) * (kWideCols * 128) + off), idesc_qk, ks > 0);
         }
         tc_commit(&sfull[slot]);
@@ -551,7 +555,8 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         const uint32_t so = (uint32_t)(slot * L::kStageBytes);
 #pragma unroll
         for (int kk = 0; kk < kWideTile / 16; ++kk)
-          tc_mma_f16(tbase + kOCol, adv(dv0, so + kk * 2048), adv(dp0, so + kk * 2048), idesc_pv,
+          tc_mma_f16(tbase + kOCol, adv(dv0, so + kk * 2 * L::kGroupBytes), adv(dp0, so + kk * 2048),
+                     idesc_pv,
                      !(first && kk == 0));
       };
       int q_slot = 0, p_slot = 0, n_qk = 0, n_pv = 0;
@@ -798,7 +803,8 @@ __global__ void __launch_bounds__(kWideThreads, 1)
           // a row past the stage's valid tokens may hold stale or NaN data: P is zero
           // there, and V must be finite (0 x NaN would poison O); warpgroup wg clears
           // column half wg of the row
-          uint8_t* sV = smem + st * L::kStageBytes + L::kKvBytes + wg * (kWideTile * 128) + r * 128;
+          uint8_t* sV = smem + st * L::kStageBytes + L::kKvBytes + (r >> 3) * L::kGroupBytes +
+                        wg * 1024 + (r & 7) * 128;
 #pragma unroll
           for (int ch = 0; ch < 8; ++ch)
             *reinterpret_cast<uint4*>(sV + ch * 16) = make_uint4(0u, 0u, 0u, 0u);
