@@ -187,13 +187,7 @@ def oracle_sample(w, bs, max_seconds=15.0, device_batch=None, nthreads=None):
         q, k, v = bits(b.q[0]), bits(b.k_caches[0]), bits(b.v_caches[0])
         tables, ctx = b.block_tables.cpu().numpy(), b.context_lens.cpu().numpy()
     else:
-        from paged_kv_cache_348_b200 import workload as wl
-        b = wl.build(w, device="cpu", block_size=bs, layers=1) if w.name != "prefix" else \
-            wl.build_prefix_decode(w, device="cpu")
-        def bits(t):
-            return t.contiguous().view(torch.int16).numpy().view(np.uint16)
-        q, k, v = bits(b.q[0]), bits(b.k_caches[0]), bits(b.v_caches[0])
-        tables, ctx = b.block_tables.numpy(), b.context_lens.numpy()
+        q, k, v, tables, ctx = oracle_inputs(w, bs)
     order = list(range(len(ctx)))
     done_bytes, spent, seqs = 0, 0.0, 0
     chunk = max(1, threads // 8)
@@ -219,6 +213,51 @@ def oracle_sample(w, bs, max_seconds=15.0, device_batch=None, nthreads=None):
         seqs += len(items)
         i += chunk
     return done_bytes, spent, seqs, threads
+
+
+def oracle_inputs(w, bs):
+    """Layer 0 of the workload for the oracle arm, built without the library: block tables
+    from the oracle's reference block manager (the same seeded pool order and, for the
+    shared-prefix workload, the same forks and appends as the GPU workload), values from
+    the seeded generators with the streams the GPU workload uses."""
+    import torch
+
+    from oracle.cow import RefBlockManager
+    from paged_kv_cache_348_b200 import inputs
+
+    ctx = [int(c) for c in inputs.context_lens(w)]
+    if w.name == "prefix":
+        need = inputs.PREFIX_PROMPTS * (inputs.PREFIX_LEN // bs) + sum(
+            -(-(c - inputs.PREFIX_LEN) // bs) for c in ctx)
+    else:
+        need = sum(-(-c // bs) for c in ctx)
+    N = w.pool_blocks if w.pool_blocks else int(math.ceil(w.pool_factor * need))
+    bm = RefBlockManager(N, bs, inputs.pool_order(N, w.seed))
+    if w.name == "prefix":
+        sids = []
+        for p in range(inputs.PREFIX_PROMPTS):
+            root = bm.new_seq(inputs.PREFIX_LEN)
+            kids = [root] + [bm.fork(root) for _ in range(inputs.PREFIX_SAMPLES - 1)]
+            for j, sid in enumerate(kids):
+                for _ in range(ctx[p * inputs.PREFIX_SAMPLES + j] - inputs.PREFIX_LEN):
+                    bm.append_slot(sid)
+                sids.append(sid)
+    else:
+        sids = [bm.new_seq(c) for c in ctx]
+    M = max(1, max(len(bm.tables[s]) for s in sids))
+    tables = np.zeros((len(sids), M), dtype=np.int32)
+    for i, s in enumerate(sids):
+        tables[i, :len(bm.tables[s])] = bm.tables[s]
+    lens = np.array([bm.ctx[s] for s in sids], dtype=np.int32)
+
+    def bits(t):
+        return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+    shape = (N, w.num_kv_heads, bs, w.head_dim)
+    k = bits(inputs.randn(shape, w.dtype, w.seed, "cpu", stream=1000))
+    v = bits(inputs.randn(shape, w.dtype, w.seed, "cpu", stream=1001))
+    q = bits(inputs.randn((len(sids), w.num_q_heads, w.head_dim), w.dtype, w.seed, "cpu",
+                          stream=5000))
+    return q, k, v, tables, lens
 
 
 def run_reference(args, w, bs, rank, world):

@@ -31,10 +31,11 @@
  *    rows one kv head serves (q heads per kv head x new tokens per sequence, or x chunk
  *    members in a cascade prefix pass) may number up to 64 for pa_decode,
  *    pa_decode_multi and the cascade's prefix pass, up to 16 for pa_decode_append,
- *    pa_decode_e4m3 and the cascade's per-sequence pass.  Up to 16 rows run on
- *    warp-level tensor-core MMAs; 17 to 64 on the 5th-generation (tcgen05) tensor cores
- *    with the accumulators in tensor memory (PAGEDKV_WIDE_MIN_COLS=n in the environment
- *    moves that threshold, for comparing the two kernels).  Pointers must be 16-byte
+ *    pa_decode_e4m3 and the cascade's per-sequence pass.  Up to 8 rows run on warp-level
+ *    tensor-core MMAs; 9 to 64 on the 5th-generation (tcgen05) tensor cores with the
+ *    accumulators in tensor memory (PAGEDKV_WIDE_MIN_COLS=n in the environment moves that
+ *    threshold, for comparing the two kernels; the fused append, 8-bit pools and the
+ *    cascade's per-sequence pass keep the warp-level kernel up to 16 rows).  Pointers must be 16-byte
  *    aligned.
  */
 #ifndef PAGEDKV_H

@@ -56,12 +56,14 @@ size_t split_workspace_bytes(int head_dim, int sms) {
 }
 
 // Query columns per kv head from which the tcgen05 kernel takes a launch (plain and prefix
-// modes; PAGEDKV_WIDE_MIN_COLS=n overrides it, for comparing the two kernels).
+// modes): 9, since at 16 columns it was measured faster than the mma.sync kernel's two
+// n-tiles (70B shape with 2 new tokens 0.105 vs 0.107 ms, 8B shape with 4: 0.078 vs
+// 0.084 ms).  PAGEDKV_WIDE_MIN_COLS=n overrides it, for comparing the two kernels.
 int wide_min_cols() {
   static const int v = [] {
     const char* e = std::getenv("PAGEDKV_WIDE_MIN_COLS");
     const int x = e ? std::atoi(e) : 0;
-    return (x >= 1 && x <= pkv::kWideCols + 1) ? x : pkv::kMaxGroup + 1;
+    return (x >= 1 && x <= pkv::kWideCols + 1) ? x : 9;
   }();
   return v;
 }

@@ -6,8 +6,9 @@
 // the launches whose query rows per kv head -- the GQA group times the new tokens of a
 // sequence ("PagedAttention -- The KV Cache Problem", "Why This Matters for Production":
 // beam search and parallel sampling), or the members of a shared-prefix chunk -- number
-// 17..64.  There the contraction is a real dense tile (up to 64 flop per KV byte), too
-// much for warp-level mma.sync, so it runs on the 5th-generation tensor cores:
+// 9..64.  There the contraction is a real dense tile (up to 64 flop per KV byte), too
+// much for warp-level mma.sync with register accumulators, so it runs on the
+// 5th-generation tensor cores:
 //
 //  * One persistent CTA per SM takes an equal range of the batch's 16-token units (the
 //    schedule of decode.cuh: segments = (sequence, kv head), weighted split, partials of
@@ -20,8 +21,8 @@
 //    accumulated in tensor memory (one S^T buffer per ring slot); then O^T[D][N] +=
 //    V^T . P^T with V read MN-major from the same tile.  It is event driven: a stage's
 //    QK^T goes out as soon as its tiles land, its PV as soon as the softmax is done.
-//  * Warps 2..9, two warpgroups that split the query columns, run the softmax: a thread
-//    owns one token row of S^T (one TMEM lane) and half of the columns.  Base 2, fp32, with
+//  * The softmax warps (warps 2..9, two warpgroups) split the query columns: a thread owns
+//    one token row of S^T (one TMEM lane) and half of the columns.  Base 2, fp32, with
 //    a lazily moved reference maximum per query row (a stage moves it only when some score
 //    exceeds it by more than 2^8, which after a portion's first stage is rare; O^T is then
 //    rescaled in tensor memory).  P^T is written in 16 bits into the stage's K tile, which
@@ -42,8 +43,12 @@ constexpr int kWideCols = 64;                     // query rows per kv head hand
 constexpr int kWideTile = 128;                    // tokens per stage (MMA M of QK^T)
 constexpr int kWideUnits = kWideTile / kUnit;     // 16-token units per stage
 constexpr int kWideStages = 3;
-constexpr int kWideSoftThreads = 256;             // softmax warps 2..9 (two warpgroups)
-constexpr int kWideThreads = 64 + kWideSoftThreads;
+// softmax warpgroups (warps 2 .. 1 + 4 * SWG): two, each owning half of the NC query columns.
+// Four (16 columns each at NC 64) measured slower: the 576-thread CTA caps a thread at 96
+// registers and the softmax spilled.
+__host__ __device__ constexpr int wide_swg(int) { return 2; }
+__host__ __device__ constexpr int wide_soft_threads(int nc) { return 128 * wide_swg(nc); }
+__host__ __device__ constexpr int wide_threads(int nc) { return 64 + wide_soft_threads(nc); }
 // tensor memory: one S^T buffer per ring slot (columns 64 s .. 64 s + NC - 1) and O^T from
 // column 256 (NC columns, or 2 NC when P's residual is a second column block)
 constexpr uint32_t kWideTmemCols = 512;
@@ -92,7 +97,7 @@ struct WideLayout {
 // Last arrival of a split segment (see merge_split in decode.cuh), for up to 64 query
 // columns: out = (sum_k acc_k 2^(m_k - M)) / (sum_k l_k 2^(m_k - M)), contributors folded
 // in CTA order.  Thread tid owns elements (column, 4 dims) e = tid + 256 i, 4 at a time.
-template <typename T, int D, int MODE>
+template <typename T, int D, int MODE, int kWideSoftThreads>
 __device__ __forceinline__ void merge_wide(const DecodeArgs& a, const SplitDesc& dsc,
                                            long long total, int G, int tid) {
   constexpr int kF4 = D / 4;
@@ -170,13 +175,14 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const float* v) {
 }
 
 template <typename T, int D, int BS, int MODE, int NC>
-__global__ void __launch_bounds__(kWideThreads, 1)
+__global__ void __launch_bounds__(wide_threads(NC), 1)
     pa_decode_wide_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
                           const __grid_constant__ CUtensorMap tmv) {
   using L = WideLayout<D>;
   static_assert(MODE == kPlain || MODE == kPrefix, "wide decode: plain (multi-token) or prefix");
   static_assert(NC == 16 || NC == 32 || NC == 64, "16, 32 or 64 query columns");
-  constexpr int CW = NC / 2;                        // columns of one softmax warpgroup
+  constexpr int kWideSoftThreads = wide_soft_threads(NC);
+  constexpr int CW = NC / wide_swg(NC);             // columns of one softmax warpgroup
   // bf16 P keeps ~16 bits as a high part (columns 0..NC-1 of P^T and O^T) plus its rounding
   // residual (columns NC..2NC-1, summed when O^T is read back); fp16 P has 11, enough here
   constexpr bool kSplit = std::is_same_v<T, __nv_bfloat16>;
@@ -909,7 +915,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
             *last_flag = last;
           }
           named_bar_sync(1, kWideSoftThreads);
-          if (*last_flag) merge_wide<T, D, MODE>(a, dsc, *total_s, G, tid);
+          if (*last_flag) merge_wide<T, D, MODE, kWideSoftThreads>(a, dsc, *total_s, G, tid);
         }
         named_bar_sync(1, kWideSoftThreads);       // red[] is reused by the next stage
 #pragma unroll

@@ -130,7 +130,7 @@ pa_status launch_wide(const pkv::DecodeArgs& a, const CUtensorMap& mk, const CUt
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynSmem) !=
       cudaSuccess)
     return PA_ERR_CUDA;
-  if (launch(k, dim3(grid), dim3(pkv::kWideThreads), L::kDynSmem, stream, a, mk, mv) !=
+  if (launch(k, dim3(grid), dim3(pkv::wide_threads(NC)), L::kDynSmem, stream, a, mk, mv) !=
       cudaSuccess)
     return PA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
