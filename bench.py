@@ -359,8 +359,7 @@ def main():
         wl.use_cascade(b)
     stream = torch.cuda.current_stream()
     L = b.layers
-    fused = not args.unfused and b.q_len == 1 and b.cascade is None and b.kv_scales is None \
-        and b.kv_bscales is None
+    fused = not args.unfused and b.q_len == 1 and b.cascade is None and b.kv_scales is None
     kv_step = b.kv_bytes_per_step()
     kv_layer = kv_step // L
 
@@ -404,13 +403,15 @@ def main():
         if b.cow_pairs is not None and b.cow_pairs.shape[0]:
             pk.pa_copy_blocks(b.k_caches, b.v_caches, b.cow_pairs, b.status)
         for l in range(L):
-            if b.kv_bscales is not None:
+            if fused:
+                pass
+            elif b.kv_bscales is not None:
                 pk.pa_cache_append_e4m3_bs(b.k_caches[l], b.v_caches[l], *b.kv_bscales[l],
                                            b.k_new[l], b.v_new[l], b.slot_mapping, b.status)
             elif b.kv_scales is not None:
                 pk.pa_cache_append_e4m3(b.k_caches[l], b.v_caches[l], b.k_new[l], b.v_new[l],
                                         b.slot_mapping, *b.kv_scales, b.status)
-            elif not fused:
+            else:
                 pk.pa_cache_append(b.k_caches[l], b.v_caches[l], b.k_new[l], b.v_new[l],
                                    b.slot_mapping, b.status)
             ev_s[s * L + l].record(stream)
@@ -438,7 +439,9 @@ def main():
         dec_avg = dec_avg_events
         dec_src = "an event pair around each launch"
     achieved = kv_layer / (dec_avg * 1e-3) / 1e9
-    variant = ("cascade" if b.cascade is not None else "append" if fused else
+    variant = ("cascade" if b.cascade is not None else
+               "e4m3bs_append" if fused and b.kv_bscales is not None else
+               "append" if fused else
                "e4m3bs" if b.kv_bscales is not None else
                "e4m3" if b.kv_scales is not None else "decode" if b.q_len == 1 else "multi")
     traffic = ncu_traffic(w.name, bs, variant)
@@ -465,6 +468,8 @@ def main():
         "kv_bytes_per_step": kv_step,
         "roofline": {"bound": "hbm", "kernel": "pa_decode_split_kernel (%s)" % (
                          "two launches per pa_decode_cascade" if b.cascade is not None else
+                         "one launch per pa_decode_append_e4m3_bs" if fused and
+                         b.kv_bscales is not None else
                          "one launch per pa_decode_append" if fused else
                          "one launch per pa_decode_e4m3_bs" if b.kv_bscales is not None else
                          "one launch per pa_decode_e4m3" if b.kv_scales is not None else
@@ -569,9 +574,15 @@ def run_e2e(b, args, world, kv_step, fused=False):
             if b.kv_bscales is not None:
                 pk.pa_cache_append_e4m3_bs(b.k_caches[l], b.v_caches[l], *b.kv_bscales[l],
                                            b.k_new[l], b.v_new[l], slots[m], b.status, comp)
-                pk.pa_decode_e4m3_bs(b.out[l], b.q[l], b.k_caches[l], b.v_caches[l],
-                                     *b.kv_bscales[l], tabs[m], ctxs[m], b.scale, b.workspace,
-                                     b.status, comp)
+                if b.cascade is not None:
+                    pk.pa_decode_cascade_e4m3_bs(b.out[l], b.q[l], b.k_caches[l],
+                                                 b.v_caches[l], *b.kv_bscales[l], tabs[m],
+                                                 ctxs[m], *b.cascade, b.scale, b.workspace,
+                                                 b.status, comp)
+                else:
+                    pk.pa_decode_e4m3_bs(b.out[l], b.q[l], b.k_caches[l], b.v_caches[l],
+                                         *b.kv_bscales[l], tabs[m], ctxs[m], b.scale,
+                                         b.workspace, b.status, comp)
                 ev_used[l].record(comp)
                 continue
             if b.kv_scales is not None:
@@ -738,6 +749,9 @@ def secondary_measurements(args, peak):
         ("llama70b_e4m3_bs", lambda: wl.build(inputs.LLAMA70B, layers=1, kv8="block"), plain,
          "70B shape, one layer, 8-bit E4M3 pools with per-(block, kv head) scales, "
          "pa_decode_e4m3_bs"),
+        ("llama70b_e4m3_bs_append", lambda: wl.build(inputs.LLAMA70B, layers=1, kv8="block"),
+         fused, "70B shape, one layer, 8-bit E4M3 pools with per-(block, kv head) scales, "
+         "pa_decode_append_e4m3_bs (the newest token quantised and appended in the launch)"),
         ("llama8b", lambda: wl.build(inputs.LLAMA8B), fused, "8B shape, pa_decode_append"),
         ("llama8b_q4", lambda: wl.build(inputs.LLAMA8B, q_len=4), plain,
          "8B shape, 4 new tokens (16 rows), pa_decode_multi"),

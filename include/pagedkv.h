@@ -30,13 +30,13 @@
  *    num_q_heads % num_kv_heads == 0; q, out and the caches share one dtype.  The query
  *    rows one kv head serves (q heads per kv head x new tokens per sequence, or x chunk
  *    members in a cascade prefix pass) may number up to 64 for pa_decode,
- *    pa_decode_multi and the cascade's prefix pass, up to 16 for pa_decode_append,
- *    pa_decode_e4m3 and the cascade's per-sequence pass.  Up to 8 rows run on warp-level
- *    tensor-core MMAs; 9 to 64 on the 5th-generation (tcgen05) tensor cores with the
- *    accumulators in tensor memory (PAGEDKV_WIDE_MIN_COLS=n in the environment moves that
- *    threshold, for comparing the two kernels; the fused append, 8-bit pools and the
- *    cascade's per-sequence pass keep the warp-level kernel up to 16 rows).  Pointers must be 16-byte
- *    aligned.
+ *    pa_decode_multi, pa_decode_append and the cascade's prefix pass over 16-bit pools,
+ *    up to 16 for 8-bit pools and the cascade's per-sequence pass.  Up to 8 rows run on
+ *    warp-level tensor-core MMAs; 9 to 64 on the 5th-generation (tcgen05) tensor cores
+ *    with the accumulators in tensor memory (PAGEDKV_WIDE_MIN_COLS=n in the environment
+ *    moves that threshold, for comparing the two kernels; 8-bit pools and the cascade's
+ *    per-sequence pass keep the warp-level kernel up to 16 rows).  Pointers must be
+ *    16-byte aligned.
  */
 #ifndef PAGEDKV_H
 #define PAGEDKV_H
@@ -284,6 +284,44 @@ pa_status pa_decode_cascade(void* out, const void* q, const void* k_cache, const
                             void* stream);
 
 /*
+ * The cascade and the fused append over 8-bit pools with per-(block, kv head) scales
+ * (the format of pa_cache_append_e4m3_bs / pa_decode_e4m3_bs; head_dim 128).
+ *
+ * pa_decode_cascade_e4m3_bs -- pa_decode_cascade over such pools: the result is that of
+ * pa_decode_e4m3_bs (q_len 1) on the same inputs, the softmax split at prefix_lens[s]
+ * and recombined exactly as for pa_decode_cascade.  Arguments, contract and errors as
+ * for pa_decode_cascade, plus the scale arrays, with one more limit: a chunk holds at
+ * most 16 query rows, (num_q_heads/num_kv_heads) * chunk_width <= 16.  Workspace:
+ * pa_decode_cascade_workspace_bytes.
+ *
+ * pa_decode_append_e4m3_bs -- pa_cache_append_e4m3_bs of each sequence's newest token
+ * (position p = context_lens[s] - 1, slot of p through block_tables) fused into
+ * pa_decode_e4m3_bs (q_len 1): the same cache codes, scales and output bits as the two
+ * calls in sequence.  When p is offset 0 of its block the token sets that block's scales
+ * (k_scales, v_scales are written there); otherwise they are read.  Arguments and errors
+ * as for pa_decode_append, plus the scale arrays; the newest token's block must not be
+ * shared with another sequence.
+ */
+pa_status pa_decode_cascade_e4m3_bs(void* out, const void* q, const void* k_cache,
+                                    const void* v_cache, const float* k_scales,
+                                    const float* v_scales, const int32_t* block_tables,
+                                    const int32_t* context_lens, const int32_t* prefix_lens,
+                                    int num_seqs, const int32_t* chunk_members, int chunk_width,
+                                    const int32_t* chunk_prefix_lens, int num_chunks,
+                                    int num_q_heads, int num_kv_heads, int head_dim,
+                                    int block_size, int max_blocks_per_seq, int num_blocks,
+                                    float scale, pa_dtype dtype, void* workspace,
+                                    size_t workspace_bytes, int32_t* dev_status, void* stream);
+pa_status pa_decode_append_e4m3_bs(void* out, const void* q, void* k_cache, void* v_cache,
+                                   float* k_scales, float* v_scales, const void* k_new,
+                                   const void* v_new, const int32_t* block_tables,
+                                   const int32_t* context_lens, int num_seqs, int num_q_heads,
+                                   int num_kv_heads, int head_dim, int block_size,
+                                   int max_blocks_per_seq, int num_blocks, float scale,
+                                   pa_dtype dtype, void* workspace, size_t workspace_bytes,
+                                   int32_t* dev_status, void* stream);
+
+/*
  * pa_cache_append -- write the new tokens' K and V into their cache slots.
  *
  * Defined by [P1] "How PagedAttention borrows OS paging" (blocks are filled on demand
@@ -361,9 +399,11 @@ pa_status pa_swap_in_blocks(void* const* k_caches, void* const* v_caches, int nu
  *
  * Same arguments, results and errors as pa_decode, minus workspace/workspace_bytes,
  * with these differences:
- *  - The scratch holds the split partials of at most 444 CTAs (3 per SM on a 148-SM
- *    B200, the most pa_decode schedules there) at head_dim <= 128: head_dim above 128
- *    returns PA_ERR_UNSUPPORTED, and a GPU with more SMs is scheduled with 444 CTAs.
+ *  - The scratch holds the split partials, at head_dim <= 128, of at most 444 CTAs of
+ *    the warp-level kernel (3 per SM on a 148-SM B200, the most pa_decode schedules
+ *    there) or 148 of the tcgen05 kernel (one per SM, 9 to 64 query rows per kv head):
+ *    head_dim above 128 returns PA_ERR_UNSUPPORTED, and a GPU with more SMs is
+ *    scheduled with at most those numbers of CTAs.
  *    The batch size does not change the scratch; num_seqs above PA_NOALLOC_MAX_SEQS
  *    returns PA_ERR_INVALID as a stated limit of this call, not of the scratch.
  *  - The first call on a device looks up the device address of the array for that
@@ -377,7 +417,7 @@ pa_status pa_swap_in_blocks(void* const* k_caches, void* const* v_caches, int nu
  *    different streams, or from different host threads) race on it and give wrong
  *    results: order them on one stream or with events.
  */
-#define PA_NOALLOC_SCRATCH_BYTES 7864320
+#define PA_NOALLOC_SCRATCH_BYTES 9852160
 #define PA_NOALLOC_MAX_SEQS 16384
 pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache, const void* v_cache,
                             const int32_t* block_tables, const int32_t* context_lens,

@@ -143,11 +143,23 @@ pa_status dispatch_mode(bool kv8, bool wide, int mode, bool bf16, int d, int bs,
       return nc == 16 ? run_wide_mode<pkv::kPrefix, 16>(bf16, d, bs, a, mk, mv, grid, s)
              : nc == 32 ? run_wide_mode<pkv::kPrefix, 32>(bf16, d, bs, a, mk, mv, grid, s)
                         : run_wide_mode<pkv::kPrefix, 64>(bf16, d, bs, a, mk, mv, grid, s);
+    if (mode == pkv::kAppend)
+      return nc == 16 ? run_wide_mode<pkv::kAppend, 16>(bf16, d, bs, a, mk, mv, grid, s)
+             : nc == 32 ? run_wide_mode<pkv::kAppend, 32>(bf16, d, bs, a, mk, mv, grid, s)
+                        : run_wide_mode<pkv::kAppend, 64>(bf16, d, bs, a, mk, mv, grid, s);
     return nc == 16 ? run_wide_mode<pkv::kPlain, 16>(bf16, d, bs, a, mk, mv, grid, s)
            : nc == 32 ? run_wide_mode<pkv::kPlain, 32>(bf16, d, bs, a, mk, mv, grid, s)
                       : run_wide_mode<pkv::kPlain, 64>(bf16, d, bs, a, mk, mv, grid, s);
   }
-  if (kv8) return run_decode_mode<pkv::kPlain, true>(bf16, d, bs, a, mk, mv, grid, s);
+  if (kv8) {
+    switch (mode) {
+      case pkv::kPlain: return run_decode_mode<pkv::kPlain, true>(bf16, d, bs, a, mk, mv, grid, s);
+      case pkv::kPrefix: return run_decode_mode<pkv::kPrefix, true>(bf16, d, bs, a, mk, mv, grid, s);
+      case pkv::kSuffix: return run_decode_mode<pkv::kSuffix, true>(bf16, d, bs, a, mk, mv, grid, s);
+      case pkv::kAppend: return run_decode_mode<pkv::kAppend, true>(bf16, d, bs, a, mk, mv, grid, s);
+    }
+    return PA_ERR_INVALID;
+  }
   switch (mode) {
     case pkv::kPlain: return run_decode_mode<pkv::kPlain, false>(bf16, d, bs, a, mk, mv, grid, s);
     case pkv::kPrefix: return run_decode_mode<pkv::kPrefix, false>(bf16, d, bs, a, mk, mv, grid, s);
@@ -192,8 +204,9 @@ pa_status decode_impl(void* out, const void* q, const void* k_cache, const void*
   const int group = num_q_heads / num_kv_heads;
   const long long ncol = (long long)group * q_len;
   // query columns per kv head: up to 16 on the mma.sync kernel (every mode), up to 64 on
-  // the tcgen05 kernel (16-bit pools, plain and prefix modes)
-  const bool wide_mode = !cx.kv8 && (cx.mode == pkv::kPlain || cx.mode == pkv::kPrefix);
+  // the tcgen05 kernel (16-bit pools: plain, prefix and fused-append modes)
+  const bool wide_mode = !cx.kv8 && (cx.mode == pkv::kPlain || cx.mode == pkv::kPrefix ||
+                                     cx.mode == pkv::kAppend);
   if (ncol > (wide_mode ? pkv::kWideCols : pkv::kMaxGroup)) return PA_ERR_UNSUPPORTED;
   const bool wide = wide_mode && ncol >= wide_min_cols();
   if ((long long)num_blocks * num_kv_heads * block_size >= (1ll << 31) ||
@@ -209,14 +222,18 @@ pa_status decode_impl(void* out, const void* q, const void* k_cache, const void*
   const int sms = sm_count();
   if (sms <= 0) return PA_ERR_CUDA;
   int grid = wide ? sms : sms * pkv::ctas_per_sm(cx.kv8, ncol <= 8 ? 1 : 2, block_size);
-  if (grid_cap > 0 && grid > grid_cap) grid = grid_cap;
+  // a cap counts mma.sync CTAs (up to kMaxCtasPerSm a SM); the tcgen05 kernel runs one a SM
+  const int cap = grid_cap > 0 ? (wide ? grid_cap / pkv::kMaxCtasPerSm : grid_cap) : 0;
+  if (cap > 0 && grid > cap) grid = cap;
   const WsLayout w = ws_layout(head_dim, grid, wide ? pkv::kWideCols : pkv::kMaxGroup);
   if (workspace_bytes < w.total) return PA_ERR_INVALID;
 
   CUtensorMap mk, mv;
   std::memset(&mk, 0, sizeof(mk));
   std::memset(&mv, 0, sizeof(mv));
-  if (cx.kv8 && (head_dim != 128 || cx.mode != pkv::kPlain)) return PA_ERR_UNSUPPORTED;
+  // 8-bit pools: head_dim 128; the cascade and fused-append modes need per-block scales
+  if (cx.kv8 && (head_dim != 128 || (cx.mode != pkv::kPlain && !cx.k_bscale)))
+    return PA_ERR_UNSUPPORTED;
   if (block_size != 1) {
     const uint64_t rows = (uint64_t)num_blocks * num_kv_heads * block_size;
     const int box_rows = block_size < 16 ? block_size : 16;
@@ -280,6 +297,58 @@ CascadeLayout cascade_layout(int num_seqs, int num_q_heads, int head_dim, int sm
   c.total = align256(c.acc_off + sizeof(float) * (size_t)num_seqs * num_q_heads * head_dim);
   return c;
 }
+
+// The two cascade passes over one pool pair; cx carries the pool's element format (8-bit
+// scales), the rest is filled in here.
+pa_status cascade_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
+                       const int32_t* block_tables, const int32_t* context_lens,
+                       const int32_t* prefix_lens, int num_seqs, const int32_t* chunk_members,
+                       int chunk_width, const int32_t* chunk_prefix_lens, int num_chunks,
+                       int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                       int max_blocks_per_seq, int num_blocks, float scale, pa_dtype dtype,
+                       void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                       void* stream, CascadeArgs cx) {
+  if (num_seqs < 0 || num_chunks < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+      num_q_heads % num_kv_heads || (num_chunks && chunk_width < 1))
+    return PA_ERR_INVALID;
+  if (num_seqs == 0) return PA_OK;
+  if (!prefix_lens || (num_chunks && (!chunk_members || !chunk_prefix_lens)) || !workspace ||
+      !aligned16(workspace))
+    return PA_ERR_INVALID;
+  const int sms = sm_count();
+  if (sms <= 0) return PA_ERR_CUDA;
+  const CascadeLayout cl = cascade_layout(num_seqs, num_q_heads, head_dim, sms);
+  if (workspace_bytes < cl.total) return PA_ERR_INVALID;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cx.ext_ml = reinterpret_cast<float2*>(ws + cl.ml_off);
+  cx.ext_acc = reinterpret_cast<float*>(ws + cl.acc_off);
+  const int group = num_q_heads / num_kv_heads;
+  // the prefix pass puts a chunk's members' query rows side by side (up to 64 columns on
+  // 16-bit pools, 16 on 8-bit ones); the suffix pass decodes one new token per sequence
+  // (up to 16)
+  const int prefix_cols = cx.kv8 ? pkv::kMaxGroup : pkv::kWideCols;
+  if (group > pkv::kMaxGroup || (num_chunks && (long long)group * chunk_width > prefix_cols))
+    return PA_ERR_UNSUPPORTED;
+  if (num_chunks > 0) {
+    // pass 1: each chunk's shared prefix once, its members' query rows as MMA columns
+    cx.mode = pkv::kPrefix;
+    cx.chunk_members = chunk_members;
+    cx.q_rows = num_seqs;
+    const pa_status r = decode_impl(out, q, k_cache, v_cache, block_tables, chunk_prefix_lens,
+                                    num_chunks, chunk_width, num_q_heads, num_kv_heads,
+                                    head_dim, block_size, max_blocks_per_seq, num_blocks, scale,
+                                    dtype, workspace, cl.split, 0, dev_status, stream, cx);
+    if (r != PA_OK) return r;
+  }
+  // pass 2: every sequence's own tokens, merged with its prefix partial
+  cx.mode = pkv::kSuffix;
+  cx.chunk_members = nullptr;
+  cx.seq_start = prefix_lens;
+  return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, 1,
+                     num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                     num_blocks, scale, dtype, workspace, cl.split, 0, dev_status, stream, cx);
+}
+
 
 }  // namespace
 
@@ -492,44 +561,57 @@ pa_status pa_decode_cascade(void* out, const void* q, const void* k_cache, const
                             int max_blocks_per_seq, int num_blocks, float scale, pa_dtype dtype,
                             void* workspace, size_t workspace_bytes, int32_t* dev_status,
                             void* stream) {
-  if (num_seqs < 0 || num_chunks < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
-      num_q_heads % num_kv_heads || (num_chunks && chunk_width < 1))
-    return PA_ERR_INVALID;
-  if (num_seqs == 0) return PA_OK;
-  if (!prefix_lens || (num_chunks && (!chunk_members || !chunk_prefix_lens)) || !workspace ||
-      !aligned16(workspace))
-    return PA_ERR_INVALID;
-  const int sms = sm_count();
-  if (sms <= 0) return PA_ERR_CUDA;
-  const CascadeLayout cl = cascade_layout(num_seqs, num_q_heads, head_dim, sms);
-  if (workspace_bytes < cl.total) return PA_ERR_INVALID;
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  return cascade_impl(out, q, k_cache, v_cache, block_tables, context_lens, prefix_lens,
+                      num_seqs, chunk_members, chunk_width, chunk_prefix_lens, num_chunks,
+                      num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                      num_blocks, scale, dtype, workspace, workspace_bytes, dev_status, stream,
+                      CascadeArgs());
+}
+
+pa_status pa_decode_cascade_e4m3_bs(void* out, const void* q, const void* k_cache,
+                                    const void* v_cache, const float* k_scales,
+                                    const float* v_scales, const int32_t* block_tables,
+                                    const int32_t* context_lens, const int32_t* prefix_lens,
+                                    int num_seqs, const int32_t* chunk_members, int chunk_width,
+                                    const int32_t* chunk_prefix_lens, int num_chunks,
+                                    int num_q_heads, int num_kv_heads, int head_dim,
+                                    int block_size, int max_blocks_per_seq, int num_blocks,
+                                    float scale, pa_dtype dtype, void* workspace,
+                                    size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  if (num_seqs > 0 && (!k_scales || !v_scales)) return PA_ERR_INVALID;
   CascadeArgs cx;
-  cx.ext_ml = reinterpret_cast<float2*>(ws + cl.ml_off);
-  cx.ext_acc = reinterpret_cast<float*>(ws + cl.acc_off);
-  const int group = num_q_heads / num_kv_heads;
-  // the prefix pass puts a chunk's members' query rows side by side (up to 64 columns);
-  // the suffix pass decodes one new token per sequence (up to 16)
-  if (group > pkv::kMaxGroup || (num_chunks && (long long)group * chunk_width > pkv::kWideCols))
-    return PA_ERR_UNSUPPORTED;
-  if (num_chunks > 0) {
-    // pass 1: each chunk's shared prefix once, its members' query rows as MMA columns
-    cx.mode = pkv::kPrefix;
-    cx.chunk_members = chunk_members;
-    cx.q_rows = num_seqs;
-    const pa_status r = decode_impl(out, q, k_cache, v_cache, block_tables, chunk_prefix_lens,
-                                    num_chunks, chunk_width, num_q_heads, num_kv_heads,
-                                    head_dim, block_size, max_blocks_per_seq, num_blocks, scale,
-                                    dtype, workspace, cl.split, 0, dev_status, stream, cx);
-    if (r != PA_OK) return r;
-  }
-  // pass 2: every sequence's own tokens, merged with its prefix partial
-  cx.mode = pkv::kSuffix;
-  cx.chunk_members = nullptr;
-  cx.seq_start = prefix_lens;
+  cx.kv8 = true;
+  cx.k_bscale = k_scales;
+  cx.v_bscale = v_scales;
+  return cascade_impl(out, q, k_cache, v_cache, block_tables, context_lens, prefix_lens,
+                      num_seqs, chunk_members, chunk_width, chunk_prefix_lens, num_chunks,
+                      num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                      num_blocks, scale, dtype, workspace, workspace_bytes, dev_status, stream,
+                      cx);
+}
+
+pa_status pa_decode_append_e4m3_bs(void* out, const void* q, void* k_cache, void* v_cache,
+                                   float* k_scales, float* v_scales, const void* k_new,
+                                   const void* v_new, const int32_t* block_tables,
+                                   const int32_t* context_lens, int num_seqs, int num_q_heads,
+                                   int num_kv_heads, int head_dim, int block_size,
+                                   int max_blocks_per_seq, int num_blocks, float scale,
+                                   pa_dtype dtype, void* workspace, size_t workspace_bytes,
+                                   int32_t* dev_status, void* stream) {
+  if (num_seqs > 0 && (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new) ||
+                       !k_scales || !v_scales))
+    return PA_ERR_INVALID;
+  CascadeArgs cx;
+  cx.mode = pkv::kAppend;
+  cx.k_new = k_new;
+  cx.v_new = v_new;
+  cx.kv8 = true;
+  cx.k_bscale = k_scales;
+  cx.v_bscale = v_scales;
   return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, 1,
                      num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
-                     num_blocks, scale, dtype, workspace, cl.split, 0, dev_status, stream, cx);
+                     num_blocks, scale, dtype, workspace, workspace_bytes, 0, dev_status, stream,
+                     cx);
 }
 
 pa_status pa_cache_append(void* k_cache, void* v_cache, const void* k, const void* v,
@@ -669,12 +751,16 @@ pa_status pa_swap_in_blocks(void* const* k_caches, void* const* v_caches, int nu
 namespace {
 
 constexpr size_t kNoallocScratchBytes = PA_NOALLOC_SCRATCH_BYTES;
-// split CTAs the scratch is sized for: 3 per SM on a 148-SM B200, the most pa_decode runs
-// there (block_size <= 8); a GPU with more SMs runs at most this many
+// split CTAs the scratch is sized for: 3 mma.sync CTAs per SM on a 148-SM B200, the most
+// pa_decode runs there (block_size <= 8), or one tcgen05 CTA per SM; a GPU with more SMs
+// runs at most this many
 constexpr int kNoallocMaxGrid = 444;
 constexpr int kNoallocMaxDevices = 64;
 static_assert(ws_layout(128, kNoallocMaxGrid, pkv::kMaxGroup).total <= kNoallocScratchBytes,
               "the scratch must hold the split partials of kNoallocMaxGrid CTAs at head_dim 128");
+static_assert(ws_layout(128, kNoallocMaxGrid / pkv::kMaxCtasPerSm, pkv::kWideCols).total <=
+                  kNoallocScratchBytes,
+              "and those of the tcgen05 kernel's CTAs (one a SM, 64 query columns)");
 
 // Lives in the module's global memory: every device that loads the library holds it
 // until the process exits.  Host code must not pass its name to a kernel (on the host

@@ -160,7 +160,7 @@ struct Layout {
   static constexpr int kMlOff = kDescOff + 2 * (int)sizeof(SplitDesc);
   // fused append: per stage the new token's K and V rows, staged by the producer
   static constexpr int kNewOff = (kMlOff + kConsumerWarps * kMaxGroup * 8 + 15) / 16 * 16;
-  static constexpr int kNewBytes = KV8 ? 16 : 2 * D * 2;
+  static constexpr int kNewBytes = 2 * D * 2;         // the new token's 16-bit K and V rows
   // 8-bit caches with per-(block, kv head) scales: per stage the K and V scale of every
   // token row, staged by the producer
   static constexpr int kScOff = kNewOff + kStages * kNewBytes;
@@ -462,7 +462,9 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
   using L = Layout<D, KV8, ctas_per_sm(KV8, NT, BS)>;
   constexpr int kStages = L::kStages;
   constexpr int kSegW = seg_weight(BS);
-  static_assert(!KV8 || (D == 128 && MODE == kPlain), "8-bit caches: head_dim 128, plain decode");
+  static_assert(!KV8 || D == 128, "8-bit caches: head_dim 128");
+  static_assert(!KV8 || MODE == kPlain || KSC,
+                "8-bit caches: the cascade and fused-append modes use per-block scales");
   static_assert(!KSC || KV8, "per-block scales belong to 8-bit caches");
   // MMA operand type: the cache's 16-bit type, or fp16 for E4M3 (exact there)
   constexpr bool kBF16 = !KV8 && std::is_same_v<T, __nv_bfloat16>;
@@ -979,7 +981,60 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
         // causal limit: new token j sees unit rows < ctx - q_len + 1 + j - t0 (a prefix
         // launch's columns are different sequences: no mask)
         const int lim0 = MODE == kPrefix ? (1 << 30) : mt.ctx - a.q_len + 1 - t0;
-        if (MODE == kAppend && mt.newrow >= 0 && (mt.ctx - 1 - mt.tok0) / kUnit == u) {
+        if (MODE == kAppend && KV8 && mt.newrow >= 0 && (mt.ctx - 1 - mt.tok0) / kUnit == u) {
+          // fused append into 8-bit pools with per-(block, kv head) scales: lanes 0..7
+          // quantise the new K row, 8..15 the V row, 16 values (one 16-byte chunk of codes)
+          // each, exactly as the block-scaled append does; a token at offset 0 of its block
+          // first fixes the block's scale from its own row.  The codes go into the tile row
+          // and the cache row, the scale into the stage's scale row and, for offset 0, the
+          // scale array.  With split columns both warps compute the same bytes; the first
+          // writes global memory.
+          const int rn = mt.ctx - 1 - mt.tok0;          // row in the stage tile
+          const int kv = (lane >> 3) & 1, ch = lane & 7;
+          const bool act = lane < 16;
+          const uint4* src = reinterpret_cast<const uint4*>(smem + L::kNewOff + st * L::kNewBytes +
+                                                            kv * D * 2 + ch * 32);
+          uint4 in[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+          if (act) {
+            in[0] = src[0];
+            in[1] = src[1];
+          }
+          const uint32_t* w = reinterpret_cast<const uint32_t*>(in);
+          float x[16];
+          float am = 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float2 f = unpack2<T>(w[e]);
+            x[2 * e] = f.x;
+            x[2 * e + 1] = f.y;
+            am = fmaxf(am, fmaxf(fabsf(f.x), fabsf(f.y)));
+          }
+          am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+          am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
+          am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 4));
+          float* scs = reinterpret_cast<float*>(smem + L::kScOff + st * L::kScBytes) + kv * kTileTokens;
+          const bool fresh = mt.newrow % BS == 0;       // offset 0: this token fixes the scale
+          const float sc = fresh ? e4m3_block_scale(am) : scs[rn];
+          __syncwarp();
+          if (act) {
+            uint32_t q[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              q[e] = f32x2_to_e4m3x2(__fdiv_rn(x[4 * e], sc), __fdiv_rn(x[4 * e + 1], sc)) |
+                     (f32x2_to_e4m3x2(__fdiv_rn(x[4 * e + 2], sc), __fdiv_rn(x[4 * e + 3], sc)) << 16);
+            const uint4 codes = make_uint4(q[0], q[1], q[2], q[3]);
+            *reinterpret_cast<uint4*>((kv ? sV : sK) + rn * 128 + ((ch ^ (rn & 7)) << 4)) = codes;
+            if (ch == 0 && fresh) scs[rn] = sc;
+            if (nb == 0) {
+              uint8_t* cache = static_cast<uint8_t*>(const_cast<void*>(kv ? a.v_cache : a.k_cache));
+              *reinterpret_cast<uint4*>(cache + (long long)mt.newrow * D + ch * 16) = codes;
+              if (ch == 0 && fresh)
+                const_cast<float*>(kv ? a.v_bscale : a.k_bscale)[mt.newrow / BS] = sc;
+            }
+          }
+          __syncwarp();
+          patched = true;
+        } else if (MODE == kAppend && !KV8 && mt.newrow >= 0 && (mt.ctx - 1 - mt.tok0) / kUnit == u) {
           // fused append: this unit holds the newest token; its K/V rows come from the
           // staging area (the cache row the TMA read may still be old) and are written to
           // the cache.  With split columns both warps of the unit patch their tile copy
@@ -1050,8 +1105,10 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
           const int r0 = u * kUnit + gid;
           sl_lo = a.scale_log2 * sc[r0];
           sl_hi = a.scale_log2 * sc[r0 + 8];
-          vs_lo = sc[kTileTokens + r0];
-          vs_hi = sc[kTileTokens + r0 + 8];
+          // a row past the valid tokens has p = 0; its scale may be that of a block whose
+          // offset 0 was never written (anything, NaN included), so it must not reach P
+          vs_lo = gid < valid ? sc[kTileTokens + r0] : 0.f;
+          vs_hi = gid + 8 < valid ? sc[kTileTokens + r0 + 8] : 0.f;
         }
         uint32_t bhi[NTW][2], blo[NTW][2];
 #pragma unroll

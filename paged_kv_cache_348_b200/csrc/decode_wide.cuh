@@ -54,7 +54,9 @@ __host__ __device__ constexpr int wide_threads(int nc) { return 64 + wide_soft_t
 constexpr uint32_t kWideTmemCols = 512;
 constexpr uint32_t kOCol = 256;
 constexpr float kRescaleLog2 = 8.f;               // a reference max moves past this gap only
-constexpr int kWideSegWeight = 40;                // see pa_decode_wide_kernel
+// see pa_decode_wide_kernel: a portion's fixed cost grows with its query columns (the
+// epilogue's row sums and output writes)
+__host__ __device__ constexpr int wide_seg_weight(int nc) { return nc <= 16 ? 32 : (nc <= 32 ? 40 : 56); }
 
 // K and V tiles: token row r, 64-dim half h (128 bytes, 128-byte swizzle) at
 // ((r / 8) * kHalves + h) * 1024 + (r % 8) * 128: 8-row atoms with the halves side by side,
@@ -179,7 +181,8 @@ __global__ void __launch_bounds__(wide_threads(NC), 1)
     pa_decode_wide_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
                           const __grid_constant__ CUtensorMap tmv) {
   using L = WideLayout<D>;
-  static_assert(MODE == kPlain || MODE == kPrefix, "wide decode: plain (multi-token) or prefix");
+  static_assert(MODE == kPlain || MODE == kPrefix || MODE == kAppend,
+                "wide decode: plain (multi-token), prefix or fused append");
   static_assert(NC == 16 || NC == 32 || NC == 64, "16, 32 or 64 query columns");
   constexpr int kWideSoftThreads = wide_soft_threads(NC);
   constexpr int CW = NC / wide_swg(NC);             // columns of one softmax warpgroup
@@ -191,7 +194,7 @@ __global__ void __launch_bounds__(wide_threads(NC), 1)
   // with its reference-max pass and Q load, end-of-portion epilogue) is worth about this
   // many 16-token units of streaming, several stages' worth (measured per CTA with
   // global-timer stamps), far more than in the mma.sync kernel
-  constexpr int kSegW = kWideSegWeight;
+  constexpr int kSegW = wide_seg_weight(NC);
   constexpr uint32_t kAB = std::is_same_v<T, __nv_bfloat16> ? 1u : 0u;
   constexpr int kFullCount = 33;       // lane 0's expect_tx arrival + 32 cp.async arrivals
   extern __shared__ uint8_t smem_raw[];
@@ -376,6 +379,30 @@ __global__ void __launch_bounds__(wide_threads(NC), 1)
                             (complete ? F_COMPLETE : 0);
           uint8_t* sK = smem + st * L::kStageBytes;
           uint8_t* sV = sK + L::kKvBytes;
+          if constexpr (MODE == kAppend) {
+            // fused append: the stage holding the newest token (position ctx-1) first
+            // writes that token's K/V rows (k_new, v_new) to its cache rows, then reads the
+            // tile, so the tile holds the new rows.  The stage is this segment's only reader
+            // of that row.  Each writing lane fences its stores against the async proxy
+            // before the warp issues the tile's TMA loads (an out-of-range block id is
+            // flagged by the tile's own table lookups and the row is not written).
+            const int tn = ctx_cur - 1;
+            if (tn >= tok0 && tn < tok0 + nun * kUnit) {   // warp-uniform
+              constexpr int CPR = D * 2 / 16;              // 16-byte chunks per row
+              const int blk = __ldg(trow + tn / BS);
+              if ((unsigned)blk < (unsigned)a.num_blocks && lane < 2 * CPR) {
+                const int kv = lane / CPR, ch = lane % CPR;
+                const long long src = ((long long)s_cur * Hkv + kvh) * D;
+                const long long row = ((long long)blk * Hkv + kvh) * BS + tn % BS;
+                const T* nrow = static_cast<const T*>(kv ? a.v_new : a.k_new) + src;
+                const uint4 val = __ldg(reinterpret_cast<const uint4*>(nrow) + ch);
+                T* cache = static_cast<T*>(const_cast<void*>(kv ? a.v_cache : a.k_cache));
+                reinterpret_cast<uint4*>(cache + row * D)[ch] = val;
+                fence_proxy_async_global();
+              }
+              __syncwarp();
+            }
+          }
           if constexpr (BS != 1) {
             constexpr int H = BS < 16 ? BS : 16;     // rows per TMA box (all column halves)
             constexpr int BPU = kUnit / H;           // boxes per unit

@@ -80,31 +80,33 @@ pa_status dispatch_d(int d, int bs, const pkv::DecodeArgs& a, const CUtensorMap&
                  : dispatch_bs<T, 128, MODE>(bs, a, mk, mv, grid, s);
 }
 
-// 8-bit (E4M3) caches: plain decode (one or several new tokens), head_dim 128; KSC: per-
-// (block, kv head) scales instead of one per pool.
-template <typename T, bool KSC = false>
+// 8-bit (E4M3) caches, head_dim 128: plain decode (one or several new tokens) with one
+// scale per pool or, KSC, per-(block, kv head) scales; the cascade passes and the fused
+// append with per-(block, kv head) scales.
+template <typename T, bool KSC = false, int MODE = pkv::kPlain>
 pa_status dispatch_e4m3(int bs, const pkv::DecodeArgs& a, const CUtensorMap& mk,
                         const CUtensorMap& mv, int grid, cudaStream_t s) {
   const bool nt1 = a.ncol <= 8;
   switch (bs) {
-    case 1: return nt1 ? launch_decode<T, 128, 1, 1, pkv::kPlain, true, KSC>(a, mk, mv, grid, s)
-                       : launch_decode<T, 128, 1, 2, pkv::kPlain, true, KSC>(a, mk, mv, grid, s);
-    case 8: return nt1 ? launch_decode<T, 128, 8, 1, pkv::kPlain, true, KSC>(a, mk, mv, grid, s)
-                       : launch_decode<T, 128, 8, 2, pkv::kPlain, true, KSC>(a, mk, mv, grid, s);
-    case 16: return nt1 ? launch_decode<T, 128, 16, 1, pkv::kPlain, true, KSC>(a, mk, mv, grid, s)
-                        : launch_decode<T, 128, 16, 2, pkv::kPlain, true, KSC>(a, mk, mv, grid, s);
-    case 32: return nt1 ? launch_decode<T, 128, 32, 1, pkv::kPlain, true, KSC>(a, mk, mv, grid, s)
-                        : launch_decode<T, 128, 32, 2, pkv::kPlain, true, KSC>(a, mk, mv, grid, s);
+    case 1: return nt1 ? launch_decode<T, 128, 1, 1, MODE, true, KSC>(a, mk, mv, grid, s)
+                       : launch_decode<T, 128, 1, 2, MODE, true, KSC>(a, mk, mv, grid, s);
+    case 8: return nt1 ? launch_decode<T, 128, 8, 1, MODE, true, KSC>(a, mk, mv, grid, s)
+                       : launch_decode<T, 128, 8, 2, MODE, true, KSC>(a, mk, mv, grid, s);
+    case 16: return nt1 ? launch_decode<T, 128, 16, 1, MODE, true, KSC>(a, mk, mv, grid, s)
+                        : launch_decode<T, 128, 16, 2, MODE, true, KSC>(a, mk, mv, grid, s);
+    case 32: return nt1 ? launch_decode<T, 128, 32, 1, MODE, true, KSC>(a, mk, mv, grid, s)
+                        : launch_decode<T, 128, 32, 2, MODE, true, KSC>(a, mk, mv, grid, s);
   }
   return PA_ERR_UNSUPPORTED;
 }
 
-// The block-scaled 8-bit instances; defined in decode_e4m3_bs.cu.
+// The block-scaled 8-bit plain-decode instances; defined in decode_e4m3_bs.cu.
 pa_status run_e4m3_bs(bool bf16, int bs, const pkv::DecodeArgs& a, const CUtensorMap& mk,
                       const CUtensorMap& mv, int grid, cudaStream_t s);
 
 // One kernel mode's instances, dispatched on the other parameters; defined in
-// decode_<mode>.cu.  kv8: 8-bit E4M3 pools (kPlain only).
+// decode_<mode>.cu.  kv8: 8-bit E4M3 pools (decode_e4m3*.cu; every mode but kPlain needs
+// per-(block, kv head) scales).
 template <int MODE, bool KV8>
 pa_status run_decode_mode(bool bf16, int d, int bs, const pkv::DecodeArgs& a,
                           const CUtensorMap& mk, const CUtensorMap& mv, int grid, cudaStream_t s);
@@ -118,9 +120,12 @@ PKV_DECL_RUN(pkv::kPrefix, false)
 PKV_DECL_RUN(pkv::kSuffix, false)
 PKV_DECL_RUN(pkv::kAppend, false)
 PKV_DECL_RUN(pkv::kPlain, true)
+PKV_DECL_RUN(pkv::kPrefix, true)
+PKV_DECL_RUN(pkv::kSuffix, true)
+PKV_DECL_RUN(pkv::kAppend, true)
 #undef PKV_DECL_RUN
 
-// ---- the tcgen05 kernel for 17..64 query rows per kv head (decode_wide.cuh); NC = the
+// ---- the tcgen05 kernel for 9..64 query rows per kv head (decode_wide.cuh); NC = the
 // query rows rounded up to 16, 32 or 64
 template <typename T, int D, int BS, int MODE, int NC>
 pa_status launch_wide(const pkv::DecodeArgs& a, const CUtensorMap& mk, const CUtensorMap& mv,
@@ -172,6 +177,9 @@ PKV_DECL_WIDE(pkv::kPlain, 64)
 PKV_DECL_WIDE(pkv::kPrefix, 16)
 PKV_DECL_WIDE(pkv::kPrefix, 32)
 PKV_DECL_WIDE(pkv::kPrefix, 64)
+PKV_DECL_WIDE(pkv::kAppend, 16)
+PKV_DECL_WIDE(pkv::kAppend, 32)
+PKV_DECL_WIDE(pkv::kAppend, 64)
 #undef PKV_DECL_WIDE
 
 }  // namespace pkv_host

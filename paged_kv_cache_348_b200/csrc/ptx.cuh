@@ -116,6 +116,12 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// orders this thread's earlier generic-proxy global writes before later async-proxy (TMA)
+// reads of global memory
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
@@ -271,6 +277,40 @@ __device__ __forceinline__ bool bar_red_or(int id, int nthreads, bool pred) {
       : "r"(id), "r"(nthreads), "r"((uint32_t)pred)
       : "memory");
   return r != 0;
+}
+
+// ---------------------------------------------------------------- 8-bit (E4M3) codes
+// Two binary32 values to two E4M3 codes (x0 in the low byte): round to nearest even,
+// magnitudes above 448 clamped to 448.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float x0, float x1) {
+  uint32_t d;
+  asm("{\n\t.reg .b16 t;\n\tcvt.rn.satfinite.e4m3x2.f32 t, %2, %1;\n\tcvt.u32.u16 %0, t;\n\t}"
+      : "=r"(d)
+      : "f"(x0), "f"(x1));
+  return d;
+}
+
+// Scale of a (block, kv head) slice of an 8-bit cache, fixed by the block's offset-0 token
+// ("PagedAttention -- The KV Cache Problem", "What's Still Unsolved": FP8 quantised KV
+// cache): the power of two s with s/16 < amax/448 <= s/8, i.e. 2^(ceil(log2 y) + 3) with
+// y = amax / 448 in binary32; 1 for a zero (or non-finite) amax.  ceil(log2 y) comes from
+// y's bits: a power of two gives its exponent, anything else one more.
+__device__ __forceinline__ float e4m3_block_scale(float amax) {
+  const float y = __fdiv_rn(amax, 448.f);
+  if (!(y > 0.f) || isinf(y)) return 1.f;
+  const uint32_t u = __float_as_uint(y);
+  const int ex = (int)((u >> 23) & 0xffu);
+  const uint32_t man = u & 0x7fffffu;
+  int c;
+  if (ex == 0) {                                  // subnormal: y = man * 2^-149
+    const int p = 31 - __clz(man);
+    c = man == (1u << p) ? p - 149 : p - 148;
+  } else {
+    c = ex - 127 + (man ? 1 : 0);
+  }
+  c += 3;
+  c = c < -126 ? -126 : (c > 127 ? 127 : c);
+  return __uint_as_float((uint32_t)(c + 127) << 23);
 }
 
 // ---------------------------------------------------------------- programmatic dependent launch

@@ -33,7 +33,7 @@ EXPORTS = ("pa_version", "pa_status_string", "pa_decode_workspace_bytes", "pa_de
            "pa_bm_context_len", "pa_bm_num_blocks_of", "pa_bm_max_blocks", "pa_bm_block_tables",
            "pa_bm_slot_of", "pa_bm_plan_cascade", "pa_plan_cascade", "pa_bm_swap_out",
            "pa_bm_swap_in", "pa_swap_out_blocks", "pa_swap_in_blocks", "pa_cache_append_e4m3_bs",
-           "pa_decode_e4m3_bs")
+           "pa_decode_e4m3_bs", "pa_decode_cascade_e4m3_bs", "pa_decode_append_e4m3_bs")
 
 _lib = None
 _lock = threading.Lock()
@@ -81,6 +81,13 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         L.pa_decode_e4m3_bs.restype = i32
         L.pa_decode_e4m3_bs.argtypes = [P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32,
                                         i32, f32, i32, P, sz, P, P]
+        L.pa_decode_cascade_e4m3_bs.restype = i32
+        L.pa_decode_cascade_e4m3_bs.argtypes = [P, P, P, P, P, P, P, P, P, i32, P, i32, P, i32,
+                                                i32, i32, i32, i32, i32, i32, f32, i32, P, sz, P,
+                                                P]
+        L.pa_decode_append_e4m3_bs.restype = i32
+        L.pa_decode_append_e4m3_bs.argtypes = [P, P, P, P, P, P, P, P, P, P, i32, i32, i32, i32,
+                                               i32, i32, i32, f32, i32, P, sz, P, P]
         L.pa_decode_cascade_workspace_bytes.restype = sz
         L.pa_decode_cascade_workspace_bytes.argtypes = [i32, i32, i32, i32]
         L.pa_decode_cascade.restype = i32
@@ -342,7 +349,7 @@ def pa_decode_cascade(out, q, k_cache, v_cache, block_tables, context_lens, pref
                       stream=None):
     """out[B,Hq,D] <- paged decode where chunks of sequences share a KV prefix (see
     pa_decode_cascade in include/pagedkv.h).  chunk_members is int32 [C, W] (-1 pad,
-    group * W <= 16), chunk_prefix_lens int32 [C], prefix_lens int32 [B]."""
+    group * W <= 64), chunk_prefix_lens int32 [C], prefix_lens int32 [B]."""
     _need(q, "q", ndim=3)
     _need(out, "out", dtype=q.dtype, ndim=3)
     _need(k_cache, "k_cache", dtype=q.dtype, ndim=4)
@@ -368,6 +375,74 @@ def pa_decode_cascade(out, q, k_cache, v_cache, block_tables, context_lens, pref
                                   _ptr(workspace), workspace.numel() * workspace.element_size(),
                                   _ptr(status), _stream(stream))
     _check(rc, "pa_decode_cascade")
+    return out
+
+
+def pa_decode_cascade_e4m3_bs(out, q, k_cache8, v_cache8, k_scales, v_scales, block_tables,
+                              context_lens, prefix_lens, chunk_members, chunk_prefix_lens,
+                              scale: float, workspace, status=None, stream=None):
+    """pa_decode_cascade over uint8 E4M3 pools with per-(block, kv head) scales (float32
+    [N,Hkv]); group * W <= 16 (see pa_decode_cascade_e4m3_bs in include/pagedkv.h)."""
+    _need(q, "q", ndim=3)
+    _need(out, "out", dtype=q.dtype, ndim=3)
+    _need(k_cache8, "k_cache", dtype=torch.uint8, ndim=4)
+    _need(v_cache8, "v_cache", dtype=torch.uint8, ndim=4)
+    _need(k_scales, "k_scales", dtype=torch.float32, ndim=2)
+    _need(v_scales, "v_scales", dtype=torch.float32, ndim=2)
+    _need(block_tables, "block_tables", dtype=torch.int32, ndim=2)
+    _need(context_lens, "context_lens", dtype=torch.int32, ndim=1)
+    _need(prefix_lens, "prefix_lens", dtype=torch.int32, ndim=1)
+    _need(chunk_members, "chunk_members", dtype=torch.int32, ndim=2)
+    _need(chunk_prefix_lens, "chunk_prefix_lens", dtype=torch.int32, ndim=1)
+    _need(workspace, "workspace")
+    B, Hq, D = q.shape
+    N, Hkv, bs, D2 = k_cache8.shape
+    C = chunk_members.shape[0]
+    if out.shape != q.shape or D2 != D or v_cache8.shape != k_cache8.shape or \
+            block_tables.shape[0] != B or context_lens.shape[0] != B or \
+            prefix_lens.shape[0] != B or chunk_prefix_lens.shape[0] != C or \
+            k_scales.shape != (N, Hkv) or v_scales.shape != (N, Hkv):
+        raise PagedKVError("pa_decode_cascade_e4m3_bs: inconsistent shapes")
+    rc = load().pa_decode_cascade_e4m3_bs(
+        _ptr(out), _ptr(q), _ptr(k_cache8), _ptr(v_cache8), _ptr(k_scales), _ptr(v_scales),
+        _ptr(block_tables), _ptr(context_lens), _ptr(prefix_lens), B, _ptr(chunk_members),
+        chunk_members.shape[1], _ptr(chunk_prefix_lens), C, Hq, Hkv, D, bs,
+        block_tables.shape[1], N, float(scale), _dtype_code(q), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(status), _stream(stream))
+    _check(rc, "pa_decode_cascade_e4m3_bs")
+    return out
+
+
+def pa_decode_append_e4m3_bs(out, q, k_cache8, v_cache8, k_scales, v_scales, k_new, v_new,
+                             block_tables, context_lens, scale: float, workspace, status=None,
+                             stream=None):
+    """Quantise each sequence's newest token (16-bit k_new/v_new [B,Hkv,D], position
+    context_lens-1) into uint8 E4M3 pools with per-(block, kv head) scales and decode, in
+    one launch (see pa_decode_append_e4m3_bs in include/pagedkv.h)."""
+    _need(q, "q", ndim=3)
+    _need(out, "out", dtype=q.dtype, ndim=3)
+    _need(k_cache8, "k_cache", dtype=torch.uint8, ndim=4)
+    _need(v_cache8, "v_cache", dtype=torch.uint8, ndim=4)
+    _need(k_scales, "k_scales", dtype=torch.float32, ndim=2)
+    _need(v_scales, "v_scales", dtype=torch.float32, ndim=2)
+    _need(k_new, "k_new", dtype=q.dtype, ndim=3)
+    _need(v_new, "v_new", dtype=q.dtype, ndim=3)
+    _need(block_tables, "block_tables", dtype=torch.int32, ndim=2)
+    _need(context_lens, "context_lens", dtype=torch.int32, ndim=1)
+    _need(workspace, "workspace")
+    B, Hq, D = q.shape
+    N, Hkv, bs, D2 = k_cache8.shape
+    if out.shape != q.shape or D2 != D or v_cache8.shape != k_cache8.shape or \
+            k_new.shape != (B, Hkv, D) or v_new.shape != k_new.shape or \
+            block_tables.shape[0] != B or context_lens.shape[0] != B or \
+            k_scales.shape != (N, Hkv) or v_scales.shape != (N, Hkv):
+        raise PagedKVError("pa_decode_append_e4m3_bs: inconsistent shapes")
+    rc = load().pa_decode_append_e4m3_bs(
+        _ptr(out), _ptr(q), _ptr(k_cache8), _ptr(v_cache8), _ptr(k_scales), _ptr(v_scales),
+        _ptr(k_new), _ptr(v_new), _ptr(block_tables), _ptr(context_lens), B, Hq, Hkv, D, bs,
+        block_tables.shape[1], N, float(scale), _dtype_code(q), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(status), _stream(stream))
+    _check(rc, "pa_decode_append_e4m3_bs")
     return out
 
 

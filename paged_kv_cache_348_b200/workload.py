@@ -215,12 +215,13 @@ def build_prefix_fork(w: inputs.Workload = inputs.PREFIX, device="cuda") -> Deco
 
 def run_step(b: DecodeBatch, stream=None, layers=None, fused: bool = False) -> None:
     """One decode step over all layers (see module docstring).  With fused=True each
-    layer is one pa_decode_append call (the newest token's append fused into decode;
-    one new token per sequence, no cascade)."""
+    layer is one pa_decode_append (pa_decode_append_e4m3_bs over block-scaled 8-bit pools)
+    call: the newest token's append fused into decode; one new token per sequence, no
+    cascade."""
     if b.cow_pairs is not None and b.cow_pairs.shape[0]:
         pk.pa_copy_blocks(b.k_caches, b.v_caches, b.cow_pairs, b.status, stream)
     for l in range(layers if layers is not None else b.layers):
-        if fused and b.kv_scales is None and b.kv_bscales is None:
+        if fused and b.kv_scales is None:
             append_decode_layer(b, l, stream)
             continue
         if b.kv_bscales is not None:
@@ -239,6 +240,13 @@ def append_decode_layer(b: DecodeBatch, l: int, stream=None, block_tables=None,
                         context_lens=None) -> None:
     """pa_decode_append of layer l: append the newest token of every sequence and decode."""
     assert b.q_len == 1 and b.cascade is None
+    if b.kv_bscales is not None:
+        pk.pa_decode_append_e4m3_bs(b.out[l], b.q[l], b.k_caches[l], b.v_caches[l],
+                                    *b.kv_bscales[l], b.k_new[l], b.v_new[l],
+                                    b.block_tables if block_tables is None else block_tables,
+                                    b.context_lens if context_lens is None else context_lens,
+                                    b.scale, b.workspace, b.status, stream)
+        return
     pk.pa_decode_append(b.out[l], b.q[l], b.k_caches[l], b.v_caches[l], b.k_new[l], b.v_new[l],
                         b.block_tables if block_tables is None else block_tables,
                         b.context_lens if context_lens is None else context_lens, b.scale,
@@ -246,10 +254,13 @@ def append_decode_layer(b: DecodeBatch, l: int, stream=None, block_tables=None,
 
 
 def use_cascade(b: DecodeBatch, width: int | None = None) -> DecodeBatch:
-    """Decode this batch with pa_decode_cascade: plan the shared-prefix chunks from its
-    block tables (the workspace grows to the cascade size)."""
+    """Decode this batch with pa_decode_cascade (pa_decode_cascade_e4m3_bs over block-scaled
+    8-bit pools, whose chunks hold up to 16 query rows): plan the shared-prefix chunks from
+    its block tables (the workspace grows to the cascade size)."""
     w = b.w
     ctx = b.context_lens.cpu().numpy()
+    if width is None and b.kv_bscales is not None:
+        width = max(1, 16 // (w.num_q_heads // w.num_kv_heads))
     prefix, members, plens = b.bm.plan_cascade(b.sids, w.num_q_heads // w.num_kv_heads, width)
     dev = b.block_tables.device
     b.cascade = (torch.from_numpy(prefix).to(dev), torch.from_numpy(members).to(dev),
@@ -262,6 +273,11 @@ def use_cascade(b: DecodeBatch, width: int | None = None) -> DecodeBatch:
 def decode_layer(b: DecodeBatch, l: int, stream=None) -> None:
     """pa_decode (one new token per sequence), pa_decode_multi (q_len > 1) or
     pa_decode_cascade (after use_cascade) of layer l."""
+    if b.cascade is not None and b.kv_bscales is not None:
+        pk.pa_decode_cascade_e4m3_bs(b.out[l], b.q[l], b.k_caches[l], b.v_caches[l],
+                                     *b.kv_bscales[l], b.block_tables, b.context_lens,
+                                     *b.cascade, b.scale, b.workspace, b.status, stream)
+        return
     if b.cascade is not None:
         pk.pa_decode_cascade(b.out[l], b.q[l], b.k_caches[l], b.v_caches[l], b.block_tables,
                              b.context_lens, *b.cascade, b.scale, b.workspace, b.status, stream)

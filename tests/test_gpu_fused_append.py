@@ -52,7 +52,10 @@ def _run_both(case, seed):
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
 @pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("bs", [1, 8, 16, 32])
-@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (32, 8), (64, 8), (16, 1)])
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (32, 8), (64, 8), (16, 1),
+                                    # 9+ query rows a kv head: the tcgen05 kernel, which
+                                    # writes the new rows before reading their tile
+                                    (12, 1), (32, 1), (64, 1)])
 def test_fused_append_equals_append_then_decode(dtype, D, bs, Hq, Hkv):
     case = make_case(len(CTX_MIX), Hq, Hkv, D, bs, CTX_MIX, dtype=dtype,
                      seed=500 + D + bs + Hq)

@@ -37,9 +37,13 @@ def _close(a: torch.Tensor, b: torch.Tensor):
 def test_noalloc_matches_workspace_entry_point_on_consecutive_calls():
     # two different batches back to back: long contexts so segments are split over CTAs
     # and the shared scratch holds partials; the second call sees the first's leftovers.
+    # The third and fourth have 16 and 64 query rows per kv head: the tcgen05 kernel, whose
+    # partials hold 64 rows per CTA.
     cases = [make_case(6, 64, 8, 128, 16, [7000, 5, 3000, 9100, 64, 4100], dtype="bf16", seed=81),
              make_case(9, 32, 8, 128, 8, [1, 2500, 700, 16, 8000, 333, 0, 4097, 60],
-                       dtype="f16", seed=82)]
+                       dtype="f16", seed=82),
+             make_case(5, 128, 8, 128, 16, [9000, 3, 4500, 8191, 600], dtype="bf16", seed=84),
+             make_case(4, 64, 1, 128, 32, [6000, 12000, 1, 2049], dtype="f16", seed=85)]
     st = pk.new_status()
     for case in cases:
         q, k, v, tables, ctx = _upload(case)
