@@ -234,6 +234,13 @@ pa_status decode_impl(void* out, const void* q, const void* k_cache, const void*
   // 8-bit pools: head_dim 128; the cascade and fused-append modes need per-block scales
   if (cx.kv8 && (head_dim != 128 || (cx.mode != pkv::kPlain && !cx.k_bscale)))
     return PA_ERR_UNSUPPORTED;
+  if (block_size == 1) {
+    // both kernels gather block_size-1 rows four at a time: one-row boxes
+    const uint64_t rows = (uint64_t)num_blocks * num_kv_heads;
+    if (!encode_pool(&mk, k_cache, dtype, head_dim, rows, 1, cx.kv8) ||
+        !encode_pool(&mv, v_cache, dtype, head_dim, rows, 1, cx.kv8))
+      return PA_ERR_CUDA;
+  }
   if (block_size != 1) {
     const uint64_t rows = (uint64_t)num_blocks * num_kv_heads * block_size;
     const int box_rows = block_size < 16 ? block_size : 16;

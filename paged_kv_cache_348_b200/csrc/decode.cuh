@@ -468,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
   static_assert(!KSC || KV8, "per-block scales belong to 8-bit caches");
   // MMA operand type: the cache's 16-bit type, or fp16 for E4M3 (exact there)
   constexpr bool kBF16 = !KV8 && std::is_same_v<T, __nv_bfloat16>;
-  constexpr int kFullCount = (BS == 1) ? 33 : 1;
+  constexpr int kFullCount = 1;        // the producer's expect_tx arrival
   constexpr int kConsumerThreads = 32 * kConsumerWarps;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -492,7 +492,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
     *last_flag = 0;
     fence_mbar_init();
   }
-  if (BS != 1 && threadIdx.x == 32) {
+  if (threadIdx.x == 32) {
     prefetch_tensormap(&tmk);
     prefetch_tensormap(&tmv);
   }
@@ -595,6 +595,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
       // head (whose segment starts at the same token), so only a CTA's first portion of a
       // sequence waits on table reads
       int s_win = -1, sw0 = 0, sw1 = 0, sn0 = 0, sn1 = 0;
+      int sm0 = 0, sm1 = 0, sp0 = 0, sp1 = 0;         // block_size 1: the deeper windows
       const int32_t* s_trow = a.block_tables;
       long long pbase = pb_a;
       while (ok && x < xend) {
@@ -630,17 +631,25 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
         }
         // Block-table window: lane l holds entries wb+l, wb+32+l (w0, w1) and the next 64
         // entries (n0, n1), loaded 64 blocks before they are needed, so no stage waits on a
-        // table read except the portion's first.
+        // table read except the portion's first.  With block_size 1 a stage uses a whole
+        // window of 64 entries, so two more windows (m, p) are kept: every entry is loaded
+        // three stages before its stage, which hides a table read that misses L2.
         const int nblk = (ctx_cur + BS - 1) / BS;
         int wb = (first_cur + (int)(x - seg0) * kUnit) / BS;
         const int32_t* trow;
-        int w0, w1, n0, n1;
+        int w0, w1, n0, n1, m0 = -1, m1 = -1, p0 = -1, p1 = -1;
         if (x == seg0 && s_cur == s_win) {            // warp-uniform
           trow = s_trow;
           w0 = sw0;
           w1 = sw1;
           n0 = sn0;
           n1 = sn1;
+          if constexpr (BS == 1) {
+            m0 = sm0;
+            m1 = sm1;
+            p0 = sp0;
+            p1 = sp1;
+          }
         } else {
           // a chunk of a prefix launch reads the prefix through its first member's table
           const long long trow_seq =
@@ -650,6 +659,12 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
           w1 = wb + 32 + lane < nblk ? trow[wb + 32 + lane] : -1;
           n0 = wb + 64 + lane < nblk ? trow[wb + 64 + lane] : -1;
           n1 = wb + 96 + lane < nblk ? trow[wb + 96 + lane] : -1;
+          if constexpr (BS == 1) {
+            m0 = wb + 128 + lane < nblk ? trow[wb + 128 + lane] : -1;
+            m1 = wb + 160 + lane < nblk ? trow[wb + 160 + lane] : -1;
+            p0 = wb + 192 + lane < nblk ? trow[wb + 192 + lane] : -1;
+            p1 = wb + 224 + lane < nblk ? trow[wb + 224 + lane] : -1;
+          }
           if (x == seg0) {
             s_win = s_cur;
             s_trow = trow;
@@ -657,6 +672,12 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
             sw1 = w1;
             sn0 = n0;
             sn1 = n1;
+            if constexpr (BS == 1) {
+              sm0 = m0;
+              sm1 = m1;
+              sp0 = p0;
+              sp1 = p1;
+            }
           }
         }
         for (long long tu = x; tu < pe; tu += kUnitsPerStage) {
@@ -666,8 +687,17 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
             w0 = n0;
             w1 = n1;
             wb += 64;
-            n0 = wb + 64 + lane < nblk ? trow[wb + 64 + lane] : -1;
-            n1 = wb + 96 + lane < nblk ? trow[wb + 96 + lane] : -1;
+            if constexpr (BS == 1) {
+              n0 = m0;
+              n1 = m1;
+              m0 = p0;
+              m1 = p1;
+              p0 = wb + 192 + lane < nblk ? trow[wb + 192 + lane] : -1;
+              p1 = wb + 224 + lane < nblk ? trow[wb + 224 + lane] : -1;
+            } else {
+              n0 = wb + 64 + lane < nblk ? trow[wb + 64 + lane] : -1;
+              n1 = wb + 96 + lane < nblk ? trow[wb + 96 + lane] : -1;
+            }
           }
           const int flags = (tu == x ? F_FIRST : 0) | (tu + kUnitsPerStage >= pe ? F_LAST : 0) |
                             (complete ? F_COMPLETE : 0) |
@@ -788,13 +818,15 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
               tma_load_2d(dst, kv ? &tmv : &tmk, &full[st], KV8 ? 0 : hf * 64, y, policy);
             }
           } else {
-            // block_size 1: every token is its own block; 16-byte cp.async with the same
-            // 128-byte swizzle the TMA path produces.  Stages are 64 tokens, so the window
-            // (w0, w1) holds exactly this stage's table entries, handed out by shuffle.  The
-            // copy loop is unrolled: one warp issues all of a stage's copies, so their
-            // address arithmetic must overlap.
-            constexpr int CPR = D * (KV8 ? 1 : 2) / 16;   // 16-byte chunks per row
-            constexpr int RPI = 32 / CPR;            // rows per warp instruction
+            // block_size 1: every token is its own block.  The rows come in by TMA
+            // gather4 loads, four rows of 128 bytes each (a column half of a 16-bit row, or
+            // a whole 8-bit row) from four table entries, into the same 128-byte-swizzled
+            // tile rows the box loads produce (the swizzle follows the shared-memory address,
+            // and each load's four rows are consecutive 128-byte lines).  Sixteen-byte
+            // cp.async copies, one warp issuing them all, were limited to ~0.4 of HBM
+            // bandwidth here.  Stages are 64 tokens, so the window (w0, w1) holds exactly
+            // this stage's table entries, handed out by shuffle.
+            constexpr int kParts = D * (KV8 ? 1 : 2) / 128;   // 128-byte pieces of a row
             const int ntok = nun * kUnit;
             // KSC: the K / V scales of rows lane and 32+lane (this stage's table entries
             // are w0, w1), read before the slot wait
@@ -825,42 +857,45 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
               sc[kTileTokens + 32 + lane] = scv1;
               __syncwarp();
             }
+            // load items: (group of 4 rows g, piece hf, pool kv), at most 16 * 2 * 2 = 64,
+            // two a lane; rows past the valid tokens (or with a bad block id) read row
+            // rows_total, out of range, which the TMA fills with zeros
+            const int nvalid = ntok < ctx_cur - tok0 ? ntok : ctx_cur - tok0;
+            const int nitems = ((nvalid + 3) >> 2) * kParts * 2;
+            static_assert(kTileTokens / 4 * kParts * 2 <= 64, "two load items a lane");
             if (lane == 0) {
               meta[st] = StageMeta{s_cur, kvh, tok0, nun, ctx_cur, flags, pidx, qslot, newrow};
-              mbar_arrive_expect_tx(&full[st], qbytes + nbytes);
+              mbar_arrive_expect_tx(&full[st], qbytes + nbytes + (uint32_t)nitems * 512u);
               if (qbytes)
                 for (int jq = 0; jq < a.q_len; ++jq)
                   bulk_load(sQ + jq * qrow_bytes, qrow_src(jq), qrow_bytes, &full[st]);
               if (nbytes) stage_new(&full[st]);
             }
-            const int ch = lane % CPR, hf = ch >> 3, cc = ch & 7, rl = lane / CPR;
-            constexpr long long kRowBytes = D * (KV8 ? 1 : 2);
-            const uint8_t* kb = static_cast<const uint8_t*>(a.k_cache) + ch * 16;
-            const uint8_t* vb = static_cast<const uint8_t*>(a.v_cache) + ch * 16;
-            uint8_t* sKl = sK + hf * (kTileTokens * 128) + rl * 128;
-            uint8_t* sVl = sV + hf * (kTileTokens * 128) + rl * 128;
-            const int nvalid = ntok < ctx_cur - tok0 ? ntok : ctx_cur - tok0;
+            __syncwarp();
 #pragma unroll
-            for (int i = 0; i < kTileTokens / RPI; ++i) {
-              const int r0 = i * RPI;
-              if (r0 >= ntok) break;
-              const int r = r0 + rl;
-              const int blk = __shfl_sync(0xffffffffu, r0 >= 32 ? w1 : w0, r & 31);
-              if (r < nvalid) {
-                uint32_t sz = 16;
-                long long row = 0;
-                if ((unsigned)blk < (unsigned)a.num_blocks) {
-                  row = (long long)blk * Hkv + kvh;
-                } else {
-                  if (a.status) atomicOr(a.status, DEV_BAD_BLOCK_ID);
-                  sz = 0;                                // zero fill, no read
+            for (int it = 0; it < 2; ++it) {
+              const int i = it * 32 + lane;
+              const int kv = i & 1, hf = (i >> 1) % kParts, g = (i >> 1) / kParts;
+              int y[4];
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4) {
+                const int r = 4 * g + q4;                // < 64 for every item issued
+                const int b0 = __shfl_sync(0xffffffffu, w0, r & 31);
+                const int b1 = __shfl_sync(0xffffffffu, w1, r & 31);
+                const int blk = r < 32 ? b0 : b1;
+                y[q4] = rows_total;
+                if (i < nitems && r < nvalid) {
+                  if ((unsigned)blk < (unsigned)a.num_blocks) {
+                    y[q4] = blk * Hkv + kvh;
+                  } else if (a.status && hf == 0 && kv == 0) {
+                    atomicOr(a.status, DEV_BAD_BLOCK_ID);
+                  }
                 }
-                const int soff = r0 * 128 + ((cc ^ (r & 7)) << 4);
-                cp_async_16_zfill(sKl + soff, kb + row * kRowBytes, sz, policy);
-                cp_async_16_zfill(sVl + soff, vb + row * kRowBytes, sz, policy);
               }
+              if (i < nitems)
+                tma_gather4((kv ? sV : sK) + hf * (kTileTokens * 128) + g * 512, kv ? &tmv : &tmk,
+                            &full[st], hf * 64, y[0], y[1], y[2], y[3], policy);
             }
-            cp_async_mbar_arrive_noinc(&full[st]);
           }
           if (++st == kStages) {
             st = 0;
@@ -874,16 +909,13 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
     if (ok) {
       if (lane == 0) meta[st].flags = F_END;
       __syncwarp();
-      if (BS == 1 || lane == 0) mbar_arrive(&full[st]);
-      if (BS == 1 && lane == 0) mbar_arrive(&full[st]);
+      if (lane == 0) mbar_arrive(&full[st]);
     } else {
       if (lane == 0) {
         *abort_flag = 1;
         if (a.status) atomicOr(a.status, DEV_TIMEOUT);
       }
     }
-    // drain: nothing this warp issued may still be landing when the CTA exits
-    if constexpr (BS == 1) asm volatile("cp.async.wait_all;" ::: "memory");
     return;
   }
 

@@ -236,7 +236,7 @@ __global__ void __launch_bounds__(wide_threads(NC), 1)
     *last_flag = 0;
     fence_mbar_init();
   }
-  if (BS != 1 && threadIdx.x == 32) {
+  if (threadIdx.x == 32) {
     prefetch_tensormap(&tmk);
     prefetch_tensormap(&tmv);
   }
@@ -371,6 +371,9 @@ __global__ void __launch_bounds__(wide_threads(NC), 1)
         const long long trow_seq = MODE == kPrefix ? (long long)chunk_member(a, s_cur, 0) : s_cur;
         const int32_t* trow = a.block_tables + trow_seq * a.max_blocks;
         const int nblk = (ctx_cur + BS - 1) / BS;
+        // block_size 1: the table entries of the portion's next stage, loaded while this
+        // stage waits for its slot (pv_tok = the token they start at, -1: none loaded)
+        int pv[4] = {-1, -1, -1, -1}, pv_tok = -1;
         for (long long tu = x; tu < pe; tu += kWideUnits) {
           const int nun = (int)((pe - tu) < kWideUnits ? (pe - tu) : kWideUnits);
           const int tok0 = (int)(tu - seg0) * kUnit;
@@ -454,53 +457,67 @@ __global__ void __launch_bounds__(wide_threads(NC), 1)
               }
             }
           } else {
-            // block_size 1: each token is its own block; 16-byte cp.async into the same
-            // 128-byte-swizzled rows the TMA path produces.  Lane l reads the table entries
-            // of rows l, 32+l, 64+l, 96+l before the slot wait.
-            constexpr int CPR = D * 2 / 16;            // 16-byte chunks per row
-            constexpr int RPI = 32 / CPR;              // rows per warp instruction
+            // block_size 1: each token is its own block.  TMA gather4 loads bring four rows
+            // of one column half (128 bytes each, four table entries) into four consecutive
+            // 128-byte lines of the same swizzled layout the box loads produce (the swizzle
+            // follows the shared-memory address).  Lane l holds the table entries of rows
+            // l, 32+l, 64+l, 96+l, read during the previous stage of the portion (for its
+            // first stage: before the slot wait).
             const int nvalid = (nun * kUnit < ctx_cur - tok0) ? nun * kUnit : ctx_cur - tok0;
             int wv[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const int r = j * 32 + lane;
-              wv[j] = r < nvalid ? __ldg(trow + tok0 + r) : -1;
+              wv[j] = pv_tok == tok0 ? pv[j] : (r < nvalid ? __ldg(trow + tok0 + r) : -1);
+            }
+            if (tu + kWideUnits < pe) {                // warp-uniform: the next stage's entries
+              const int t1 = tok0 + kWideTile;
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const int r = j * 32 + lane;
+                pv[j] = t1 + r < ctx_cur ? __ldg(trow + t1 + r) : -1;
+              }
+              pv_tok = t1;
             }
             if (!mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, kWaitLimitNs)) {
               ok = false;
               break;
             }
+            // load items (group of 4 rows g, half hf, pool kv): at most 32 * 2 * 2 = 128,
+            // four a lane; rows past the valid tokens or with a bad block id read row
+            // rows_total, out of range, which the TMA fills with zeros
+            const int nitems = ((nvalid + 3) >> 2) * L::kHalves * 2;
+            static_assert(kWideTile / 4 * L::kHalves * 2 <= 128, "four load items a lane");
             if (lane == 0) {
               meta[st] = StageMeta{s_cur, kvh, tok0, nun, ctx_cur, flags, pidx, qslot, -1};
-              mbar_arrive_expect_tx(&full[st], 0u);
+              mbar_arrive_expect_tx(&full[st], (uint32_t)nitems * 512u);
             }
-            const int ch = lane % CPR, hf = ch >> 3, cc = ch & 7, rl = lane / CPR;
-            const uint8_t* kb = static_cast<const uint8_t*>(a.k_cache) + ch * 16;
-            const uint8_t* vb = static_cast<const uint8_t*>(a.v_cache) + ch * 16;
-#pragma unroll 4
-            for (int i = 0; i < kWideTile / RPI; ++i) {
-              const int r0 = i * RPI;
-              if (r0 >= nvalid) break;
-              const int r = r0 + rl;
-              const int v0 = __shfl_sync(0xffffffffu, wv[0], r & 31);
-              const int v1 = __shfl_sync(0xffffffffu, wv[1], r & 31);
-              const int v2 = __shfl_sync(0xffffffffu, wv[2], r & 31);
-              const int v3 = __shfl_sync(0xffffffffu, wv[3], r & 31);
-              const int blk = r < 32 ? v0 : (r < 64 ? v1 : (r < 96 ? v2 : v3));
-              if (r < nvalid) {
-                uint32_t sz = 16;
-                long long row = 0;
-                if ((unsigned)blk < (unsigned)a.num_blocks) {
-                  row = (long long)blk * Hkv + kvh;
-                } else {
-                  if (a.status) atomicOr(a.status, DEV_BAD_BLOCK_ID);
-                  sz = 0;                              // zero fill, no read
+            __syncwarp();
+#pragma unroll
+            for (int it = 0; it < 4; ++it) {
+              const int i = it * 32 + lane;
+              const int kv = i & 1, hf = (i >> 1) % L::kHalves, g = (i >> 1) / L::kHalves;
+              int y[4];
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4) {
+                const int r = 4 * g + q4;                // < 128 for every item issued
+                const int v0 = __shfl_sync(0xffffffffu, wv[0], r & 31);
+                const int v1 = __shfl_sync(0xffffffffu, wv[1], r & 31);
+                const int v2 = __shfl_sync(0xffffffffu, wv[2], r & 31);
+                const int v3 = __shfl_sync(0xffffffffu, wv[3], r & 31);
+                const int blk = (r & 127) < 32 ? v0 : ((r & 127) < 64 ? v1 : ((r & 127) < 96 ? v2 : v3));
+                y[q4] = rows_total;
+                if (i < nitems && r < nvalid) {
+                  if ((unsigned)blk < (unsigned)a.num_blocks) {
+                    y[q4] = blk * Hkv + kvh;
+                  } else if (a.status && hf == 0 && kv == 0) {
+                    atomicOr(a.status, DEV_BAD_BLOCK_ID);
+                  }
                 }
-                const int soff = ((r >> 3) * L::kHalves + hf) * 1024 + (r & 7) * 128 +
-                                 ((cc ^ (r & 7)) << 4);
-                cp_async_16_zfill(sK + soff, kb + row * (D * 2), sz, policy);
-                cp_async_16_zfill(sV + soff, vb + row * (D * 2), sz, policy);
               }
+              if (i < nitems)
+                tma_gather4((kv ? sV : sK) + ((g >> 1) * L::kHalves + hf) * 1024 + (g & 1) * 512,
+                            kv ? &tmv : &tmk, &full[st], hf * 64, y[0], y[1], y[2], y[3], policy);
             }
           }
           if (first_stage) {
