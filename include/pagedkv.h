@@ -526,18 +526,24 @@ pa_status pa_bm_swap_in(pa_block_manager* bm, int32_t seq, int32_t* blocks, int*
  * sharing group (groups in order of first appearance, members in row order).  A group's
  * prefix is the leading table entries common to all its members, in tokens, capped at
  * its shortest member's context length; a group of one row, or with a prefix of 0,
- * gets no chunk.  Each group is cut, in row order, into chunks of at most chunk_width
- * members (the last padded with -1), all with the group's prefix; prefix_lens[i] is the
- * prefix of row i's chunk, 0 for a row in no chunk.  Identical blocks hold identical
- * K/V, so this is exactly the contract pa_decode_cascade states.
+ * gets no chunk.  Each group is cut, in row order, into chunks of at most W members
+ * (the last padded with -1), all with the group's prefix; prefix_lens[i] is the prefix
+ * of row i's chunk, 0 for a row in no chunk.  Identical blocks hold identical K/V, so
+ * this is exactly the contract pa_decode_cascade states.
  *
  *   group         q heads per kv head (num_q_heads / num_kv_heads), >= 1
- *   chunk_width   members per chunk; <= 0 picks 64 / group (at least 1).  group *
- *                 chunk_width must be <= 64 (PA_ERR_UNSUPPORTED otherwise).
+ *   chunk_width   W, members per chunk: group * W must be <= 64 (PA_ERR_UNSUPPORTED
+ *                 otherwise).  <= 0 fits W to the batch: with Wmax = max(1, 64 / group),
+ *                 W is the largest over sharing groups of ceil(m / ceil(m / Wmax)) for
+ *                 a group of m members -- each group in the fewest chunks Wmax allows,
+ *                 spread evenly -- or Wmax when no group shares a prefix.  The query
+ *                 rows of a chunk are MMA columns, so unused member slots cost work.
  *   prefix_lens   HOST int32 [num_seqs] (written)
- *   chunk_members HOST int32 [num_seqs][chunk_width] (written: the first *num_chunks
- *                 rows; there are never more chunks than rows)
+ *   chunk_members HOST int32 [num_seqs][W] (written, row stride W: the first
+ *                 *num_chunks rows; there are never more chunks than rows; with
+ *                 chunk_width <= 0 allocate for W = Wmax)
  *   chunk_prefix_lens  HOST int32 [num_seqs] (written: the first *num_chunks entries)
+ *   chunk_width_out    HOST int (written: W), or NULL
  * Host-only, no GPU.  pa_plan_cascade reads the tables (HOST int32
  * [num_seqs][max_blocks_per_seq], each holding ceil(context_lens[i]/block_size) valid
  * entries, else PA_ERR_INVALID); pa_bm_plan_cascade reads the manager's tables of
@@ -546,10 +552,10 @@ pa_status pa_bm_swap_in(pa_block_manager* bm, int32_t seq, int32_t* blocks, int*
 pa_status pa_plan_cascade(const int32_t* block_tables, int max_blocks_per_seq,
                           const int32_t* context_lens, int num_seqs, int block_size, int group,
                           int chunk_width, int32_t* prefix_lens, int32_t* chunk_members,
-                          int32_t* chunk_prefix_lens, int* num_chunks);
+                          int32_t* chunk_prefix_lens, int* num_chunks, int* chunk_width_out);
 pa_status pa_bm_plan_cascade(const pa_block_manager* bm, const int32_t* seqs, int n, int group,
                              int chunk_width, int32_t* prefix_lens, int32_t* chunk_members,
-                             int32_t* chunk_prefix_lens, int* num_chunks);
+                             int32_t* chunk_prefix_lens, int* num_chunks, int* chunk_width_out);
 
 #ifdef __cplusplus
 }

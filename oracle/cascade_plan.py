@@ -16,6 +16,12 @@ which prefix:
   3. a group of one row, or one whose prefix is empty, shares nothing;
   4. the members of a sharing group are dealt, in row order, into chunks of at most
      `width` rows (the last chunk padded with -1), each carrying the group's prefix.
+
+The chunk width is a scheduling choice the pages leave open (a chunk's query rows are the
+columns of one decode tile, at most 64).  When the caller gives none, the width is the
+smallest that still puts each sharing group in the fewest chunks of at most 64 // group
+rows: for a group of m rows that is ceil(m / ceil(m / Wmax)), and the batch takes the
+largest over its sharing groups (Wmax when no group shares anything).
 """
 from __future__ import annotations
 
@@ -23,11 +29,12 @@ import numpy as np
 
 
 def plan_cascade(tables, ctx, block_size: int, group: int, width: int | None = None):
-    """Returns (prefix_lens int32 [B], chunk_members int32 [C, width],
-    chunk_prefix_lens int32 [C]); width defaults to 64 // group members (64 query rows)."""
+    """Returns (prefix_lens int32 [B], chunk_members int32 [C, W],
+    chunk_prefix_lens int32 [C]); W = width, or fitted to the sharing groups (see the
+    module docstring)."""
     tables = np.asarray(tables)
     ctx = [int(c) for c in np.asarray(ctx)]
-    W = width or max(1, 64 // group)
+    wmax = max(1, 64 // group)
     order, groups = [], {}
     for i, c in enumerate(ctx):
         if c <= 0:
@@ -37,8 +44,7 @@ def plan_cascade(tables, ctx, block_size: int, group: int, width: int | None = N
             groups[first] = []
             order.append(first)
         groups[first].append(i)
-    prefix = [0] * len(ctx)
-    chunks, plens = [], []
+    sharing = []                                       # (rows, prefix) of each sharing group
     for first in order:
         rows = groups[first]
         if len(rows) < 2:
@@ -49,8 +55,17 @@ def plan_cascade(tables, ctx, block_size: int, group: int, width: int | None = N
         while k < usable and len({int(tables[i][k]) for i in rows}) == 1:
             k += 1
         plen = min(k * block_size, shortest)
-        if plen == 0:
-            continue
+        if plen > 0:
+            sharing.append((rows, plen))
+    if width:
+        W = width
+    elif sharing:
+        W = max(-(-len(rows) // -(-len(rows) // wmax)) for rows, _ in sharing)
+    else:
+        W = wmax
+    prefix = [0] * len(ctx)
+    chunks, plens = [], []
+    for rows, plen in sharing:
         for start in range(0, len(rows), W):
             part = rows[start:start + W]
             chunks.append(part + [-1] * (W - len(part)))

@@ -62,9 +62,9 @@ def _lib():
         L.pa_bm_block_tables.restype = i32
         L.pa_bm_slot_of.argtypes = [P, i32, i64, P]
         L.pa_bm_slot_of.restype = i32
-        L.pa_bm_plan_cascade.argtypes = [P, P, i32, i32, i32, P, P, P, P]
+        L.pa_bm_plan_cascade.argtypes = [P, P, i32, i32, i32, P, P, P, P, P]
         L.pa_bm_plan_cascade.restype = i32
-        L.pa_plan_cascade.argtypes = [P, i32, P, i32, i32, i32, i32, P, P, P, P]
+        L.pa_plan_cascade.argtypes = [P, i32, P, i32, i32, i32, i32, P, P, P, P, P]
         L.pa_plan_cascade.restype = i32
         L.pa_bm_swap_out.argtypes = [P, i32, P, P]
         L.pa_bm_swap_out.restype = i32
@@ -86,8 +86,9 @@ def plan_cascade_tables(tables: np.ndarray, ctx: np.ndarray, block_size: int, gr
                         width: int | None = None):
     """Shared-prefix chunks of a batch for pa_decode_cascade, from its block tables
     (pa_plan_cascade in include/pagedkv.h).  Returns (prefix_lens int32 [B],
-    chunk_members int32 [C, width], chunk_prefix_lens int32 [C]); the default width puts
-    64 query rows in a chunk (64 // group members)."""
+    chunk_members int32 [C, W], chunk_prefix_lens int32 [C]); W = width, or by default
+    fitted to the sharing groups (each in the fewest chunks of at most 64 // group
+    members, spread evenly)."""
     t = np.ascontiguousarray(np.asarray(tables, dtype=np.int32))
     c = np.ascontiguousarray(np.asarray(ctx, dtype=np.int32))
     B = c.shape[0]
@@ -95,13 +96,18 @@ def plan_cascade_tables(tables: np.ndarray, ctx: np.ndarray, block_size: int, gr
     prefix = np.zeros(max(B, 1), dtype=np.int32)
     members = np.zeros((max(B, 1), W), dtype=np.int32)
     plens = np.zeros(max(B, 1), dtype=np.int32)
-    nc = ctypes.c_int()
+    nc, wo = ctypes.c_int(), ctypes.c_int()
     rc = _lib().pa_plan_cascade(_ptr(t), t.shape[1] if t.ndim == 2 else 0, _ptr(c), B,
-                                int(block_size), int(group), W, _ptr(prefix), _ptr(members),
-                                _ptr(plens), ctypes.byref(nc))
+                                int(block_size), int(group), int(width or 0), _ptr(prefix),
+                                _ptr(members), _ptr(plens), ctypes.byref(nc), ctypes.byref(wo))
     if rc != pk.PA_OK:
         raise ValueError("pa_plan_cascade failed (%d)" % rc)
-    return prefix[:B].copy(), members[:nc.value].copy(), plens[:nc.value].copy()
+    return _unpack_plan(prefix, members, plens, B, nc.value, wo.value)
+
+
+def _unpack_plan(prefix, members, plens, B, nc, w):
+    m = members.reshape(-1)[:nc * w].reshape(nc, w)
+    return prefix[:B].copy(), m.copy(), plens[:nc].copy()
 
 
 class BlockManager:
@@ -254,11 +260,12 @@ class BlockManager:
         prefix = np.zeros(max(B, 1), dtype=np.int32)
         members = np.zeros((max(B, 1), W), dtype=np.int32)
         plens = np.zeros(max(B, 1), dtype=np.int32)
-        nc = ctypes.c_int()
-        rc = self._L.pa_bm_plan_cascade(self._h, _ptr(s), B, int(group), W, _ptr(prefix),
-                                        _ptr(members), _ptr(plens), ctypes.byref(nc))
+        nc, wo = ctypes.c_int(), ctypes.c_int()
+        rc = self._L.pa_bm_plan_cascade(self._h, _ptr(s), B, int(group), int(width or 0),
+                                        _ptr(prefix), _ptr(members), _ptr(plens),
+                                        ctypes.byref(nc), ctypes.byref(wo))
         self._check(rc, "plan_cascade")
-        return prefix[:B].copy(), members[:nc.value].copy(), plens[:nc.value].copy()
+        return _unpack_plan(prefix, members, plens, B, nc.value, wo.value)
 
     def tail_waste(self, sids) -> float:
         """Fraction of held slots that hold no token: only the unused tail of each

@@ -296,12 +296,12 @@ constexpr int kCascadeMaxRows = 64;     // query rows a prefix chunk holds (grou
 template <typename RowFn, typename LenFn>
 pa_status plan_rows(int n, int block_size, int group, int chunk_width, RowFn row, LenFn len,
                     int32_t* prefix_lens, int32_t* chunk_members, int32_t* chunk_prefix_lens,
-                    int* num_chunks) {
+                    int* num_chunks, int* width_out) {
   if (n < 0 || block_size <= 0 || group <= 0 || !num_chunks ||
       (n && (!prefix_lens || !chunk_members || !chunk_prefix_lens)))
     return PA_ERR_INVALID;
-  const int width = chunk_width > 0 ? chunk_width : std::max(1, kCascadeMaxRows / group);
-  if ((int64_t)group * width > kCascadeMaxRows) return PA_ERR_UNSUPPORTED;
+  const int wmax = std::max(1, kCascadeMaxRows / group);
+  if (chunk_width > 0 && (int64_t)group * chunk_width > kCascadeMaxRows) return PA_ERR_UNSUPPORTED;
   *num_chunks = 0;
   // sharing groups: rows with a non-empty context whose first physical block is the same,
   // in order of first appearance, members in batch order
@@ -319,10 +319,14 @@ pa_status plan_rows(int n, int block_size, int group, int chunk_width, RowFn row
       groups[(size_t)it->second].push_back(i);
     }
   }
-  int nc = 0;
-  for (const std::vector<int>& mem : groups) {
+  // each sharing group's prefix: the leading table entries common to every member,
+  // capped at the shortest member (0: the group shares nothing)
+  std::vector<int64_t> plens(groups.size(), 0);
+  int fit = 0;      // the default width: the widest group's members spread evenly over the
+                    // fewest chunks of at most wmax members
+  for (size_t gi = 0; gi < groups.size(); ++gi) {
+    const std::vector<int>& mem = groups[gi];
     if (mem.size() < 2) continue;
-    // the leading table entries common to every member, capped at the shortest member
     int64_t minlen = INT64_MAX;
     for (int i : mem) minlen = std::min<int64_t>(minlen, len(i));
     const int64_t nb = (minlen + block_size - 1) / block_size;
@@ -334,8 +338,18 @@ pa_status plan_rows(int n, int block_size, int group, int chunk_width, RowFn row
       if (!same) break;
       ++common;
     }
-    const int64_t plen = std::min<int64_t>(common * block_size, minlen);
-    if (plen == 0) continue;
+    plens[gi] = std::min<int64_t>(common * block_size, minlen);
+    if (plens[gi] == 0) continue;
+    const int m = (int)mem.size(), k = (m + wmax - 1) / wmax;
+    fit = std::max(fit, (m + k - 1) / k);
+  }
+  const int width = chunk_width > 0 ? chunk_width : (fit > 0 ? fit : wmax);
+  if (width_out) *width_out = width;
+  int nc = 0;
+  for (size_t gi = 0; gi < groups.size(); ++gi) {
+    const std::vector<int>& mem = groups[gi];
+    const int64_t plen = plens[gi];
+    if (mem.size() < 2 || plen == 0) continue;
     for (size_t k = 0; k < mem.size(); k += (size_t)width) {
       int32_t* out = chunk_members + (int64_t)nc * width;
       for (int j = 0; j < width; ++j) {
@@ -358,7 +372,7 @@ extern "C" {
 pa_status pa_plan_cascade(const int32_t* block_tables, int max_blocks_per_seq,
                           const int32_t* context_lens, int num_seqs, int block_size, int group,
                           int chunk_width, int32_t* prefix_lens, int32_t* chunk_members,
-                          int32_t* chunk_prefix_lens, int* num_chunks) {
+                          int32_t* chunk_prefix_lens, int* num_chunks, int* chunk_width_out) {
   if (block_size <= 0 || (num_seqs > 0 && (!block_tables || !context_lens || max_blocks_per_seq <= 0)))
     return PA_ERR_INVALID;
   for (int i = 0; i < num_seqs; ++i) {     // every table must hold its sequence's blocks
@@ -369,12 +383,12 @@ pa_status pa_plan_cascade(const int32_t* block_tables, int max_blocks_per_seq,
       num_seqs, block_size, group, chunk_width,
       [&](int i) { return block_tables + (int64_t)i * max_blocks_per_seq; },
       [&](int i) { return (int64_t)context_lens[i]; }, prefix_lens, chunk_members,
-      chunk_prefix_lens, num_chunks);
+      chunk_prefix_lens, num_chunks, chunk_width_out);
 }
 
 pa_status pa_bm_plan_cascade(const pa_block_manager* bm, const int32_t* seqs, int n, int group,
                              int chunk_width, int32_t* prefix_lens, int32_t* chunk_members,
-                             int32_t* chunk_prefix_lens, int* num_chunks) {
+                             int32_t* chunk_prefix_lens, int* num_chunks, int* chunk_width_out) {
   if (!bm || n < 0 || (n && !seqs)) return PA_ERR_INVALID;
   std::vector<const pa_block_manager::Seq*> rows((size_t)n);
   for (int i = 0; i < n; ++i) {
@@ -385,7 +399,7 @@ pa_status pa_bm_plan_cascade(const pa_block_manager* bm, const int32_t* seqs, in
       n, bm->block_size, group, chunk_width,
       [&](int i) { return rows[(size_t)i]->table.data(); },
       [&](int i) { return rows[(size_t)i]->len; }, prefix_lens, chunk_members, chunk_prefix_lens,
-      num_chunks);
+      num_chunks, chunk_width_out);
 }
 
 }  // extern "C"

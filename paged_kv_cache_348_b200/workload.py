@@ -301,7 +301,8 @@ def plan_cascade(tables: np.ndarray, ctx: np.ndarray, block_size: int, group: in
     pa_decode_cascade, planned by the library (pa_plan_cascade): sequences whose first
     block is the same physical block form a sharing group; its prefix is the leading
     table entries common to all members, capped at the shortest member's length; a
-    chunk holds at most `width` members (default 64 // group, 64 query rows)."""
+    chunk holds at most `width` members (by default fitted to the sharing groups: each
+    in the fewest chunks of at most 64 // group members, spread evenly)."""
     from .block_manager import plan_cascade_tables
 
     return plan_cascade_tables(tables, ctx, block_size, group, width)

@@ -54,10 +54,28 @@ def test_chunk_width_and_padding_are_exact():
     prefix2, members2, plens2 = wl.plan_cascade(_tables(rows), ctx, bs, group=4, width=2)
     assert members2.tolist() == [[0, 1], [2, 3], [4, -1]] and plens2.tolist() == [40] * 3
     assert np.array_equal(prefix2, prefix)
-    # default width: 64 query rows per chunk, 64 // 4 = 16 members
+    # default width: fitted to the sharing group, 5 members fit one chunk of <= 16
     prefix3, members3, plens3 = wl.plan_cascade(_tables(rows), ctx, bs, group=4)
-    assert members3.tolist() == [[0, 1, 2, 3, 4] + [-1] * 11] and plens3.tolist() == [40]
+    assert members3.tolist() == [[0, 1, 2, 3, 4]] and plens3.tolist() == [40]
     assert np.array_equal(prefix3, prefix)
+
+
+def test_default_width_spreads_a_large_group_evenly():
+    # group 4: at most 16 members a chunk.  20 sharers need 2 chunks, so 10 each; a second
+    # group of 3 is padded to that width; a group of 40 would need 3 chunks of 14.
+    bs = 8
+    rows = [[7, 8]] * 20 + [[3, 4]] * 3
+    ctx = np.array([16] * 23, dtype=np.int32)
+    prefix, members, plens = wl.plan_cascade(_tables(rows), ctx, bs, group=4)
+    assert members.tolist() == [list(range(10)), list(range(10, 20)),
+                                [20, 21, 22] + [-1] * 7]
+    assert plens.tolist() == [16, 16, 16] and prefix.tolist() == [16] * 23
+    rows40 = [[7, 8]] * 40
+    _, m40, _ = wl.plan_cascade(_tables(rows40), np.full(40, 16, np.int32), bs, group=4)
+    assert m40.shape == (3, 14) and m40[2].tolist() == list(range(28, 40)) + [-1, -1]
+    # an explicit width is kept as given
+    _, m2, _ = wl.plan_cascade(_tables(rows), ctx, bs, group=4, width=16)
+    assert m2.shape == (3, 16)
 
 
 def test_no_sharing_and_empty_sequences_give_no_chunks():
@@ -73,7 +91,7 @@ def test_divergence_inside_the_first_block_shares_nothing_beyond_it():
     rows = [[5, 6, 7], [5, 8, 9]]
     ctx = np.array([40, 40], dtype=np.int32)
     prefix, members, plens = wl.plan_cascade(_tables(rows), ctx, 16, group=8)
-    assert prefix.tolist() == [16, 16] and members.tolist() == [[0, 1] + [-1] * 6]
+    assert prefix.tolist() == [16, 16] and members.tolist() == [[0, 1]]
 
 
 def _random_sharing_batch(rng, bs):
