@@ -249,10 +249,11 @@ pa_status pa_decode_e4m3_bs(void* out, const void* q, const void* k_cache, const
  * the sequence's own part, each reduced to (max, sum, unnormalised acc), and the two
  * are combined exactly (log-sum-exp); only the rounding order differs from pa_decode.
  *
- * Two launches on `stream`: pass 1 decodes every chunk's prefix (tokens
+ Two launches on `stream`: pass 1 decodes every chunk's prefix (tokens
  * 0..chunk_prefix_lens[c]-1, read through the block table of the chunk's first member)
  * with the query rows of all its members at once; pass 2 decodes every sequence's
- * tokens prefix_lens[s]..context_lens[s]-1 and merges the prefix result.
+ * tokens prefix_lens[s]..context_lens[s]-1 and merges the prefix result.  Pass 2 waits
+ * for pass 1 only where it reads pass 1's partials, so the two overlap.
  *
  *   q, out, caches, block_tables, context_lens   as for pa_decode
  *   prefix_lens        device int32 [num_seqs]: shared-prefix length of each sequence,
@@ -264,9 +265,13 @@ pa_status pa_decode_e4m3_bs(void* out, const void* q, const void* k_cache, const
  *                      of them (pa_plan_cascade plans such chunks)
  *   chunk_prefix_lens  device int32 [num_chunks]
  *   workspace          >= pa_decode_cascade_workspace_bytes(...) bytes, 256-byte aligned
- * Contract (not checked on the device): every sequence with prefix_lens[s] > 0 is a
+ Contract (not checked on the device): every sequence with prefix_lens[s] > 0 is a
  * member of exactly one chunk, whose prefix length equals prefix_lens[s], and the block
- * tables of a chunk's members agree on their first ceil(prefix/block_size) entries.
+ * tables of a chunk's members agree on their first ceil(prefix/block_size) entries; a
+ * member's context is at least its prefix, and a prefix that is not a multiple of
+ * block_size ends its members' contexts (true of tables kept with copy-on-write, where a
+ * block stays shared only while no sharer writes into it; pa_plan_cascade plans such
+ * chunks).
  * Member ids outside [0, num_seqs) count as padding; a chunk whose first member is
  * padding is empty.  num_q_heads/num_kv_heads must be <= 16 (the per-sequence pass).
  * Other arguments, limits and errors as for pa_decode.

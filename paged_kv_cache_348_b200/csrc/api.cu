@@ -179,6 +179,7 @@ struct CascadeArgs {
   float* ext_acc = nullptr;
   const void* k_new = nullptr;   // kAppend
   const void* v_new = nullptr;
+  int late_wait = 0;             // kSuffix: wait for the prefix pass only where it is needed
   bool kv8 = false;              // 8-bit E4M3 caches with these scales
   float k_scale = 1.f, v_scale = 1.f;
   const float* k_bscale = nullptr;   // 8-bit caches: per-(block, kv head) scales instead
@@ -253,7 +254,7 @@ pa_status decode_impl(void* out, const void* q, const void* k_cache, const void*
       return PA_ERR_CUDA;
     }
   }
-  pkv::DecodeArgs a;
+  pkv::DecodeArgs a{};
   a.out = out;
   a.q = q;
   a.k_cache = k_cache;
@@ -284,6 +285,7 @@ pa_status decode_impl(void* out, const void* q, const void* k_cache, const void*
   a.ext_acc = cx.ext_acc;
   a.k_new = cx.k_new;
   a.v_new = cx.v_new;
+  a.late_wait = cx.late_wait;
   a.k_bscale = cx.k_bscale;
   a.v_bscale = cx.v_bscale;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -291,15 +293,17 @@ pa_status decode_impl(void* out, const void* q, const void* k_cache, const void*
                        grid, st);
 }
 
-// Cascade workspace: the split scratch, then the external partials (max, sum)[B][Hq]
-// and acc[B][Hq][D].
+// Cascade workspace: two split scratches (the two passes may run at the same time), then
+// the external partials (max, sum)[B][Hq] and acc[B][Hq][D] that carry the prefix pass's
+// result to the suffix pass.
 struct CascadeLayout {
-  size_t split, ml_off, acc_off, total;
+  size_t split, split2_off, ml_off, acc_off, total;
 };
 CascadeLayout cascade_layout(int num_seqs, int num_q_heads, int head_dim, int sms) {
   CascadeLayout c{};
   c.split = split_workspace_bytes(head_dim, sms);
-  c.ml_off = align256(c.split);
+  c.split2_off = align256(c.split);
+  c.ml_off = align256(c.split2_off + c.split);
   c.acc_off = align256(c.ml_off + sizeof(float2) * (size_t)num_seqs * num_q_heads);
   c.total = align256(c.acc_off + sizeof(float) * (size_t)num_seqs * num_q_heads * head_dim);
   return c;
@@ -327,8 +331,6 @@ pa_status cascade_impl(void* out, const void* q, const void* k_cache, const void
   const CascadeLayout cl = cascade_layout(num_seqs, num_q_heads, head_dim, sms);
   if (workspace_bytes < cl.total) return PA_ERR_INVALID;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  cx.ext_ml = reinterpret_cast<float2*>(ws + cl.ml_off);
-  cx.ext_acc = reinterpret_cast<float*>(ws + cl.acc_off);
   const int group = num_q_heads / num_kv_heads;
   // the prefix pass puts a chunk's members' query rows side by side (up to 64 columns on
   // 16-bit pools, 16 on 8-bit ones); the suffix pass decodes one new token per sequence
@@ -336,6 +338,12 @@ pa_status cascade_impl(void* out, const void* q, const void* k_cache, const void
   const int prefix_cols = cx.kv8 ? pkv::kMaxGroup : pkv::kWideCols;
   if (group > pkv::kMaxGroup || (num_chunks && (long long)group * chunk_width > prefix_cols))
     return PA_ERR_UNSUPPORTED;
+  // pass 1 writes each chunk's prefix partial for its members (the external partials);
+  // pass 2 decodes every sequence's own tokens and merges that partial.  Pass 2 uses a
+  // split scratch of its own and reads the partials only when it merges, so it waits for
+  // pass 1 there (and at its end) rather than at its start, and overlaps pass 1's end.
+  cx.ext_ml = reinterpret_cast<float2*>(ws + cl.ml_off);
+  cx.ext_acc = reinterpret_cast<float*>(ws + cl.acc_off);
   if (num_chunks > 0) {
     // pass 1: each chunk's shared prefix once, its members' query rows as MMA columns
     cx.mode = pkv::kPrefix;
@@ -351,9 +359,11 @@ pa_status cascade_impl(void* out, const void* q, const void* k_cache, const void
   cx.mode = pkv::kSuffix;
   cx.chunk_members = nullptr;
   cx.seq_start = prefix_lens;
+  cx.late_wait = num_chunks > 0 ? 1 : 0;      // its previous grid is then pass 1
   return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, 1,
                      num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
-                     num_blocks, scale, dtype, workspace, cl.split, 0, dev_status, stream, cx);
+                     num_blocks, scale, dtype, ws + cl.split2_off, cl.split, 0, dev_status,
+                     stream, cx);
 }
 
 

@@ -126,6 +126,10 @@ struct DecodeArgs {
   const int32_t* seq_start;     // kSuffix: first token of each sequence's own part
   const int32_t* chunk_members; // kPrefix: [num_seqs][q_len] member sequences, -1 pad
   int q_rows;                   // kPrefix: sequences in q / block_tables (valid member ids)
+  int late_wait;                // kSuffix: wait for the previous grid (the cascade's prefix
+                                // pass, whose only output this launch reads is the external
+                                // partials) before reading those, and at the end, not at
+                                // the start
   float2* ext_ml;               // [members][Hq] (max, sum) of the prefix part, base 2
   float* ext_acc;               // [members][Hq][D] its unnormalised accumulator
   // kAppend: K/V of each sequence's newest token, [seqs][Hkv][D]
@@ -497,7 +501,13 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
     prefetch_tensormap(&tmv);
   }
   __syncthreads();
-  pdl_wait();      // nothing global is read or written before the previous grid is done
+  // Nothing global is read or written before the previous grid is done -- except in a
+  // late-wait suffix launch: its previous grid is the cascade's prefix pass, which writes
+  // nothing this launch touches but the external partials, so it waits for that grid only
+  // before it reads them (CTA 0's rows without units, every end-of-portion merge) and
+  // before it exits; it overlaps the prefix pass's end and still completes after it.
+  const bool late_wait = MODE == kSuffix && a.late_wait;
+  if (!late_wait) pdl_wait();
   pdl_trigger();
 
   const int G = gridDim.x, c = blockIdx.x;
@@ -505,6 +515,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
 
   if (warp == 0) {
     // ============================== producer ==============================
+    if (late_wait && c == 0) pdl_wait();
     const int B = a.num_seqs;
     // pass 1 over the batch: total units; CTA 0 also writes the zero rows of empty
     // sequences (they own no unit).  For B <= 32 the lane values are kept for pass 2.
@@ -916,6 +927,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
         if (a.status) atomicOr(a.status, DEV_TIMEOUT);
       }
     }
+    if (late_wait) pdl_wait();
     return;
   }
 
@@ -1270,6 +1282,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
       }
     }
     if (mt.flags & F_LAST) {
+      if (late_wait) pdl_wait();                 // the prefix partials are complete
       // ---- merge the four warps' (m, l, O) for this segment portion
 #pragma unroll
       for (int n = 0; n < NTW; ++n)
@@ -1413,6 +1426,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
       ph ^= 1u;
     }
   }
+  if (late_wait) pdl_wait();
 }
 
 }  // namespace pkv

@@ -258,7 +258,6 @@ __global__ void __launch_bounds__(wide_threads(NC), 1)
 
   const int G = gridDim.x, c = blockIdx.x;
   const int Hkv = a.num_kv_heads, group = a.group;
-  constexpr int nq = NC;                            // MMA N: the query rows rounded up
 
   if (warp == 0) {
     // ============================== producer ==============================
