@@ -16,6 +16,12 @@
  *    allocates no device memory and keeps no state between calls.
  *  - Synchrony: every call only enqueues work on `stream` (a cudaStream_t; NULL is
  *    the legacy default stream) and returns; results are ready when the stream is.
+ *    The kernels are launched as programmatic dependents of the previous kernel on the
+ *    stream: a decode kernel may begin reading its context lengths, block tables,
+ *    prefix lengths and chunk members while a previous kernel of THIS library is still
+ *    running (none of them writes those arrays); everything else waits for it.  A
+ *    kernel of other code that writes those arrays must finish before the call (plain
+ *    stream order does that, unless that kernel itself releases its dependents early).
  *  - Errors: arguments are validated on the host before anything is enqueued; a
  *    failed check returns an error code and enqueues nothing.  A CUDA launch error
  *    returns PA_ERR_CUDA.  Range violations found on the device (a block id outside

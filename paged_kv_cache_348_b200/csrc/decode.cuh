@@ -501,21 +501,24 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
     prefetch_tensormap(&tmv);
   }
   __syncthreads();
-  // Nothing global is read or written before the previous grid is done -- except in a
-  // late-wait suffix launch: its previous grid is the cascade's prefix pass, which writes
-  // nothing this launch touches but the external partials, so it waits for that grid only
-  // before it reads them (CTA 0's rows without units, every end-of-portion merge) and
-  // before it exits; it overlaps the prefix pass's end and still completes after it.
+  // Nothing global is written, and nothing a previous kernel may write is read, before the
+  // previous grid is done.  The producer of every CTA but CTA 0 (which writes the rows of
+  // sequences without units) computes its schedule first: that reads only the launch's
+  // lengths, starts and block tables, which no kernel of this library writes.  A late-wait
+  // suffix launch's previous grid is the cascade's prefix pass, which writes nothing this
+  // launch touches but the external partials, so it waits for that grid only before it
+  // reads them (CTA 0's rows without units, every end-of-portion merge) and before it
+  // exits; it overlaps the prefix pass's end and still completes after it.
   const bool late_wait = MODE == kSuffix && a.late_wait;
-  if (!late_wait) pdl_wait();
-  pdl_trigger();
+  if (warp != 0 && !late_wait) pdl_wait();
+  if (warp != 0) pdl_trigger();
 
   const int G = gridDim.x, c = blockIdx.x;
   const int Hkv = a.num_kv_heads, group = a.group;
 
   if (warp == 0) {
     // ============================== producer ==============================
-    if (late_wait && c == 0) pdl_wait();
+    if (c == 0) pdl_wait();
     const int B = a.num_seqs;
     // pass 1 over the batch: total units; CTA 0 also writes the zero rows of empty
     // sequences (they own no unit).  For B <= 32 the lane values are kept for pass 2.
@@ -592,6 +595,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
     }
     if (lane == 0) *total_s = total;
     __syncwarp();
+    if (c != 0 && !late_wait) pdl_wait();
 
     const uint64_t policy = policy_evict_first();
     const int rows_total = a.num_blocks * Hkv * BS;

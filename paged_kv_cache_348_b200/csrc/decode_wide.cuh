@@ -253,14 +253,21 @@ __global__ void __launch_bounds__(wide_threads(NC), 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  pdl_wait();      // nothing global is read or written before the previous grid is done
-  pdl_trigger();
+  // Nothing global is written, and nothing a previous kernel may write is read, before the
+  // previous grid is done; the producer of every CTA but CTA 0 (which writes the rows of
+  // sequences without units) computes its schedule first, from the launch's lengths and
+  // chunk members, which no kernel of this library writes.
+  if (warp != 0) {
+    pdl_wait();
+    pdl_trigger();
+  }
 
   const int G = gridDim.x, c = blockIdx.x;
   const int Hkv = a.num_kv_heads, group = a.group;
 
   if (warp == 0) {
     // ============================== producer ==============================
+    if (c == 0) pdl_wait();
     const int B = a.num_seqs;
     long long run = 0;
     int keep_ctx = 0, keep_u = 0, keep_x = 0;
@@ -328,6 +335,7 @@ __global__ void __launch_bounds__(wide_threads(NC), 1)
     }
     if (lane == 0) *total_s = total;
     __syncwarp();
+    if (c != 0) pdl_wait();
 
     const uint64_t policy = policy_evict_first();
     const int rows_total = a.num_blocks * Hkv * BS;
