@@ -145,8 +145,11 @@ struct DecodeArgs {
 
 // Shared-memory layout of a CTA.  16-bit caches: K and V tiles of 64 tokens in D/64
 // column halves of 128-byte lines; 8-bit (E4M3) caches: one line of D bytes per token
-// (D = 128), and, since a stage is half the size, a deeper ring.  CPS = CTAs per SM.
-template <int D, bool KV8 = false, int CPS = 2>
+// (D = 128), and, since a stage is half the size, a deeper ring.  CPS = CTAs per SM;
+// NEW: the fused append's staged rows, SC: the 8-bit per-row scales (regions left out
+// when the launch has no use for them: every byte of shared memory a CTA takes is L1 the
+// spilled registers of the 3-CTA configurations no longer have).
+template <int D, bool KV8 = false, int CPS = 2, bool NEW = true, bool SC = KV8>
 struct Layout {
   static constexpr int kStages = KV8 ? (CPS == 2 ? 5 : 3) : (CPS == 2 ? 3 : 2);
   static_assert(CPS == 2 || CPS == 3, "2 or 3 CTAs per SM");
@@ -164,11 +167,11 @@ struct Layout {
   static constexpr int kMlOff = kDescOff + 2 * (int)sizeof(SplitDesc);
   // fused append: per stage the new token's K and V rows, staged by the producer
   static constexpr int kNewOff = (kMlOff + kConsumerWarps * kMaxGroup * 8 + 15) / 16 * 16;
-  static constexpr int kNewBytes = 2 * D * 2;         // the new token's 16-bit K and V rows
+  static constexpr int kNewBytes = NEW ? 2 * D * 2 : 0;   // the new token's 16-bit K, V rows
   // 8-bit caches with per-(block, kv head) scales: per stage the K and V scale of every
   // token row, staged by the producer
   static constexpr int kScOff = kNewOff + kStages * kNewBytes;
-  static constexpr int kScBytes = KV8 ? 2 * kTileTokens * 4 : 0;
+  static constexpr int kScBytes = SC ? 2 * kTileTokens * 4 : 0;
   static constexpr int kBytes = kScOff + kStages * kScBytes;
   static constexpr int kDynSmem = kBytes + 1024;           // slack for 1024-byte alignment
   static_assert(kBarOff % 8 == 0 && kMiscOff % 8 == 0 && kDescOff % 8 == 0 && kMlOff % 8 == 0 &&
@@ -463,7 +466,7 @@ template <typename T, int D, int BS, int NT, int MODE, bool KV8 = false, bool KS
 __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
     pa_decode_split_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
                            const __grid_constant__ CUtensorMap tmv) {
-  using L = Layout<D, KV8, ctas_per_sm(KV8, NT, BS)>;
+  using L = Layout<D, KV8, ctas_per_sm(KV8, NT, BS), MODE == kAppend, KSC>;
   constexpr int kStages = L::kStages;
   constexpr int kSegW = seg_weight(BS);
   static_assert(!KV8 || D == 128, "8-bit caches: head_dim 128");
