@@ -189,7 +189,7 @@ pa_status pa_decode_append(void* out, const void* q, void* k_cache, void* v_cach
  * code, everything else as for pa_decode (q and out 16-bit, dtype).  Inside, the codes
  * are converted exactly to fp16 and the products use fp16 tensor-core MMAs with fp32
  * accumulation (q is converted to fp16: values beyond fp16's range are not supported).
- * head_dim 128 only (PA_ERR_UNSUPPORTED otherwise); workspace as for pa_decode.
+ * head_dim 64 or 128; workspace as for pa_decode.
  */
 pa_status pa_cache_append_e4m3(void* k_cache, void* v_cache, const void* k, const void* v,
                                const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
@@ -227,7 +227,8 @@ pa_status pa_decode_e4m3(void* out, const void* q, const void* k_cache, const vo
  * q_len = 1 is pa_decode) over such pools: K_s[t] = k_scales[b][h] * code with b the
  * physical block of position t, V likewise.  Inside, each token row's K scale multiplies
  * its scores and its V scale its softmax weights before the fp16 tensor-core PV product.
- * head_dim 128, (num_q_heads/num_kv_heads) * q_len <= 16; workspace as for pa_decode.
+ * head_dim 64 or 128, (num_q_heads/num_kv_heads) * q_len <= 16; workspace as for
+ * pa_decode.
  */
 pa_status pa_cache_append_e4m3_bs(void* k_cache, void* v_cache, float* k_scales,
                                   float* v_scales, const void* k, const void* v,
@@ -296,7 +297,7 @@ pa_status pa_decode_cascade(void* out, const void* q, const void* k_cache, const
 
 /*
  * The cascade and the fused append over 8-bit pools with per-(block, kv head) scales
- * (the format of pa_cache_append_e4m3_bs / pa_decode_e4m3_bs; head_dim 128).
+ * (the format of pa_cache_append_e4m3_bs / pa_decode_e4m3_bs; head_dim 64 or 128).
  *
  * pa_decode_cascade_e4m3_bs -- pa_decode_cascade over such pools: the result is that of
  * pa_decode_e4m3_bs (q_len 1) on the same inputs, the softmax split at prefix_lens[s]

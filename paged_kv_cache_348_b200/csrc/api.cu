@@ -84,7 +84,8 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 // 2-D view of one pool: rows = num_blocks*kv_heads*block_size, each head_dim elements;
 // box = 64 dims x box_rows rows, 128-byte swizzle, out-of-range rows read as zero.
-// kv8: an 8-bit (E4M3) pool, rows of head_dim bytes, box = head_dim x box_rows (128 B).
+// kv8: an 8-bit (E4M3) pool, rows of head_dim bytes, box = head_dim x box_rows, with the
+// 128-byte swizzle at head_dim 128 and the 64-byte one at head_dim 64 (one row a line).
 bool encode_pool(CUtensorMap* map, const void* base, pa_dtype dtype, int head_dim,
                  uint64_t rows, int box_rows, bool kv8 = false) {
   auto enc = tensor_map_encoder();
@@ -97,7 +98,8 @@ bool encode_pool(CUtensorMap* map, const void* base, pa_dtype dtype, int head_di
                             : dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                                : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
                    2, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   (kv8 && head_dim == 64) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -232,9 +234,8 @@ pa_status decode_impl(void* out, const void* q, const void* k_cache, const void*
   CUtensorMap mk, mv;
   std::memset(&mk, 0, sizeof(mk));
   std::memset(&mv, 0, sizeof(mv));
-  // 8-bit pools: head_dim 128; the cascade and fused-append modes need per-block scales
-  if (cx.kv8 && (head_dim != 128 || (cx.mode != pkv::kPlain && !cx.k_bscale)))
-    return PA_ERR_UNSUPPORTED;
+  // 8-bit pools: the cascade and fused-append modes need per-block scales
+  if (cx.kv8 && cx.mode != pkv::kPlain && !cx.k_bscale) return PA_ERR_UNSUPPORTED;
   if (block_size == 1) {
     // both kernels gather block_size-1 rows four at a time: one-row boxes
     const uint64_t rows = (uint64_t)num_blocks * num_kv_heads;

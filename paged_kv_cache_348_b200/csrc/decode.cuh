@@ -65,6 +65,14 @@ constexpr int kThreads = 32 * (1 + kConsumerWarps); // warp 0 produces, 1..4 con
 // codes (half-size stages keep a 3-deep ring), and block_size <= 8, whose producer issues
 // a copy per 16 bytes (block_size 1) or per 1 KB box (block_size 8); 16-bit stages then
 // form a 2-deep ring.
+// 8-bit tile rows: D bytes at D = 128 or 64, 16-byte chunk c of row r stored at chunk
+// c ^ kv8_swz(r): the 128-byte swizzle (the row's low 3 bits) or the 64-byte one (bits 1-2:
+// two 64-byte rows share a 128-byte line), the patterns TMA writes
+template <int D>
+__host__ __device__ constexpr int kv8_swz(int r) {
+  return D == 128 ? (r & 7) : ((r >> 1) & 3);
+}
+
 __host__ __device__ constexpr int ctas_per_sm(bool kv8, int nt, int bs) {
   return (kv8 || bs <= 8) && nt == 1 ? 3 : 2;
 }
@@ -144,8 +152,9 @@ struct DecodeArgs {
 
 
 // Shared-memory layout of a CTA.  16-bit caches: K and V tiles of 64 tokens in D/64
-// column halves of 128-byte lines; 8-bit (E4M3) caches: one line of D bytes per token
-// (D = 128), and, since a stage is half the size, a deeper ring.  CPS = CTAs per SM;
+// column halves of 128-byte lines; 8-bit (E4M3) caches: one row of D bytes per token
+// (D = 128: a 128-byte line, 128-byte swizzle; D = 64: a 64-byte row, 64-byte swizzle),
+// and, since a stage is half the size, a deeper ring.  CPS = CTAs per SM;
 // NEW: the fused append's staged rows, SC: the 8-bit per-row scales (regions left out
 // when the launch has no use for them: every byte of shared memory a CTA takes is L1 the
 // spilled registers of the 3-CTA configurations no longer have).
@@ -472,7 +481,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
   using L = Layout<D, KV8, ctas_per_sm(KV8, NT, BS), MODE == kAppend, KSC>;
   constexpr int kStages = L::kStages;
   constexpr int kSegW = seg_weight(BS);
-  static_assert(!KV8 || D == 128, "8-bit caches: head_dim 128");
+  static_assert(!KV8 || D == 128 || D == 64, "8-bit caches: head_dim 128 or 64");
   static_assert(!KV8 || MODE == kPlain || KSC,
                 "8-bit caches: the cascade and fused-append modes use per-block scales");
   static_assert(!KSC || KV8, "per-block scales belong to 8-bit caches");
@@ -772,7 +781,8 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
             constexpr int H = BS < 16 ? BS : 16;     // rows per TMA box
             constexpr int BPU = kUnit / H;           // boxes per unit and column half
             constexpr int kParts = KV8 ? 1 : L::kHalves;   // boxes per row of a token
-            constexpr int kBoxBytes = H * 128;       // D = 128 8-bit values or 64 16-bit
+            constexpr int kRowB = KV8 ? D : 128;     // tile bytes per row and box
+            constexpr int kBoxBytes = H * kRowB;     // D 8-bit values or 64 16-bit
             static_assert(kUnitsPerStage * BPU * kParts * 2 <= 32, "one box per lane");
             // this lane's box and its block-table entry, read before the slot wait
             const int nbox = nun * BPU * kParts * 2;
@@ -835,7 +845,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
             }
             __syncwarp();
             if (mine) {
-              uint8_t* dst = (kv ? sV : sK) + hf * (kTileTokens * 128) + (j * kUnit + b * H) * 128;
+              uint8_t* dst = (kv ? sV : sK) + hf * (kTileTokens * 128) + (j * kUnit + b * H) * kRowB;
               tma_load_2d(dst, kv ? &tmv : &tmk, &full[st], KV8 ? 0 : hf * 64, y, policy);
             }
           } else {
@@ -847,7 +857,9 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
             // cp.async copies, one warp issuing them all, were limited to ~0.4 of HBM
             // bandwidth here.  Stages are 64 tokens, so the window (w0, w1) holds exactly
             // this stage's table entries, handed out by shuffle.
-            constexpr int kParts = D * (KV8 ? 1 : 2) / 128;   // 128-byte pieces of a row
+            // 128-byte pieces of a row (a 64-byte 8-bit row is one piece of its own size)
+            constexpr int kParts = D * (KV8 ? 1 : 2) >= 128 ? D * (KV8 ? 1 : 2) / 128 : 1;
+            constexpr int kPieceB = KV8 ? (D < 128 ? D : 128) : 128;
             const int ntok = nun * kUnit;
             // KSC: the K / V scales of rows lane and 32+lane (this stage's table entries
             // are w0, w1), read before the slot wait
@@ -886,7 +898,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
             static_assert(kTileTokens / 4 * kParts * 2 <= 64, "two load items a lane");
             if (lane == 0) {
               meta[st] = StageMeta{s_cur, kvh, tok0, nun, ctx_cur, flags, pidx, qslot, newrow};
-              mbar_arrive_expect_tx(&full[st], qbytes + nbytes + (uint32_t)nitems * 512u);
+              mbar_arrive_expect_tx(&full[st], qbytes + nbytes + (uint32_t)nitems * (4u * kPieceB));
               if (qbytes)
                 for (int jq = 0; jq < a.q_len; ++jq)
                   bulk_load(sQ + jq * qrow_bytes, qrow_src(jq), qrow_bytes, &full[st]);
@@ -914,7 +926,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
                 }
               }
               if (i < nitems)
-                tma_gather4((kv ? sV : sK) + hf * (kTileTokens * 128) + g * 512, kv ? &tmv : &tmk,
+                tma_gather4((kv ? sV : sK) + hf * (kTileTokens * 128) + g * 4 * kPieceB, kv ? &tmv : &tmk,
                             &full[st], hf * 64, y[0], y[1], y[2], y[3], policy);
             }
           }
@@ -1036,16 +1048,17 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
         // launch's columns are different sequences: no mask)
         const int lim0 = MODE == kPrefix ? (1 << 30) : mt.ctx - a.q_len + 1 - t0;
         if (MODE == kAppend && KV8 && mt.newrow >= 0 && (mt.ctx - 1 - mt.tok0) / kUnit == u) {
-          // fused append into 8-bit pools with per-(block, kv head) scales: lanes 0..7
-          // quantise the new K row, 8..15 the V row, 16 values (one 16-byte chunk of codes)
-          // each, exactly as the block-scaled append does; a token at offset 0 of its block
-          // first fixes the block's scale from its own row.  The codes go into the tile row
-          // and the cache row, the scale into the stage's scale row and, for offset 0, the
-          // scale array.  With split columns both warps compute the same bytes; the first
-          // writes global memory.
+          // fused append into 8-bit pools with per-(block, kv head) scales: D/16 lanes
+          // quantise the new K row and as many the V row, 16 values (one 16-byte chunk of
+          // codes) each, exactly as the block-scaled append does; a token at offset 0 of its
+          // block first fixes the block's scale from its own row.  The codes go into the tile
+          // row and the cache row, the scale into the stage's scale row and, for offset 0,
+          // the scale array.  With split columns both warps compute the same bytes; the
+          // first writes global memory.
+          constexpr int CPR8 = D / 16;                  // 16-byte chunks of codes per row
           const int rn = mt.ctx - 1 - mt.tok0;          // row in the stage tile
-          const int kv = (lane >> 3) & 1, ch = lane & 7;
-          const bool act = lane < 16;
+          const int kv = (lane / CPR8) & 1, ch = lane % CPR8;
+          const bool act = lane < 2 * CPR8;
           const uint4* src = reinterpret_cast<const uint4*>(smem + L::kNewOff + st * L::kNewBytes +
                                                             kv * D * 2 + ch * 32);
           uint4 in[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
@@ -1063,9 +1076,8 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
             x[2 * e + 1] = f.y;
             am = fmaxf(am, fmaxf(fabsf(f.x), fabsf(f.y)));
           }
-          am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
-          am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
-          am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 4));
+#pragma unroll
+          for (int o = 1; o < CPR8; o <<= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
           float* scs = reinterpret_cast<float*>(smem + L::kScOff + st * L::kScBytes) + kv * kTileTokens;
           const bool fresh = mt.newrow % BS == 0;       // offset 0: this token fixes the scale
           const float sc = fresh ? e4m3_block_scale(am) : scs[rn];
@@ -1077,7 +1089,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
               q[e] = f32x2_to_e4m3x2(__fdiv_rn(x[4 * e], sc), __fdiv_rn(x[4 * e + 1], sc)) |
                      (f32x2_to_e4m3x2(__fdiv_rn(x[4 * e + 2], sc), __fdiv_rn(x[4 * e + 3], sc)) << 16);
             const uint4 codes = make_uint4(q[0], q[1], q[2], q[3]);
-            *reinterpret_cast<uint4*>((kv ? sV : sK) + rn * 128 + ((ch ^ (rn & 7)) << 4)) = codes;
+            *reinterpret_cast<uint4*>((kv ? sV : sK) + rn * D + ((ch ^ kv8_swz<D>(rn)) << 4)) = codes;
             if (ch == 0 && fresh) scs[rn] = sc;
             if (nb == 0) {
               uint8_t* cache = static_cast<uint8_t*>(const_cast<void*>(kv ? a.v_cache : a.k_cache));
@@ -1122,7 +1134,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
 #pragma unroll
           for (int ks = 0; ks < KS; ks += 2) {
             const int chunk = ks + (j >> 1);
-            const uint32_t addr = kbase + r * 128 + ((chunk ^ (r & 7)) << 4);
+            const uint32_t addr = kbase + r * D + ((chunk ^ kv8_swz<D>(r)) << 4);
             uint32_t m0, m1, m2, m3;
             ldsm_x4(addr, m0, m1, m2, m3);
             uint32_t x0, x1, x2, x3, y0, y1, y2, y3;
@@ -1238,7 +1250,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
 #pragma unroll
             for (int mtile = 0; mtile < KS; mtile += 2) {
               const int chunk = mtile + (j >> 1);
-              const uint32_t addr = vbase + r * 128 + ((chunk ^ (r & 7)) << 4);
+              const uint32_t addr = vbase + r * D + ((chunk ^ kv8_swz<D>(r)) << 4);
               uint32_t m[4];
               ldsm_x4_t(addr, m[0], m[1], m[2], m[3]);
 #pragma unroll

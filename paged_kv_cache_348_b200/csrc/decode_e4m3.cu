@@ -7,10 +7,9 @@ template <>
 pa_status run_decode_mode<pkv::kPlain, true>(bool bf16, int d, int bs, const pkv::DecodeArgs& a,
                                        const CUtensorMap& mk, const CUtensorMap& mv, int grid,
                                        cudaStream_t s) {
-  (void)d;
-  if (a.k_bscale) return run_e4m3_bs(bf16, bs, a, mk, mv, grid, s);
-  if (bf16) return dispatch_e4m3<__nv_bfloat16>(bs, a, mk, mv, grid, s);
-  return dispatch_e4m3<__half>(bs, a, mk, mv, grid, s);
+  if (a.k_bscale) return run_e4m3_bs(bf16, d, bs, a, mk, mv, grid, s);
+  if (bf16) return dispatch_e4m3<__nv_bfloat16>(d, bs, a, mk, mv, grid, s);
+  return dispatch_e4m3<__half>(d, bs, a, mk, mv, grid, s);
 }
 
 }  // namespace pkv_host

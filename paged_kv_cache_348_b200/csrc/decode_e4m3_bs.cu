@@ -4,10 +4,10 @@
 
 namespace pkv_host {
 
-pa_status run_e4m3_bs(bool bf16, int bs, const pkv::DecodeArgs& a, const CUtensorMap& mk,
+pa_status run_e4m3_bs(bool bf16, int d, int bs, const pkv::DecodeArgs& a, const CUtensorMap& mk,
                       const CUtensorMap& mv, int grid, cudaStream_t s) {
-  if (bf16) return dispatch_e4m3<__nv_bfloat16, true>(bs, a, mk, mv, grid, s);
-  return dispatch_e4m3<__half, true>(bs, a, mk, mv, grid, s);
+  if (bf16) return dispatch_e4m3<__nv_bfloat16, true>(d, bs, a, mk, mv, grid, s);
+  return dispatch_e4m3<__half, true>(d, bs, a, mk, mv, grid, s);
 }
 
 }  // namespace pkv_host

@@ -8,10 +8,9 @@ template <>
 pa_status run_decode_mode<pkv::kAppend, true>(bool bf16, int d, int bs, const pkv::DecodeArgs& a,
                                           const CUtensorMap& mk, const CUtensorMap& mv,
                                           int grid, cudaStream_t s) {
-  (void)d;
   if (!a.k_bscale || !a.v_bscale) return PA_ERR_UNSUPPORTED;
-  if (bf16) return dispatch_e4m3<__nv_bfloat16, true, pkv::kAppend>(bs, a, mk, mv, grid, s);
-  return dispatch_e4m3<__half, true, pkv::kAppend>(bs, a, mk, mv, grid, s);
+  if (bf16) return dispatch_e4m3<__nv_bfloat16, true, pkv::kAppend>(d, bs, a, mk, mv, grid, s);
+  return dispatch_e4m3<__half, true, pkv::kAppend>(d, bs, a, mk, mv, grid, s);
 }
 
 }  // namespace pkv_host

@@ -80,28 +80,34 @@ pa_status dispatch_d(int d, int bs, const pkv::DecodeArgs& a, const CUtensorMap&
                  : dispatch_bs<T, 128, MODE>(bs, a, mk, mv, grid, s);
 }
 
-// 8-bit (E4M3) caches, head_dim 128: plain decode (one or several new tokens) with one
-// scale per pool or, KSC, per-(block, kv head) scales; the cascade passes and the fused
+// 8-bit (E4M3) caches, head_dim 128 or 64: plain decode (one or several new tokens) with
+// one scale per pool or, KSC, per-(block, kv head) scales; the cascade passes and the fused
 // append with per-(block, kv head) scales.
-template <typename T, bool KSC = false, int MODE = pkv::kPlain>
-pa_status dispatch_e4m3(int bs, const pkv::DecodeArgs& a, const CUtensorMap& mk,
-                        const CUtensorMap& mv, int grid, cudaStream_t s) {
+template <typename T, int D, bool KSC, int MODE>
+pa_status dispatch_e4m3_d(int bs, const pkv::DecodeArgs& a, const CUtensorMap& mk,
+                          const CUtensorMap& mv, int grid, cudaStream_t s) {
   const bool nt1 = a.ncol <= 8;
   switch (bs) {
-    case 1: return nt1 ? launch_decode<T, 128, 1, 1, MODE, true, KSC>(a, mk, mv, grid, s)
-                       : launch_decode<T, 128, 1, 2, MODE, true, KSC>(a, mk, mv, grid, s);
-    case 8: return nt1 ? launch_decode<T, 128, 8, 1, MODE, true, KSC>(a, mk, mv, grid, s)
-                       : launch_decode<T, 128, 8, 2, MODE, true, KSC>(a, mk, mv, grid, s);
-    case 16: return nt1 ? launch_decode<T, 128, 16, 1, MODE, true, KSC>(a, mk, mv, grid, s)
-                        : launch_decode<T, 128, 16, 2, MODE, true, KSC>(a, mk, mv, grid, s);
-    case 32: return nt1 ? launch_decode<T, 128, 32, 1, MODE, true, KSC>(a, mk, mv, grid, s)
-                        : launch_decode<T, 128, 32, 2, MODE, true, KSC>(a, mk, mv, grid, s);
+    case 1: return nt1 ? launch_decode<T, D, 1, 1, MODE, true, KSC>(a, mk, mv, grid, s)
+                       : launch_decode<T, D, 1, 2, MODE, true, KSC>(a, mk, mv, grid, s);
+    case 8: return nt1 ? launch_decode<T, D, 8, 1, MODE, true, KSC>(a, mk, mv, grid, s)
+                       : launch_decode<T, D, 8, 2, MODE, true, KSC>(a, mk, mv, grid, s);
+    case 16: return nt1 ? launch_decode<T, D, 16, 1, MODE, true, KSC>(a, mk, mv, grid, s)
+                        : launch_decode<T, D, 16, 2, MODE, true, KSC>(a, mk, mv, grid, s);
+    case 32: return nt1 ? launch_decode<T, D, 32, 1, MODE, true, KSC>(a, mk, mv, grid, s)
+                        : launch_decode<T, D, 32, 2, MODE, true, KSC>(a, mk, mv, grid, s);
   }
   return PA_ERR_UNSUPPORTED;
 }
+template <typename T, bool KSC = false, int MODE = pkv::kPlain>
+pa_status dispatch_e4m3(int d, int bs, const pkv::DecodeArgs& a, const CUtensorMap& mk,
+                        const CUtensorMap& mv, int grid, cudaStream_t s) {
+  return d == 64 ? dispatch_e4m3_d<T, 64, KSC, MODE>(bs, a, mk, mv, grid, s)
+                 : dispatch_e4m3_d<T, 128, KSC, MODE>(bs, a, mk, mv, grid, s);
+}
 
 // The block-scaled 8-bit plain-decode instances; defined in decode_e4m3_bs.cu.
-pa_status run_e4m3_bs(bool bf16, int bs, const pkv::DecodeArgs& a, const CUtensorMap& mk,
+pa_status run_e4m3_bs(bool bf16, int d, int bs, const pkv::DecodeArgs& a, const CUtensorMap& mk,
                       const CUtensorMap& mv, int grid, cudaStream_t s);
 
 // One kernel mode's instances, dispatched on the other parameters; defined in

@@ -21,8 +21,8 @@ NTHREADS = 8
 NAN8 = 0x7F
 
 
-def e4m3_case(ctx, Hq, Hkv, bs, dtype, seed, ks=0.02, vs=0.03, shuffle=True, poison=True):
-    case = make_case(len(ctx), Hq, Hkv, 128, bs, ctx, dtype=dtype, seed=seed, shuffle=shuffle,
+def e4m3_case(ctx, Hq, Hkv, bs, dtype, seed, ks=0.02, vs=0.03, shuffle=True, poison=True, D=128):
+    case = make_case(len(ctx), Hq, Hkv, D, bs, ctx, dtype=dtype, seed=seed, shuffle=shuffle,
                      poison=False)
     shape = case["k"].shape
     case["k8"] = inputs.randn_e4m3(shape, ks, seed, stream=31).numpy()
@@ -42,7 +42,7 @@ def run_e4m3(case):
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
     q = from_bits(case["q"], case["dtype"]).cuda()
     out = torch.full_like(q, float("nan"))
-    ws = pk.new_workspace(case["B"], case["Hq"], case["Hkv"], 128)
+    ws = pk.new_workspace(case["B"], case["Hq"], case["Hkv"], case["D"])
     ws.fill_(0xFF)
     st = pk.new_status()
     pk.pa_decode_e4m3(out, q, dev(case["k8"]), dev(case["v8"]), case["ks"], case["vs"],
@@ -55,16 +55,17 @@ CTX_MIX = [0, 1, 2, 15, 16, 17, 31, 63, 64, 65, 100, 129, 255, 300, 511, 1000, 2
 
 
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("bs", [1, 8, 16, 32])
 @pytest.mark.parametrize("Hq,Hkv", [(4, 4), (32, 8), (64, 8), (16, 1)])
-def test_e4m3_decode_matches_oracle(dtype, bs, Hq, Hkv):
-    case = e4m3_case(CTX_MIX, Hq, Hkv, bs, dtype, seed=600 + bs + Hq)
+def test_e4m3_decode_matches_oracle(dtype, D, bs, Hq, Hkv):
+    case = e4m3_case(CTX_MIX, Hq, Hkv, bs, dtype, seed=600 + bs + Hq + D, D=D)
     out, st = run_e4m3(case)
     assert st == 0
     ref, _ = oracle.decode_e4m3(case["q"], case["k8"], case["v8"], case["ks"], case["vs"],
                                 case["tables"], case["ctx"], case["scale"], dtype,
                                 nthreads=NTHREADS)
-    assert_attn_close(out, ref, what="e4m3 %s bs%d %d/%d" % (dtype, bs, Hq, Hkv))
+    assert_attn_close(out, ref, what="e4m3 %s D%d bs%d %d/%d" % (dtype, D, bs, Hq, Hkv))
     assert not out[0].float().abs().max().item()
 
 
@@ -106,13 +107,13 @@ def test_e4m3_append_bit_exact(dtype, scales):
 
 
 def test_e4m3_unsupported_head_dim_is_rejected():
-    q = torch.zeros((2, 4, 64), dtype=torch.float16, device="cuda")
-    k8 = torch.zeros((4, 4, 16, 64), dtype=torch.uint8, device="cuda")
+    q = torch.zeros((2, 4, 96), dtype=torch.float16, device="cuda")
+    k8 = torch.zeros((4, 4, 16, 96), dtype=torch.uint8, device="cuda")
     t = torch.zeros((2, 1), dtype=torch.int32, device="cuda")
     c = torch.ones(2, dtype=torch.int32, device="cuda")
     with pytest.raises(pk.PagedKVError, match="unsupported"):
         pk.pa_decode_e4m3(torch.empty_like(q), q, k8, k8, 0.1, 0.1, t, c, 0.125,
-                          pk.new_workspace(2, 4, 4, 64))
+                          pk.new_workspace(2, 4, 4, 96))
 
 
 def test_e4m3_llama70b_shape_step_full_size():

@@ -26,16 +26,16 @@ def _dev(a):
     return torch.from_numpy(np.ascontiguousarray(a)).cuda()
 
 
-def bs_case(ctx, Hq, Hkv, bs, dtype, seed, q_len=1, skip_last=False):
+def bs_case(ctx, Hq, Hkv, bs, dtype, seed, q_len=1, skip_last=False, D=128):
     """8-bit pools filled the way a server fills them: every cached token appended in
     position order through the oracle's block-scaled append (so each block's scale is the
     one its first token fixed); free blocks and tails hold NaN codes, blocks without a
     token NaN scales.  skip_last: each sequence's newest token (position ctx-1) is left
     out, for the fused append to write."""
-    case = make_case(len(ctx), Hq, Hkv, 128, bs, ctx, dtype=dtype, seed=seed, poison=False)
+    case = make_case(len(ctx), Hq, Hkv, D, bs, ctx, dtype=dtype, seed=seed, poison=False)
     N = case["N"]
-    k8 = np.full((N, Hkv, bs, 128), NAN8, np.uint8)
-    v8 = np.full((N, Hkv, bs, 128), NAN8, np.uint8)
+    k8 = np.full((N, Hkv, bs, D), NAN8, np.uint8)
+    v8 = np.full((N, Hkv, bs, D), NAN8, np.uint8)
     ks = np.full((N, Hkv), np.nan, np.float32)
     vs = np.full((N, Hkv), np.nan, np.float32)
     slots = []
@@ -45,20 +45,20 @@ def bs_case(ctx, Hq, Hkv, bs, dtype, seed, q_len=1, skip_last=False):
         slots += [t[p // bs] * bs + p % bs for p in range(n)]
     slots = np.array(slots, np.int64)
     T = max(1, len(slots))
-    rng_k = bits(inputs.randn((T, Hkv, 128), dtype, seed, stream=41))
-    rng_v = bits(inputs.randn((T, Hkv, 128), dtype, seed, stream=42))
+    rng_k = bits(inputs.randn((T, Hkv, D), dtype, seed, stream=41))
+    rng_v = bits(inputs.randn((T, Hkv, D), dtype, seed, stream=42))
     oracle.cache_append_e4m3_bs(k8, v8, ks, vs, rng_k[:len(slots)], rng_v[:len(slots)], slots,
                                 dtype)
     case.update(k8=k8, v8=v8, ks=ks, vs=vs)
     if q_len > 1:
-        case["q"] = bits(inputs.randn((len(ctx), q_len, Hq, 128), dtype, seed, stream=43))
+        case["q"] = bits(inputs.randn((len(ctx), q_len, Hq, D), dtype, seed, stream=43))
     return case
 
 
 def run_bs(case):
     q = from_bits(case["q"], case["dtype"]).cuda()
     out = torch.full_like(q, float("nan"))
-    ws = pk.new_workspace(case["B"], case["Hq"], case["Hkv"], 128)
+    ws = pk.new_workspace(case["B"], case["Hq"], case["Hkv"], case["D"])
     ws.fill_(0xFF)
     st = pk.new_status()
     pk.pa_decode_e4m3_bs(out, q, _dev(case["k8"]), _dev(case["v8"]), _dev(case["ks"]),
@@ -107,17 +107,19 @@ CTX_MIX = [0, 1, 2, 15, 16, 17, 31, 63, 64, 65, 100, 129, 255, 300, 511, 1000, 2
 
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
 @pytest.mark.parametrize("bs", [1, 8, 16, 32])
-@pytest.mark.parametrize("Hq,Hkv,q_len", [(4, 4, 1), (32, 8, 1), (64, 8, 1), (16, 1, 1),
-                                          (32, 8, 4), (64, 8, 2), (8, 8, 3)])
-def test_block_scaled_decode_matches_oracle(dtype, bs, Hq, Hkv, q_len):
-    case = bs_case(CTX_MIX, Hq, Hkv, bs, dtype, seed=710 + bs + Hq + q_len, q_len=q_len)
+@pytest.mark.parametrize("Hq,Hkv,q_len,D", [(4, 4, 1, 128), (32, 8, 1, 128), (64, 8, 1, 128),
+                                            (16, 1, 1, 128), (32, 8, 4, 128), (64, 8, 2, 128),
+                                            (8, 8, 3, 128), (4, 4, 1, 64), (32, 8, 1, 64),
+                                            (16, 1, 1, 64), (8, 2, 4, 64)])
+def test_block_scaled_decode_matches_oracle(dtype, bs, Hq, Hkv, q_len, D):
+    case = bs_case(CTX_MIX, Hq, Hkv, bs, dtype, seed=710 + bs + Hq + q_len + D, q_len=q_len, D=D)
     out, st = run_bs(case)
     assert st == 0
     ref, _ = oracle.decode_e4m3_bs(case["q"], case["k8"], case["v8"], case["ks"], case["vs"],
                                    case["tables"], case["ctx"], case["scale"], dtype,
                                    nthreads=NTHREADS)
-    assert_attn_close(out, ref, what="e4m3 block scales %s bs%d %d/%d q_len %d" % (
-        dtype, bs, Hq, Hkv, q_len))
+    assert_attn_close(out, ref, what="e4m3 block scales %s D%d bs%d %d/%d q_len %d" % (
+        dtype, D, bs, Hq, Hkv, q_len))
     assert not out[0].float().abs().max().item()
 
 
@@ -171,21 +173,22 @@ def _newest_slots(case):
 
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
 @pytest.mark.parametrize("bs", [1, 8, 16, 32])
-@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (32, 8), (64, 8), (16, 1)])
-def test_block_scaled_fused_append_equals_append_then_decode(dtype, bs, Hq, Hkv):
+@pytest.mark.parametrize("Hq,Hkv,D", [(4, 4, 128), (32, 8, 128), (64, 8, 128), (16, 1, 128),
+                                      (32, 8, 64), (16, 1, 64)])
+def test_block_scaled_fused_append_equals_append_then_decode(dtype, bs, Hq, Hkv, D):
     """pa_decode_append_e4m3_bs: the same codes, scales and output bits as
     pa_cache_append_e4m3_bs of the newest tokens followed by pa_decode_e4m3_bs; codes and
     scales bit-exact against the oracle's append, the output within tolerance of its
     decode.  The mix has newest tokens at offset 0 of a fresh block (NaN scale before the
     call) and later offsets."""
-    seed = 760 + bs + Hq
-    case = bs_case(CTX_APPEND, Hq, Hkv, bs, dtype, seed=seed, skip_last=True)
+    seed = 760 + bs + Hq + D
+    case = bs_case(CTX_APPEND, Hq, Hkv, bs, dtype, seed=seed, skip_last=True, D=D)
     B = case["B"]
-    kn = inputs.randn((B, Hkv, 128), dtype, seed, "cuda", stream=21) * 2
-    vn = inputs.randn((B, Hkv, 128), dtype, seed, "cuda", stream=22) * 0.1
+    kn = inputs.randn((B, Hkv, D), dtype, seed, "cuda", stream=21) * 2
+    vn = inputs.randn((B, Hkv, D), dtype, seed, "cuda", stream=22) * 0.1
     q = from_bits(case["q"], dtype).cuda()
     tables, ctx = _dev(case["tables"]), _dev(case["ctx"])
-    ws = pk.new_workspace(B, Hq, Hkv, 128)
+    ws = pk.new_workspace(B, Hq, Hkv, D)
     pools = lambda: [_dev(case[x]) for x in ("k8", "v8", "ks", "vs")]
     k1, v1, ks1, vs1 = pools()
     st1 = pk.new_status()
@@ -210,8 +213,8 @@ def test_block_scaled_fused_append_equals_append_then_decode(dtype, bs, Hq, Hkv)
     assert np.array_equal(vs2.cpu().numpy().view(np.uint32), vs.view(np.uint32))
     ref, _ = oracle.decode_e4m3_bs(case["q"], k8, v8, ks, vs, case["tables"], case["ctx"],
                                    case["scale"], dtype, nthreads=NTHREADS)
-    assert_attn_close(o2, ref, what="e4m3 block-scaled fused append %s bs%d %d/%d" % (
-        dtype, bs, Hq, Hkv))
+    assert_attn_close(o2, ref, what="e4m3 block-scaled fused append %s D%d bs%d %d/%d" % (
+        dtype, D, bs, Hq, Hkv))
 
 
 def test_block_scaled_fused_append_llama70b_layer_full_size():
@@ -241,12 +244,12 @@ def test_block_scaled_fused_append_llama70b_layer_full_size():
 
 # ---- the cascade over block-scaled pools
 
-def shared_bs_case(groups, Hq, Hkv, bs, dtype, seed):
+def shared_bs_case(groups, Hq, Hkv, bs, dtype, seed, D=128):
     """test_gpu_cascade's forked sequences, their 8-bit pools filled through the oracle's
     block-scaled append: every physical slot some sequence uses is appended once (a
     shared block's tokens once for all its sharers)."""
     from tests.test_gpu_cascade import shared_case
-    case = shared_case(groups, Hq, Hkv, 128, bs, dtype, seed, poison=False)
+    case = shared_case(groups, Hq, Hkv, D, bs, dtype, seed, poison=False)
     N = case["N"]
     used = sorted({int(case["tables"][i, p // bs]) * bs + p % bs
                    for i in range(case["B"]) for p in range(int(case["ctx"][i]))})
@@ -254,8 +257,8 @@ def shared_bs_case(groups, Hq, Hkv, bs, dtype, seed):
     blk, off = slots // bs, slots % bs
     rows_k = case["k"][blk, :, off, :]                     # [T, Hkv, D]
     rows_v = case["v"][blk, :, off, :]
-    k8 = np.full((N, Hkv, bs, 128), NAN8, np.uint8)
-    v8 = np.full((N, Hkv, bs, 128), NAN8, np.uint8)
+    k8 = np.full((N, Hkv, bs, D), NAN8, np.uint8)
+    v8 = np.full((N, Hkv, bs, D), NAN8, np.uint8)
     ks = np.full((N, Hkv), np.nan, np.float32)
     vs = np.full((N, Hkv), np.nan, np.float32)
     oracle.cache_append_e4m3_bs(k8, v8, ks, vs, np.ascontiguousarray(rows_k),
@@ -268,7 +271,7 @@ def run_cascade_bs(case, plan):
     q = from_bits(case["q"], case["dtype"]).cuda()
     prefix, members, plens = plan
     out = torch.full_like(q, float("nan"))
-    ws = pk.new_cascade_workspace(case["B"], case["Hq"], case["Hkv"], 128)
+    ws = pk.new_cascade_workspace(case["B"], case["Hq"], case["Hkv"], case["D"])
     ws.fill_(0xFF)
     st = pk.new_status()
     pk.pa_decode_cascade_e4m3_bs(out, q, _dev(case["k8"]), _dev(case["v8"]), _dev(case["ks"]),
@@ -285,10 +288,11 @@ CASCADE_GROUPS = [(40, [3, 0, 17, 1]), (0, [5]), (33, [0, 0]),
 
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
 @pytest.mark.parametrize("bs", [1, 8, 16, 32])
-@pytest.mark.parametrize("Hq,Hkv,width", [(8, 2, 2), (8, 2, 4), (32, 8, 2), (4, 4, 8),
-                                          (4, 4, 16), (16, 1, 1)])
-def test_block_scaled_cascade_matches_oracle(dtype, bs, Hq, Hkv, width):
-    case = shared_bs_case(CASCADE_GROUPS, Hq, Hkv, bs, dtype, seed=780 + bs + Hq + width)
+@pytest.mark.parametrize("Hq,Hkv,width,D", [(8, 2, 2, 128), (8, 2, 4, 128), (32, 8, 2, 128),
+                                            (4, 4, 8, 128), (4, 4, 16, 128), (16, 1, 1, 128),
+                                            (8, 2, 4, 64), (4, 4, 16, 64)])
+def test_block_scaled_cascade_matches_oracle(dtype, bs, Hq, Hkv, width, D):
+    case = shared_bs_case(CASCADE_GROUPS, Hq, Hkv, bs, dtype, seed=780 + bs + Hq + width + D, D=D)
     plan = wl.plan_cascade(case["tables"], case["ctx"], bs, Hq // Hkv, width)
     out, st = run_cascade_bs(case, plan)
     assert st == 0
@@ -296,8 +300,8 @@ def test_block_scaled_cascade_matches_oracle(dtype, bs, Hq, Hkv, width):
     ref, _ = oracle.decode_e4m3_bs(case["q"], case["k8"], case["v8"], case["ks"], case["vs"],
                                    case["tables"], case["ctx"], case["scale"], dtype,
                                    nthreads=NTHREADS)
-    assert_attn_close(out, ref, what="e4m3 block-scaled cascade %s bs%d %d/%d w%d" % (
-        dtype, bs, Hq, Hkv, width))
+    assert_attn_close(out, ref, what="e4m3 block-scaled cascade %s D%d bs%d %d/%d w%d" % (
+        dtype, D, bs, Hq, Hkv, width))
 
 
 def test_block_scaled_cascade_without_chunks_is_decode_and_repeats_bit_identical():
