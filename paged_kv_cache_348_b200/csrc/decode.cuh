@@ -20,23 +20,27 @@
 //    contributors per L2 round trip: it sits at the end of most CTAs' ranges, on the
 //    kernel's critical path.
 //  * The producer keeps a window of block-table entries in registers, loaded 64 blocks
-//    ahead of use, so the only table read a stage waits for is a portion's first.
+//    ahead of use (at block_size 1, three windows ahead), so the only table read a stage
+//    waits for is a portion's first.
 //  * Per CTA: one producer warp walks the CTA's range and streams K/V tiles of 64
-//    tokens into a 3-stage shared-memory ring: for block_size >= 8 with 2-D TMA
-//    tensor copies (128-byte swizzle, box = min(block_size,16) rows x 64 dims) whose
-//    row coordinate is the physical block id read from the block table; for
-//    block_size 1 with 16-byte cp.async copies.  Stages complete on mbarriers.
+//    tokens into a shared-memory ring (2-5 stages by configuration): for block_size >= 8
+//    with 2-D TMA tensor copies (128-byte swizzle, box = min(block_size,16) rows x 64
+//    dims) whose row coordinate is the physical block id read from the block table; for
+//    block_size 1 with TMA gather4 loads of four 128-byte rows from four table entries.
+//    Stages complete on mbarriers with transaction counts.
 //  * Four consumer warps each take one 16-token unit of a stage.  All query rows of a
 //    kv head -- the GQA group's heads times the new tokens of the sequence -- share
 //    every K/V byte: S^T = K q^T and O^T += V^T P^T run as m16n8k16 tensor-core MMAs
 //    with the tokens (resp. head dims) on M and those query rows on N (a group of 8
-//    heads fills one n-tile exactly; up to 16 rows are supported).  With several new
-//    tokens, token j is masked from the cached positions after its own.  Softmax is an fp32 online softmax
-//    in base 2; P is split into a 16-bit high part and a 16-bit residual so the PV
-//    product keeps ~16 mantissa bits.
+//    heads fills one n-tile exactly; up to 16 rows here, 9 to 64 also on the tcgen05
+//    kernel of decode_wide.cuh).  With several new tokens, token j is masked from the
+//    cached positions after its own.  Softmax is an fp32 online softmax in base 2; P is
+//    split into a 16-bit high part and a 16-bit residual so the PV product keeps ~16
+//    mantissa bits.  8-bit (E4M3) tiles are converted to fp16 fragments after ldmatrix.
 //  * Every wait is bounded (2 s); on give-up the CTA sets PA_DEV_TIMEOUT and leaves.
-//  * Launched with programmatic dependent launch: the prologue overlaps the previous
-//    kernel's tail, and no global memory is touched before griddepcontrol.wait.
+//  * Launched with programmatic dependent launch: the prologue -- and the producer's
+//    schedule, which reads only lengths, starts and block tables -- overlaps the previous
+//    kernel's tail; nothing else global is touched before griddepcontrol.wait.
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -53,7 +57,7 @@ constexpr int kUnit = 16;                           // tokens per schedule unit
 // end-of-portion merge) is worth about this many units of streaming, so a CTA whose range
 // holds many short segments gets fewer units.  The weight is a tail of virtual units after
 // each segment's real ones; ranges that fall on it do no work.  With block_size 1 a unit
-// costs more (the producer issues a copy per 16 bytes), so the tail is shorter.
+// costs more (the producer issues a gather per 4 rows), so the tail is shorter.
 __host__ __device__ constexpr int seg_weight(int bs) { return bs == 1 ? 2 : 8; }
 constexpr int kConsumerWarps = 4;
 constexpr int kUnitsPerStage = kConsumerWarps;      // one unit per consumer warp
@@ -279,14 +283,6 @@ template <typename T>
 __device__ __forceinline__ T from_float(float x) {
   if constexpr (std::is_same_v<T, __nv_bfloat16>) return __float2bfloat16_rn(x);
   else return __float2half_rn(x);
-}
-
-__device__ __forceinline__ void cp_async_16_zfill(void* dst, const void* src, uint32_t src_bytes,
-                                                  uint64_t policy) {
-  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(
-                   smem_u32(dst)),
-               "l"(src), "r"(src_bytes), "l"(policy)
-               : "memory");
 }
 
 // Finish one output value from this launch's (M, L, acc) of a column: kPlain writes

@@ -13,8 +13,9 @@
 //  * One persistent CTA per SM takes an equal range of the batch's 16-token units (the
 //    schedule of decode.cuh: segments = (sequence, kv head), weighted split, partials of
 //    segments shared between CTAs merged by the last arrival).
-//  * Warp 0 streams 128-token K and V tiles into a 3-stage ring with 2-D TMA copies whose
-//    row coordinate comes from the block table (128-byte swizzle, tokens as rows), and the
+//  * Warp 0 streams 128-token K and V tiles into a 3-stage ring with 4-D TMA copies whose
+//    row coordinate comes from the block table (128-byte swizzle, tokens as rows, a unit's
+//    two column halves in one box; at block_size 1 gather4 loads of four rows), and the
 //    segment's query rows into a Q tile with cp.async (same swizzle).
 //  * Warp 1 (one thread) issues the MMAs: S^T[128 tokens][N] = K . Q^T with the tokens on
 //    M = 128 and the query rows on N = 16..64 (no padding of the query side to 64 or 128),
@@ -624,8 +625,8 @@ __global__ void __launch_bounds__(wide_threads(NC), 1)
       while (ok) {
         bool progress = false;
         if (!q_end && n_qk - n_pv < kWideStages && mbar_try_wait(&full[q_slot], q_ph)) {
-          // Q (and, at block_size 1, K/V) arrive by cp.async: generic-proxy writes the
-          // tensor cores read through the async proxy
+          // Q arrives by cp.async: generic-proxy writes the tensor cores read through the
+          // async proxy
           fence_proxy_async_smem();
           const int f = meta[q_slot].flags;
           if (f & F_END) {
