@@ -162,7 +162,7 @@ struct DecodeArgs {
 // NEW: the fused append's staged rows, SC: the 8-bit per-row scales (regions left out
 // when the launch has no use for them: every byte of shared memory a CTA takes is L1 the
 // spilled registers of the 3-CTA configurations no longer have).
-template <int D, bool KV8 = false, int CPS = 2, bool NEW = true, bool SC = KV8>
+template <int D, bool KV8 = false, int CPS = 2, bool NEW = true, bool SC = KV8, bool G1 = false>
 struct Layout {
   // 8-bit pools with per-row scales at 3 CTAs per SM: a 2-deep ring leaves the spilling
   // consumers more L1 (the fused append over them: 6.11 -> 5.61 ms per 70B-shape step);
@@ -171,7 +171,8 @@ struct Layout {
   static_assert(CPS == 2 || CPS == 3, "2 or 3 CTAs per SM");
   static constexpr int kHalves = D / 64;                   // 128-byte swizzled column halves
   static constexpr int kKvBytes = KV8 ? kTileTokens * D : kHalves * kTileTokens * 128;
-  static constexpr int kQBytes = kMaxGroup * D * 2;
+  // the 16-bit query rows of the stage's columns: at 3 CTAs per SM (one n-tile) at most 8
+  static constexpr int kQBytes = (CPS == 3 ? 8 : kMaxGroup) * D * 2;
   static constexpr int kStageBytes = 2 * kKvBytes + kQBytes;
   static_assert(kStageBytes % 1024 == 0, "stage must keep 1024-byte alignment");
   static constexpr int kMetaOff = kStages * kStageBytes;
@@ -188,10 +189,18 @@ struct Layout {
   // token row, staged by the producer
   static constexpr int kScOff = kNewOff + kStages * kNewBytes;
   static constexpr int kScBytes = SC ? 2 * kTileTokens * 4 : 0;
-  static constexpr int kBytes = kScOff + kStages * kScBytes;
+  // block size 1 (G1), for the consumer warp that issues the V gathers: per stage the row
+  // coordinates of the fill, a barrier the producer arrives on once they are written and
+  // the fill's count of 4-row groups (0: the producer is done); then that warp's count of
+  // the arrivals it has taken
+  static constexpr int kYOff = (kScOff + kStages * kScBytes + 15) / 16 * 16;
+  static constexpr int kYBytes = G1 ? kTileTokens * 4 : 0;
+  static constexpr int kYBarOff = kYOff + kStages * kYBytes;
+  static constexpr int kYMarkOff = kYBarOff + (G1 ? kStages * 8 : 0);
+  static constexpr int kBytes = kYMarkOff + (G1 ? (kStages + 1) * 4 : 0);
   static constexpr int kDynSmem = kBytes + 1024;           // slack for 1024-byte alignment
   static_assert(kBarOff % 8 == 0 && kMiscOff % 8 == 0 && kDescOff % 8 == 0 && kMlOff % 8 == 0 &&
-                    kNewOff % 16 == 0 && kNewBytes % 16 == 0,
+                    kNewOff % 16 == 0 && kNewBytes % 16 == 0 && kYBarOff % 8 == 0,
                 "mbarriers and 64-bit fields need 8-byte, bulk-copy targets 16-byte alignment");
   static_assert(CPS * (kDynSmem + 1024) <= 233472, "CPS CTAs per SM must fit");
 };
@@ -474,13 +483,14 @@ template <typename T, int D, int BS, int NT, int MODE, bool KV8 = false, bool KS
 __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
     pa_decode_split_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
                            const __grid_constant__ CUtensorMap tmv) {
-  using L = Layout<D, KV8, ctas_per_sm(KV8, NT, BS), MODE == kAppend, KSC>;
+  using L = Layout<D, KV8, ctas_per_sm(KV8, NT, BS), MODE == kAppend, KSC, BS == 1>;
   constexpr int kStages = L::kStages;
   constexpr int kSegW = seg_weight(BS);
   static_assert(!KV8 || D == 128 || D == 64, "8-bit caches: head_dim 128 or 64");
   static_assert(!KV8 || MODE == kPlain || KSC,
                 "8-bit caches: the cascade and fused-append modes use per-block scales");
   static_assert(!KSC || KV8, "per-block scales belong to 8-bit caches");
+  static_assert(ctas_per_sm(KV8, NT, BS) == 2 || NT == 1, "the 3-CTA layout holds 8 columns");
   // MMA operand type: the cache's 16-bit type, or fp16 for E4M3 (exact there)
   constexpr bool kBF16 = !KV8 && std::is_same_v<T, __nv_bfloat16>;
   constexpr int kFullCount = 1;        // the producer's expect_tx arrival
@@ -497,12 +507,26 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
   SplitDesc* desc = reinterpret_cast<SplitDesc*>(smem + L::kDescOff);
   float2* mls = reinterpret_cast<float2*>(smem + L::kMlOff);
 
+  // block size 1: the producer issues the K gathers and consumer warp kHelperWarp the V
+  // gathers of every fill (a warp issues TMA loads at a bounded rate, and at four rows a
+  // load this path is bound by it).  A gather load moves four 128-byte pieces (a column
+  // half of a 16-bit row, or a whole 8-bit row; a 64-byte 8-bit row is one piece of its
+  // own size).
+  constexpr int kHelperWarp = kConsumerWarps - 1;
+  constexpr int kGParts = D * (KV8 ? 1 : 2) >= 128 ? D * (KV8 ? 1 : 2) / 128 : 1;
+  constexpr int kGPieceB = KV8 ? (D < 128 ? D : 128) : 128;
+  uint64_t* yready = reinterpret_cast<uint64_t*>(smem + L::kYBarOff);
+  volatile int* ymark = reinterpret_cast<volatile int*>(smem + L::kYMarkOff);
+  volatile int* yseen = ymark + kStages;
+  int* ycoord = reinterpret_cast<int*>(smem + L::kYOff);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&full[i], kFullCount);
       mbar_init(&empty[i], kConsumerWarps);
+      if constexpr (BS == 1) mbar_init(&yready[i], 1);
     }
+    if constexpr (BS == 1) *yseen = 0;
     *abort_flag = 0;
     *last_flag = 0;
     fence_mbar_init();
@@ -613,6 +637,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
     int st = 0, nq = 0;
     uint32_t ph = 0;
     bool ok = true;
+    [[maybe_unused]] int nfill = 0;                  // block size 1: coordinate sets published
     {
       long long x = start;
       const long long xend = end;
@@ -853,9 +878,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
             // cp.async copies, one warp issuing them all, were limited to ~0.4 of HBM
             // bandwidth here.  Stages are 64 tokens, so the window (w0, w1) holds exactly
             // this stage's table entries, handed out by shuffle.
-            // 128-byte pieces of a row (a 64-byte 8-bit row is one piece of its own size)
-            constexpr int kParts = D * (KV8 ? 1 : 2) >= 128 ? D * (KV8 ? 1 : 2) / 128 : 1;
-            constexpr int kPieceB = KV8 ? (D < 128 ? D : 128) : 128;
+            constexpr int kParts = kGParts, kPieceB = kGPieceB;
             const int ntok = nun * kUnit;
             // KSC: the K / V scales of rows lane and 32+lane (this stage's table entries
             // are w0, w1), read before the slot wait
@@ -900,30 +923,30 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
                   bulk_load(sQ + jq * qrow_bytes, qrow_src(jq), qrow_bytes, &full[st]);
               if (nbytes) stage_new(&full[st]);
             }
-            __syncwarp();
+            // every row's coordinate (rows lane and 32+lane), published for the helper warp
+            int* yc = ycoord + st * kTileTokens;
 #pragma unroll
-            for (int it = 0; it < 2; ++it) {
-              const int i = it * 32 + lane;
-              const int kv = i & 1, hf = (i >> 1) % kParts, g = (i >> 1) / kParts;
-              int y[4];
-#pragma unroll
-              for (int q4 = 0; q4 < 4; ++q4) {
-                const int r = 4 * g + q4;                // < 64 for every item issued
-                const int b0 = __shfl_sync(0xffffffffu, w0, r & 31);
-                const int b1 = __shfl_sync(0xffffffffu, w1, r & 31);
-                const int blk = r < 32 ? b0 : b1;
-                y[q4] = rows_total;
-                if (i < nitems && r < nvalid) {
-                  if ((unsigned)blk < (unsigned)a.num_blocks) {
-                    y[q4] = blk * Hkv + kvh;
-                  } else if (a.status && hf == 0 && kv == 0) {
-                    atomicOr(a.status, DEV_BAD_BLOCK_ID);
-                  }
-                }
+            for (int h = 0; h < 2; ++h) {
+              const int r = h * 32 + lane, blk = h ? w1 : w0;
+              int y = rows_total;
+              if (r < nvalid) {
+                if ((unsigned)blk < (unsigned)a.num_blocks) y = blk * Hkv + kvh;
+                else if (a.status) atomicOr(a.status, DEV_BAD_BLOCK_ID);
               }
-              if (i < nitems)
-                tma_gather4((kv ? sV : sK) + hf * (kTileTokens * 128) + g * 4 * kPieceB, kv ? &tmv : &tmk,
-                            &full[st], hf * 64, y[0], y[1], y[2], y[3], policy);
+              yc[r] = y;
+            }
+            __syncwarp();
+            if (lane == 0) {
+              ymark[st] = (nvalid + 3) >> 2;
+              mbar_arrive(&yready[st]);                 // releases the coordinates
+            }
+            ++nfill;
+            // the K gathers: (group of 4 rows g, piece hf), one a lane
+            static_assert(kTileTokens / 4 * kParts <= 32, "one K load item a lane");
+            if (lane < nitems / 2) {
+              const int hf = lane % kParts, g = lane / kParts;
+              tma_gather4(sK + hf * (kTileTokens * 128) + g * 4 * kPieceB, &tmk, &full[st], hf * 64,
+                          yc[4 * g], yc[4 * g + 1], yc[4 * g + 2], yc[4 * g + 3], policy);
             }
           }
           if (++st == kStages) {
@@ -939,6 +962,23 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
       if (lane == 0) meta[st].flags = F_END;
       __syncwarp();
       if (lane == 0) mbar_arrive(&full[st]);
+      if constexpr (BS == 1) {
+        // the V-gather warp waits for the next fill of every slot: one more arrival on each
+        // slot's barrier, with no groups, tells it there is none.  It must have taken every
+        // earlier arrival first (two phases completing before its wait would read as none,
+        // and the group count would be overwritten), which its count shows.
+        bool seen = true;
+        if (lane == 0) seen = wait_count_bounded(yseen, nfill, abort_flag, kWaitLimitNs);
+        seen = __shfl_sync(0xffffffffu, seen, 0);
+        if (seen && lane < kStages) {
+          ymark[lane] = 0;
+          mbar_arrive(&yready[lane]);
+        }
+        if (!seen && lane == 0) {
+          *abort_flag = 1;
+          if (a.status) atomicOr(a.status, DEV_TIMEOUT);
+        }
+      }
     } else {
       if (lane == 0) {
         *abort_flag = 1;
@@ -984,6 +1024,41 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
   for (int n = 0; n < NTW; ++n) {
     jcol[n][0] = ((nb + n) * 8 + 2 * tig) / group;
     jcol[n][1] = ((nb + n) * 8 + 2 * tig + 1) / group;
+  }
+
+  // block size 1, warp kHelperWarp: take the next fill of slot s (the producer's arrival
+  // of parity par on yready[s]) and issue its V gathers, one (group of 4 rows, piece) a
+  // lane, into the slot's V tile; false when the wait gave up
+  [[maybe_unused]] auto take_fill = [&](int s, uint32_t par) -> bool {
+    if (!mbar_wait_bounded(&yready[s], par, abort_flag, kWaitLimitNs)) return false;
+    const int ngrp = __shfl_sync(0xffffffffu, lane == 0 ? ymark[s] : 0, 0);
+    if (lane == 0) {
+      __threadfence_block();                        // the count is read before it is taken
+      *yseen = *yseen + 1;
+    }
+    if (lane < ngrp * kGParts) {
+      const int hf = lane % kGParts, g = lane / kGParts;
+      const int* yc = ycoord + s * kTileTokens + 4 * g;
+      uint8_t* sV = smem + s * L::kStageBytes + L::kKvBytes;
+      tma_gather4(sV + hf * (kTileTokens * 128) + g * 4 * kGPieceB, &tmv, &full[s], hf * 64,
+                  yc[0], yc[1], yc[2], yc[3], policy_evict_first());
+    }
+    return true;
+  };
+  // a failed wait leaves this warp in the loop (the others may reach a named barrier with
+  // it); the abort flag ends every later wait
+  auto helper_abort = [&]() {
+    if (lane == 0) {
+      *abort_flag = 1;
+      if (a.status) atomicOr(a.status, DEV_TIMEOUT);
+    }
+  };
+  if constexpr (BS == 1) {
+    if (cw == kHelperWarp) {
+      bool okh = true;
+      for (int s = 0; s < kStages && okh; ++s) okh = take_fill(s, 0u);
+      if (!okh) helper_abort();
+    }
   }
 
   int st = 0;
@@ -1439,6 +1514,8 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm(KV8, NT, BS))
     if (patched) fence_proxy_async_smem();   // the patched row precedes the next TMA fill
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[st]);
+    if constexpr (BS == 1)
+      if (cw == kHelperWarp && !take_fill(st, ph ^ 1u)) helper_abort();
     if (++st == kStages) {
       st = 0;
       ph ^= 1u;

@@ -43,7 +43,7 @@ cudaError_t launch(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream
 template <typename T, int D, int BS, int NT, int MODE, bool KV8 = false, bool KSC = false>
 pa_status launch_decode(const pkv::DecodeArgs& a, const CUtensorMap& mk, const CUtensorMap& mv,
                         int grid, cudaStream_t stream) {
-  using L = pkv::Layout<D, KV8, pkv::ctas_per_sm(KV8, NT, BS), MODE == pkv::kAppend, KSC>;
+  using L = pkv::Layout<D, KV8, pkv::ctas_per_sm(KV8, NT, BS), MODE == pkv::kAppend, KSC, BS == 1>;
   auto split = pkv::pa_decode_split_kernel<T, D, BS, NT, MODE, KV8, KSC>;
   if (cudaFuncSetAttribute(split, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kDynSmem) !=
       cudaSuccess)

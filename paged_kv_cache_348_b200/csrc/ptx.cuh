@@ -60,6 +60,22 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+// Spin until *p >= n (a count another warp of the CTA raises), bounded as above.
+__device__ __forceinline__ bool wait_count_bounded(volatile int* p, int n, volatile int* abort,
+                                                   uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (*p >= n) {
+      __threadfence_block();                       // what follows is ordered after the read
+      return true;
+    }
+    if ((it & 63u) == 0u) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
+  }
+}
+
 // A cp.async (non-bulk) arrive-on: the barrier's arrival fires once every prior
 // cp.async of this thread has landed; .noinc makes it count as one expected arrival.
 __device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t* bar) {
