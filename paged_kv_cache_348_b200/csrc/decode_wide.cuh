@@ -13,10 +13,13 @@
 //  * One persistent CTA per SM takes an equal range of the batch's 16-token units (the
 //    schedule of decode.cuh: segments = (sequence, kv head), weighted split, partials of
 //    segments shared between CTAs merged by the last arrival).
-//  * Warp 0 streams 128-token K and V tiles into a 3-stage ring with 4-D TMA copies whose
-//    row coordinate comes from the block table (128-byte swizzle, tokens as rows, a unit's
-//    two column halves in one box; at block_size 1 gather4 loads of four rows), and the
-//    segment's query rows into a Q tile with cp.async (same swizzle).
+//  * Warp 0 streams 128-token K tiles into a 3-stage ring with 4-D TMA copies whose row
+//    coordinate comes from the block table (128-byte swizzle, tokens as rows, a unit's two
+//    column halves in one box; at block_size 1 gather4 loads of four rows), and the
+//    segment's query rows into a Q tile with cp.async (same swizzle); with 32 query
+//    columns or fewer warp 10 walks the same schedule and issues the V tiles (one warp
+//    issuing every load capped the stream at ~0.8 of HBM bandwidth with no compute at all;
+//    at 64 columns the extra warp's registers cost the softmax more than it gains).
 //  * Warp 1 (one thread) issues the MMAs: S^T[128 tokens][N] = K . Q^T with the tokens on
 //    M = 128 and the query rows on N = 16..64 (no padding of the query side to 64 or 128),
 //    accumulated in tensor memory (one S^T buffer per ring slot); then O^T[D][N] +=
@@ -49,7 +52,12 @@ constexpr int kWideStages = 3;
 // registers and the softmax spilled.
 __host__ __device__ constexpr int wide_swg(int) { return 2; }
 __host__ __device__ constexpr int wide_soft_threads(int nc) { return 128 * wide_swg(nc); }
-__host__ __device__ constexpr int wide_threads(int nc) { return 64 + wide_soft_threads(nc); }
+// warps: 0 producer (K, Q; V too at 64 columns), 1 MMA, 2 .. 1 + 4 * SWG softmax, then at
+// up to 32 columns the V producer
+__host__ __device__ constexpr bool wide_vprod(int nc) { return nc <= 32; }
+__host__ __device__ constexpr int wide_threads(int nc) {
+  return 64 + wide_soft_threads(nc) + (wide_vprod(nc) ? 32 : 0);
+}
 // tensor memory: one S^T buffer per ring slot (columns 64 s .. 64 s + NC - 1) and O^T from
 // column 256 (NC columns, or 2 NC when P's residual is a second column block)
 constexpr uint32_t kWideTmemCols = 512;
@@ -221,6 +229,8 @@ __global__ void __launch_bounds__(wide_threads(NC), 1)
   uint8_t* sQ = smem + L::kQOff;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // the V producer (none: an index no warp has)
+  constexpr int kVWarp = wide_vprod(NC) ? 2 + kWideSoftThreads / 32 : -1;
   if (threadIdx.x == 0) {
     for (int i = 0; i < kWideStages; ++i) {
       mbar_init(&full[i], kFullCount);
@@ -255,10 +265,10 @@ __global__ void __launch_bounds__(wide_threads(NC), 1)
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
   // Nothing global is written, and nothing a previous kernel may write is read, before the
-  // previous grid is done; the producer of every CTA but CTA 0 (which writes the rows of
-  // sequences without units) computes its schedule first, from the launch's lengths and
-  // chunk members, which no kernel of this library writes.
-  if (warp != 0) {
+  // previous grid is done; the producers of every CTA but CTA 0's K producer (which writes
+  // the rows of sequences without units) compute their schedule first, from the launch's
+  // lengths and chunk members, which no kernel of this library writes.
+  if (warp != 0 && warp != kVWarp) {
     pdl_wait();
     pdl_trigger();
   }
@@ -266,16 +276,24 @@ __global__ void __launch_bounds__(wide_threads(NC), 1)
   const int G = gridDim.x, c = blockIdx.x;
   const int Hkv = a.num_kv_heads, group = a.group;
 
-  if (warp == 0) {
-    // ============================== producer ==============================
-    if (c == 0) pdl_wait();
+  if (warp == 0 || warp == kVWarp) {
+    // ============================== producers ==============================
+    // Both walk the CTA's schedule; warp 0 (kw) issues the K tiles and the Q tile, sets each
+    // stage's meta and byte count and ends the ring, the V warp issues the V tiles.  Each
+    // waits for a slot's release on its own; the V loads of a fill may land before warp 0's
+    // expect_tx (the transaction count goes negative, and the phase still waits for warp
+    // 0's arrival).  Without a V warp, warp 0 issues both pools' tiles.
+    const bool kw = warp == 0;
+    constexpr int nkv = wide_vprod(NC) ? 1 : 2;    // pools this warp loads: kv0 .. kv0+nkv-1
+    const int kv0 = kw ? 0 : 1;
+    if (c == 0 && kw) pdl_wait();
     const int B = a.num_seqs;
     long long run = 0;
     int keep_ctx = 0, keep_u = 0, keep_x = 0;
     for (int base = 0; base < B; base += 32) {
       const int s = base + lane;
       SeqSpan sp{0, 0};
-      if (s < B) sp = span_of<MODE>(a, s, c == 0 ? a.status : nullptr);
+      if (s < B) sp = span_of<MODE>(a, s, c == 0 && kw ? a.status : nullptr);
       const int u = (sp.ctx + kUnit - 1) / kUnit;
       int x = u ? u + kSegW : 0;
 #pragma unroll
@@ -287,7 +305,7 @@ __global__ void __launch_bounds__(wide_threads(NC), 1)
       keep_u = u;
       keep_x = x;
       run += __shfl_sync(0xffffffffu, x, 31);
-      if (c == 0) {
+      if (c == 0 && kw) {
         unsigned zero = __ballot_sync(0xffffffffu, s < B && u == 0);
         while (zero) {
           const int src = __ffs(zero) - 1;
@@ -334,9 +352,9 @@ __global__ void __launch_bounds__(wide_threads(NC), 1)
         r2 += __shfl_sync(0xffffffffu, x, 31);
       }
     }
-    if (lane == 0) *total_s = total;
+    if (lane == 0 && kw) *total_s = total;
     __syncwarp();
-    if (c != 0) pdl_wait();
+    if (c != 0 || !kw) pdl_wait();
 
     const uint64_t policy = policy_evict_first();
     const int rows_total = a.num_blocks * Hkv * BS;
@@ -367,7 +385,7 @@ __global__ void __launch_bounds__(wide_threads(NC), 1)
         int qslot = 0;
         if (!complete) {
           qslot = nqs++;
-          if (lane == 0) {
+          if (lane == 0 && kw) {
             const int cf = cta_of(seg0, total, G), cl = cta_of(seg1 - 1, total, G);
             int ncontrib = 0;
             for (int cc = cf; cc <= cl; ++cc)
@@ -401,8 +419,8 @@ __global__ void __launch_bounds__(wide_threads(NC), 1)
             if (tn >= tok0 && tn < tok0 + nun * kUnit) {   // warp-uniform
               constexpr int CPR = D * 2 / 16;              // 16-byte chunks per row
               const int blk = __ldg(trow + tn / BS);
-              if ((unsigned)blk < (unsigned)a.num_blocks && lane < 2 * CPR) {
-                const int kv = lane / CPR, ch = lane % CPR;
+              if ((unsigned)blk < (unsigned)a.num_blocks && lane < nkv * CPR) {
+                const int kv = kv0 + lane / CPR, ch = lane % CPR;   // this warp's pools
                 const long long src = ((long long)s_cur * Hkv + kvh) * D;
                 const long long row = ((long long)blk * Hkv + kvh) * BS + tn % BS;
                 const T* nrow = static_cast<const T*>(kv ? a.v_new : a.k_new) + src;
@@ -418,15 +436,15 @@ __global__ void __launch_bounds__(wide_threads(NC), 1)
             constexpr int H = BS < 16 ? BS : 16;     // rows per TMA box (all column halves)
             constexpr int BPU = kUnit / H;           // boxes per unit
             constexpr int kBoxBytes = H * 128 * L::kHalves;
-            constexpr int kMaxBox = kWideUnits * BPU * 2;
+            constexpr int kMaxBox = kWideUnits * BPU;    // of this warp's pool
             constexpr int kRep = (kMaxBox + 31) / 32;
-            const int nbox = nun * BPU * 2;
+            const int nbox = nun * BPU;
             // this lane's boxes and their block-table entries, read before the slot wait
             int ys[kRep];
 #pragma unroll
             for (int rp = 0; rp < kRep; ++rp) {
               const int bi = lane + 32 * rp;
-              const int jb = bi >> 1;
+              const int jb = bi;
               const int t = tok0 + (jb / BPU) * kUnit + (jb % BPU) * H;
               ys[rp] = -1;
               if (bi < nbox && t < ctx_cur) {
@@ -434,7 +452,7 @@ __global__ void __launch_bounds__(wide_threads(NC), 1)
                 if ((unsigned)blk < (unsigned)a.num_blocks) {
                   ys[rp] = (blk * Hkv + kvh) * BS + (t % BS);
                 } else {
-                  if (a.status) atomicOr(a.status, DEV_BAD_BLOCK_ID);
+                  if (a.status && kw) atomicOr(a.status, DEV_BAD_BLOCK_ID);
                   ys[rp] = rows_total;                 // out of range: TMA fills zeros
                 }
               }
@@ -449,19 +467,22 @@ __global__ void __launch_bounds__(wide_threads(NC), 1)
               ok = false;
               break;
             }
-            if (lane == 0) {
+            if (lane == 0 && kw) {
               meta[st] = StageMeta{s_cur, kvh, tok0, nun, ctx_cur, flags, pidx, qslot, -1};
               mbar_arrive_expect_tx(&full[st], bytes);
             }
             __syncwarp();
 #pragma unroll
             for (int rp = 0; rp < kRep; ++rp) {
-              const int bi = lane + 32 * rp;
+              const int jb = lane + 32 * rp;
               if (ys[rp] >= 0) {
-                const int kv = bi & 1, jb = bi >> 1;
                 const int row0 = (jb / BPU) * kUnit + (jb % BPU) * H;   // a multiple of 8
-                uint8_t* dst = (kv ? sV : sK) + (row0 >> 3) * L::kGroupBytes;
-                tma_load_4d(dst, kv ? &tmv : &tmk, &full[st], ys[rp] >> 3, policy);
+#pragma unroll
+                for (int kk = 0; kk < nkv; ++kk) {
+                  const int kv = kv0 + kk;
+                  uint8_t* dst = (kv ? sV : sK) + (row0 >> 3) * L::kGroupBytes;
+                  tma_load_4d(dst, kv ? &tmv : &tmk, &full[st], ys[rp] >> 3, policy);
+                }
               }
             }
           } else {
@@ -491,20 +512,20 @@ __global__ void __launch_bounds__(wide_threads(NC), 1)
               ok = false;
               break;
             }
-            // load items (group of 4 rows g, half hf, pool kv): at most 32 * 2 * 2 = 128,
-            // four a lane; rows past the valid tokens or with a bad block id read row
+            // load items (group of 4 rows g, half hf) of this warp's pool: at most 32 * 2 =
+            // 64, two a lane; rows past the valid tokens or with a bad block id read row
             // rows_total, out of range, which the TMA fills with zeros
-            const int nitems = ((nvalid + 3) >> 2) * L::kHalves * 2;
-            static_assert(kWideTile / 4 * L::kHalves * 2 <= 128, "four load items a lane");
-            if (lane == 0) {
+            const int nitems = ((nvalid + 3) >> 2) * L::kHalves;
+            static_assert(kWideTile / 4 * L::kHalves <= 64, "two load items a lane");
+            if (lane == 0 && kw) {
               meta[st] = StageMeta{s_cur, kvh, tok0, nun, ctx_cur, flags, pidx, qslot, -1};
-              mbar_arrive_expect_tx(&full[st], (uint32_t)nitems * 512u);
+              mbar_arrive_expect_tx(&full[st], (uint32_t)nitems * 2u * 512u);
             }
             __syncwarp();
 #pragma unroll
-            for (int it = 0; it < 4; ++it) {
-              const int i = it * 32 + lane;
-              const int kv = i & 1, hf = (i >> 1) % L::kHalves, g = (i >> 1) / L::kHalves;
+            for (int it = 0; it < 2 * nkv; ++it) {
+              const int i = (it & 1) * 32 + lane;
+              const int kv = kv0 + (it >> 1), hf = i % L::kHalves, g = i / L::kHalves;
               int y[4];
 #pragma unroll
               for (int q4 = 0; q4 < 4; ++q4) {
@@ -528,7 +549,7 @@ __global__ void __launch_bounds__(wide_threads(NC), 1)
                             kv ? &tmv : &tmk, &full[st], hf * 64, y[0], y[1], y[2], y[3], policy);
             }
           }
-          if (first_stage) {
+          if (first_stage && kw) {
             // the segment's query rows: column cq = token (or chunk member) j * group + head,
             // row cq of the Q tile, 128-byte swizzle.  The previous portion's last QK^T must
             // be done with the single Q tile first.
@@ -559,7 +580,7 @@ __global__ void __launch_bounds__(wide_threads(NC), 1)
             }
             ++portions;
           }
-          cp_async_mbar_arrive_noinc(&full[st]);
+          if (kw) cp_async_mbar_arrive_noinc(&full[st]);
           if (++st == kWideStages) {
             st = 0;
             ph ^= 1u;
@@ -568,15 +589,18 @@ __global__ void __launch_bounds__(wide_threads(NC), 1)
         x = pe == seg1 ? seg0 + w_cur : pe;          // past the virtual tail
       }
     }
-    if (ok) ok = mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, kWaitLimitNs);
-    if (ok) {
+    if (kw && ok) ok = mbar_wait_bounded(&empty[st], ph ^ 1u, abort_flag, kWaitLimitNs);
+    if (!kw) {
+      // the V producer is done with its last fill
+    } else if (ok) {
       if (lane == 0) {
         meta[st].flags = F_END;
         mbar_arrive(&full[st]);
       }
       __syncwarp();
       cp_async_mbar_arrive_noinc(&full[st]);
-    } else if (lane == 0) {
+    }
+    if (!ok && lane == 0) {
       *abort_flag = 1;
       if (a.status) atomicOr(a.status, DEV_TIMEOUT);
     }
