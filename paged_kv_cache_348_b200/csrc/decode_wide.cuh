@@ -65,7 +65,7 @@ constexpr uint32_t kOCol = 256;
 constexpr float kRescaleLog2 = 8.f;               // a reference max moves past this gap only
 // see pa_decode_wide_kernel: a portion's fixed cost grows with its query columns (the
 // epilogue's row sums and output writes)
-__host__ __device__ constexpr int wide_seg_weight(int nc) { return nc <= 16 ? 32 : (nc <= 32 ? 40 : 56); }
+__host__ __device__ constexpr int wide_seg_weight(int nc) { return nc <= 16 ? 24 : (nc <= 32 ? 40 : 56); }
 
 // K and V tiles: token row r, 64-dim half h (128 bytes, 128-byte swizzle) at
 // ((r / 8) * kHalves + h) * 1024 + (r % 8) * 128: 8-row atoms with the halves side by side,
@@ -202,7 +202,8 @@ __global__ void __launch_bounds__(wide_threads(NC), 1)
   // a segment's schedule weight beyond its units: a portion's fixed cost here (first stage
   // with its reference-max pass and Q load, end-of-portion epilogue) is worth about this
   // many 16-token units of streaming, several stages' worth (measured per CTA with
-  // global-timer stamps), far more than in the mma.sync kernel
+  // global-timer stamps, then timed: at 16 columns 24 against 16, 20, 32 and 48), far
+  // more than in the mma.sync kernel
   constexpr int kSegW = wide_seg_weight(NC);
   constexpr uint32_t kAB = std::is_same_v<T, __nv_bfloat16> ? 1u : 0u;
   constexpr int kFullCount = 33;       // lane 0's expect_tx arrival + 32 cp.async arrivals
