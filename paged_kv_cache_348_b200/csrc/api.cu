@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -186,6 +187,7 @@ struct CascadeArgs {
   float k_scale = 1.f, v_scale = 1.f;
   const float* k_bscale = nullptr;   // 8-bit caches: per-(block, kv head) scales instead
   const float* v_bscale = nullptr;
+  int max_grid = 0;              // > 0: at most this many CTAs (one per segment)
 };
 
 // Validation, workspace layout, tensor maps and launch shared by the decode entry points.
@@ -228,6 +230,7 @@ pa_status decode_impl(void* out, const void* q, const void* k_cache, const void*
   // a cap counts mma.sync CTAs (up to kMaxCtasPerSm a SM); the tcgen05 kernel runs one a SM
   const int cap = grid_cap > 0 ? (wide ? grid_cap / pkv::kMaxCtasPerSm : grid_cap) : 0;
   if (cap > 0 && grid > cap) grid = cap;
+  if (cx.max_grid > 0 && grid > cx.max_grid) grid = cx.max_grid;
   const WsLayout w = ws_layout(head_dim, grid, wide ? pkv::kWideCols : pkv::kMaxGroup);
   if (workspace_bytes < w.total) return PA_ERR_INVALID;
 
@@ -350,6 +353,10 @@ pa_status cascade_impl(void* out, const void* q, const void* k_cache, const void
     cx.mode = pkv::kPrefix;
     cx.chunk_members = chunk_members;
     cx.q_rows = num_seqs;
+    // no more CTAs than (chunk, kv head) segments: the weighted split still balances the
+    // CTAs, but segments of equal length are no longer split (no partials, arrivals or
+    // merges), and the SMs left over start the suffix pass at once
+    cx.max_grid = (int)std::min<long long>((long long)num_chunks * num_kv_heads, 1 << 30);
     const pa_status r = decode_impl(out, q, k_cache, v_cache, block_tables, chunk_prefix_lens,
                                     num_chunks, chunk_width, num_q_heads, num_kv_heads,
                                     head_dim, block_size, max_blocks_per_seq, num_blocks, scale,
@@ -358,6 +365,7 @@ pa_status cascade_impl(void* out, const void* q, const void* k_cache, const void
   }
   // pass 2: every sequence's own tokens, merged with its prefix partial
   cx.mode = pkv::kSuffix;
+  cx.max_grid = 0;
   cx.chunk_members = nullptr;
   cx.seq_start = prefix_lens;
   cx.late_wait = num_chunks > 0 ? 1 : 0;      // its previous grid is then pass 1
