@@ -34,6 +34,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "paged decode attn: KV-read HBM GB/s (% of B200 peak) and seq-steps/s"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0        # B200 HBM3e, nominal (the measured copy peak is the roofline)
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -464,6 +465,8 @@ def main():
                    "l2": "inputs larger than L2 (%.2f GB of K/V per layer)" % (kv_layer / 1e9)},
         "pct_of_peak_hbm": 100.0 * value / world / peak,
         "peak_hbm_gbs": peak, "peak_kind": peak_kind,
+        "pct_of_nominal_hbm": 100.0 * value / world / NOMINAL_HBM_GBS,
+        "nominal_hbm_gbs": NOMINAL_HBM_GBS,
         "seq_steps_per_s": world * w.num_seqs / (ms_step * 1e-3),
         "kv_bytes_per_step": kv_step,
         "roofline": {"bound": "hbm", "kernel": "pa_decode_split_kernel (%s)" % (
