@@ -522,10 +522,12 @@ def run_e2e(b, args, world, kv_step, fused=False):
     """The step through the public API with host buffers.  Every step copies, from pinned
     host memory, every layer's new q / k / v, the block tables, context lens and slot
     mapping, runs append + decode per layer, and copies every layer's output back.
-    Copies run on their own streams, ordered per layer by events: layer l's inputs are
-    uploaded while earlier layers compute, and its output is read back while later
-    layers compute (the step metadata is double-buffered across steps).  Timed with CUDA
-    events from the first upload to the last read-back."""
+    Copies run on their own streams and the device buffers of a step are double-buffered
+    across steps: step i+1's inputs upload while step i computes, and step i's outputs
+    are read back while step i+1 computes; the compute stream waits twice per step (its
+    inputs are in, the read-back of the outputs it overwrites is done), so the layers'
+    launches follow each other directly.  Timed with CUDA events from the first upload to
+    the last read-back."""
     import torch
 
     from paged_kv_cache_348_b200 import pagedkv as pk
@@ -543,95 +545,82 @@ def run_e2e(b, args, world, kv_step, fused=False):
     d2h_bytes = sum(t.numel() * t.element_size() for t in hout)
     comp = torch.cuda.current_stream()
     up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    # two sets of a step's device buffers (set m serves the steps i with i % 2 == m)
+    own = (b.q, b.k_new, b.v_new, b.out, b.block_tables, b.context_lens, b.slot_mapping)
+    qs = [b.q, [t.clone() for t in b.q]]
+    ks = [b.k_new, [t.clone() for t in b.k_new]]
+    vs = [b.v_new, [t.clone() for t in b.v_new]]
+    outs = [b.out, [t.clone() for t in b.out]]
     tabs = [b.block_tables, b.block_tables.clone()]
     ctxs = [b.context_lens, b.context_lens.clone()]
     slots = [b.slot_mapping, b.slot_mapping.clone()]
-    ev_in = [torch.cuda.Event() for _ in range(L)]      # layer l's inputs are on the device
-    ev_used = [torch.cuda.Event() for _ in range(L)]    # layer l computed (inputs free, output ready)
-    ev_out = [torch.cuda.Event() for _ in range(L)]     # layer l's output is on the host
-    ev_meta = [torch.cuda.Event(), torch.cuda.Event()]
-    ev_meta_free = [torch.cuda.Event(), torch.cuda.Event()]
+    ev_in = [torch.cuda.Event(), torch.cuda.Event()]     # set m's inputs are on the device
+    ev_used = [torch.cuda.Event(), torch.cuda.Event()]   # set m's step computed
+    ev_out = [torch.cuda.Event(), torch.cuda.Event()]    # set m's outputs are on the host
 
     def step(i):
         m = i % 2
         with torch.cuda.stream(up):
-            up.wait_event(ev_meta_free[m])
+            up.wait_event(ev_used[m])                    # step i-2 is done with set m
             tabs[m].copy_(htab, non_blocking=True)
             ctxs[m].copy_(hctx, non_blocking=True)
             slots[m].copy_(hslot, non_blocking=True)
-            ev_meta[m].record(up)
             for l in range(L):
-                up.wait_event(ev_used[l])
-                b.q[l].copy_(hq[l], non_blocking=True)
-                b.k_new[l].copy_(hk[l], non_blocking=True)
-                b.v_new[l].copy_(hv[l], non_blocking=True)
-                ev_in[l].record(up)
-        comp.wait_event(ev_meta[m])
-        for l in range(L):
-            comp.wait_event(ev_in[l])
-            comp.wait_event(ev_out[l])
-            if fused:
-                wl.append_decode_layer(b, l, comp, tabs[m], ctxs[m])
-                ev_used[l].record(comp)
-                continue
-            if b.kv_bscales is not None:
-                pk.pa_cache_append_e4m3_bs(b.k_caches[l], b.v_caches[l], *b.kv_bscales[l],
-                                           b.k_new[l], b.v_new[l], slots[m], b.status, comp)
-                if b.cascade is not None:
-                    pk.pa_decode_cascade_e4m3_bs(b.out[l], b.q[l], b.k_caches[l],
-                                                 b.v_caches[l], *b.kv_bscales[l], tabs[m],
-                                                 ctxs[m], *b.cascade, b.scale, b.workspace,
-                                                 b.status, comp)
+                qs[m][l].copy_(hq[l], non_blocking=True)
+                ks[m][l].copy_(hk[l], non_blocking=True)
+                vs[m][l].copy_(hv[l], non_blocking=True)
+            ev_in[m].record(up)
+        comp.wait_event(ev_in[m])
+        comp.wait_event(ev_out[m])                       # step i-2's outputs are read back
+        b.q, b.k_new, b.v_new, b.out = qs[m], ks[m], vs[m], outs[m]
+        b.block_tables, b.context_lens, b.slot_mapping = tabs[m], ctxs[m], slots[m]
+        if fused:
+            wl.run_step(b, comp, fused=True)
+        else:
+            for l in range(L):
+                if b.kv_bscales is not None:
+                    pk.pa_cache_append_e4m3_bs(b.k_caches[l], b.v_caches[l], *b.kv_bscales[l],
+                                               b.k_new[l], b.v_new[l], b.slot_mapping, b.status,
+                                               comp)
+                elif b.kv_scales is not None:
+                    pk.pa_cache_append_e4m3(b.k_caches[l], b.v_caches[l], b.k_new[l],
+                                            b.v_new[l], b.slot_mapping, *b.kv_scales, b.status,
+                                            comp)
                 else:
-                    pk.pa_decode_e4m3_bs(b.out[l], b.q[l], b.k_caches[l], b.v_caches[l],
-                                         *b.kv_bscales[l], tabs[m], ctxs[m], b.scale,
-                                         b.workspace, b.status, comp)
-                ev_used[l].record(comp)
-                continue
-            if b.kv_scales is not None:
-                pk.pa_cache_append_e4m3(b.k_caches[l], b.v_caches[l], b.k_new[l], b.v_new[l],
-                                        slots[m], *b.kv_scales, b.status, comp)
-                pk.pa_decode_e4m3(b.out[l], b.q[l], b.k_caches[l], b.v_caches[l], *b.kv_scales,
-                                  tabs[m], ctxs[m], b.scale, b.workspace, b.status, comp)
-                ev_used[l].record(comp)
-                continue
-            pk.pa_cache_append(b.k_caches[l], b.v_caches[l], b.k_new[l], b.v_new[l], slots[m],
-                               b.status, comp)
-            if b.cascade is not None:
-                pk.pa_decode_cascade(b.out[l], b.q[l], b.k_caches[l], b.v_caches[l], tabs[m],
-                                     ctxs[m], *b.cascade, b.scale, b.workspace, b.status, comp)
-            else:
-                fn = pk.pa_decode if b.q_len == 1 else pk.pa_decode_multi
-                fn(b.out[l], b.q[l], b.k_caches[l], b.v_caches[l], tabs[m], ctxs[m], b.scale,
-                   b.workspace, b.status, comp)
-            ev_used[l].record(comp)
-        ev_meta_free[m].record(comp)
+                    pk.pa_cache_append(b.k_caches[l], b.v_caches[l], b.k_new[l], b.v_new[l],
+                                       b.slot_mapping, b.status, comp)
+                wl.decode_layer(b, l, comp)
+        ev_used[m].record(comp)
         with torch.cuda.stream(down):
+            down.wait_event(ev_used[m])
             for l in range(L):
-                down.wait_event(ev_used[l])
-                hout[l].copy_(b.out[l], non_blocking=True)
-                ev_out[l].record(down)
+                hout[l].copy_(outs[m][l], non_blocking=True)
+            ev_out[m].record(down)
 
-    for i in range(max(1, args.warmup)):
-        step(i)
-    torch.cuda.synchronize()
-    s = torch.cuda.Event(enable_timing=True)
-    e = torch.cuda.Event(enable_timing=True)
-    s.record(comp)
-    up.wait_event(s)
-    down.wait_event(s)
-    for i in range(args.steps):
-        step(i)
-    comp.wait_event(ev_out[L - 1])
-    e.record(comp)
-    torch.cuda.synchronize()
+    try:
+        for i in range(max(1, args.warmup)):
+            step(i)
+        torch.cuda.synchronize()
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record(comp)
+        up.wait_event(s)
+        down.wait_event(s)
+        for i in range(args.steps):
+            step(i)
+        comp.wait_event(ev_out[(args.steps - 1) % 2])
+        e.record(comp)
+        torch.cuda.synchronize()
+    finally:
+        b.q, b.k_new, b.v_new, b.out, b.block_tables, b.context_lens, b.slot_mapping = own
     ms = max_over_ranks(s.elapsed_time(e), world)
     ms_step = ms / args.steps
     return {"value": job_gbs(world, kv_step, ms_step), "unit": "GB/s",
             "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,
             "ms_per_step": ms_step,
             "copies": "pinned host buffers; uploads and read-backs on two copy streams, "
-                      "overlapped with compute layer by layer"}
+                      "device buffers double-buffered across steps (each step's copies "
+                      "overlap the neighbouring steps' compute)"}
 
 
 
