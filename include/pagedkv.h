@@ -569,6 +569,22 @@ pa_status pa_bm_plan_cascade(const pa_block_manager* bm, const int32_t* seqs, in
                              int chunk_width, int32_t* prefix_lens, int32_t* chunk_members,
                              int32_t* chunk_prefix_lens, int* num_chunks, int* chunk_width_out);
 
+/*
+ * pa_check_bounded_waits -- a diagnostic of the bounded waits.  Every wait of a decode
+ * kernel's pipeline (a stage barrier, a slot release, the count the block-size-1 V-gather
+ * warp keeps) gives up after 2 s, sets PA_DEV_TIMEOUT in dev_status and lets the kernel
+ * leave, so a pipeline that cannot finish reports an error instead of hanging the GPU.
+ * This call runs the same two wait helpers, on one warp, against a barrier that nothing
+ * arrives on and a count that nothing raises, each with a limit of limit_us microseconds.
+ *   result    DEVICE int32 [4], 4-byte aligned (written): [0] 1 if the barrier wait gave
+ *             up, [1] 1 if the count wait gave up (both 1 when the mechanism works),
+ *             [2], [3] how long each wait took, in microseconds
+ *   limit_us  1 .. 2,000,000
+ * PA_ERR_INVALID for a null or misaligned result or a limit out of range.  Stream-ordered
+ * like every call; the GPU stays usable afterwards.
+ */
+pa_status pa_check_bounded_waits(int32_t* result, int limit_us, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -17,6 +17,7 @@
 #include "kv_ops.cuh"
 #include "launch.cuh"
 #include "pagedkv.h"
+#include "wait_check.cuh"
 
 namespace {
 
@@ -693,6 +694,14 @@ pa_status pa_copy_blocks(void* const* k_caches, void* const* v_caches, int num_l
       return PA_ERR_CUDA;
   }
   return PA_OK;
+}
+
+pa_status pa_check_bounded_waits(int32_t* result, int limit_us, void* stream) {
+  if (!result || (reinterpret_cast<uintptr_t>(result) & 3) || limit_us < 1 || limit_us > 2000000)
+    return PA_ERR_INVALID;
+  pkv::pa_wait_check_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      result, (uint64_t)limit_us * 1000ull);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 }  // extern "C"

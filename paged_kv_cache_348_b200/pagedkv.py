@@ -33,7 +33,8 @@ EXPORTS = ("pa_version", "pa_status_string", "pa_decode_workspace_bytes", "pa_de
            "pa_bm_context_len", "pa_bm_num_blocks_of", "pa_bm_max_blocks", "pa_bm_block_tables",
            "pa_bm_slot_of", "pa_bm_plan_cascade", "pa_plan_cascade", "pa_bm_swap_out",
            "pa_bm_swap_in", "pa_swap_out_blocks", "pa_swap_in_blocks", "pa_cache_append_e4m3_bs",
-           "pa_decode_e4m3_bs", "pa_decode_cascade_e4m3_bs", "pa_decode_append_e4m3_bs")
+           "pa_decode_e4m3_bs", "pa_decode_cascade_e4m3_bs", "pa_decode_append_e4m3_bs",
+           "pa_check_bounded_waits")
 
 _lib = None
 _lock = threading.Lock()
@@ -66,6 +67,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         L.pa_decode_multi.restype = i32
         L.pa_decode_multi.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, i32,
                                       f32, i32, P, sz, P, P]
+        L.pa_check_bounded_waits.restype = i32
+        L.pa_check_bounded_waits.argtypes = [P, i32, P]
         L.pa_decode_append.restype = i32
         L.pa_decode_append.argtypes = [P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32,
                                        f32, i32, P, sz, P, P]
@@ -152,6 +155,16 @@ def pa_decode_workspace_bytes(num_seqs: int, num_q_heads: int, num_kv_heads: int
 def new_workspace(num_seqs, num_q_heads, num_kv_heads, head_dim, device=None) -> torch.Tensor:
     n = pa_decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim)
     return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def pa_check_bounded_waits(limit_us: int, stream=None) -> list:
+    """Run the library's bounded-wait diagnostic (see pa_check_bounded_waits in
+    include/pagedkv.h) on the current device and return its four results: barrier wait
+    gave up, count wait gave up, and how long each took in microseconds."""
+    result = torch.full((4,), -1, dtype=torch.int32, device="cuda")
+    _check(load().pa_check_bounded_waits(_ptr(result), int(limit_us), _stream(stream)),
+           "pa_check_bounded_waits")
+    return [int(x) for x in result.cpu()]
 
 
 def new_status(device=None) -> torch.Tensor:

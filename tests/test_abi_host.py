@@ -78,6 +78,15 @@ def test_append_and_copy_host_validation(lib):
     assert lib.pa_copy_blocks(bad, arr, 2, p, 3, 10, 4096, None, None) == pk.PA_ERR_INVALID
 
 
+def test_wait_check_host_validation(lib):
+    """pa_check_bounded_waits rejects a null or misaligned result and limits out of range
+    on the host, before anything is launched."""
+    assert lib.pa_check_bounded_waits(None, 100, None) == pk.PA_ERR_INVALID
+    assert lib.pa_check_bounded_waits(P(4098), 100, None) == pk.PA_ERR_INVALID
+    assert lib.pa_check_bounded_waits(P(4096), 0, None) == pk.PA_ERR_INVALID
+    assert lib.pa_check_bounded_waits(P(4096), 2000001, None) == pk.PA_ERR_INVALID
+
+
 def test_binding_refuses_cpu_tensors(lib):
     q = torch.zeros(2, 4, 64, dtype=torch.float16)
     with pytest.raises(pk.PagedKVError, match="CUDA tensor"):

@@ -301,3 +301,17 @@ def test_workload_heavytail_sampled(bs):
     longest = list(np.argsort(ctx)[-6:])
     items = sorted(set(longest + list(range(0, 256, 17))))
     _step_and_check(b, [0], items=[int(i) for i in items])
+
+
+def test_bounded_waits_give_up_and_the_gpu_stays_usable():
+    """The wait helpers every decode pipeline uses give up after their limit when nothing
+    completes the barrier or raises the count (the kernels then set PA_DEV_TIMEOUT and
+    leave), and the device stays usable: a decode right after matches the oracle."""
+    res = pk.pa_check_bounded_waits(20000)             # 20 ms limit
+    assert res[0] == 1 and res[1] == 1, res
+    assert 20000 <= res[2] < 1000000 and 20000 <= res[3] < 1000000, res
+    case = make_case(3, 8, 2, 128, 16, [5, 40, 100], dtype="f16", seed=610)
+    out, status = run_case(case)
+    assert status == 0
+    ref, _ = oracle_of(case)
+    assert_attn_close(out, ref, what="decode after the wait check")
